@@ -1,0 +1,121 @@
+"""fp64 CPU oracle for the WKV7 recurrence -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this package.  The product path (``linear_attention_rnn_wkv7_b200``)
+never does; the two share no code.
+
+``fwd`` runs the plain sequential recurrence of the generalized delta rule
+(rwkv-ops 0.9.0 README, "rwkv7op 使用方法", generalized_delta_rule docstring:
+shapes [B,T,H,K], log-space decay, mask[B,T] 1 = update / 0 = keep, initial
+and final state [N,H,K,V]) in C, fp64, OpenMP over (sequence, head) units;
+see ``wkv7_oracle.c`` for the equations.  ``step`` is the length-one case
+(rwkv-ops 0.9.0 README, "rwkv7_op_rnn 使用方法": inputs (B,1,H,K), state
+(B,H,K,K)).  ``brute`` holds an independent dense-product form used only to
+pin this one on tiny inputs.
+
+Every input is converted exactly to float64 (bf16 and fp32 values are exactly
+representable), so the oracle sees the very values a kernel sees.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wkv7_oracle.c")
+_LIB = os.path.join(_HERE, "libwkv7_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (-O2, OpenMP) next to its source."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def load_library(path: str):
+    """Open a compiled oracle library (the default one, or a test's variant)."""
+    lib = ctypes.CDLL(path)
+    p = ctypes.c_void_p
+    i = ctypes.c_int
+    lib.wkv7_oracle_fwd.restype = ctypes.c_int
+    lib.wkv7_oracle_fwd.argtypes = [p, p, p, p, p, p, p, p, p, p,
+                                    i, i, i, i, i, p, i, i, ctypes.POINTER(ctypes.c_int)]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor (any float dtype, CPU)
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(x):
+    return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
+
+
+def fwd(r, w, k, v, a, b, s0=None, mask=None, cu_seqlens=None,
+        output_final_state: bool = True, nthreads: int = 0, library=None):
+    """Oracle forward.  Returns (o [B,T,H,V] f64, sT [N,H,K,V] f64 or None, threads).
+
+    r,w,k,a,b: [B,T,H,K]; v: [B,T,H,V]; s0: [N,H,K,V] or None (zeros);
+    mask: [B,T] (nonzero = update) or None; cu_seqlens: [N+1] ints or None.
+    """
+    r, w, k, v, a, b = (_f64(x) for x in (r, w, k, v, a, b))
+    B, T, H, K = r.shape
+    V = v.shape[-1]
+    for x in (w, k, a, b):
+        assert x.shape == (B, T, H, K)
+    assert v.shape == (B, T, H, V)
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int32))
+        N = cu.shape[0] - 1
+    else:
+        N = B
+    s0 = _f64(s0)
+    if s0 is not None:
+        assert s0.shape == (N, H, K, V)
+    m = None
+    if mask is not None:
+        m = mask.cpu().numpy() if hasattr(mask, "cpu") else np.asarray(mask)
+        m = np.ascontiguousarray((m != 0).astype(np.uint8))
+        assert m.shape == (B, T)
+    o = np.zeros((B, T, H, V), dtype=np.float64)
+    sT = np.zeros((N, H, K, V), dtype=np.float64) if output_final_state else None
+    used = ctypes.c_int(0)
+    lib = _load() if library is None else library
+    rc = lib.wkv7_oracle_fwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                 _ptr(s0), _ptr(m), _ptr(o), _ptr(sT), B, T, H, K, V,
+                                 _ptr(cu), N, int(nthreads), ctypes.byref(used))
+    if rc != 0:
+        raise ValueError("wkv7_oracle_fwd rejected its arguments")
+    return o, sT, used.value
+
+
+def step(r, w, k, v, a, b, state, nthreads: int = 0):
+    """One decode step: inputs [B,H,K] / v [B,H,V], state [B,H,K,V] (not modified).
+
+    Returns (o [B,H,V], new_state [B,H,K,V]) in float64.
+    """
+    r, w, k, v, a, b = (_f64(x)[:, None] for x in (r, w, k, v, a, b))
+    o, sT, _ = fwd(r, w, k, v, a, b, s0=_f64(state), nthreads=nthreads)
+    return o[:, 0], sT

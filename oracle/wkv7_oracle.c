@@ -1,0 +1,142 @@
+/*
+ * wkv7_oracle.c -- plain, slow, fp64 CPU oracle for the RWKV-7 "generalized
+ * delta rule" (WKV7) recurrence.  TEST INFRASTRUCTURE ONLY: it is built and
+ * called by the tests, by the smoke check and by the benchmark's CPU-baseline
+ * leg, never by the product path.  It shares no code, header or constant with
+ * the CUDA library.
+ *
+ * What it computes (rwkv-ops 0.9.0 README, "rwkv7op 使用方法": the
+ * generalized_delta_rule signature and docstring; rwkv-ops 0.7.4 README, same
+ * section).  Per (sequence, head) a K x V state S, stored row-major [k][v]
+ * exactly like the documented initial_state / final_state layout [N, H, K, V],
+ * evolves token by token:
+ *
+ *     u_t = S_{t-1}^T a_t                            (read the old state with a)
+ *     S_t = diag(exp(w_t)) S_{t-1} + b_t u_t^T + k_t v_t^T
+ *     o_t = S_t^T r_t
+ *
+ * w is the decay "in log space" (docstring: gk is the decay term in log
+ * space), so the per-step factor is exp(w).  The docstring's mask[B,T]
+ * decides whether the state is updated (1 update, 0 no update); at a masked
+ * step the state is carried unchanged and the output is read from it,
+ * o_t = S_{t-1}^T r_t.  initial_state=None means a zero state.  With
+ * cu_seqlens (the packed variable-length form: initial_state has one entry
+ * per sequence, N = number of sequences), sequence n occupies packed rows
+ * [cu_seqlens[n], cu_seqlens[n+1]) of a batch of one and starts from its own
+ * initial state.
+ *
+ * Layouts (all dense, row-major): r,w,k,a,b [B,T,H,K]; v [B,T,H,V];
+ * o [B,T,H,V]; s0 / sT [N,H,K,V]; mask [B,T] (nonzero = update).
+ * Without cu_seqlens N == B.  With cu_seqlens B == 1 and T == cu_seqlens[N].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* One (sequence, head) unit, rows [bos, eos) of batch row bb. */
+static void oracle_unit(const double* r, const double* w, const double* k,
+                        const double* v, const double* a, const double* b,
+                        const double* s0, const unsigned char* mask,
+                        double* o, double* sT, int T, int H, int K, int V,
+                        int bb, int bos, int eos, int n, int h, double* S,
+                        double* u) {
+    const size_t state_off = ((size_t)n * H + h) * (size_t)K * V;
+    if (s0)
+        memcpy(S, s0 + state_off, sizeof(double) * (size_t)K * V);
+    else
+        memset(S, 0, sizeof(double) * (size_t)K * V);
+
+    for (int t = bos; t < eos; ++t) {
+        const size_t rowK = (((size_t)bb * T + t) * H + h) * (size_t)K;
+        const size_t rowV = (((size_t)bb * T + t) * H + h) * (size_t)V;
+        const int update = mask ? (mask[(size_t)bb * T + t] != 0) : 1;
+        if (update) {
+            /* u = S^T a  (uses the state before this token) */
+            for (int j = 0; j < V; ++j) u[j] = 0.0;
+            for (int i = 0; i < K; ++i) {
+                const double ai = a[rowK + i];
+                for (int j = 0; j < V; ++j) u[j] += S[(size_t)i * V + j] * ai;
+            }
+            /* S = diag(exp(w)) S + b u^T + k v^T */
+            for (int i = 0; i < K; ++i) {
+                const double di = exp(w[rowK + i]);
+                const double bi = b[rowK + i];
+                const double ki = k[rowK + i];
+                for (int j = 0; j < V; ++j) {
+                    double* s = &S[(size_t)i * V + j];
+                    *s = di * (*s) + bi * u[j] + ki * v[rowV + j];
+                }
+            }
+        }
+        /* o = S^T r */
+        for (int j = 0; j < V; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < K; ++i) acc += S[(size_t)i * V + j] * r[rowK + i];
+            o[rowV + j] = acc;
+        }
+    }
+    if (sT) memcpy(sT + state_off, S, sizeof(double) * (size_t)K * V);
+}
+
+/*
+ * Returns 0 on success, 1 on an invalid argument.  nthreads <= 0 lets OpenMP
+ * choose; the number of threads actually used is written to *threads_used
+ * when that pointer is non-NULL.
+ */
+int wkv7_oracle_fwd(const double* r, const double* w, const double* k,
+                    const double* v, const double* a, const double* b,
+                    const double* s0, const unsigned char* mask, double* o,
+                    double* sT, int B, int T, int H, int K, int V,
+                    const int32_t* cu_seqlens, int N, int nthreads,
+                    int* threads_used) {
+    if (!r || !w || !k || !v || !a || !b || !o) return 1;
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0) return 1;
+    if (cu_seqlens) {
+        if (B != 1 || N < 0 || cu_seqlens[0] != 0 || cu_seqlens[N] != T) return 1;
+        for (int n = 0; n < N; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n]) return 1;
+    } else {
+        N = B;
+    }
+    const long units = (long)N * H;
+    int used = 1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel
+    {
+#pragma omp single
+        used = omp_get_num_threads();
+        double* S = (double*)malloc(sizeof(double) * ((size_t)K * V + V));
+#pragma omp for schedule(dynamic, 1)
+        for (long unit = 0; unit < units; ++unit) {
+            const int n = (int)(unit / H), h = (int)(unit % H);
+            const int bb = cu_seqlens ? 0 : n;
+            const int bos = cu_seqlens ? cu_seqlens[n] : 0;
+            const int eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+            oracle_unit(r, w, k, v, a, b, s0, mask, o, sT, T, H, K, V, bb, bos,
+                        eos, n, h, S, S + (size_t)K * V);
+        }
+        free(S);
+    }
+#else
+    (void)nthreads;
+    {
+        double* S = (double*)malloc(sizeof(double) * ((size_t)K * V + V));
+        for (long unit = 0; unit < units; ++unit) {
+            const int n = (int)(unit / H), h = (int)(unit % H);
+            const int bb = cu_seqlens ? 0 : n;
+            const int bos = cu_seqlens ? cu_seqlens[n] : 0;
+            const int eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+            oracle_unit(r, w, k, v, a, b, s0, mask, o, sT, T, H, K, V, bb, bos,
+                        eos, n, h, S, S + (size_t)K * V);
+        }
+        free(S);
+    }
+#endif
+    if (threads_used) *threads_used = used;
+    return 0;
+}
