@@ -1,0 +1,365 @@
+#!/usr/bin/env python
+"""Benchmark of the WKV7 hot path on B200.
+
+One step = one wkv7_fwd over the B=8, T=4096, H=64, K=V=64 bf16 workload
+(fp32 initial state in, fp32 final state out), inputs resident in HBM.  The
+line also carries the decode step (wkv7_step over 1024 x 32 fp32 states, 256
+consecutive steps) as HBM GB/s against the measured copy bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (the
+(sequence, head) units are independent, no collective on the data path) and
+rank 0 prints the whole-job throughput: all ranks' tokens / max-over-ranks time.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_rnn_wkv7_b200 import synth  # noqa: E402
+
+METRIC = "WKV7 fwd tokens/s (B=8,T=4096,H=64,D=64 bf16) + decode HBM GB/s vs peak"
+FWD = synth.WORKLOADS["fwd_bf16_b8_t4096_h64"]
+DEC = synth.WORKLOADS["step_bf16_b1024_h32_256steps"]
+TOKEN_HEAD_BYTES = 6 * 64 * 2 + 64 * 2  # r,w,k,v,a,b in + o out, bf16
+STATE_BYTES = 64 * 64 * 4
+FALLBACK_HBM_GBS = 6650.0
+
+
+def fwd_algorithmic_bytes(B, T, H) -> int:
+    return B * T * H * TOKEN_HEAD_BYTES + 2 * B * H * STATE_BYTES
+
+
+def step_algorithmic_bytes(B, H) -> int:
+    return B * H * (2 * STATE_BYTES + 7 * 64 * 2)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_rnn_wkv7_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entries = json.load(f)
+    e = entries.get(kernel)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(target_s: float = 12.0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the B=8,T=4096,H=64
+    workload: whole (b, h) units of T=4096 tokens.  Returns the cpu_baseline dict."""
+    import oracle  # test infrastructure; used here only for the CPU baseline leg
+    x = synth.fwd_inputs(1, FWD["T"], FWD["H"], dtype=torch.bfloat16, seed=FWD["seed"],
+                         s0_std=FWD["s0_std"])
+    H = FWD["H"]
+
+    def run(units):
+        sl = {n: x[n][:, :, :units] for n in "rwkvab"}
+        t0 = time.perf_counter()
+        _, _, used = oracle.fwd(*(sl[n] for n in "rwkvab"), s0=x["s0"][:, :units])
+        return time.perf_counter() - t0, used
+
+    probe_units = min(H, max(2, os.cpu_count() or 1))
+    dt, used = run(probe_units)
+    units = int(min(H, max(probe_units, probe_units * target_s / max(dt, 1e-3))))
+    dt, used = run(units)
+    token_heads = units * FWD["T"]
+    return {"value": token_heads / H / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{units} of the 512 (b,h) units of B=8,T=4096,H=64 (b=0, h<{units}), "
+                      f"full T=4096 each; tokens/s = token-heads / 64 / wall time"}
+
+
+def reference_arm(args, rank: int):
+    """The oracle as the reference arm: each step is one bounded sample."""
+    if rank != 0:
+        return
+    import oracle
+    H, T = FWD["H"], FWD["T"]
+    x = synth.fwd_inputs(1, T, H, dtype=torch.bfloat16, seed=FWD["seed"], s0_std=FWD["s0_std"])
+    units = 4
+    sl = {n: x[n][:, :, :units] for n in "rwkvab"}
+
+    def one():
+        return oracle.fwd(*(sl[n] for n in "rwkvab"), s0=x["s0"][:, :units])[2]
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    used = 0
+    for _ in range(args.steps):
+        used = one()
+    dt = time.perf_counter() - t0
+    tokens = args.steps * units * T / H
+    value = tokens / dt
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "fwd_bf16_b8_t4096_h64", "B": 8, "T": T, "H": H, "K": 64,
+                       "V": 64},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                             "sample": f"each step: {units} of the 512 (b,h) units, full "
+                                       f"T={T}, fp64 sequential recurrence"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--algo", choices=["auto", "recurrent", "chunked"], default="auto")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode leg")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    from linear_attention_rnn_wkv7_b200 import wkv7_fwd, wkv7_step, library
+    library()  # fail loudly if the CUDA library is missing
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if pg is None:
+            return v
+        t = torch.tensor([v], device=device, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    hbm_peak, peak_kind = load_peaks()
+    B, T, H = FWD["B"], FWD["T"], FWD["H"]
+    x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16, seed=FWD["seed"] + 1000 * rank,
+                         s0_std=FWD["s0_std"])
+    xd = {k: v.to(device) for k, v in x.items()}
+    o = torch.empty(B, T, H, 64, dtype=torch.bfloat16, device=device)
+    sT = torch.empty(B, H, 64, 64, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
+                 algo=args.algo, o=o, sT=sT)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    clock_info = clocks.stop()
+    barrier()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_step = ms_total / args.steps
+    tokens_per_step = B * T
+    value = world * tokens_per_step * args.steps / (ms_total / 1e3)
+
+    fwd_bytes = fwd_algorithmic_bytes(B, T, H)
+    achieved = fwd_bytes / (ms_step / 1e3) / 1e9
+    kernel = "chunked" if args.algo in ("auto", "chunked") else "recurrent"
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
+                "traffic": profiled_traffic(f"fwd_{kernel}_b8_t4096_h64"),
+                "algorithmic_bytes_per_launch": fwd_bytes}
+
+    # End to end through the public call with host buffers: pinned H2D of every
+    # input, the forward, D2H of o and the final state, every step.
+    host = {k: v.pin_memory() for k, v in x.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    s_host = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o.numel() * o.element_size() + sT.numel() * sT.element_size()
+
+    def e2e_step():
+        for k in host:
+            xd[k].copy_(host[k], non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+        s_host.copy_(sT, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1)) / args.e2e_steps
+    e2e = {"value": world * tokens_per_step / (ms_e2e / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+    del host, o_host, s_host
+
+    decode = None
+    if not args.no_decode:
+        decode = decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks,
+                            barrier, rank)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_oracle_sample()
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "fwd_bf16_b8_t4096_h64", "B": B, "T": T, "H": H,
+                           "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out",
+                           "algo": args.algo, "parallelism": f"replicas x{world}",
+                           "l2": "inputs (1.9 GB per step) larger than L2; no flush"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": args.steps, "clocks": clock_info, "decode": decode}
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank):
+    """256 consecutive wkv7_step calls over 1024 x 32 fp32 states (512 MiB, > L2).
+    Step inputs: 32 independently drawn step sets, used in turn."""
+    B, H, steps = DEC["B"], DEC["H"], DEC["steps"]
+    state = synth.decode_state(B, H, seed=DEC["seed"] + 1000 * rank, std=DEC["s0_std"]).to(device)
+    sets = []
+    for i in range(32):
+        x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16, seed=DEC["seed"] + 1000 * rank,
+                                     step=i)
+        sets.append({k: v.to(device) for k, v in x.items()})
+    o = torch.empty(B, H, 64, dtype=torch.bfloat16, device=device)
+
+    def run(n):
+        for i in range(n):
+            x = sets[i % len(sets)]
+            wkv7_step(x["r"], x["w"], x["k"], x["v"], x["a"], x["b"], state, o=o)
+
+    run(3)
+    torch.cuda.synchronize(device)
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    run(steps)
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
+    nbytes = step_algorithmic_bytes(B, H)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": "step_bf16_b1024_h32_256steps", "steps": steps, "us_per_step": 1e3 * ms,
+            "algorithmic_bytes_per_step": nbytes, "GB/s": gbs, "peak": hbm_peak,
+            "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
+            "tokens/s": B / (ms / 1e3), "gpu_launches": steps,
+            "traffic": profiled_traffic("step_b1024_h32")}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,128 @@
+/*
+ * wkv7.h -- C ABI of the B200 (sm_100a) WKV7 library (libwkv7.so).
+ *
+ * WKV7 is the RWKV-7 "generalized delta rule" recurrence behind
+ * generalized_delta_rule(r, w, k, v, a, b, initial_state, output_final_state,
+ * head_first, mask) and its length-one decode form rwkv7_op_rnn (rwkv-ops
+ * 0.9.0 README, sections "rwkv7op 使用方法" and "rwkv7_op_rnn 使用方法";
+ * rwkv-ops 0.7.4 README, same sections).  Per (sequence, head) a K x V fp32
+ * state S, stored row-major [k][v], evolves token by token:
+ *
+ *     u_t = S_{t-1}^T a_t                      (a reads the old state)
+ *     S_t = diag(exp(w_t)) S_{t-1} + b_t u_t^T + k_t v_t^T
+ *     o_t = S_t^T r_t
+ *
+ * w is the per-channel decay in log space (the README's docstring: "decay
+ * term in log space"); q in the docstring is r here, gk is w.  mask[b,t] = 0
+ * means the state is not updated at that token (docstring: 1 update, 0 no
+ * update); the output there is read from the unchanged state,
+ * o_t = S_{t-1}^T r_t.
+ *
+ * Conventions shared by every entry point:
+ *  - All pointers are DEVICE pointers of the current CUDA device, dense,
+ *    row-major and 16-byte aligned.  The caller owns and allocates every
+ *    buffer; the library allocates nothing and frees nothing.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *    stream).  A non-OK return means either nothing was launched (argument
+ *    check on the host) or the launch itself failed (WKV7_ERR_CUDA).
+ *  - Problems only the device can see (a cu_seqlens entry out of order or out
+ *    of range) are recorded in a device-side flag; the affected sequence is
+ *    skipped (its outputs are left unwritten) and wkv7_get_last_error reports
+ *    it.  No kernel traps, asserts or spins without a bound.
+ *  - Inputs r, w, k, a, b are [B, T, H, K]; v is [B, T, H, V]; the output o is
+ *    [B, T, H, V]; all of them share one element type (wkv7_dtype).  States
+ *    are fp32 [N, H, K, V] (the README's initial_state / final_state layout).
+ *  - Supported head sizes: K == V == 64 (the README's default head_size).
+ *    Other sizes return WKV7_ERR_UNSUPPORTED.
+ */
+#ifndef WKV7_H
+#define WKV7_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WKV7_OK = 0,
+    WKV7_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad size, bad combination   */
+    WKV7_ERR_UNSUPPORTED = 2,    /* valid request outside the supported set (e.g. K != 64) */
+    WKV7_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed                    */
+    WKV7_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait gave up (reported later)    */
+    WKV7_ERR_DEVICE_BAD_SEQLENS = 5 /* a kernel found cu_seqlens out of order / range       */
+} wkv7_status;
+
+typedef enum {
+    WKV7_BF16 = 0, /* r, w, k, v, a, b and o are bfloat16 */
+    WKV7_F32 = 1   /* r, w, k, v, a, b and o are float32  */
+} wkv7_dtype;
+
+typedef enum {
+    WKV7_ALGO_AUTO = 0,      /* library's choice (chunked tensor-core form for bf16 when built) */
+    WKV7_ALGO_RECURRENT = 1, /* token-by-token fp32 recurrence on CUDA cores                  */
+    WKV7_ALGO_CHUNKED = 2    /* 64-token chunks, WY form, tcgen05 tensor cores (bf16 only)    */
+} wkv7_algo;
+
+/*
+ * wkv7_fwd -- forward over whole sequences (generalized_delta_rule /
+ * generalized_delta_rule_inference; forward only, no autograd state kept).
+ *
+ *   r, w, k, a, b  [B, T, H, K]  dtype   receptance, log decay, key, a (read), b (write)
+ *   v              [B, T, H, V]  dtype
+ *   s0             [N, H, K, V]  fp32    initial states, or NULL for zeros
+ *                                        (README: initial_state=None)
+ *   mask           [B, T]        uint8   nonzero = update, 0 = keep the state; NULL = all 1
+ *   o              [B, T, H, V]  dtype   output, fully written (must not alias an input)
+ *   sT             [N, H, K, V]  fp32    final states, or NULL to skip
+ *                                        (README: output_final_state=False); may equal s0
+ *   cu_seqlens     [N + 1]       int32   packed variable-length form, or NULL.  When given,
+ *                                        B must be 1, sequence n is rows
+ *                                        [cu_seqlens[n], cu_seqlens[n+1]) of the packed T,
+ *                                        cu_seqlens[0] = 0, cu_seqlens[N] = T, non-decreasing.
+ *                                        When NULL, N must equal B.
+ *   algo           wkv7_algo             kernel family (WKV7_ALGO_AUTO unless testing)
+ *
+ * Returns WKV7_OK after enqueueing the kernel(s) on `stream`.
+ * B, T or N may be 0 (nothing to compute; with T == 0, sT receives s0 or zeros).
+ */
+wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
+                     const void* a, const void* b, const float* s0, const uint8_t* mask,
+                     void* o, float* sT, int B, int T, int H, int K, int V,
+                     const int32_t* cu_seqlens, int N, wkv7_dtype dtype, wkv7_algo algo,
+                     void* stream);
+
+/*
+ * wkv7_step -- one decode token for B independent states (rwkv7_op_rnn with
+ * T = 1; README: inputs (B, 1, H, K), state (B, H, K, K)).
+ *
+ *   r, w, k, a, b  [B, H, K]     dtype
+ *   v              [B, H, V]     dtype
+ *   state          [B, H, K, V]  fp32    read and updated IN PLACE (S_{t-1} -> S_t)
+ *   o              [B, H, V]     dtype   o = S_t^T r (must not alias state or inputs)
+ *
+ * Each state is streamed from HBM once and written back once.
+ */
+wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v,
+                      const void* a, const void* b, float* state, void* o, int B, int H,
+                      int K, int V, wkv7_dtype dtype, void* stream);
+
+/*
+ * wkv7_get_last_error -- synchronises `stream`, returns and clears the sticky
+ * device-side flag (WKV7_ERR_DEVICE_TIMEOUT / WKV7_ERR_DEVICE_BAD_SEQLENS) of
+ * the current device, or WKV7_ERR_CUDA if the stream reports a CUDA error,
+ * else WKV7_OK.
+ */
+wkv7_status wkv7_get_last_error(void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* wkv7_status_string(wkv7_status s);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int wkv7_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV7_H */

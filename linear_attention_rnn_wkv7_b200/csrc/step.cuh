@@ -1,0 +1,132 @@
+// step.cuh -- single-token WKV7 decode step (rwkv7_op_rnn, rwkv-ops 0.9.0
+// README, "rwkv7_op_rnn 使用方法": the T = 1 case used for decoding).
+//
+// Per (batch, head) unit the 64 x 64 fp32 state is read from HBM once,
+// updated and written back once:
+//     u = S^T a;   S <- diag(exp w) S + b u^T + k v^T;   o = S^T r.
+// The step is purely HBM-bound (32 KiB of state traffic per unit against
+// ~9 flops per state element), so the kernel is organised around coalesced
+// 128-bit state loads and stores and enough bytes in flight per SM:
+//   - one warp owns one unit; lane l holds columns 4*(l%16) .. +3 of rows
+//     32*(l/16) .. +31, i.e. 32 float4 registers;  one warp-wide load
+//     instruction covers two full 256-byte state rows;
+//   - the two K-halves of u = S^T a and o = S^T r are combined with one
+//     shuffle (xor 16) per column;
+//   - the per-token vectors (r, exp w, k, a, b) go through a 1.25 KiB per-warp
+//     shared-memory stage so each lane reads its 32 rows as float4 broadcasts.
+#pragma once
+#include "common.cuh"
+
+namespace wkv7 {
+
+constexpr int kStepWarps = 4;  // units per block
+
+template <typename Tin>
+__global__ void __launch_bounds__(kStepWarps * 32)
+step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
+            const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
+            float* __restrict__ state, Tin* __restrict__ o, long long units) {
+    __shared__ __align__(16) float vec[kStepWarps][5][64];  // r, d = exp(w), k, a, b
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const long long unit = (long long)blockIdx.x * kStepWarps + warp;
+    if (unit >= units) return;  // warp-uniform; only __syncwarp is used below
+
+    const size_t voff = (size_t)unit * 64;
+    float4* S_g = reinterpret_cast<float4*>(state + (size_t)unit * 64 * 64);
+    const int c = lane & 15;  // float4 column group
+    const int p = lane >> 4;  // row half
+
+    // Issue the 16 KiB state read first so it overlaps the vector staging.
+    float4 S[32];
+#pragma unroll
+    for (int m = 0; m < 32; ++m) S[m] = S_g[(32 * p + m) * 16 + c];
+
+    {
+        const float2 rr = load2(r + voff + 2 * lane);
+        const float2 ww = load2(w + voff + 2 * lane);
+        const float2 kk = load2(k + voff + 2 * lane);
+        const float2 aa = load2(a + voff + 2 * lane);
+        const float2 bb = load2(b + voff + 2 * lane);
+        float* vv = &vec[warp][0][0];
+        reinterpret_cast<float2*>(vv + 0 * 64)[lane] = rr;
+        reinterpret_cast<float2*>(vv + 1 * 64)[lane] = make_float2(expf(ww.x), expf(ww.y));
+        reinterpret_cast<float2*>(vv + 2 * 64)[lane] = kk;
+        reinterpret_cast<float2*>(vv + 3 * 64)[lane] = aa;
+        reinterpret_cast<float2*>(vv + 4 * 64)[lane] = bb;
+    }
+    const float4 vcol = load4(v + voff + 4 * c);
+    __syncwarp();
+
+    const float* sr = &vec[warp][0][32 * p];
+    const float* sd = &vec[warp][1][32 * p];
+    const float* sk = &vec[warp][2][32 * p];
+    const float* sa = &vec[warp][3][32 * p];
+    const float* sb = &vec[warp][4][32 * p];
+
+    // u = S^T a over this lane's 32 rows, then across the two row halves.
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m4 = 0; m4 < 8; ++m4) {
+        const float4 a4 = reinterpret_cast<const float4*>(sa)[m4];
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 s = S[4 * m4 + q];
+            u.x = fmaf(s.x, av[q], u.x);
+            u.y = fmaf(s.y, av[q], u.y);
+            u.z = fmaf(s.z, av[q], u.z);
+            u.w = fmaf(s.w, av[q], u.w);
+        }
+    }
+    u.x += __shfl_xor_sync(0xffffffffu, u.x, 16);
+    u.y += __shfl_xor_sync(0xffffffffu, u.y, 16);
+    u.z += __shfl_xor_sync(0xffffffffu, u.z, 16);
+    u.w += __shfl_xor_sync(0xffffffffu, u.w, 16);
+
+    // S <- diag(d) S + b u^T + k v^T;  o = S^T r;  store S.
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m4 = 0; m4 < 8; ++m4) {
+        const float4 d4 = reinterpret_cast<const float4*>(sd)[m4];
+        const float4 k4 = reinterpret_cast<const float4*>(sk)[m4];
+        const float4 b4 = reinterpret_cast<const float4*>(sb)[m4];
+        const float4 r4 = reinterpret_cast<const float4*>(sr)[m4];
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+        const float rv[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float4 s = S[4 * m4 + q];
+            s.x = fmaf(s.x, dv[q], fmaf(bv[q], u.x, kv[q] * vcol.x));
+            s.y = fmaf(s.y, dv[q], fmaf(bv[q], u.y, kv[q] * vcol.y));
+            s.z = fmaf(s.z, dv[q], fmaf(bv[q], u.z, kv[q] * vcol.z));
+            s.w = fmaf(s.w, dv[q], fmaf(bv[q], u.w, kv[q] * vcol.w));
+            acc.x = fmaf(s.x, rv[q], acc.x);
+            acc.y = fmaf(s.y, rv[q], acc.y);
+            acc.z = fmaf(s.z, rv[q], acc.z);
+            acc.w = fmaf(s.w, rv[q], acc.w);
+            S_g[(32 * p + 4 * m4 + q) * 16 + c] = s;
+        }
+    }
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+    if (p == 0) store4(o + voff + 4 * c, acc);
+}
+
+template <typename Tin>
+cudaError_t launch_step(const void* r, const void* w, const void* k, const void* v,
+                        const void* a, const void* b, float* state, void* o, long long units,
+                        cudaStream_t stream) {
+    const long long blocks = (units + kStepWarps - 1) / kStepWarps;
+    step_kernel<Tin><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
+        static_cast<const Tin*>(r), static_cast<const Tin*>(w), static_cast<const Tin*>(k),
+        static_cast<const Tin*>(v), static_cast<const Tin*>(a), static_cast<const Tin*>(b),
+        state, static_cast<Tin*>(o), units);
+    return cudaGetLastError();
+}
+
+}  // namespace wkv7

@@ -1,0 +1,123 @@
+// wkv7_api.cu -- the C ABI of libwkv7.so (declared in include/wkv7.h): host-side
+// argument checks and kernel dispatch.  Everything the recurrence computes runs
+// in the kernels included below; this file only validates and launches.
+#include <cuda_runtime.h>
+
+#include "wkv7.h"
+#include "common.cuh"
+#include "step.cuh"
+#include "recurrent.cuh"
+#include "chunked.cuh"
+
+namespace {
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+
+}  // namespace
+
+extern "C" {
+
+const char* wkv7_status_string(wkv7_status s) {
+    switch (s) {
+        case WKV7_OK: return "WKV7_OK";
+        case WKV7_ERR_INVALID_ARG: return "WKV7_ERR_INVALID_ARG";
+        case WKV7_ERR_UNSUPPORTED: return "WKV7_ERR_UNSUPPORTED";
+        case WKV7_ERR_CUDA: return "WKV7_ERR_CUDA";
+        case WKV7_ERR_DEVICE_TIMEOUT: return "WKV7_ERR_DEVICE_TIMEOUT";
+        case WKV7_ERR_DEVICE_BAD_SEQLENS: return "WKV7_ERR_DEVICE_BAD_SEQLENS";
+    }
+    return "WKV7_UNKNOWN_STATUS";
+}
+
+int wkv7_version(void) { return kVersion; }
+
+wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
+                     const void* a, const void* b, const float* s0, const uint8_t* mask,
+                     void* o, float* sT, int B, int T, int H, int K, int V,
+                     const int32_t* cu_seqlens, int N, wkv7_dtype dtype, wkv7_algo algo,
+                     void* stream_) {
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0 || N < 0) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_RECURRENT && algo != WKV7_ALGO_CHUNKED)
+        return WKV7_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (B != 1) return WKV7_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return WKV7_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return WKV7_ERR_INVALID_ARG;
+    }
+    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)N * H;
+    const long long rows = (long long)B * T * H;
+    if (units > 0x7fffffffLL || rows > (1LL << 40)) return WKV7_ERR_UNSUPPORTED;
+    const bool tokens = rows > 0;
+    if (tokens && (!ok_ptr(r) || !ok_ptr(w) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(a) ||
+                   !ok_ptr(b) || !ok_ptr(o)))
+        return WKV7_ERR_INVALID_ARG;
+    if ((s0 && !aligned16(s0)) || (sT && !aligned16(sT))) return WKV7_ERR_INVALID_ARG;
+    if (tokens && (o == r || o == w || o == k || o == v || o == a || o == b))
+        return WKV7_ERR_INVALID_ARG;
+    if (units == 0) return WKV7_OK;
+
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool chunked = algo == WKV7_ALGO_CHUNKED ||
+                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && wkv7::kChunkedBuilt);
+    cudaError_t err;
+    if (chunked) {
+        if (dtype != WKV7_BF16 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
+        err = wkv7::launch_chunked(r, w, k, v, a, b, s0, mask, o, sT, B, T, H, N, cu_seqlens,
+                                   stream);
+    } else if (dtype == WKV7_BF16) {
+        err = wkv7::launch_recurrent<__nv_bfloat16>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
+                                                    cu_seqlens, stream);
+    } else {
+        err = wkv7::launch_recurrent<float>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
+                                            cu_seqlens, stream);
+    }
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v,
+                      const void* a, const void* b, float* state, void* o, int B, int H,
+                      int K, int V, wkv7_dtype dtype, void* stream_) {
+    if (B < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)B * H;
+    if (units == 0) return WKV7_OK;
+    if (units > (1LL << 33)) return WKV7_ERR_UNSUPPORTED;
+    if (!ok_ptr(r) || !ok_ptr(w) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(a) || !ok_ptr(b) ||
+        !ok_ptr(state) || !ok_ptr(o))
+        return WKV7_ERR_INVALID_ARG;
+    if (o == state || o == r || o == w || o == k || o == v || o == a || o == b)
+        return WKV7_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const cudaError_t err =
+        dtype == WKV7_BF16
+            ? wkv7::launch_step<__nv_bfloat16>(r, w, k, v, a, b, state, o, units, stream)
+            : wkv7::launch_step<float>(r, w, k, v, a, b, state, o, units, stream);
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+wkv7_status wkv7_get_last_error(void* stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    unsigned int flags = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return WKV7_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&flags, wkv7::g_error_flags, sizeof(flags)) != cudaSuccess)
+        return WKV7_ERR_CUDA;
+    if (flags) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(wkv7::g_error_flags, &zero, sizeof(zero)) != cudaSuccess)
+            return WKV7_ERR_CUDA;
+        if (flags & (1u << WKV7_ERR_DEVICE_TIMEOUT)) return WKV7_ERR_DEVICE_TIMEOUT;
+        if (flags & (1u << WKV7_ERR_DEVICE_BAD_SEQLENS)) return WKV7_ERR_DEVICE_BAD_SEQLENS;
+        return WKV7_ERR_CUDA;
+    }
+    return WKV7_OK;
+}
+
+}  // extern "C"

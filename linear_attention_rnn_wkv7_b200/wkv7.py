@@ -1,0 +1,156 @@
+"""Thin Python binding of libwkv7.so (argument marshalling only).
+
+Every step of the recurrence runs in the library's CUDA kernels; this module
+only checks tensors, allocates outputs with PyTorch and passes raw device
+pointers plus the current CUDA stream through the C ABI declared in
+``include/wkv7.h``.  There is no CPU or PyTorch fallback: if the library is
+missing or the tensors are not on a CUDA device, the call raises.
+
+Names follow the C ABI: ``wkv7_fwd`` (generalized_delta_rule /
+generalized_delta_rule_inference, forward only) and ``wkv7_step``
+(rwkv7_op_rnn) -- rwkv-ops 0.9.0 README, sections "rwkv7op 使用方法" and
+"rwkv7_op_rnn 使用方法".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwkv7.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_DEVICE_BAD_SEQLENS = range(6)
+BF16, F32 = 0, 1
+ALGO = {"auto": 0, "recurrent": 1, "chunked": 2}
+
+_lib = None
+
+
+class WKV7Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def library() -> ctypes.CDLL:
+    """Load libwkv7.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libwkv7.so not built ({LIB_PATH}); run "
+                              "python -m linear_attention_rnn_wkv7_b200.build")
+        lib = ctypes.CDLL(LIB_PATH)
+        p, i = ctypes.c_void_p, ctypes.c_int
+        lib.wkv7_fwd.restype = i
+        lib.wkv7_fwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i, i, i, i, i, p, i, i, i, p]
+        lib.wkv7_step.restype = i
+        lib.wkv7_step.argtypes = [p, p, p, p, p, p, p, p, i, i, i, i, i, p]
+        lib.wkv7_get_last_error.restype = i
+        lib.wkv7_get_last_error.argtypes = [p]
+        lib.wkv7_status_string.restype = ctypes.c_char_p
+        lib.wkv7_status_string.argtypes = [i]
+        lib.wkv7_version.restype = i
+        lib.wkv7_version.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return library().wkv7_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _check(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def wkv7_fwd(r, w, k, v, a, b, s0=None, mask=None, cu_seqlens=None,
+             output_final_state: bool = True, algo: str = "auto", o=None, sT=None):
+    """WKV7 forward.  r,w,k,a,b [B,T,H,K]; v [B,T,H,V] (bf16 or fp32, all alike);
+    s0 [N,H,K,V] fp32 or None; mask [B,T] uint8/bool or None; cu_seqlens [N+1]
+    int32 (B must be 1) or None.  Returns (o [B,T,H,V], sT [N,H,K,V] or None)."""
+    _check(r, "r")
+    dt = r.dtype
+    B, T, H, K = r.shape
+    V = v.shape[-1]
+    for name, t in (("w", w), ("k", k), ("a", a), ("b", b)):
+        _check(t, name, dt, (B, T, H, K))
+    _check(v, "v", dt, (B, T, H, V))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if s0 is not None:
+        _check(s0, "s0", torch.float32, (N, H, K, V))
+    if mask is not None:
+        if mask.dtype == torch.bool:
+            mask = mask.to(torch.uint8)
+        _check(mask, "mask", torch.uint8, (B, T))
+    if o is None:
+        o = torch.empty((B, T, H, V), dtype=dt, device=r.device)
+    else:
+        _check(o, "o", dt, (B, T, H, V))
+    if output_final_state and sT is None:
+        sT = torch.empty((N, H, K, V), dtype=torch.float32, device=r.device)
+    elif sT is not None:
+        _check(sT, "sT", torch.float32, (N, H, K, V))
+    st = library().wkv7_fwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0),
+                            _ptr(mask), _ptr(o), _ptr(sT), B, T, H, K, V, _ptr(cu_seqlens), N,
+                            _dtype_code(r), ALGO[algo], _stream(r.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_fwd")
+    return o, sT
+
+
+def wkv7_step(r, w, k, v, a, b, state, o=None):
+    """One decode token.  r,w,k,a,b [B,H,K]; v [B,H,V]; state [B,H,K,V] fp32,
+    updated in place.  Returns o [B,H,V] (dtype of the inputs)."""
+    _check(r, "r")
+    dt = r.dtype
+    B, H, K = r.shape
+    V = v.shape[-1]
+    for name, t in (("w", w), ("k", k), ("a", a), ("b", b)):
+        _check(t, name, dt, (B, H, K))
+    _check(v, "v", dt, (B, H, V))
+    _check(state, "state", torch.float32, (B, H, K, V))
+    if o is None:
+        o = torch.empty((B, H, V), dtype=dt, device=r.device)
+    else:
+        _check(o, "o", dt, (B, H, V))
+    st = library().wkv7_step(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(state),
+                             _ptr(o), B, H, K, V, _dtype_code(r), _stream(r.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_step")
+    return o
+
+
+def wkv7_get_last_error(device=None) -> int:
+    """Synchronise the current stream; return and clear the device-side flag."""
+    return library().wkv7_get_last_error(_stream(device))

@@ -1,0 +1,111 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports every
+entry point that include/wkv7.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_rnn_wkv7_b200 as wkv7
+from linear_attention_rnn_wkv7_b200 import build as wkv7_build
+from linear_attention_rnn_wkv7_b200.wkv7 import (ERR_INVALID_ARG, ERR_UNSUPPORTED, OK, BF16, F32)
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    wkv7_build.build()
+    return wkv7.library()
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*"
+                            r"(wkv7_[A-Za-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for required in ("wkv7_fwd", "wkv7_step", "wkv7_get_last_error", "wkv7_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libwkv7.so does not export {name}"
+
+
+def test_status_strings(lib):
+    assert wkv7.status_string(OK) == "WKV7_OK"
+    assert wkv7.status_string(ERR_UNSUPPORTED) == "WKV7_ERR_UNSUPPORTED"
+    assert lib.wkv7_version() >= 10000
+
+
+# Fake, 16-byte aligned device addresses: every call below must be rejected by
+# the host-side checks, so nothing is ever dereferenced or launched.
+P = 0x7f0000000000
+MIS = P + 2
+
+
+def fwd(lib, ptrs=None, B=1, T=8, H=2, K=64, V=64, cu=None, N=None, dtype=BF16, algo=0,
+        s0=None, sT=None, o=None, mask=None):
+    ptrs = ptrs or [P + 0x1000 * i for i in range(6)]
+    o = P + 0x10000 if o is None else o
+    N = B if N is None else N
+    return lib.wkv7_fwd(*[ctypes.c_void_p(x) if x else None for x in ptrs],
+                        ctypes.c_void_p(s0) if s0 else None, ctypes.c_void_p(mask) if mask else None,
+                        ctypes.c_void_p(o) if o else None, ctypes.c_void_p(sT) if sT else None,
+                        B, T, H, K, V, ctypes.c_void_p(cu) if cu else None, N, dtype, algo, None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert fwd(lib, K=32, V=32) == ERR_UNSUPPORTED
+    assert fwd(lib, K=64, V=128) == ERR_UNSUPPORTED
+    assert fwd(lib, H=0) == ERR_INVALID_ARG
+    assert fwd(lib, B=-1) == ERR_INVALID_ARG
+    assert fwd(lib, T=-3) == ERR_INVALID_ARG
+    assert fwd(lib, dtype=7) == ERR_INVALID_ARG
+    assert fwd(lib, algo=9) == ERR_INVALID_ARG
+    assert fwd(lib, ptrs=[P, 0, P + 32, P + 48, P + 64, P + 80]) == ERR_INVALID_ARG  # null w
+    assert fwd(lib, ptrs=[P, MIS, P + 32, P + 48, P + 64, P + 80]) == ERR_INVALID_ARG
+    assert fwd(lib, o=0) == ERR_INVALID_ARG
+    assert fwd(lib, o=P) == ERR_INVALID_ARG  # o aliases r
+    assert fwd(lib, s0=MIS) == ERR_INVALID_ARG
+    assert fwd(lib, sT=MIS) == ERR_INVALID_ARG
+    assert fwd(lib, B=2, N=3) == ERR_INVALID_ARG  # N must equal B without cu_seqlens
+    assert fwd(lib, B=2, cu=P + 0x20000, N=2) == ERR_INVALID_ARG  # varlen needs B == 1
+    assert fwd(lib, cu=P + 0x20001, N=2) == ERR_INVALID_ARG  # misaligned cu_seqlens
+    assert fwd(lib, dtype=F32, algo=2) == ERR_UNSUPPORTED  # chunked form is bf16 only
+    # nothing to do: zero sequences, no launch
+    assert fwd(lib, B=0, N=0) == OK
+    assert fwd(lib, cu=P + 0x20000, N=0, T=0) == OK
+
+
+def test_step_rejects_bad_arguments(lib):
+    ptrs = [ctypes.c_void_p(P + 0x1000 * i) for i in range(6)]
+    st, o = ctypes.c_void_p(P + 0x10000), ctypes.c_void_p(P + 0x20000)
+    assert lib.wkv7_step(*ptrs, st, o, 4, 2, 32, 32, BF16, None) == ERR_UNSUPPORTED
+    assert lib.wkv7_step(*ptrs, st, o, 4, 0, 64, 64, BF16, None) == ERR_INVALID_ARG
+    assert lib.wkv7_step(*ptrs, st, o, 4, 2, 64, 64, 5, None) == ERR_INVALID_ARG
+    assert lib.wkv7_step(*ptrs, st, st, 4, 2, 64, 64, BF16, None) == ERR_INVALID_ARG  # o == state
+    assert lib.wkv7_step(*ptrs, None, o, 4, 2, 64, 64, BF16, None) == ERR_INVALID_ARG
+    assert lib.wkv7_step(*ptrs, ctypes.c_void_p(P + 0x10004), o, 4, 2, 64, 64, BF16,
+                         None) == ERR_INVALID_ARG
+    assert lib.wkv7_step(*ptrs, st, o, 0, 2, 64, 64, BF16, None) == OK  # empty batch
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        wkv7.wkv7_fwd(x, x, x, x, x, x)
+    with pytest.raises(ValueError, match="CUDA"):
+        wkv7.wkv7_step(x[:, 0], x[:, 0], x[:, 0], x[:, 0], x[:, 0], x[:, 0],
+                       torch.zeros(1, 1, 64, 64))

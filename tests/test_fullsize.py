@@ -1,0 +1,92 @@
+"""Parity at the full workload sizes, in the launch configuration the benchmark
+times, on sampled (sequence, head) units that the oracle computes one by one.
+
+Workloads: B=8,T=4096,H=64 bf16 (seed 1); B=16,T=4096,H=32 bf16 with a padding
+mask (seed 2); 64 packed sequences of log-uniform length in [16, 8192], H=32
+(seed 3); 1024 x 32 decode states (seed 4)."""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_rnn_wkv7_b200 import synth, wkv7_fwd, wkv7_step
+from parity_util import check, oracle_units, rel_err, BF16_O_REL, BF16_S_REL
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample_units(B, H, n, seed):
+    g = np.random.default_rng(seed)
+    units = {(0, 0), (B - 1, H - 1)}
+    while len(units) < n:
+        units.add((int(g.integers(B)), int(g.integers(H))))
+    return sorted(units)
+
+
+@functools.lru_cache(maxsize=1)
+def _inputs(name):
+    p = synth.WORKLOADS[name]
+    x = synth.fwd_inputs(p["B"], p["T"], p["H"], dtype=torch.bfloat16, seed=p["seed"],
+                         s0_std=p["s0_std"])
+    mask = synth.padding_mask(p["B"], p["T"], seed=p["seed"]) if p.get("mask") else None
+    return x, mask
+
+
+def _fwd_full(cuda_device, name, algo):
+    p = synth.WORKLOADS[name]
+    x, mask = _inputs(name)
+    xd = {k: v.to(cuda_device) for k, v in x.items()}
+    o, s = wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
+                    mask=None if mask is None else mask.to(cuda_device), algo=algo)
+    units = _sample_units(p["B"], p["H"], 6, p["seed"])
+    o_ref, s_ref = oracle_units(x, units, mask)
+    og = torch.stack([o[bb, :, h] for bb, h in units])
+    sg = torch.stack([s[bb, h] for bb, h in units])
+    return check(og, sg, o_ref, s_ref, torch.bfloat16, f"{name} {algo}")
+
+
+@pytest.mark.parametrize("algo", ["auto", "recurrent"])
+def test_fwd_b8_t4096_h64(cuda_device, algo):
+    _fwd_full(cuda_device, "fwd_bf16_b8_t4096_h64", algo)
+
+
+@pytest.mark.parametrize("algo", ["auto", "recurrent"])
+def test_fwd_masked_b16_t4096_h32(cuda_device, algo):
+    _fwd_full(cuda_device, "fwd_bf16_masked_b16_t4096_h32", algo)
+
+
+def test_fwd_varlen_64seq_h32(cuda_device):
+    p = synth.WORKLOADS["fwd_bf16_varlen_64seq_h32"]
+    lengths = synth.varlen_lengths(p["n_seqs"], p["lo"], p["hi"], seed=p["seed"])
+    x = synth.varlen_inputs(lengths, p["H"], dtype=torch.bfloat16, seed=p["seed"],
+                            s0_std=p["s0_std"])
+    xd = {k: v.to(cuda_device) for k, v in x.items()}
+    o, s = wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
+                    cu_seqlens=xd["cu_seqlens"])
+    cu = x["cu_seqlens"].tolist()
+    order = np.argsort(lengths.numpy())
+    for n in {int(order[0]), int(order[-1]), int(order[len(order) // 2])}:  # short, long, median
+        lo, hi = cu[n], cu[n + 1]
+        part = {k: x[k][:, lo:hi] for k in "rwkvab"}
+        o_ref, s_ref, _ = oracle.fwd(*(part[k] for k in "rwkvab"), s0=x["s0"][n:n + 1])
+        check(o[:, lo:hi], s[n:n + 1], o_ref, s_ref, torch.bfloat16, f"varlen seq {n}")
+
+
+def test_step_b1024_h32(cuda_device):
+    p = synth.WORKLOADS["step_bf16_b1024_h32_256steps"]
+    B, H, steps = p["B"], p["H"], 16
+    state = synth.decode_state(B, H, seed=p["seed"], std=p["s0_std"])
+    units = _sample_units(B, H, 8, p["seed"])
+    idx_b = [u[0] for u in units]
+    idx_h = [u[1] for u in units]
+    ref = state[idx_b, idx_h].double().numpy()[:, None]  # [U,1,K,V]
+    st = state.to(cuda_device)
+    for i in range(steps):
+        x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16, seed=p["seed"], step=i)
+        o = wkv7_step(*(x[n].to(cuda_device) for n in "rwkvab"), st)
+        sub = {n: x[n][idx_b, idx_h][:, None] for n in "rwkvab"}  # [U,1,K]
+        o_ref, ref = oracle.step(*(sub[n] for n in "rwkvab"), ref)
+        assert rel_err(o[idx_b, idx_h][:, None], o_ref) <= BF16_O_REL
+    assert rel_err(st[idx_b, idx_h][:, None], ref) <= BF16_S_REL
