@@ -197,6 +197,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=FWD["B"],
+                    help="forward batch (default 8; smaller only for profiling captures)")
+    ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
+                    help="run only one leg (profiling captures)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -232,13 +236,46 @@ def main():
         return float(t.item())
 
     hbm_peak, peak_kind = load_peaks()
-    B, T, H = FWD["B"], FWD["T"], FWD["H"]
+    stream = torch.cuda.current_stream(device)
+    fwd = None
+    if args.only in ("all", "fwd"):
+        fwd = fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
+                      barrier, rank, world)
+    decode = None
+    if args.only in ("all", "decode") and not args.no_decode:
+        decode = decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks,
+                            barrier, rank)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu and args.only == "all":
+        cpu = cpu_oracle_sample()
+
+    if rank == 0:
+        B, T, H = args.batch, FWD["T"], FWD["H"]
+        line = {"metric": METRIC, "value": fwd and fwd["value"], "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": fwd and fwd["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"fwd_bf16_b{B}_t{T}_h{H}", "B": B, "T": T, "H": H,
+                           "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out",
+                           "algo": args.algo, "parallelism": f"replicas x{world}",
+                           "l2": "inputs (1.9 GB per step) larger than L2; no flush"},
+                "roofline": fwd and fwd["roofline"], "cpu_baseline": cpu,
+                "e2e": fwd and fwd["e2e"], "gpu_launches": args.steps if fwd else 0,
+                "clocks": fwd and fwd["clocks"], "decode": decode}
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks, barrier,
+            rank, world):
+    """K timed forward launches on resident inputs, then the host-buffer e2e pass."""
+    B, T, H = args.batch, FWD["T"], FWD["H"]
     x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16, seed=FWD["seed"] + 1000 * rank,
                          s0_std=FWD["s0_std"])
     xd = {k: v.to(device) for k, v in x.items()}
     o = torch.empty(B, T, H, 64, dtype=torch.bfloat16, device=device)
     sT = torch.empty(B, H, 64, 64, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
 
     def step():
         wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
@@ -268,7 +305,8 @@ def main():
     kernel = "chunked" if args.algo in ("auto", "chunked") else "recurrent"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
-                "traffic": profiled_traffic(f"fwd_{kernel}_b8_t4096_h64"),
+                "kernel": kernel,
+                "traffic": profiled_traffic(f"fwd_{kernel}_b{B}_t{T}_h{H}"),
                 "algorithmic_bytes_per_launch": fwd_bytes}
 
     # End to end through the public call with host buffers: pinned H2D of every
@@ -298,31 +336,8 @@ def main():
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1)) / args.e2e_steps
     e2e = {"value": world * tokens_per_step / (ms_e2e / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
-    del host, o_host, s_host
-
-    decode = None
-    if not args.no_decode:
-        decode = decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks,
-                            barrier, rank)
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_oracle_sample()
-
-    if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": "fwd_bf16_b8_t4096_h64", "B": B, "T": T, "H": H,
-                           "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out",
-                           "algo": args.algo, "parallelism": f"replicas x{world}",
-                           "l2": "inputs (1.9 GB per step) larger than L2; no flush"},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps, "clocks": clock_info, "decode": decode}
-        print(json.dumps(line), flush=True)
-    if pg is not None:
-        pg.destroy_process_group()
+    return {"value": value, "ms_per_step": ms_step, "roofline": roofline, "e2e": e2e,
+            "clocks": clock_info}
 
 
 def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank):

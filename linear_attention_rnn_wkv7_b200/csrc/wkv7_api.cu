@@ -64,8 +64,9 @@ wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
     if (units == 0) return WKV7_OK;
 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    const bool chunked = algo == WKV7_ALGO_CHUNKED ||
-                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && wkv7::kChunkedBuilt);
+    // T == 0 (nothing but the state copy) always takes the recurrent kernel.
+    const bool chunked = rows > 0 && (algo == WKV7_ALGO_CHUNKED ||
+                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && wkv7::kChunkedBuilt));
     cudaError_t err;
     if (chunked) {
         if (dtype != WKV7_BF16 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
