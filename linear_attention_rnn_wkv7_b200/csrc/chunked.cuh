@@ -40,28 +40,32 @@ namespace chunked {
 
 constexpr int kThreads = 256;
 // Shared-memory map (bytes; every tile 1024-aligned, 64 rows x 128 B, 128B swizzle).
-constexpr uint32_t OFF_R = 0;          // raw r -> r~        (Gram B rows 0..63)
-constexpr uint32_t OFF_A = 8192;       // raw a -> a~        (Gram B rows 64..127)
-constexpr uint32_t OFF_K = 16384;      // raw k -> k~        (Gram A rows 0..63)
-constexpr uint32_t OFF_B = 24576;      // raw b -> b~        (Gram A rows 64..127)
+constexpr uint32_t OFF_R = 0;          // raw r -> r~        (Gram A rows 0..63)
+constexpr uint32_t OFF_A = 8192;       // raw a -> a~        (Gram A rows 64..127)
+constexpr uint32_t OFF_K = 16384;      // raw k -> k~        (Gram B rows 0..63)
+constexpr uint32_t OFF_B = 24576;      // raw b -> b~        (Gram B rows 64..127)
 constexpr uint32_t OFF_W = 32768;      // raw w -> Bhat      (MMA-3 A, MN-major atom 0)
 constexpr uint32_t OFF_V = 40960;      // raw v              (final MMA B, MN-major)
 constexpr uint32_t OFF_ABAR = 49152;   // Abar [s][k]        (MMA-2 A, MN-major atom 0)
 constexpr uint32_t OFF_AAK = 57344;    // A_ak [s][s']       (MMA-2 A, MN-major atom 1)
 constexpr uint32_t OFF_ARBT = 65536;   // A_rb^T [s][t]      (MMA-3 A, MN-major atom 1)
-constexpr uint32_t OFF_ARKT = 73728;   // A_rk^T [s][t]      (epilogue 3); prologue scratch
+constexpr uint32_t OFF_ARK = 73728;    // A_rk [t][s]        (epilogue 3); prologue scratch
 constexpr uint32_t OFF_RBAR = 81920;   // Rbar [t][k]        (epilogue 3)
 constexpr uint32_t OFF_S0 = 90112;     // S0 bf16 [k][v]     (final MMA B, MN-major)
 constexpr uint32_t OFF_F0 = 98304;     // fp32 64x64: E_t, then Khat [s][k]
 constexpr uint32_t OFF_MISC = 114688;  // mbarriers, TMEM address, abort flag
-constexpr uint32_t kSmemBytes = OFF_MISC + 32;
+constexpr uint32_t OFF_GAMMA = OFF_MISC + 64;  // e^{g_L} per channel (64 fp32)
+constexpr uint32_t kSmemBytes = OFF_GAMMA + 256;
 // Aliases (lifetimes do not overlap).
 constexpr uint32_t OFF_AAB = OFF_R;    // fp32 A_ab [t][s] (epilogue 1 -> solve), 16 KB
-constexpr uint32_t OFF_TT = OFF_K;     // T^T [s][t]      (solve -> MMA-2 B, MN-major)
+constexpr uint32_t OFF_TF = OFF_K;     // fp32 T [t][s]    (solve), 16 KB
+constexpr uint32_t OFF_TT = OFF_R;     // T^T [s][t]      (solve -> MMA-2 B, MN-major)
 constexpr uint32_t OFF_WZT = OFF_K;    // [W^T; Z^T] [n][t] 128 rows (MMA-3 B, K-major)
 constexpr uint32_t OFF_FIN0 = OFF_R;   // final A, K block 0: [M'; Rbar + A_rb W]
 constexpr uint32_t OFF_FIN1 = OFF_ABAR;// final A, K block 1: [P_N hi; A_rk + A_rb Z]
 constexpr uint32_t OFF_FIN2 = OFF_K;   // final A, K block 2: [P_N lo; 0]
+// Prologue scratch inside the A_rk tile (free until epilogue 1), in floats.
+constexpr int SCR_TOT = 0, SCR_EC = 512, SCR_EMC = 576, SCR_ELC = 640, SCR_VALID = 704;
 // Tensor-memory columns (fp32 accumulators, 128 lanes).
 constexpr uint32_t TM_D1 = 0;    // Gram, later MMA-3 (128 cols)
 constexpr uint32_t TM_D2 = 128;  // [W^T; Z^T] (64 cols)
@@ -76,6 +80,13 @@ __device__ __forceinline__ uint32_t sw(uint32_t row, uint32_t c) {
 // Byte offset of bf16 element (row, col) in a 128B-swizzled 64-column tile.
 __device__ __forceinline__ uint32_t swe(uint32_t row, uint32_t col) {
     return sw(row, col >> 3) + ((col & 7u) << 1);
+}
+
+// Float index of (row, col) in a 64x64 fp32 tile whose 16-byte chunks are permuted
+// within each 64-byte group by bits 2..3 of the row, so that four rows 4 apart
+// read with float4 loads hit different banks.
+__device__ __forceinline__ int fidx(int row, int col) {
+    return row * 64 + ((((col >> 2) ^ ((row >> 2) & 3)) << 2) | (col & 3));
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -112,6 +123,51 @@ __device__ __forceinline__ void tmem_row(uint32_t tmem, int wq, uint32_t col, fl
         for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
     }
     sm100::tmem_ld_wait();
+}
+
+// One level L of the blocked triangular inverse: blocks (i, j) = (j + L, j),
+// j = 0 .. 3 - L.  Four threads per output column c, each owning four rows.
+template <int L>
+__device__ __forceinline__ void solve_level(const float* A, float* Tf, int tid, int lane) {
+    if (tid >= (4 - L) * 64) return;  // whole warps
+    const int j = tid >> 6, i = j + L, c = (tid >> 2) & 15, rq = tid & 3;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int d = 0; d < L; ++d) {
+        const int mb = j + d;  // Y += A_{i,mb} T_{mb,j}[:, c]
+        float tc[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) tc[m] = Tf[fidx(16 * mb + m, 16 * j + c)];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int row = 16 * i + 4 * rq + r;
+#pragma unroll
+            for (int m4 = 0; m4 < 16; m4 += 4) {
+                const float4 a4 = *reinterpret_cast<const float4*>(A + fidx(row, 16 * mb + m4));
+                y[r] = fmaf(a4.x, tc[m4], y[r]);
+                y[r] = fmaf(a4.y, tc[m4 + 1], y[r]);
+                y[r] = fmaf(a4.z, tc[m4 + 2], y[r]);
+                y[r] = fmaf(a4.w, tc[m4 + 3], y[r]);
+            }
+        }
+    }
+    float yc[16];  // the whole column Y[:, c], gathered from the four row owners
+#pragma unroll
+    for (int m = 0; m < 16; ++m) yc[m] = __shfl_sync(0xffffffffu, y[m & 3], (lane & ~3) | (m >> 2));
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = 16 * i + 4 * rq + r;
+        float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+        for (int m4 = 0; m4 < 16; m4 += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(Tf + fidx(row, 16 * i + m4));
+            z0 = fmaf(t4.x, yc[m4], z0);
+            z1 = fmaf(t4.y, yc[m4 + 1], z1);
+            z0 = fmaf(t4.z, yc[m4 + 2], z0);
+            z1 = fmaf(t4.w, yc[m4 + 3], z1);
+        }
+        Tf[fidx(row, 16 * j + c)] = z0 + z1;
+    }
 }
 
 __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int* abort_flag) {
@@ -190,11 +246,10 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         for (int c = 0; c < 4; ++c)
             *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(S + 8 * c);
     }
-    float gamma = 1.f;  // e^{g_L} for this thread's channel (state threads)
-
-    float* scratch = reinterpret_cast<float*>(smem + OFF_ARKT);  // prologue only
-    uint8_t* validb = reinterpret_cast<uint8_t*>(scratch + 448);
+    float* scratch = reinterpret_cast<float*>(smem + OFF_ARK);  // prologue only
+    uint8_t* validb = reinterpret_cast<uint8_t*>(scratch + SCR_VALID);
     float* F0 = reinterpret_cast<float*>(smem + OFF_F0);
+    float* gamma_s = reinterpret_cast<float*>(smem + OFF_GAMMA);
     uint32_t mma_phase = 0;
     int iter = 0;
     for (int c0 = 0; c0 < len; c0 += 64, ++iter) {
@@ -214,59 +269,73 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
 
         // ---- 2. prefix sums of w (mask folded), E_t = e^{g_t - c} ------------------------
         {
-            const int kk = tid & 63, q = tid >> 6;
-            float gl[16];
-            float acc = 0.f;
+            const int p = tid & 31, q = tid >> 5;  // channels 2p, 2p+1; tokens 8q .. 8q+7
+            float2 gl[8];
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = 16 * q + i;
+            for (int i = 0; i < 8; ++i) {
+                const int t = 8 * q + i;
                 const bool val = t < nv && (!mask || mask[row0 + c0 + t] != 0);
-                acc += val ? bf16_at(smem + OFF_W, t, kk) : 0.f;
+                const float2 wv = __bfloat1622float2(
+                    *reinterpret_cast<const __nv_bfloat162*>(smem + OFF_W + swe(t, 2 * p)));
+                acc.x += val ? wv.x : 0.f;
+                acc.y += val ? wv.y : 0.f;
                 gl[i] = acc;
-                if (kk == 0) validb[t] = val ? 1 : 0;
+                if (p == 0) validb[t] = val ? 1 : 0;
             }
-            scratch[q * 64 + kk] = acc;
+            reinterpret_cast<float2*>(scratch + SCR_TOT + q * 64)[p] = acc;
             __syncthreads();
-            const float t0 = scratch[kk], t1 = scratch[64 + kk], t2 = scratch[128 + kk],
-                        t3 = scratch[192 + kk];
-            const float prefix = q == 0 ? 0.f : (q == 1 ? t0 : (q == 2 ? t0 + t1 : t0 + t1 + t2));
-            const float c = t0 + t1;
-            const float gL = (t0 + t1) + (t2 + t3);
+            float2 prefix = make_float2(0.f, 0.f), c = prefix, gL = prefix;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) F0[(16 * q + i) * 64 + kk] = clamped_exp(prefix + gl[i] - c);
-            if (q == 0) {
-                scratch[256 + kk] = clamped_exp(c);
-                scratch[320 + kk] = clamped_exp(-c);
-                scratch[384 + kk] = clamped_exp(gL - c);
+            for (int qq = 0; qq < 8; ++qq) {
+                const float2 tq = reinterpret_cast<const float2*>(scratch + SCR_TOT + qq * 64)[p];
+                if (qq < q) { prefix.x += tq.x; prefix.y += tq.y; }
+                if (qq < 4) { c.x += tq.x; c.y += tq.y; }
+                gL.x += tq.x; gL.y += tq.y;
             }
-            gamma = __expf(gL);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                reinterpret_cast<float2*>(F0 + (8 * q + i) * 64)[p] =
+                    make_float2(clamped_exp(prefix.x + gl[i].x - c.x),
+                                clamped_exp(prefix.y + gl[i].y - c.y));
+            if (q == 0) {
+                reinterpret_cast<float2*>(scratch + SCR_EC)[p] =
+                    make_float2(clamped_exp(c.x), clamped_exp(c.y));
+                reinterpret_cast<float2*>(scratch + SCR_EMC)[p] =
+                    make_float2(clamped_exp(-c.x), clamped_exp(-c.y));
+                reinterpret_cast<float2*>(scratch + SCR_ELC)[p] =
+                    make_float2(clamped_exp(gL.x - c.x), clamped_exp(gL.y - c.y));
+                reinterpret_cast<float2*>(gamma_s)[p] = make_float2(__expf(gL.x), __expf(gL.y));
+            }
             __syncthreads();
         }
 
-        // ---- 3. scaled operands (two 8-channel pieces per thread) ------------------------
+        // ---- 3. scaled operands (two 8-channel pieces per thread); each thread rewrites
+        //         only the chunks it read, and Khat waits until every E_t read is done ----
         {
-            uint4 o_r[2], o_a[2], o_k[2], o_b[2], o_abar[2], o_bhat[2], o_rbar[2];
             float4 o_khat[2][2];
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const int item = tid + 256 * it;
                 const int t = item >> 3, j = item & 7;
                 const bool val = validb[t] != 0;
+                const uint32_t off = sw(t, j);
                 float rv[8], av[8], kv[8], bv[8];
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_R + sw(t, j)), rv);
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_A + sw(t, j)), av);
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_K + sw(t, j)), kv);
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_B + sw(t, j)), bv);
+                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_R + off), rv);
+                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_A + off), av);
+                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_K + off), kv);
+                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_B + off), bv);
                 float E[8], Em[8], ec[8], elc[8];
                 const float* Erow = F0 + t * 64 + 8 * j;
-                const float* Emrow = t > 0 ? F0 + (t - 1) * 64 + 8 * j : scratch + 320 + 8 * j;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    E[e] = Erow[e];
-                    Em[e] = Emrow[e];
-                    ec[e] = scratch[256 + 8 * j + e];
-                    elc[e] = scratch[384 + 8 * j + e];
-                }
+                const float* Emrow = t > 0 ? F0 + (t - 1) * 64 + 8 * j : scratch + SCR_EMC + 8 * j;
+                *reinterpret_cast<float4*>(E) = reinterpret_cast<const float4*>(Erow)[0];
+                *reinterpret_cast<float4*>(E + 4) = reinterpret_cast<const float4*>(Erow)[1];
+                *reinterpret_cast<float4*>(Em) = reinterpret_cast<const float4*>(Emrow)[0];
+                *reinterpret_cast<float4*>(Em + 4) = reinterpret_cast<const float4*>(Emrow)[1];
+                *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[0];
+                *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[1];
+                *reinterpret_cast<float4*>(elc) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[0];
+                *reinterpret_cast<float4*>(elc + 4) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[1];
                 float rt[8], at[8], kt[8], btl[8], abar[8], bhat[8], khat[8], rbar[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -282,13 +351,13 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                     khat[e] = k_ * elc[e] * inv;
                     rbar[e] = rt[e] * ec[e];
                 }
-                o_r[it] = pack8(rt);
-                o_a[it] = pack8(at);
-                o_k[it] = pack8(kt);
-                o_b[it] = pack8(btl);
-                o_abar[it] = pack8(abar);
-                o_bhat[it] = pack8(bhat);
-                o_rbar[it] = pack8(rbar);
+                *reinterpret_cast<uint4*>(smem + OFF_R + off) = pack8(rt);
+                *reinterpret_cast<uint4*>(smem + OFF_A + off) = pack8(at);
+                *reinterpret_cast<uint4*>(smem + OFF_K + off) = pack8(kt);
+                *reinterpret_cast<uint4*>(smem + OFF_B + off) = pack8(btl);
+                *reinterpret_cast<uint4*>(smem + OFF_W + off) = pack8(bhat);
+                *reinterpret_cast<uint4*>(smem + OFF_ABAR + off) = pack8(abar);
+                *reinterpret_cast<uint4*>(smem + OFF_RBAR + off) = pack8(rbar);
                 o_khat[it][0] = make_float4(khat[0], khat[1], khat[2], khat[3]);
                 o_khat[it][1] = make_float4(khat[4], khat[5], khat[6], khat[7]);
             }
@@ -297,14 +366,6 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             for (int it = 0; it < 2; ++it) {
                 const int item = tid + 256 * it;
                 const int t = item >> 3, j = item & 7;
-                const uint32_t off = sw(t, j);
-                *reinterpret_cast<uint4*>(smem + OFF_R + off) = o_r[it];
-                *reinterpret_cast<uint4*>(smem + OFF_A + off) = o_a[it];
-                *reinterpret_cast<uint4*>(smem + OFF_K + off) = o_k[it];
-                *reinterpret_cast<uint4*>(smem + OFF_B + off) = o_b[it];
-                *reinterpret_cast<uint4*>(smem + OFF_W + off) = o_bhat[it];
-                *reinterpret_cast<uint4*>(smem + OFF_ABAR + off) = o_abar[it];
-                *reinterpret_cast<uint4*>(smem + OFF_RBAR + off) = o_rbar[it];
                 float4* kh = reinterpret_cast<float4*>(F0 + t * 64 + 8 * j);
                 kh[0] = o_khat[it][0];
                 kh[1] = o_khat[it][1];
@@ -314,54 +375,61 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             __syncthreads();
         }
 
-        // ---- 4. Gram: D1 = [k~; b~] [r~; a~]^T  (128 x 128 x 64) ---------------------------
+        // ---- 4. Gram: D1 = [r~; a~] [k~; b~]^T  (128 x 128 x 64) ---------------------------
         if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t id = idesc_bf16(128, 128, false, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_D1, smem_desc(sbase + OFF_K + 32 * kk, 16, 1024),
-                          smem_desc(sbase + OFF_R + 32 * kk, 16, 1024), id, kk > 0);
+                umma_bf16(tmem + TM_D1, smem_desc(sbase + OFF_R + 32 * kk, 16, 1024),
+                          smem_desc(sbase + OFF_K + 32 * kk, 16, 1024), id, kk > 0);
             umma_commit(bar_mma);
         }
         wait_or_abort(bar_mma, mma_phase, abort_flag);
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 5. epilogue 1: masked A_rk^T, A_ak, A_rb^T (bf16), A_ab (fp32) ----------------
+        // ---- 5. epilogue 1: rows t of D1 -> masked A_rk, A_rb^T, A_ak (bf16), A_ab (fp32) --
         {
             float v[64];
             tmem_row<4>(tmem + TM_D1, wq, 64 * wh, v);
             if (wq < 2) {
-                const int s = m_row;  // row of k~
-                if (wh == 0) {  // A_rk[t][s] = v[t], kept for s <= t -> A_rk^T row s
+                const int t = m_row;  // row of r~
+                if (wh == 0) {  // A_rk[t][s] = v[s], kept for s <= t -> row t
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         float x[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = (s <= 8 * c + e) ? v[8 * c + e] : 0.f;
-                        *reinterpret_cast<uint4*>(smem + OFF_ARKT + sw(s, c)) = pack8(x);
+                        for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
+                        *reinterpret_cast<uint4*>(smem + OFF_ARK + sw(t, c)) = pack8(x);
                     }
-                } else {  // A_ak[t][s] = v[t], kept for s < t -> column s of the A_ak tile
+                } else {  // A_rb[t][s] = v[s], kept for s <= t -> column t of A_rb^T
 #pragma unroll
-                    for (int t = 0; t < 64; ++t)
-                        *reinterpret_cast<__nv_bfloat16*>(smem + OFF_AAK + swe(t, s)) =
-                            __float2bfloat16_rn(s < t ? v[t] : 0.f);
+                    for (int s_ = 0; s_ < 64; ++s_)
+                        *reinterpret_cast<__nv_bfloat16*>(smem + OFF_ARBT + swe(s_, t)) =
+                            __float2bfloat16_rn(s_ <= t ? v[s_] : 0.f);
                 }
             } else {
-                const int s = m_row - 64;  // row of b~
-                if (wh == 0) {  // A_rb[t][s], s <= t -> A_rb^T row s
+                const int t = m_row - 64;  // row of a~
+                if (wh == 0) {  // A_ak[t][s] = v[s], kept for s < t -> row t
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         float x[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = (s <= 8 * c + e) ? v[8 * c + e] : 0.f;
-                        *reinterpret_cast<uint4*>(smem + OFF_ARBT + sw(s, c)) = pack8(x);
+                        for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
+                        *reinterpret_cast<uint4*>(smem + OFF_AAK + sw(t, c)) = pack8(x);
                     }
-                } else {  // A_ab[t][s], s < t -> fp32 [t][s]
+                } else {  // A_ab[t][s], kept for s < t -> fp32 row t
                     float* aab = reinterpret_cast<float*>(smem + OFF_AAB);
 #pragma unroll
-                    for (int t = 0; t < 64; ++t) aab[t * 64 + s] = s < t ? v[t] : 0.f;
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        float4 x;
+                        x.x = (4 * c4 + 0 < t) ? v[4 * c4 + 0] : 0.f;
+                        x.y = (4 * c4 + 1 < t) ? v[4 * c4 + 1] : 0.f;
+                        x.z = (4 * c4 + 2 < t) ? v[4 * c4 + 2] : 0.f;
+                        x.w = (4 * c4 + 3 < t) ? v[4 * c4 + 3] : 0.f;
+                        *reinterpret_cast<float4*>(aab + fidx(t, 4 * c4)) = x;
+                    }
                 }
             }
             fence_proxy_async();
@@ -369,39 +437,54 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             __syncthreads();
         }
 
-        // ---- 6. T = (I - A_ab)^-1 by forward substitution, 4 threads per column -----------
+        // ---- 6. T = (I - A_ab)^-1 (fp32): 16x16 diagonal blocks by forward substitution,
+        //         then the off-diagonal blocks level by level,
+        //         T_ij = T_ii * sum_{m=j}^{i-1} A_im T_mj ------------------------------------
         {
-            const int jj = lane >> 2, hq = lane & 3;
-            const int j = 8 * warp + jj;
-            const float* aab = reinterpret_cast<const float*>(smem + OFF_AAB);
-            float x[16];
+            const float* A = reinterpret_cast<const float*>(smem + OFF_AAB);
+            float* Tf = reinterpret_cast<float*>(smem + OFF_TF);
+            if (tid < 64) {  // diagonal block b, column c
+                const int b = tid >> 4, c = tid & 15, base = 16 * b;
+                float x[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = 0.f;
+                for (int i = 0; i < 16; ++i) x[i] = 0.f;
 #pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                float acc = 0.f;
-                if (t > 0) {
+                for (int t = 0; t < 16; ++t) {
+                    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                    for (int i = 0; i <= (t - 1) / 16; ++i) {
-                        const float4 arow =
-                            *reinterpret_cast<const float4*>(aab + t * 64 + 16 * i + 4 * hq);
-                        acc = fmaf(arow.x, x[4 * i + 0], acc);
-                        acc = fmaf(arow.y, x[4 * i + 1], acc);
-                        acc = fmaf(arow.z, x[4 * i + 2], acc);
-                        acc = fmaf(arow.w, x[4 * i + 3], acc);
+                    for (int s4 = 0; s4 < t; s4 += 4) {
+                        const float4 a4 =
+                            *reinterpret_cast<const float4*>(A + fidx(base + t, base + s4));
+                        acc0 = fmaf(a4.x, x[s4 + 0], acc0);
+                        acc1 = fmaf(a4.y, x[s4 + 1], acc1);
+                        acc0 = fmaf(a4.z, x[s4 + 2], acc0);
+                        acc1 = fmaf(a4.w, x[s4 + 3], acc1);
                     }
+                    x[t] = (t == c) ? 1.f : acc0 + acc1;
                 }
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                const float val = (t == j) ? 1.f : acc;
-                if (hq == ((t >> 2) & 3)) x[(t >> 4) * 4 + (t & 3)] = val;
-            }
-            // T^T row j (MN-major B of MMA-2): elements (j, t) = T[t][j]
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int t0 = 16 * i + 4 * hq;
-                uint2 u = make_uint2(pack2(x[4 * i], x[4 * i + 1]), pack2(x[4 * i + 2], x[4 * i + 3]));
-                *reinterpret_cast<uint2*>(smem + OFF_TT + swe(j, t0)) = u;
+                for (int t = 0; t < 16; ++t) Tf[fidx(base + t, base + c)] = x[t];
+            }
+            __syncthreads();
+            solve_level<1>(A, Tf, tid, lane);
+            __syncthreads();
+            solve_level<2>(A, Tf, tid, lane);
+            __syncthreads();
+            solve_level<3>(A, Tf, tid, lane);
+            __syncthreads();
+            // T^T row j (MN-major B of MMA-2): elements (j, t) = T[t][j]; zero above the
+            // diagonal blocks
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int item = tid + 256 * it;
+                const int j = item >> 3, hc = item & 7;
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 8 * hc + e;
+                    x[e] = ((t >> 4) < (j >> 4)) ? 0.f : Tf[fidx(t, j)];
+                }
+                *reinterpret_cast<uint4*>(smem + OFF_TT + sw(j, hc)) = pack8(x);
             }
             fence_proxy_async();
             tc_fence_before();
@@ -488,9 +571,9 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         float po[8];
+                        unpack8(*reinterpret_cast<const uint4*>(smem + OFF_ARK + sw(tp, c)), po);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            po[e] = v[8 * c + e] + bf16_at(smem + OFF_ARKT, 8 * c + e, tp);
+                        for (int e = 0; e < 8; ++e) po[e] += v[8 * c + e];
                         *reinterpret_cast<uint4*>(smem + OFF_FIN1 + sw(m_row, c)) = pack8(po);
                         *reinterpret_cast<uint4*>(smem + OFF_FIN2 + sw(m_row, c)) = make_uint4(0, 0, 0, 0);
                     }
@@ -525,6 +608,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             float v[32];
             tmem_row<2>(tmem + TM_DF, wq, 32 * wh, v);
             if (state_thread) {
+                const float gamma = gamma_s[m_row];  // e^{g_L} of this state row's channel
 #pragma unroll
                 for (int j = 0; j < 32; ++j) S[j] = fmaf(gamma, S[j], v[j]);
 #pragma unroll
