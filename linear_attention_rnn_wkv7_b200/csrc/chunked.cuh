@@ -125,49 +125,71 @@ __device__ __forceinline__ void tmem_row(uint32_t tmem, int wq, uint32_t col, fl
     sm100::tmem_ld_wait();
 }
 
-// One level L of the blocked triangular inverse: blocks (i, j) = (j + L, j),
-// j = 0 .. 3 - L.  Four threads per output column c, each owning four rows.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// Warp-level D += A * B, m16n8k8, tf32 operands, fp32 accumulate.  Fragment
+// ownership (g = lane / 4, q = lane % 4): A (g|g+8, q|q+4), B (k = q|q+4, n = g),
+// C/D (g|g+8, 2q|2q+1).
+__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 16x16x16 product of fp32 blocks in an fidx tile: acc += X[xr.., xc..] * Y[yr.., yc..].
+__device__ __forceinline__ void block_mma(float (&acc)[2][4], const float* X, int xr, int xc,
+                                          const float* Y, int yr, int yc, int lane) {
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = to_tf32(X[fidx(xr + g, xc + 8 * ks + q)]);
+        const uint32_t a1 = to_tf32(X[fidx(xr + g + 8, xc + 8 * ks + q)]);
+        const uint32_t a2 = to_tf32(X[fidx(xr + g, xc + 8 * ks + q + 4)]);
+        const uint32_t a3 = to_tf32(X[fidx(xr + g + 8, xc + 8 * ks + q + 4)]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = to_tf32(Y[fidx(yr + 8 * ks + q, yc + 8 * nt + g)]);
+            const uint32_t b1 = to_tf32(Y[fidx(yr + 8 * ks + q + 4, yc + 8 * nt + g)]);
+            mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
+        }
+    }
+}
+
+__device__ __forceinline__ void store_block(float* Tf, int r0, int c0, const float (&acc)[2][4],
+                                            int lane) {
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        Tf[fidx(r0 + g, c0 + 8 * nt + 2 * q)] = acc[nt][0];
+        Tf[fidx(r0 + g, c0 + 8 * nt + 2 * q + 1)] = acc[nt][1];
+        Tf[fidx(r0 + g + 8, c0 + 8 * nt + 2 * q)] = acc[nt][2];
+        Tf[fidx(r0 + g + 8, c0 + 8 * nt + 2 * q + 1)] = acc[nt][3];
+    }
+}
+
+// Level L of the blocked inverse on warp-level tensor-core MMAs (tf32 operands,
+// fp32 accumulation): warp j computes block (i, j), i = j + L, as
+// T_ij = T_ii * sum_{m=j}^{i-1} A_im T_mj, staging the sum in block (i, j) itself.
 template <int L>
-__device__ __forceinline__ void solve_level(const float* A, float* Tf, int tid, int lane) {
-    if (tid >= (4 - L) * 64) return;  // whole warps
-    const int j = tid >> 6, i = j + L, c = (tid >> 2) & 15, rq = tid & 3;
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
+__device__ __forceinline__ void solve_level_mma(const float* A, float* Tf, int warp, int lane) {
+    if (warp >= 4 - L) return;
+    const int j = warp, i = j + L;
+    float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int d = 0; d < L; ++d) {
-        const int mb = j + d;  // Y += A_{i,mb} T_{mb,j}[:, c]
-        float tc[16];
-#pragma unroll
-        for (int m = 0; m < 16; ++m) tc[m] = Tf[fidx(16 * mb + m, 16 * j + c)];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int row = 16 * i + 4 * rq + r;
-#pragma unroll
-            for (int m4 = 0; m4 < 16; m4 += 4) {
-                const float4 a4 = *reinterpret_cast<const float4*>(A + fidx(row, 16 * mb + m4));
-                y[r] = fmaf(a4.x, tc[m4], y[r]);
-                y[r] = fmaf(a4.y, tc[m4 + 1], y[r]);
-                y[r] = fmaf(a4.z, tc[m4 + 2], y[r]);
-                y[r] = fmaf(a4.w, tc[m4 + 3], y[r]);
-            }
-        }
-    }
-    float yc[16];  // the whole column Y[:, c], gathered from the four row owners
-#pragma unroll
-    for (int m = 0; m < 16; ++m) yc[m] = __shfl_sync(0xffffffffu, y[m & 3], (lane & ~3) | (m >> 2));
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int row = 16 * i + 4 * rq + r;
-        float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-        for (int m4 = 0; m4 < 16; m4 += 4) {
-            const float4 t4 = *reinterpret_cast<const float4*>(Tf + fidx(row, 16 * i + m4));
-            z0 = fmaf(t4.x, yc[m4], z0);
-            z1 = fmaf(t4.y, yc[m4 + 1], z1);
-            z0 = fmaf(t4.z, yc[m4 + 2], z0);
-            z1 = fmaf(t4.w, yc[m4 + 3], z1);
-        }
-        Tf[fidx(row, 16 * j + c)] = z0 + z1;
-    }
+    for (int d = 0; d < L; ++d) block_mma(y, A, 16 * i, 16 * (j + d), Tf, 16 * (j + d), 16 * j, lane);
+    store_block(Tf, 16 * i, 16 * j, y, lane);
+    __syncwarp();
+    float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    block_mma(z, Tf, 16 * i, 16 * i, Tf, 16 * i, 16 * j, lane);
+    __syncwarp();
+    store_block(Tf, 16 * i, 16 * j, z, lane);
 }
 
 __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int* abort_flag) {
@@ -437,8 +459,8 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             __syncthreads();
         }
 
-        // ---- 6. T = (I - A_ab)^-1 (fp32): 16x16 diagonal blocks by forward substitution,
-        //         then the off-diagonal blocks level by level,
+        // ---- 6. T = (I - A_ab)^-1: 16x16 diagonal blocks by fp32 forward substitution,
+        //         then the off-diagonal blocks level by level on warp MMAs,
         //         T_ij = T_ii * sum_{m=j}^{i-1} A_im T_mj ------------------------------------
         {
             const float* A = reinterpret_cast<const float*>(smem + OFF_AAB);
@@ -466,11 +488,11 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                 for (int t = 0; t < 16; ++t) Tf[fidx(base + t, base + c)] = x[t];
             }
             __syncthreads();
-            solve_level<1>(A, Tf, tid, lane);
+            solve_level_mma<1>(A, Tf, warp, lane);
             __syncthreads();
-            solve_level<2>(A, Tf, tid, lane);
+            solve_level_mma<2>(A, Tf, warp, lane);
             __syncthreads();
-            solve_level<3>(A, Tf, tid, lane);
+            solve_level_mma<3>(A, Tf, warp, lane);
             __syncthreads();
             // T^T row j (MN-major B of MMA-2): elements (j, t) = T[t][j]; zero above the
             // diagonal blocks
