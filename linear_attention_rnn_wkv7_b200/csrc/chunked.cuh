@@ -13,13 +13,16 @@
 //   W = T Abar, Z = T A_ak              (so the read vectors are U = W S0 + Z V)
 //   S_L = diag(e^{g_L}) S0 + (Bhat^T W) S0 + (Khat^T + Bhat^T Z) V
 //   O   = (Rbar + A_rb W) S0 + (A_rk + A_rb Z) V
-// Only the last product depends on S0, so one chunk costs five tcgen05 MMA groups
-// (Gram, W|Z, the two Bhat/A_rb products, final) with everything else on CUDA
-// cores: the prefix sums and exps, the 64x64 triangular solve (fp32) and the
-// TMEM -> shared-memory epilogues that re-layout each result as the next
-// product's operand.  The write term Khat^T + Bhat^T Z enters the final MMA as a
-// hi/lo pair of bf16 matrices (about 16 significant bits), which keeps the fp32
-// final state within 1e-3 of the fp64 recurrence; all other operands are bf16.
+// Only the last product depends on S0.  One chunk costs three tcgen05 MMA groups
+// (the Gram matrix, the Bhat/A_rb products with [W | Z], and the final product
+// with [S0; V]) with fp32 accumulators in tensor memory.  [W | Z] = T [Abar | A_ak]
+// comes from a block forward substitution on warp-level tf32 MMAs (each warp owns
+// 16 of its 128 columns), after the 16x16 diagonal blocks of T by fp32 forward
+// substitution.  CUDA cores do the prefix sums and exps and the tensor-memory ->
+// shared-memory epilogues that re-layout each result as the next product's operand.
+// The write term Khat^T + Bhat^T Z enters the final MMA as a hi/lo pair of bf16
+// matrices (about 16 significant bits), which keeps the fp32 final state within
+// 1e-3 of the fp64 recurrence; all other tensor-core operands are bf16 or tf32.
 //
 // A masked or out-of-range token is folded into the loads as w = a = k = b = 0:
 // its transition is then the identity and it writes nothing, and its output is
@@ -39,36 +42,74 @@ constexpr bool kChunkedBuilt = true;
 namespace chunked {
 
 constexpr int kThreads = 256;
-// Shared-memory map (bytes; every tile 1024-aligned, 64 rows x 128 B, 128B swizzle).
-constexpr uint32_t OFF_R = 0;          // raw r -> r~        (Gram A rows 0..63)
-constexpr uint32_t OFF_A = 8192;       // raw a -> a~        (Gram A rows 64..127)
-constexpr uint32_t OFF_K = 16384;      // raw k -> k~        (Gram B rows 0..63)
-constexpr uint32_t OFF_B = 24576;      // raw b -> b~        (Gram B rows 64..127)
-constexpr uint32_t OFF_W = 32768;      // raw w -> Bhat      (MMA-3 A, MN-major atom 0)
-constexpr uint32_t OFF_V = 40960;      // raw v              (final MMA B, MN-major)
-constexpr uint32_t OFF_ABAR = 49152;   // Abar [s][k]        (MMA-2 A, MN-major atom 0)
-constexpr uint32_t OFF_AAK = 57344;    // A_ak [s][s']       (MMA-2 A, MN-major atom 1)
-constexpr uint32_t OFF_ARBT = 65536;   // A_rb^T [s][t]      (MMA-3 A, MN-major atom 1)
-constexpr uint32_t OFF_ARK = 73728;    // A_rk [t][s]        (epilogue 3); prologue scratch
-constexpr uint32_t OFF_RBAR = 81920;   // Rbar [t][k]        (epilogue 3)
-constexpr uint32_t OFF_S0 = 90112;     // S0 bf16 [k][v]     (final MMA B, MN-major)
-constexpr uint32_t OFF_F0 = 98304;     // fp32 64x64: E_t, then Khat [s][k]
-constexpr uint32_t OFF_MISC = 114688;  // mbarriers, TMEM address, abort flag
+// Shared-memory map.  Fourteen 8 KB tiles (64 rows x 128 B, 1024-aligned, 128B
+// swizzle) plus a small control block.  Consecutive chunks alternate between two
+// layouts of the same tiles, so that the next chunk's six input tiles can be
+// loaded by TMA into tiles this chunk no longer needs while its final MMA runs.
+constexpr uint32_t kTile = 8192;
+constexpr uint32_t OFF_S0 = 11 * kTile;    // S0 bf16 [k][v] (final MMA B, MN-major), both layouts
+constexpr uint32_t OFF_MISC = 14 * kTile;  // mbarriers, TMEM address, abort flag
 constexpr uint32_t OFF_GAMMA = OFF_MISC + 64;  // e^{g_L} per channel (64 fp32)
 constexpr uint32_t kSmemBytes = OFF_GAMMA + 256;
-// Aliases (lifetimes do not overlap).
-constexpr uint32_t OFF_AAB = OFF_R;    // fp32 A_ab [t][s] (epilogue 1 -> solve), 16 KB
-constexpr uint32_t OFF_TF = OFF_K;     // fp32 T [t][s]    (solve), 16 KB
-constexpr uint32_t OFF_TT = OFF_R;     // T^T [s][t]      (solve -> MMA-2 B, MN-major)
-constexpr uint32_t OFF_WZT = OFF_K;    // [W^T; Z^T] [n][t] 128 rows (MMA-3 B, K-major)
-constexpr uint32_t OFF_FIN0 = OFF_R;   // final A, K block 0: [M'; Rbar + A_rb W]
-constexpr uint32_t OFF_FIN1 = OFF_ABAR;// final A, K block 1: [P_N hi; A_rk + A_rb Z]
-constexpr uint32_t OFF_FIN2 = OFF_K;   // final A, K block 2: [P_N lo; 0]
+
+template <int P>
+struct Lay;
+// Even chunks.
+template <>
+struct Lay<0> {
+    static constexpr uint32_t R = 0 * kTile;      // raw r -> r~   (Gram A rows 0..63)
+    static constexpr uint32_t A = 1 * kTile;      // raw a -> a~   (Gram A rows 64..127)
+    static constexpr uint32_t K = 2 * kTile;      // raw k -> k~   (Gram B rows 0..63)
+    static constexpr uint32_t B = 3 * kTile;      // raw b -> b~   (Gram B rows 64..127)
+    static constexpr uint32_t W = 4 * kTile;      // raw w -> Bhat (MMA-3 A, MN-major atom 0)
+    static constexpr uint32_t V = 5 * kTile;      // raw v         (final MMA B, MN-major)
+    static constexpr uint32_t ABAR = 6 * kTile;   // Abar [s][k] -> W [t][k]  (MMA-3 B, MN-major atom 0)
+    static constexpr uint32_t AAK = 7 * kTile;    // A_ak [s][s'] -> Z [t][s'] (MMA-3 B, MN-major atom 1)
+    static constexpr uint32_t ARBT = 8 * kTile;   // A_rb^T [s][t] (MMA-3 A, MN-major atom 1)
+    static constexpr uint32_t ARK = 9 * kTile;    // A_rk [t][s] (epilogue 3); prologue scratch
+    static constexpr uint32_t RBAR = 10 * kTile;  // Rbar [t][k] (epilogue 3)
+    static constexpr uint32_t F0 = 12 * kTile;    // fp32 64x64 (2 tiles): E_t, then Khat [s][k]
+};
+// Odd chunks: the six input tiles land in tiles the even layout no longer needs
+// once its epilogue 3 is done (Bhat, A_rb^T, A_rk, Rbar, Khat), and vice versa.
+template <>
+struct Lay<1> {
+    static constexpr uint32_t R = 12 * kTile;
+    static constexpr uint32_t A = 13 * kTile;
+    static constexpr uint32_t K = 8 * kTile;
+    static constexpr uint32_t B = 9 * kTile;
+    static constexpr uint32_t W = 4 * kTile;
+    static constexpr uint32_t V = 10 * kTile;
+    static constexpr uint32_t ABAR = 6 * kTile;
+    static constexpr uint32_t AAK = 7 * kTile;
+    static constexpr uint32_t ARBT = 5 * kTile;
+    static constexpr uint32_t ARK = 0 * kTile;
+    static constexpr uint32_t RBAR = 1 * kTile;
+    static constexpr uint32_t F0 = 2 * kTile;
+};
+// The two layouts as run-time offsets (one copy of the chunk code keeps the
+// kernel's instruction footprint small).
+struct LayR {
+    uint32_t R, A, K, B, W, V, ABAR, AAK, ARBT, ARK, RBAR, F0;
+};
+template <int P>
+__device__ __forceinline__ LayR lay_const() {
+    return LayR{Lay<P>::R,    Lay<P>::A,   Lay<P>::K,    Lay<P>::B,   Lay<P>::W,    Lay<P>::V,
+                Lay<P>::ABAR, Lay<P>::AAK, Lay<P>::ARBT, Lay<P>::ARK, Lay<P>::RBAR, Lay<P>::F0};
+}
+__device__ __forceinline__ LayR lay_of(int par) {
+    return par ? lay_const<1>() : lay_const<0>();
+}
+// Aliases inside one chunk (lifetimes do not overlap):
+//   fp32 A_ab [t][s]     R (2 tiles)   epilogue 1 -> W|Z substitution
+//   fp32 T_ii + scratch  K (2 tiles)   W|Z substitution
+//   [M'; Rbar + A_rb W]  R (2 tiles)   epilogue 3 -> final MMA A, K block 0
+//   [P_N hi; A_rk+A_rb Z] ABAR (2)     epilogue 3 -> final MMA A, K block 1
+//   [P_N lo; 0]          K (2 tiles)   epilogue 3 -> final MMA A, K block 2
 // Prologue scratch inside the A_rk tile (free until epilogue 1), in floats.
 constexpr int SCR_TOT = 0, SCR_EC = 512, SCR_EMC = 576, SCR_ELC = 640, SCR_VALID = 704;
 // Tensor-memory columns (fp32 accumulators, 128 lanes).
 constexpr uint32_t TM_D1 = 0;    // Gram, later MMA-3 (128 cols)
-constexpr uint32_t TM_D2 = 128;  // [W^T; Z^T] (64 cols)
 constexpr uint32_t TM_DF = 192;  // [S update; O] (64 cols)
 constexpr uint32_t kTmemCols = 256;
 constexpr float kExpClamp = 40.f;
@@ -143,55 +184,6 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 16x16x16 product of fp32 blocks in an fidx tile: acc += X[xr.., xc..] * Y[yr.., yc..].
-__device__ __forceinline__ void block_mma(float (&acc)[2][4], const float* X, int xr, int xc,
-                                          const float* Y, int yr, int yc, int lane) {
-    const int g = lane >> 2, q = lane & 3;
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t a0 = to_tf32(X[fidx(xr + g, xc + 8 * ks + q)]);
-        const uint32_t a1 = to_tf32(X[fidx(xr + g + 8, xc + 8 * ks + q)]);
-        const uint32_t a2 = to_tf32(X[fidx(xr + g, xc + 8 * ks + q + 4)]);
-        const uint32_t a3 = to_tf32(X[fidx(xr + g + 8, xc + 8 * ks + q + 4)]);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const uint32_t b0 = to_tf32(Y[fidx(yr + 8 * ks + q, yc + 8 * nt + g)]);
-            const uint32_t b1 = to_tf32(Y[fidx(yr + 8 * ks + q + 4, yc + 8 * nt + g)]);
-            mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
-        }
-    }
-}
-
-__device__ __forceinline__ void store_block(float* Tf, int r0, int c0, const float (&acc)[2][4],
-                                            int lane) {
-    const int g = lane >> 2, q = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        Tf[fidx(r0 + g, c0 + 8 * nt + 2 * q)] = acc[nt][0];
-        Tf[fidx(r0 + g, c0 + 8 * nt + 2 * q + 1)] = acc[nt][1];
-        Tf[fidx(r0 + g + 8, c0 + 8 * nt + 2 * q)] = acc[nt][2];
-        Tf[fidx(r0 + g + 8, c0 + 8 * nt + 2 * q + 1)] = acc[nt][3];
-    }
-}
-
-// Level L of the blocked inverse on warp-level tensor-core MMAs (tf32 operands,
-// fp32 accumulation): warp j computes block (i, j), i = j + L, as
-// T_ij = T_ii * sum_{m=j}^{i-1} A_im T_mj, staging the sum in block (i, j) itself.
-template <int L>
-__device__ __forceinline__ void solve_level_mma(const float* A, float* Tf, int warp, int lane) {
-    if (warp >= 4 - L) return;
-    const int j = warp, i = j + L;
-    float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int d = 0; d < L; ++d) block_mma(y, A, 16 * i, 16 * (j + d), Tf, 16 * (j + d), 16 * j, lane);
-    store_block(Tf, 16 * i, 16 * j, y, lane);
-    __syncwarp();
-    float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    block_mma(z, Tf, 16 * i, 16 * i, Tf, 16 * i, 16 * j, lane);
-    __syncwarp();
-    store_block(Tf, 16 * i, 16 * j, z, lane);
-}
-
 __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int* abort_flag) {
     if (!sm100::mbar_wait(bar, parity)) {
         raise_flag(4 /* WKV7_ERR_DEVICE_TIMEOUT */);
@@ -199,95 +191,60 @@ __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
-chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
-               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-               const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
-               float* sT, int T, int H, const int32_t* __restrict__ cu_seqlens) {
-    extern __shared__ __align__(1024) uint8_t smem[];
+// Everything one CTA keeps for its (sequence, head) between chunks.
+struct Ctx {
+    uint8_t* smem;
+    uint32_t sbase, tmem, bar_tma, bar_mma, mma_phase;
+    int tid, warp, lane, wq, wh, m_row, h, H;
+    bool state_thread;
+    long long row0;  // token row of the sequence start
+    int len;
+    const uint8_t* mask;
+    __nv_bfloat16* o;
+    int* abort_flag;
+    float* gamma_s;
+    const CUtensorMap *tm_r, *tm_w, *tm_k, *tm_v, *tm_a, *tm_b;
+};
+
+// Lanes 0..5 of the calling warp: request the six 64 x 64 bf16 input tiles of the chunk
+// starting at token c0 into layout `par` (lane 0 arms the barrier first; the
+// six copies are issued in parallel).
+__device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
+    const LayR L = lay_of(par);
     using namespace sm100;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
-    const uint32_t sbase = smem_u32(smem);
-    if (sbase & 1023u) {  // the swizzled tiles need a 1024-byte aligned base
-        if (tid == 0) raise_flag(3 /* WKV7_ERR_CUDA */);
-        return;
+    const int lane = cx.lane;
+    if (lane == 0) mbar_arrive_expect_tx(cx.bar_tma, 6 * kTile);
+    __syncwarp();
+    const int row = (int)(cx.row0 + c0);
+    if (lane < 6) {
+        const CUtensorMap* map = lane == 0 ? cx.tm_r : lane == 1 ? cx.tm_a : lane == 2 ? cx.tm_k
+                               : lane == 3 ? cx.tm_b : lane == 4 ? cx.tm_w : cx.tm_v;
+        const uint32_t dst = lane == 0 ? L.R : lane == 1 ? L.A : lane == 2 ? L.K
+                           : lane == 3 ? L.B : lane == 4 ? L.W : L.V;
+        tma_load_3d(cx.sbase + dst, map, cx.bar_tma, 0, cx.h, row);
     }
-    const int h = blockIdx.x % H;
-    const int n = blockIdx.x / H;
-    int bb = n, bos = 0, eos = T;
-    if (cu_seqlens) {
-        bb = 0;
-        bos = cu_seqlens[n];
-        eos = cu_seqlens[n + 1];
-        if (bos < 0 || eos < bos || eos > T) {
-            if (tid == 0) raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
-            return;
-        }
-    }
-    const int len = eos - bos;
-    const long long row0 = (long long)bb * T + bos;  // token row of the sequence start
+}
 
-    const uint32_t bar_tma = sbase + OFF_MISC, bar_mma = sbase + OFF_MISC + 8;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 16);
-    int* abort_flag = reinterpret_cast<int*>(smem + OFF_MISC + 20);
-    if (warp == 0) {
-        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-        tmem_relinquish();
-    }
-    if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(bar_mma, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    // State rows: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
-    // [32*wh, 32*wh + 32), in fp32 registers for the whole sequence.
-    const bool state_thread = wq < 2;
-    const int m_row = 32 * wq + lane;
-    const size_t state_off = ((size_t)n * H + h) * 4096;
-    float S[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) S[j] = 0.f;
-    if (state_thread) {
-        if (s0) {
-            const float4* src = reinterpret_cast<const float4*>(s0 + state_off + m_row * 64 + 32 * wh);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 f = src[j];
-                S[4 * j] = f.x; S[4 * j + 1] = f.y; S[4 * j + 2] = f.z; S[4 * j + 3] = f.w;
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(S + 8 * c);
-    }
-    float* scratch = reinterpret_cast<float*>(smem + OFF_ARK);  // prologue only
+// One 64-token chunk starting at token c0, in layout P (its inputs already requested).
+__device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_next, int par) {
+    const LayR L = lay_of(par);
+    using namespace sm100;
+    uint8_t* smem = cx.smem;
+    const uint32_t sbase = cx.sbase, tmem = cx.tmem, bar_mma = cx.bar_mma;
+    const int tid = cx.tid, warp = cx.warp, lane = cx.lane, wq = cx.wq, wh = cx.wh;
+    const int m_row = cx.m_row, H = cx.H, h = cx.h;
+    const bool state_thread = cx.state_thread;
+    const long long row0 = cx.row0;
+    const uint8_t* mask = cx.mask;
+    __nv_bfloat16* o = cx.o;
+    int* abort_flag = cx.abort_flag;
+    float* gamma_s = cx.gamma_s;
+    uint32_t& mma_phase = cx.mma_phase;
+    float* scratch = reinterpret_cast<float*>(smem + L.ARK);  // prologue only
     uint8_t* validb = reinterpret_cast<uint8_t*>(scratch + SCR_VALID);
-    float* F0 = reinterpret_cast<float*>(smem + OFF_F0);
-    float* gamma_s = reinterpret_cast<float*>(smem + OFF_GAMMA);
-    uint32_t mma_phase = 0;
-    int iter = 0;
-    for (int c0 = 0; c0 < len; c0 += 64, ++iter) {
-        const int nv = min(64, len - c0);
-        // ---- 1. TMA: the chunk's six 64 x 64 bf16 tiles ------------------------------
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar_tma, 6 * 8192);
-            const int row = (int)(row0 + c0);
-            tma_load_3d(sbase + OFF_R, &tm_r, bar_tma, 0, h, row);
-            tma_load_3d(sbase + OFF_A, &tm_a, bar_tma, 0, h, row);
-            tma_load_3d(sbase + OFF_K, &tm_k, bar_tma, 0, h, row);
-            tma_load_3d(sbase + OFF_B, &tm_b, bar_tma, 0, h, row);
-            tma_load_3d(sbase + OFF_W, &tm_w, bar_tma, 0, h, row);
-            tma_load_3d(sbase + OFF_V, &tm_v, bar_tma, 0, h, row);
-        }
-        wait_or_abort(bar_tma, iter & 1, abort_flag);
+    float* F0 = reinterpret_cast<float*>(smem + L.F0);
+    const int nv = min(64, cx.len - c0);
+    wait_or_abort(cx.bar_tma, par, abort_flag);
 
         // ---- 2. prefix sums of w (mask folded), E_t = e^{g_t - c} ------------------------
         {
@@ -299,7 +256,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                 const int t = 8 * q + i;
                 const bool val = t < nv && (!mask || mask[row0 + c0 + t] != 0);
                 const float2 wv = __bfloat1622float2(
-                    *reinterpret_cast<const __nv_bfloat162*>(smem + OFF_W + swe(t, 2 * p)));
+                    *reinterpret_cast<const __nv_bfloat162*>(smem + L.W + swe(t, 2 * p)));
                 acc.x += val ? wv.x : 0.f;
                 acc.y += val ? wv.y : 0.f;
                 gl[i] = acc;
@@ -343,10 +300,10 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                 const bool val = validb[t] != 0;
                 const uint32_t off = sw(t, j);
                 float rv[8], av[8], kv[8], bv[8];
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_R + off), rv);
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_A + off), av);
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_K + off), kv);
-                unpack8(*reinterpret_cast<const uint4*>(smem + OFF_B + off), bv);
+                unpack8(*reinterpret_cast<const uint4*>(smem + L.R + off), rv);
+                unpack8(*reinterpret_cast<const uint4*>(smem + L.A + off), av);
+                unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv);
+                unpack8(*reinterpret_cast<const uint4*>(smem + L.B + off), bv);
                 float E[8], Em[8], ec[8], elc[8];
                 const float* Erow = F0 + t * 64 + 8 * j;
                 const float* Emrow = t > 0 ? F0 + (t - 1) * 64 + 8 * j : scratch + SCR_EMC + 8 * j;
@@ -373,13 +330,13 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                     khat[e] = k_ * elc[e] * inv;
                     rbar[e] = rt[e] * ec[e];
                 }
-                *reinterpret_cast<uint4*>(smem + OFF_R + off) = pack8(rt);
-                *reinterpret_cast<uint4*>(smem + OFF_A + off) = pack8(at);
-                *reinterpret_cast<uint4*>(smem + OFF_K + off) = pack8(kt);
-                *reinterpret_cast<uint4*>(smem + OFF_B + off) = pack8(btl);
-                *reinterpret_cast<uint4*>(smem + OFF_W + off) = pack8(bhat);
-                *reinterpret_cast<uint4*>(smem + OFF_ABAR + off) = pack8(abar);
-                *reinterpret_cast<uint4*>(smem + OFF_RBAR + off) = pack8(rbar);
+                *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rt);
+                *reinterpret_cast<uint4*>(smem + L.A + off) = pack8(at);
+                *reinterpret_cast<uint4*>(smem + L.K + off) = pack8(kt);
+                *reinterpret_cast<uint4*>(smem + L.B + off) = pack8(btl);
+                *reinterpret_cast<uint4*>(smem + L.W + off) = pack8(bhat);
+                *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8(abar);
+                *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8(rbar);
                 o_khat[it][0] = make_float4(khat[0], khat[1], khat[2], khat[3]);
                 o_khat[it][1] = make_float4(khat[4], khat[5], khat[6], khat[7]);
             }
@@ -403,8 +360,8 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             constexpr uint32_t id = idesc_bf16(128, 128, false, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_D1, smem_desc(sbase + OFF_R + 32 * kk, 16, 1024),
-                          smem_desc(sbase + OFF_K + 32 * kk, 16, 1024), id, kk > 0);
+                umma_bf16(tmem + TM_D1, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
+                          smem_desc(sbase + L.K + 32 * kk, 16, 1024), id, kk > 0);
             umma_commit(bar_mma);
         }
         wait_or_abort(bar_mma, mma_phase, abort_flag);
@@ -423,12 +380,12 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                         float x[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
-                        *reinterpret_cast<uint4*>(smem + OFF_ARK + sw(t, c)) = pack8(x);
+                        *reinterpret_cast<uint4*>(smem + L.ARK + sw(t, c)) = pack8(x);
                     }
                 } else {  // A_rb[t][s] = v[s], kept for s <= t -> column t of A_rb^T
 #pragma unroll
                     for (int s_ = 0; s_ < 64; ++s_)
-                        *reinterpret_cast<__nv_bfloat16*>(smem + OFF_ARBT + swe(s_, t)) =
+                        *reinterpret_cast<__nv_bfloat16*>(smem + L.ARBT + swe(s_, t)) =
                             __float2bfloat16_rn(s_ <= t ? v[s_] : 0.f);
                 }
             } else {
@@ -439,10 +396,10 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                         float x[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
-                        *reinterpret_cast<uint4*>(smem + OFF_AAK + sw(t, c)) = pack8(x);
+                        *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8(x);
                     }
                 } else {  // A_ab[t][s], kept for s < t -> fp32 row t
-                    float* aab = reinterpret_cast<float*>(smem + OFF_AAB);
+                    float* aab = reinterpret_cast<float*>(smem + L.R);
 #pragma unroll
                     for (int c4 = 0; c4 < 16; ++c4) {
                         float4 x;
@@ -459,12 +416,16 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             __syncthreads();
         }
 
-        // ---- 6. T = (I - A_ab)^-1: 16x16 diagonal blocks by fp32 forward substitution,
-        //         then the off-diagonal blocks level by level on warp MMAs,
-        //         T_ij = T_ii * sum_{m=j}^{i-1} A_im T_mj ------------------------------------
+        // ---- 6. [W | Z] = T [Abar | A_ak], T = (I - A_ab)^-1, by block forward
+        //         substitution over four 16-row blocks:
+        //             X_i = T_ii (RHS_i + sum_{m<i} A_im X_m).
+        //         The 16x16 diagonal inverses T_ii come from fp32 forward substitution;
+        //         then each warp solves its own 16 of the 128 right-hand-side columns
+        //         with warp-level tf32 MMAs, writing X in place over the right-hand
+        //         side (bf16), where MMA-3 reads it as its MN-major B operand ---------
         {
-            const float* A = reinterpret_cast<const float*>(smem + OFF_AAB);
-            float* Tf = reinterpret_cast<float*>(smem + OFF_TF);
+            const float* A = reinterpret_cast<const float*>(smem + L.R);  // A_ab [t][s]
+            float* Td = reinterpret_cast<float*>(smem + L.K);             // T_bb, rows of 20
             if (tid < 64) {  // diagonal block b, column c
                 const int b = tid >> 4, c = tid & 15, base = 16 * b;
                 float x[16];
@@ -485,75 +446,95 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                     x[t] = (t == c) ? 1.f : acc0 + acc1;
                 }
 #pragma unroll
-                for (int t = 0; t < 16; ++t) Tf[fidx(base + t, base + c)] = x[t];
+                for (int t = 0; t < 16; ++t) Td[(base + t) * 20 + c] = x[t];
             }
             __syncthreads();
-            solve_level_mma<1>(A, Tf, warp, lane);
-            __syncthreads();
-            solve_level_mma<2>(A, Tf, warp, lane);
-            __syncthreads();
-            solve_level_mma<3>(A, Tf, warp, lane);
-            __syncthreads();
-            // T^T row j (MN-major B of MMA-2): elements (j, t) = T[t][j]; zero above the
-            // diagonal blocks
+            const int g = lane >> 2, q = lane & 3;
+            uint8_t* xt = smem + (warp < 4 ? L.ABAR : L.AAK);  // tile of this warp's columns
+            const int nc = 16 * (warp & 3);                    // first column inside it
+            float* ys = reinterpret_cast<float*>(smem + L.K + 5120) + warp * 320;  // 16 x 20
 #pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int item = tid + 256 * it;
-                const int j = item >> 3, hc = item & 7;
-                float x[8];
+            for (int i = 0; i < 4; ++i) {
+                float y[2][4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int t = 8 * hc + e;
-                    x[e] = ((t >> 4) < (j >> 4)) ? 0.f : Tf[fidx(t, j)];
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int col = nc + 8 * nt + 2 * q;
+                    const float2 lo = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162*>(xt + swe(16 * i + g, col)));
+                    const float2 hi = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162*>(xt + swe(16 * i + g + 8, col)));
+                    y[nt][0] = lo.x; y[nt][1] = lo.y; y[nt][2] = hi.x; y[nt][3] = hi.y;
                 }
-                *reinterpret_cast<uint4*>(smem + OFF_TT + sw(j, hc)) = pack8(x);
+#pragma unroll
+                for (int m = 0; m < i; ++m) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const int ac = 16 * m + 8 * ks + q;
+                        const uint32_t a0 = to_tf32(A[fidx(16 * i + g, ac)]);
+                        const uint32_t a1 = to_tf32(A[fidx(16 * i + g + 8, ac)]);
+                        const uint32_t a2 = to_tf32(A[fidx(16 * i + g, ac + 4)]);
+                        const uint32_t a3 = to_tf32(A[fidx(16 * i + g + 8, ac + 4)]);
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt) {
+                            const int col = nc + 8 * nt + g;
+                            const uint32_t b0 = to_tf32(bf16_at(xt, 16 * m + 8 * ks + q, col));
+                            const uint32_t b1 = to_tf32(bf16_at(xt, 16 * m + 8 * ks + q + 4, col));
+                            mma_tf32(y[nt], a0, a1, a2, a3, b0, b1);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    ys[g * 20 + 8 * nt + 2 * q] = y[nt][0];
+                    ys[g * 20 + 8 * nt + 2 * q + 1] = y[nt][1];
+                    ys[(g + 8) * 20 + 8 * nt + 2 * q] = y[nt][2];
+                    ys[(g + 8) * 20 + 8 * nt + 2 * q + 1] = y[nt][3];
+                }
+                __syncwarp();
+                float xo[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    const float* tr = Td + (16 * i) * 20 + 8 * ks + q;
+                    const uint32_t a0 = to_tf32(tr[g * 20]);
+                    const uint32_t a1 = to_tf32(tr[(g + 8) * 20]);
+                    const uint32_t a2 = to_tf32(tr[g * 20 + 4]);
+                    const uint32_t a3 = to_tf32(tr[(g + 8) * 20 + 4]);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const uint32_t b0 = to_tf32(ys[(8 * ks + q) * 20 + 8 * nt + g]);
+                        const uint32_t b1 = to_tf32(ys[(8 * ks + q + 4) * 20 + 8 * nt + g]);
+                        mma_tf32(xo[nt], a0, a1, a2, a3, b0, b1);
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int col = nc + 8 * nt + 2 * q;
+                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g, col)) = pack2(xo[nt][0], xo[nt][1]);
+                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g + 8, col)) = pack2(xo[nt][2], xo[nt][3]);
+                }
+                __syncwarp();
             }
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
         }
 
-        // ---- 7. MMA-2: [W^T; Z^T] = [Abar^T; A_ak^T] T^T  (128 x 64 x 64) -----------------
+        // ---- 7. MMA-3: [Bhat^T; A_rb] [W | Z]  (128 x 128 x 64) ----------------------------
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+            constexpr uint32_t id = idesc_bf16(128, 128, true, true);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_D2, smem_desc(sbase + OFF_ABAR + 2048 * kk, OFF_AAK - OFF_ABAR, 1024),
-                          smem_desc(sbase + OFF_TT + 2048 * kk, 8192, 1024), id, kk > 0);
+                umma_bf16(tmem + TM_D1, smem_desc(sbase + L.W + 2048 * kk, L.ARBT - L.W, 1024),
+                          smem_desc(sbase + L.ABAR + 2048 * kk, L.AAK - L.ABAR, 1024), id, kk > 0);
             umma_commit(bar_mma);
         }
         wait_or_abort(bar_mma, mma_phase, abort_flag);
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 8. epilogue 2: [W^T; Z^T] -> bf16 K-major B of MMA-3 ---------------------------
-        {
-            float v[32];
-            tmem_row<2>(tmem + TM_D2, wq, 32 * wh, v);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<uint4*>(smem + OFF_WZT + sw(m_row, 4 * wh + c)) = pack8(v + 8 * c);
-            fence_proxy_async();
-            tc_fence_before();
-            __syncthreads();
-        }
-
-        // ---- 9. MMA-3: [Bhat^T; A_rb] [W | Z]  (128 x 128 x 64) ----------------------------
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 128, true, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_D1, smem_desc(sbase + OFF_W + 2048 * kk, OFF_ARBT - OFF_W, 1024),
-                          smem_desc(sbase + OFF_WZT + 32 * kk, 16, 1024), id, kk > 0);
-            umma_commit(bar_mma);
-        }
-        wait_or_abort(bar_mma, mma_phase, abort_flag);
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- 10. epilogue 3: assemble the final A operand ---------------------------------
+        // ---- 8. epilogue 3: assemble the final A operand ---------------------------------
         {
             float v[64];
             tmem_row<4>(tmem + TM_D1, wq, 64 * wh, v);
@@ -562,7 +543,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                 if (wh == 0) {  // M' = Bhat^T W
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(smem + OFF_FIN0 + sw(k, c)) = pack8(v + 8 * c);
+                        *reinterpret_cast<uint4*>(smem + L.R + sw(k, c)) = pack8(v + 8 * c);
                 } else {  // P_N = Bhat^T Z + Khat^T, split into bf16 hi + lo
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -574,8 +555,8 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                             hi[e] = __bfloat162float(__float2bfloat16_rn(p));
                             lo[e] = p - hi[e];
                         }
-                        *reinterpret_cast<uint4*>(smem + OFF_FIN1 + sw(k, c)) = pack8(hi);
-                        *reinterpret_cast<uint4*>(smem + OFF_FIN2 + sw(k, c)) = pack8(lo);
+                        *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, c)) = pack8(hi);
+                        *reinterpret_cast<uint4*>(smem + L.K + sw(k, c)) = pack8(lo);
                     }
                 }
             } else {
@@ -584,20 +565,20 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         float rb[8];
-                        unpack8(*reinterpret_cast<const uint4*>(smem + OFF_RBAR + sw(tp, c)), rb);
+                        unpack8(*reinterpret_cast<const uint4*>(smem + L.RBAR + sw(tp, c)), rb);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) rb[e] += v[8 * c + e];
-                        *reinterpret_cast<uint4*>(smem + OFF_FIN0 + sw(m_row, c)) = pack8(rb);
+                        *reinterpret_cast<uint4*>(smem + L.R + sw(m_row, c)) = pack8(rb);
                     }
                 } else {  // P_O = A_rb Z + A_rk; the lo block is zero for these rows
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         float po[8];
-                        unpack8(*reinterpret_cast<const uint4*>(smem + OFF_ARK + sw(tp, c)), po);
+                        unpack8(*reinterpret_cast<const uint4*>(smem + L.ARK + sw(tp, c)), po);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) po[e] += v[8 * c + e];
-                        *reinterpret_cast<uint4*>(smem + OFF_FIN1 + sw(m_row, c)) = pack8(po);
-                        *reinterpret_cast<uint4*>(smem + OFF_FIN2 + sw(m_row, c)) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(smem + L.ABAR + sw(m_row, c)) = pack8(po);
+                        *reinterpret_cast<uint4*>(smem + L.K + sw(m_row, c)) = make_uint4(0, 0, 0, 0);
                     }
                 }
             }
@@ -606,14 +587,18 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             __syncthreads();
         }
 
-        // ---- 11. final MMA: [S upd; O] = A_fin [S0; V; V]  (128 x 64 x 192) --------------
+        // The next chunk's inputs go to the other layout's input tiles, all of which
+        // are dead now; the copy overlaps this chunk's final MMA and epilogue.
+        if (has_next && warp == 1) issue_loads(cx, c0 + 64, par ^ 1);
+
+        // ---- 9. final MMA: [S upd; O] = A_fin [S0; V; V]  (128 x 64 x 192) --------------
         if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
             for (int blk = 0; blk < 3; ++blk) {
-                const uint32_t aoff = blk == 0 ? OFF_FIN0 : (blk == 1 ? OFF_FIN1 : OFF_FIN2);
-                const uint32_t boff = blk == 0 ? OFF_S0 : OFF_V;
+                const uint32_t aoff = blk == 0 ? L.R : (blk == 1 ? L.ABAR : L.K);
+                const uint32_t boff = blk == 0 ? OFF_S0 : L.V;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem + TM_DF, smem_desc(sbase + aoff + 32 * kk, 16, 1024),
@@ -625,7 +610,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 12. epilogue 4: state carry (fp32) and the chunk's outputs ---------------------
+        // ---- 10. epilogue 4: state carry (fp32) and the chunk's outputs ---------------------
         {
             float v[32];
             tmem_row<2>(tmem + TM_DF, wq, 32 * wh, v);
@@ -648,19 +633,125 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             tc_fence_before();
             __syncthreads();
         }
-        if (*abort_flag) break;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
+               float* sT, int T, int H, const int32_t* __restrict__ cu_seqlens) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    using namespace sm100;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
+    const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {  // the swizzled tiles need a 1024-byte aligned base
+        if (tid == 0) raise_flag(3 /* WKV7_ERR_CUDA */);
+        return;
+    }
+    const int h = blockIdx.x % H;
+    const int n = blockIdx.x / H;
+    int bb = n, bos = 0, eos = T;
+    if (cu_seqlens) {
+        bb = 0;
+        bos = cu_seqlens[n];
+        eos = cu_seqlens[n + 1];
+        if (bos < 0 || eos < bos || eos > T) {
+            if (tid == 0) raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
+            return;
+        }
     }
 
-    if (state_thread && sT && !*abort_flag) {
+    Ctx cx;
+    cx.smem = smem;
+    cx.sbase = sbase;
+    cx.bar_tma = sbase + OFF_MISC;
+    cx.bar_mma = sbase + OFF_MISC + 8;
+    cx.mma_phase = 0;
+    cx.tid = tid;
+    cx.warp = warp;
+    cx.lane = lane;
+    cx.wq = wq;
+    cx.wh = wh;
+    cx.m_row = 32 * wq + lane;
+    cx.h = h;
+    cx.H = H;
+    cx.state_thread = wq < 2;
+    cx.row0 = (long long)bb * T + bos;
+    cx.len = eos - bos;
+    cx.mask = mask;
+    cx.o = o;
+    cx.abort_flag = reinterpret_cast<int*>(smem + OFF_MISC + 20);
+    cx.gamma_s = reinterpret_cast<float*>(smem + OFF_GAMMA);
+    cx.tm_r = &tm_r;
+    cx.tm_w = &tm_w;
+    cx.tm_k = &tm_k;
+    cx.tm_v = &tm_v;
+    cx.tm_a = &tm_a;
+    cx.tm_b = &tm_b;
+
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 16);
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(cx.bar_tma, 1);
+        mbar_init(cx.bar_mma, 1);
+        *cx.abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cx.tmem = *tmem_slot;
+    if (warp == 0 && lane < 6)
+        prefetch_tensormap(lane == 0 ? &tm_r : lane == 1 ? &tm_a : lane == 2 ? &tm_k
+                           : lane == 3 ? &tm_b : lane == 4 ? &tm_w : &tm_v);
+    if (warp == 0 && cx.len > 0) issue_loads(cx, 0, 0);
+
+    // State rows: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
+    // [32*wh, 32*wh + 32), in fp32 registers for the whole sequence.
+    const int m_row = cx.m_row;
+    const size_t state_off = ((size_t)n * H + h) * 4096;
+    float S[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) S[j] = 0.f;
+    if (cx.state_thread) {
+        if (s0) {
+            const float4* src = reinterpret_cast<const float4*>(s0 + state_off + m_row * 64 + 32 * wh);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 f = src[j];
+                S[4 * j] = f.x;
+                S[4 * j + 1] = f.y;
+                S[4 * j + 2] = f.z;
+                S[4 * j + 3] = f.w;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(S + 8 * c);
+    }
+
+    // Chunks alternate between the two shared-memory layouts.
+    for (int c0 = 0, par = 0; c0 < cx.len; c0 += 64, par ^= 1) {
+        chunk(cx, S, c0, c0 + 64 < cx.len, par);
+        if (*cx.abort_flag) break;
+    }
+
+    if (cx.state_thread && sT && !*cx.abort_flag) {
         float4* dst = reinterpret_cast<float4*>(sT + state_off + m_row * 64 + 32 * wh);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+        for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(cx.tmem, kTmemCols);
     }
 }
 
