@@ -110,6 +110,7 @@ __device__ __forceinline__ LayR lay_of(int par) {
 constexpr int SCR_TOT = 0, SCR_EC = 512, SCR_EMC = 576, SCR_ELC = 640, SCR_VALID = 704;
 // Tensor-memory columns (fp32 accumulators, 128 lanes).
 constexpr uint32_t TM_D1 = 0;    // Gram, later MMA-3 (128 cols)
+constexpr uint32_t TM_D1B = 128; // A_rb^T = b~ r~^T (64 cols)
 constexpr uint32_t TM_DF = 192;  // [S update; O] (64 cols)
 constexpr uint32_t kTmemCols = 256;
 constexpr float kExpClamp = 40.f;
@@ -124,10 +125,10 @@ __device__ __forceinline__ uint32_t swe(uint32_t row, uint32_t col) {
 }
 
 // Float index of (row, col) in a 64x64 fp32 tile whose 16-byte chunks are permuted
-// within each 64-byte group by bits 2..3 of the row, so that four rows 4 apart
-// read with float4 loads hit different banks.
+// by the low three bits of the row, so that eight consecutive rows written or
+// read at the same column hit different banks.
 __device__ __forceinline__ int fidx(int row, int col) {
-    return row * 64 + ((((col >> 2) ^ ((row >> 2) & 3)) << 2) | (col & 3));
+    return row * 64 + ((((col >> 2) ^ (row & 7)) << 2) | (col & 3));
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -362,16 +363,24 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
             for (int kk = 0; kk < 4; ++kk)
                 umma_bf16(tmem + TM_D1, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
                           smem_desc(sbase + L.K + 32 * kk, 16, 1024), id, kk > 0);
+            // A_rb^T directly: rows s of b~ against r~ (rows 64..127 of this A operand
+            // read the next tile and are never used).
+            constexpr uint32_t id2 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.B + 32 * kk, 16, 1024),
+                          smem_desc(sbase + L.R + 32 * kk, 16, 1024), id2, kk > 0);
             umma_commit(bar_mma);
         }
         wait_or_abort(bar_mma, mma_phase, abort_flag);
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 5. epilogue 1: rows t of D1 -> masked A_rk, A_rb^T, A_ak (bf16), A_ab (fp32) --
+        // ---- 5. epilogue 1: masked A_rk, A_rb^T, A_ak (bf16) and A_ab (fp32), each row-wise --
         {
             float v[64];
-            tmem_row<4>(tmem + TM_D1, wq, 64 * wh, v);
+            // Warps 4 and 5 read A_rb^T (lanes 0..63 of D1b); the others read D1.
+            tmem_row<4>(tmem + ((wq < 2 && wh == 1) ? TM_D1B : TM_D1 + 64 * wh), wq, 0, v);
             if (wq < 2) {
                 const int t = m_row;  // row of r~
                 if (wh == 0) {  // A_rk[t][s] = v[s], kept for s <= t -> row t
@@ -382,11 +391,15 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
                         for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
                         *reinterpret_cast<uint4*>(smem + L.ARK + sw(t, c)) = pack8(x);
                     }
-                } else {  // A_rb[t][s] = v[s], kept for s <= t -> column t of A_rb^T
+                } else {  // row s = m_row of A_rb^T: A_rb[t][s] = v[t], kept for s <= t
+                    const int s_ = m_row;
 #pragma unroll
-                    for (int s_ = 0; s_ < 64; ++s_)
-                        *reinterpret_cast<__nv_bfloat16*>(smem + L.ARBT + swe(s_, t)) =
-                            __float2bfloat16_rn(s_ <= t ? v[s_] : 0.f);
+                    for (int c = 0; c < 8; ++c) {
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] = (s_ <= 8 * c + e) ? v[8 * c + e] : 0.f;
+                        *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8(x);
+                    }
                 }
             } else {
                 const int t = m_row - 64;  // row of a~
@@ -451,67 +464,74 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
             __syncthreads();
             const int g = lane >> 2, q = lane & 3;
             uint8_t* xt = smem + (warp < 4 ? L.ABAR : L.AAK);  // tile of this warp's columns
-            const int nc = 16 * (warp & 3);                    // first column inside it
+            const int nb = 2 * (warp & 3);                     // first 16-byte chunk of them
             float* ys = reinterpret_cast<float*>(smem + L.K + 5120) + warp * 320;  // 16 x 20
+            // Per-lane byte / float offsets of the fragment elements (rows advance in
+            // multiples of 8, which leave the swizzle phase unchanged).
+            uint32_t yoff[2], boff[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                yoff[nt] = g * 128 + ((((uint32_t)(nb + nt)) ^ g) << 4) + 4 * q;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    boff[nt][hh] = (q + 4 * hh) * 128 + ((((uint32_t)(nb + nt)) ^ (q + 4 * hh)) << 4) + 2 * g;
+            }
+            auto bf16_bits = [](const uint8_t* p) -> uint32_t {
+                return (uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16;  // exact in tf32
+            };
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float y[2][4];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    const int col = nc + 8 * nt + 2 * q;
-                    const float2 lo = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162*>(xt + swe(16 * i + g, col)));
-                    const float2 hi = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162*>(xt + swe(16 * i + g + 8, col)));
+                    const uint8_t* py = xt + 16 * i * 128 + yoff[nt];
+                    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(py));
+                    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(py + 1024));
                     y[nt][0] = lo.x; y[nt][1] = lo.y; y[nt][2] = hi.x; y[nt][3] = hi.y;
                 }
 #pragma unroll
                 for (int m = 0; m < i; ++m) {
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
-                        const int ac = 16 * m + 8 * ks + q;
-                        const uint32_t a0 = to_tf32(A[fidx(16 * i + g, ac)]);
-                        const uint32_t a1 = to_tf32(A[fidx(16 * i + g + 8, ac)]);
-                        const uint32_t a2 = to_tf32(A[fidx(16 * i + g, ac + 4)]);
-                        const uint32_t a3 = to_tf32(A[fidx(16 * i + g + 8, ac + 4)]);
+                        // rows 16i + g (+8) share the swizzle phase g
+                        const float* Ab = A + (16 * i + g) * 64 + q;
+                        const int c0i = ((4 * m + 2 * ks) ^ g) << 2, c1i = ((4 * m + 2 * ks + 1) ^ g) << 2;
+                        const uint32_t a0 = to_tf32(Ab[c0i]);
+                        const uint32_t a1 = to_tf32(Ab[8 * 64 + c0i]);
+                        const uint32_t a2 = to_tf32(Ab[c1i]);
+                        const uint32_t a3 = to_tf32(Ab[8 * 64 + c1i]);
+                        const uint8_t* xb = xt + (16 * m + 8 * ks) * 128;
 #pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const int col = nc + 8 * nt + g;
-                            const uint32_t b0 = to_tf32(bf16_at(xt, 16 * m + 8 * ks + q, col));
-                            const uint32_t b1 = to_tf32(bf16_at(xt, 16 * m + 8 * ks + q + 4, col));
-                            mma_tf32(y[nt], a0, a1, a2, a3, b0, b1);
-                        }
+                        for (int nt = 0; nt < 2; ++nt)
+                            mma_tf32(y[nt], a0, a1, a2, a3, bf16_bits(xb + boff[nt][0]),
+                                     bf16_bits(xb + boff[nt][1]));
                     }
                 }
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    ys[g * 20 + 8 * nt + 2 * q] = y[nt][0];
-                    ys[g * 20 + 8 * nt + 2 * q + 1] = y[nt][1];
-                    ys[(g + 8) * 20 + 8 * nt + 2 * q] = y[nt][2];
-                    ys[(g + 8) * 20 + 8 * nt + 2 * q + 1] = y[nt][3];
+                    *reinterpret_cast<float2*>(ys + g * 20 + 8 * nt + 2 * q) = make_float2(y[nt][0], y[nt][1]);
+                    *reinterpret_cast<float2*>(ys + (g + 8) * 20 + 8 * nt + 2 * q) = make_float2(y[nt][2], y[nt][3]);
                 }
                 __syncwarp();
                 float xo[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
-                    const float* tr = Td + (16 * i) * 20 + 8 * ks + q;
-                    const uint32_t a0 = to_tf32(tr[g * 20]);
-                    const uint32_t a1 = to_tf32(tr[(g + 8) * 20]);
-                    const uint32_t a2 = to_tf32(tr[g * 20 + 4]);
-                    const uint32_t a3 = to_tf32(tr[(g + 8) * 20 + 4]);
+                    const float* tr = Td + (16 * i + g) * 20 + 8 * ks + q;
+                    const uint32_t a0 = to_tf32(tr[0]);
+                    const uint32_t a1 = to_tf32(tr[8 * 20]);
+                    const uint32_t a2 = to_tf32(tr[4]);
+                    const uint32_t a3 = to_tf32(tr[8 * 20 + 4]);
+                    const float* yb = ys + (8 * ks + q) * 20 + g;
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const uint32_t b0 = to_tf32(ys[(8 * ks + q) * 20 + 8 * nt + g]);
-                        const uint32_t b1 = to_tf32(ys[(8 * ks + q + 4) * 20 + 8 * nt + g]);
-                        mma_tf32(xo[nt], a0, a1, a2, a3, b0, b1);
-                    }
+                    for (int nt = 0; nt < 2; ++nt)
+                        mma_tf32(xo[nt], a0, a1, a2, a3, to_tf32(yb[8 * nt]), to_tf32(yb[4 * 20 + 8 * nt]));
                 }
                 __syncwarp();
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    const int col = nc + 8 * nt + 2 * q;
-                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g, col)) = pack2(xo[nt][0], xo[nt][1]);
-                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g + 8, col)) = pack2(xo[nt][2], xo[nt][3]);
+                    uint8_t* px = xt + 16 * i * 128 + yoff[nt];
+                    *reinterpret_cast<uint32_t*>(px) = pack2(xo[nt][0], xo[nt][1]);
+                    *reinterpret_cast<uint32_t*>(px + 1024) = pack2(xo[nt][2], xo[nt][3]);
                 }
                 __syncwarp();
             }
