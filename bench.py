@@ -29,7 +29,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from linear_attention_rnn_wkv7_b200 import synth  # noqa: E402
+from linear_attention_rnn_wkv7_b200 import replicas, synth  # noqa: E402
 
 METRIC = "WKV7 fwd tokens/s (B=8,T=4096,H=64,D=64 bf16) + decode HBM GB/s vs peak"
 FWD = synth.WORKLOADS["fwd_bf16_b8_t4096_h64"]
@@ -201,6 +201,9 @@ def main():
                     help="forward batch (default 8; smaller only for profiling captures)")
     ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
                     help="run only one leg (profiling captures)")
+    ap.add_argument("--workload", choices=["b8_t4096_h64", "masked_b16_t4096_h32",
+                                           "varlen_64seq_h32"], default="b8_t4096_h64",
+                    help="forward workload (the metric is quoted on b8_t4096_h64)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -229,11 +232,7 @@ def main():
             pg.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if pg is None:
-            return v
-        t = torch.tensor([v], device=device, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, device=device)
 
     hbm_peak, peak_kind = load_peaks()
     stream = torch.cuda.current_stream(device)
@@ -250,15 +249,14 @@ def main():
         cpu = cpu_oracle_sample()
 
     if rank == 0:
-        B, T, H = args.batch, FWD["T"], FWD["H"]
+        desc = fwd["desc"] if fwd else {"workload": "none"}
         line = {"metric": METRIC, "value": fwd and fwd["value"], "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": fwd and fwd["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": f"fwd_bf16_b{B}_t{T}_h{H}", "B": B, "T": T, "H": H,
-                           "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out",
+                "config": {**desc, "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out",
                            "algo": args.algo, "parallelism": f"replicas x{world}",
-                           "l2": "inputs (1.9 GB per step) larger than L2; no flush"},
+                           "l2": "inputs larger than L2 (>= 0.1 GB per step); no flush"},
                 "roofline": fwd and fwd["roofline"], "cpu_baseline": cpu,
                 "e2e": fwd and fwd["e2e"], "gpu_launches": args.steps if fwd else 0,
                 "clocks": fwd and fwd["clocks"], "decode": decode}
@@ -267,19 +265,59 @@ def main():
         pg.destroy_process_group()
 
 
+def fwd_workload(args, rank):
+    """Synthetic inputs, tokens per step and algorithmic bytes per launch of a workload."""
+    mask = cu = None
+    if args.workload == "b8_t4096_h64":
+        B, T, H = args.batch, FWD["T"], FWD["H"]
+        x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16,
+                             seed=replicas.replica_seed(FWD["seed"], rank), s0_std=FWD["s0_std"])
+        tokens = B * T
+        nbytes = fwd_algorithmic_bytes(B, T, H)
+        desc = {"workload": f"fwd_bf16_b{B}_t{T}_h{H}", "B": B, "T": T, "H": H}
+    elif args.workload == "masked_b16_t4096_h32":
+        p = synth.WORKLOADS["fwd_bf16_masked_b16_t4096_h32"]
+        B, T, H = p["B"], p["T"], p["H"]
+        x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16,
+                             seed=replicas.replica_seed(p["seed"], rank), s0_std=p["s0_std"])
+        mask = synth.padding_mask(B, T, seed=replicas.replica_seed(p["seed"], rank))
+        kept = int(mask.sum())
+        tokens = B * T
+        # masked tokens only need r in and o out; the mask itself is read once
+        nbytes = (kept * H * TOKEN_HEAD_BYTES + (B * T - kept) * H * 2 * 64 * 2 + B * T
+                  + 2 * B * H * STATE_BYTES)
+        desc = {"workload": "fwd_bf16_masked_b16_t4096_h32", "B": B, "T": T, "H": H,
+                "masked_fraction": 1 - kept / (B * T)}
+    else:
+        p = synth.WORKLOADS["fwd_bf16_varlen_64seq_h32"]
+        lengths = synth.varlen_lengths(p["n_seqs"], p["lo"], p["hi"],
+                                       seed=replicas.replica_seed(p["seed"], rank))
+        H = p["H"]
+        x = synth.varlen_inputs(lengths, H, dtype=torch.bfloat16,
+                                seed=replicas.replica_seed(p["seed"], rank), s0_std=p["s0_std"])
+        cu = x.pop("cu_seqlens")
+        B, T = 1, int(lengths.sum())
+        tokens = T
+        nbytes = T * H * TOKEN_HEAD_BYTES + 2 * lengths.numel() * H * STATE_BYTES
+        desc = {"workload": "fwd_bf16_varlen_64seq_h32", "n_seqs": lengths.numel(),
+                "total_tokens": T, "max_len": int(lengths.max()), "H": H}
+    return x, mask, cu, B, T, H, tokens, nbytes, desc
+
+
 def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks, barrier,
             rank, world):
     """K timed forward launches on resident inputs, then the host-buffer e2e pass."""
-    B, T, H = args.batch, FWD["T"], FWD["H"]
-    x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16, seed=FWD["seed"] + 1000 * rank,
-                         s0_std=FWD["s0_std"])
+    x, mask, cu, B, T, H, tokens_per_step, fwd_bytes, desc = fwd_workload(args, rank)
     xd = {k: v.to(device) for k, v in x.items()}
+    maskd = None if mask is None else mask.to(device)
+    cud = None if cu is None else cu.to(device)
+    N = xd["s0"].shape[0]
     o = torch.empty(B, T, H, 64, dtype=torch.bfloat16, device=device)
-    sT = torch.empty(B, H, 64, 64, dtype=torch.float32, device=device)
+    sT = torch.empty(N, H, 64, 64, dtype=torch.float32, device=device)
 
     def step():
         wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
-                 algo=args.algo, o=o, sT=sT)
+                 mask=maskd, cu_seqlens=cud, algo=args.algo, o=o, sT=sT)
 
     for _ in range(args.warmup):
         step()
@@ -297,21 +335,24 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
     barrier()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1))
     ms_step = ms_total / args.steps
-    tokens_per_step = B * T
     value = world * tokens_per_step * args.steps / (ms_total / 1e3)
 
-    fwd_bytes = fwd_algorithmic_bytes(B, T, H)
     achieved = fwd_bytes / (ms_step / 1e3) / 1e9
     kernel = "chunked" if args.algo in ("auto", "chunked") else "recurrent"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
                 "kernel": kernel,
-                "traffic": profiled_traffic(f"fwd_{kernel}_b{B}_t{T}_h{H}"),
+                "traffic": profiled_traffic(f"fwd_{kernel}_{args.workload}"),
                 "algorithmic_bytes_per_launch": fwd_bytes}
 
     # End to end through the public call with host buffers: pinned H2D of every
     # input, the forward, D2H of o and the final state, every step.
     host = {k: v.pin_memory() for k, v in x.items()}
+    dev = dict(xd)
+    if mask is not None:
+        host["mask"], dev["mask"] = mask.pin_memory(), maskd
+    if cu is not None:
+        host["cu_seqlens"], dev["cu_seqlens"] = cu.pin_memory(), cud
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     s_host = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
@@ -319,7 +360,7 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
 
     def e2e_step():
         for k in host:
-            xd[k].copy_(host[k], non_blocking=True)
+            dev[k].copy_(host[k], non_blocking=True)
         step()
         o_host.copy_(o, non_blocking=True)
         s_host.copy_(sT, non_blocking=True)
@@ -337,17 +378,18 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
     e2e = {"value": world * tokens_per_step / (ms_e2e / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
     return {"value": value, "ms_per_step": ms_step, "roofline": roofline, "e2e": e2e,
-            "clocks": clock_info}
+            "clocks": clock_info, "desc": desc}
 
 
 def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank):
     """256 consecutive wkv7_step calls over 1024 x 32 fp32 states (512 MiB, > L2).
     Step inputs: 32 independently drawn step sets, used in turn."""
     B, H, steps = DEC["B"], DEC["H"], DEC["steps"]
-    state = synth.decode_state(B, H, seed=DEC["seed"] + 1000 * rank, std=DEC["s0_std"]).to(device)
+    state = synth.decode_state(B, H, seed=replicas.replica_seed(DEC["seed"], rank),
+                               std=DEC["s0_std"]).to(device)
     sets = []
     for i in range(32):
-        x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16, seed=DEC["seed"] + 1000 * rank,
+        x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16, seed=replicas.replica_seed(DEC["seed"], rank),
                                      step=i)
         sets.append({k: v.to(device) for k, v in x.items()})
     o = torch.empty(B, H, 64, dtype=torch.bfloat16, device=device)
