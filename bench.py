@@ -389,7 +389,8 @@ def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, b
                                std=DEC["s0_std"]).to(device)
     sets = []
     for i in range(32):
-        x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16, seed=replicas.replica_seed(DEC["seed"], rank),
+        x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16,
+                                     seed=replicas.replica_seed(DEC["seed"], rank),
                                      step=i)
         sets.append({k: v.to(device) for k, v in x.items()})
     o = torch.empty(B, H, 64, dtype=torch.bfloat16, device=device)
