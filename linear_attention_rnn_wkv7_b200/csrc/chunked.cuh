@@ -554,33 +554,44 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 8. epilogue 3: assemble the final A operand ---------------------------------
+        // ---- 8. epilogue 3: assemble the final A operand.  Rows k (lanes 0..63): M'
+        //         and the hi/lo split of P_N, whose 64 columns are shared by warps 0/1
+        //         (after M') and 4/5.  Rows t (lanes 64..127): Q and P_O. --------------
         {
-            float v[64];
-            tmem_row<4>(tmem + TM_D1, wq, 64 * wh, v);
             if (wq < 2) {
                 const int k = m_row;
-                if (wh == 0) {  // M' = Bhat^T W
+                auto split_pn = [&](const float* v, int c0n) {  // P_N = Bhat^T Z + Khat^T
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(smem + L.R + sw(k, c)) = pack8(v + 8 * c);
-                } else {  // P_N = Bhat^T Z + Khat^T, split into bf16 hi + lo
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         float hi[8], lo[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const int s = 8 * c + e;
-                            const float p = v[s] + F0[s * 64 + k];
-                            hi[e] = __bfloat162float(__float2bfloat16_rn(p));
-                            lo[e] = p - hi[e];
+                            const int s_ = 8 * (c0n + c) + e;
+                            const float pn = v[8 * c + e] + F0[s_ * 64 + k];
+                            hi[e] = __bfloat162float(__float2bfloat16_rn(pn));
+                            lo[e] = pn - hi[e];
                         }
-                        *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, c)) = pack8(hi);
-                        *reinterpret_cast<uint4*>(smem + L.K + sw(k, c)) = pack8(lo);
+                        *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, c0n + c)) = pack8(hi);
+                        *reinterpret_cast<uint4*>(smem + L.K + sw(k, c0n + c)) = pack8(lo);
                     }
+                };
+                if (wh == 0) {
+                    float v[64];
+                    tmem_row<4>(tmem + TM_D1, wq, 0, v);  // M' = Bhat^T W
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(smem + L.R + sw(k, c)) = pack8(v + 8 * c);
+                    tmem_row<2>(tmem + TM_D1, wq, 64, v);  // P_N columns 0..31
+                    split_pn(v, 0);
+                } else {
+                    float v[32];
+                    tmem_row<2>(tmem + TM_D1, wq, 96, v);  // P_N columns 32..63
+                    split_pn(v, 4);
                 }
             } else {
                 const int tp = m_row - 64;
+                float v[64];
+                tmem_row<4>(tmem + TM_D1, wq, 64 * wh, v);
                 if (wh == 0) {  // Q = A_rb W + Rbar
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -649,9 +660,11 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
                     for (int c = 0; c < 4; ++c) dst[c] = pack8(v + 8 * c);
                 }
             }
+            // No barrier: nothing the next chunk does before its own first barrier
+            // touches what this epilogue reads or writes (S0 tile, o, TMEM columns
+            // of the final product, e^{g_L}).
             fence_proxy_async();
             tc_fence_before();
-            __syncthreads();
         }
 }
 
