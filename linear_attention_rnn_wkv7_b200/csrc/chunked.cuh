@@ -167,6 +167,17 @@ __device__ __forceinline__ void tmem_row(uint32_t tmem, int wq, uint32_t col, fl
     sm100::tmem_ld_wait();
 }
 
+// Store 32 fp32 columns [col, col + 32) of this warp's lanes.
+__device__ __forceinline__ void tmem_row_st32(uint32_t tmem, int wq, uint32_t col, const float* v) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        float tmp[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) tmp[j] = v[16 * i + j];
+        sm100::tmem_st16(tmem + ((uint32_t)(32 * wq) << 16) + col + 16 * i, tmp);
+    }
+}
+
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -227,7 +238,7 @@ __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
 }
 
 // One 64-token chunk starting at token c0, in layout P (its inputs already requested).
-__device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_next, int par) {
+__device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
     const LayR L = lay_of(par);
     using namespace sm100;
     uint8_t* smem = cx.smem;
@@ -613,6 +624,22 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
                     }
                 }
             }
+            // The final MMA accumulates onto its tensor-memory columns: rows 0..63 hold
+            // the fp32 state, scaled here by e^{g_L}; rows 64..127 (outputs) start at 0.
+            {
+                float sv[32];
+                if (state_thread) {
+                    const float gamma = gamma_s[m_row];
+                    tmem_row<2>(tmem + TM_DF, wq, 32 * wh, sv);
+#pragma unroll
+                    for (int j2 = 0; j2 < 32; ++j2) sv[j2] *= gamma;
+                } else {
+#pragma unroll
+                    for (int j2 = 0; j2 < 32; ++j2) sv[j2] = 0.f;
+                }
+                tmem_row_st32(tmem + TM_DF, wq, 32 * wh, sv);
+                tmem_st_wait();
+            }
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
@@ -633,7 +660,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem + TM_DF, smem_desc(sbase + aoff + 32 * kk, 16, 1024),
-                              smem_desc(sbase + boff + 2048 * kk, 8192, 1024), id, (blk | kk) != 0);
+                              smem_desc(sbase + boff + 2048 * kk, 8192, 1024), id, 1u);
             }
             umma_commit(bar_mma);
         }
@@ -645,13 +672,10 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
         {
             float v[32];
             tmem_row<2>(tmem + TM_DF, wq, 32 * wh, v);
-            if (state_thread) {
-                const float gamma = gamma_s[m_row];  // e^{g_L} of this state row's channel
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = fmaf(gamma, S[j], v[j]);
+            if (state_thread) {  // v = the new fp32 state row; its bf16 copy feeds the next chunk
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(S + 8 * c);
+                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(v + 8 * c);
             } else {
                 const int t = m_row - 64;
                 if (t < nv) {
@@ -661,8 +685,8 @@ __device__ __forceinline__ void chunk(Ctx& cx, float (&S)[32], int c0, bool has_
                 }
             }
             // No barrier: nothing the next chunk does before its own first barrier
-            // touches what this epilogue reads or writes (S0 tile, o, TMEM columns
-            // of the final product, e^{g_L}).
+            // touches what this epilogue reads or writes (S0 tile, o, the final
+            // product's tensor-memory columns).
             fence_proxy_async();
             tc_fence_before();
         }
@@ -744,41 +768,48 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                            : lane == 3 ? &tm_b : lane == 4 ? &tm_w : &tm_v);
     if (warp == 0 && cx.len > 0) issue_loads(cx, 0, 0);
 
-    // State rows: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
-    // [32*wh, 32*wh + 32), in fp32 registers for the whole sequence.
+    // The fp32 state lives in tensor memory, rows 0..63 of the final product's
+    // columns: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
+    // [32*wh, 32*wh + 32).  A bf16 copy in shared memory feeds the final MMA.
     const int m_row = cx.m_row;
     const size_t state_off = ((size_t)n * H + h) * 4096;
-    float S[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) S[j] = 0.f;
     if (cx.state_thread) {
+        float sv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[j] = 0.f;
         if (s0) {
             const float4* src = reinterpret_cast<const float4*>(s0 + state_off + m_row * 64 + 32 * wh);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float4 f = src[j];
-                S[4 * j] = f.x;
-                S[4 * j + 1] = f.y;
-                S[4 * j + 2] = f.z;
-                S[4 * j + 3] = f.w;
+                sv[4 * j] = f.x;
+                sv[4 * j + 1] = f.y;
+                sv[4 * j + 2] = f.z;
+                sv[4 * j + 3] = f.w;
             }
         }
+        tmem_row_st32(cx.tmem + TM_DF, wq, 32 * wh, sv);
+        tmem_st_wait();
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(S + 8 * c);
+            *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(sv + 8 * c);
     }
+    tc_fence_before();
 
     // Chunks alternate between the two shared-memory layouts.
     for (int c0 = 0, par = 0; c0 < cx.len; c0 += 64, par ^= 1) {
-        chunk(cx, S, c0, c0 + 64 < cx.len, par);
+        chunk(cx, c0, c0 + 64 < cx.len, par);
         if (*cx.abort_flag) break;
     }
 
+    tc_fence_after();
     if (cx.state_thread && sT && !*cx.abort_flag) {
+        float sv[32];
+        tmem_row<2>(cx.tmem + TM_DF, wq, 32 * wh, sv);
         float4* dst = reinterpret_cast<float4*>(sT + state_off + m_row * 64 + 32 * wh);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+            dst[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
     }
     tc_fence_before();
     __syncthreads();
