@@ -442,11 +442,12 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 
         // ---- 6. [W | Z] = T [Abar | A_ak], T = (I - A_ab)^-1, by block forward
         //         substitution over four 16-row blocks:
-        //             X_i = T_ii (RHS_i + sum_{m<i} A_im X_m).
+        //             X_i = T_ii RHS_i + sum_{m<i} (T_ii A_im) X_m.
         //         The 16x16 diagonal inverses T_ii come from fp32 forward substitution;
-        //         then each warp solves its own 16 of the 128 right-hand-side columns
-        //         with warp-level tf32 MMAs, writing X in place over the right-hand
-        //         side (bf16), where MMA-3 reads it as its MN-major B operand ---------
+        //         the products T_ii A_im and T_ii RHS_i are independent and run in
+        //         parallel on warp-level tf32 MMAs; then each warp finishes its own 16
+        //         of the 128 right-hand-side columns, writing X in place over the
+        //         right-hand side (bf16), where MMA-3 reads it as its MN-major B operand
         {
             const float* A = reinterpret_cast<const float*>(smem + L.R);  // A_ab [t][s]
             float* Td = reinterpret_cast<float*>(smem + L.K);             // T_bb, rows of 20
@@ -476,9 +477,11 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             const int g = lane >> 2, q = lane & 3;
             uint8_t* xt = smem + (warp < 4 ? L.ABAR : L.AAK);  // tile of this warp's columns
             const int nb = 2 * (warp & 3);                     // first 16-byte chunk of them
-            float* ys = reinterpret_cast<float*>(smem + L.K + 5120) + warp * 320;  // 16 x 20
-            // Per-lane byte / float offsets of the fragment elements (rows advance in
-            // multiples of 8, which leave the swizzle phase unchanged).
+            // Precomputed T_ii A_im for the six blocks below the diagonal, fp32 16 x 16
+            // with rows of 20, after the four T_ii.
+            float* Ta = Td + 4 * 16 * 20;
+            // Per-lane byte offsets of the fragment elements in the bf16 tile (rows
+            // advance in multiples of 8, which leave the swizzle phase unchanged).
             uint32_t yoff[2], boff[2][2];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -490,59 +493,82 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             auto bf16_bits = [](const uint8_t* p) -> uint32_t {
                 return (uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16;  // exact in tf32
             };
+            // A fragment of a 16 x 16 fp32 block with rows of 20 floats.
+            auto afrag20 = [&](const float* blk, int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2,
+                               uint32_t& a3) {
+                const float* tr = blk + g * 20 + 8 * ks + q;
+                a0 = to_tf32(tr[0]);
+                a1 = to_tf32(tr[8 * 20]);
+                a2 = to_tf32(tr[4]);
+                a3 = to_tf32(tr[8 * 20 + 4]);
+            };
+            // (a) warps 0..5: Ta(i, m) = T_ii A_im, one block each.
+            if (warp < 6) {
+                const int i = warp < 1 ? 1 : (warp < 3 ? 2 : 3);
+                const int m = warp < 1 ? 0 : (warp < 3 ? warp - 1 : warp - 3);
+                float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float y[2][4];
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t a0, a1, a2, a3;
+                    afrag20(Td + 16 * i * 20, ks, a0, a1, a2, a3);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        // B = A_im: k = row 16i + 8ks + q (+4), n = column 16m + 8nt + g
+                        const int r0 = 16 * i + 8 * ks + q, cn = 16 * m + 8 * nt + g;
+                        mma_tf32(z[nt], a0, a1, a2, a3, to_tf32(A[fidx(r0, cn)]),
+                                 to_tf32(A[fidx(r0 + 4, cn)]));
+                    }
+                }
+                float* dst = Ta + warp * 320;  // blocks in order (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    const uint8_t* py = xt + 16 * i * 128 + yoff[nt];
-                    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(py));
-                    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(py + 1024));
-                    y[nt][0] = lo.x; y[nt][1] = lo.y; y[nt][2] = hi.x; y[nt][3] = hi.y;
+                    *reinterpret_cast<float2*>(dst + g * 20 + 8 * nt + 2 * q) = make_float2(z[nt][0], z[nt][1]);
+                    *reinterpret_cast<float2*>(dst + (g + 8) * 20 + 8 * nt + 2 * q) = make_float2(z[nt][2], z[nt][3]);
                 }
+            }
+            // (b) every warp, its 16 columns: Y_i = T_ii RHS_i for the four block rows.
+            float y[4][2][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) y[i][nt][e] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t a0, a1, a2, a3;
+                    afrag20(Td + 16 * i * 20, ks, a0, a1, a2, a3);
+                    const uint8_t* xb = xt + (16 * i + 8 * ks) * 128;
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+                        mma_tf32(y[i][nt], a0, a1, a2, a3, bf16_bits(xb + boff[nt][0]),
+                                 bf16_bits(xb + boff[nt][1]));
+                }
+            }
+            __syncthreads();  // Ta visible; every warp has read its right-hand side
+            // (c) X_i = Y_i + sum_{m<i} Ta(i, m) X_m, written in place over the right-hand
+            //     side in bf16 (X_m is read back from there by the later block rows).
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
 #pragma unroll
                 for (int m = 0; m < i; ++m) {
+                    const int blk = (i == 1) ? 0 : (i == 2 ? 1 + m : 3 + m);
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
-                        // rows 16i + g (+8) share the swizzle phase g
-                        const float* Ab = A + (16 * i + g) * 64 + q;
-                        const int c0i = ((4 * m + 2 * ks) ^ g) << 2, c1i = ((4 * m + 2 * ks + 1) ^ g) << 2;
-                        const uint32_t a0 = to_tf32(Ab[c0i]);
-                        const uint32_t a1 = to_tf32(Ab[8 * 64 + c0i]);
-                        const uint32_t a2 = to_tf32(Ab[c1i]);
-                        const uint32_t a3 = to_tf32(Ab[8 * 64 + c1i]);
+                        uint32_t a0, a1, a2, a3;
+                        afrag20(Ta + blk * 320, ks, a0, a1, a2, a3);
                         const uint8_t* xb = xt + (16 * m + 8 * ks) * 128;
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt)
-                            mma_tf32(y[nt], a0, a1, a2, a3, bf16_bits(xb + boff[nt][0]),
+                            mma_tf32(y[i][nt], a0, a1, a2, a3, bf16_bits(xb + boff[nt][0]),
                                      bf16_bits(xb + boff[nt][1]));
                     }
                 }
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    *reinterpret_cast<float2*>(ys + g * 20 + 8 * nt + 2 * q) = make_float2(y[nt][0], y[nt][1]);
-                    *reinterpret_cast<float2*>(ys + (g + 8) * 20 + 8 * nt + 2 * q) = make_float2(y[nt][2], y[nt][3]);
-                }
-                __syncwarp();
-                float xo[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    const float* tr = Td + (16 * i + g) * 20 + 8 * ks + q;
-                    const uint32_t a0 = to_tf32(tr[0]);
-                    const uint32_t a1 = to_tf32(tr[8 * 20]);
-                    const uint32_t a2 = to_tf32(tr[4]);
-                    const uint32_t a3 = to_tf32(tr[8 * 20 + 4]);
-                    const float* yb = ys + (8 * ks + q) * 20 + g;
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-                        mma_tf32(xo[nt], a0, a1, a2, a3, to_tf32(yb[8 * nt]), to_tf32(yb[4 * 20 + 8 * nt]));
-                }
-                __syncwarp();
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
                     uint8_t* px = xt + 16 * i * 128 + yoff[nt];
-                    *reinterpret_cast<uint32_t*>(px) = pack2(xo[nt][0], xo[nt][1]);
-                    *reinterpret_cast<uint32_t*>(px + 1024) = pack2(xo[nt][2], xo[nt][3]);
+                    *reinterpret_cast<uint32_t*>(px) = pack2(y[i][nt][0], y[i][nt][1]);
+                    *reinterpret_cast<uint32_t*>(px + 1024) = pack2(y[i][nt][2], y[i][nt][3]);
                 }
                 __syncwarp();
             }
