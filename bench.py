@@ -151,6 +151,12 @@ def cpu_oracle_sample(target_s: float = 12.0):
                       f"full T=4096 each; tokens/s = token-heads / 64 / wall time"}
 
 
+def fwd_config(desc: dict, algo: str, world: int) -> dict:
+    return {**desc, "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out", "algo": algo,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (>= 0.1 GB per step); no flush"}
+
+
 def reference_arm(args, rank: int):
     """The oracle as the reference arm: each step is one bounded sample."""
     if rank != 0:
@@ -158,7 +164,7 @@ def reference_arm(args, rank: int):
     import oracle
     H, T = FWD["H"], FWD["T"]
     x = synth.fwd_inputs(1, T, H, dtype=torch.bfloat16, seed=FWD["seed"], s0_std=FWD["s0_std"])
-    units = 4
+    units = min(H, max(4, os.cpu_count() or 1))  # one whole (b, h) unit per host thread
     sl = {n: x[n][:, :, :units] for n in "rwkvab"}
 
     def one():
@@ -177,11 +183,12 @@ def reference_arm(args, rank: int):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "fwd_bf16_b8_t4096_h64", "B": 8, "T": T, "H": H, "K": 64,
-                       "V": 64},
+            "config": fwd_config({"workload": "fwd_bf16_b8_t4096_h64", "B": FWD["B"], "T": T,
+                                  "H": H}, "oracle", args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
-                             "sample": f"each step: {units} of the 512 (b,h) units, full "
-                                       f"T={T}, fp64 sequential recurrence"},
+                             "sample": f"each step: {units} of the 512 (b,h) units of "
+                                       f"B=8,T={T},H={H}, full T each, fp64 sequential "
+                                       f"recurrence; tokens/s = token-heads / {H} / time"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -254,9 +261,7 @@ def main():
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": fwd and fwd["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {**desc, "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out",
-                           "algo": args.algo, "parallelism": f"replicas x{world}",
-                           "l2": "inputs larger than L2 (>= 0.1 GB per step); no flush"},
+                "config": fwd_config(desc, args.algo, world),
                 "roofline": fwd and fwd["roofline"], "cpu_baseline": cpu,
                 "e2e": fwd and fwd["e2e"], "gpu_launches": args.steps if fwd else 0,
                 "clocks": fwd and fwd["clocks"], "decode": decode}
