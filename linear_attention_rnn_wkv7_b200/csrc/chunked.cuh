@@ -301,14 +301,26 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             __syncthreads();
         }
 
-        // ---- 3. scaled operands (two 8-channel pieces per thread); each thread rewrites
-        //         only the chunks it read, and Khat waits until every E_t read is done ----
+        // ---- 3. scaled operands.  Thread (q, j) owns tokens 2q, 2q+1 and channels
+        //         8j..8j+7, so E_{t-1} of its second token is E_t of its first and the
+        //         per-channel constants are read once; each thread rewrites only the
+        //         chunks it read, and Khat waits until every E_t read is done. ---------
         {
+            const int j = tid & 7, t0 = 2 * (tid >> 3);
+            float ec[8], elc[8], Ep[8];
+            *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[0];
+            *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[1];
+            *reinterpret_cast<float4*>(elc) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[0];
+            *reinterpret_cast<float4*>(elc + 4) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[1];
+            {
+                const float* Emrow = t0 > 0 ? F0 + (t0 - 1) * 64 + 8 * j : scratch + SCR_EMC + 8 * j;
+                *reinterpret_cast<float4*>(Ep) = reinterpret_cast<const float4*>(Emrow)[0];
+                *reinterpret_cast<float4*>(Ep + 4) = reinterpret_cast<const float4*>(Emrow)[1];
+            }
             float4 o_khat[2][2];
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
-                const int item = tid + 256 * it;
-                const int t = item >> 3, j = item & 7;
+                const int t = t0 + it;
                 const bool val = validb[t] != 0;
                 const uint32_t off = sw(t, j);
                 float rv[8], av[8], kv[8], bv[8];
@@ -316,31 +328,25 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.A + off), av);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.B + off), bv);
-                float E[8], Em[8], ec[8], elc[8];
-                const float* Erow = F0 + t * 64 + 8 * j;
-                const float* Emrow = t > 0 ? F0 + (t - 1) * 64 + 8 * j : scratch + SCR_EMC + 8 * j;
-                *reinterpret_cast<float4*>(E) = reinterpret_cast<const float4*>(Erow)[0];
-                *reinterpret_cast<float4*>(E + 4) = reinterpret_cast<const float4*>(Erow)[1];
-                *reinterpret_cast<float4*>(Em) = reinterpret_cast<const float4*>(Emrow)[0];
-                *reinterpret_cast<float4*>(Em + 4) = reinterpret_cast<const float4*>(Emrow)[1];
-                *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[0];
-                *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[1];
-                *reinterpret_cast<float4*>(elc) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[0];
-                *reinterpret_cast<float4*>(elc + 4) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[1];
+                float E[8];
+                *reinterpret_cast<float4*>(E) = reinterpret_cast<const float4*>(F0 + t * 64 + 8 * j)[0];
+                *reinterpret_cast<float4*>(E + 4) = reinterpret_cast<const float4*>(F0 + t * 64 + 8 * j)[1];
                 float rt[8], at[8], kt[8], btl[8], abar[8], bhat[8], khat[8], rbar[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float inv = __frcp_rn(E[e]);
                     const float a_ = val ? av[e] : 0.f, k_ = val ? kv[e] : 0.f,
                                 b_ = val ? bv[e] : 0.f;
+                    const float il = elc[e] * inv;  // e^{g_L - g_t}
                     rt[e] = rv[e] * E[e];
-                    at[e] = a_ * Em[e];
+                    at[e] = a_ * Ep[e];
                     kt[e] = k_ * inv;
                     btl[e] = b_ * inv;
                     abar[e] = at[e] * ec[e];
-                    bhat[e] = b_ * elc[e] * inv;
-                    khat[e] = k_ * elc[e] * inv;
+                    bhat[e] = b_ * il;
+                    khat[e] = k_ * il;
                     rbar[e] = rt[e] * ec[e];
+                    Ep[e] = E[e];  // E_{t-1} of the next token
                 }
                 *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rt);
                 *reinterpret_cast<uint4*>(smem + L.A + off) = pack8(at);
@@ -355,9 +361,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             __syncthreads();  // every E_t read before F0 is overwritten by Khat
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
-                const int item = tid + 256 * it;
-                const int t = item >> 3, j = item & 7;
-                float4* kh = reinterpret_cast<float4*>(F0 + t * 64 + 8 * j);
+                float4* kh = reinterpret_cast<float4*>(F0 + (t0 + it) * 64 + 8 * j);
                 kh[0] = o_khat[it][0];
                 kh[1] = o_khat[it][1];
             }
