@@ -178,6 +178,31 @@ __device__ __forceinline__ void tmem_row_st32(uint32_t tmem, int wq, uint32_t co
     }
 }
 
+// Warp-level D += A * B, m16n8k16, bf16 operands, fp32 accumulate.  Fragment
+// ownership (g = lane / 4, q = lane % 4): A (g|g+8, 2q..2q+1 | 2q+8..2q+9),
+// B (k = 2q..2q+1 | 2q+8..2q+9, n = g), C/D (g|g+8, 2q|2q+1).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Four 8x8 b16 matrices; lane l gives the address of row (l % 8) of matrix l / 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -449,12 +474,15 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         //             X_i = T_ii RHS_i + sum_{m<i} (T_ii A_im) X_m.
         //         The 16x16 diagonal inverses T_ii come from fp32 forward substitution;
         //         the products T_ii A_im and T_ii RHS_i are independent and run in
-        //         parallel on warp-level tf32 MMAs; then each warp finishes its own 16
-        //         of the 128 right-hand-side columns, writing X in place over the
-        //         right-hand side (bf16), where MMA-3 reads it as its MN-major B operand
+        //         parallel on warp-level bf16 MMAs (fp32 accumulate); then each warp
+        //         finishes its own 16 of the 128 right-hand-side columns, writing X in
+        //         place over the right-hand side (bf16), where MMA-3 reads it as its
+        //         MN-major B operand. ------------------------------------------------
         {
             const float* A = reinterpret_cast<const float*>(smem + L.R);  // A_ab [t][s]
-            float* Td = reinterpret_cast<float*>(smem + L.K);             // T_bb, rows of 20
+            // bf16 16x16 blocks with rows of 48 bytes: T_ii (4), then T_ii A_im (6).
+            uint8_t* Tb = smem + L.K;
+            uint8_t* Tab = Tb + 4 * 768;
             if (tid < 64) {  // diagonal block b, column c
                 const int b = tid >> 4, c = tid & 15, base = 16 * b;
                 float x[16];
@@ -475,59 +503,46 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     x[t] = (t == c) ? 1.f : acc0 + acc1;
                 }
 #pragma unroll
-                for (int t = 0; t < 16; ++t) Td[(base + t) * 20 + c] = x[t];
+                for (int t = 0; t < 16; ++t)
+                    *reinterpret_cast<__nv_bfloat16*>(Tb + b * 768 + t * 48 + 2 * c) =
+                        __float2bfloat16_rn(x[t]);
             }
             __syncthreads();
             const int g = lane >> 2, q = lane & 3;
             uint8_t* xt = smem + (warp < 4 ? L.ABAR : L.AAK);  // tile of this warp's columns
             const int nb = 2 * (warp & 3);                     // first 16-byte chunk of them
-            // Precomputed T_ii A_im for the six blocks below the diagonal, fp32 16 x 16
-            // with rows of 20, after the four T_ii.
-            float* Ta = Td + 4 * 16 * 20;
-            // Per-lane byte offsets of the fragment elements in the bf16 tile (rows
-            // advance in multiples of 8, which leave the swizzle phase unchanged).
-            uint32_t yoff[2], boff[2][2];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                yoff[nt] = g * 128 + ((((uint32_t)(nb + nt)) ^ g) << 4) + 4 * q;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-                    boff[nt][hh] = (q + 4 * hh) * 128 + ((((uint32_t)(nb + nt)) ^ (q + 4 * hh)) << 4) + 2 * g;
-            }
-            auto bf16_bits = [](const uint8_t* p) -> uint32_t {
-                return (uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16;  // exact in tf32
+            const uint32_t xs = smem_u32(xt);
+            // ldmatrix row addresses of this lane: A blocks (48-byte rows) and the
+            // transposed B fragments of rows kb..kb+15 of this warp's 16 columns.
+            const int lr = (lane & 7) + 8 * ((lane >> 3) & 1), lc = 8 * (lane >> 4);
+            const uint32_t a_lane = lr * 48 + 2 * lc;
+            auto b_addr = [&](int kb) -> uint32_t {
+                const int row = kb + (lane & 7) + 8 * ((lane >> 3) & 1);
+                return xs + sw(row, nb + (lane >> 4));
             };
-            // A fragment of a 16 x 16 fp32 block with rows of 20 floats.
-            auto afrag20 = [&](const float* blk, int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2,
-                               uint32_t& a3) {
-                const float* tr = blk + g * 20 + 8 * ks + q;
-                a0 = to_tf32(tr[0]);
-                a1 = to_tf32(tr[8 * 20]);
-                a2 = to_tf32(tr[4]);
-                a3 = to_tf32(tr[8 * 20 + 4]);
+            auto a_frag = [&](const uint8_t* blk, uint32_t (&af)[4]) {
+                ldsm_x4(smem_u32(blk) + a_lane, af[0], af[1], af[2], af[3]);
             };
-            // (a) warps 0..5: Ta(i, m) = T_ii A_im, one block each.
+            // (a) warps 0..5: T_ii A_im, one block each, stored bf16.
             if (warp < 6) {
                 const int i = warp < 1 ? 1 : (warp < 3 ? 2 : 3);
                 const int m = warp < 1 ? 0 : (warp < 3 ? warp - 1 : warp - 3);
+                uint32_t af[4];
+                a_frag(Tb + i * 768, af);
                 float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    uint32_t a0, a1, a2, a3;
-                    afrag20(Td + 16 * i * 20, ks, a0, a1, a2, a3);
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        // B = A_im: k = row 16i + 8ks + q (+4), n = column 16m + 8nt + g
-                        const int r0 = 16 * i + 8 * ks + q, cn = 16 * m + 8 * nt + g;
-                        mma_tf32(z[nt], a0, a1, a2, a3, to_tf32(A[fidx(r0, cn)]),
-                                 to_tf32(A[fidx(r0 + 4, cn)]));
-                    }
+                for (int nt = 0; nt < 2; ++nt) {
+                    // B = A_im: k = row 16i + (2q, 2q+1 | 2q+8, 2q+9), n = column 16m + 8nt + g
+                    const int r0 = 16 * i + 2 * q, cn = 16 * m + 8 * nt + g;
+                    const uint32_t b0 = pack2(A[fidx(r0, cn)], A[fidx(r0 + 1, cn)]);
+                    const uint32_t b1 = pack2(A[fidx(r0 + 8, cn)], A[fidx(r0 + 9, cn)]);
+                    mma_bf16_16816(z[nt], af[0], af[1], af[2], af[3], b0, b1);
                 }
-                float* dst = Ta + warp * 320;  // blocks in order (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+                uint8_t* dst = Tab + warp * 768;  // blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    *reinterpret_cast<float2*>(dst + g * 20 + 8 * nt + 2 * q) = make_float2(z[nt][0], z[nt][1]);
-                    *reinterpret_cast<float2*>(dst + (g + 8) * 20 + 8 * nt + 2 * q) = make_float2(z[nt][2], z[nt][3]);
+                    *reinterpret_cast<uint32_t*>(dst + g * 48 + 2 * (8 * nt + 2 * q)) = pack2(z[nt][0], z[nt][1]);
+                    *reinterpret_cast<uint32_t*>(dst + (g + 8) * 48 + 2 * (8 * nt + 2 * q)) = pack2(z[nt][2], z[nt][3]);
                 }
             }
             // (b) every warp, its 16 columns: Y_i = T_ii RHS_i for the four block rows.
@@ -538,41 +553,31 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) y[i][nt][e] = 0.f;
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    uint32_t a0, a1, a2, a3;
-                    afrag20(Td + 16 * i * 20, ks, a0, a1, a2, a3);
-                    const uint8_t* xb = xt + (16 * i + 8 * ks) * 128;
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-                        mma_tf32(y[i][nt], a0, a1, a2, a3, bf16_bits(xb + boff[nt][0]),
-                                 bf16_bits(xb + boff[nt][1]));
-                }
+                uint32_t af[4], bf[4];
+                a_frag(Tb + i * 768, af);
+                ldsm_x4_t(b_addr(16 * i), bf[0], bf[1], bf[2], bf[3]);
+                mma_bf16_16816(y[i][0], af[0], af[1], af[2], af[3], bf[0], bf[1]);
+                mma_bf16_16816(y[i][1], af[0], af[1], af[2], af[3], bf[2], bf[3]);
             }
-            __syncthreads();  // Ta visible; every warp has read its right-hand side
-            // (c) X_i = Y_i + sum_{m<i} Ta(i, m) X_m, written in place over the right-hand
+            __syncthreads();  // T_ii A_im visible; every warp has read its right-hand side
+            // (c) X_i = Y_i + sum_{m<i} (T_ii A_im) X_m, written in place over the right-hand
             //     side in bf16 (X_m is read back from there by the later block rows).
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
 #pragma unroll
                 for (int m = 0; m < i; ++m) {
                     const int blk = (i == 1) ? 0 : (i == 2 ? 1 + m : 3 + m);
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        uint32_t a0, a1, a2, a3;
-                        afrag20(Ta + blk * 320, ks, a0, a1, a2, a3);
-                        const uint8_t* xb = xt + (16 * m + 8 * ks) * 128;
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt)
-                            mma_tf32(y[i][nt], a0, a1, a2, a3, bf16_bits(xb + boff[nt][0]),
-                                     bf16_bits(xb + boff[nt][1]));
-                    }
+                    uint32_t af[4], bf[4];
+                    a_frag(Tab + blk * 768, af);
+                    ldsm_x4_t(b_addr(16 * m), bf[0], bf[1], bf[2], bf[3]);
+                    mma_bf16_16816(y[i][0], af[0], af[1], af[2], af[3], bf[0], bf[1]);
+                    mma_bf16_16816(y[i][1], af[0], af[1], af[2], af[3], bf[2], bf[3]);
                 }
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    uint8_t* px = xt + 16 * i * 128 + yoff[nt];
-                    *reinterpret_cast<uint32_t*>(px) = pack2(y[i][nt][0], y[i][nt][1]);
-                    *reinterpret_cast<uint32_t*>(px + 1024) = pack2(y[i][nt][2], y[i][nt][3]);
+                    const int col = 8 * (nb + nt) + 2 * q;
+                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g, col)) = pack2(y[i][nt][0], y[i][nt][1]);
+                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g + 8, col)) = pack2(y[i][nt][2], y[i][nt][3]);
                 }
                 __syncwarp();
             }
