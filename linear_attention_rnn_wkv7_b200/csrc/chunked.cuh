@@ -107,7 +107,7 @@ __device__ __forceinline__ LayR lay_of(int par) {
 //   [P_N hi; A_rk+A_rb Z] ABAR (2)     epilogue 3 -> final MMA A, K block 1
 //   [P_N lo; 0]          K (2 tiles)   epilogue 3 -> final MMA A, K block 2
 // Prologue scratch inside the A_rk tile (free until epilogue 1), in floats.
-constexpr int SCR_TOT = 0, SCR_EC = 512, SCR_EMC = 576, SCR_ELC = 640, SCR_VALID = 704;
+constexpr int SCR_TOT = 0, SCR_C = 512, SCR_EC = 576, SCR_ELC = 640;  // floats
 // Tensor-memory columns (fp32 accumulators, 128 lanes).
 constexpr uint32_t TM_D1 = 0;    // Gram, later MMA-3 (128 cols)
 constexpr uint32_t TM_D1B = 128; // A_rb^T = b~ r~^T (64 cols)
@@ -278,92 +278,106 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
     float* gamma_s = cx.gamma_s;
     uint32_t& mma_phase = cx.mma_phase;
     float* scratch = reinterpret_cast<float*>(smem + L.ARK);  // prologue only
-    uint8_t* validb = reinterpret_cast<uint8_t*>(scratch + SCR_VALID);
     float* F0 = reinterpret_cast<float*>(smem + L.F0);
     const int nv = min(64, cx.len - c0);
     wait_or_abort(cx.bar_tma, par, abort_flag);
 
-        // ---- 2. prefix sums of w (mask folded), E_t = e^{g_t - c} ------------------------
-        {
-            const int p = tid & 31, q = tid >> 5;  // channels 2p, 2p+1; tokens 8q .. 8q+7
-            float2 gl[8];
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int t = 8 * q + i;
-                const bool val = t < nv && (!mask || mask[row0 + c0 + t] != 0);
-                const float2 wv = __bfloat1622float2(
-                    *reinterpret_cast<const __nv_bfloat162*>(smem + L.W + swe(t, 2 * p)));
-                acc.x += val ? wv.x : 0.f;
-                acc.y += val ? wv.y : 0.f;
-                gl[i] = acc;
-                if (p == 0) validb[t] = val ? 1 : 0;
-            }
-            reinterpret_cast<float2*>(scratch + SCR_TOT + q * 64)[p] = acc;
-            __syncthreads();
-            float2 prefix = make_float2(0.f, 0.f), c = prefix, gL = prefix;
-#pragma unroll
-            for (int qq = 0; qq < 8; ++qq) {
-                const float2 tq = reinterpret_cast<const float2*>(scratch + SCR_TOT + qq * 64)[p];
-                if (qq < q) { prefix.x += tq.x; prefix.y += tq.y; }
-                if (qq < 4) { c.x += tq.x; c.y += tq.y; }
-                gL.x += tq.x; gL.y += tq.y;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                reinterpret_cast<float2*>(F0 + (8 * q + i) * 64)[p] =
-                    make_float2(clamped_exp(prefix.x + gl[i].x - c.x),
-                                clamped_exp(prefix.y + gl[i].y - c.y));
-            if (q == 0) {
-                reinterpret_cast<float2*>(scratch + SCR_EC)[p] =
-                    make_float2(clamped_exp(c.x), clamped_exp(c.y));
-                reinterpret_cast<float2*>(scratch + SCR_EMC)[p] =
-                    make_float2(clamped_exp(-c.x), clamped_exp(-c.y));
-                reinterpret_cast<float2*>(scratch + SCR_ELC)[p] =
-                    make_float2(clamped_exp(gL.x - c.x), clamped_exp(gL.y - c.y));
-                reinterpret_cast<float2*>(gamma_s)[p] = make_float2(__expf(gL.x), __expf(gL.y));
-            }
-            __syncthreads();
-        }
-
-        // ---- 3. scaled operands.  Thread (q, j) owns tokens 2q, 2q+1 and channels
-        //         8j..8j+7, so E_{t-1} of its second token is E_t of its first and the
-        //         per-channel constants are read once; each thread rewrites only the
-        //         chunks it read, and Khat waits until every E_t read is done. ---------
+        // ---- 2. prefix sums of w (mask folded) and every scaled operand, in one pass.
+        //         Thread (q, j) owns tokens 2q, 2q+1 and channels 8j..8j+7: a shuffle
+        //         scan over the warp's four token pairs, warp totals exchanged through
+        //         shared memory, per-channel constants from warp 0, then E_t and the
+        //         operands, written in place. ------------------------------------------
         {
             const int j = tid & 7, t0 = 2 * (tid >> 3);
-            float ec[8], elc[8], Ep[8];
+            const bool va = t0 < nv && (!mask || mask[row0 + c0 + t0] != 0);
+            const bool vb = t0 + 1 < nv && (!mask || mask[row0 + c0 + t0 + 1] != 0);
+            const uint32_t offa = sw(t0, j), offb = sw(t0 + 1, j);
+            float wa[8], wb[8], incl[8];
+            unpack8(*reinterpret_cast<const uint4*>(smem + L.W + offa), wa);
+            unpack8(*reinterpret_cast<const uint4*>(smem + L.W + offb), wb);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                wa[e] = va ? wa[e] : 0.f;
+                wb[e] = vb ? wb[e] : 0.f;
+                incl[e] = wa[e] + wb[e];
+            }
+#pragma unroll
+            for (int d = 8; d < 32; d *= 2) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float up = __shfl_up_sync(0xffffffffu, incl[e], d);
+                    if (lane >= d) incl[e] += up;
+                }
+            }
+            float* wt = scratch + SCR_TOT;  // [warp][channel] sums of w over the warp's 8 tokens
+            if (lane >= 24) {
+                *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j) =
+                    make_float4(incl[0], incl[1], incl[2], incl[3]);
+                *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j + 4) =
+                    make_float4(incl[4], incl[5], incl[6], incl[7]);
+            }
+            __syncthreads();
+            if (warp == 0) {  // per channel: c = g_31, g_L, and the exps built from them
+                const int ch = 2 * lane;
+                float2 c = make_float2(0.f, 0.f), gL = c;
+#pragma unroll
+                for (int w2 = 0; w2 < 8; ++w2) {
+                    const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
+                    if (w2 < 4) { c.x += x.x; c.y += x.y; }
+                    gL.x += x.x; gL.y += x.y;
+                }
+                reinterpret_cast<float2*>(scratch + SCR_C)[lane] = c;
+                reinterpret_cast<float2*>(scratch + SCR_EC)[lane] =
+                    make_float2(clamped_exp(c.x), clamped_exp(c.y));
+                reinterpret_cast<float2*>(scratch + SCR_ELC)[lane] =
+                    make_float2(clamped_exp(gL.x - c.x), clamped_exp(gL.y - c.y));
+                reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(__expf(gL.x), __expf(gL.y));
+            }
+            float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ga[e] = incl[e] - wb[e];
+#pragma unroll
+            for (int w2 = 0; w2 < 7; ++w2) {
+                if (w2 < warp) {
+                    const float4 x0 = *reinterpret_cast<const float4*>(wt + w2 * 64 + 8 * j);
+                    const float4 x1 = *reinterpret_cast<const float4*>(wt + w2 * 64 + 8 * j + 4);
+                    ga[0] += x0.x; ga[1] += x0.y; ga[2] += x0.z; ga[3] += x0.w;
+                    ga[4] += x1.x; ga[5] += x1.y; ga[6] += x1.z; ga[7] += x1.w;
+                }
+            }
+            __syncthreads();  // per-channel constants ready
+            float cc[8], ec[8], elc[8];
+            *reinterpret_cast<float4*>(cc) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[0];
+            *reinterpret_cast<float4*>(cc + 4) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[1];
             *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[0];
             *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[1];
             *reinterpret_cast<float4*>(elc) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[0];
             *reinterpret_cast<float4*>(elc + 4) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[1];
-            {
-                const float* Emrow = t0 > 0 ? F0 + (t0 - 1) * 64 + 8 * j : scratch + SCR_EMC + 8 * j;
-                *reinterpret_cast<float4*>(Ep) = reinterpret_cast<const float4*>(Emrow)[0];
-                *reinterpret_cast<float4*>(Ep + 4) = reinterpret_cast<const float4*>(Emrow)[1];
+            float Ep[8];  // E at token t0 - 1
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float prev = __shfl_up_sync(0xffffffffu, ga[e] + wb[e], 8);  // g_{t0-1}
+                Ep[e] = clamped_exp(((lane >= 8) ? prev : ga[e] - wa[e]) - cc[e]);
             }
-            float4 o_khat[2][2];
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
-                const int t = t0 + it;
-                const bool val = validb[t] != 0;
-                const uint32_t off = sw(t, j);
+                const uint32_t off = it ? offb : offa;
+                const bool val = it ? vb : va;
                 float rv[8], av[8], kv[8], bv[8];
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.R + off), rv);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.A + off), av);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.B + off), bv);
-                float E[8];
-                *reinterpret_cast<float4*>(E) = reinterpret_cast<const float4*>(F0 + t * 64 + 8 * j)[0];
-                *reinterpret_cast<float4*>(E + 4) = reinterpret_cast<const float4*>(F0 + t * 64 + 8 * j)[1];
                 float rt[8], at[8], kt[8], btl[8], abar[8], bhat[8], khat[8], rbar[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float inv = __frcp_rn(E[e]);
+                    const float g = it ? ga[e] + wb[e] : ga[e];
+                    const float E = clamped_exp(g - cc[e]);
+                    const float inv = clamped_exp(cc[e] - g);
                     const float a_ = val ? av[e] : 0.f, k_ = val ? kv[e] : 0.f,
                                 b_ = val ? bv[e] : 0.f;
                     const float il = elc[e] * inv;  // e^{g_L - g_t}
-                    rt[e] = rv[e] * E[e];
+                    rt[e] = rv[e] * E;
                     at[e] = a_ * Ep[e];
                     kt[e] = k_ * inv;
                     btl[e] = b_ * inv;
@@ -371,7 +385,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     bhat[e] = b_ * il;
                     khat[e] = k_ * il;
                     rbar[e] = rt[e] * ec[e];
-                    Ep[e] = E[e];  // E_{t-1} of the next token
+                    Ep[e] = E;  // E_{t-1} of the next token
                 }
                 *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rt);
                 *reinterpret_cast<uint4*>(smem + L.A + off) = pack8(at);
@@ -380,15 +394,9 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 *reinterpret_cast<uint4*>(smem + L.W + off) = pack8(bhat);
                 *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8(abar);
                 *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8(rbar);
-                o_khat[it][0] = make_float4(khat[0], khat[1], khat[2], khat[3]);
-                o_khat[it][1] = make_float4(khat[4], khat[5], khat[6], khat[7]);
-            }
-            __syncthreads();  // every E_t read before F0 is overwritten by Khat
-#pragma unroll
-            for (int it = 0; it < 2; ++it) {
                 float4* kh = reinterpret_cast<float4*>(F0 + (t0 + it) * 64 + 8 * j);
-                kh[0] = o_khat[it][0];
-                kh[1] = o_khat[it][1];
+                kh[0] = make_float4(khat[0], khat[1], khat[2], khat[3]);
+                kh[1] = make_float4(khat[4], khat[5], khat[6], khat[7]);
             }
             fence_proxy_async();
             tc_fence_before();
