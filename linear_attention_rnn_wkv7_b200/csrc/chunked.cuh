@@ -150,9 +150,17 @@ __device__ __forceinline__ void unpack8(uint4 u, float* v) {
 __device__ __forceinline__ float bf16_at(const uint8_t* tile, uint32_t row, uint32_t col) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + swe(row, col)));
 }
-__device__ __forceinline__ float clamped_exp(float x) {
-    return __expf(fminf(fmaxf(x, -kExpClamp), kExpClamp));
+// 2^x by the hardware approximation (relative error about 2^-22, subnormal results
+// flushed to zero); the prologue keeps
+// log decays in log2 units so that every exponential is one such instruction.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kClamp2 = kExpClamp * kLog2e;  // the exponent clamp in log2 units
+__device__ __forceinline__ float clamp2(float x) { return fminf(fmaxf(x, -kClamp2), kClamp2); }
 
 // Load `n16` groups of 16 TMEM columns starting at column `col` for this warp's lanes.
 template <int N16>
@@ -296,9 +304,9 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             unpack8(*reinterpret_cast<const uint4*>(smem + L.W + offa), wa);
             unpack8(*reinterpret_cast<const uint4*>(smem + L.W + offb), wb);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                wa[e] = va ? wa[e] : 0.f;
-                wb[e] = vb ? wb[e] : 0.f;
+            for (int e = 0; e < 8; ++e) {  // log decays in log2 units from here on
+                wa[e] = va ? wa[e] * kLog2e : 0.f;
+                wb[e] = vb ? wb[e] * kLog2e : 0.f;
                 incl[e] = wa[e] + wb[e];
             }
 #pragma unroll
@@ -328,10 +336,10 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 }
                 reinterpret_cast<float2*>(scratch + SCR_C)[lane] = c;
                 reinterpret_cast<float2*>(scratch + SCR_EC)[lane] =
-                    make_float2(clamped_exp(c.x), clamped_exp(c.y));
+                    make_float2(ex2(clamp2(c.x)), ex2(clamp2(c.y)));
                 reinterpret_cast<float2*>(scratch + SCR_ELC)[lane] =
-                    make_float2(clamped_exp(gL.x - c.x), clamped_exp(gL.y - c.y));
-                reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(__expf(gL.x), __expf(gL.y));
+                    make_float2(ex2(clamp2(gL.x - c.x)), ex2(clamp2(gL.y - c.y)));
+                reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(ex2(gL.x), ex2(gL.y));
             }
             float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
 #pragma unroll
@@ -357,8 +365,9 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float prev = __shfl_up_sync(0xffffffffu, ga[e] + wb[e], 8);  // g_{t0-1}
-                Ep[e] = clamped_exp(((lane >= 8) ? prev : ga[e] - wa[e]) - cc[e]);
+                Ep[e] = ex2(clamp2(((lane >= 8) ? prev : ga[e] - wa[e]) - cc[e]));
             }
+            float rts[2][8], ats[2][8];  // fp32 r~ and a~, kept for Rbar and Abar
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const uint32_t off = it ? offb : offa;
@@ -368,32 +377,29 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.A + off), av);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.B + off), bv);
-                float rt[8], at[8], kt[8], btl[8], abar[8], bhat[8], khat[8], rbar[8];
+                float kt[8], btl[8], bhat[8], khat[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float g = it ? ga[e] + wb[e] : ga[e];
-                    const float E = clamped_exp(g - cc[e]);
-                    const float inv = clamped_exp(cc[e] - g);
-                    const float a_ = val ? av[e] : 0.f, k_ = val ? kv[e] : 0.f,
-                                b_ = val ? bv[e] : 0.f;
+                    const float d = clamp2(g - cc[e]);
+                    const float E = ex2(d);
+                    // A masked token writes nothing: its a, k, b scales are zero.
+                    const float inv = val ? ex2(-d) : 0.f;
+                    const float ep = val ? Ep[e] : 0.f;
                     const float il = elc[e] * inv;  // e^{g_L - g_t}
-                    rt[e] = rv[e] * E;
-                    at[e] = a_ * Ep[e];
-                    kt[e] = k_ * inv;
-                    btl[e] = b_ * inv;
-                    abar[e] = at[e] * ec[e];
-                    bhat[e] = b_ * il;
-                    khat[e] = k_ * il;
-                    rbar[e] = rt[e] * ec[e];
+                    rts[it][e] = rv[e] * E;
+                    ats[it][e] = av[e] * ep;
+                    kt[e] = kv[e] * inv;
+                    btl[e] = bv[e] * inv;
+                    bhat[e] = bv[e] * il;
+                    khat[e] = kv[e] * il;
                     Ep[e] = E;  // E_{t-1} of the next token
                 }
-                *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rt);
-                *reinterpret_cast<uint4*>(smem + L.A + off) = pack8(at);
+                *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rts[it]);
+                *reinterpret_cast<uint4*>(smem + L.A + off) = pack8(ats[it]);
                 *reinterpret_cast<uint4*>(smem + L.K + off) = pack8(kt);
                 *reinterpret_cast<uint4*>(smem + L.B + off) = pack8(btl);
                 *reinterpret_cast<uint4*>(smem + L.W + off) = pack8(bhat);
-                *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8(abar);
-                *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8(rbar);
                 float4* kh = reinterpret_cast<float4*>(F0 + (t0 + it) * 64 + 8 * j);
                 kh[0] = make_float4(khat[0], khat[1], khat[2], khat[3]);
                 kh[1] = make_float4(khat[4], khat[5], khat[6], khat[7]);
@@ -401,25 +407,41 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
+
+            // Gram: D1 = [r~; a~] [k~; b~]^T  (128 x 128 x 64) on the tensor cores.
+            if (tid == 0) {
+                tc_fence_after();
+                constexpr uint32_t id = idesc_bf16(128, 128, false, false);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_D1, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
+                              smem_desc(sbase + L.K + 32 * kk, 16, 1024), id, kk > 0);
+                // A_rb^T directly: rows s of b~ against r~ (rows 64..127 of this A operand
+                // read the next tile and are never used).
+                constexpr uint32_t id2 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.B + 32 * kk, 16, 1024),
+                              smem_desc(sbase + L.R + 32 * kk, 16, 1024), id2, kk > 0);
+                umma_commit(bar_mma);
+            }
+            // While it runs: Abar = a~ e^c and Rbar = r~ e^c (tiles the Gram does not read,
+            // first read after epilogue 1's barrier).
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const uint32_t off = it ? offb : offa;
+                float abar[8], rbar[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    abar[e] = ats[it][e] * ec[e];
+                    rbar[e] = rts[it][e] * ec[e];
+                }
+                *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8(abar);
+                *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8(rbar);
+            }
         }
 
-        // ---- 4. Gram: D1 = [r~; a~] [k~; b~]^T  (128 x 128 x 64) ---------------------------
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 128, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_D1, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
-                          smem_desc(sbase + L.K + 32 * kk, 16, 1024), id, kk > 0);
-            // A_rb^T directly: rows s of b~ against r~ (rows 64..127 of this A operand
-            // read the next tile and are never used).
-            constexpr uint32_t id2 = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.B + 32 * kk, 16, 1024),
-                          smem_desc(sbase + L.R + 32 * kk, 16, 1024), id2, kk > 0);
-            umma_commit(bar_mma);
-        }
+        // ---- 4. Gram wait ------------------------------------------------------------------
         wait_or_abort(bar_mma, mma_phase, abort_flag);
         mma_phase ^= 1;
         tc_fence_after();
@@ -609,62 +631,56 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         tc_fence_after();
 
         // ---- 8. epilogue 3: assemble the final A operand.  Rows k (lanes 0..63): M'
-        //         and the hi/lo split of P_N, whose 64 columns are shared by warps 0/1
-        //         (after M') and 4/5.  Rows t (lanes 64..127): Q and P_O. --------------
+        //         and the hi/lo split of P_N; warps 0/1 take columns 0..31 of both,
+        //         warps 4/5 columns 32..63.  Rows t (lanes 64..127): Q (warps 2/3) and
+        //         P_O (warps 6/7). ---------------------------------------------------
         {
             if (wq < 2) {
                 const int k = m_row;
-                auto split_pn = [&](const float* v, int c0n) {  // P_N = Bhat^T Z + Khat^T
+                float v[64];  // M' = Bhat^T W, then P_N - Khat^T = Bhat^T Z, 32 columns each
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float hi[8], lo[8];
+                for (int i = 0; i < 4; ++i) {
+                    float tmp[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1 + (i >> 1) * 64 + 32 * wh + 16 * (i & 1),
+                              tmp);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int s_ = 8 * (c0n + c) + e;
-                            const float pn = v[8 * c + e] + F0[s_ * 64 + k];
-                            hi[e] = __bfloat162float(__float2bfloat16_rn(pn));
-                            lo[e] = pn - hi[e];
-                        }
-                        *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, c0n + c)) = pack8(hi);
-                        *reinterpret_cast<uint4*>(smem + L.K + sw(k, c0n + c)) = pack8(lo);
+                    for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
+                }
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(smem + L.R + sw(k, 4 * wh + c)) = pack8(v + 8 * c);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {  // P_N = Bhat^T Z + Khat^T, split into bf16 hi + lo
+                    float hi[8], lo[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int s_ = 8 * (4 * wh + c) + e;
+                        const float pn = v[32 + 8 * c + e] + F0[s_ * 64 + k];
+                        hi[e] = __bfloat162float(__float2bfloat16_rn(pn));
+                        lo[e] = pn - hi[e];
                     }
-                };
-                if (wh == 0) {
-                    float v[64];
-                    tmem_row<4>(tmem + TM_D1, wq, 0, v);  // M' = Bhat^T W
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(smem + L.R + sw(k, c)) = pack8(v + 8 * c);
-                    tmem_row<2>(tmem + TM_D1, wq, 64, v);  // P_N columns 0..31
-                    split_pn(v, 0);
-                } else {
-                    float v[32];
-                    tmem_row<2>(tmem + TM_D1, wq, 96, v);  // P_N columns 32..63
-                    split_pn(v, 4);
+                    *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, 4 * wh + c)) = pack8(hi);
+                    *reinterpret_cast<uint4*>(smem + L.K + sw(k, 4 * wh + c)) = pack8(lo);
                 }
             } else {
                 const int tp = m_row - 64;
                 float v[64];
                 tmem_row<4>(tmem + TM_D1, wq, 64 * wh, v);
-                if (wh == 0) {  // Q = A_rb W + Rbar
+                // Q = A_rb W + Rbar (wh 0) or P_O = A_rb Z + A_rk (wh 1); P_O's lo block is zero.
+                const uint32_t src = wh ? L.ARK : L.RBAR, dst = wh ? L.ABAR : L.R;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float rb[8];
-                        unpack8(*reinterpret_cast<const uint4*>(smem + L.RBAR + sw(tp, c)), rb);
+                for (int c = 0; c < 8; ++c) {
+                    float x[8];
+                    unpack8(*reinterpret_cast<const uint4*>(smem + src + sw(tp, c)), x);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) rb[e] += v[8 * c + e];
-                        *reinterpret_cast<uint4*>(smem + L.R + sw(m_row, c)) = pack8(rb);
-                    }
-                } else {  // P_O = A_rb Z + A_rk; the lo block is zero for these rows
+                    for (int e = 0; e < 8; ++e) x[e] += v[8 * c + e];
+                    *reinterpret_cast<uint4*>(smem + dst + sw(m_row, c)) = pack8(x);
+                }
+                if (wh) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float po[8];
-                        unpack8(*reinterpret_cast<const uint4*>(smem + L.ARK + sw(tp, c)), po);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) po[e] += v[8 * c + e];
-                        *reinterpret_cast<uint4*>(smem + L.ABAR + sw(m_row, c)) = pack8(po);
+                    for (int c = 0; c < 8; ++c)
                         *reinterpret_cast<uint4*>(smem + L.K + sw(m_row, c)) = make_uint4(0, 0, 0, 0);
-                    }
                 }
             }
             // The final MMA accumulates onto its tensor-memory columns: rows 0..63 hold
