@@ -211,6 +211,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                  : "r"(addr));
 }
 
+// Transpose of an 8x8 b16 matrix held one 32-bit pair per lane (lane l: row l / 4,
+// columns 2 (l % 4), +1), returned in the same layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -446,54 +454,73 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 5. epilogue 1: masked A_rk, A_rb^T, A_ak (bf16) and A_ab (fp32), each row-wise --
+        // ---- 5. epilogue 1: masked A_rk, A_rb^T, A_ak (bf16) and A_ab (fp32), each row-wise;
+        //         the second 32 columns load from tensor memory while the first are stored.
         {
             float v[64];
             // Warps 4 and 5 read A_rb^T (lanes 0..63 of D1b); the others read D1.
-            tmem_row<4>(tmem + ((wq < 2 && wh == 1) ? TM_D1B : TM_D1 + 64 * wh), wq, 0, v);
-            if (wq < 2) {
-                const int t = m_row;  // row of r~
-                if (wh == 0) {  // A_rk[t][s] = v[s], kept for s <= t -> row t
+            const uint32_t ta = tmem + ((uint32_t)(32 * wq) << 16) +
+                                ((wq < 2 && wh == 1) ? TM_D1B : TM_D1 + 64 * wh);
+            auto load32 = [&](int h) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float x[8];
+                for (int i = 0; i < 2; ++i) {
+                    float tmp[16];
+                    tmem_ld16(ta + 32 * h + 16 * i, tmp);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
-                        *reinterpret_cast<uint4*>(smem + L.ARK + sw(t, c)) = pack8(x);
+                    for (int j2 = 0; j2 < 16; ++j2) v[32 * h + 16 * i + j2] = tmp[j2];
+                }
+            };
+            auto emit = [&](int h) {  // columns [32h, 32h + 32)
+                if (wq < 2) {
+                    const int t = m_row;  // row of r~
+                    if (wh == 0) {  // A_rk[t][s] = v[s], kept for s <= t -> row t
+#pragma unroll
+                        for (int c = 4 * h; c < 4 * h + 4; ++c) {
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
+                            *reinterpret_cast<uint4*>(smem + L.ARK + sw(t, c)) = pack8(x);
+                        }
+                    } else {  // row s = m_row of A_rb^T: A_rb[t][s] = v[t], kept for s <= t
+                        const int s_ = m_row;
+#pragma unroll
+                        for (int c = 4 * h; c < 4 * h + 4; ++c) {
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = (s_ <= 8 * c + e) ? v[8 * c + e] : 0.f;
+                            *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8(x);
+                        }
                     }
-                } else {  // row s = m_row of A_rb^T: A_rb[t][s] = v[t], kept for s <= t
-                    const int s_ = m_row;
+                } else {
+                    const int t = m_row - 64;  // row of a~
+                    if (wh == 0) {  // A_ak[t][s] = v[s], kept for s < t -> row t
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float x[8];
+                        for (int c = 4 * h; c < 4 * h + 4; ++c) {
+                            float x[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = (s_ <= 8 * c + e) ? v[8 * c + e] : 0.f;
-                        *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8(x);
+                            for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
+                            *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8(x);
+                        }
+                    } else {  // A_ab[t][s], kept for s < t -> fp32 row t
+                        float* aab = reinterpret_cast<float*>(smem + L.R);
+#pragma unroll
+                        for (int c4 = 8 * h; c4 < 8 * h + 8; ++c4) {
+                            float4 x;
+                            x.x = (4 * c4 + 0 < t) ? v[4 * c4 + 0] : 0.f;
+                            x.y = (4 * c4 + 1 < t) ? v[4 * c4 + 1] : 0.f;
+                            x.z = (4 * c4 + 2 < t) ? v[4 * c4 + 2] : 0.f;
+                            x.w = (4 * c4 + 3 < t) ? v[4 * c4 + 3] : 0.f;
+                            *reinterpret_cast<float4*>(aab + fidx(t, 4 * c4)) = x;
+                        }
                     }
                 }
-            } else {
-                const int t = m_row - 64;  // row of a~
-                if (wh == 0) {  // A_ak[t][s] = v[s], kept for s < t -> row t
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float x[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
-                        *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8(x);
-                    }
-                } else {  // A_ab[t][s], kept for s < t -> fp32 row t
-                    float* aab = reinterpret_cast<float*>(smem + L.R);
-#pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        float4 x;
-                        x.x = (4 * c4 + 0 < t) ? v[4 * c4 + 0] : 0.f;
-                        x.y = (4 * c4 + 1 < t) ? v[4 * c4 + 1] : 0.f;
-                        x.z = (4 * c4 + 2 < t) ? v[4 * c4 + 2] : 0.f;
-                        x.w = (4 * c4 + 3 < t) ? v[4 * c4 + 3] : 0.f;
-                        *reinterpret_cast<float4*>(aab + fidx(t, 4 * c4)) = x;
-                    }
-                }
-            }
+            };
+            load32(0);
+            tmem_ld_wait();
+            load32(1);
+            emit(0);
+            tmem_ld_wait();
+            emit(1);
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
@@ -591,25 +618,31 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             }
             __syncthreads();  // T_ii A_im visible; every warp has read its right-hand side
             // (c) X_i = Y_i + sum_{m<i} (T_ii A_im) X_m, written in place over the right-hand
-            //     side in bf16 (X_m is read back from there by the later block rows).
+            //     side in bf16 for MMA-3.  Later block rows take X_m as their B operand
+            //     straight from registers: the bf16 C fragments, transposed 8x8 at a time.
+            uint32_t xb[3][4];  // B fragments of X_0..X_2 (n-tile 0: b0 b1, n-tile 1: b0 b1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
 #pragma unroll
                 for (int m = 0; m < i; ++m) {
                     const int blk = (i == 1) ? 0 : (i == 2 ? 1 + m : 3 + m);
-                    uint32_t af[4], bf[4];
+                    uint32_t af[4];
                     a_frag(Tab + blk * 768, af);
-                    ldsm_x4_t(b_addr(16 * m), bf[0], bf[1], bf[2], bf[3]);
-                    mma_bf16_16816(y[i][0], af[0], af[1], af[2], af[3], bf[0], bf[1]);
-                    mma_bf16_16816(y[i][1], af[0], af[1], af[2], af[3], bf[2], bf[3]);
+                    mma_bf16_16816(y[i][0], af[0], af[1], af[2], af[3], xb[m][0], xb[m][1]);
+                    mma_bf16_16816(y[i][1], af[0], af[1], af[2], af[3], xb[m][2], xb[m][3]);
                 }
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int col = 8 * (nb + nt) + 2 * q;
-                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g, col)) = pack2(y[i][nt][0], y[i][nt][1]);
-                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g + 8, col)) = pack2(y[i][nt][2], y[i][nt][3]);
+                    const uint32_t top = pack2(y[i][nt][0], y[i][nt][1]);
+                    const uint32_t bot = pack2(y[i][nt][2], y[i][nt][3]);
+                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g, col)) = top;
+                    *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g + 8, col)) = bot;
+                    if (i < 3) {
+                        xb[i][2 * nt] = movmatrix_t(top);
+                        xb[i][2 * nt + 1] = movmatrix_t(bot);
+                    }
                 }
-                __syncwarp();
             }
             fence_proxy_async();
             tc_fence_before();
@@ -638,18 +671,22 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             if (wq < 2) {
                 const int k = m_row;
                 float v[64];  // M' = Bhat^T W, then P_N - Khat^T = Bhat^T Z, 32 columns each
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                auto load16 = [&](int i) {
                     float tmp[16];
                     tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1 + (i >> 1) * 64 + 32 * wh + 16 * (i & 1),
                               tmp);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
-                }
+                };
+                load16(0);
+                load16(1);
                 tmem_ld_wait();
+                load16(2);  // P_N columns load while M' is stored
+                load16(3);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     *reinterpret_cast<uint4*>(smem + L.R + sw(k, 4 * wh + c)) = pack8(v + 8 * c);
+                tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {  // P_N = Bhat^T Z + Khat^T, split into bf16 hi + lo
                     float hi[8], lo[8];
@@ -666,17 +703,33 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             } else {
                 const int tp = m_row - 64;
                 float v[64];
-                tmem_row<4>(tmem + TM_D1, wq, 64 * wh, v);
-                // Q = A_rb W + Rbar (wh 0) or P_O = A_rb Z + A_rk (wh 1); P_O's lo block is zero.
+                auto load16 = [&](int i) {
+                    float tmp[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1 + 64 * wh + 16 * i, tmp);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
+                };
+                // Q = A_rb W + Rbar (wh 0) or P_O = A_rb Z + A_rk (wh 1); P_O's lo block is
+                // zero.  The second 32 columns load while the first are stored.
                 const uint32_t src = wh ? L.ARK : L.RBAR, dst = wh ? L.ABAR : L.R;
+                auto emit = [&](int h) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float x[8];
-                    unpack8(*reinterpret_cast<const uint4*>(smem + src + sw(tp, c)), x);
+                    for (int c = 4 * h; c < 4 * h + 4; ++c) {
+                        float x[8];
+                        unpack8(*reinterpret_cast<const uint4*>(smem + src + sw(tp, c)), x);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] += v[8 * c + e];
-                    *reinterpret_cast<uint4*>(smem + dst + sw(m_row, c)) = pack8(x);
-                }
+                        for (int e = 0; e < 8; ++e) x[e] += v[8 * c + e];
+                        *reinterpret_cast<uint4*>(smem + dst + sw(m_row, c)) = pack8(x);
+                    }
+                };
+                load16(0);
+                load16(1);
+                tmem_ld_wait();
+                load16(2);
+                load16(3);
+                emit(0);
+                tmem_ld_wait();
+                emit(1);
                 if (wh) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
