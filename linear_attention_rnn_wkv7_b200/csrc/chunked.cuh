@@ -4,31 +4,33 @@
 // The recurrence (rwkv-ops 0.9.0 README, "rwkv7op 使用方法")
 //     u_t = S_{t-1}^T a_t;  S_t = diag(exp w_t) S_{t-1} + b_t u_t^T + k_t v_t^T;  o_t = S_t^T r_t
 // is rewritten exactly for a chunk of L = 64 tokens (t = 0..63, state S0 at the
-// chunk start).  With g_t = sum_{j<=t} w_j (per channel, log space), a
-// reference c = g_31 and E_t = exp(g_t - c):
+// chunk start).  With g_t = sum_{j<=t} w_j (per channel, log space), the chunk's
+// last prefix g_L = g_63 as reference and E_t = exp(g_t - g_L) (>= 1):
 //   r~ = r E_t, a~ = a E_{t-1}, k~ = k / E_t, b~ = b / E_t        (Gram operands)
 //   A_rk[t][s] = r~_t.k~_s (s<=t), A_rb = r~.b~ (s<=t), A_ak = a~.k~ (s<t), A_ab = a~.b~ (s<t)
 //   T = (I - A_ab)^-1 (the UT / WY representation of the chunk's rank-1 products)
-//   Abar = a e^{g_{t-1}}, Rbar = r e^{g_t}, Bhat = b e^{g_L - g_t}, Khat = k e^{g_L - g_t}
+//   Abar = a e^{g_{t-1}} = a~ e^{g_L}, Rbar = r e^{g_t} = r~ e^{g_L},
+//   Bhat = b e^{g_L - g_t} = b~, Khat = k e^{g_L - g_t} = k~ (kept in fp32)
 //   W = T Abar, Z = T A_ak              (so the read vectors are U = W S0 + Z V)
 //   S_L = diag(e^{g_L}) S0 + (Bhat^T W) S0 + (Khat^T + Bhat^T Z) V
 //   O   = (Rbar + A_rb W) S0 + (A_rk + A_rb Z) V
 // Only the last product depends on S0.  One chunk costs three tcgen05 MMA groups
 // (the Gram matrix, the Bhat/A_rb products with [W | Z], and the final product
 // with [S0; V]) with fp32 accumulators in tensor memory.  [W | Z] = T [Abar | A_ak]
-// comes from a block forward substitution on warp-level tf32 MMAs (each warp owns
+// comes from a block forward substitution on warp-level bf16 MMAs (each warp owns
 // 16 of its 128 columns), after the 16x16 diagonal blocks of T by fp32 forward
 // substitution.  CUDA cores do the prefix sums and exps and the tensor-memory ->
 // shared-memory epilogues that re-layout each result as the next product's operand.
 // The write term Khat^T + Bhat^T Z enters the final MMA as a hi/lo pair of bf16
 // matrices (about 16 significant bits), which keeps the fp32 final state within
-// 1e-3 of the fp64 recurrence; all other tensor-core operands are bf16 or tf32.
+// 1e-3 of the fp64 recurrence; all other tensor-core operands are bf16.
 //
-// A masked or out-of-range token is folded into the loads as w = a = k = b = 0:
-// its transition is then the identity and it writes nothing, and its output is
-// read from the carried state.  Exps are clamped to [-40, 40] around c, so the
-// factorisation is exact while |g_t - g_31| <= 40 inside a chunk (per-step log
-// decay >= -1.2; the RWKV-7 parametrisation keeps it >= -0.607).
+// A masked or out-of-range token is folded into the loads as w = 0 and zero a, k, b
+// scales: its transition is then the identity and it writes nothing, and its output
+// is read from the carried state.  Exps are clamped to [-80, 80] (every operand and
+// Gram entry stays finite in fp32 and bf16), so the factorisation is exact while
+// g_t - g_L <= 80 inside a chunk (per-step log decay >= -1.26; the RWKV-7
+// parametrisation keeps it >= -0.607).
 #pragma once
 #include <cuda.h>
 
@@ -107,13 +109,13 @@ __device__ __forceinline__ LayR lay_of(int par) {
 //   [P_N hi; A_rk+A_rb Z] ABAR (2)     epilogue 3 -> final MMA A, K block 1
 //   [P_N lo; 0]          K (2 tiles)   epilogue 3 -> final MMA A, K block 2
 // Prologue scratch inside the A_rk tile (free until epilogue 1), in floats.
-constexpr int SCR_TOT = 0, SCR_C = 512, SCR_EC = 576, SCR_ELC = 640;  // floats
+constexpr int SCR_TOT = 0, SCR_C = 512;  // floats
 // Tensor-memory columns (fp32 accumulators, 128 lanes).
 constexpr uint32_t TM_D1 = 0;    // Gram, later MMA-3 (128 cols)
 constexpr uint32_t TM_D1B = 128; // A_rb^T = b~ r~^T (64 cols)
 constexpr uint32_t TM_DF = 192;  // [S update; O] (64 cols)
 constexpr uint32_t kTmemCols = 256;
-constexpr float kExpClamp = 40.f;
+constexpr float kExpClamp = 80.f;
 
 // Byte offset of 16-byte chunk `c` of row `row` in a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t sw(uint32_t row, uint32_t c) {
@@ -137,6 +139,17 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 __device__ __forceinline__ uint4 pack8(const float* v) {
     return make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
+}
+// fp16 pairs, rounded to nearest and saturated at +-65504 (never inf).  fp16 keeps
+// three more significant bits than bf16; it carries the operands of the [W | Z]
+// substitution and of MMA-3, whose magnitudes stay near 1.
+__device__ __forceinline__ uint32_t pack2h(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+__device__ __forceinline__ uint4 pack8h(const float* v) {
+    return make_uint4(pack2h(v[0], v[1]), pack2h(v[2], v[3]), pack2h(v[4], v[5]), pack2h(v[6], v[7]));
 }
 __device__ __forceinline__ void unpack8(uint4 u, float* v) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -193,6 +206,15 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// The same with fp16 operands.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
         "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -333,20 +355,15 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     make_float4(incl[4], incl[5], incl[6], incl[7]);
             }
             __syncthreads();
-            if (warp == 0) {  // per channel: c = g_31, g_L, and the exps built from them
+            if (warp == 0) {  // per channel: the reference c = g_L and e^{g_L}
                 const int ch = 2 * lane;
-                float2 c = make_float2(0.f, 0.f), gL = c;
+                float2 gL = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int w2 = 0; w2 < 8; ++w2) {
                     const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
-                    if (w2 < 4) { c.x += x.x; c.y += x.y; }
                     gL.x += x.x; gL.y += x.y;
                 }
-                reinterpret_cast<float2*>(scratch + SCR_C)[lane] = c;
-                reinterpret_cast<float2*>(scratch + SCR_EC)[lane] =
-                    make_float2(ex2(clamp2(c.x)), ex2(clamp2(c.y)));
-                reinterpret_cast<float2*>(scratch + SCR_ELC)[lane] =
-                    make_float2(ex2(clamp2(gL.x - c.x)), ex2(clamp2(gL.y - c.y)));
+                reinterpret_cast<float2*>(scratch + SCR_C)[lane] = gL;
                 reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(ex2(gL.x), ex2(gL.y));
             }
             float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
@@ -362,13 +379,11 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 }
             }
             __syncthreads();  // per-channel constants ready
-            float cc[8], ec[8], elc[8];
+            float cc[8], ec[8];  // c = g_L (log2 units) and e^{g_L}
             *reinterpret_cast<float4*>(cc) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[0];
             *reinterpret_cast<float4*>(cc + 4) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[1];
-            *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[0];
-            *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(scratch + SCR_EC + 8 * j)[1];
-            *reinterpret_cast<float4*>(elc) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[0];
-            *reinterpret_cast<float4*>(elc + 4) = reinterpret_cast<const float4*>(scratch + SCR_ELC + 8 * j)[1];
+            *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[0];
+            *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[1];
             float Ep[8];  // E at token t0 - 1
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -385,32 +400,37 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.A + off), av);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv);
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.B + off), bv);
-                float kt[8], btl[8], bhat[8], khat[8];
+                float kt[8], btl[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float g = it ? ga[e] + wb[e] : ga[e];
                     const float d = clamp2(g - cc[e]);
-                    const float E = ex2(d);
+                    const float E = ex2(d);  // e^{g_t - g_L}
                     // A masked token writes nothing: its a, k, b scales are zero.
                     const float inv = val ? ex2(-d) : 0.f;
                     const float ep = val ? Ep[e] : 0.f;
-                    const float il = elc[e] * inv;  // e^{g_L - g_t}
                     rts[it][e] = rv[e] * E;
                     ats[it][e] = av[e] * ep;
-                    kt[e] = kv[e] * inv;
-                    btl[e] = bv[e] * inv;
-                    bhat[e] = bv[e] * il;
-                    khat[e] = kv[e] * il;
+                    kt[e] = kv[e] * inv;   // = Khat (fp32)
+                    btl[e] = bv[e] * inv;  // = Bhat
                     Ep[e] = E;  // E_{t-1} of the next token
                 }
                 *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rts[it]);
                 *reinterpret_cast<uint4*>(smem + L.A + off) = pack8(ats[it]);
-                *reinterpret_cast<uint4*>(smem + L.K + off) = pack8(kt);
+                const uint4 kq = pack8(kt);
+                *reinterpret_cast<uint4*>(smem + L.K + off) = kq;
+                {  // k~ - bf16(k~) in bf16: the Gram adds [r~; a~] k~_lo^T to A_rk and A_ak
+                    float khi[8], klo[8];
+                    unpack8(kq, khi);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) klo[e] = kt[e] - khi[e];
+                    *reinterpret_cast<uint4*>(smem + L.ARBT + off) = pack8(klo);
+                }
                 *reinterpret_cast<uint4*>(smem + L.B + off) = pack8(btl);
-                *reinterpret_cast<uint4*>(smem + L.W + off) = pack8(bhat);
+                *reinterpret_cast<uint4*>(smem + L.W + off) = pack8h(btl);  // Bhat (fp16)
                 float4* kh = reinterpret_cast<float4*>(F0 + (t0 + it) * 64 + 8 * j);
-                kh[0] = make_float4(khat[0], khat[1], khat[2], khat[3]);
-                kh[1] = make_float4(khat[4], khat[5], khat[6], khat[7]);
+                kh[0] = make_float4(kt[0], kt[1], kt[2], kt[3]);
+                kh[1] = make_float4(kt[4], kt[5], kt[6], kt[7]);
             }
             fence_proxy_async();
             tc_fence_before();
@@ -431,10 +451,17 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.B + 32 * kk, 16, 1024),
                               smem_desc(sbase + L.R + 32 * kk, 16, 1024), id2, kk > 0);
+                // The low part of k~ into the A_rk and A_ak columns (A_ak feeds Z and the
+                // write term P_N, where bf16 rounding of k~ would dominate the state error).
+                constexpr uint32_t id3 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_D1, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
+                              smem_desc(sbase + L.ARBT + 32 * kk, 16, 1024), id3, 1u);
                 umma_commit(bar_mma);
             }
-            // While it runs: Abar = a~ e^c and Rbar = r~ e^c (tiles the Gram does not read,
-            // first read after epilogue 1's barrier).
+            // While it runs: Abar = a~ e^{g_L} (fp16) and Rbar = r~ e^{g_L} (tiles the Gram
+            // does not read, first read after epilogue 1's barrier).
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const uint32_t off = it ? offb : offa;
@@ -444,7 +471,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     abar[e] = ats[it][e] * ec[e];
                     rbar[e] = rts[it][e] * ec[e];
                 }
-                *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8(abar);
+                *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8h(abar);
                 *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8(rbar);
             }
         }
@@ -488,7 +515,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                             float x[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) x[e] = (s_ <= 8 * c + e) ? v[8 * c + e] : 0.f;
-                            *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8(x);
+                            *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8h(x);
                         }
                     }
                 } else {
@@ -499,7 +526,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                             float x[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
-                            *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8(x);
+                            *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8h(x);
                         }
                     } else {  // A_ab[t][s], kept for s < t -> fp32 row t
                         float* aab = reinterpret_cast<float*>(smem + L.R);
@@ -560,9 +587,12 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     x[t] = (t == c) ? 1.f : acc0 + acc1;
                 }
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    *reinterpret_cast<__nv_bfloat16*>(Tb + b * 768 + t * 48 + 2 * c) =
-                        __float2bfloat16_rn(x[t]);
+#pragma unroll
+                for (int t = 0; t < 16; t += 2) {  // fp16, column c: rows t and t + 1
+                    const uint32_t hp = pack2h(x[t], x[t + 1]);
+                    *reinterpret_cast<uint16_t*>(Tb + b * 768 + t * 48 + 2 * c) = (uint16_t)(hp & 0xFFFFu);
+                    *reinterpret_cast<uint16_t*>(Tb + b * 768 + (t + 1) * 48 + 2 * c) = (uint16_t)(hp >> 16);
+                }
             }
             __syncthreads();
             const int g = lane >> 2, q = lane & 3;
@@ -591,15 +621,15 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int nt = 0; nt < 2; ++nt) {
                     // B = A_im: k = row 16i + (2q, 2q+1 | 2q+8, 2q+9), n = column 16m + 8nt + g
                     const int r0 = 16 * i + 2 * q, cn = 16 * m + 8 * nt + g;
-                    const uint32_t b0 = pack2(A[fidx(r0, cn)], A[fidx(r0 + 1, cn)]);
-                    const uint32_t b1 = pack2(A[fidx(r0 + 8, cn)], A[fidx(r0 + 9, cn)]);
-                    mma_bf16_16816(z[nt], af[0], af[1], af[2], af[3], b0, b1);
+                    const uint32_t b0 = pack2h(A[fidx(r0, cn)], A[fidx(r0 + 1, cn)]);
+                    const uint32_t b1 = pack2h(A[fidx(r0 + 8, cn)], A[fidx(r0 + 9, cn)]);
+                    mma_f16_16816(z[nt], af[0], af[1], af[2], af[3], b0, b1);
                 }
                 uint8_t* dst = Tab + warp * 768;  // blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    *reinterpret_cast<uint32_t*>(dst + g * 48 + 2 * (8 * nt + 2 * q)) = pack2(z[nt][0], z[nt][1]);
-                    *reinterpret_cast<uint32_t*>(dst + (g + 8) * 48 + 2 * (8 * nt + 2 * q)) = pack2(z[nt][2], z[nt][3]);
+                    *reinterpret_cast<uint32_t*>(dst + g * 48 + 2 * (8 * nt + 2 * q)) = pack2h(z[nt][0], z[nt][1]);
+                    *reinterpret_cast<uint32_t*>(dst + (g + 8) * 48 + 2 * (8 * nt + 2 * q)) = pack2h(z[nt][2], z[nt][3]);
                 }
             }
             // (b) every warp, its 16 columns: Y_i = T_ii RHS_i for the four block rows.
@@ -613,8 +643,8 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 uint32_t af[4], bf[4];
                 a_frag(Tb + i * 768, af);
                 ldsm_x4_t(b_addr(16 * i), bf[0], bf[1], bf[2], bf[3]);
-                mma_bf16_16816(y[i][0], af[0], af[1], af[2], af[3], bf[0], bf[1]);
-                mma_bf16_16816(y[i][1], af[0], af[1], af[2], af[3], bf[2], bf[3]);
+                mma_f16_16816(y[i][0], af[0], af[1], af[2], af[3], bf[0], bf[1]);
+                mma_f16_16816(y[i][1], af[0], af[1], af[2], af[3], bf[2], bf[3]);
             }
             __syncthreads();  // T_ii A_im visible; every warp has read its right-hand side
             // (c) X_i = Y_i + sum_{m<i} (T_ii A_im) X_m, written in place over the right-hand
@@ -628,14 +658,14 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     const int blk = (i == 1) ? 0 : (i == 2 ? 1 + m : 3 + m);
                     uint32_t af[4];
                     a_frag(Tab + blk * 768, af);
-                    mma_bf16_16816(y[i][0], af[0], af[1], af[2], af[3], xb[m][0], xb[m][1]);
-                    mma_bf16_16816(y[i][1], af[0], af[1], af[2], af[3], xb[m][2], xb[m][3]);
+                    mma_f16_16816(y[i][0], af[0], af[1], af[2], af[3], xb[m][0], xb[m][1]);
+                    mma_f16_16816(y[i][1], af[0], af[1], af[2], af[3], xb[m][2], xb[m][3]);
                 }
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int col = 8 * (nb + nt) + 2 * q;
-                    const uint32_t top = pack2(y[i][nt][0], y[i][nt][1]);
-                    const uint32_t bot = pack2(y[i][nt][2], y[i][nt][3]);
+                    const uint32_t top = pack2h(y[i][nt][0], y[i][nt][1]);
+                    const uint32_t bot = pack2h(y[i][nt][2], y[i][nt][3]);
                     *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g, col)) = top;
                     *reinterpret_cast<uint32_t*>(xt + swe(16 * i + g + 8, col)) = bot;
                     if (i < 3) {
@@ -652,7 +682,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         // ---- 7. MMA-3: [Bhat^T; A_rb] [W | Z]  (128 x 128 x 64) ----------------------------
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 128, true, true);
+            constexpr uint32_t id = idesc_f16(128, 128, true, true);  // fp16 operands
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 umma_bf16(tmem + TM_D1, smem_desc(sbase + L.W + 2048 * kk, L.ARBT - L.W, 1024),

@@ -1,5 +1,8 @@
 """Parity at the full workload sizes, in the launch configuration the benchmark
-times, on sampled (sequence, head) units that the oracle computes one by one.
+times.  The forward workloads are compared on every (sequence, head) unit with one
+oracle call over the whole problem (a few seconds on the host's cores), so the
+relative errors use the same denominators as the tolerances' definition; the decode
+workload on sampled states.
 
 Workloads: B=8,T=4096,H=64 bf16 (seed 1); B=16,T=4096,H=32 bf16 with a padding
 mask (seed 2); 64 packed sequences of log-uniform length in [16, 8192], H=32
@@ -12,7 +15,7 @@ import torch
 
 import oracle
 from linear_attention_rnn_wkv7_b200 import synth, wkv7_fwd, wkv7_step
-from parity_util import check, oracle_units, rel_err, BF16_O_REL, BF16_S_REL
+from parity_util import check, rel_err, BF16_O_REL, BF16_S_REL
 
 pytestmark = pytest.mark.gpu
 
@@ -35,16 +38,20 @@ def _inputs(name):
 
 
 def _fwd_full(cuda_device, name, algo):
-    p = synth.WORKLOADS[name]
     x, mask = _inputs(name)
     xd = {k: v.to(cuda_device) for k, v in x.items()}
     o, s = wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
                     mask=None if mask is None else mask.to(cuda_device), algo=algo)
-    units = _sample_units(p["B"], p["H"], 6, p["seed"])
-    o_ref, s_ref = oracle_units(x, units, mask)
-    og = torch.stack([o[bb, :, h] for bb, h in units])
-    sg = torch.stack([s[bb, h] for bb, h in units])
-    return check(og, sg, o_ref, s_ref, torch.bfloat16, f"{name} {algo}")
+    o_ref, s_ref = _oracle_full(name)
+    return check(o, s, o_ref, s_ref, torch.bfloat16, f"{name} {algo}")
+
+
+@functools.lru_cache(maxsize=1)
+def _oracle_full(name):
+    x, mask = _inputs(name)
+    o_ref, s_ref, _ = oracle.fwd(x["r"], x["w"], x["k"], x["v"], x["a"], x["b"], s0=x["s0"],
+                                 mask=mask)
+    return o_ref, s_ref
 
 
 @pytest.mark.parametrize("algo", ["auto", "recurrent"])
@@ -65,13 +72,9 @@ def test_fwd_varlen_64seq_h32(cuda_device):
     xd = {k: v.to(cuda_device) for k, v in x.items()}
     o, s = wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
                     cu_seqlens=xd["cu_seqlens"])
-    cu = x["cu_seqlens"].tolist()
-    order = np.argsort(lengths.numpy())
-    for n in {int(order[0]), int(order[-1]), int(order[len(order) // 2])}:  # short, long, median
-        lo, hi = cu[n], cu[n + 1]
-        part = {k: x[k][:, lo:hi] for k in "rwkvab"}
-        o_ref, s_ref, _ = oracle.fwd(*(part[k] for k in "rwkvab"), s0=x["s0"][n:n + 1])
-        check(o[:, lo:hi], s[n:n + 1], o_ref, s_ref, torch.bfloat16, f"varlen seq {n}")
+    o_ref, s_ref, _ = oracle.fwd(x["r"], x["w"], x["k"], x["v"], x["a"], x["b"], s0=x["s0"],
+                                 cu_seqlens=x["cu_seqlens"])
+    check(o, s, o_ref, s_ref, torch.bfloat16, "varlen 64 sequences")
 
 
 def test_step_b1024_h32(cuda_device):
