@@ -17,13 +17,17 @@
 // Only the last product depends on S0.  One chunk costs three tcgen05 MMA groups
 // (the Gram matrix, the Bhat/A_rb products with [W | Z], and the final product
 // with [S0; V]) with fp32 accumulators in tensor memory.  [W | Z] = T [Abar | A_ak]
-// comes from a block forward substitution on warp-level bf16 MMAs (each warp owns
-// 16 of its 128 columns), after the 16x16 diagonal blocks of T by fp32 forward
+// comes from a block forward substitution on warp-level MMAs (each warp owns 16 of
+// its 128 columns), after the 16x16 diagonal blocks of T by fp32 forward
 // substitution.  CUDA cores do the prefix sums and exps and the tensor-memory ->
 // shared-memory epilogues that re-layout each result as the next product's operand.
-// The write term Khat^T + Bhat^T Z enters the final MMA as a hi/lo pair of bf16
-// matrices (about 16 significant bits), which keeps the fp32 final state within
-// 1e-3 of the fp64 recurrence; all other tensor-core operands are bf16.
+// Precision: the Gram operands need bf16's exponent range (E_t spans e^{+-40}), and
+// the low part of k~ (k~ - bf16(k~)) is added into A_rk and A_ak by a fourth Gram
+// group, since A_ak feeds the write term Khat^T + Bhat^T Z where rounding of k~ would
+// dominate the state error.  Every later operand (the substitution, MMA-3, the final
+// product, the bf16 copy of S0 and V) stays near 1 in magnitude and is fp16, with
+// three more significant bits than bf16; that keeps the fp32 final state well within
+// 1e-3 of the fp64 recurrence.
 //
 // A masked or out-of-range token is folded into the loads as w = 0 and zero a, k, b
 // scales: its transition is then the identity and it writes nothing, and its output
@@ -473,6 +477,9 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 }
                 *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8h(abar);
                 *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8(rbar);
+                float vf[8];  // V to fp16 in place (the final MMA's B operand)
+                unpack8(*reinterpret_cast<const uint4*>(smem + L.V + off), vf);
+                *reinterpret_cast<uint4*>(smem + L.V + off) = pack8h(vf);
             }
         }
 
@@ -715,20 +722,14 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 load16(3);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + L.R + sw(k, 4 * wh + c)) = pack8(v + 8 * c);
+                    *reinterpret_cast<uint4*>(smem + L.R + sw(k, 4 * wh + c)) = pack8h(v + 8 * c);
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {  // P_N = Bhat^T Z + Khat^T, split into bf16 hi + lo
-                    float hi[8], lo[8];
+                for (int c = 0; c < 4; ++c) {  // P_N = Bhat^T Z + Khat^T
+                    float pn[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int s_ = 8 * (4 * wh + c) + e;
-                        const float pn = v[32 + 8 * c + e] + F0[s_ * 64 + k];
-                        hi[e] = __bfloat162float(__float2bfloat16_rn(pn));
-                        lo[e] = pn - hi[e];
-                    }
-                    *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, 4 * wh + c)) = pack8(hi);
-                    *reinterpret_cast<uint4*>(smem + L.K + sw(k, 4 * wh + c)) = pack8(lo);
+                    for (int e = 0; e < 8; ++e) pn[e] = v[32 + 8 * c + e] + F0[(8 * (4 * wh + c) + e) * 64 + k];
+                    *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, 4 * wh + c)) = pack8h(pn);
                 }
             } else {
                 const int tp = m_row - 64;
@@ -739,8 +740,8 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
                 };
-                // Q = A_rb W + Rbar (wh 0) or P_O = A_rb Z + A_rk (wh 1); P_O's lo block is
-                // zero.  The second 32 columns load while the first are stored.
+                // Q = A_rb W + Rbar (wh 0) or P_O = A_rb Z + A_rk (wh 1).  The second 32
+                // columns load while the first are stored.
                 const uint32_t src = wh ? L.ARK : L.RBAR, dst = wh ? L.ABAR : L.R;
                 auto emit = [&](int h) {
 #pragma unroll
@@ -749,7 +750,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                         unpack8(*reinterpret_cast<const uint4*>(smem + src + sw(tp, c)), x);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) x[e] += v[8 * c + e];
-                        *reinterpret_cast<uint4*>(smem + dst + sw(m_row, c)) = pack8(x);
+                        *reinterpret_cast<uint4*>(smem + dst + sw(m_row, c)) = pack8h(x);
                     }
                 };
                 load16(0);
@@ -760,11 +761,6 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 emit(0);
                 tmem_ld_wait();
                 emit(1);
-                if (wh) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(smem + L.K + sw(m_row, c)) = make_uint4(0, 0, 0, 0);
-                }
             }
             // The final MMA accumulates onto its tensor-memory columns: rows 0..63 hold
             // the fp32 state, scaled here by e^{g_L}; rows 64..127 (outputs) start at 0.
@@ -791,13 +787,13 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         // are dead now; the copy overlaps this chunk's final MMA and epilogue.
         if (has_next && warp == 1) issue_loads(cx, c0 + 64, par ^ 1);
 
-        // ---- 9. final MMA: [S upd; O] = A_fin [S0; V; V]  (128 x 64 x 192) --------------
+        // ---- 9. final MMA: [S upd; O] = A_fin [S0; V]  (128 x 64 x 128, fp16) ------------
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+            constexpr uint32_t id = idesc_f16(128, 64, false, true);
 #pragma unroll
-            for (int blk = 0; blk < 3; ++blk) {
-                const uint32_t aoff = blk == 0 ? L.R : (blk == 1 ? L.ABAR : L.K);
+            for (int blk = 0; blk < 2; ++blk) {
+                const uint32_t aoff = blk == 0 ? L.R : L.ABAR;
                 const uint32_t boff = blk == 0 ? OFF_S0 : L.V;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
@@ -817,7 +813,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             if (state_thread) {  // v = the new fp32 state row; its bf16 copy feeds the next chunk
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(v + 8 * c);
+                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8h(v + 8 * c);
             } else {
                 const int t = m_row - 64;
                 if (t < nv) {
@@ -934,7 +930,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         tmem_st_wait();
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8(sv + 8 * c);
+            *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8h(sv + 8 * c);
     }
     tc_fence_before();
 
