@@ -85,6 +85,12 @@ typedef enum {
  *
  * Returns WKV7_OK after enqueueing the kernel(s) on `stream`.
  * B, T or N may be 0 (nothing to compute; with T == 0, sT receives s0 or zeros).
+ *
+ * Range of the chunked form (WKV7_ALGO_CHUNKED, and AUTO for bf16): exact while a
+ * 64-token chunk's decay stays within e^{-80} (per-step log decay >= -1.26 on
+ * average); the state and v enter its last tensor-core product as fp16 operands,
+ * so their magnitudes must stay below 65504 (larger values saturate).  The
+ * recurrent form has neither limit.
  */
 wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
                      const void* a, const void* b, const float* s0, const uint8_t* mask,

@@ -67,6 +67,37 @@ def test_bf16_null_states(cuda_device, algo):
 
 
 @pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("decay", ["none", "strong", "mixed"])
+def test_extreme_decays(cuda_device, algo, decay):
+    """Per-step log decays at both ends of the range the chunked form is exact for:
+    w = 0 (no decay: E_t = 1, a pure delta rule), w = -1.2 (a chunk's decay spans
+    e^{-76}, near the exponent clamp of 80), and channels mixing the two."""
+    x = synth.fwd_inputs(2, 200, 2, dtype=torch.bfloat16, seed=11, s0_std=0.1)
+    w = x["w"].float()
+    if decay == "none":
+        w = torch.zeros_like(w)
+    elif decay == "strong":
+        w = torch.full_like(w, -1.2)
+    else:
+        w = torch.where(torch.arange(64) % 2 == 0, torch.zeros_like(w), torch.full_like(w, -1.2))
+    x["w"] = w.to(torch.bfloat16).contiguous()
+    o_ref, s_ref = ref(x)
+    o, s = run(to_dev(x, cuda_device), algo)
+    check(o, s, o_ref, s_ref, torch.bfloat16, f"{algo} decay={decay}")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_larger_magnitudes(cuda_device, algo):
+    """State entries around 10 and values around 100 (the chunked form carries S0 and
+    V as fp16 operands, exact in range up to 65504)."""
+    x = synth.fwd_inputs(2, 200, 2, dtype=torch.bfloat16, seed=13, s0_std=10.0)
+    x["v"] = (x["v"].float() * 100.0).to(torch.bfloat16).contiguous()
+    o_ref, s_ref = ref(x)
+    o, s = run(to_dev(x, cuda_device), algo)
+    check(o, s, o_ref, s_ref, torch.bfloat16, f"{algo} larger magnitudes")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_mask(cuda_device, algo, dtype):
     if algo == "chunked" and dtype == torch.float32:
