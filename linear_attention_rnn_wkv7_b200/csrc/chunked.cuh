@@ -107,7 +107,8 @@ __device__ __forceinline__ LayR lay_of(int par) {
     return par ? lay_const<1>() : lay_const<0>();
 }
 // Aliases inside one chunk (lifetimes do not overlap):
-//   fp32 A_ab [t][s]     R (2 tiles)   epilogue 1 -> W|Z substitution
+//   A_ab [t][s]          R: fp16 blocks left of the diagonal; A: fp32 diagonal
+//                        blocks (epilogue 1 -> W|Z substitution)
 //   fp32 T_ii + scratch  K (2 tiles)   W|Z substitution
 //   [M'; Rbar + A_rb W]  R (2 tiles)   epilogue 3 -> final MMA A, K block 0
 //   [P_N hi; A_rk+A_rb Z] ABAR (2)     epilogue 3 -> final MMA A, K block 1
@@ -130,11 +131,11 @@ __device__ __forceinline__ uint32_t swe(uint32_t row, uint32_t col) {
     return sw(row, col >> 3) + ((col & 7u) << 1);
 }
 
-// Float index of (row, col) in a 64x64 fp32 tile whose 16-byte chunks are permuted
-// by the low three bits of the row, so that eight consecutive rows written or
-// read at the same column hit different banks.
-__device__ __forceinline__ int fidx(int row, int col) {
-    return row * 64 + ((((col >> 2) ^ (row & 7)) << 2) | (col & 3));
+// Float index of element (r, c) of diagonal 16x16 block bb of A_ab, kept in fp32
+// (blocks 260 floats apart and 16-byte chunks permuted by r % 4, so the rows a warp
+// writes together and the blocks it reads together fall in different banks).
+__device__ __forceinline__ int didx(int bb, int r, int c) {
+    return bb * 260 + r * 16 + ((((c >> 2) ^ (r & 3)) << 2) | (c & 3));
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -535,16 +536,29 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                             for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
                             *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8h(x);
                         }
-                    } else {  // A_ab[t][s], kept for s < t -> fp32 row t
-                        float* aab = reinterpret_cast<float*>(smem + L.R);
+                    } else {  // A_ab[t][s], s < t: the blocks left of row t's diagonal block
+                        // (all kept) as fp16 for the T_ii A_im products, the diagonal block
+                        // (masked) in fp32 for the T_ii substitution.
+                        const int bt = t >> 4;
 #pragma unroll
-                        for (int c4 = 8 * h; c4 < 8 * h + 8; ++c4) {
-                            float4 x;
-                            x.x = (4 * c4 + 0 < t) ? v[4 * c4 + 0] : 0.f;
-                            x.y = (4 * c4 + 1 < t) ? v[4 * c4 + 1] : 0.f;
-                            x.z = (4 * c4 + 2 < t) ? v[4 * c4 + 2] : 0.f;
-                            x.w = (4 * c4 + 3 < t) ? v[4 * c4 + 3] : 0.f;
-                            *reinterpret_cast<float4*>(aab + fidx(t, 4 * c4)) = x;
+                        for (int c = 4 * h; c < 4 * h + 4; ++c)
+                            if (c < 2 * bt)
+                                *reinterpret_cast<uint4*>(smem + L.R + sw(t, c)) = pack8h(v + 8 * c);
+                        float* dg = reinterpret_cast<float*>(smem + L.A);
+#pragma unroll
+                        for (int b2 = 2 * h; b2 < 2 * h + 2; ++b2) {
+                            if (bt == b2) {
+#pragma unroll
+                                for (int c4 = 0; c4 < 4; ++c4) {
+                                    const int s0_ = 16 * b2 + 4 * c4;
+                                    float4 x;
+                                    x.x = (s0_ + 0 < t) ? v[s0_ + 0] : 0.f;
+                                    x.y = (s0_ + 1 < t) ? v[s0_ + 1] : 0.f;
+                                    x.z = (s0_ + 2 < t) ? v[s0_ + 2] : 0.f;
+                                    x.w = (s0_ + 3 < t) ? v[s0_ + 3] : 0.f;
+                                    *reinterpret_cast<float4*>(dg + didx(b2, t & 15, 4 * c4)) = x;
+                                }
+                            }
                         }
                     }
                 }
@@ -570,12 +584,12 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         //         place over the right-hand side (bf16), where MMA-3 reads it as its
         //         MN-major B operand. ------------------------------------------------
         {
-            const float* A = reinterpret_cast<const float*>(smem + L.R);  // A_ab [t][s]
+            const float* Dg = reinterpret_cast<const float*>(smem + L.A);  // diagonal blocks of A_ab
             // bf16 16x16 blocks with rows of 48 bytes: T_ii (4), then T_ii A_im (6).
             uint8_t* Tb = smem + L.K;
             uint8_t* Tab = Tb + 4 * 768;
             if (tid < 64) {  // diagonal block b, column c
-                const int b = tid >> 4, c = tid & 15, base = 16 * b;
+                const int b = tid >> 4, c = tid & 15;
                 float x[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) x[i] = 0.f;
@@ -584,8 +598,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
                     for (int s4 = 0; s4 < t; s4 += 4) {
-                        const float4 a4 =
-                            *reinterpret_cast<const float4*>(A + fidx(base + t, base + s4));
+                        const float4 a4 = *reinterpret_cast<const float4*>(Dg + didx(b, t, s4));
                         acc0 = fmaf(a4.x, x[s4 + 0], acc0);
                         acc1 = fmaf(a4.y, x[s4 + 1], acc1);
                         acc0 = fmaf(a4.z, x[s4 + 2], acc0);
@@ -624,14 +637,12 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 uint32_t af[4];
                 a_frag(Tb + i * 768, af);
                 float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    // B = A_im: k = row 16i + (2q, 2q+1 | 2q+8, 2q+9), n = column 16m + 8nt + g
-                    const int r0 = 16 * i + 2 * q, cn = 16 * m + 8 * nt + g;
-                    const uint32_t b0 = pack2h(A[fidx(r0, cn)], A[fidx(r0 + 1, cn)]);
-                    const uint32_t b1 = pack2h(A[fidx(r0 + 8, cn)], A[fidx(r0 + 9, cn)]);
-                    mma_f16_16816(z[nt], af[0], af[1], af[2], af[3], b0, b1);
-                }
+                uint32_t bfa[4];  // B = A_im (fp16 rows 16i.., columns 16m..), transposed fragments
+                ldsm_x4_t(smem_u32(smem + L.R) +
+                              sw(16 * i + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * m + (lane >> 4)),
+                          bfa[0], bfa[1], bfa[2], bfa[3]);
+                mma_f16_16816(z[0], af[0], af[1], af[2], af[3], bfa[0], bfa[1]);
+                mma_f16_16816(z[1], af[0], af[1], af[2], af[3], bfa[2], bfa[3]);
                 uint8_t* dst = Tab + warp * 768;  // blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
