@@ -114,7 +114,7 @@ __device__ __forceinline__ LayR lay_of(int par) {
 //   [P_N hi; A_rk+A_rb Z] ABAR (2)     epilogue 3 -> final MMA A, K block 1
 //   [P_N lo; 0]          K (2 tiles)   epilogue 3 -> final MMA A, K block 2
 // Prologue scratch inside the A_rk tile (free until epilogue 1), in floats.
-constexpr int SCR_TOT = 0, SCR_C = 512;  // floats
+constexpr int SCR_TOT = 0, SCR_C = 512, SCR_PRE = 576;  // floats (SCR_PRE: 8 x 64)
 // Tensor-memory columns (fp32 accumulators, 128 lanes).
 constexpr uint32_t TM_D1 = 0;    // Gram, later MMA-3 (128 cols)
 constexpr uint32_t TM_D1B = 128; // A_rb^T = b~ r~^T (64 cols)
@@ -328,20 +328,28 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         // ---- 2. prefix sums of w (mask folded) and every scaled operand, in one pass.
         //         Thread (q, j) owns tokens 2q, 2q+1 and channels 8j..8j+7: a shuffle
         //         scan over the warp's four token pairs, warp totals exchanged through
-        //         shared memory, per-channel constants from warp 0, then E_t and the
-        //         operands, written in place. ------------------------------------------
+        //         shared memory, each warp's exclusive prefix and the per-channel
+        //         constants from warp 0, then E_t and the operands, written in
+        //         place. ----------------------------------------------------------------
         {
             const int j = tid & 7, t0 = 2 * (tid >> 3);
             const bool va = t0 < nv && (!mask || mask[row0 + c0 + t0] != 0);
             const bool vb = t0 + 1 < nv && (!mask || mask[row0 + c0 + t0 + 1] != 0);
             const uint32_t offa = sw(t0, j), offb = sw(t0 + 1, j);
             float wa[8], wb[8], incl[8];
-            unpack8(*reinterpret_cast<const uint4*>(smem + L.W + offa), wa);
-            unpack8(*reinterpret_cast<const uint4*>(smem + L.W + offb), wb);
+            {  // a masked token's w is zero (cleared on the packed words)
+                const uint32_t ma = va ? 0xFFFFFFFFu : 0u, mb = vb ? 0xFFFFFFFFu : 0u;
+                uint4 qa = *reinterpret_cast<const uint4*>(smem + L.W + offa);
+                uint4 qb = *reinterpret_cast<const uint4*>(smem + L.W + offb);
+                qa.x &= ma; qa.y &= ma; qa.z &= ma; qa.w &= ma;
+                qb.x &= mb; qb.y &= mb; qb.z &= mb; qb.w &= mb;
+                unpack8(qa, wa);
+                unpack8(qb, wb);
+            }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {  // log decays in log2 units from here on
-                wa[e] = va ? wa[e] * kLog2e : 0.f;
-                wb[e] = vb ? wb[e] * kLog2e : 0.f;
+                wa[e] *= kLog2e;
+                wb[e] *= kLog2e;
                 incl[e] = wa[e] + wb[e];
             }
 #pragma unroll
@@ -360,41 +368,35 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     make_float4(incl[4], incl[5], incl[6], incl[7]);
             }
             __syncthreads();
-            if (warp == 0) {  // per channel: the reference c = g_L and e^{g_L}
+            if (warp == 0) {  // per channel: exclusive prefixes over the warps, c = g_L, e^{g_L}
                 const int ch = 2 * lane;
                 float2 gL = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int w2 = 0; w2 < 8; ++w2) {
                     const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
+                    reinterpret_cast<float2*>(scratch + SCR_PRE + w2 * 64)[lane] = gL;
                     gL.x += x.x; gL.y += x.y;
                 }
                 reinterpret_cast<float2*>(scratch + SCR_C)[lane] = gL;
                 reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(ex2(gL.x), ex2(gL.y));
             }
-            float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
-#pragma unroll
-            for (int e = 0; e < 8; ++e) ga[e] = incl[e] - wb[e];
-#pragma unroll
-            for (int w2 = 0; w2 < 7; ++w2) {
-                if (w2 < warp) {
-                    const float4 x0 = *reinterpret_cast<const float4*>(wt + w2 * 64 + 8 * j);
-                    const float4 x1 = *reinterpret_cast<const float4*>(wt + w2 * 64 + 8 * j + 4);
-                    ga[0] += x0.x; ga[1] += x0.y; ga[2] += x0.z; ga[3] += x0.w;
-                    ga[4] += x1.x; ga[5] += x1.y; ga[6] += x1.z; ga[7] += x1.w;
-                }
-            }
             __syncthreads();  // per-channel constants ready
+            float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
+            {
+                const float4 x0 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j);
+                const float4 x1 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j + 4);
+                const float pre[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ga[e] = pre[e] + (incl[e] - wb[e]);
+            }
             float cc[8], ec[8];  // c = g_L (log2 units) and e^{g_L}
             *reinterpret_cast<float4*>(cc) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[0];
             *reinterpret_cast<float4*>(cc + 4) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[1];
             *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[0];
             *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[1];
-            float Ep[8];  // E at token t0 - 1
+            float Ep[8];  // E at token t0 - 1 (g_{t0-1} = g_{t0} - w_{t0})
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float prev = __shfl_up_sync(0xffffffffu, ga[e] + wb[e], 8);  // g_{t0-1}
-                Ep[e] = ex2(clamp2(((lane >= 8) ? prev : ga[e] - wa[e]) - cc[e]));
-            }
+            for (int e = 0; e < 8; ++e) Ep[e] = ex2(clamp2(ga[e] - wa[e] - cc[e]));
             float rts[2][8], ats[2][8];  // fp32 r~ and a~, kept for Rbar and Abar
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
