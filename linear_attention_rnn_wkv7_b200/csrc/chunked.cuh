@@ -165,9 +165,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float* v) {
         v[2 * i + 1] = f.y;
     }
 }
-__device__ __forceinline__ float bf16_at(const uint8_t* tile, uint32_t row, uint32_t col) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + swe(row, col)));
-}
 // 2^x by the hardware approximation (relative error about 2^-22, subnormal results
 // flushed to zero); the prologue keeps
 // log decays in log2 units so that every exponential is one such instruction.
@@ -204,18 +201,9 @@ __device__ __forceinline__ void tmem_row_st32(uint32_t tmem, int wq, uint32_t co
     }
 }
 
-// Warp-level D += A * B, m16n8k16, bf16 operands, fp32 accumulate.  Fragment
+// Warp-level D += A * B, m16n8k16, fp16 operands, fp32 accumulate.  Fragment
 // ownership (g = lane / 4, q = lane % 4): A (g|g+8, 2q..2q+1 | 2q+8..2q+9),
 // B (k = 2q..2q+1 | 2q+8..2q+9, n = g), C/D (g|g+8, 2q|2q+1).
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-// The same with fp16 operands.
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                               uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -246,23 +234,6 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     return y;
 }
 
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
-// Warp-level D += A * B, m16n8k8, tf32 operands, fp32 accumulate.  Fragment
-// ownership (g = lane / 4, q = lane % 4): A (g|g+8, q|q+4), B (k = q|q+4, n = g),
-// C/D (g|g+8, 2q|2q+1).
-__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int* abort_flag) {
     if (!sm100::mbar_wait(bar, parity)) {
