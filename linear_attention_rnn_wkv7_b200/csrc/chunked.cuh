@@ -699,14 +699,28 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
                 };
+                float sv[32];  // this thread's fp32 state row, loaded with M'
                 load16(0);
                 load16(1);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float tmp[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_DF + 32 * wh + 16 * i, tmp);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sv[16 * i + j] = tmp[j];
+                }
                 tmem_ld_wait();
-                load16(2);  // P_N columns load while M' is stored
+                load16(2);  // P_N columns load while M' is stored and the state is scaled
                 load16(3);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     *reinterpret_cast<uint4*>(smem + L.R + sw(k, 4 * wh + c)) = pack8h(v + 8 * c);
+                {  // the final MMA accumulates onto the state row scaled by e^{g_L}
+                    const float gamma = gamma_s[m_row];
+#pragma unroll
+                    for (int j2 = 0; j2 < 32; ++j2) sv[j2] *= gamma;
+                    tmem_row_st32(tmem + TM_DF, wq, 32 * wh, sv);
+                }
                 tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {  // P_N = Bhat^T Z + Khat^T
@@ -715,6 +729,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     for (int e = 0; e < 8; ++e) pn[e] = v[32 + 8 * c + e] + F0[(8 * (4 * wh + c) + e) * 64 + k];
                     *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, 4 * wh + c)) = pack8h(pn);
                 }
+                tmem_st_wait();
             } else {
                 const int tp = m_row - 64;
                 float v[64];
@@ -747,18 +762,11 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 emit(1);
             }
             // The final MMA accumulates onto its tensor-memory columns: rows 0..63 hold
-            // the fp32 state, scaled here by e^{g_L}; rows 64..127 (outputs) start at 0.
-            {
+            // the scaled fp32 state (above); rows 64..127 (outputs) start at 0.
+            if (!state_thread) {
                 float sv[32];
-                if (state_thread) {
-                    const float gamma = gamma_s[m_row];
-                    tmem_row<2>(tmem + TM_DF, wq, 32 * wh, sv);
 #pragma unroll
-                    for (int j2 = 0; j2 < 32; ++j2) sv[j2] *= gamma;
-                } else {
-#pragma unroll
-                    for (int j2 = 0; j2 < 32; ++j2) sv[j2] = 0.f;
-                }
+                for (int j2 = 0; j2 < 32; ++j2) sv[j2] = 0.f;
                 tmem_row_st32(tmem + TM_DF, wq, 32 * wh, sv);
                 tmem_st_wait();
             }
