@@ -715,6 +715,10 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     *reinterpret_cast<uint4*>(smem + L.R + sw(k, 4 * wh + c)) = pack8h(v + 8 * c);
+                // The final MMA's S0 operand: the fp16 copy of the state this chunk starts from.
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(k, 4 * wh + c)) = pack8h(sv + 8 * c);
                 {  // the final MMA accumulates onto the state row scaled by e^{g_L}
                     const float gamma = gamma_s[m_row];
 #pragma unroll
@@ -798,28 +802,22 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 10. epilogue 4: state carry (fp32) and the chunk's outputs ---------------------
-        {
+        // ---- 10. epilogue 4: the chunk's outputs (rows 64..127 of the final product); the
+        //          new fp32 state stays in tensor memory (its fp16 copy is written by the
+        //          next chunk's epilogue 3) ----------------------------------------------
+        if (!state_thread) {
             float v[32];
             tmem_row<2>(tmem + TM_DF, wq, 32 * wh, v);
-            if (state_thread) {  // v = the new fp32 state row; its bf16 copy feeds the next chunk
+            const int t = m_row - 64;
+            if (t < nv) {
+                uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(row0 + c0 + t) * H + h) * 64 + 32 * wh);
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8h(v + 8 * c);
-            } else {
-                const int t = m_row - 64;
-                if (t < nv) {
-                    uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(row0 + c0 + t) * H + h) * 64 + 32 * wh);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) dst[c] = pack8(v + 8 * c);
-                }
+                for (int c = 0; c < 4; ++c) dst[c] = pack8(v + 8 * c);
             }
-            // No barrier: nothing the next chunk does before its own first barrier
-            // touches what this epilogue reads or writes (S0 tile, o, the final
-            // product's tensor-memory columns).
-            fence_proxy_async();
-            tc_fence_before();
         }
+        // No barrier: nothing the next chunk does before its own first barrier touches
+        // what this epilogue reads or writes (o, the final product's output rows).
+        tc_fence_before();
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -900,7 +898,8 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
 
     // The fp32 state lives in tensor memory, rows 0..63 of the final product's
     // columns: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
-    // [32*wh, 32*wh + 32).  A bf16 copy in shared memory feeds the final MMA.
+    // [32*wh, 32*wh + 32).  Each chunk's epilogue 3 writes the fp16 copy in shared
+    // memory that feeds its final MMA.
     const int m_row = cx.m_row;
     const size_t state_off = ((size_t)n * H + h) * 4096;
     if (cx.state_thread) {
@@ -920,9 +919,6 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         }
         tmem_row_st32(cx.tmem + TM_DF, wq, 32 * wh, sv);
         tmem_st_wait();
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(m_row, 4 * wh + c)) = pack8h(sv + 8 * c);
     }
     tc_fence_before();
 
