@@ -685,9 +685,8 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         tc_fence_after();
 
         // ---- 8. epilogue 3: assemble the final A operand.  Rows k (lanes 0..63): M'
-        //         and the hi/lo split of P_N; warps 0/1 take columns 0..31 of both,
-        //         warps 4/5 columns 32..63.  Rows t (lanes 64..127): Q (warps 2/3) and
-        //         P_O (warps 6/7). ---------------------------------------------------
+        //         and P_N; warps 0/1 take columns 0..31 of both, warps 4/5 columns
+        //         32..63.  Rows t (lanes 64..127): Q (warps 2/3) and P_O (warps 6/7). --
         {
             if (wq < 2) {
                 const int k = m_row;
