@@ -765,14 +765,8 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 emit(1);
             }
             // The final MMA accumulates onto its tensor-memory columns: rows 0..63 hold
-            // the scaled fp32 state (above); rows 64..127 (outputs) start at 0.
-            if (!state_thread) {
-                float sv[32];
-#pragma unroll
-                for (int j2 = 0; j2 < 32; ++j2) sv[j2] = 0.f;
-                tmem_row_st32(tmem + TM_DF, wq, 32 * wh, sv);
-                tmem_st_wait();
-            }
+            // the scaled fp32 state (above); rows 64..127 (outputs) were cleared by the
+            // previous chunk's epilogue 4 (or at the start).
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
@@ -807,6 +801,12 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         if (!state_thread) {
             float v[32];
             tmem_row<2>(tmem + TM_DF, wq, 32 * wh, v);
+            {  // cleared for the next chunk's final MMA, which accumulates onto them
+                float z[32];
+#pragma unroll
+                for (int j2 = 0; j2 < 32; ++j2) z[j2] = 0.f;
+                tmem_row_st32(tmem + TM_DF, wq, 32 * wh, z);
+            }
             const int t = m_row - 64;
             if (t < nv) {
                 uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(row0 + c0 + t) * H + h) * 64 + 32 * wh);
@@ -814,6 +814,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int c = 0; c < 4; ++c) dst[c] = pack8(v + 8 * c);
             }
         }
+        if (!state_thread) tmem_st_wait();
         // No barrier: nothing the next chunk does before its own first barrier touches
         // what this epilogue reads or writes (o, the final product's output rows).
         tc_fence_before();
@@ -917,6 +918,12 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             }
         }
         tmem_row_st32(cx.tmem + TM_DF, wq, 32 * wh, sv);
+        tmem_st_wait();
+    } else {  // output rows start at 0 (the final MMA accumulates onto them)
+        float z[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = 0.f;
+        tmem_row_st32(cx.tmem + TM_DF, wq, 32 * wh, z);
         tmem_st_wait();
     }
     tc_fence_before();
