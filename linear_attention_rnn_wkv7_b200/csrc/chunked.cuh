@@ -825,7 +825,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
-               float* sT, int T, int H, const int32_t* __restrict__ cu_seqlens) {
+               float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens) {
     extern __shared__ __align__(1024) uint8_t smem[];
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -836,7 +836,28 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         return;
     }
     const int h = blockIdx.x % H;
-    const int n = blockIdx.x / H;
+    int n = blockIdx.x / H;
+    if (cu_seqlens && N <= kThreads) {
+        // Packed sequences are taken longest first (ties by index): blocks start in
+        // index order, so the long sequences do not end up in the last wave.  Each CTA
+        // ranks the lengths itself, in a tile that is free until the first chunk.
+        int* lens = reinterpret_cast<int*>(smem + 9 * kTile);
+        int* pick = lens + kThreads;
+        if (tid < N) lens[tid] = cu_seqlens[tid + 1] - cu_seqlens[tid];
+        __syncthreads();
+        if (tid < N) {
+            const int mine = lens[tid];
+            int rank = 0;
+            for (int j = 0; j < N; ++j) {
+                const int lj = lens[j];
+                rank += (lj > mine) || (lj == mine && j < tid);
+            }
+            if (rank == n) *pick = tid;
+        }
+        __syncthreads();
+        n = *pick;
+        __syncthreads();  // the tile is reused later
+    }
     int bb = n, bos = 0, eos = T;
     if (cu_seqlens) {
         bb = 0;
@@ -1003,7 +1024,7 @@ inline cudaError_t launch_chunked(const void* r, const void* w, const void* k, c
     }
     chunked_kernel<<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], s0, mask,
-        static_cast<__nv_bfloat16*>(o), sT, T, H, cu_seqlens);
+        static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens);
     return cudaGetLastError();
 }
 
