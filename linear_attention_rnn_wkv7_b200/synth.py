@@ -12,6 +12,11 @@ Value recipe (the RWKV-7 parametrisation the workloads use):
   initial states ~ N(0, std) fp32.
 Draw order: r, k, v, z, eta, then the initial state, then the mask.  Values are
 drawn in fp32 and rounded to the requested dtype once.
+
+Gated DeltaNet inputs (``gdn_inputs``): q, k, v ~ N(0, 1) as drawn (the operator
+normalises q and k itself); g = -exp(-0.5 - softplus(z)), z ~ N(0, 1), one log
+decay per (b, t, h); beta = sigmoid(y), y ~ N(0, 1), per (b, t, h).  Draw order:
+q, k, v, z, y, then the initial state.
 """
 from __future__ import annotations
 
@@ -21,7 +26,8 @@ import torch
 import torch.nn.functional as F
 
 __all__ = ["fwd_inputs", "padding_mask", "varlen_lengths", "decode_state",
-           "decode_step_inputs", "WORKLOADS"]
+           "decode_step_inputs", "gdn_inputs", "gdn_varlen_inputs", "gdn_step_inputs",
+           "WORKLOADS"]
 
 
 def _token_vectors(g: torch.Generator, shape_k, shape_v, dtype):
@@ -53,6 +59,51 @@ def fwd_inputs(B: int, T: int, H: int, K: int = 64, V: int = 64,
     else:
         out["s0"] = (torch.randn(N, H, K, V, generator=g) * s0_std).contiguous()
     return out
+
+
+def _gdn_vectors(g: torch.Generator, shape_k, shape_v, dtype):
+    q = torch.randn(shape_k, generator=g)
+    k = torch.randn(shape_k, generator=g)
+    v = torch.randn(shape_v, generator=g)
+    z = torch.randn(shape_k[:-1], generator=g)
+    gate = -torch.exp(-0.5 - F.softplus(z))
+    beta = torch.sigmoid(torch.randn(shape_k[:-1], generator=g))
+    return {name: t.to(dtype).contiguous() for name, t in
+            (("q", q), ("k", k), ("v", v), ("g", gate), ("beta", beta))}
+
+
+def gdn_inputs(B: int, T: int, H: int, K: int = 64, V: int = 64,
+               dtype: torch.dtype = torch.bfloat16, seed: int = 0,
+               s0_std: float | None = 0.1, n_states: int | None = None):
+    """Gated DeltaNet inputs q, k [B,T,H,K], v [B,T,H,V], g, beta [B,T,H];
+    s0 [N,H,K,V] fp32 (or None)."""
+    g = torch.Generator().manual_seed(seed)
+    out = _gdn_vectors(g, (B, T, H, K), (B, T, H, V), dtype)
+    N = B if n_states is None else n_states
+    if s0_std is None:
+        out["s0"] = None
+    elif s0_std == 0.0:
+        out["s0"] = torch.zeros(N, H, K, V, dtype=torch.float32)
+    else:
+        out["s0"] = (torch.randn(N, H, K, V, generator=g) * s0_std).contiguous()
+    return out
+
+
+def gdn_varlen_inputs(lengths: torch.Tensor, H: int, K: int = 64, V: int = 64,
+                      dtype: torch.dtype = torch.bfloat16, seed: int = 0,
+                      s0_std: float | None = 0.1):
+    """Packed [1, sum(lengths), H, *] Gated DeltaNet inputs, per-sequence s0, cu_seqlens."""
+    out = gdn_inputs(1, int(lengths.sum()), H, K, V, dtype, seed, s0_std,
+                     n_states=lengths.numel())
+    out["cu_seqlens"] = cu_seqlens_of(lengths)
+    return out
+
+
+def gdn_step_inputs(B: int, H: int, K: int = 64, V: int = 64,
+                    dtype: torch.dtype = torch.bfloat16, seed: int = 6, step: int = 0):
+    """One Gated DeltaNet decode step: q, k [B,H,K], v [B,H,V], g, beta [B,H]."""
+    g = torch.Generator().manual_seed(seed * 1_000_003 + 1 + step)
+    return _gdn_vectors(g, (B, H, K), (B, H, V), dtype)
 
 
 def padding_mask(B: int, T: int, seed: int, max_suffix: int = 1024,
@@ -105,7 +156,7 @@ def decode_step_inputs(B: int, H: int, K: int = 64, V: int = 64,
     return _token_vectors(g, (B, H, K), (B, H, V), dtype)
 
 
-# The five workloads: name -> description of sizes (used by tests and bench).
+# The workloads: name -> description of sizes (used by tests and bench).
 WORKLOADS = {
     "fwd_fp32_small": dict(B=1, T=64, H=2, K=64, V=64, dtype="f32", seed=0, s0_std=0.0),
     "fwd_bf16_b8_t4096_h64": dict(B=8, T=4096, H=64, K=64, V=64, dtype="bf16", seed=1,
@@ -116,4 +167,9 @@ WORKLOADS = {
                                       dtype="bf16", seed=3, s0_std=0.1),
     "step_bf16_b1024_h32_256steps": dict(B=1024, H=32, K=64, V=64, dtype="bf16", seed=4,
                                          steps=256, s0_std=0.1),
+    # Gated DeltaNet through the same kernels (same shapes as the WKV7 workloads)
+    "gdn_fwd_bf16_b8_t4096_h64": dict(B=8, T=4096, H=64, K=64, V=64, dtype="bf16", seed=5,
+                                      s0_std=0.1),
+    "gdn_step_bf16_b1024_h32_256steps": dict(B=1024, H=32, K=64, V=64, dtype="bf16", seed=6,
+                                             steps=256, s0_std=0.1),
 }

@@ -13,6 +13,11 @@ see ``wkv7_oracle.c`` for the equations.  ``step`` is the length-one case
 (B,H,K,K)).  ``brute`` holds an independent dense-product form used only to
 pin this one on tiny inputs.
 
+``gdn_fwd`` / ``gdn_step`` are the Gated DeltaNet operator of the same README
+(sections "gdn_recurrent 使用方法" and "gdn_chunk 使用方法": q, k L2-normalised
+inside, g a log-space decay gate per (b, t, h), beta a write strength in (0, 1)
+per (b, t, h)), written in its delta-rule form in ``wkv7_oracle.c``.
+
 Every input is converted exactly to float64 (bf16 and fp32 values are exactly
 representable), so the oracle sees the very values a kernel sees.
 """
@@ -48,6 +53,10 @@ def load_library(path: str):
     lib.wkv7_oracle_fwd.restype = ctypes.c_int
     lib.wkv7_oracle_fwd.argtypes = [p, p, p, p, p, p, p, p, p, p,
                                     i, i, i, i, i, p, i, i, ctypes.POINTER(ctypes.c_int)]
+    if hasattr(lib, "gdn_oracle_fwd"):
+        lib.gdn_oracle_fwd.restype = ctypes.c_int
+        lib.gdn_oracle_fwd.argtypes = [p, p, p, p, p, p, i, p, p,
+                                       i, i, i, i, i, p, i, i, ctypes.POINTER(ctypes.c_int)]
     return lib
 
 
@@ -118,4 +127,50 @@ def step(r, w, k, v, a, b, state, nthreads: int = 0):
     """
     r, w, k, v, a, b = (_f64(x)[:, None] for x in (r, w, k, v, a, b))
     o, sT, _ = fwd(r, w, k, v, a, b, s0=_f64(state), nthreads=nthreads)
+    return o[:, 0], sT
+
+
+def _cu(cu_seqlens):
+    if cu_seqlens is None:
+        return None
+    return np.ascontiguousarray(np.asarray(
+        cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int32))
+
+
+def gdn_fwd(q, k, v, g, beta, s0=None, cu_seqlens=None, output_final_state: bool = True,
+            nthreads: int = 0, library=None):
+    """Gated DeltaNet oracle forward.  Returns (o [B,T,H,V], sT [N,H,K,V] or None, threads).
+
+    q, k: [B,T,H,K]; v: [B,T,H,V]; g, beta: [B,T,H]; s0: [N,H,K,V], [1,H,K,V]
+    (one state shared by every sequence) or None (zeros); cu_seqlens: [N+1] or None.
+    """
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    assert k.shape == (B, T, H, K) and v.shape == (B, T, H, V)
+    assert g.shape == (B, T, H) and beta.shape == (B, T, H)
+    cu = _cu(cu_seqlens)
+    N = B if cu is None else cu.shape[0] - 1
+    s0 = _f64(s0)
+    shared = 0
+    if s0 is not None:
+        assert s0.shape in ((N, H, K, V), (1, H, K, V))
+        shared = int(s0.shape[0] == 1 and N != 1)
+    o = np.zeros((B, T, H, V), dtype=np.float64)
+    sT = np.zeros((N, H, K, V), dtype=np.float64) if output_final_state else None
+    used = ctypes.c_int(0)
+    lib = _load() if library is None else library
+    rc = lib.gdn_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0), shared,
+                            _ptr(o), _ptr(sT), B, T, H, K, V, _ptr(cu), N, int(nthreads),
+                            ctypes.byref(used))
+    if rc != 0:
+        raise ValueError("gdn_oracle_fwd rejected its arguments")
+    return o, sT, used.value
+
+
+def gdn_step(q, k, v, g, beta, state, nthreads: int = 0):
+    """One Gated DeltaNet decode step: q, k [B,H,K], v [B,H,V], g, beta [B,H],
+    state [B,H,K,V] (not modified).  Returns (o [B,H,V], new_state) in float64."""
+    q, k, v, g, beta = (_f64(x)[:, None] for x in (q, k, v, g, beta))
+    o, sT, _ = gdn_fwd(q, k, v, g, beta, s0=_f64(state), nthreads=nthreads)
     return o[:, 0], sT

@@ -28,6 +28,9 @@
  * Layouts (all dense, row-major): r,w,k,a,b [B,T,H,K]; v [B,T,H,V];
  * o [B,T,H,V]; s0 / sT [N,H,K,V]; mask [B,T] (nonzero = update).
  * Without cu_seqlens N == B.  With cu_seqlens B == 1 and T == cu_seqlens[N].
+ *
+ * gdn_oracle_fwd, at the end of this file, is the Gated DeltaNet operator of
+ * the same README, written on its own (it does not call the function above).
  */
 #include <math.h>
 #include <stdint.h>
@@ -133,6 +136,120 @@ int wkv7_oracle_fwd(const double* r, const double* w, const double* k,
             const int eos = cu_seqlens ? cu_seqlens[n + 1] : T;
             oracle_unit(r, w, k, v, a, b, s0, mask, o, sT, T, H, K, V, bb, bos,
                         eos, n, h, S, S + (size_t)K * V);
+        }
+        free(S);
+    }
+#endif
+    if (threads_used) *threads_used = used;
+    return 0;
+}
+
+/*
+ * Gated DeltaNet (rwkv-ops 0.9.0 README, "gdn_recurrent 使用方法" and
+ * "gdn_chunk 使用方法": gated_delta_net_recurrent / _chunk / _single_step).
+ * q, k [B,T,H,K] are L2-normalised over K inside the op; v [B,T,H,V]; g [B,T,H]
+ * is the log-space decay gate; beta [B,T,H] the write strength, already in (0,1).
+ * initial_state is [N,H,K,V], or [1,H,K,V] shared by every sequence.  The
+ * README names the operator but prints no formula; this is the Gated DeltaNet
+ * rule in its delta-rule form, per (sequence, head) and token:
+ *
+ *     qh = q / |q|,  kh = k / |k|          (a zero vector stays zero)
+ *     S  <- exp(g) S                        (the gate decays the old state)
+ *     e   = v - S^T kh                      (what the gated state predicts for kh)
+ *     S  <- S + beta kh e^T                 (delta-rule correction)
+ *     o   = S^T qh
+ *
+ * No further scaling of q (the README states none).
+ */
+static void unit_normalise(const double* x, double* y, int n) {
+    double ss = 0.0;
+    for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+    const double nrm = sqrt(ss);
+    for (int i = 0; i < n; ++i) y[i] = nrm > 0.0 ? x[i] / nrm : 0.0;
+}
+
+static void gdn_unit(const double* q, const double* k, const double* v,
+                     const double* g, const double* beta, const double* s0,
+                     int s0_shared, double* o, double* sT, int T, int H, int K,
+                     int V, int bb, int bos, int eos, int n, int h, double* S,
+                     double* work) {
+    double* qh = work;
+    double* kh = work + K;
+    double* e = work + 2 * (size_t)K;
+    const size_t state_off = ((size_t)n * H + h) * (size_t)K * V;
+    const size_t init_off = ((size_t)(s0_shared ? 0 : n) * H + h) * (size_t)K * V;
+    if (s0)
+        memcpy(S, s0 + init_off, sizeof(double) * (size_t)K * V);
+    else
+        memset(S, 0, sizeof(double) * (size_t)K * V);
+
+    for (int t = bos; t < eos; ++t) {
+        const size_t tok = ((size_t)bb * T + t) * H + h;
+        unit_normalise(q + tok * K, qh, K);
+        unit_normalise(k + tok * K, kh, K);
+        const double alpha = exp(g[tok]);
+        const double bt = beta[tok];
+        for (size_t i = 0; i < (size_t)K * V; ++i) S[i] *= alpha;
+        for (int j = 0; j < V; ++j) {
+            double pred = 0.0;
+            for (int i = 0; i < K; ++i) pred += S[(size_t)i * V + j] * kh[i];
+            e[j] = v[tok * V + j] - pred;
+        }
+        for (int i = 0; i < K; ++i)
+            for (int j = 0; j < V; ++j) S[(size_t)i * V + j] += bt * kh[i] * e[j];
+        for (int j = 0; j < V; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < K; ++i) acc += S[(size_t)i * V + j] * qh[i];
+            o[tok * V + j] = acc;
+        }
+    }
+    if (sT) memcpy(sT + state_off, S, sizeof(double) * (size_t)K * V);
+}
+
+/* Same conventions and return codes as wkv7_oracle_fwd; s0_shared != 0 means
+ * s0 holds one [H,K,V] state used by every sequence. */
+int gdn_oracle_fwd(const double* q, const double* k, const double* v,
+                   const double* g, const double* beta, const double* s0,
+                   int s0_shared, double* o, double* sT, int B, int T, int H,
+                   int K, int V, const int32_t* cu_seqlens, int N, int nthreads,
+                   int* threads_used) {
+    if (!q || !k || !v || !g || !beta || !o) return 1;
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0) return 1;
+    if (cu_seqlens) {
+        if (B != 1 || N < 0 || cu_seqlens[0] != 0 || cu_seqlens[N] != T) return 1;
+        for (int n = 0; n < N; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n]) return 1;
+    } else {
+        N = B;
+    }
+    const long units = (long)N * H;
+    const size_t scratch = (size_t)K * V + 2 * (size_t)K + V;
+    int used = 1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel
+    {
+#pragma omp single
+        used = omp_get_num_threads();
+        double* S = (double*)malloc(sizeof(double) * scratch);
+#pragma omp for schedule(dynamic, 1)
+        for (long unit = 0; unit < units; ++unit) {
+            const int n = (int)(unit / H), h = (int)(unit % H);
+            gdn_unit(q, k, v, g, beta, s0, s0_shared, o, sT, T, H, K, V,
+                     cu_seqlens ? 0 : n, cu_seqlens ? cu_seqlens[n] : 0,
+                     cu_seqlens ? cu_seqlens[n + 1] : T, n, h, S, S + (size_t)K * V);
+        }
+        free(S);
+    }
+#else
+    (void)nthreads;
+    {
+        double* S = (double*)malloc(sizeof(double) * scratch);
+        for (long unit = 0; unit < units; ++unit) {
+            const int n = (int)(unit / H), h = (int)(unit % H);
+            gdn_unit(q, k, v, g, beta, s0, s0_shared, o, sT, T, H, K, V,
+                     cu_seqlens ? 0 : n, cu_seqlens ? cu_seqlens[n] : 0,
+                     cu_seqlens ? cu_seqlens[n + 1] : T, n, h, S, S + (size_t)K * V);
         }
         free(S);
     }
