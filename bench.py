@@ -12,6 +12,8 @@ Under torchrun (N > 1) every rank runs its own replica of the workload (the
 (sequence, head) units are independent, no collective on the data path) and
 rank 0 prints the whole-job throughput: all ranks' tokens / max-over-ranks time.
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample instead.
+``--family gdn`` measures the Gated DeltaNet entry points (wkv7_gdn_fwd /
+wkv7_gdn_step) on workloads of the same shapes instead.
 """
 from __future__ import annotations
 
@@ -36,6 +38,10 @@ FWD = synth.WORKLOADS["fwd_bf16_b8_t4096_h64"]
 DEC = synth.WORKLOADS["step_bf16_b1024_h32_256steps"]
 TOKEN_HEAD_BYTES = 6 * 64 * 2 + 64 * 2  # r,w,k,v,a,b in + o out, bf16
 STATE_BYTES = 64 * 64 * 4
+GDN_METRIC = "Gated DeltaNet fwd tokens/s (B=8,T=4096,H=64,D=64 bf16) + decode HBM GB/s vs peak"
+GDN_FWD = synth.WORKLOADS["gdn_fwd_bf16_b8_t4096_h64"]
+GDN_DEC = synth.WORKLOADS["gdn_step_bf16_b1024_h32_256steps"]
+GDN_TOKEN_HEAD_BYTES = 3 * 64 * 2 + 2 * 2 + 64 * 2  # q,k,v + g,beta in, o out, bf16
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -45,6 +51,14 @@ def fwd_algorithmic_bytes(B, T, H) -> int:
 
 def step_algorithmic_bytes(B, H) -> int:
     return B * H * (2 * STATE_BYTES + 7 * 64 * 2)
+
+
+def gdn_fwd_algorithmic_bytes(B, T, H) -> int:
+    return B * T * H * GDN_TOKEN_HEAD_BYTES + 2 * B * H * STATE_BYTES
+
+
+def gdn_step_algorithmic_bytes(B, H) -> int:
+    return B * H * (2 * STATE_BYTES + GDN_TOKEN_HEAD_BYTES)
 
 
 def load_peaks():
@@ -127,18 +141,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_oracle_sample(target_s: float = 12.0):
+def cpu_oracle_sample(target_s: float = 12.0, gdn: bool = False):
     """Time the fp64 oracle (as it stands) on a bounded sample of the B=8,T=4096,H=64
     workload: whole (b, h) units of T=4096 tokens.  Returns the cpu_baseline dict."""
     import oracle  # test infrastructure; used here only for the CPU baseline leg
-    x = synth.fwd_inputs(1, FWD["T"], FWD["H"], dtype=torch.bfloat16, seed=FWD["seed"],
-                         s0_std=FWD["s0_std"])
+    if gdn:
+        x = synth.gdn_inputs(1, GDN_FWD["T"], GDN_FWD["H"], dtype=torch.bfloat16,
+                             seed=GDN_FWD["seed"], s0_std=GDN_FWD["s0_std"])
+        names, call = ("q", "k", "v", "g", "beta"), oracle.gdn_fwd
+    else:
+        x = synth.fwd_inputs(1, FWD["T"], FWD["H"], dtype=torch.bfloat16, seed=FWD["seed"],
+                             s0_std=FWD["s0_std"])
+        names, call = tuple("rwkvab"), oracle.fwd
     H = FWD["H"]
 
     def run(units):
-        sl = {n: x[n][:, :, :units] for n in "rwkvab"}
+        sl = {n: x[n][:, :, :units] for n in names}
         t0 = time.perf_counter()
-        _, _, used = oracle.fwd(*(sl[n] for n in "rwkvab"), s0=x["s0"][:, :units])
+        _, _, used = call(*(sl[n] for n in names), s0=x["s0"][:, :units])
         return time.perf_counter() - t0, used
 
     probe_units = min(H, max(2, os.cpu_count() or 1))
@@ -211,6 +231,9 @@ def main():
     ap.add_argument("--workload", choices=["b8_t4096_h64", "masked_b16_t4096_h32",
                                            "varlen_64seq_h32"], default="b8_t4096_h64",
                     help="forward workload (the metric is quoted on b8_t4096_h64)")
+    ap.add_argument("--family", choices=["wkv7", "gdn"], default="wkv7",
+                    help="gdn: the Gated DeltaNet entry points on the B=8,T=4096,H=64 "
+                         "forward and 1024x32 decode workloads")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -222,7 +245,8 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
-    from linear_attention_rnn_wkv7_b200 import wkv7_fwd, wkv7_step, library
+    from linear_attention_rnn_wkv7_b200 import (library, wkv7_fwd, wkv7_gdn_fwd, wkv7_gdn_step,
+                                                wkv7_step)
     library()  # fail loudly if the CUDA library is missing
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
@@ -244,20 +268,22 @@ def main():
     hbm_peak, peak_kind = load_peaks()
     stream = torch.cuda.current_stream(device)
     fwd = None
+    gdn = args.family == "gdn"
     if args.only in ("all", "fwd"):
-        fwd = fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
-                      barrier, rank, world)
+        fwd = fwd_leg(args, device, stream, wkv7_gdn_fwd if gdn else wkv7_fwd, hbm_peak,
+                      peak_kind, max_over_ranks, barrier, rank, world)
     decode = None
     if args.only in ("all", "decode") and not args.no_decode:
-        decode = decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks,
-                            barrier, rank)
+        decode = decode_leg(device, stream, wkv7_gdn_step if gdn else wkv7_step, hbm_peak,
+                            peak_kind, max_over_ranks, barrier, rank, gdn)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu and args.only == "all":
-        cpu = cpu_oracle_sample()
+        cpu = cpu_oracle_sample(gdn=gdn)
 
     if rank == 0:
         desc = fwd["desc"] if fwd else {"workload": "none"}
-        line = {"metric": METRIC, "value": fwd and fwd["value"], "unit": "tokens/s",
+        line = {"metric": GDN_METRIC if gdn else METRIC, "value": fwd and fwd["value"],
+                "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": fwd and fwd["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -273,6 +299,15 @@ def main():
 def fwd_workload(args, rank):
     """Synthetic inputs, tokens per step and algorithmic bytes per launch of a workload."""
     mask = cu = None
+    if args.family == "gdn":
+        if args.workload != "b8_t4096_h64":
+            raise SystemExit("--family gdn runs the b8_t4096_h64 workload only")
+        B, T, H = args.batch, GDN_FWD["T"], GDN_FWD["H"]
+        x = synth.gdn_inputs(B, T, H, dtype=torch.bfloat16,
+                             seed=replicas.replica_seed(GDN_FWD["seed"], rank),
+                             s0_std=GDN_FWD["s0_std"])
+        return (x, None, None, B, T, H, B * T, gdn_fwd_algorithmic_bytes(B, T, H),
+                {"workload": f"gdn_fwd_bf16_b{B}_t{T}_h{H}", "B": B, "T": T, "H": H})
     if args.workload == "b8_t4096_h64":
         B, T, H = args.batch, FWD["T"], FWD["H"]
         x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16,
@@ -320,9 +355,14 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
     o = torch.empty(B, T, H, 64, dtype=torch.bfloat16, device=device)
     sT = torch.empty(N, H, 64, 64, dtype=torch.float32, device=device)
 
-    def step():
-        wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
-                 mask=maskd, cu_seqlens=cud, algo=args.algo, o=o, sT=sT)
+    if args.family == "gdn":
+        def step():
+            wkv7_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], s0=xd["s0"],
+                     algo=args.algo, o=o, sT=sT)
+    else:
+        def step():
+            wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
+                     mask=maskd, cu_seqlens=cud, algo=args.algo, o=o, sT=sT)
 
     for _ in range(args.warmup):
         step()
@@ -344,6 +384,8 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
 
     achieved = fwd_bytes / (ms_step / 1e3) / 1e9
     kernel = "chunked" if args.algo in ("auto", "chunked") else "recurrent"
+    if args.family == "gdn":
+        kernel = "gdn_" + kernel
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
                 "kernel": kernel,
@@ -386,24 +428,25 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
             "clocks": clock_info, "desc": desc}
 
 
-def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank):
-    """256 consecutive wkv7_step calls over 1024 x 32 fp32 states (512 MiB, > L2).
-    Step inputs: 32 independently drawn step sets, used in turn."""
-    B, H, steps = DEC["B"], DEC["H"], DEC["steps"]
-    state = synth.decode_state(B, H, seed=replicas.replica_seed(DEC["seed"], rank),
-                               std=DEC["s0_std"]).to(device)
+def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank,
+               gdn=False):
+    """256 consecutive wkv7_step (or wkv7_gdn_step) calls over 1024 x 32 fp32 states
+    (512 MiB, > L2).  Step inputs: 32 independently drawn step sets, used in turn."""
+    p = GDN_DEC if gdn else DEC
+    B, H, steps = p["B"], p["H"], p["steps"]
+    state = synth.decode_state(B, H, seed=replicas.replica_seed(p["seed"], rank),
+                               std=p["s0_std"]).to(device)
     sets = []
+    names = ("q", "k", "v", "g", "beta") if gdn else ("r", "w", "k", "v", "a", "b")
+    draw = synth.gdn_step_inputs if gdn else synth.decode_step_inputs
     for i in range(32):
-        x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16,
-                                     seed=replicas.replica_seed(DEC["seed"], rank),
-                                     step=i)
-        sets.append({k: v.to(device) for k, v in x.items()})
+        x = draw(B, H, dtype=torch.bfloat16, seed=replicas.replica_seed(p["seed"], rank), step=i)
+        sets.append(tuple(x[n].to(device) for n in names))
     o = torch.empty(B, H, 64, dtype=torch.bfloat16, device=device)
 
     def run(n):
         for i in range(n):
-            x = sets[i % len(sets)]
-            wkv7_step(x["r"], x["w"], x["k"], x["v"], x["a"], x["b"], state, o=o)
+            wkv7_step(*sets[i % len(sets)], state, o=o)
 
     run(3)
     torch.cuda.synchronize(device)
@@ -415,13 +458,14 @@ def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, b
     torch.cuda.synchronize(device)
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
-    nbytes = step_algorithmic_bytes(B, H)
+    nbytes = gdn_step_algorithmic_bytes(B, H) if gdn else step_algorithmic_bytes(B, H)
     gbs = nbytes / (ms / 1e3) / 1e9
-    return {"workload": "step_bf16_b1024_h32_256steps", "steps": steps, "us_per_step": 1e3 * ms,
+    return {"workload": ("gdn_" if gdn else "") + "step_bf16_b1024_h32_256steps", "steps": steps,
+            "us_per_step": 1e3 * ms,
             "algorithmic_bytes_per_step": nbytes, "GB/s": gbs, "peak": hbm_peak,
             "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
             "tokens/s": B / (ms / 1e3), "gpu_launches": steps,
-            "traffic": profiled_traffic("step_b1024_h32")}
+            "traffic": profiled_traffic(("gdn_" if gdn else "") + "step_b1024_h32")}
 
 
 if __name__ == "__main__":

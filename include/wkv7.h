@@ -114,6 +114,57 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
                       int K, int V, wkv7_dtype dtype, void* stream);
 
 /*
+ * wkv7_gdn_fwd -- Gated DeltaNet forward over whole sequences
+ * (gated_delta_net_recurrent / gated_delta_net_recurrent_inference /
+ * gated_delta_net_chunk; rwkv-ops 0.9.0 README, "gdn_recurrent 使用方法" and
+ * "gdn_chunk 使用方法"), computed by the same kernels as wkv7_fwd.  Per
+ * (sequence, head) and token, with qh = q / |q| and kh = k / |k| over K (the
+ * README: q and k are L2-normalised inside; a zero vector stays zero):
+ *
+ *     S_t = exp(g_t) (I - beta_t kh_t kh_t^T) S_{t-1} + beta_t kh_t v_t^T
+ *     o_t = S_t^T qh_t
+ *
+ * i.e. the generalized rule above with w_t = g_t on every channel, a_t = kh_t,
+ * b_t = -exp(g_t) beta_t kh_t and write key beta_t kh_t.  q is not scaled
+ * further (the README states no scale).
+ *
+ *   q, k           [B, T, H, K]  dtype   query and key (normalised inside)
+ *   v              [B, T, H, V]  dtype
+ *   g              [B, T, H]     dtype   log-space decay gate (exp(g) multiplies the state)
+ *   beta           [B, T, H]     dtype   write strength, expected in (0, 1) (README: already
+ *                                        passed through a sigmoid; not checked)
+ *   s0             [N, H, K, V]  fp32    initial states, or NULL for zeros; with s0_shared = 1
+ *                                        a single [1, H, K, V] state used by every sequence
+ *   o              [B, T, H, V]  dtype   output (must not alias an input)
+ *   sT             [N, H, K, V]  fp32    final states, or NULL; may equal s0 unless s0_shared
+ *                                        and N > 1
+ *   cu_seqlens, N, algo, stream          as for wkv7_fwd (no mask: the README's operator has none)
+ *
+ * q, k, v, o, s0, sT must be 16-byte aligned; g and beta only aligned to their element.
+ * The chunked form has the range stated for wkv7_fwd: a chunk's summed gate within
+ * -80, and state / v magnitudes below 65504.
+ */
+wkv7_status wkv7_gdn_fwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* s0, int s0_shared, void* o, float* sT,
+                         int B, int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
+                         wkv7_dtype dtype, wkv7_algo algo, void* stream);
+
+/*
+ * wkv7_gdn_step -- one Gated DeltaNet decode token for B independent states
+ * (gated_delta_net_recurrent_single_step; README: q, k (B, H, K), v (B, H, V),
+ * g, beta (B, H), state (B, H, K, V)).
+ *
+ *   q, k           [B, H, K]     dtype
+ *   v              [B, H, V]     dtype
+ *   g, beta        [B, H]        dtype   (element-aligned)
+ *   state          [B, H, K, V]  fp32    read and updated IN PLACE
+ *   o              [B, H, V]     dtype   o = S_t^T qh (must not alias state or inputs)
+ */
+wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const void* g,
+                          const void* beta, float* state, void* o, int B, int H, int K, int V,
+                          wkv7_dtype dtype, void* stream);
+
+/*
  * wkv7_get_last_error -- synchronises `stream`, returns and clears the sticky
  * device-side flag (WKV7_ERR_DEVICE_TIMEOUT / WKV7_ERR_DEVICE_BAD_SEQLENS) of
  * the current device, or WKV7_ERR_CUDA if the stream reports a CUDA error,

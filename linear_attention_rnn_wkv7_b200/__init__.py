@@ -1,12 +1,13 @@
 """B200-native (sm_100a) WKV7: the RWKV-7 generalized delta rule behind a C ABI.
 
-``wkv7_fwd`` / ``wkv7_step`` call libwkv7.so (hand-written CUDA kernels);
+``wkv7_fwd`` / ``wkv7_step`` (and the Gated DeltaNet ``wkv7_gdn_fwd`` /
+``wkv7_gdn_step``) call libwkv7.so (hand-written CUDA kernels);
 ``synth`` draws the seeded synthetic workloads.  Importing this package does
 not load the CUDA library; the first call does, and fails loudly if it is
 missing.
 """
-from .wkv7 import (WKV7Error, library, status_string, wkv7_fwd, wkv7_get_last_error,  # noqa: F401
-                   wkv7_step)
+from .wkv7 import (WKV7Error, library, status_string, wkv7_fwd, wkv7_gdn_fwd,  # noqa: F401
+                   wkv7_gdn_step, wkv7_get_last_error, wkv7_step)
 
-__all__ = ["wkv7_fwd", "wkv7_step", "wkv7_get_last_error", "library", "status_string",
-           "WKV7Error"]
+__all__ = ["wkv7_fwd", "wkv7_step", "wkv7_gdn_fwd", "wkv7_gdn_step", "wkv7_get_last_error",
+           "library", "status_string", "WKV7Error"]

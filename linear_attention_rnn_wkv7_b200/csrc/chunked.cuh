@@ -35,6 +35,14 @@
 // Gram entry stays finite in fp32 and bf16), so the factorisation is exact while
 // g_t - g_L <= 80 inside a chunk (per-step log decay >= -1.26; the RWKV-7
 // parametrisation keeps it >= -0.607).
+//
+// Gated DeltaNet (rwkv-ops 0.9.0 README, "gdn_recurrent 使用方法" / "gdn_chunk
+// 使用方法") runs through the same kernel (template flag kGdn): its transition
+// e^{g} (I - beta kh kh^T) and write beta kh v^T are the generalized rule with one
+// log decay per token on every channel (w_t = g_t), a = kh, b = -e^{g} beta kh and
+// write key beta kh, where qh and kh are q and k L2-normalised over K.  Only the
+// loads (q, k, v by TMA; g and beta per token) and the prologue differ: the scan is
+// over one scalar per token, and the operands are built from qh and kh in registers.
 #pragma once
 #include <cuda.h>
 
@@ -255,19 +263,28 @@ struct Ctx {
     int* abort_flag;
     float* gamma_s;
     const CUtensorMap *tm_r, *tm_w, *tm_k, *tm_v, *tm_a, *tm_b;
+    const __nv_bfloat16 *g, *beta;  // Gated DeltaNet only: [rows, H]
 };
 
 // Lanes 0..5 of the calling warp: request the six 64 x 64 bf16 input tiles of the chunk
 // starting at token c0 into layout `par` (lane 0 arms the barrier first; the
-// six copies are issued in parallel).
+// six copies are issued in parallel).  Gated DeltaNet loads three (q, k, v into the
+// r, k, v tiles).
+template <bool kGdn>
 __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
     const LayR L = lay_of(par);
     using namespace sm100;
     const int lane = cx.lane;
-    if (lane == 0) mbar_arrive_expect_tx(cx.bar_tma, 6 * kTile);
+    if (lane == 0) mbar_arrive_expect_tx(cx.bar_tma, (kGdn ? 3 : 6) * kTile);
     __syncwarp();
     const int row = (int)(cx.row0 + c0);
-    if (lane < 6) {
+    if constexpr (kGdn) {
+        if (lane < 3) {
+            const CUtensorMap* map = lane == 0 ? cx.tm_r : lane == 1 ? cx.tm_k : cx.tm_v;
+            const uint32_t dst = lane == 0 ? L.R : lane == 1 ? L.K : L.V;
+            tma_load_3d(cx.sbase + dst, map, cx.bar_tma, 0, cx.h, row);
+        }
+    } else if (lane < 6) {
         const CUtensorMap* map = lane == 0 ? cx.tm_r : lane == 1 ? cx.tm_a : lane == 2 ? cx.tm_k
                                : lane == 3 ? cx.tm_b : lane == 4 ? cx.tm_w : cx.tm_v;
         const uint32_t dst = lane == 0 ? L.R : lane == 1 ? L.A : lane == 2 ? L.K
@@ -277,6 +294,7 @@ __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
 }
 
 // One 64-token chunk starting at token c0, in layout P (its inputs already requested).
+template <bool kGdn>
 __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
     const LayR L = lay_of(par);
     using namespace sm100;
@@ -294,6 +312,19 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
     float* scratch = reinterpret_cast<float*>(smem + L.ARK);  // prologue only
     float* F0 = reinterpret_cast<float*>(smem + L.F0);
     const int nv = min(64, cx.len - c0);
+    float gq[2] = {0.f, 0.f}, bq[2] = {0.f, 0.f};  // Gated DeltaNet: g, beta of tokens t0, t0+1
+    if constexpr (kGdn) {  // issued before the tile wait, so their latency overlaps it
+        const int t0 = 2 * (tid >> 3);
+        const long long tok = (row0 + c0 + t0) * H + h;
+        if (t0 < nv) {
+            gq[0] = __bfloat162float(cx.g[tok]);
+            bq[0] = __bfloat162float(cx.beta[tok]);
+        }
+        if (t0 + 1 < nv) {
+            gq[1] = __bfloat162float(cx.g[tok + H]);
+            bq[1] = __bfloat162float(cx.beta[tok + H]);
+        }
+    }
     wait_or_abort(cx.bar_tma, par, abort_flag);
 
         // ---- 2. prefix sums of w (mask folded) and every scaled operand, in one pass.
@@ -307,92 +338,11 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             const bool va = t0 < nv && (!mask || mask[row0 + c0 + t0] != 0);
             const bool vb = t0 + 1 < nv && (!mask || mask[row0 + c0 + t0 + 1] != 0);
             const uint32_t offa = sw(t0, j), offb = sw(t0 + 1, j);
-            float wa[8], wb[8], incl[8];
-            {  // a masked token's w is zero (cleared on the packed words)
-                const uint32_t ma = va ? 0xFFFFFFFFu : 0u, mb = vb ? 0xFFFFFFFFu : 0u;
-                uint4 qa = *reinterpret_cast<const uint4*>(smem + L.W + offa);
-                uint4 qb = *reinterpret_cast<const uint4*>(smem + L.W + offb);
-                qa.x &= ma; qa.y &= ma; qa.z &= ma; qa.w &= ma;
-                qb.x &= mb; qb.y &= mb; qb.z &= mb; qb.w &= mb;
-                unpack8(qa, wa);
-                unpack8(qb, wb);
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {  // log decays in log2 units from here on
-                wa[e] *= kLog2e;
-                wb[e] *= kLog2e;
-                incl[e] = wa[e] + wb[e];
-            }
-#pragma unroll
-            for (int d = 8; d < 32; d *= 2) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float up = __shfl_up_sync(0xffffffffu, incl[e], d);
-                    if (lane >= d) incl[e] += up;
-                }
-            }
-            float* wt = scratch + SCR_TOT;  // [warp][channel] sums of w over the warp's 8 tokens
-            if (lane >= 24) {
-                *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j) =
-                    make_float4(incl[0], incl[1], incl[2], incl[3]);
-                *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j + 4) =
-                    make_float4(incl[4], incl[5], incl[6], incl[7]);
-            }
-            __syncthreads();
-            if (warp == 0) {  // per channel: exclusive prefixes over the warps, c = g_L, e^{g_L}
-                const int ch = 2 * lane;
-                float2 gL = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int w2 = 0; w2 < 8; ++w2) {
-                    const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
-                    reinterpret_cast<float2*>(scratch + SCR_PRE + w2 * 64)[lane] = gL;
-                    gL.x += x.x; gL.y += x.y;
-                }
-                reinterpret_cast<float2*>(scratch + SCR_C)[lane] = gL;
-                reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(ex2(gL.x), ex2(gL.y));
-            }
-            __syncthreads();  // per-channel constants ready
-            float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
-            {
-                const float4 x0 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j);
-                const float4 x1 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j + 4);
-                const float pre[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ga[e] = pre[e] + (incl[e] - wb[e]);
-            }
-            float cc[8], ec[8];  // c = g_L (log2 units) and e^{g_L}
-            *reinterpret_cast<float4*>(cc) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[0];
-            *reinterpret_cast<float4*>(cc + 4) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[1];
-            *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[0];
-            *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[1];
-            float Ep[8];  // E at token t0 - 1 (g_{t0-1} = g_{t0} - w_{t0})
-#pragma unroll
-            for (int e = 0; e < 8; ++e) Ep[e] = ex2(clamp2(ga[e] - wa[e] - cc[e]));
-            float rts[2][8], ats[2][8];  // fp32 r~ and a~, kept for Rbar and Abar
-#pragma unroll
-            for (int it = 0; it < 2; ++it) {
+            float rts[2][8], ats[2][8], ec[8];  // fp32 r~ and a~, kept for Rbar and Abar; e^{g_L}
+            // The token's operands to shared memory: r~, a~, k~ (bf16; the bf16 low part of
+            // k~ for the Gram's fourth group), b~ (bf16 and fp16 as Bhat), Khat (fp32).
+            auto put = [&](int it, const float* kt, const float* btl) {
                 const uint32_t off = it ? offb : offa;
-                const bool val = it ? vb : va;
-                float rv[8], av[8], kv[8], bv[8];
-                unpack8(*reinterpret_cast<const uint4*>(smem + L.R + off), rv);
-                unpack8(*reinterpret_cast<const uint4*>(smem + L.A + off), av);
-                unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv);
-                unpack8(*reinterpret_cast<const uint4*>(smem + L.B + off), bv);
-                float kt[8], btl[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float g = it ? ga[e] + wb[e] : ga[e];
-                    const float d = clamp2(g - cc[e]);
-                    const float E = ex2(d);  // e^{g_t - g_L}
-                    // A masked token writes nothing: its a, k, b scales are zero.
-                    const float inv = val ? ex2(-d) : 0.f;
-                    const float ep = val ? Ep[e] : 0.f;
-                    rts[it][e] = rv[e] * E;
-                    ats[it][e] = av[e] * ep;
-                    kt[e] = kv[e] * inv;   // = Khat (fp32)
-                    btl[e] = bv[e] * inv;  // = Bhat
-                    Ep[e] = E;  // E_{t-1} of the next token
-                }
                 *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rts[it]);
                 *reinterpret_cast<uint4*>(smem + L.A + off) = pack8(ats[it]);
                 const uint4 kq = pack8(kt);
@@ -409,6 +359,162 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 float4* kh = reinterpret_cast<float4*>(F0 + (t0 + it) * 64 + 8 * j);
                 kh[0] = make_float4(kt[0], kt[1], kt[2], kt[3]);
                 kh[1] = make_float4(kt[4], kt[5], kt[6], kt[7]);
+            };
+            if constexpr (kGdn) {
+                // Gated DeltaNet: one log decay per token, so the scan runs on one value per
+                // token pair; qh, kh from the tiles with norms reduced over the pair's 8 lanes.
+                const float wa = va ? gq[0] * kLog2e : 0.f, wb = vb ? gq[1] * kLog2e : 0.f;
+                float incl = wa + wb;
+#pragma unroll
+                for (int d = 8; d < 32; d *= 2) {
+                    const float up = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += up;
+                }
+                if (lane == 24) scratch[SCR_TOT + warp] = incl;  // the warp's 8-token sum
+                float qv[2][8], kv[2][8], nq[2], nk[2];
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const uint32_t off = it ? offb : offa;
+                    unpack8(*reinterpret_cast<const uint4*>(smem + L.R + off), qv[it]);
+                    unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv[it]);
+                    float sq = 0.f, sk = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        sq = fmaf(qv[it][e], qv[it][e], sq);
+                        sk = fmaf(kv[it][e], kv[it][e], sk);
+                    }
+#pragma unroll
+                    for (int m = 1; m < 8; m *= 2) {
+                        sq += __shfl_xor_sync(0xffffffffu, sq, m);
+                        sk += __shfl_xor_sync(0xffffffffu, sk, m);
+                    }
+                    nq[it] = sq > 0.f ? rsqrtf(sq) : 0.f;  // a zero vector stays zero
+                    nk[it] = sk > 0.f ? rsqrtf(sk) : 0.f;
+                }
+                __syncthreads();
+                float pre = 0.f, gL = 0.f;  // earlier warps' sum; g_L (log2 units)
+#pragma unroll
+                for (int w2 = 0; w2 < 8; ++w2) {
+                    const float x = scratch[SCR_TOT + w2];
+                    pre += (w2 < warp) ? x : 0.f;
+                    gL += x;
+                }
+                const float eg = ex2(gL);
+                if (tid < 64) gamma_s[tid] = eg;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ec[e] = eg;
+                const float ga = pre + (incl - wb);  // g at token t0
+                float Ep = ex2(clamp2(ga - wa - gL));   // E_{t0-1}
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const bool val = it ? vb : va;
+                    const float d = clamp2((it ? ga + wb : ga) - gL);
+                    const float E = ex2(d);
+                    const float inv = val ? ex2(-d) : 0.f;  // a masked token writes nothing
+                    const float ep = val ? Ep : 0.f;
+                    const float bw = bq[it] * inv;                   // beta / E
+                    const float bb = -ex2(it ? wb : wa) * bw;       // -e^{g} beta / E
+                    const float rq = nq[it] * E, ak = nk[it] * ep;
+                    float kt[8], btl[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float kn = kv[it][e] * nk[it];
+                        rts[it][e] = qv[it][e] * rq;
+                        ats[it][e] = kv[it][e] * ak;
+                        kt[e] = kn * bw;
+                        btl[e] = kn * bb;
+                    }
+                    Ep = E;
+                    put(it, kt, btl);
+                }
+            } else {
+                float wa[8], wb[8], incl[8];
+                {  // a masked token's w is zero (cleared on the packed words)
+                    const uint32_t ma = va ? 0xFFFFFFFFu : 0u, mb = vb ? 0xFFFFFFFFu : 0u;
+                    uint4 qa = *reinterpret_cast<const uint4*>(smem + L.W + offa);
+                    uint4 qb = *reinterpret_cast<const uint4*>(smem + L.W + offb);
+                    qa.x &= ma; qa.y &= ma; qa.z &= ma; qa.w &= ma;
+                    qb.x &= mb; qb.y &= mb; qb.z &= mb; qb.w &= mb;
+                    unpack8(qa, wa);
+                    unpack8(qb, wb);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {  // log decays in log2 units from here on
+                    wa[e] *= kLog2e;
+                    wb[e] *= kLog2e;
+                    incl[e] = wa[e] + wb[e];
+                }
+#pragma unroll
+                for (int d = 8; d < 32; d *= 2) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float up = __shfl_up_sync(0xffffffffu, incl[e], d);
+                        if (lane >= d) incl[e] += up;
+                    }
+                }
+                float* wt = scratch + SCR_TOT;  // [warp][channel] sums of w over the warp's 8 tokens
+                if (lane >= 24) {
+                    *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j) =
+                        make_float4(incl[0], incl[1], incl[2], incl[3]);
+                    *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j + 4) =
+                        make_float4(incl[4], incl[5], incl[6], incl[7]);
+                }
+                __syncthreads();
+                if (warp == 0) {  // per channel: exclusive prefixes over the warps, c = g_L, e^{g_L}
+                    const int ch = 2 * lane;
+                    float2 gL = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int w2 = 0; w2 < 8; ++w2) {
+                        const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
+                        reinterpret_cast<float2*>(scratch + SCR_PRE + w2 * 64)[lane] = gL;
+                        gL.x += x.x; gL.y += x.y;
+                    }
+                    reinterpret_cast<float2*>(scratch + SCR_C)[lane] = gL;
+                    reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(ex2(gL.x), ex2(gL.y));
+                }
+                __syncthreads();  // per-channel constants ready
+                float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
+                {
+                    const float4 x0 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j);
+                    const float4 x1 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j + 4);
+                    const float pre[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ga[e] = pre[e] + (incl[e] - wb[e]);
+                }
+                float cc[8];  // c = g_L (log2 units)
+                *reinterpret_cast<float4*>(cc) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[0];
+                *reinterpret_cast<float4*>(cc + 4) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[1];
+                *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[0];
+                *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[1];
+                float Ep[8];  // E at token t0 - 1 (g_{t0-1} = g_{t0} - w_{t0})
+#pragma unroll
+                for (int e = 0; e < 8; ++e) Ep[e] = ex2(clamp2(ga[e] - wa[e] - cc[e]));
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const uint32_t off = it ? offb : offa;
+                    const bool val = it ? vb : va;
+                    float rv[8], av[8], kv[8], bv[8];
+                    unpack8(*reinterpret_cast<const uint4*>(smem + L.R + off), rv);
+                    unpack8(*reinterpret_cast<const uint4*>(smem + L.A + off), av);
+                    unpack8(*reinterpret_cast<const uint4*>(smem + L.K + off), kv);
+                    unpack8(*reinterpret_cast<const uint4*>(smem + L.B + off), bv);
+                    float kt[8], btl[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float g = it ? ga[e] + wb[e] : ga[e];
+                        const float d = clamp2(g - cc[e]);
+                        const float E = ex2(d);  // e^{g_t - g_L}
+                        // A masked token writes nothing: its a, k, b scales are zero.
+                        const float inv = val ? ex2(-d) : 0.f;
+                        const float ep = val ? Ep[e] : 0.f;
+                        rts[it][e] = rv[e] * E;
+                        ats[it][e] = av[e] * ep;
+                        kt[e] = kv[e] * inv;   // = Khat (fp32)
+                        btl[e] = bv[e] * inv;  // = Bhat
+                        Ep[e] = E;  // E_{t-1} of the next token
+                    }
+                    put(it, kt, btl);
+                }
             }
             fence_proxy_async();
             tc_fence_before();
@@ -774,7 +880,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 
         // The next chunk's inputs go to the other layout's input tiles, all of which
         // are dead now; the copy overlaps this chunk's final MMA and epilogue.
-        if (has_next && warp == 1) issue_loads(cx, c0 + 64, par ^ 1);
+        if (has_next && warp == 1) issue_loads<kGdn>(cx, c0 + 64, par ^ 1);
 
         // ---- 9. final MMA: [S upd; O] = A_fin [S0; V]  (128 x 64 x 128, fp16) ------------
         if (tid == 0) {
@@ -820,12 +926,17 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         tc_fence_before();
 }
 
+// kGdn: Gated DeltaNet (tm_r, tm_k, tm_v map q, k, v; g and beta per token; s0 may be
+// one state per head shared by every sequence, s0_shared != 0).
+template <bool kGdn>
 __global__ void __launch_bounds__(kThreads, 2)
 chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
-               float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens) {
+               float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens,
+               const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ beta,
+               int s0_shared) {
     extern __shared__ __align__(1024) uint8_t smem[];
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -896,6 +1007,8 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     cx.tm_v = &tm_v;
     cx.tm_a = &tm_a;
     cx.tm_b = &tm_b;
+    cx.g = g;
+    cx.beta = beta;
 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 16);
     if (warp == 0) {
@@ -915,7 +1028,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     if (warp == 0 && lane < 6)
         prefetch_tensormap(lane == 0 ? &tm_r : lane == 1 ? &tm_a : lane == 2 ? &tm_k
                            : lane == 3 ? &tm_b : lane == 4 ? &tm_w : &tm_v);
-    if (warp == 0 && cx.len > 0) issue_loads(cx, 0, 0);
+    if (warp == 0 && cx.len > 0) issue_loads<kGdn>(cx, 0, 0);
 
     // The fp32 state lives in tensor memory, rows 0..63 of the final product's
     // columns: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
@@ -928,7 +1041,8 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
 #pragma unroll
         for (int j = 0; j < 32; ++j) sv[j] = 0.f;
         if (s0) {
-            const float4* src = reinterpret_cast<const float4*>(s0 + state_off + m_row * 64 + 32 * wh);
+            const size_t init_off = s0_shared ? (size_t)h * 4096 : state_off;
+            const float4* src = reinterpret_cast<const float4*>(s0 + init_off + m_row * 64 + 32 * wh);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float4 f = src[j];
@@ -951,7 +1065,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
 
     // Chunks alternate between the two shared-memory layouts.
     for (int c0 = 0, par = 0; c0 < cx.len; c0 += 64, par ^= 1) {
-        chunk(cx, c0, c0 + 64 < cx.len, par);
+        chunk<kGdn>(cx, c0, c0 + 64 < cx.len, par);
         if (*cx.abort_flag) break;
     }
 
@@ -1005,27 +1119,51 @@ inline bool make_map(CUtensorMap* map, const void* ptr, long long rows, int H) {
 
 }  // namespace chunked
 
-inline cudaError_t launch_chunked(const void* r, const void* w, const void* k, const void* v,
-                                  const void* a, const void* b, const float* s0,
-                                  const uint8_t* mask, void* o, float* sT, int B, int T, int H,
-                                  int N, const int32_t* cu_seqlens, cudaStream_t stream) {
-    using namespace chunked;
+namespace chunked {
+template <bool kGdn>
+inline cudaError_t launch(const void* const* ptrs, int nmaps, const float* s0,
+                          const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
+                          const int32_t* cu_seqlens, const void* g, const void* beta,
+                          int s0_shared, cudaStream_t stream) {
     const long long rows = (long long)B * T;
     CUtensorMap maps[6];
-    const void* ptrs[6] = {r, w, k, v, a, b};
-    for (int i = 0; i < 6; ++i)
+    for (int i = 0; i < nmaps; ++i)
         if (!make_map(&maps[i], ptrs[i], rows, H)) return cudaErrorInvalidValue;
+    for (int i = nmaps; i < 6; ++i) maps[i] = maps[0];  // unused by the kernel
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    chunked_kernel<<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
+    chunked_kernel<kGdn><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], s0, mask,
-        static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens);
+        static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens,
+        static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(beta), s0_shared);
     return cudaGetLastError();
+}
+}  // namespace chunked
+
+inline cudaError_t launch_chunked(const void* r, const void* w, const void* k, const void* v,
+                                  const void* a, const void* b, const float* s0,
+                                  const uint8_t* mask, void* o, float* sT, int B, int T, int H,
+                                  int N, const int32_t* cu_seqlens, cudaStream_t stream) {
+    const void* ptrs[6] = {r, w, k, v, a, b};
+    return chunked::launch<false>(ptrs, 6, s0, mask, o, sT, B, T, H, N, cu_seqlens, nullptr,
+                                  nullptr, 0, stream);
+}
+
+// Gated DeltaNet: q, k, v [B*T, H, 64] bf16 through the r, k, v maps; g, beta [B*T, H].
+inline cudaError_t launch_chunked_gdn(const void* q, const void* k, const void* v,
+                                      const void* g, const void* beta, const float* s0,
+                                      int s0_shared, void* o, float* sT, int B, int T, int H,
+                                      int N, const int32_t* cu_seqlens, cudaStream_t stream) {
+    // map order r, w, k, v: the unused w slot repeats q
+    const void* ptrs[4] = {q, q, k, v};
+    return chunked::launch<true>(ptrs, 4, s0, nullptr, o, sT, B, T, H, N, cu_seqlens, g, beta,
+                                 s0_shared, stream);
 }
 
 }  // namespace wkv7

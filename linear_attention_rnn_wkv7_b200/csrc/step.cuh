@@ -14,6 +14,12 @@
 //     shuffle (xor 16) per column;
 //   - the per-token vectors (r, exp w, k, a, b) go through a 1.25 KiB per-warp
 //     shared-memory stage so each lane reads its 32 rows as float4 broadcasts.
+//
+// kGdn: the Gated DeltaNet single step (rwkv-ops 0.9.0 README,
+// gated_delta_net_recurrent_single_step).  The stage holds r = qh, exp(w) = e^{g},
+// write key beta kh, a = kh, b = -e^{g} beta kh (qh, kh: q and k over their L2
+// norms, reduced across the warp), so the same update applies
+// e^{g} (I - beta kh kh^T) S + beta kh v^T.
 #pragma once
 #include "common.cuh"
 
@@ -21,11 +27,12 @@ namespace wkv7 {
 
 constexpr int kStepWarps = 4;  // units per block
 
-template <typename Tin>
+template <typename Tin, bool kGdn>
 __global__ void __launch_bounds__(kStepWarps * 32)
 step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
             const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
-            float* __restrict__ state, Tin* __restrict__ o, long long units) {
+            float* __restrict__ state, Tin* __restrict__ o, long long units,
+            const Tin* __restrict__ g, const Tin* __restrict__ beta) {
     __shared__ __align__(16) float vec[kStepWarps][5][64];  // r, d = exp(w), k, a, b
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -42,7 +49,26 @@ step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
 #pragma unroll
     for (int m = 0; m < 32; ++m) S[m] = S_g[(32 * p + m) * 16 + c];
 
-    {
+    if constexpr (kGdn) {
+        const float2 qq = load2(r + voff + 2 * lane);
+        const float2 kk = load2(k + voff + 2 * lane);
+        float sq = qq.x * qq.x + qq.y * qq.y, sk = kk.x * kk.x + kk.y * kk.y;
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, m);
+            sk += __shfl_xor_sync(0xffffffffu, sk, m);
+        }
+        const float nq = sq > 0.f ? rsqrtf(sq) : 0.f, nk = sk > 0.f ? rsqrtf(sk) : 0.f;
+        const float alpha = expf(to_f32(g[unit])), bt = to_f32(beta[unit]);
+        const float2 kn = make_float2(kk.x * nk, kk.y * nk);
+        float* vv = &vec[warp][0][0];
+        reinterpret_cast<float2*>(vv + 0 * 64)[lane] = make_float2(qq.x * nq, qq.y * nq);
+        reinterpret_cast<float2*>(vv + 1 * 64)[lane] = make_float2(alpha, alpha);
+        reinterpret_cast<float2*>(vv + 2 * 64)[lane] = make_float2(bt * kn.x, bt * kn.y);
+        reinterpret_cast<float2*>(vv + 3 * 64)[lane] = kn;
+        reinterpret_cast<float2*>(vv + 4 * 64)[lane] =
+            make_float2(-alpha * bt * kn.x, -alpha * bt * kn.y);
+    } else {
         const float2 rr = load2(r + voff + 2 * lane);
         const float2 ww = load2(w + voff + 2 * lane);
         const float2 kk = load2(k + voff + 2 * lane);
@@ -122,10 +148,23 @@ cudaError_t launch_step(const void* r, const void* w, const void* k, const void*
                         const void* a, const void* b, float* state, void* o, long long units,
                         cudaStream_t stream) {
     const long long blocks = (units + kStepWarps - 1) / kStepWarps;
-    step_kernel<Tin><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
+    step_kernel<Tin, false><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
         static_cast<const Tin*>(r), static_cast<const Tin*>(w), static_cast<const Tin*>(k),
         static_cast<const Tin*>(v), static_cast<const Tin*>(a), static_cast<const Tin*>(b),
-        state, static_cast<Tin*>(o), units);
+        state, static_cast<Tin*>(o), units, nullptr, nullptr);
+    return cudaGetLastError();
+}
+
+// Gated DeltaNet step: q, k [units, 64], v [units, 64], g, beta [units].
+template <typename Tin>
+cudaError_t launch_step_gdn(const void* q, const void* k, const void* v, const void* g,
+                            const void* beta, float* state, void* o, long long units,
+                            cudaStream_t stream) {
+    const long long blocks = (units + kStepWarps - 1) / kStepWarps;
+    step_kernel<Tin, true><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
+        static_cast<const Tin*>(q), nullptr, static_cast<const Tin*>(k),
+        static_cast<const Tin*>(v), nullptr, nullptr, state, static_cast<Tin*>(o), units,
+        static_cast<const Tin*>(g), static_cast<const Tin*>(beta));
     return cudaGetLastError();
 }
 

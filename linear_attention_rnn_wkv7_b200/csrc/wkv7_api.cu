@@ -17,6 +17,12 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 
+// Non-null and aligned to its element (g, beta are read one element at a time).
+inline bool ok_scalar_ptr(const void* p, wkv7_dtype dtype) {
+    const uintptr_t m = dtype == WKV7_BF16 ? 1u : 3u;
+    return p != nullptr && (reinterpret_cast<uintptr_t>(p) & m) == 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -101,6 +107,76 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
         dtype == WKV7_BF16
             ? wkv7::launch_step<__nv_bfloat16>(r, w, k, v, a, b, state, o, units, stream)
             : wkv7::launch_step<float>(r, w, k, v, a, b, state, o, units, stream);
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+wkv7_status wkv7_gdn_fwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* s0, int s0_shared, void* o, float* sT,
+                         int B, int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
+                         wkv7_dtype dtype, wkv7_algo algo, void* stream_) {
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0 || N < 0) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_RECURRENT && algo != WKV7_ALGO_CHUNKED)
+        return WKV7_ERR_INVALID_ARG;
+    if (s0_shared != 0 && s0_shared != 1) return WKV7_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (B != 1) return WKV7_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return WKV7_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return WKV7_ERR_INVALID_ARG;
+    }
+    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)N * H;
+    const long long rows = (long long)B * T * H;
+    if (units > 0x7fffffffLL || rows > (1LL << 40)) return WKV7_ERR_UNSUPPORTED;
+    const bool tokens = rows > 0;
+    if (tokens && (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) ||
+                   !ok_scalar_ptr(g, dtype) || !ok_scalar_ptr(beta, dtype)))
+        return WKV7_ERR_INVALID_ARG;
+    if ((s0 && !aligned16(s0)) || (sT && !aligned16(sT))) return WKV7_ERR_INVALID_ARG;
+    if (tokens && (o == q || o == k || o == v || o == g || o == beta))
+        return WKV7_ERR_INVALID_ARG;
+    if (s0_shared && sT && s0 == sT && N > 1) return WKV7_ERR_INVALID_ARG;
+    if (units == 0) return WKV7_OK;
+    if (!s0) s0_shared = 0;
+
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool chunked = rows > 0 && (algo == WKV7_ALGO_CHUNKED ||
+                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && wkv7::kChunkedBuilt));
+    cudaError_t err;
+    if (chunked) {
+        if (dtype != WKV7_BF16 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
+        err = wkv7::launch_chunked_gdn(q, k, v, g, beta, s0, s0_shared, o, sT, B, T, H, N,
+                                       cu_seqlens, stream);
+    } else if (dtype == WKV7_BF16) {
+        err = wkv7::launch_recurrent_gdn<__nv_bfloat16>(q, k, v, g, beta, s0, s0_shared, o, sT,
+                                                        T, H, N, cu_seqlens, stream);
+    } else {
+        err = wkv7::launch_recurrent_gdn<float>(q, k, v, g, beta, s0, s0_shared, o, sT, T, H,
+                                                N, cu_seqlens, stream);
+    }
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const void* g,
+                          const void* beta, float* state, void* o, int B, int H, int K, int V,
+                          wkv7_dtype dtype, void* stream_) {
+    if (B < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)B * H;
+    if (units == 0) return WKV7_OK;
+    if (units > (1LL << 33)) return WKV7_ERR_UNSUPPORTED;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(state) || !ok_ptr(o) ||
+        !ok_scalar_ptr(g, dtype) || !ok_scalar_ptr(beta, dtype))
+        return WKV7_ERR_INVALID_ARG;
+    if (o == state || o == q || o == k || o == v || o == g || o == beta)
+        return WKV7_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const cudaError_t err =
+        dtype == WKV7_BF16
+            ? wkv7::launch_step_gdn<__nv_bfloat16>(q, k, v, g, beta, state, o, units, stream)
+            : wkv7::launch_step_gdn<float>(q, k, v, g, beta, state, o, units, stream);
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 

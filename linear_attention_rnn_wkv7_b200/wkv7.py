@@ -9,7 +9,9 @@ missing or the tensors are not on a CUDA device, the call raises.
 Names follow the C ABI: ``wkv7_fwd`` (generalized_delta_rule /
 generalized_delta_rule_inference, forward only) and ``wkv7_step``
 (rwkv7_op_rnn) -- rwkv-ops 0.9.0 README, sections "rwkv7op 使用方法" and
-"rwkv7_op_rnn 使用方法".
+"rwkv7_op_rnn 使用方法"; ``wkv7_gdn_fwd`` / ``wkv7_gdn_step`` (Gated DeltaNet:
+gated_delta_net_recurrent / _chunk / _single_step, same README, "gdn_recurrent
+使用方法" and "gdn_chunk 使用方法").
 """
 from __future__ import annotations
 
@@ -47,6 +49,10 @@ def library() -> ctypes.CDLL:
         lib.wkv7_fwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i, i, i, i, i, p, i, i, i, p]
         lib.wkv7_step.restype = i
         lib.wkv7_step.argtypes = [p, p, p, p, p, p, p, p, i, i, i, i, i, p]
+        lib.wkv7_gdn_fwd.restype = i
+        lib.wkv7_gdn_fwd.argtypes = [p, p, p, p, p, p, i, p, p, i, i, i, i, i, p, i, i, i, p]
+        lib.wkv7_gdn_step.restype = i
+        lib.wkv7_gdn_step.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, p]
         lib.wkv7_get_last_error.restype = i
         lib.wkv7_get_last_error.argtypes = [p]
         lib.wkv7_status_string.restype = ctypes.c_char_p
@@ -148,6 +154,70 @@ def wkv7_step(r, w, k, v, a, b, state, o=None):
                              _ptr(o), B, H, K, V, _dtype_code(r), _stream(r.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_step")
+    return o
+
+
+def wkv7_gdn_fwd(q, k, v, g, beta, s0=None, cu_seqlens=None, output_final_state: bool = True,
+                 algo: str = "auto", o=None, sT=None):
+    """Gated DeltaNet forward.  q, k [B,T,H,K]; v [B,T,H,V]; g, beta [B,T,H] (bf16 or
+    fp32, all alike); s0 [N,H,K,V] or [1,H,K,V] (shared) fp32 or None; cu_seqlens
+    [N+1] int32 (B must be 1) or None.  Returns (o [B,T,H,V], sT [N,H,K,V] or None)."""
+    _check(q, "q")
+    dt = q.dtype
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    _check(k, "k", dt, (B, T, H, K))
+    _check(v, "v", dt, (B, T, H, V))
+    _check(g, "g", dt, (B, T, H))
+    _check(beta, "beta", dt, (B, T, H))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    shared = 0
+    if s0 is not None:
+        _check(s0, "s0", torch.float32)
+        if tuple(s0.shape) == (1, H, K, V) and N != 1:
+            shared = 1
+        elif tuple(s0.shape) != (N, H, K, V):
+            raise ValueError(f"s0 must have shape {(N, H, K, V)} or {(1, H, K, V)}")
+    if o is None:
+        o = torch.empty((B, T, H, V), dtype=dt, device=q.device)
+    else:
+        _check(o, "o", dt, (B, T, H, V))
+    if output_final_state and sT is None:
+        sT = torch.empty((N, H, K, V), dtype=torch.float32, device=q.device)
+    elif sT is not None:
+        _check(sT, "sT", torch.float32, (N, H, K, V))
+    st = library().wkv7_gdn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0), shared,
+                                _ptr(o), _ptr(sT), B, T, H, K, V, _ptr(cu_seqlens), N,
+                                _dtype_code(q), ALGO[algo], _stream(q.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_gdn_fwd")
+    return o, sT
+
+
+def wkv7_gdn_step(q, k, v, g, beta, state, o=None):
+    """One Gated DeltaNet decode token.  q, k [B,H,K]; v [B,H,V]; g, beta [B,H];
+    state [B,H,K,V] fp32, updated in place.  Returns o [B,H,V]."""
+    _check(q, "q")
+    dt = q.dtype
+    B, H, K = q.shape
+    V = v.shape[-1]
+    _check(k, "k", dt, (B, H, K))
+    _check(v, "v", dt, (B, H, V))
+    _check(g, "g", dt, (B, H))
+    _check(beta, "beta", dt, (B, H))
+    _check(state, "state", torch.float32, (B, H, K, V))
+    if o is None:
+        o = torch.empty((B, H, V), dtype=dt, device=q.device)
+    else:
+        _check(o, "o", dt, (B, H, V))
+    st = library().wkv7_gdn_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                 _ptr(o), B, H, K, V, _dtype_code(q), _stream(q.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_gdn_step")
     return o
 
 

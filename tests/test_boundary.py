@@ -33,7 +33,8 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     names = declared_functions()
-    for required in ("wkv7_fwd", "wkv7_step", "wkv7_get_last_error", "wkv7_status_string"):
+    for required in ("wkv7_fwd", "wkv7_step", "wkv7_gdn_fwd", "wkv7_gdn_step",
+                     "wkv7_get_last_error", "wkv7_status_string"):
         assert required in names
 
 
@@ -109,3 +110,54 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         wkv7.wkv7_step(x[:, 0], x[:, 0], x[:, 0], x[:, 0], x[:, 0], x[:, 0],
                        torch.zeros(1, 1, 64, 64))
+
+
+def gdn(lib, ptrs=None, B=1, T=8, H=2, K=64, V=64, cu=None, N=None, dtype=BF16, algo=0,
+        s0=None, shared=0, sT=None, o=None):
+    ptrs = ptrs or [P + 0x1000 * i for i in range(5)]
+    o = P + 0x10000 if o is None else o
+    N = B if N is None else N
+    return lib.wkv7_gdn_fwd(*[ctypes.c_void_p(x) if x else None for x in ptrs],
+                            ctypes.c_void_p(s0) if s0 else None, shared,
+                            ctypes.c_void_p(o) if o else None, ctypes.c_void_p(sT) if sT else None,
+                            B, T, H, K, V, ctypes.c_void_p(cu) if cu else None, N, dtype, algo,
+                            None)
+
+
+def test_gdn_fwd_rejects_bad_arguments(lib):
+    assert gdn(lib, K=128) == ERR_UNSUPPORTED
+    assert gdn(lib, H=0) == ERR_INVALID_ARG
+    assert gdn(lib, dtype=3) == ERR_INVALID_ARG
+    assert gdn(lib, algo=5) == ERR_INVALID_ARG
+    assert gdn(lib, shared=2) == ERR_INVALID_ARG
+    assert gdn(lib, ptrs=[P, P + 16, P + 32, 0, P + 64]) == ERR_INVALID_ARG  # null g
+    assert gdn(lib, ptrs=[P, P + 16, P + 32, P + 49, P + 64]) == ERR_INVALID_ARG  # odd bf16 g
+    assert gdn(lib, ptrs=[P, P + 16, P + 32, P + 50, P + 66], dtype=F32) == ERR_INVALID_ARG
+    assert gdn(lib, ptrs=[P, P + 8, P + 32, P + 48, P + 64]) == ERR_INVALID_ARG  # k not 16-aligned
+    assert gdn(lib, o=P) == ERR_INVALID_ARG  # o aliases q
+    assert gdn(lib, B=2, N=3) == ERR_INVALID_ARG
+    assert gdn(lib, B=2, s0=P + 0x30000, sT=P + 0x30000, shared=1) == ERR_INVALID_ARG
+    assert gdn(lib, dtype=F32, algo=2) == ERR_UNSUPPORTED
+    assert gdn(lib, B=0, N=0) == OK
+
+
+def test_gdn_step_rejects_bad_arguments(lib):
+    ptrs = [ctypes.c_void_p(P + 0x1000 * i) for i in range(5)]
+    st, o = ctypes.c_void_p(P + 0x10000), ctypes.c_void_p(P + 0x20000)
+    assert lib.wkv7_gdn_step(*ptrs, st, o, 4, 2, 32, 64, BF16, None) == ERR_UNSUPPORTED
+    assert lib.wkv7_gdn_step(*ptrs, st, o, 4, 0, 64, 64, BF16, None) == ERR_INVALID_ARG
+    assert lib.wkv7_gdn_step(*ptrs, st, st, 4, 2, 64, 64, BF16, None) == ERR_INVALID_ARG
+    bad = ptrs[:3] + [ctypes.c_void_p(P + 0x3001), ptrs[4]]
+    assert lib.wkv7_gdn_step(*bad, st, o, 4, 2, 64, 64, BF16, None) == ERR_INVALID_ARG
+    assert lib.wkv7_gdn_step(*ptrs, st, o, 0, 2, 64, 64, BF16, None) == OK
+
+
+def test_gdn_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
+    s = torch.zeros(1, 4, 1, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        wkv7.wkv7_gdn_fwd(x, x, x, s, s)
+    with pytest.raises(ValueError, match="CUDA"):
+        wkv7.wkv7_gdn_step(x[:, 0], x[:, 0], x[:, 0], s[:, 0], s[:, 0],
+                           torch.zeros(1, 1, 64, 64))
