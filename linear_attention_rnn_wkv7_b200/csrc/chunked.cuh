@@ -63,7 +63,7 @@ constexpr int kThreads = 256;
 constexpr uint32_t kTile = 8192;
 constexpr uint32_t OFF_S0 = 11 * kTile;    // S0 bf16 [k][v] (final MMA B, MN-major), both layouts
 constexpr uint32_t OFF_MISC = 14 * kTile;  // mbarriers, TMEM address, abort flag
-constexpr uint32_t OFF_GAMMA = OFF_MISC + 64;  // e^{g_L} per channel (64 fp32)
+constexpr uint32_t OFF_GAMMA = OFF_MISC + 64;  // e^{g_L}, channel c at cswz(c) (64 fp32)
 constexpr uint32_t kSmemBytes = OFF_GAMMA + 256;
 
 template <int P>
@@ -82,7 +82,7 @@ struct Lay<0> {
     static constexpr uint32_t ARBT = 8 * kTile;   // A_rb^T [s][t] (MMA-3 A, MN-major atom 1)
     static constexpr uint32_t ARK = 9 * kTile;    // A_rk [t][s] (epilogue 3); prologue scratch
     static constexpr uint32_t RBAR = 10 * kTile;  // Rbar [t][k] (epilogue 3)
-    static constexpr uint32_t F0 = 12 * kTile;    // fp32 64x64 (2 tiles): E_t, then Khat [s][k]
+    static constexpr uint32_t F0 = 12 * kTile;    // fp32 64x64 (2 tiles): Khat [s][cswz(k)]
 };
 // Odd chunks: the six input tiles land in tiles the even layout no longer needs
 // once its epilogue 3 is done (Bhat, A_rb^T, A_rk, Rbar, Khat), and vice versa.
@@ -117,10 +117,9 @@ __device__ __forceinline__ LayR lay_of(int par) {
 // Aliases inside one chunk (lifetimes do not overlap):
 //   A_ab [t][s]          R: fp16 blocks left of the diagonal; A: fp32 diagonal
 //                        blocks (epilogue 1 -> W|Z substitution)
-//   fp32 T_ii + scratch  K (2 tiles)   W|Z substitution
-//   [M'; Rbar + A_rb W]  R (2 tiles)   epilogue 3 -> final MMA A, K block 0
-//   [P_N hi; A_rk+A_rb Z] ABAR (2)     epilogue 3 -> final MMA A, K block 1
-//   [P_N lo; 0]          K (2 tiles)   epilogue 3 -> final MMA A, K block 2
+//   T_ii, T_ii A_im      K: fp16 16x16 blocks with 48-byte rows (W|Z substitution)
+//   [M'; Rbar + A_rb W]  R (2 tiles)   epilogue 3 -> final MMA A, K block 0 (B: S0)
+//   [P_N; A_rk + A_rb Z] ABAR (2)      epilogue 3 -> final MMA A, K block 1 (B: V)
 // Prologue scratch inside the A_rk tile (free until epilogue 1), in floats.
 constexpr int SCR_TOT = 0, SCR_C = 512, SCR_PRE = 576;  // floats (SCR_PRE: 8 x 64)
 // Tensor-memory columns (fp32 accumulators, 128 lanes).
@@ -140,11 +139,18 @@ __device__ __forceinline__ uint32_t swe(uint32_t row, uint32_t col) {
 }
 
 // Float index of element (r, c) of diagonal 16x16 block bb of A_ab, kept in fp32
-// (blocks 260 floats apart and 16-byte chunks permuted by r % 4, so the rows a warp
-// writes together and the blocks it reads together fall in different banks).
+// (rows 20 floats apart, so the float4 chunks eight rows write together fall in eight
+// different bank groups; blocks 324 floats apart, so the two blocks a warp reads
+// together do too).
 __device__ __forceinline__ int didx(int bb, int r, int c) {
-    return bb * 260 + r * 16 + ((((c >> 2) ^ (r & 3)) << 2) | (c & 3));
+    return bb * 324 + r * 20 + c;
 }
+
+// Position of channel c in a 64-float per-channel row (prologue scratch, e^{g_L},
+// Khat rows): the two 16-byte halves of each 32-byte group swap places in the upper
+// half of the row, so that lanes j and j + 4 of a thread's eight 32-byte strided
+// float4 accesses land in different banks.
+__device__ __forceinline__ int cswz(int c) { return c ^ ((c & 32) >> 3); }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -338,6 +344,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             const bool va = t0 < nv && (!mask || mask[row0 + c0 + t0] != 0);
             const bool vb = t0 + 1 < nv && (!mask || mask[row0 + c0 + t0 + 1] != 0);
             const uint32_t offa = sw(t0, j), offb = sw(t0 + 1, j);
+            const int h0 = cswz(8 * j), h1 = cswz(8 * j + 4);  // this thread's channel halves
             float rts[2][8], ats[2][8], ec[8];  // fp32 r~ and a~, kept for Rbar and Abar; e^{g_L}
             // The token's operands to shared memory: r~, a~, k~ (bf16; the bf16 low part of
             // k~ for the Gram's fourth group), b~ (bf16 and fp16 as Bhat), Khat (fp32).
@@ -356,9 +363,9 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 }
                 *reinterpret_cast<uint4*>(smem + L.B + off) = pack8(btl);
                 *reinterpret_cast<uint4*>(smem + L.W + off) = pack8h(btl);  // Bhat (fp16)
-                float4* kh = reinterpret_cast<float4*>(F0 + (t0 + it) * 64 + 8 * j);
-                kh[0] = make_float4(kt[0], kt[1], kt[2], kt[3]);
-                kh[1] = make_float4(kt[4], kt[5], kt[6], kt[7]);
+                float* kh = F0 + (t0 + it) * 64;
+                *reinterpret_cast<float4*>(kh + h0) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+                *reinterpret_cast<float4*>(kh + h1) = make_float4(kt[4], kt[5], kt[6], kt[7]);
             };
             if constexpr (kGdn) {
                 // Gated DeltaNet: one log decay per token, so the scan runs on one value per
@@ -454,38 +461,38 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 }
                 float* wt = scratch + SCR_TOT;  // [warp][channel] sums of w over the warp's 8 tokens
                 if (lane >= 24) {
-                    *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j) =
+                    *reinterpret_cast<float4*>(wt + warp * 64 + h0) =
                         make_float4(incl[0], incl[1], incl[2], incl[3]);
-                    *reinterpret_cast<float4*>(wt + warp * 64 + 8 * j + 4) =
+                    *reinterpret_cast<float4*>(wt + warp * 64 + h1) =
                         make_float4(incl[4], incl[5], incl[6], incl[7]);
                 }
                 __syncthreads();
                 if (warp == 0) {  // per channel: exclusive prefixes over the warps, c = g_L, e^{g_L}
-                    const int ch = 2 * lane;
+                    const int ch = cswz(2 * lane);  // channels 2 lane, 2 lane + 1
                     float2 gL = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int w2 = 0; w2 < 8; ++w2) {
                         const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
-                        reinterpret_cast<float2*>(scratch + SCR_PRE + w2 * 64)[lane] = gL;
+                        *reinterpret_cast<float2*>(scratch + SCR_PRE + w2 * 64 + ch) = gL;
                         gL.x += x.x; gL.y += x.y;
                     }
-                    reinterpret_cast<float2*>(scratch + SCR_C)[lane] = gL;
-                    reinterpret_cast<float2*>(gamma_s)[lane] = make_float2(ex2(gL.x), ex2(gL.y));
+                    *reinterpret_cast<float2*>(scratch + SCR_C + ch) = gL;
+                    *reinterpret_cast<float2*>(gamma_s + ch) = make_float2(ex2(gL.x), ex2(gL.y));
                 }
                 __syncthreads();  // per-channel constants ready
                 float ga[8];  // g at token t0: earlier warps + this warp's pairs up to t0
                 {
-                    const float4 x0 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j);
-                    const float4 x1 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + 8 * j + 4);
+                    const float4 x0 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + h0);
+                    const float4 x1 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + h1);
                     const float pre[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) ga[e] = pre[e] + (incl[e] - wb[e]);
                 }
                 float cc[8];  // c = g_L (log2 units)
-                *reinterpret_cast<float4*>(cc) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[0];
-                *reinterpret_cast<float4*>(cc + 4) = reinterpret_cast<const float4*>(scratch + SCR_C + 8 * j)[1];
-                *reinterpret_cast<float4*>(ec) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[0];
-                *reinterpret_cast<float4*>(ec + 4) = reinterpret_cast<const float4*>(gamma_s + 8 * j)[1];
+                *reinterpret_cast<float4*>(cc) = *reinterpret_cast<const float4*>(scratch + SCR_C + h0);
+                *reinterpret_cast<float4*>(cc + 4) = *reinterpret_cast<const float4*>(scratch + SCR_C + h1);
+                *reinterpret_cast<float4*>(ec) = *reinterpret_cast<const float4*>(gamma_s + h0);
+                *reinterpret_cast<float4*>(ec + 4) = *reinterpret_cast<const float4*>(gamma_s + h1);
                 float Ep[8];  // E at token t0 - 1 (g_{t0-1} = g_{t0} - w_{t0})
 #pragma unroll
                 for (int e = 0; e < 8; ++e) Ep[e] = ex2(clamp2(ga[e] - wa[e] - cc[e]));
@@ -658,13 +665,13 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         //             X_i = T_ii RHS_i + sum_{m<i} (T_ii A_im) X_m.
         //         The 16x16 diagonal inverses T_ii come from fp32 forward substitution;
         //         the products T_ii A_im and T_ii RHS_i are independent and run in
-        //         parallel on warp-level bf16 MMAs (fp32 accumulate); then each warp
+        //         parallel on warp-level fp16 MMAs (fp32 accumulate); then each warp
         //         finishes its own 16 of the 128 right-hand-side columns, writing X in
-        //         place over the right-hand side (bf16), where MMA-3 reads it as its
+        //         place over the right-hand side (fp16), where MMA-3 reads it as its
         //         MN-major B operand. ------------------------------------------------
         {
             const float* Dg = reinterpret_cast<const float*>(smem + L.A);  // diagonal blocks of A_ab
-            // bf16 16x16 blocks with rows of 48 bytes: T_ii (4), then T_ii A_im (6).
+            // fp16 16x16 blocks with rows of 48 bytes: T_ii (4), then T_ii A_im (6).
             uint8_t* Tb = smem + L.K;
             uint8_t* Tab = Tb + 4 * 768;
             if (tid < 64) {  // diagonal block b, column c
@@ -825,7 +832,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int c = 0; c < 4; ++c)
                     *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(k, 4 * wh + c)) = pack8h(sv + 8 * c);
                 {  // the final MMA accumulates onto the state row scaled by e^{g_L}
-                    const float gamma = gamma_s[m_row];
+                    const float gamma = gamma_s[cswz(m_row)];
 #pragma unroll
                     for (int j2 = 0; j2 < 32; ++j2) sv[j2] *= gamma;
                     tmem_row_st32(tmem + TM_DF, wq, 32 * wh, sv);
@@ -835,7 +842,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int c = 0; c < 4; ++c) {  // P_N = Bhat^T Z + Khat^T
                     float pn[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) pn[e] = v[32 + 8 * c + e] + F0[(8 * (4 * wh + c) + e) * 64 + k];
+                    for (int e = 0; e < 8; ++e) pn[e] = v[32 + 8 * c + e] + F0[(8 * (4 * wh + c) + e) * 64 + cswz(k)];
                     *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, 4 * wh + c)) = pack8h(pn);
                 }
                 tmem_st_wait();
