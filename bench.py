@@ -45,20 +45,22 @@ GDN_TOKEN_HEAD_BYTES = 3 * 64 * 2 + 2 * 2 + 64 * 2  # q,k,v + g,beta in, o out, 
 FALLBACK_HBM_GBS = 6650.0
 
 
-def fwd_algorithmic_bytes(B, T, H) -> int:
-    return B * T * H * TOKEN_HEAD_BYTES + 2 * B * H * STATE_BYTES
+def fwd_algorithmic_bytes(B, T, H, D=64) -> int:
+    """bf16 r,w,k,v,a,b in and o out per token-head; fp32 s0 in and sT out per unit."""
+    return B * T * H * 7 * D * 2 + 2 * B * H * D * D * 4
 
 
-def step_algorithmic_bytes(B, H) -> int:
-    return B * H * (2 * STATE_BYTES + 7 * 64 * 2)
+def step_algorithmic_bytes(B, H, D=64) -> int:
+    return B * H * (2 * D * D * 4 + 7 * D * 2)
 
 
-def gdn_fwd_algorithmic_bytes(B, T, H) -> int:
-    return B * T * H * GDN_TOKEN_HEAD_BYTES + 2 * B * H * STATE_BYTES
+def gdn_fwd_algorithmic_bytes(B, T, H, D=64) -> int:
+    """bf16 q,k,v in, o out, g and beta in per token-head; fp32 states per unit."""
+    return B * T * H * (4 * D * 2 + 2 * 2) + 2 * B * H * D * D * 4
 
 
-def gdn_step_algorithmic_bytes(B, H) -> int:
-    return B * H * (2 * STATE_BYTES + GDN_TOKEN_HEAD_BYTES)
+def gdn_step_algorithmic_bytes(B, H, D=64) -> int:
+    return B * H * (2 * D * D * 4 + 4 * D * 2 + 2 * 2)
 
 
 def load_peaks():
@@ -171,8 +173,8 @@ def cpu_oracle_sample(target_s: float = 12.0, gdn: bool = False):
                       f"full T=4096 each; tokens/s = token-heads / 64 / wall time"}
 
 
-def fwd_config(desc: dict, algo: str, world: int) -> dict:
-    return {**desc, "K": 64, "V": 64, "state": "fp32 s0 in, fp32 sT out", "algo": algo,
+def fwd_config(desc: dict, algo: str, world: int, D: int = 64) -> dict:
+    return {**desc, "K": D, "V": D, "state": "fp32 s0 in, fp32 sT out", "algo": algo,
             "parallelism": f"replicas x{world}",
             "l2": "inputs larger than L2 (>= 0.1 GB per step); no flush"}
 
@@ -231,6 +233,9 @@ def main():
     ap.add_argument("--workload", choices=["b8_t4096_h64", "masked_b16_t4096_h32",
                                            "varlen_64seq_h32"], default="b8_t4096_h64",
                     help="forward workload (the metric is quoted on b8_t4096_h64)")
+    ap.add_argument("--head-size", type=int, choices=[64, 128, 256], default=64,
+                    help="K = V; 128 / 256 keep C = H x head size at 4096 (forward) and "
+                         "2048 (decode), and run on the CUDA-core kernels")
     ap.add_argument("--family", choices=["wkv7", "gdn"], default="wkv7",
                     help="gdn: the Gated DeltaNet entry points on the B=8,T=4096,H=64 "
                          "forward and 1024x32 decode workloads")
@@ -275,9 +280,9 @@ def main():
     decode = None
     if args.only in ("all", "decode") and not args.no_decode:
         decode = decode_leg(device, stream, wkv7_gdn_step if gdn else wkv7_step, hbm_peak,
-                            peak_kind, max_over_ranks, barrier, rank, gdn)
+                            peak_kind, max_over_ranks, barrier, rank, gdn, args.head_size)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu and args.only == "all":
+    if rank == 0 and world == 1 and not args.no_cpu and args.only == "all" and args.head_size == 64:
         cpu = cpu_oracle_sample(gdn=gdn)
 
     if rank == 0:
@@ -287,7 +292,7 @@ def main():
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": fwd and fwd["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": fwd_config(desc, args.algo, world),
+                "config": fwd_config(desc, args.algo, world, args.head_size),
                 "roofline": fwd and fwd["roofline"], "cpu_baseline": cpu,
                 "e2e": fwd and fwd["e2e"], "gpu_launches": args.steps if fwd else 0,
                 "clocks": fwd and fwd["clocks"], "decode": decode}
@@ -302,19 +307,25 @@ def fwd_workload(args, rank):
     if args.family == "gdn":
         if args.workload != "b8_t4096_h64":
             raise SystemExit("--family gdn runs the b8_t4096_h64 workload only")
-        B, T, H = args.batch, GDN_FWD["T"], GDN_FWD["H"]
-        x = synth.gdn_inputs(B, T, H, dtype=torch.bfloat16,
+        D = args.head_size
+        B, T, H = args.batch, GDN_FWD["T"], GDN_FWD["H"] * 64 // D
+        x = synth.gdn_inputs(B, T, H, K=D, V=D, dtype=torch.bfloat16,
                              seed=replicas.replica_seed(GDN_FWD["seed"], rank),
                              s0_std=GDN_FWD["s0_std"])
-        return (x, None, None, B, T, H, B * T, gdn_fwd_algorithmic_bytes(B, T, H),
-                {"workload": f"gdn_fwd_bf16_b{B}_t{T}_h{H}", "B": B, "T": T, "H": H})
+        tag = "" if D == 64 else f"_d{D}"
+        return (x, None, None, B, T, H, B * T, gdn_fwd_algorithmic_bytes(B, T, H, D),
+                {"workload": f"gdn_fwd_bf16_b{B}_t{T}_h{H}{tag}", "B": B, "T": T, "H": H})
+    if args.head_size != 64 and args.workload != "b8_t4096_h64":
+        raise SystemExit("--head-size applies to the b8_t4096_h64 workload only")
     if args.workload == "b8_t4096_h64":
-        B, T, H = args.batch, FWD["T"], FWD["H"]
-        x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16,
+        D = args.head_size
+        B, T, H = args.batch, FWD["T"], FWD["H"] * 64 // D
+        x = synth.fwd_inputs(B, T, H, K=D, V=D, dtype=torch.bfloat16,
                              seed=replicas.replica_seed(FWD["seed"], rank), s0_std=FWD["s0_std"])
         tokens = B * T
-        nbytes = fwd_algorithmic_bytes(B, T, H)
-        desc = {"workload": f"fwd_bf16_b{B}_t{T}_h{H}", "B": B, "T": T, "H": H}
+        nbytes = fwd_algorithmic_bytes(B, T, H, D)
+        tag = "" if D == 64 else f"_d{D}"
+        desc = {"workload": f"fwd_bf16_b{B}_t{T}_h{H}{tag}", "B": B, "T": T, "H": H}
     elif args.workload == "masked_b16_t4096_h32":
         p = synth.WORKLOADS["fwd_bf16_masked_b16_t4096_h32"]
         B, T, H = p["B"], p["T"], p["H"]
@@ -352,8 +363,9 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
     maskd = None if mask is None else mask.to(device)
     cud = None if cu is None else cu.to(device)
     N = xd["s0"].shape[0]
-    o = torch.empty(B, T, H, 64, dtype=torch.bfloat16, device=device)
-    sT = torch.empty(N, H, 64, 64, dtype=torch.float32, device=device)
+    D = xd["v"].shape[-1]
+    o = torch.empty(B, T, H, D, dtype=torch.bfloat16, device=device)
+    sT = torch.empty(N, H, D, D, dtype=torch.float32, device=device)
 
     if args.family == "gdn":
         def step():
@@ -383,13 +395,14 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
     value = world * tokens_per_step * args.steps / (ms_total / 1e3)
 
     achieved = fwd_bytes / (ms_step / 1e3) / 1e9
-    kernel = "chunked" if args.algo in ("auto", "chunked") else "recurrent"
+    kernel = "chunked" if args.algo in ("auto", "chunked") and D == 64 else "recurrent"
     if args.family == "gdn":
         kernel = "gdn_" + kernel
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
                 "kernel": kernel,
-                "traffic": profiled_traffic(f"fwd_{kernel}_{args.workload}"),
+                "traffic": profiled_traffic(f"fwd_{kernel}_{args.workload}"
+                                            + ("" if D == 64 else f"_d{D}")),
                 "algorithmic_bytes_per_launch": fwd_bytes}
 
     # End to end through the public call with host buffers: pinned H2D of every
@@ -429,20 +442,21 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
 
 
 def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank,
-               gdn=False):
+               gdn=False, D=64):
     """256 consecutive wkv7_step (or wkv7_gdn_step) calls over 1024 x 32 fp32 states
     (512 MiB, > L2).  Step inputs: 32 independently drawn step sets, used in turn."""
     p = GDN_DEC if gdn else DEC
-    B, H, steps = p["B"], p["H"], p["steps"]
-    state = synth.decode_state(B, H, seed=replicas.replica_seed(p["seed"], rank),
+    B, H, steps = p["B"], p["H"] * 64 // D, p["steps"]
+    state = synth.decode_state(B, H, K=D, V=D, seed=replicas.replica_seed(p["seed"], rank),
                                std=p["s0_std"]).to(device)
     sets = []
     names = ("q", "k", "v", "g", "beta") if gdn else ("r", "w", "k", "v", "a", "b")
     draw = synth.gdn_step_inputs if gdn else synth.decode_step_inputs
     for i in range(32):
-        x = draw(B, H, dtype=torch.bfloat16, seed=replicas.replica_seed(p["seed"], rank), step=i)
+        x = draw(B, H, K=D, V=D, dtype=torch.bfloat16,
+                 seed=replicas.replica_seed(p["seed"], rank), step=i)
         sets.append(tuple(x[n].to(device) for n in names))
-    o = torch.empty(B, H, 64, dtype=torch.bfloat16, device=device)
+    o = torch.empty(B, H, D, dtype=torch.bfloat16, device=device)
 
     def run(n):
         for i in range(n):
@@ -458,14 +472,16 @@ def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, b
     torch.cuda.synchronize(device)
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
-    nbytes = gdn_step_algorithmic_bytes(B, H) if gdn else step_algorithmic_bytes(B, H)
+    nbytes = gdn_step_algorithmic_bytes(B, H, D) if gdn else step_algorithmic_bytes(B, H, D)
     gbs = nbytes / (ms / 1e3) / 1e9
-    return {"workload": ("gdn_" if gdn else "") + "step_bf16_b1024_h32_256steps", "steps": steps,
+    tag = "" if D == 64 else f"_d{D}"
+    return {"workload": ("gdn_" if gdn else "") + f"step_bf16_b{B}_h{H}_256steps{tag}",
+            "steps": steps,
             "us_per_step": 1e3 * ms,
             "algorithmic_bytes_per_step": nbytes, "GB/s": gbs, "peak": hbm_peak,
             "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
             "tokens/s": B / (ms / 1e3), "gpu_launches": steps,
-            "traffic": profiled_traffic(("gdn_" if gdn else "") + "step_b1024_h32")}
+            "traffic": profiled_traffic(("gdn_" if gdn else "") + f"step_b{B}_h{H}{tag}")}
 
 
 if __name__ == "__main__":

@@ -30,8 +30,10 @@
  *    skipped (its outputs are left unwritten) and wkv7_get_last_error reports
  *    it.  No kernel traps, asserts or spins without a bound.
  *  - Inputs r, w, k, a, b are [B, T, H, K]; v is [B, T, H, V]; the output o is
- *    [B, T, H, V]; all of them share one element type (wkv7_dtype).  States
- *    are fp32 [N, H, K, V] (the README's initial_state / final_state layout).
+ *    [B, T, H, V]; all of them share one element type (wkv7_dtype).  With
+ *    WKV7_LAYOUT_BHTK (the README's head_first=True) they are [B, H, T, K] /
+ *    [B, H, T, V] instead.  States are fp32 [N, H, K, V] in both layouts (the
+ *    README's initial_state / final_state layout).
  *  - Supported head sizes: K == V == 64 (the README's default head_size).
  *    Other sizes return WKV7_ERR_UNSUPPORTED.
  */
@@ -59,6 +61,11 @@ typedef enum {
 } wkv7_dtype;
 
 typedef enum {
+    WKV7_LAYOUT_BTHK = 0, /* [B, T, H, *]: token-major (README default, head_first=False) */
+    WKV7_LAYOUT_BHTK = 1  /* [B, H, T, *]: head-first (README head_first=True)            */
+} wkv7_layout;
+
+typedef enum {
     WKV7_ALGO_AUTO = 0,      /* library's choice (chunked tensor-core form for bf16 when built) */
     WKV7_ALGO_RECURRENT = 1, /* token-by-token fp32 recurrence on CUDA cores                  */
     WKV7_ALGO_CHUNKED = 2    /* 64-token chunks, WY form, tcgen05 tensor cores (bf16 only)    */
@@ -81,6 +88,8 @@ typedef enum {
  *                                        [cu_seqlens[n], cu_seqlens[n+1]) of the packed T,
  *                                        cu_seqlens[0] = 0, cu_seqlens[N] = T, non-decreasing.
  *                                        When NULL, N must equal B.
+ *   layout         wkv7_layout           token-major or head-first inputs and o (mask stays
+ *                                        [B, T], states [N, H, K, V])
  *   algo           wkv7_algo             kernel family (WKV7_ALGO_AUTO unless testing)
  *
  * Returns WKV7_OK after enqueueing the kernel(s) on `stream`.
@@ -95,8 +104,8 @@ typedef enum {
 wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
                      const void* a, const void* b, const float* s0, const uint8_t* mask,
                      void* o, float* sT, int B, int T, int H, int K, int V,
-                     const int32_t* cu_seqlens, int N, wkv7_dtype dtype, wkv7_algo algo,
-                     void* stream);
+                     const int32_t* cu_seqlens, int N, wkv7_layout layout, wkv7_dtype dtype,
+                     wkv7_algo algo, void* stream);
 
 /*
  * wkv7_step -- one decode token for B independent states (rwkv7_op_rnn with
@@ -138,7 +147,8 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
  *   o              [B, T, H, V]  dtype   output (must not alias an input)
  *   sT             [N, H, K, V]  fp32    final states, or NULL; may equal s0 unless s0_shared
  *                                        and N > 1
- *   cu_seqlens, N, algo, stream          as for wkv7_fwd (no mask: the README's operator has none)
+ *   cu_seqlens, N, layout, algo, stream  as for wkv7_fwd (no mask: the README's operator has
+ *                                        none); head-first g and beta are [B, H, T]
  *
  * q, k, v, o, s0, sT must be 16-byte aligned; g and beta only aligned to their element.
  * The chunked form has the range stated for wkv7_fwd: a chunk's summed gate within
@@ -147,7 +157,7 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
 wkv7_status wkv7_gdn_fwd(const void* q, const void* k, const void* v, const void* g,
                          const void* beta, const float* s0, int s0_shared, void* o, float* sT,
                          int B, int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
-                         wkv7_dtype dtype, wkv7_algo algo, void* stream);
+                         wkv7_layout layout, wkv7_dtype dtype, wkv7_algo algo, void* stream);
 
 /*
  * wkv7_gdn_step -- one Gated DeltaNet decode token for B independent states

@@ -260,12 +260,16 @@ __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int
 struct Ctx {
     uint8_t* smem;
     uint32_t sbase, tmem, bar_tma, bar_mma, mma_phase;
-    int tid, warp, lane, wq, wh, m_row, h, H;
+    int tid, warp, lane, wq, wh, m_row;
     bool state_thread;
-    long long row0;  // token row of the sequence start
+    long long row0;  // token row of the sequence start in the [B*T] token space (mask)
     int len;
     const uint8_t* mask;
-    __nv_bfloat16* o;
+    __nv_bfloat16* o;  // this unit's first output row; rows o_ts elements apart
+    long long o_ts;
+    long long gb0;     // Gated DeltaNet: index of the first token's g / beta; gbs apart
+    int gbs;
+    int tma_y, tma_z;  // tile coordinates of the sequence start (dims 1 and 2 of the maps)
     int* abort_flag;
     float* gamma_s;
     const CUtensorMap *tm_r, *tm_w, *tm_k, *tm_v, *tm_a, *tm_b;
@@ -276,38 +280,41 @@ struct Ctx {
 // starting at token c0 into layout `par` (lane 0 arms the barrier first; the
 // six copies are issued in parallel).  Gated DeltaNet loads three (q, k, v into the
 // r, k, v tiles).
-template <bool kGdn>
+template <bool kGdn, bool kHf>
 __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
     const LayR L = lay_of(par);
     using namespace sm100;
     const int lane = cx.lane;
     if (lane == 0) mbar_arrive_expect_tx(cx.bar_tma, (kGdn ? 3 : 6) * kTile);
     __syncwarp();
-    const int row = (int)(cx.row0 + c0);
+    // token-major maps are (channel, head, token row); head-first maps (channel, token,
+    // batch x head): the chunk start advances dimension 2 or dimension 1
+    const int cy = kHf ? cx.tma_y + c0 : cx.tma_y;
+    const int cz = kHf ? cx.tma_z : cx.tma_z + c0;
     if constexpr (kGdn) {
         if (lane < 3) {
             const CUtensorMap* map = lane == 0 ? cx.tm_r : lane == 1 ? cx.tm_k : cx.tm_v;
             const uint32_t dst = lane == 0 ? L.R : lane == 1 ? L.K : L.V;
-            tma_load_3d(cx.sbase + dst, map, cx.bar_tma, 0, cx.h, row);
+            tma_load_3d(cx.sbase + dst, map, cx.bar_tma, 0, cy, cz);
         }
     } else if (lane < 6) {
         const CUtensorMap* map = lane == 0 ? cx.tm_r : lane == 1 ? cx.tm_a : lane == 2 ? cx.tm_k
                                : lane == 3 ? cx.tm_b : lane == 4 ? cx.tm_w : cx.tm_v;
         const uint32_t dst = lane == 0 ? L.R : lane == 1 ? L.A : lane == 2 ? L.K
                            : lane == 3 ? L.B : lane == 4 ? L.W : L.V;
-        tma_load_3d(cx.sbase + dst, map, cx.bar_tma, 0, cx.h, row);
+        tma_load_3d(cx.sbase + dst, map, cx.bar_tma, 0, cy, cz);
     }
 }
 
 // One 64-token chunk starting at token c0, in layout P (its inputs already requested).
-template <bool kGdn>
+template <bool kGdn, bool kHf>
 __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
     const LayR L = lay_of(par);
     using namespace sm100;
     uint8_t* smem = cx.smem;
     const uint32_t sbase = cx.sbase, tmem = cx.tmem, bar_mma = cx.bar_mma;
     const int tid = cx.tid, warp = cx.warp, lane = cx.lane, wq = cx.wq, wh = cx.wh;
-    const int m_row = cx.m_row, H = cx.H, h = cx.h;
+    const int m_row = cx.m_row;
     const bool state_thread = cx.state_thread;
     const long long row0 = cx.row0;
     const uint8_t* mask = cx.mask;
@@ -321,14 +328,15 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
     float gq[2] = {0.f, 0.f}, bq[2] = {0.f, 0.f};  // Gated DeltaNet: g, beta of tokens t0, t0+1
     if constexpr (kGdn) {  // issued before the tile wait, so their latency overlaps it
         const int t0 = 2 * (tid >> 3);
-        const long long tok = (row0 + c0 + t0) * H + h;
+        const long long gbs = kHf ? 1 : cx.gbs;
+        const long long tok = cx.gb0 + (long long)(c0 + t0) * gbs;
         if (t0 < nv) {
             gq[0] = __bfloat162float(cx.g[tok]);
             bq[0] = __bfloat162float(cx.beta[tok]);
         }
         if (t0 + 1 < nv) {
-            gq[1] = __bfloat162float(cx.g[tok + H]);
-            bq[1] = __bfloat162float(cx.beta[tok + H]);
+            gq[1] = __bfloat162float(cx.g[tok + gbs]);
+            bq[1] = __bfloat162float(cx.beta[tok + gbs]);
         }
     }
     wait_or_abort(cx.bar_tma, par, abort_flag);
@@ -887,7 +895,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 
         // The next chunk's inputs go to the other layout's input tiles, all of which
         // are dead now; the copy overlaps this chunk's final MMA and epilogue.
-        if (has_next && warp == 1) issue_loads<kGdn>(cx, c0 + 64, par ^ 1);
+        if (has_next && warp == 1) issue_loads<kGdn, kHf>(cx, c0 + 64, par ^ 1);
 
         // ---- 9. final MMA: [S upd; O] = A_fin [S0; V]  (128 x 64 x 128, fp16) ------------
         if (tid == 0) {
@@ -922,7 +930,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             }
             const int t = m_row - 64;
             if (t < nv) {
-                uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(row0 + c0 + t) * H + h) * 64 + 32 * wh);
+                uint4* dst = reinterpret_cast<uint4*>(o + (c0 + t) * (kHf ? 64 : cx.o_ts) + 32 * wh);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) dst[c] = pack8(v + 8 * c);
             }
@@ -934,8 +942,9 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
 }
 
 // kGdn: Gated DeltaNet (tm_r, tm_k, tm_v map q, k, v; g and beta per token; s0 may be
-// one state per head shared by every sequence, s0_shared != 0).
-template <bool kGdn>
+// one state per head shared by every sequence, s0_shared != 0).  kHf (head first):
+// inputs, o (and g, beta) are [B, H, T, *] instead of [B, T, H, *]; the maps follow.
+template <bool kGdn, bool kHf>
 __global__ void __launch_bounds__(kThreads, 2)
 chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -999,13 +1008,26 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     cx.wq = wq;
     cx.wh = wh;
     cx.m_row = 32 * wq + lane;
-    cx.h = h;
-    cx.H = H;
     cx.state_thread = wq < 2;
     cx.row0 = (long long)bb * T + bos;
     cx.len = eos - bos;
     cx.mask = mask;
-    cx.o = o;
+    if (kHf) {
+        const long long u0 = ((long long)bb * H + h) * T + bos;  // [B, H, T] token index
+        cx.o = o + u0 * 64;
+        cx.o_ts = 64;
+        cx.gb0 = u0;
+        cx.gbs = 1;
+        cx.tma_y = bos;
+        cx.tma_z = bb * H + h;
+    } else {
+        cx.o = o + (cx.row0 * H + h) * 64;
+        cx.o_ts = (long long)H * 64;
+        cx.gb0 = cx.row0 * H + h;
+        cx.gbs = H;
+        cx.tma_y = h;
+        cx.tma_z = (int)cx.row0;
+    }
     cx.abort_flag = reinterpret_cast<int*>(smem + OFF_MISC + 20);
     cx.gamma_s = reinterpret_cast<float*>(smem + OFF_GAMMA);
     cx.tm_r = &tm_r;
@@ -1035,7 +1057,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     if (warp == 0 && lane < 6)
         prefetch_tensormap(lane == 0 ? &tm_r : lane == 1 ? &tm_a : lane == 2 ? &tm_k
                            : lane == 3 ? &tm_b : lane == 4 ? &tm_w : &tm_v);
-    if (warp == 0 && cx.len > 0) issue_loads<kGdn>(cx, 0, 0);
+    if (warp == 0 && cx.len > 0) issue_loads<kGdn, kHf>(cx, 0, 0);
 
     // The fp32 state lives in tensor memory, rows 0..63 of the final product's
     // columns: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
@@ -1072,7 +1094,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
 
     // Chunks alternate between the two shared-memory layouts.
     for (int c0 = 0, par = 0; c0 < cx.len; c0 += 64, par ^= 1) {
-        chunk<kGdn>(cx, c0, c0 + 64 < cx.len, par);
+        chunk<kGdn, kHf>(cx, c0, c0 + 64 < cx.len, par);
         if (*cx.abort_flag) break;
     }
 
@@ -1111,13 +1133,23 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, H, 64] bf16 tensor viewed as (64, H, rows); box = 64 tokens of one head.
-inline bool make_map(CUtensorMap* map, const void* ptr, long long rows, int H) {
+// [B*T, H, 64] bf16 tensor viewed as (64, H, B*T), box = 64 tokens of one head; or,
+// head first, [B*H, T, 64] viewed as (64, T, B*H), box = 64 tokens of one (b, h).  Both
+// boxes land as 64 rows of 128 bytes, token-major.
+inline bool make_map(CUtensorMap* map, const void* ptr, int B, int T, int H, int head_first) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[3] = {64, (cuuint64_t)H, (cuuint64_t)rows};
+    const cuuint64_t rows = (cuuint64_t)B * T;
+    cuuint64_t dims[3] = {64, (cuuint64_t)H, rows};
     cuuint64_t strides[2] = {64 * 2, (cuuint64_t)H * 64 * 2};
     cuuint32_t box[3] = {64, 1, 64};
+    if (head_first) {
+        dims[1] = (cuuint64_t)T;
+        dims[2] = (cuuint64_t)B * H;
+        strides[1] = (cuuint64_t)T * 64 * 2;
+        box[1] = 64;
+        box[2] = 1;
+    }
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1127,50 +1159,63 @@ inline bool make_map(CUtensorMap* map, const void* ptr, long long rows, int H) {
 }  // namespace chunked
 
 namespace chunked {
-template <bool kGdn>
-inline cudaError_t launch(const void* const* ptrs, int nmaps, const float* s0,
+template <bool kGdn, bool kHf>
+inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float* s0,
                           const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
                           const int32_t* cu_seqlens, const void* g, const void* beta,
                           int s0_shared, cudaStream_t stream) {
-    const long long rows = (long long)B * T;
     CUtensorMap maps[6];
     for (int i = 0; i < nmaps; ++i)
-        if (!make_map(&maps[i], ptrs[i], rows, H)) return cudaErrorInvalidValue;
+        if (!make_map(&maps[i], ptrs[i], B, T, H, kHf)) return cudaErrorInvalidValue;
     for (int i = nmaps; i < 6; ++i) maps[i] = maps[0];  // unused by the kernel
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn>,
+        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    chunked_kernel<kGdn><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
+    chunked_kernel<kGdn, kHf><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], s0, mask,
         static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens,
         static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(beta), s0_shared);
     return cudaGetLastError();
+}
+template <bool kGdn>
+inline cudaError_t launch(const void* const* ptrs, int nmaps, const float* s0,
+                          const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
+                          const int32_t* cu_seqlens, const void* g, const void* beta,
+                          int s0_shared, int head_first, cudaStream_t stream) {
+    return head_first
+               ? launch_layout<kGdn, true>(ptrs, nmaps, s0, mask, o, sT, B, T, H, N, cu_seqlens,
+                                           g, beta, s0_shared, stream)
+               : launch_layout<kGdn, false>(ptrs, nmaps, s0, mask, o, sT, B, T, H, N, cu_seqlens,
+                                            g, beta, s0_shared, stream);
 }
 }  // namespace chunked
 
 inline cudaError_t launch_chunked(const void* r, const void* w, const void* k, const void* v,
                                   const void* a, const void* b, const float* s0,
                                   const uint8_t* mask, void* o, float* sT, int B, int T, int H,
-                                  int N, const int32_t* cu_seqlens, cudaStream_t stream) {
+                                  int N, const int32_t* cu_seqlens, int head_first,
+                                  cudaStream_t stream) {
     const void* ptrs[6] = {r, w, k, v, a, b};
     return chunked::launch<false>(ptrs, 6, s0, mask, o, sT, B, T, H, N, cu_seqlens, nullptr,
-                                  nullptr, 0, stream);
+                                  nullptr, 0, head_first, stream);
 }
 
-// Gated DeltaNet: q, k, v [B*T, H, 64] bf16 through the r, k, v maps; g, beta [B*T, H].
+// Gated DeltaNet: q, k, v [B*T, H, 64] bf16 through the r, k, v maps; g, beta [B*T, H]
+// (head first: [B*H, T, 64] and [B*H, T]).
 inline cudaError_t launch_chunked_gdn(const void* q, const void* k, const void* v,
                                       const void* g, const void* beta, const float* s0,
                                       int s0_shared, void* o, float* sT, int B, int T, int H,
-                                      int N, const int32_t* cu_seqlens, cudaStream_t stream) {
+                                      int N, const int32_t* cu_seqlens, int head_first,
+                                      cudaStream_t stream) {
     // map order r, w, k, v: the unused w slot repeats q
     const void* ptrs[4] = {q, q, k, v};
     return chunked::launch<true>(ptrs, 4, s0, nullptr, o, sT, B, T, H, N, cu_seqlens, g, beta,
-                                 s0_shared, stream);
+                                 s0_shared, head_first, stream);
 }
 
 }  // namespace wkv7

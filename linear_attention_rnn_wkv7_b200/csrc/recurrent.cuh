@@ -3,11 +3,15 @@
 // The recurrence (rwkv-ops 0.9.0 README, "rwkv7op 使用方法"):
 //     u_t = S_{t-1}^T a_t;  S_t = diag(exp w_t) S_{t-1} + b_t u_t^T + k_t v_t^T;  o_t = S_t^T r_t
 // decouples over the V columns of the state: column j only needs u_t[j],
-// which is the dot product of column j with a_t.  So one thread owns one state
-// column (64 fp32 registers) and every reduction over K stays inside a thread;
-// a block of 64 threads owns one (sequence, head).  Tokens are staged 16 at a
-// time in shared memory (r, exp(w), k, a, b, v as fp32) so that each thread
-// reads the shared vectors as float4 broadcasts.
+// which is the dot product of column j with a_t.  So a block owns a slab of 64
+// state columns of one (sequence, head), and each column is held by P = K / 64
+// threads of adjacent lanes, 64 rows (64 fp32 registers) each: the reductions over
+// K are a thread's own sum plus log2(P) shuffles.  K = V = 64 is one block of 64
+// threads per (sequence, head); the README's other head sizes (128, 256) take
+// K / 64 column slabs of 64 x P threads, every slab reading the whole K-side vectors.
+// Tokens are staged 1024 / K at a time in shared memory (r, exp(w), k, a, b over K
+// and the slab's 64 entries of v, as fp32) so that each thread reads the shared
+// vectors as float4 broadcasts.
 //
 // This is the fp32-input path (its accuracy is that of an fp32 recurrence)
 // and the anchor the chunked tensor-core kernel is checked against; masks,
@@ -24,89 +28,102 @@
 
 namespace wkv7 {
 
-constexpr int kRecTile = 16;
-
-template <typename Tin, bool kGdn>
-__global__ void __launch_bounds__(64)
+// K (= V): head size.  Block: 64 columns x P = K / 64 threads per column.
+template <typename Tin, bool kGdn, int K>
+__global__ void __launch_bounds__(K)
 recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
                  const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
                  const float* s0, const uint8_t* __restrict__ mask, Tin* __restrict__ o,
                  float* sT, int T, int H, const int32_t* __restrict__ cu_seqlens,
-                 const Tin* __restrict__ g, const Tin* __restrict__ beta, int s0_shared) {
-    __shared__ __align__(16) float sm[6][kRecTile][64];  // r, d, k, a, b, v
-    __shared__ uint8_t smask[kRecTile];
-    __shared__ float sgb[4][kRecTile];  // Gated DeltaNet: g, beta, 1/|q|, 1/|k|
+                 const Tin* __restrict__ g, const Tin* __restrict__ beta, int s0_shared,
+                 int head_first) {
+    constexpr int P = K / 64;        // threads per state column
+    constexpr int kTile = 1024 / K;  // tokens per staging round
+    constexpr int kSlabs = K / 64;   // 64-column slabs per (sequence, head)
+    __shared__ __align__(16) float sm[5][kTile][K];  // r, d, k, a, b
+    __shared__ __align__(16) float sv[kTile][64];    // this slab's v
+    __shared__ uint8_t smask[kTile];
+    __shared__ float sgb[4][kTile];  // Gated DeltaNet: g, beta, 1/|q|, 1/|k|
 
-    const int h = blockIdx.x % H;
-    const int n = blockIdx.x / H;
-    const int j = threadIdx.x;
+    const int slab = blockIdx.x % kSlabs;
+    const int unit = blockIdx.x / kSlabs;
+    const int h = unit % H;
+    const int n = unit / H;
+    const int tid = threadIdx.x;
+    const int c = tid / P, part = tid % P;  // column of the slab, 64-row part of it
+    const int col = 64 * slab + c;          // state column
     int bb = n, bos = 0, eos = T;
     if (cu_seqlens) {
         bb = 0;
         bos = cu_seqlens[n];
         eos = cu_seqlens[n + 1];
         if (bos < 0 || eos < bos || eos > T) {  // block-uniform
-            if (j == 0) raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
+            if (tid == 0 && slab == 0) raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
             return;
         }
     }
-    const size_t state_off = ((size_t)n * H + h) * 4096;
-    const size_t init_off = s0_shared ? (size_t)h * 4096 : state_off;
+    // token t of this unit is row tb + t * ts of the [*, K] inputs and outputs (and
+    // element tb + t * ts of g and beta): [B, T, H, *] or, head first, [B, H, T, *]
+    const size_t tb = head_first ? ((size_t)bb * H + h) * T : (size_t)bb * T * H + h;
+    const size_t ts = head_first ? 1 : (size_t)H;
+    const size_t state_off = ((size_t)n * H + h) * K * K;
+    const size_t init_off = s0_shared ? (size_t)h * K * K : state_off;
 
-    float S[64];
+    float S[64];  // rows 64 part .. 64 part + 63 of column col
 #pragma unroll
-    for (int i = 0; i < 64; ++i) S[i] = s0 ? s0[init_off + i * 64 + j] : 0.f;
+    for (int i = 0; i < 64; ++i)
+        S[i] = s0 ? s0[init_off + (size_t)(64 * part + i) * K + col] : 0.f;
 
-    for (int t0 = bos; t0 < eos; t0 += kRecTile) {
-        const int cnt = min(kRecTile, eos - t0);
+    for (int t0 = bos; t0 < eos; t0 += kTile) {
+        const int cnt = min(kTile, eos - t0);
         __syncthreads();
         if constexpr (kGdn) {
             for (int tt = 0; tt < cnt; ++tt) {
-                const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
-                sm[0][tt][j] = to_f32(r[row + j]);  // q
-                sm[3][tt][j] = to_f32(k[row + j]);
-                sm[5][tt][j] = to_f32(v[row + j]);
+                const size_t row = (tb + (size_t)(t0 + tt) * ts) * K;
+                sm[0][tt][tid] = to_f32(r[row + tid]);  // q
+                sm[3][tt][tid] = to_f32(k[row + tid]);
+                if (tid < 64) sv[tt][tid] = to_f32(v[row + 64 * slab + tid]);
             }
-            if (j < cnt) {
-                const size_t tok = ((size_t)bb * T + t0 + j) * H + h;
-                sgb[0][j] = to_f32(g[tok]);
-                sgb[1][j] = to_f32(beta[tok]);
-                smask[j] = 1;
+            if (tid < cnt) {
+                const size_t tok = tb + (size_t)(t0 + tid) * ts;
+                sgb[0][tid] = to_f32(g[tok]);
+                sgb[1][tid] = to_f32(beta[tok]);
+                smask[tid] = 1;
             }
             __syncthreads();
-            if (j < 2 * cnt) {  // thread 2 tt + e: the inverse norm of q (e = 0) or k (e = 1)
-                const float* x = sm[(j & 1) ? 3 : 0][j >> 1];
+            if (tid < 2 * cnt) {  // thread 2 tt + e: the inverse norm of q (e = 0) or k (e = 1)
+                const float* x = sm[(tid & 1) ? 3 : 0][tid >> 1];
                 float ss = 0.f;
-                for (int i = 0; i < 64; ++i) ss = fmaf(x[i], x[i], ss);
-                sgb[2 + (j & 1)][j >> 1] = ss > 0.f ? rsqrtf(ss) : 0.f;  // zero stays zero
+                for (int i = 0; i < K; ++i) ss = fmaf(x[i], x[i], ss);
+                sgb[2 + (tid & 1)][tid >> 1] = ss > 0.f ? rsqrtf(ss) : 0.f;  // zero stays zero
             }
             __syncthreads();
             for (int tt = 0; tt < cnt; ++tt) {
-                const float kn = sm[3][tt][j] * sgb[3][tt];
+                const float kn = sm[3][tt][tid] * sgb[3][tt];
                 const float alpha = expf(sgb[0][tt]), bt = sgb[1][tt];
-                sm[0][tt][j] *= sgb[2][tt];
-                sm[1][tt][j] = alpha;
-                sm[2][tt][j] = bt * kn;
-                sm[3][tt][j] = kn;
-                sm[4][tt][j] = -alpha * bt * kn;
+                sm[0][tt][tid] *= sgb[2][tt];
+                sm[1][tt][tid] = alpha;
+                sm[2][tt][tid] = bt * kn;
+                sm[3][tt][tid] = kn;
+                sm[4][tt][tid] = -alpha * bt * kn;
             }
         } else {
             for (int tt = 0; tt < cnt; ++tt) {
-                const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
-                sm[0][tt][j] = to_f32(r[row + j]);
-                sm[1][tt][j] = expf(to_f32(w[row + j]));
-                sm[2][tt][j] = to_f32(k[row + j]);
-                sm[3][tt][j] = to_f32(a[row + j]);
-                sm[4][tt][j] = to_f32(b[row + j]);
-                sm[5][tt][j] = to_f32(v[row + j]);
+                const size_t row = (tb + (size_t)(t0 + tt) * ts) * K;
+                sm[0][tt][tid] = to_f32(r[row + tid]);
+                sm[1][tt][tid] = expf(to_f32(w[row + tid]));
+                sm[2][tt][tid] = to_f32(k[row + tid]);
+                sm[3][tt][tid] = to_f32(a[row + tid]);
+                sm[4][tt][tid] = to_f32(b[row + tid]);
+                if (tid < 64) sv[tt][tid] = to_f32(v[row + 64 * slab + tid]);
             }
-            if (j < cnt) smask[j] = mask ? (mask[(size_t)bb * T + t0 + j] != 0) : 1;
+            if (tid < cnt) smask[tid] = mask ? (mask[(size_t)bb * T + t0 + tid] != 0) : 1;
         }
         __syncthreads();
 
         for (int tt = 0; tt < cnt; ++tt) {
             if (smask[tt]) {
-                const float4* a4 = reinterpret_cast<const float4*>(sm[3][tt]);
+                const float4* a4 = reinterpret_cast<const float4*>(sm[3][tt] + 64 * part);
                 float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
 #pragma unroll
                 for (int i4 = 0; i4 < 16; ++i4) {
@@ -116,11 +133,13 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
                     u2 = fmaf(S[4 * i4 + 2], av.z, u2);
                     u3 = fmaf(S[4 * i4 + 3], av.w, u3);
                 }
-                const float u = (u0 + u1) + (u2 + u3);
-                const float vj = sm[5][tt][j];
-                const float4* d4 = reinterpret_cast<const float4*>(sm[1][tt]);
-                const float4* k4 = reinterpret_cast<const float4*>(sm[2][tt]);
-                const float4* b4 = reinterpret_cast<const float4*>(sm[4][tt]);
+                float u = (u0 + u1) + (u2 + u3);
+#pragma unroll
+                for (int m = 1; m < P; m *= 2) u += __shfl_xor_sync(0xffffffffu, u, m);
+                const float vj = sv[tt][c];
+                const float4* d4 = reinterpret_cast<const float4*>(sm[1][tt] + 64 * part);
+                const float4* k4 = reinterpret_cast<const float4*>(sm[2][tt] + 64 * part);
+                const float4* b4 = reinterpret_cast<const float4*>(sm[4][tt] + 64 * part);
 #pragma unroll
                 for (int i4 = 0; i4 < 16; ++i4) {
                     const float4 dv = d4[i4], kv = k4[i4], bv = b4[i4];
@@ -130,7 +149,7 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
                     S[4 * i4 + 3] = fmaf(S[4 * i4 + 3], dv.w, fmaf(bv.w, u, kv.w * vj));
                 }
             }
-            const float4* r4 = reinterpret_cast<const float4*>(sm[0][tt]);
+            const float4* r4 = reinterpret_cast<const float4*>(sm[0][tt] + 64 * part);
             float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
 #pragma unroll
             for (int i4 = 0; i4 < 16; ++i4) {
@@ -140,41 +159,79 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
                 o2 = fmaf(S[4 * i4 + 2], rv.z, o2);
                 o3 = fmaf(S[4 * i4 + 3], rv.w, o3);
             }
-            const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
-            o[row + j] = from_f32<Tin>((o0 + o1) + (o2 + o3));
+            float ov = (o0 + o1) + (o2 + o3);
+#pragma unroll
+            for (int m = 1; m < P; m *= 2) ov += __shfl_xor_sync(0xffffffffu, ov, m);
+            if (part == 0) {
+                const size_t row = (tb + (size_t)(t0 + tt) * ts) * K;
+                o[row + col] = from_f32<Tin>(ov);
+            }
         }
     }
     if (sT) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) sT[state_off + i * 64 + j] = S[i];
+        for (int i = 0; i < 64; ++i) sT[state_off + (size_t)(64 * part + i) * K + col] = S[i];
     }
 }
 
+template <typename Tin, bool kGdn, int K>
+cudaError_t launch_recurrent_k(const void* r, const void* w, const void* k, const void* v,
+                               const void* a, const void* b, const float* s0,
+                               const uint8_t* mask, void* o, float* sT, int T, int H, int N,
+                               const int32_t* cu_seqlens, const void* g, const void* beta,
+                               int s0_shared, int head_first, cudaStream_t stream) {
+    const long long blocks = (long long)N * H * (K / 64);
+    recurrent_kernel<Tin, kGdn, K><<<(unsigned)blocks, K, 0, stream>>>(
+        static_cast<const Tin*>(r), static_cast<const Tin*>(w), static_cast<const Tin*>(k),
+        static_cast<const Tin*>(v), static_cast<const Tin*>(a), static_cast<const Tin*>(b), s0,
+        mask, static_cast<Tin*>(o), sT, T, H, cu_seqlens, static_cast<const Tin*>(g),
+        static_cast<const Tin*>(beta), s0_shared, head_first);
+    return cudaGetLastError();
+}
+
+template <typename Tin, bool kGdn>
+cudaError_t launch_recurrent_any(int K, const void* r, const void* w, const void* k,
+                                 const void* v, const void* a, const void* b, const float* s0,
+                                 const uint8_t* mask, void* o, float* sT, int T, int H, int N,
+                                 const int32_t* cu_seqlens, const void* g, const void* beta,
+                                 int s0_shared, int head_first, cudaStream_t stream) {
+    switch (K) {
+        case 64:
+            return launch_recurrent_k<Tin, kGdn, 64>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
+                                                     cu_seqlens, g, beta, s0_shared, head_first,
+                                                     stream);
+        case 128:
+            return launch_recurrent_k<Tin, kGdn, 128>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
+                                                      cu_seqlens, g, beta, s0_shared, head_first,
+                                                      stream);
+        case 256:
+            return launch_recurrent_k<Tin, kGdn, 256>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
+                                                      cu_seqlens, g, beta, s0_shared, head_first,
+                                                      stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// WKV7: r, w, k, a, b [rows, H, K], v and o [rows, H, K] (K = V in {64, 128, 256}).
 template <typename Tin>
 cudaError_t launch_recurrent(const void* r, const void* w, const void* k, const void* v,
                              const void* a, const void* b, const float* s0,
                              const uint8_t* mask, void* o, float* sT, int T, int H, int N,
-                             const int32_t* cu_seqlens, cudaStream_t stream) {
-    const long long blocks = (long long)N * H;
-    recurrent_kernel<Tin, false><<<(unsigned)blocks, 64, 0, stream>>>(
-        static_cast<const Tin*>(r), static_cast<const Tin*>(w), static_cast<const Tin*>(k),
-        static_cast<const Tin*>(v), static_cast<const Tin*>(a), static_cast<const Tin*>(b), s0,
-        mask, static_cast<Tin*>(o), sT, T, H, cu_seqlens, nullptr, nullptr, 0);
-    return cudaGetLastError();
+                             const int32_t* cu_seqlens, int head_first, int K,
+                             cudaStream_t stream) {
+    return launch_recurrent_any<Tin, false>(K, r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
+                                            cu_seqlens, nullptr, nullptr, 0, head_first, stream);
 }
 
-// Gated DeltaNet: q, k [rows, H, 64], v [rows, H, 64], g, beta [rows, H].
+// Gated DeltaNet: q, k [rows, H, K], v [rows, H, K], g, beta [rows, H].
 template <typename Tin>
 cudaError_t launch_recurrent_gdn(const void* q, const void* k, const void* v, const void* g,
                                  const void* beta, const float* s0, int s0_shared, void* o,
                                  float* sT, int T, int H, int N, const int32_t* cu_seqlens,
-                                 cudaStream_t stream) {
-    const long long blocks = (long long)N * H;
-    recurrent_kernel<Tin, true><<<(unsigned)blocks, 64, 0, stream>>>(
-        static_cast<const Tin*>(q), nullptr, static_cast<const Tin*>(k),
-        static_cast<const Tin*>(v), nullptr, nullptr, s0, nullptr, static_cast<Tin*>(o), sT, T,
-        H, cu_seqlens, static_cast<const Tin*>(g), static_cast<const Tin*>(beta), s0_shared);
-    return cudaGetLastError();
+                                 int head_first, int K, cudaStream_t stream) {
+    return launch_recurrent_any<Tin, true>(K, q, nullptr, k, v, nullptr, nullptr, s0, nullptr,
+                                           o, sT, T, H, N, cu_seqlens, g, beta, s0_shared,
+                                           head_first, stream);
 }
 
 }  // namespace wkv7

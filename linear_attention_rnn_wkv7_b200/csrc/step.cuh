@@ -20,6 +20,11 @@
 // write key beta kh, a = kh, b = -e^{g} beta kh (qh, kh: q and k over their L2
 // norms, reduced across the warp), so the same update applies
 // e^{g} (I - beta kh kh^T) S + beta kh v^T.
+//
+// Head sizes 128 and 256 (step_kernel_wide): one block per (unit, 64-column slab)
+// with K / 64 warps, warp p holding rows 64 p .. 64 p + 63 of the slab in the same
+// lane layout as above; the K-reductions of u and o add the warps' partial sums
+// through shared memory (two block barriers per step).
 #pragma once
 #include "common.cuh"
 
@@ -143,29 +148,191 @@ step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
     if (p == 0) store4(o + voff + 4 * c, acc);
 }
 
-template <typename Tin>
-cudaError_t launch_step(const void* r, const void* w, const void* k, const void* v,
-                        const void* a, const void* b, float* state, void* o, long long units,
-                        cudaStream_t stream) {
-    const long long blocks = (units + kStepWarps - 1) / kStepWarps;
-    step_kernel<Tin, false><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
-        static_cast<const Tin*>(r), static_cast<const Tin*>(w), static_cast<const Tin*>(k),
-        static_cast<const Tin*>(v), static_cast<const Tin*>(a), static_cast<const Tin*>(b),
-        state, static_cast<Tin*>(o), units, nullptr, nullptr);
+// K = V in {128, 256}: block = K / 64 warps on one 64-column slab of one unit.
+template <typename Tin, bool kGdn, int K>
+__global__ void __launch_bounds__(32 * (K / 64))
+step_kernel_wide(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
+                 const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
+                 float* __restrict__ state, Tin* __restrict__ o, const Tin* __restrict__ g,
+                 const Tin* __restrict__ beta) {
+    constexpr int P = K / 64;  // warps = row parts = column slabs per unit
+    __shared__ __align__(16) float vec[5][K];  // r, d = exp(w), k, a, b
+    __shared__ __align__(16) float part_u[P][64];
+    __shared__ __align__(16) float part_o[P][64];
+    __shared__ float nrm[2][P];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;  // row part
+    const long long unit = blockIdx.x / P;
+    const int slab = blockIdx.x % P;
+    const size_t voff = (size_t)unit * K;
+    float* Su = state + (size_t)unit * K * K;
+    const int c = lane & 15;  // float4 column group of the slab
+    const int ph = lane >> 4; // row half of the part
+    const int row0 = 64 * warp + 32 * ph;
+    const int col0 = 64 * slab + 4 * c;
+
+    float4 S[32];
+#pragma unroll
+    for (int m = 0; m < 32; ++m)
+        S[m] = *reinterpret_cast<const float4*>(Su + (size_t)(row0 + m) * K + col0);
+
+    const int e0 = 64 * warp + 2 * lane;  // this lane's two vector entries
+    if constexpr (kGdn) {
+        const float2 qq = load2(r + voff + e0);
+        const float2 kk = load2(k + voff + e0);
+        float sq = qq.x * qq.x + qq.y * qq.y, sk = kk.x * kk.x + kk.y * kk.y;
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, m);
+            sk += __shfl_xor_sync(0xffffffffu, sk, m);
+        }
+        if (lane == 0) {
+            nrm[0][warp] = sq;
+            nrm[1][warp] = sk;
+        }
+        __syncthreads();
+        sq = 0.f;
+        sk = 0.f;
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            sq += nrm[0][p];
+            sk += nrm[1][p];
+        }
+        const float nq = sq > 0.f ? rsqrtf(sq) : 0.f, nk = sk > 0.f ? rsqrtf(sk) : 0.f;
+        const float alpha = expf(to_f32(g[unit])), bt = to_f32(beta[unit]);
+        const float2 kn = make_float2(kk.x * nk, kk.y * nk);
+        *reinterpret_cast<float2*>(&vec[0][e0]) = make_float2(qq.x * nq, qq.y * nq);
+        *reinterpret_cast<float2*>(&vec[1][e0]) = make_float2(alpha, alpha);
+        *reinterpret_cast<float2*>(&vec[2][e0]) = make_float2(bt * kn.x, bt * kn.y);
+        *reinterpret_cast<float2*>(&vec[3][e0]) = kn;
+        *reinterpret_cast<float2*>(&vec[4][e0]) = make_float2(-alpha * bt * kn.x, -alpha * bt * kn.y);
+    } else {
+        const float2 ww = load2(w + voff + e0);
+        *reinterpret_cast<float2*>(&vec[0][e0]) = load2(r + voff + e0);
+        *reinterpret_cast<float2*>(&vec[1][e0]) = make_float2(expf(ww.x), expf(ww.y));
+        *reinterpret_cast<float2*>(&vec[2][e0]) = load2(k + voff + e0);
+        *reinterpret_cast<float2*>(&vec[3][e0]) = load2(a + voff + e0);
+        *reinterpret_cast<float2*>(&vec[4][e0]) = load2(b + voff + e0);
+    }
+    const float4 vcol = load4(v + voff + col0);
+    __syncwarp();  // a warp reads only the rows its own lanes wrote
+
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m4 = 0; m4 < 8; ++m4) {
+        const float4 a4 = reinterpret_cast<const float4*>(&vec[3][row0])[m4];
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 s = S[4 * m4 + q];
+            u.x = fmaf(s.x, av[q], u.x);
+            u.y = fmaf(s.y, av[q], u.y);
+            u.z = fmaf(s.z, av[q], u.z);
+            u.w = fmaf(s.w, av[q], u.w);
+        }
+    }
+    u.x += __shfl_xor_sync(0xffffffffu, u.x, 16);
+    u.y += __shfl_xor_sync(0xffffffffu, u.y, 16);
+    u.z += __shfl_xor_sync(0xffffffffu, u.z, 16);
+    u.w += __shfl_xor_sync(0xffffffffu, u.w, 16);
+    if (ph == 0) *reinterpret_cast<float4*>(&part_u[warp][4 * c]) = u;
+    __syncthreads();
+    u = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const float4 x = *reinterpret_cast<const float4*>(&part_u[p][4 * c]);
+        u.x += x.x;
+        u.y += x.y;
+        u.z += x.z;
+        u.w += x.w;
+    }
+
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m4 = 0; m4 < 8; ++m4) {
+        const float4 d4 = reinterpret_cast<const float4*>(&vec[1][row0])[m4];
+        const float4 k4 = reinterpret_cast<const float4*>(&vec[2][row0])[m4];
+        const float4 b4 = reinterpret_cast<const float4*>(&vec[4][row0])[m4];
+        const float4 r4 = reinterpret_cast<const float4*>(&vec[0][row0])[m4];
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+        const float rv[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float4 s = S[4 * m4 + q];
+            s.x = fmaf(s.x, dv[q], fmaf(bv[q], u.x, kv[q] * vcol.x));
+            s.y = fmaf(s.y, dv[q], fmaf(bv[q], u.y, kv[q] * vcol.y));
+            s.z = fmaf(s.z, dv[q], fmaf(bv[q], u.z, kv[q] * vcol.z));
+            s.w = fmaf(s.w, dv[q], fmaf(bv[q], u.w, kv[q] * vcol.w));
+            acc.x = fmaf(s.x, rv[q], acc.x);
+            acc.y = fmaf(s.y, rv[q], acc.y);
+            acc.z = fmaf(s.z, rv[q], acc.z);
+            acc.w = fmaf(s.w, rv[q], acc.w);
+            *reinterpret_cast<float4*>(Su + (size_t)(row0 + 4 * m4 + q) * K + col0) = s;
+        }
+    }
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+    if (ph == 0) *reinterpret_cast<float4*>(&part_o[warp][4 * c]) = acc;
+    __syncthreads();
+    if (warp == 0 && ph == 0) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            const float4 y = *reinterpret_cast<const float4*>(&part_o[p][4 * c]);
+            x.x += y.x;
+            x.y += y.y;
+            x.z += y.z;
+            x.w += y.w;
+        }
+        store4(o + voff + col0, x);
+    }
+}
+
+template <typename Tin, bool kGdn>
+cudaError_t launch_step_any(int K, const void* r, const void* w, const void* k, const void* v,
+                            const void* a, const void* b, float* state, void* o, long long units,
+                            const void* g, const void* beta, cudaStream_t stream) {
+    const Tin *r_ = static_cast<const Tin*>(r), *w_ = static_cast<const Tin*>(w),
+              *k_ = static_cast<const Tin*>(k), *v_ = static_cast<const Tin*>(v),
+              *a_ = static_cast<const Tin*>(a), *b_ = static_cast<const Tin*>(b),
+              *g_ = static_cast<const Tin*>(g), *be_ = static_cast<const Tin*>(beta);
+    Tin* o_ = static_cast<Tin*>(o);
+    if (K == 64) {
+        const long long blocks = (units + kStepWarps - 1) / kStepWarps;
+        step_kernel<Tin, kGdn><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
+            r_, w_, k_, v_, a_, b_, state, o_, units, g_, be_);
+    } else if (K == 128) {
+        step_kernel_wide<Tin, kGdn, 128><<<(unsigned)(units * 2), 64, 0, stream>>>(
+            r_, w_, k_, v_, a_, b_, state, o_, g_, be_);
+    } else if (K == 256) {
+        step_kernel_wide<Tin, kGdn, 256><<<(unsigned)(units * 4), 128, 0, stream>>>(
+            r_, w_, k_, v_, a_, b_, state, o_, g_, be_);
+    } else {
+        return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 
-// Gated DeltaNet step: q, k [units, 64], v [units, 64], g, beta [units].
+// WKV7 step: r, w, k, a, b, v, o [units, K]; state [units, K, K] (K in {64, 128, 256}).
+template <typename Tin>
+cudaError_t launch_step(const void* r, const void* w, const void* k, const void* v,
+                        const void* a, const void* b, float* state, void* o, long long units,
+                        int K, cudaStream_t stream) {
+    return launch_step_any<Tin, false>(K, r, w, k, v, a, b, state, o, units, nullptr, nullptr,
+                                       stream);
+}
+
+// Gated DeltaNet step: q, k, v, o [units, K], g, beta [units].
 template <typename Tin>
 cudaError_t launch_step_gdn(const void* q, const void* k, const void* v, const void* g,
-                            const void* beta, float* state, void* o, long long units,
+                            const void* beta, float* state, void* o, long long units, int K,
                             cudaStream_t stream) {
-    const long long blocks = (units + kStepWarps - 1) / kStepWarps;
-    step_kernel<Tin, true><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
-        static_cast<const Tin*>(q), nullptr, static_cast<const Tin*>(k),
-        static_cast<const Tin*>(v), nullptr, nullptr, state, static_cast<Tin*>(o), units,
-        static_cast<const Tin*>(g), static_cast<const Tin*>(beta));
-    return cudaGetLastError();
+    return launch_step_any<Tin, true>(K, q, nullptr, k, v, nullptr, nullptr, state, o, units, g,
+                                      beta, stream);
 }
 
 }  // namespace wkv7

@@ -17,6 +17,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 
+// Head sizes with a kernel: K == V in {64, 128, 256} (the chunked form: 64 only).
+inline bool head_size_ok(int K, int V) { return K == V && (K == 64 || K == 128 || K == 256); }
+
 // Non-null and aligned to its element (g, beta are read one element at a time).
 inline bool ok_scalar_ptr(const void* p, wkv7_dtype dtype) {
     const uintptr_t m = dtype == WKV7_BF16 ? 1u : 3u;
@@ -44,9 +47,10 @@ int wkv7_version(void) { return kVersion; }
 wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
                      const void* a, const void* b, const float* s0, const uint8_t* mask,
                      void* o, float* sT, int B, int T, int H, int K, int V,
-                     const int32_t* cu_seqlens, int N, wkv7_dtype dtype, wkv7_algo algo,
-                     void* stream_) {
+                     const int32_t* cu_seqlens, int N, wkv7_layout layout, wkv7_dtype dtype,
+                     wkv7_algo algo, void* stream_) {
     if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0 || N < 0) return WKV7_ERR_INVALID_ARG;
+    if (layout != WKV7_LAYOUT_BTHK && layout != WKV7_LAYOUT_BHTK) return WKV7_ERR_INVALID_ARG;
     if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
     if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_RECURRENT && algo != WKV7_ALGO_CHUNKED)
         return WKV7_ERR_INVALID_ARG;
@@ -56,10 +60,11 @@ wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
     } else if (N != B) {
         return WKV7_ERR_INVALID_ARG;
     }
-    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    if (!head_size_ok(K, V)) return WKV7_ERR_UNSUPPORTED;
     const long long units = (long long)N * H;
     const long long rows = (long long)B * T * H;
-    if (units > 0x7fffffffLL || rows > (1LL << 40)) return WKV7_ERR_UNSUPPORTED;
+    if (units * (K / 64) > 0x7fffffffLL || rows > (1LL << 40) || (long long)B * T > 0x7fffffffLL)
+        return WKV7_ERR_UNSUPPORTED;
     const bool tokens = rows > 0;
     if (tokens && (!ok_ptr(r) || !ok_ptr(w) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(a) ||
                    !ok_ptr(b) || !ok_ptr(o)))
@@ -70,20 +75,22 @@ wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
     if (units == 0) return WKV7_OK;
 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const int hf = layout == WKV7_LAYOUT_BHTK;
     // T == 0 (nothing but the state copy) always takes the recurrent kernel.
     const bool chunked = rows > 0 && (algo == WKV7_ALGO_CHUNKED ||
-                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && wkv7::kChunkedBuilt));
+                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && K == 64 &&
+                          wkv7::kChunkedBuilt));
     cudaError_t err;
     if (chunked) {
-        if (dtype != WKV7_BF16 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
+        if (dtype != WKV7_BF16 || K != 64 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
         err = wkv7::launch_chunked(r, w, k, v, a, b, s0, mask, o, sT, B, T, H, N, cu_seqlens,
-                                   stream);
+                                   hf, stream);
     } else if (dtype == WKV7_BF16) {
         err = wkv7::launch_recurrent<__nv_bfloat16>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
-                                                    cu_seqlens, stream);
+                                                    cu_seqlens, hf, K, stream);
     } else {
         err = wkv7::launch_recurrent<float>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
-                                            cu_seqlens, stream);
+                                            cu_seqlens, hf, K, stream);
     }
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
@@ -93,10 +100,10 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
                       int K, int V, wkv7_dtype dtype, void* stream_) {
     if (B < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
     if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
-    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    if (!head_size_ok(K, V)) return WKV7_ERR_UNSUPPORTED;
     const long long units = (long long)B * H;
     if (units == 0) return WKV7_OK;
-    if (units > (1LL << 33)) return WKV7_ERR_UNSUPPORTED;
+    if (units > (1LL << 33) || units * (K / 64) > 0x7fffffffLL) return WKV7_ERR_UNSUPPORTED;
     if (!ok_ptr(r) || !ok_ptr(w) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(a) || !ok_ptr(b) ||
         !ok_ptr(state) || !ok_ptr(o))
         return WKV7_ERR_INVALID_ARG;
@@ -105,16 +112,17 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const cudaError_t err =
         dtype == WKV7_BF16
-            ? wkv7::launch_step<__nv_bfloat16>(r, w, k, v, a, b, state, o, units, stream)
-            : wkv7::launch_step<float>(r, w, k, v, a, b, state, o, units, stream);
+            ? wkv7::launch_step<__nv_bfloat16>(r, w, k, v, a, b, state, o, units, K, stream)
+            : wkv7::launch_step<float>(r, w, k, v, a, b, state, o, units, K, stream);
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 
 wkv7_status wkv7_gdn_fwd(const void* q, const void* k, const void* v, const void* g,
                          const void* beta, const float* s0, int s0_shared, void* o, float* sT,
                          int B, int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
-                         wkv7_dtype dtype, wkv7_algo algo, void* stream_) {
+                         wkv7_layout layout, wkv7_dtype dtype, wkv7_algo algo, void* stream_) {
     if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0 || N < 0) return WKV7_ERR_INVALID_ARG;
+    if (layout != WKV7_LAYOUT_BTHK && layout != WKV7_LAYOUT_BHTK) return WKV7_ERR_INVALID_ARG;
     if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
     if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_RECURRENT && algo != WKV7_ALGO_CHUNKED)
         return WKV7_ERR_INVALID_ARG;
@@ -125,10 +133,11 @@ wkv7_status wkv7_gdn_fwd(const void* q, const void* k, const void* v, const void
     } else if (N != B) {
         return WKV7_ERR_INVALID_ARG;
     }
-    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    if (!head_size_ok(K, V)) return WKV7_ERR_UNSUPPORTED;
     const long long units = (long long)N * H;
     const long long rows = (long long)B * T * H;
-    if (units > 0x7fffffffLL || rows > (1LL << 40)) return WKV7_ERR_UNSUPPORTED;
+    if (units * (K / 64) > 0x7fffffffLL || rows > (1LL << 40) || (long long)B * T > 0x7fffffffLL)
+        return WKV7_ERR_UNSUPPORTED;
     const bool tokens = rows > 0;
     if (tokens && (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) ||
                    !ok_scalar_ptr(g, dtype) || !ok_scalar_ptr(beta, dtype)))
@@ -141,19 +150,21 @@ wkv7_status wkv7_gdn_fwd(const void* q, const void* k, const void* v, const void
     if (!s0) s0_shared = 0;
 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const int hf = layout == WKV7_LAYOUT_BHTK;
     const bool chunked = rows > 0 && (algo == WKV7_ALGO_CHUNKED ||
-                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && wkv7::kChunkedBuilt));
+                         (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16 && K == 64 &&
+                          wkv7::kChunkedBuilt));
     cudaError_t err;
     if (chunked) {
-        if (dtype != WKV7_BF16 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
+        if (dtype != WKV7_BF16 || K != 64 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
         err = wkv7::launch_chunked_gdn(q, k, v, g, beta, s0, s0_shared, o, sT, B, T, H, N,
-                                       cu_seqlens, stream);
+                                       cu_seqlens, hf, stream);
     } else if (dtype == WKV7_BF16) {
         err = wkv7::launch_recurrent_gdn<__nv_bfloat16>(q, k, v, g, beta, s0, s0_shared, o, sT,
-                                                        T, H, N, cu_seqlens, stream);
+                                                        T, H, N, cu_seqlens, hf, K, stream);
     } else {
         err = wkv7::launch_recurrent_gdn<float>(q, k, v, g, beta, s0, s0_shared, o, sT, T, H,
-                                                N, cu_seqlens, stream);
+                                                N, cu_seqlens, hf, K, stream);
     }
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
@@ -163,10 +174,10 @@ wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const voi
                           wkv7_dtype dtype, void* stream_) {
     if (B < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
     if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
-    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    if (!head_size_ok(K, V)) return WKV7_ERR_UNSUPPORTED;
     const long long units = (long long)B * H;
     if (units == 0) return WKV7_OK;
-    if (units > (1LL << 33)) return WKV7_ERR_UNSUPPORTED;
+    if (units > (1LL << 33) || units * (K / 64) > 0x7fffffffLL) return WKV7_ERR_UNSUPPORTED;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(state) || !ok_ptr(o) ||
         !ok_scalar_ptr(g, dtype) || !ok_scalar_ptr(beta, dtype))
         return WKV7_ERR_INVALID_ARG;
@@ -175,8 +186,8 @@ wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const voi
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const cudaError_t err =
         dtype == WKV7_BF16
-            ? wkv7::launch_step_gdn<__nv_bfloat16>(q, k, v, g, beta, state, o, units, stream)
-            : wkv7::launch_step_gdn<float>(q, k, v, g, beta, state, o, units, stream);
+            ? wkv7::launch_step_gdn<__nv_bfloat16>(q, k, v, g, beta, state, o, units, K, stream)
+            : wkv7::launch_step_gdn<float>(q, k, v, g, beta, state, o, units, K, stream);
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 

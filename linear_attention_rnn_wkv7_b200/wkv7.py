@@ -46,11 +46,11 @@ def library() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         p, i = ctypes.c_void_p, ctypes.c_int
         lib.wkv7_fwd.restype = i
-        lib.wkv7_fwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i, i, i, i, i, p, i, i, i, p]
+        lib.wkv7_fwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i, i, i, i, i, p, i, i, i, i, p]
         lib.wkv7_step.restype = i
         lib.wkv7_step.argtypes = [p, p, p, p, p, p, p, p, i, i, i, i, i, p]
         lib.wkv7_gdn_fwd.restype = i
-        lib.wkv7_gdn_fwd.argtypes = [p, p, p, p, p, p, i, p, p, i, i, i, i, i, p, i, i, i, p]
+        lib.wkv7_gdn_fwd.argtypes = [p, p, p, p, p, p, i, p, p, i, i, i, i, i, p, i, i, i, i, p]
         lib.wkv7_gdn_step.restype = i
         lib.wkv7_gdn_step.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, p]
         lib.wkv7_get_last_error.restype = i
@@ -97,17 +97,24 @@ def _stream(device) -> ctypes.c_void_p:
 
 
 def wkv7_fwd(r, w, k, v, a, b, s0=None, mask=None, cu_seqlens=None,
-             output_final_state: bool = True, algo: str = "auto", o=None, sT=None):
-    """WKV7 forward.  r,w,k,a,b [B,T,H,K]; v [B,T,H,V] (bf16 or fp32, all alike);
-    s0 [N,H,K,V] fp32 or None; mask [B,T] uint8/bool or None; cu_seqlens [N+1]
-    int32 (B must be 1) or None.  Returns (o [B,T,H,V], sT [N,H,K,V] or None)."""
+             output_final_state: bool = True, algo: str = "auto", o=None, sT=None,
+             head_first: bool = False):
+    """WKV7 forward.  r,w,k,a,b [B,T,H,K]; v [B,T,H,V] (bf16 or fp32, all alike), or
+    [B,H,T,*] with head_first; s0 [N,H,K,V] fp32 or None; mask [B,T] uint8/bool or
+    None; cu_seqlens [N+1] int32 (B must be 1) or None.
+    Returns (o shaped like v, sT [N,H,K,V] or None)."""
     _check(r, "r")
     dt = r.dtype
-    B, T, H, K = r.shape
+    if head_first:
+        B, H, T, K = r.shape
+    else:
+        B, T, H, K = r.shape
     V = v.shape[-1]
+    kshape = (B, H, T, K) if head_first else (B, T, H, K)
+    vshape = (B, H, T, V) if head_first else (B, T, H, V)
     for name, t in (("w", w), ("k", k), ("a", a), ("b", b)):
-        _check(t, name, dt, (B, T, H, K))
-    _check(v, "v", dt, (B, T, H, V))
+        _check(t, name, dt, kshape)
+    _check(v, "v", dt, vshape)
     if cu_seqlens is not None:
         _check(cu_seqlens, "cu_seqlens", torch.int32)
         N = cu_seqlens.numel() - 1
@@ -120,16 +127,16 @@ def wkv7_fwd(r, w, k, v, a, b, s0=None, mask=None, cu_seqlens=None,
             mask = mask.to(torch.uint8)
         _check(mask, "mask", torch.uint8, (B, T))
     if o is None:
-        o = torch.empty((B, T, H, V), dtype=dt, device=r.device)
+        o = torch.empty(vshape, dtype=dt, device=r.device)
     else:
-        _check(o, "o", dt, (B, T, H, V))
+        _check(o, "o", dt, vshape)
     if output_final_state and sT is None:
         sT = torch.empty((N, H, K, V), dtype=torch.float32, device=r.device)
     elif sT is not None:
         _check(sT, "sT", torch.float32, (N, H, K, V))
     st = library().wkv7_fwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0),
                             _ptr(mask), _ptr(o), _ptr(sT), B, T, H, K, V, _ptr(cu_seqlens), N,
-                            _dtype_code(r), ALGO[algo], _stream(r.device))
+                            int(bool(head_first)), _dtype_code(r), ALGO[algo], _stream(r.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_fwd")
     return o, sT
@@ -158,18 +165,24 @@ def wkv7_step(r, w, k, v, a, b, state, o=None):
 
 
 def wkv7_gdn_fwd(q, k, v, g, beta, s0=None, cu_seqlens=None, output_final_state: bool = True,
-                 algo: str = "auto", o=None, sT=None):
+                 algo: str = "auto", o=None, sT=None, head_first: bool = False):
     """Gated DeltaNet forward.  q, k [B,T,H,K]; v [B,T,H,V]; g, beta [B,T,H] (bf16 or
-    fp32, all alike); s0 [N,H,K,V] or [1,H,K,V] (shared) fp32 or None; cu_seqlens
-    [N+1] int32 (B must be 1) or None.  Returns (o [B,T,H,V], sT [N,H,K,V] or None)."""
+    fp32, all alike), or [B,H,T,*] / [B,H,T] with head_first; s0 [N,H,K,V] or
+    [1,H,K,V] (shared) fp32 or None; cu_seqlens [N+1] int32 (B must be 1) or None.
+    Returns (o shaped like v, sT [N,H,K,V] or None)."""
     _check(q, "q")
     dt = q.dtype
-    B, T, H, K = q.shape
+    if head_first:
+        B, H, T, K = q.shape
+    else:
+        B, T, H, K = q.shape
     V = v.shape[-1]
-    _check(k, "k", dt, (B, T, H, K))
-    _check(v, "v", dt, (B, T, H, V))
-    _check(g, "g", dt, (B, T, H))
-    _check(beta, "beta", dt, (B, T, H))
+    kshape = (B, H, T, K) if head_first else (B, T, H, K)
+    vshape = (B, H, T, V) if head_first else (B, T, H, V)
+    _check(k, "k", dt, kshape)
+    _check(v, "v", dt, vshape)
+    _check(g, "g", dt, kshape[:3])
+    _check(beta, "beta", dt, kshape[:3])
     if cu_seqlens is not None:
         _check(cu_seqlens, "cu_seqlens", torch.int32)
         N = cu_seqlens.numel() - 1
@@ -183,16 +196,17 @@ def wkv7_gdn_fwd(q, k, v, g, beta, s0=None, cu_seqlens=None, output_final_state:
         elif tuple(s0.shape) != (N, H, K, V):
             raise ValueError(f"s0 must have shape {(N, H, K, V)} or {(1, H, K, V)}")
     if o is None:
-        o = torch.empty((B, T, H, V), dtype=dt, device=q.device)
+        o = torch.empty(vshape, dtype=dt, device=q.device)
     else:
-        _check(o, "o", dt, (B, T, H, V))
+        _check(o, "o", dt, vshape)
     if output_final_state and sT is None:
         sT = torch.empty((N, H, K, V), dtype=torch.float32, device=q.device)
     elif sT is not None:
         _check(sT, "sT", torch.float32, (N, H, K, V))
     st = library().wkv7_gdn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0), shared,
                                 _ptr(o), _ptr(sT), B, T, H, K, V, _ptr(cu_seqlens), N,
-                                _dtype_code(q), ALGO[algo], _stream(q.device))
+                                int(bool(head_first)), _dtype_code(q), ALGO[algo],
+                                _stream(q.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_gdn_fwd")
     return o, sT

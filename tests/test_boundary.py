@@ -56,14 +56,15 @@ MIS = P + 2
 
 
 def fwd(lib, ptrs=None, B=1, T=8, H=2, K=64, V=64, cu=None, N=None, dtype=BF16, algo=0,
-        s0=None, sT=None, o=None, mask=None):
+        s0=None, sT=None, o=None, mask=None, layout=0):
     ptrs = ptrs or [P + 0x1000 * i for i in range(6)]
     o = P + 0x10000 if o is None else o
     N = B if N is None else N
     return lib.wkv7_fwd(*[ctypes.c_void_p(x) if x else None for x in ptrs],
                         ctypes.c_void_p(s0) if s0 else None, ctypes.c_void_p(mask) if mask else None,
                         ctypes.c_void_p(o) if o else None, ctypes.c_void_p(sT) if sT else None,
-                        B, T, H, K, V, ctypes.c_void_p(cu) if cu else None, N, dtype, algo, None)
+                        B, T, H, K, V, ctypes.c_void_p(cu) if cu else None, N, layout, dtype, algo,
+                        None)
 
 
 def test_fwd_rejects_bad_arguments(lib):
@@ -74,6 +75,7 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, T=-3) == ERR_INVALID_ARG
     assert fwd(lib, dtype=7) == ERR_INVALID_ARG
     assert fwd(lib, algo=9) == ERR_INVALID_ARG
+    assert fwd(lib, layout=2) == ERR_INVALID_ARG
     assert fwd(lib, ptrs=[P, 0, P + 32, P + 48, P + 64, P + 80]) == ERR_INVALID_ARG  # null w
     assert fwd(lib, ptrs=[P, MIS, P + 32, P + 48, P + 64, P + 80]) == ERR_INVALID_ARG
     assert fwd(lib, o=0) == ERR_INVALID_ARG
@@ -113,15 +115,15 @@ def test_binding_refuses_cpu_tensors():
 
 
 def gdn(lib, ptrs=None, B=1, T=8, H=2, K=64, V=64, cu=None, N=None, dtype=BF16, algo=0,
-        s0=None, shared=0, sT=None, o=None):
+        s0=None, shared=0, sT=None, o=None, layout=0):
     ptrs = ptrs or [P + 0x1000 * i for i in range(5)]
     o = P + 0x10000 if o is None else o
     N = B if N is None else N
     return lib.wkv7_gdn_fwd(*[ctypes.c_void_p(x) if x else None for x in ptrs],
                             ctypes.c_void_p(s0) if s0 else None, shared,
                             ctypes.c_void_p(o) if o else None, ctypes.c_void_p(sT) if sT else None,
-                            B, T, H, K, V, ctypes.c_void_p(cu) if cu else None, N, dtype, algo,
-                            None)
+                            B, T, H, K, V, ctypes.c_void_p(cu) if cu else None, N, layout, dtype,
+                            algo, None)
 
 
 def test_gdn_fwd_rejects_bad_arguments(lib):
@@ -130,6 +132,7 @@ def test_gdn_fwd_rejects_bad_arguments(lib):
     assert gdn(lib, dtype=3) == ERR_INVALID_ARG
     assert gdn(lib, algo=5) == ERR_INVALID_ARG
     assert gdn(lib, shared=2) == ERR_INVALID_ARG
+    assert gdn(lib, layout=-1) == ERR_INVALID_ARG
     assert gdn(lib, ptrs=[P, P + 16, P + 32, 0, P + 64]) == ERR_INVALID_ARG  # null g
     assert gdn(lib, ptrs=[P, P + 16, P + 32, P + 49, P + 64]) == ERR_INVALID_ARG  # odd bf16 g
     assert gdn(lib, ptrs=[P, P + 16, P + 32, P + 50, P + 66], dtype=F32) == ERR_INVALID_ARG

@@ -159,3 +159,17 @@ def test_steps_equal_forward(cuda_device):
     torch.testing.assert_close(state, s_fwd, rtol=0, atol=2e-5)
     o_ref, s_ref = ref(x)
     assert rel_err(state, s_ref) < 1e-5
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("T", [1, 65, 200])
+def test_head_first_layout(cuda_device, algo, T):
+    """head_first=True (README: q, k, v [B,H,T,*], g and beta [B,H,T]) gives the
+    token-major results."""
+    x = synth.gdn_inputs(2, T, 3, dtype=torch.bfloat16, seed=400 + T, s0_std=0.1)
+    o_ref, s_ref = ref(x)
+    xd = to_dev(x, cuda_device)
+    hf = {n: (xd[n].transpose(1, 2).contiguous() if n != "s0" else xd[n]) for n in xd}
+    o, s = wkv7_gdn_fwd(*(hf[n] for n in NAMES), s0=hf["s0"], algo=algo, head_first=True)
+    assert o.shape == (2, 3, T, 64)
+    check(o.transpose(1, 2), s, o_ref, s_ref, torch.bfloat16, f"gdn head_first {algo} T={T}")

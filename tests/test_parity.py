@@ -211,3 +211,39 @@ def test_bad_cu_seqlens_flagged_not_faulting(cuda_device, algo):
         raise
     assert wkv7_get_last_error() == ERR_DEVICE_BAD_SEQLENS
     assert wkv7_get_last_error() == OK  # the flag is cleared once read
+
+
+def _head_first(t):
+    return t.transpose(1, 2).contiguous()
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("T", [1, 64, 130])
+def test_head_first_layout(cuda_device, algo, T):
+    """head_first=True ([B,H,T,*] inputs and output, README generalized_delta_rule
+    argument): the same results as the token-major run, with and without a mask."""
+    x = synth.fwd_inputs(2, T, 3, dtype=torch.bfloat16, seed=300 + T, s0_std=0.1)
+    mask = torch.ones(2, T, dtype=torch.uint8)
+    mask[1, T // 3:T // 2] = 0
+    for m in (None, mask):
+        o_ref, s_ref = ref(x, mask=m)
+        xd = to_dev(x, cuda_device)
+        hf = {n: (_head_first(xd[n]) if n != "s0" else xd[n]) for n in xd}
+        o, s = wkv7_fwd(*(hf[n] for n in "rwkvab"), s0=hf["s0"],
+                        mask=None if m is None else m.to(cuda_device), algo=algo,
+                        head_first=True)
+        assert o.shape == (2, 3, T, 64)
+        check(o.transpose(1, 2), s, o_ref, s_ref, torch.bfloat16, f"head_first {algo} T={T}")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_head_first_varlen(cuda_device, algo):
+    lengths = torch.tensor([70, 0, 1, 129])
+    x = synth.varlen_inputs(lengths, 2, dtype=torch.bfloat16, seed=310, s0_std=0.1)
+    cu = x.pop("cu_seqlens")
+    o_ref, s_ref = ref(x, cu=cu)
+    xd = to_dev(x, cuda_device)
+    hf = {n: (_head_first(xd[n]) if n != "s0" else xd[n]) for n in xd}
+    o, s = wkv7_fwd(*(hf[n] for n in "rwkvab"), s0=hf["s0"], cu_seqlens=cu.to(cuda_device),
+                    algo=algo, head_first=True)
+    check(o.transpose(1, 2), s, o_ref, s_ref, torch.bfloat16, f"head_first varlen {algo}")
