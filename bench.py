@@ -184,13 +184,21 @@ def reference_arm(args, rank: int):
     if rank != 0:
         return
     import oracle
+    gdn = args.family == "gdn"
     H, T = FWD["H"], FWD["T"]
-    x = synth.fwd_inputs(1, T, H, dtype=torch.bfloat16, seed=FWD["seed"], s0_std=FWD["s0_std"])
+    if gdn:
+        x = synth.gdn_inputs(1, T, H, dtype=torch.bfloat16, seed=GDN_FWD["seed"],
+                             s0_std=GDN_FWD["s0_std"])
+        names, call = ("q", "k", "v", "g", "beta"), oracle.gdn_fwd
+    else:
+        x = synth.fwd_inputs(1, T, H, dtype=torch.bfloat16, seed=FWD["seed"],
+                             s0_std=FWD["s0_std"])
+        names, call = tuple("rwkvab"), oracle.fwd
     units = min(H, max(4, os.cpu_count() or 1))  # one whole (b, h) unit per host thread
-    sl = {n: x[n][:, :, :units] for n in "rwkvab"}
+    sl = {n: x[n][:, :, :units] for n in names}
 
     def one():
-        return oracle.fwd(*(sl[n] for n in "rwkvab"), s0=x["s0"][:, :units])[2]
+        return call(*(sl[n] for n in names), s0=x["s0"][:, :units])[2]
 
     for _ in range(args.warmup):
         one()
@@ -201,12 +209,13 @@ def reference_arm(args, rank: int):
     dt = time.perf_counter() - t0
     tokens = args.steps * units * T / H
     value = tokens / dt
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+    line = {"metric": GDN_METRIC if gdn else METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": fwd_config({"workload": "fwd_bf16_b8_t4096_h64", "B": FWD["B"], "T": T,
-                                  "H": H}, "oracle", args.gpus),
+            "config": fwd_config({"workload": ("gdn_" if gdn else "") + "fwd_bf16_b8_t4096_h64",
+                                  "B": FWD["B"], "T": T, "H": H}, "oracle", args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
                              "sample": f"each step: {units} of the 512 (b,h) units of "
                                        f"B=8,T={T},H={H}, full T each, fp64 sequential "

@@ -34,8 +34,10 @@
  *    WKV7_LAYOUT_BHTK (the README's head_first=True) they are [B, H, T, K] /
  *    [B, H, T, V] instead.  States are fp32 [N, H, K, V] in both layouts (the
  *    README's initial_state / final_state layout).
- *  - Supported head sizes: K == V == 64 (the README's default head_size).
- *    Other sizes return WKV7_ERR_UNSUPPORTED.
+ *  - Supported head sizes: K == V in {64, 128, 256} (the README's head_size,
+ *    default 64).  The chunked tensor-core kernel takes 64 only; other sizes
+ *    run on the fp32 CUDA-core kernels.  Anything else returns
+ *    WKV7_ERR_UNSUPPORTED.
  */
 #ifndef WKV7_H
 #define WKV7_H
@@ -66,7 +68,7 @@ typedef enum {
 } wkv7_layout;
 
 typedef enum {
-    WKV7_ALGO_AUTO = 0,      /* library's choice (chunked tensor-core form for bf16 when built) */
+    WKV7_ALGO_AUTO = 0,      /* library's choice (chunked tensor-core form for bf16, K = 64)   */
     WKV7_ALGO_RECURRENT = 1, /* token-by-token fp32 recurrence on CUDA cores                  */
     WKV7_ALGO_CHUNKED = 2    /* 64-token chunks, WY form, tcgen05 tensor cores (bf16 only)    */
 } wkv7_algo;

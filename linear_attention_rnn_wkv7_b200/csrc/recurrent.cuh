@@ -9,9 +9,15 @@
 // K are a thread's own sum plus log2(P) shuffles.  K = V = 64 is one block of 64
 // threads per (sequence, head); the README's other head sizes (128, 256) take
 // K / 64 column slabs of 64 x P threads, every slab reading the whole K-side vectors.
-// Tokens are staged 1024 / K at a time in shared memory (r, exp(w), k, a, b over K
-// and the slab's 64 entries of v, as fp32) so that each thread reads the shared
-// vectors as float4 broadcasts.
+// (Four threads per column at every head size, i.e. more warps with shorter
+// chains, measured slower: the extra shuffles sit on each token's dependency chain.)
+//
+// Tokens go through shared memory in tiles of 512 / K: while a tile is computed,
+// cp.async copies the next tile's raw inputs (r, w, k, a, b rows and the slab's 64
+// entries of v) into the other half of a double buffer, so the recurrence never
+// waits for global memory.  Each tile is then converted once to fp32 (exp(w)
+// included) in a layout whose 64-float parts are 68 floats apart, so the P parts a
+// warp reads as float4 broadcasts sit in different banks.
 //
 // This is the fp32-input path (its accuracy is that of an fp32 recurrence)
 // and the anchor the chunked tensor-core kernel is checked against; masks,
@@ -19,7 +25,7 @@
 // chunked kernel.
 //
 // kGdn: Gated DeltaNet (rwkv-ops 0.9.0 README, "gdn_recurrent 使用方法").  The
-// staging turns q, k, v, g, beta into the generalized rule's per-token vectors:
+// conversion turns q, k, v, g, beta into the generalized rule's per-token vectors:
 // r = qh, exp(w) = e^{g} on every channel, write key beta kh, a = kh and
 // b = -e^{g} beta kh (qh, kh: q and k over their L2 norms), so the loop below
 // applies e^{g} (I - beta kh kh^T) S + beta kh v^T.
@@ -28,7 +34,24 @@
 
 namespace wkv7 {
 
-// K (= V): head size.  Block: 64 columns x P = K / 64 threads per column.
+namespace rec {
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+}  // namespace rec
+
+// K (= V): head size.  Block: 64 columns x P = K / 64 threads per column, 64 rows each.
 template <typename Tin, bool kGdn, int K>
 __global__ void __launch_bounds__(K)
 recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
@@ -37,11 +60,23 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
                  float* sT, int T, int H, const int32_t* __restrict__ cu_seqlens,
                  const Tin* __restrict__ g, const Tin* __restrict__ beta, int s0_shared,
                  int head_first) {
+    using namespace rec;
     constexpr int P = K / 64;        // threads per state column
-    constexpr int kTile = 1024 / K;  // tokens per staging round
+    constexpr int R = 64;            // rows per thread
+    constexpr int kSeg = R + 4;      // floats between the parts of a converted row
+    constexpr int kThreads = K;
+    constexpr int kTile = 512 / K;   // tokens per tile
     constexpr int kSlabs = K / 64;   // 64-column slabs per (sequence, head)
-    __shared__ __align__(16) float sm[5][kTile][K];  // r, d, k, a, b
-    __shared__ __align__(16) float sv[kTile][64];    // this slab's v
+    constexpr int KP = P * kSeg;     // converted row length (padded parts)
+    constexpr int EPC = 16 / (int)sizeof(Tin);  // elements per 16-byte copy
+    constexpr int CR = K / EPC;      // copies per K-row
+    constexpr int CV = 64 / EPC;     // copies per v slab row
+    constexpr int NV = kGdn ? 2 : 5; // K-rows per token: q, k  or  r, w, k, a, b
+    constexpr int PER_TOK = NV * CR + CV;
+    __shared__ __align__(16) Tin raw[2][5][kTile][K];  // r (q), w, k, a, b as loaded
+    __shared__ __align__(16) Tin rawv[2][kTile][64];
+    __shared__ __align__(16) float sm[5][kTile][KP];   // r, d = exp(w), k, a, b (fp32)
+    __shared__ __align__(16) float sv[kTile][64];      // this slab's v
     __shared__ uint8_t smask[kTile];
     __shared__ float sgb[4][kTile];  // Gated DeltaNet: g, beta, 1/|q|, 1/|k|
 
@@ -50,7 +85,7 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
     const int h = unit % H;
     const int n = unit / H;
     const int tid = threadIdx.x;
-    const int c = tid / P, part = tid % P;  // column of the slab, 64-row part of it
+    const int c = tid / P, part = tid % P;  // column of the slab, R-row part of it
     const int col = 64 * slab + c;          // state column
     int bb = n, bos = 0, eos = T;
     if (cu_seqlens) {
@@ -69,64 +104,96 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
     const size_t state_off = ((size_t)n * H + h) * K * K;
     const size_t init_off = s0_shared ? (size_t)h * K * K : state_off;
 
-    float S[64];  // rows 64 part .. 64 part + 63 of column col
-#pragma unroll
-    for (int i = 0; i < 64; ++i)
-        S[i] = s0 ? s0[init_off + (size_t)(64 * part + i) * K + col] : 0.f;
-
-    for (int t0 = bos; t0 < eos; t0 += kTile) {
-        const int cnt = min(kTile, eos - t0);
-        __syncthreads();
-        if constexpr (kGdn) {
-            for (int tt = 0; tt < cnt; ++tt) {
-                const size_t row = (tb + (size_t)(t0 + tt) * ts) * K;
-                sm[0][tt][tid] = to_f32(r[row + tid]);  // q
-                sm[3][tt][tid] = to_f32(k[row + tid]);
-                if (tid < 64) sv[tt][tid] = to_f32(v[row + 64 * slab + tid]);
+    // Copies of tile [t0, t0 + cnt) into buffer buf; per-token scalars (mask or g,
+    // beta) are read into registers here and stored at the tile's conversion.
+    float pre_g = 0.f, pre_b = 0.f;
+    uint8_t pre_m = 1;
+    auto issue = [&](int buf, int t0, int cnt) {
+        for (int idx = tid; idx < cnt * PER_TOK; idx += kThreads) {
+            const int tt = idx / PER_TOK, rem = idx - tt * PER_TOK;
+            const size_t row = (tb + (size_t)(t0 + tt) * ts) * K;
+            if (rem < NV * CR) {
+                const int vi = rem / CR, e = (rem - vi * CR) * EPC;
+                const int slot = kGdn ? 2 * vi : vi;  // q -> slot 0, k -> slot 2
+                const Tin* src = slot == 0 ? r : slot == 1 ? w : slot == 2 ? k : slot == 3 ? a : b;
+                cp_async16(&raw[buf][slot][tt][e], src + row + e);
+            } else {
+                const int e = (rem - NV * CR) * EPC;
+                cp_async16(&rawv[buf][tt][e], v + row + 64 * slab + e);
             }
+        }
+        if (tid < cnt) {
+            const size_t tok = tb + (size_t)(t0 + tid) * ts;
+            if constexpr (kGdn) {
+                pre_g = to_f32(g[tok]);
+                pre_b = to_f32(beta[tok]);
+            } else {
+                pre_m = mask ? (mask[(size_t)bb * T + t0 + tid] != 0) : 1;
+            }
+        }
+    };
+
+    float S[R];  // rows R part .. R part + R - 1 of column col
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+        S[i] = s0 ? s0[init_off + (size_t)(R * part + i) * K + col] : 0.f;
+
+    if (bos < eos) issue(0, bos, min(kTile, eos - bos));
+    cp_async_commit();
+    const int pe = tid + (kSeg - R) * (tid / R);  // element tid, padded
+    for (int t0 = bos, buf = 0; t0 < eos; t0 += kTile, buf ^= 1) {
+        const int cnt = min(kTile, eos - t0);
+        const float my_g = pre_g, my_b = pre_b;
+        const uint8_t my_m = pre_m;
+        if (t0 + kTile < eos) issue(buf ^ 1, t0 + kTile, min(kTile, eos - t0 - kTile));
+        cp_async_commit();
+        cp_async_wait<1>();  // this tile's copies (the next tile's may still be in flight)
+        __syncthreads();     // every thread's copies visible; the last tile's reads done
+        if constexpr (kGdn) {
             if (tid < cnt) {
-                const size_t tok = tb + (size_t)(t0 + tid) * ts;
-                sgb[0][tid] = to_f32(g[tok]);
-                sgb[1][tid] = to_f32(beta[tok]);
+                sgb[0][tid] = my_g;
+                sgb[1][tid] = my_b;
                 smask[tid] = 1;
             }
-            __syncthreads();
             if (tid < 2 * cnt) {  // thread 2 tt + e: the inverse norm of q (e = 0) or k (e = 1)
-                const float* x = sm[(tid & 1) ? 3 : 0][tid >> 1];
+                const Tin* x = raw[buf][(tid & 1) ? 2 : 0][tid >> 1];
                 float ss = 0.f;
-                for (int i = 0; i < K; ++i) ss = fmaf(x[i], x[i], ss);
+                for (int i = 0; i < K; ++i) {
+                    const float xi = to_f32(x[i]);
+                    ss = fmaf(xi, xi, ss);
+                }
                 sgb[2 + (tid & 1)][tid >> 1] = ss > 0.f ? rsqrtf(ss) : 0.f;  // zero stays zero
             }
             __syncthreads();
             for (int tt = 0; tt < cnt; ++tt) {
-                const float kn = sm[3][tt][tid] * sgb[3][tt];
+                const float kn = to_f32(raw[buf][2][tt][tid]) * sgb[3][tt];
                 const float alpha = expf(sgb[0][tt]), bt = sgb[1][tt];
-                sm[0][tt][tid] *= sgb[2][tt];
-                sm[1][tt][tid] = alpha;
-                sm[2][tt][tid] = bt * kn;
-                sm[3][tt][tid] = kn;
-                sm[4][tt][tid] = -alpha * bt * kn;
+                sm[0][tt][pe] = to_f32(raw[buf][0][tt][tid]) * sgb[2][tt];
+                sm[1][tt][pe] = alpha;
+                sm[2][tt][pe] = bt * kn;
+                sm[3][tt][pe] = kn;
+                sm[4][tt][pe] = -alpha * bt * kn;
+                if (tid < 64) sv[tt][tid] = to_f32(rawv[buf][tt][tid]);
             }
         } else {
             for (int tt = 0; tt < cnt; ++tt) {
-                const size_t row = (tb + (size_t)(t0 + tt) * ts) * K;
-                sm[0][tt][tid] = to_f32(r[row + tid]);
-                sm[1][tt][tid] = expf(to_f32(w[row + tid]));
-                sm[2][tt][tid] = to_f32(k[row + tid]);
-                sm[3][tt][tid] = to_f32(a[row + tid]);
-                sm[4][tt][tid] = to_f32(b[row + tid]);
-                if (tid < 64) sv[tt][tid] = to_f32(v[row + 64 * slab + tid]);
+                sm[0][tt][pe] = to_f32(raw[buf][0][tt][tid]);
+                sm[1][tt][pe] = expf(to_f32(raw[buf][1][tt][tid]));
+                sm[2][tt][pe] = to_f32(raw[buf][2][tt][tid]);
+                sm[3][tt][pe] = to_f32(raw[buf][3][tt][tid]);
+                sm[4][tt][pe] = to_f32(raw[buf][4][tt][tid]);
+                if (tid < 64) sv[tt][tid] = to_f32(rawv[buf][tt][tid]);
             }
-            if (tid < cnt) smask[tid] = mask ? (mask[(size_t)bb * T + t0 + tid] != 0) : 1;
+            if (tid < cnt) smask[tid] = my_m;
         }
         __syncthreads();
 
         for (int tt = 0; tt < cnt; ++tt) {
             if (smask[tt]) {
-                const float4* a4 = reinterpret_cast<const float4*>(sm[3][tt] + 64 * part);
+                const float4* a4 = reinterpret_cast<const float4*>(sm[3][tt] + kSeg * part);
                 float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
 #pragma unroll
-                for (int i4 = 0; i4 < 16; ++i4) {
+                for (int i4 = 0; i4 < R / 4; ++i4) {
                     const float4 av = a4[i4];
                     u0 = fmaf(S[4 * i4 + 0], av.x, u0);
                     u1 = fmaf(S[4 * i4 + 1], av.y, u1);
@@ -137,11 +204,11 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
 #pragma unroll
                 for (int m = 1; m < P; m *= 2) u += __shfl_xor_sync(0xffffffffu, u, m);
                 const float vj = sv[tt][c];
-                const float4* d4 = reinterpret_cast<const float4*>(sm[1][tt] + 64 * part);
-                const float4* k4 = reinterpret_cast<const float4*>(sm[2][tt] + 64 * part);
-                const float4* b4 = reinterpret_cast<const float4*>(sm[4][tt] + 64 * part);
+                const float4* d4 = reinterpret_cast<const float4*>(sm[1][tt] + kSeg * part);
+                const float4* k4 = reinterpret_cast<const float4*>(sm[2][tt] + kSeg * part);
+                const float4* b4 = reinterpret_cast<const float4*>(sm[4][tt] + kSeg * part);
 #pragma unroll
-                for (int i4 = 0; i4 < 16; ++i4) {
+                for (int i4 = 0; i4 < R / 4; ++i4) {
                     const float4 dv = d4[i4], kv = k4[i4], bv = b4[i4];
                     S[4 * i4 + 0] = fmaf(S[4 * i4 + 0], dv.x, fmaf(bv.x, u, kv.x * vj));
                     S[4 * i4 + 1] = fmaf(S[4 * i4 + 1], dv.y, fmaf(bv.y, u, kv.y * vj));
@@ -149,10 +216,10 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
                     S[4 * i4 + 3] = fmaf(S[4 * i4 + 3], dv.w, fmaf(bv.w, u, kv.w * vj));
                 }
             }
-            const float4* r4 = reinterpret_cast<const float4*>(sm[0][tt] + 64 * part);
+            const float4* r4 = reinterpret_cast<const float4*>(sm[0][tt] + kSeg * part);
             float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
 #pragma unroll
-            for (int i4 = 0; i4 < 16; ++i4) {
+            for (int i4 = 0; i4 < R / 4; ++i4) {
                 const float4 rv = r4[i4];
                 o0 = fmaf(S[4 * i4 + 0], rv.x, o0);
                 o1 = fmaf(S[4 * i4 + 1], rv.y, o1);
@@ -168,9 +235,10 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
             }
         }
     }
+    cp_async_wait<0>();  // nothing is left in flight when the block exits
     if (sT) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) sT[state_off + (size_t)(64 * part + i) * K + col] = S[i];
+        for (int i = 0; i < R; ++i) sT[state_off + (size_t)(R * part + i) * K + col] = S[i];
     }
 }
 
