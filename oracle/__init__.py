@@ -13,6 +13,9 @@ see ``wkv7_oracle.c`` for the equations.  ``step`` is the length-one case
 (B,H,K,K)).  ``brute`` holds an independent dense-product form used only to
 pin this one on tiny inputs.
 
+``bwd`` is the backward of ``fwd`` (plain reverse-mode differentiation of the
+same recurrence, every state kept), for dL/do and dL/dS_T given.
+
 ``gdn_fwd`` / ``gdn_step`` are the Gated DeltaNet operator of the same README
 (sections "gdn_recurrent 使用方法" and "gdn_chunk 使用方法": q, k L2-normalised
 inside, g a log-space decay gate per (b, t, h), beta a write strength in (0, 1)
@@ -53,6 +56,10 @@ def load_library(path: str):
     lib.wkv7_oracle_fwd.restype = ctypes.c_int
     lib.wkv7_oracle_fwd.argtypes = [p, p, p, p, p, p, p, p, p, p,
                                     i, i, i, i, i, p, i, i, ctypes.POINTER(ctypes.c_int)]
+    if hasattr(lib, "wkv7_oracle_bwd"):
+        lib.wkv7_oracle_bwd.restype = ctypes.c_int
+        lib.wkv7_oracle_bwd.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i,
+                                                   ctypes.POINTER(ctypes.c_int)]
     if hasattr(lib, "gdn_oracle_fwd"):
         lib.gdn_oracle_fwd.restype = ctypes.c_int
         lib.gdn_oracle_fwd.argtypes = [p, p, p, p, p, p, i, p, p,
@@ -174,3 +181,33 @@ def gdn_step(q, k, v, g, beta, state, nthreads: int = 0):
     q, k, v, g, beta = (_f64(x)[:, None] for x in (q, k, v, g, beta))
     o, sT, _ = gdn_fwd(q, k, v, g, beta, s0=_f64(state), nthreads=nthreads)
     return o[:, 0], sT
+
+
+def bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=None,
+        nthreads: int = 0, library=None):
+    """Oracle backward.  Returns a dict of float64 arrays: dr, dw, dk, da, db [B,T,H,K],
+    dv [B,T,H,V], ds0 [N,H,K,V]."""
+    r, w, k, v, a, b, dout = (_f64(x) for x in (r, w, k, v, a, b, dout))
+    B, T, H, K = r.shape
+    V = v.shape[-1]
+    assert dout.shape == (B, T, H, V)
+    cu = _cu(cu_seqlens)
+    N = B if cu is None else cu.shape[0] - 1
+    s0, dsT = _f64(s0), _f64(dsT)
+    m = None
+    if mask is not None:
+        m = mask.cpu().numpy() if hasattr(mask, "cpu") else np.asarray(mask)
+        m = np.ascontiguousarray((m != 0).astype(np.uint8))
+    g = {n: np.zeros((B, T, H, K)) for n in ("dr", "dw", "dk", "da", "db")}
+    g["dv"] = np.zeros((B, T, H, V))
+    g["ds0"] = np.zeros((N, H, K, V))
+    used = ctypes.c_int(0)
+    lib = _load() if library is None else library
+    rc = lib.wkv7_oracle_bwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0),
+                             _ptr(m), _ptr(dout), _ptr(dsT), _ptr(g["dr"]), _ptr(g["dw"]),
+                             _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["db"]),
+                             _ptr(g["ds0"]), B, T, H, K, V, _ptr(cu), N, int(nthreads),
+                             ctypes.byref(used))
+    if rc != 0:
+        raise ValueError("wkv7_oracle_bwd rejected its arguments")
+    return g

@@ -257,3 +257,164 @@ int gdn_oracle_fwd(const double* q, const double* k, const double* v,
     if (threads_used) *threads_used = used;
     return 0;
 }
+
+/*
+ * Backward of the generalized delta rule above (the README: the chunked
+ * generalized_delta_rule entry supports backpropagation; rwkv-ops 0.9.0 README,
+ * "rwkv7op 使用方法").  Given dL/do (dout, [B,T,H,V]) and dL/dS_T (dsT, [N,H,K,V]
+ * or NULL), returns dL/dr, dw, dk, dv, da, db ([B,T,H,*]) and dL/ds0 ([N,H,K,V]).
+ * Plain reverse-mode differentiation of the forward recurrence, token by token,
+ * with every state of the unit kept (S_0 .. S_L):
+ *
+ *   o_t = S_t^T r_t            ->  G += r_t do_t^T,   dr_t = S_t do_t
+ *   S_t = D_t S_{t-1} + b_t u_t^T + k_t v_t^T,  u_t = S_{t-1}^T a_t,  D_t = diag(e^{w_t}):
+ *        dv_t = G^T k_t,   dk_t = G v_t,   du_t = G^T b_t,   db_t = G u_t,
+ *        da_t = S_{t-1} du_t,   dw_t = e^{w_t} * rowsum(G * S_{t-1}),
+ *        G <- D_t G + a_t du_t^T                 (G becomes dL/dS_{t-1})
+ *   a masked token passes G through unchanged and has zero dw, dk, dv, da, db.
+ * At the end dL/ds0 = G.
+ */
+static void oracle_unit_bwd(const double* r, const double* w, const double* k,
+                            const double* v, const double* a, const double* b,
+                            const double* s0, const unsigned char* mask,
+                            const double* dout, const double* dsT, double* dr,
+                            double* dw, double* dk, double* dv, double* da,
+                            double* db, double* ds0, int T, int H, int K, int V,
+                            int bb, int bos, int eos, int n, int h) {
+    const size_t KV = (size_t)K * V;
+    const size_t state_off = ((size_t)n * H + h) * KV;
+    const int L = eos - bos;
+    double* S = (double*)malloc(sizeof(double) * KV * (size_t)(L + 1));
+    double* G = (double*)malloc(sizeof(double) * KV);
+    double* u = (double*)malloc(sizeof(double) * V);
+    double* du = (double*)malloc(sizeof(double) * V);
+    if (s0)
+        memcpy(S, s0 + state_off, sizeof(double) * KV);
+    else
+        memset(S, 0, sizeof(double) * KV);
+    for (int p = 0; p < L; ++p) {  /* forward, keeping S_{p+1} */
+        const int t = bos + p;
+        const size_t rowK = (((size_t)bb * T + t) * H + h) * (size_t)K;
+        const size_t rowV = (((size_t)bb * T + t) * H + h) * (size_t)V;
+        const double* Sp = S + KV * (size_t)p;
+        double* Sn = S + KV * (size_t)(p + 1);
+        if (mask && mask[(size_t)bb * T + t] == 0) {
+            memcpy(Sn, Sp, sizeof(double) * KV);
+            continue;
+        }
+        for (int j = 0; j < V; ++j) {
+            u[j] = 0.0;
+            for (int i = 0; i < K; ++i) u[j] += Sp[(size_t)i * V + j] * a[rowK + i];
+        }
+        for (int i = 0; i < K; ++i)
+            for (int j = 0; j < V; ++j)
+                Sn[(size_t)i * V + j] = exp(w[rowK + i]) * Sp[(size_t)i * V + j] +
+                                        b[rowK + i] * u[j] + k[rowK + i] * v[rowV + j];
+    }
+    if (dsT)
+        memcpy(G, dsT + state_off, sizeof(double) * KV);
+    else
+        memset(G, 0, sizeof(double) * KV);
+    for (int p = L - 1; p >= 0; --p) {
+        const int t = bos + p;
+        const size_t rowK = (((size_t)bb * T + t) * H + h) * (size_t)K;
+        const size_t rowV = (((size_t)bb * T + t) * H + h) * (size_t)V;
+        const double* Sp = S + KV * (size_t)p;        /* S_{t-1} */
+        const double* St = S + KV * (size_t)(p + 1);  /* S_t */
+        for (int i = 0; i < K; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < V; ++j) {
+                G[(size_t)i * V + j] += r[rowK + i] * dout[rowV + j];
+                acc += St[(size_t)i * V + j] * dout[rowV + j];
+            }
+            dr[rowK + i] = acc;
+        }
+        if (mask && mask[(size_t)bb * T + t] == 0) {
+            for (int i = 0; i < K; ++i) dw[rowK + i] = dk[rowK + i] = da[rowK + i] = db[rowK + i] = 0.0;
+            for (int j = 0; j < V; ++j) dv[rowV + j] = 0.0;
+            continue;
+        }
+        for (int j = 0; j < V; ++j) {
+            double su = 0.0, sv = 0.0, sd = 0.0;
+            for (int i = 0; i < K; ++i) {
+                su += Sp[(size_t)i * V + j] * a[rowK + i];
+                sv += G[(size_t)i * V + j] * k[rowK + i];
+                sd += G[(size_t)i * V + j] * b[rowK + i];
+            }
+            u[j] = su;
+            dv[rowV + j] = sv;
+            du[j] = sd;
+        }
+        for (int i = 0; i < K; ++i) {
+            double sk = 0.0, sb = 0.0, sa = 0.0, sw = 0.0;
+            for (int j = 0; j < V; ++j) {
+                const double g = G[(size_t)i * V + j];
+                sk += g * v[rowV + j];
+                sb += g * u[j];
+                sa += Sp[(size_t)i * V + j] * du[j];
+                sw += g * Sp[(size_t)i * V + j];
+            }
+            const double di = exp(w[rowK + i]);
+            dk[rowK + i] = sk;
+            db[rowK + i] = sb;
+            da[rowK + i] = sa;
+            dw[rowK + i] = di * sw;
+            for (int j = 0; j < V; ++j)
+                G[(size_t)i * V + j] = di * G[(size_t)i * V + j] + a[rowK + i] * du[j];
+        }
+    }
+    if (ds0) memcpy(ds0 + state_off, G, sizeof(double) * KV);
+    free(S);
+    free(G);
+    free(u);
+    free(du);
+}
+
+/* Same conventions and return codes as wkv7_oracle_fwd.  dout is required; dsT
+ * and ds0 may be NULL. */
+int wkv7_oracle_bwd(const double* r, const double* w, const double* k,
+                    const double* v, const double* a, const double* b,
+                    const double* s0, const unsigned char* mask, const double* dout,
+                    const double* dsT, double* dr, double* dw, double* dk,
+                    double* dv, double* da, double* db, double* ds0, int B,
+                    int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
+                    int nthreads, int* threads_used) {
+    if (!r || !w || !k || !v || !a || !b || !dout) return 1;
+    if (!dr || !dw || !dk || !dv || !da || !db) return 1;
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0) return 1;
+    if (cu_seqlens) {
+        if (B != 1 || N < 0 || cu_seqlens[0] != 0 || cu_seqlens[N] != T) return 1;
+        for (int n = 0; n < N; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n]) return 1;
+    } else {
+        N = B;
+    }
+    const long units = (long)N * H;
+    int used = 1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel
+    {
+#pragma omp single
+        used = omp_get_num_threads();
+#pragma omp for schedule(dynamic, 1)
+        for (long unit = 0; unit < units; ++unit) {
+            const int n = (int)(unit / H), h = (int)(unit % H);
+            oracle_unit_bwd(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da, db,
+                            ds0, T, H, K, V, cu_seqlens ? 0 : n,
+                            cu_seqlens ? cu_seqlens[n] : 0,
+                            cu_seqlens ? cu_seqlens[n + 1] : T, n, h);
+        }
+    }
+#else
+    (void)nthreads;
+    for (long unit = 0; unit < units; ++unit) {
+        const int n = (int)(unit / H), h = (int)(unit % H);
+        oracle_unit_bwd(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da, db, ds0,
+                        T, H, K, V, cu_seqlens ? 0 : n, cu_seqlens ? cu_seqlens[n] : 0,
+                        cu_seqlens ? cu_seqlens[n + 1] : T, n, h);
+    }
+#endif
+    if (threads_used) *threads_used = used;
+    return 0;
+}
