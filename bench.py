@@ -237,7 +237,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--batch", type=int, default=FWD["B"],
                     help="forward batch (default 8; smaller only for profiling captures)")
-    ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward leg")
+    ap.add_argument("--only", choices=["all", "fwd", "decode", "bwd"], default="all",
                     help="run only one leg (profiling captures)")
     ap.add_argument("--workload", choices=["b8_t4096_h64", "masked_b16_t4096_h32",
                                            "varlen_64seq_h32"], default="b8_t4096_h64",
@@ -259,8 +260,8 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
-    from linear_attention_rnn_wkv7_b200 import (library, wkv7_fwd, wkv7_gdn_fwd, wkv7_gdn_step,
-                                                wkv7_step)
+    from linear_attention_rnn_wkv7_b200 import (library, wkv7_bwd, wkv7_fwd, wkv7_gdn_fwd,
+                                                wkv7_gdn_step, wkv7_step)
     library()  # fail loudly if the CUDA library is missing
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
@@ -290,6 +291,11 @@ def main():
     if args.only in ("all", "decode") and not args.no_decode:
         decode = decode_leg(device, stream, wkv7_gdn_step if gdn else wkv7_step, hbm_peak,
                             peak_kind, max_over_ranks, barrier, rank, gdn, args.head_size)
+    backward = None
+    if (args.only in ("all", "bwd") and not args.no_bwd and not gdn and args.head_size == 64
+            and args.workload == "b8_t4096_h64"):
+        backward = bwd_leg(args, device, stream, wkv7_bwd, hbm_peak, peak_kind, max_over_ranks,
+                           barrier, rank)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu and args.only == "all" and args.head_size == 64:
         cpu = cpu_oracle_sample(gdn=gdn)
@@ -304,7 +310,7 @@ def main():
                 "config": fwd_config(desc, args.algo, world, args.head_size),
                 "roofline": fwd and fwd["roofline"], "cpu_baseline": cpu,
                 "e2e": fwd and fwd["e2e"], "gpu_launches": args.steps if fwd else 0,
-                "clocks": fwd and fwd["clocks"], "decode": decode}
+                "clocks": fwd and fwd["clocks"], "decode": decode, "backward": backward}
         print(json.dumps(line), flush=True)
     if pg is not None:
         pg.destroy_process_group()
@@ -448,6 +454,51 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
     return {"value": value, "ms_per_step": ms_step, "roofline": roofline, "e2e": e2e,
             "clocks": clock_info, "desc": desc}
+
+
+def bwd_leg(args, device, stream, wkv7_bwd, hbm_peak, peak_kind, max_over_ranks, barrier, rank):
+    """wkv7_bwd on the B=8, T=4096, H=64 bf16 forward workload (random dL/do and
+    dL/dS_T), inputs and workspace resident; up to 20 timed launches."""
+    B, T, H = args.batch, FWD["T"], FWD["H"]
+    x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16,
+                         seed=replicas.replica_seed(FWD["seed"], rank), s0_std=FWD["s0_std"])
+    gen = torch.Generator().manual_seed(replicas.replica_seed(620, rank))
+    dout = torch.randn(B, T, H, 64, generator=gen).to(torch.bfloat16).to(device)
+    dsT = (torch.randn(B, H, 64, 64, generator=gen) * 0.1).to(device)
+    xd = {k: v.to(device) for k, v in x.items()}
+    ws = torch.empty(wkv7_bwd_workspace_nbytes(B, T, H), dtype=torch.uint8, device=device)
+
+    def step():
+        wkv7_bwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], dout, s0=xd["s0"],
+                 dsT=dsT, workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    barrier()
+    steps = max(1, min(args.steps, 20))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
+    # inputs r,w,k,v,a,b and dout read, six gradients written (bf16), s0 and dsT read and
+    # ds0 written (fp32); the workspace (checkpoints, u) is not counted
+    nbytes = B * T * H * 13 * 64 * 2 + 3 * B * H * STATE_BYTES
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"bwd_bf16_b{B}_t{T}_h{H}", "steps": steps, "ms_per_step": ms,
+            "tokens/s": B * T / (ms / 1e3), "algorithmic_bytes_per_step": nbytes, "GB/s": gbs,
+            "peak": hbm_peak, "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
+            "workspace_bytes": ws.numel(), "gpu_launches": 2 * steps,
+            "kernels": "ckpt_kernel (forward, checkpoints) + bwd_kernel (reverse)"}
+
+
+def wkv7_bwd_workspace_nbytes(B, T, H):
+    from linear_attention_rnn_wkv7_b200 import library
+    return int(library().wkv7_bwd_workspace_bytes(B, T, H, 64, 64))
 
 
 def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank,

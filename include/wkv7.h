@@ -42,6 +42,7 @@
 #ifndef WKV7_H
 #define WKV7_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -123,6 +124,40 @@ wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
 wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v,
                       const void* a, const void* b, float* state, void* o, int B, int H,
                       int K, int V, wkv7_dtype dtype, void* stream);
+
+/*
+ * wkv7_bwd -- backward of wkv7_fwd (the README's training entry,
+ * generalized_delta_rule, supports backpropagation; rwkv-ops 0.9.0 README,
+ * "rwkv7op 使用方法").  For the loss L = sum(o * dout) + sum(S_T * dsT) it writes
+ * the gradients of every forward input, by reverse-mode differentiation of the
+ * recurrence:
+ *
+ *     G = dL/dS_t;  G += r_t do_t^T;  dr_t = S_t do_t;  dv_t = G^T k_t;  dk_t = G v_t;
+ *     du_t = G^T b_t;  db_t = G u_t;  da_t = S_{t-1} du_t;
+ *     dw_t = e^{w_t} * rowsum(G * S_{t-1});  G <- diag(e^{w_t}) G + a_t du_t^T;
+ *     ds0 = G after the first token.
+ *
+ *   r, w, k, v, a, b, s0, mask   as for wkv7_fwd ([B, T, H, 64], token-major, no varlen)
+ *   dout           [B, T, H, V]  dtype   dL/do (required)
+ *   dsT            [B, H, K, V]  fp32    dL/dS_T, or NULL for zero
+ *   dr, dw, dk, da, db [B, T, H, K], dv [B, T, H, V]   dtype   outputs (fully written;
+ *                                        must not alias an input)
+ *   ds0            [B, H, K, V]  fp32    dL/ds0, or NULL to skip
+ *   workspace      device buffer of at least wkv7_bwd_workspace_bytes(B, T, H, K, V)
+ *                  bytes (16-byte aligned; the caller owns it): the forward states
+ *                  every 8 tokens and every token's u = S_{t-1}^T a, recomputed here
+ *
+ * K = V = 64 only.  A masked token passes the state gradient through and has zero
+ * dw, dk, dv, da, db.  Two kernels on `stream`: a forward that writes the
+ * checkpoints, then the reverse pass.
+ */
+size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V);
+
+wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
+                     const void* b, const float* s0, const uint8_t* mask, const void* dout,
+                     const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
+                     void* db, float* ds0, int B, int T, int H, int K, int V,
+                     wkv7_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * wkv7_gdn_fwd -- Gated DeltaNet forward over whole sequences

@@ -1,0 +1,306 @@
+// backward.cuh -- backward of the WKV7 forward (the README's training entry,
+// generalized_delta_rule, supports backpropagation; rwkv-ops 0.9.0 README,
+// "rwkv7op 使用方法"), K = V = 64, fp32 on CUDA cores.
+//
+// Given dL/do and dL/dS_T, reverse-mode differentiation of
+//     u_t = S_{t-1}^T a_t,  S_t = D_t S_{t-1} + b_t u_t^T + k_t v_t^T,  o_t = S_t^T r_t
+// runs backwards with the adjoint G = dL/dS_t:
+//     G += r_t do_t^T;  dr_t = S_t do_t;  dv_t = G^T k_t;  dk_t = G v_t;
+//     du_t = G^T b_t;   db_t = G u_t;     da_t = S_{t-1} du_t;
+//     dw_t = e^{w_t} * rowsum(G * S_{t-1});  G <- D_t G + a_t du_t^T
+// and finally dL/ds0 = G.  Two kernels:
+//   ckpt_kernel  re-runs the forward with one thread per state column (as the
+//                recurrent forward) and writes the state before every kCkpt-th token
+//                and the final state (the checkpoints), and every token's u_t;
+//   bwd_kernel   walks the tokens backwards with one thread per state row: it holds
+//                row i of S_t and of G, so dr, dk, db, da, dw are in-thread sums over
+//                the row; dv and du (sums over rows) go through G written to shared
+//                memory once per token.  S_{t-1} is rebuilt from S_t with the stored
+//                u_t, S_{t-1} = D_t^{-1} (S_t - b_t u_t^T - k_t v_t^T), at most
+//                kCkpt - 1 times in a row before the next checkpoint replaces it
+//                (the rebuild scales errors by e^{-w} per step; with the checkpoint
+//                interval of 8 that stays below e^{4.3} for per-step decays >= -0.607).
+// A masked token passes G through unchanged and gets zero dw, dk, dv, da, db.
+#pragma once
+#include "common.cuh"
+
+namespace wkv7 {
+
+namespace bwd {
+
+constexpr int kCkpt = 8;  // tokens between checkpoints (one reverse tile)
+constexpr int kRow = 68;  // padded row length of the adjoint in shared memory
+
+// Workspace: checkpoints [units][nC + 1][64][64] fp32, then u [units][T][64] fp32.
+inline size_t workspace_floats(long long units, int T) {
+    const long long nC = (T + kCkpt - 1) / kCkpt;
+    return (size_t)units * ((size_t)(nC + 1) * 4096 + (size_t)T * 64);
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(64)
+ckpt_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
+            const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
+            const float* __restrict__ s0, const uint8_t* __restrict__ mask,
+            float* __restrict__ ckpt, float* __restrict__ uws, int T, int H) {
+    constexpr int kTile = 16;
+    __shared__ __align__(16) float sm[4][kTile][64];  // d = exp(w), k, a, b
+    __shared__ float sv[kTile][64];
+    __shared__ uint8_t smask[kTile];
+    const int unit = blockIdx.x;
+    const int h = unit % H, bb = unit / H;
+    const int j = threadIdx.x;
+    const int nC = (T + kCkpt - 1) / kCkpt;
+    float* ck = ckpt + (size_t)unit * (nC + 1) * 4096;
+    float* uu = uws + (size_t)unit * T * 64;
+    (void)r;
+
+    float S[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) S[i] = s0 ? s0[(size_t)unit * 4096 + i * 64 + j] : 0.f;
+
+    for (int t0 = 0; t0 < T; t0 += kTile) {
+        const int cnt = min(kTile, T - t0);
+        __syncthreads();
+        for (int tt = 0; tt < cnt; ++tt) {
+            const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
+            sm[0][tt][j] = expf(to_f32(w[row + j]));
+            sm[1][tt][j] = to_f32(k[row + j]);
+            sm[2][tt][j] = to_f32(a[row + j]);
+            sm[3][tt][j] = to_f32(b[row + j]);
+            sv[tt][j] = to_f32(v[row + j]);
+        }
+        if (j < cnt) smask[j] = mask ? (mask[(size_t)bb * T + t0 + j] != 0) : 1;
+        __syncthreads();
+        for (int tt = 0; tt < cnt; ++tt) {
+            const int p = t0 + tt;
+            if (p % kCkpt == 0) {  // the state before token p
+                float* dst = ck + (size_t)(p / kCkpt) * 4096;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) dst[i * 64 + j] = S[i];
+            }
+            if (!smask[tt]) {
+                uu[(size_t)p * 64 + j] = 0.f;
+                continue;
+            }
+            const float4* a4 = reinterpret_cast<const float4*>(sm[2][tt]);
+            float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
+#pragma unroll
+            for (int i4 = 0; i4 < 16; ++i4) {
+                const float4 av = a4[i4];
+                u0 = fmaf(S[4 * i4 + 0], av.x, u0);
+                u1 = fmaf(S[4 * i4 + 1], av.y, u1);
+                u2 = fmaf(S[4 * i4 + 2], av.z, u2);
+                u3 = fmaf(S[4 * i4 + 3], av.w, u3);
+            }
+            const float u = (u0 + u1) + (u2 + u3);
+            uu[(size_t)p * 64 + j] = u;
+            const float vj = sv[tt][j];
+            const float4* d4 = reinterpret_cast<const float4*>(sm[0][tt]);
+            const float4* k4 = reinterpret_cast<const float4*>(sm[1][tt]);
+            const float4* b4 = reinterpret_cast<const float4*>(sm[3][tt]);
+#pragma unroll
+            for (int i4 = 0; i4 < 16; ++i4) {
+                const float4 dv = d4[i4], kv = k4[i4], bv = b4[i4];
+                S[4 * i4 + 0] = fmaf(S[4 * i4 + 0], dv.x, fmaf(bv.x, u, kv.x * vj));
+                S[4 * i4 + 1] = fmaf(S[4 * i4 + 1], dv.y, fmaf(bv.y, u, kv.y * vj));
+                S[4 * i4 + 2] = fmaf(S[4 * i4 + 2], dv.z, fmaf(bv.z, u, kv.z * vj));
+                S[4 * i4 + 3] = fmaf(S[4 * i4 + 3], dv.w, fmaf(bv.w, u, kv.w * vj));
+            }
+        }
+    }
+    float* dst = ck + (size_t)nC * 4096;  // the final state
+#pragma unroll
+    for (int i = 0; i < 64; ++i) dst[i * 64 + j] = S[i];
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(64)
+bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
+           const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
+           const uint8_t* __restrict__ mask, const Tin* __restrict__ dout,
+           const float* __restrict__ dsT, const float* __restrict__ ckpt,
+           const float* __restrict__ uws, Tin* __restrict__ dr, Tin* __restrict__ dw,
+           Tin* __restrict__ dk, Tin* __restrict__ dv, Tin* __restrict__ da,
+           Tin* __restrict__ db, float* __restrict__ ds0, int T, int H) {
+    // per token of the tile: K-side r, e^{w}, e^{-w}, k, a, b; V-side v, do, u
+    __shared__ __align__(16) float sK[6][kCkpt][64];
+    __shared__ __align__(16) float sV[3][kCkpt][64];
+    __shared__ __align__(16) float sG[64 * kRow];  // G rows (one token at a time)
+    __shared__ __align__(16) float sdu[64];
+    __shared__ uint8_t smask[kCkpt];
+    const int unit = blockIdx.x;
+    const int h = unit % H, bb = unit / H;
+    const int i = threadIdx.x;  // state row
+    const int nC = (T + kCkpt - 1) / kCkpt;
+    const float* ck = ckpt + (size_t)unit * (nC + 1) * 4096;
+    const float* uu = uws + (size_t)unit * T * 64;
+
+    float S[64], G[64];
+    {
+        const float4* src = reinterpret_cast<const float4*>(ck + (size_t)nC * 4096 + i * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const float4 x = src[q];
+            S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
+        }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 64; ++jj) G[jj] = dsT ? dsT[(size_t)unit * 4096 + i * 64 + jj] : 0.f;
+
+    for (int c = nC - 1; c >= 0; --c) {
+        const int t0 = c * kCkpt, cnt = min(kCkpt, T - t0);
+        __syncthreads();  // the previous tile's reads of the stage are done
+        for (int tt = 0; tt < cnt; ++tt) {
+            const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
+            const float wv = to_f32(w[row + i]);
+            sK[0][tt][i] = to_f32(r[row + i]);
+            sK[1][tt][i] = expf(wv);
+            sK[2][tt][i] = expf(-wv);
+            sK[3][tt][i] = to_f32(k[row + i]);
+            sK[4][tt][i] = to_f32(a[row + i]);
+            sK[5][tt][i] = to_f32(b[row + i]);
+            sV[0][tt][i] = to_f32(v[row + i]);
+            sV[1][tt][i] = to_f32(dout[row + i]);
+            sV[2][tt][i] = uu[(size_t)(t0 + tt) * 64 + i];
+        }
+        if (i < cnt) smask[i] = mask ? (mask[(size_t)bb * T + t0 + i] != 0) : 1;
+        __syncthreads();
+
+        for (int tt = cnt - 1; tt >= 0; --tt) {
+            const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
+            const float ri = sK[0][tt][i];
+            const float4* do4 = reinterpret_cast<const float4*>(sV[1][tt]);
+            float dri = 0.f;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {  // G += r do^T;  dr = S_t do
+                const float4 x = do4[q];
+                G[4 * q] = fmaf(ri, x.x, G[4 * q]);
+                G[4 * q + 1] = fmaf(ri, x.y, G[4 * q + 1]);
+                G[4 * q + 2] = fmaf(ri, x.z, G[4 * q + 2]);
+                G[4 * q + 3] = fmaf(ri, x.w, G[4 * q + 3]);
+                dri = fmaf(S[4 * q], x.x, fmaf(S[4 * q + 1], x.y,
+                      fmaf(S[4 * q + 2], x.z, fmaf(S[4 * q + 3], x.w, dri))));
+            }
+            dr[row + i] = from_f32<Tin>(dri);
+            const bool upd = smask[tt] != 0;  // block-uniform
+            if (!upd) {
+                dw[row + i] = from_f32<Tin>(0.f);
+                dk[row + i] = from_f32<Tin>(0.f);
+                dv[row + i] = from_f32<Tin>(0.f);
+                da[row + i] = from_f32<Tin>(0.f);
+                db[row + i] = from_f32<Tin>(0.f);
+                if (tt == 0) {  // the state before the tile is the checkpoint (unchanged here)
+                    const float4* src = reinterpret_cast<const float4*>(ck + (size_t)c * 4096 + i * 64);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 x = src[q];
+                        S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
+                    }
+                }
+                continue;
+            }
+            // dk = G v, db = G u (row sums); G row to shared memory for the column sums
+            const float4* v4 = reinterpret_cast<const float4*>(sV[0][tt]);
+            const float4* u4 = reinterpret_cast<const float4*>(sV[2][tt]);
+            float dki = 0.f, dbi = 0.f;
+            float4* gr = reinterpret_cast<float4*>(sG + i * kRow);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const float4 xv = v4[q], xu = u4[q];
+                dki = fmaf(G[4 * q], xv.x, fmaf(G[4 * q + 1], xv.y,
+                      fmaf(G[4 * q + 2], xv.z, fmaf(G[4 * q + 3], xv.w, dki))));
+                dbi = fmaf(G[4 * q], xu.x, fmaf(G[4 * q + 1], xu.y,
+                      fmaf(G[4 * q + 2], xu.z, fmaf(G[4 * q + 3], xu.w, dbi))));
+                gr[q] = make_float4(G[4 * q], G[4 * q + 1], G[4 * q + 2], G[4 * q + 3]);
+            }
+            dk[row + i] = from_f32<Tin>(dki);
+            db[row + i] = from_f32<Tin>(dbi);
+            __syncthreads();
+            {  // thread i as column i: dv_i = sum_m G[m][i] k_m, du_i = sum_m G[m][i] b_m
+                const float* kk = sK[3][tt];
+                const float* bbv = sK[5][tt];
+                float sv0 = 0.f, sv1 = 0.f, su0 = 0.f, su1 = 0.f;
+#pragma unroll 16
+                for (int m = 0; m < 64; m += 2) {
+                    const float g0 = sG[m * kRow + i], g1 = sG[(m + 1) * kRow + i];
+                    sv0 = fmaf(g0, kk[m], sv0);
+                    sv1 = fmaf(g1, kk[m + 1], sv1);
+                    su0 = fmaf(g0, bbv[m], su0);
+                    su1 = fmaf(g1, bbv[m + 1], su1);
+                }
+                dv[row + i] = from_f32<Tin>(sv0 + sv1);
+                sdu[i] = su0 + su1;
+            }
+            __syncthreads();
+            // S becomes S_{t-1}: the checkpoint at the tile start, else rebuilt from S_t
+            if (tt == 0) {
+                const float4* src = reinterpret_cast<const float4*>(ck + (size_t)c * 4096 + i * 64);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float4 x = src[q];
+                    S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
+                }
+            } else {
+                const float ki = sK[3][tt][i], bi = sK[5][tt][i], dinv = sK[2][tt][i];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float4 xv = v4[q], xu = u4[q];
+                    S[4 * q] = (S[4 * q] - fmaf(bi, xu.x, ki * xv.x)) * dinv;
+                    S[4 * q + 1] = (S[4 * q + 1] - fmaf(bi, xu.y, ki * xv.y)) * dinv;
+                    S[4 * q + 2] = (S[4 * q + 2] - fmaf(bi, xu.z, ki * xv.z)) * dinv;
+                    S[4 * q + 3] = (S[4 * q + 3] - fmaf(bi, xu.w, ki * xv.w)) * dinv;
+                }
+            }
+            const float4* du4 = reinterpret_cast<const float4*>(sdu);
+            const float di = sK[1][tt][i], ai = sK[4][tt][i];
+            float dai = 0.f, dwi = 0.f;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const float4 x = du4[q];
+                dai = fmaf(S[4 * q], x.x, fmaf(S[4 * q + 1], x.y,
+                      fmaf(S[4 * q + 2], x.z, fmaf(S[4 * q + 3], x.w, dai))));
+                dwi = fmaf(G[4 * q], S[4 * q], fmaf(G[4 * q + 1], S[4 * q + 1],
+                      fmaf(G[4 * q + 2], S[4 * q + 2], fmaf(G[4 * q + 3], S[4 * q + 3], dwi))));
+                G[4 * q] = fmaf(di, G[4 * q], ai * x.x);
+                G[4 * q + 1] = fmaf(di, G[4 * q + 1], ai * x.y);
+                G[4 * q + 2] = fmaf(di, G[4 * q + 2], ai * x.z);
+                G[4 * q + 3] = fmaf(di, G[4 * q + 3], ai * x.w);
+            }
+            da[row + i] = from_f32<Tin>(dai);
+            dw[row + i] = from_f32<Tin>(di * dwi);
+        }
+    }
+    if (ds0) {
+        float4* dst = reinterpret_cast<float4*>(ds0 + (size_t)unit * 4096 + i * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            dst[q] = make_float4(G[4 * q], G[4 * q + 1], G[4 * q + 2], G[4 * q + 3]);
+    }
+}
+
+}  // namespace bwd
+
+template <typename Tin>
+cudaError_t launch_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
+                       const void* b, const float* s0, const uint8_t* mask, const void* dout,
+                       const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
+                       void* db, float* ds0, int B, int T, int H, float* ws,
+                       cudaStream_t stream) {
+    const long long units = (long long)B * H;
+    const long long nC = (T + bwd::kCkpt - 1) / bwd::kCkpt;
+    float* ckpt = ws;
+    float* uws = ws + (size_t)units * (nC + 1) * 4096;
+    const Tin *r_ = static_cast<const Tin*>(r), *w_ = static_cast<const Tin*>(w),
+              *k_ = static_cast<const Tin*>(k), *v_ = static_cast<const Tin*>(v),
+              *a_ = static_cast<const Tin*>(a), *b_ = static_cast<const Tin*>(b);
+    bwd::ckpt_kernel<Tin><<<(unsigned)units, 64, 0, stream>>>(r_, w_, k_, v_, a_, b_, s0, mask,
+                                                              ckpt, uws, T, H);
+    bwd::bwd_kernel<Tin><<<(unsigned)units, 64, 0, stream>>>(
+        r_, w_, k_, v_, a_, b_, mask, static_cast<const Tin*>(dout), dsT, ckpt, uws,
+        static_cast<Tin*>(dr), static_cast<Tin*>(dw), static_cast<Tin*>(dk),
+        static_cast<Tin*>(dv), static_cast<Tin*>(da), static_cast<Tin*>(db), ds0, T, H);
+    return cudaGetLastError();
+}
+
+}  // namespace wkv7

@@ -8,6 +8,7 @@
 #include "step.cuh"
 #include "recurrent.cuh"
 #include "chunked.cuh"
+#include "backward.cuh"
 
 namespace {
 
@@ -188,6 +189,48 @@ wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const voi
         dtype == WKV7_BF16
             ? wkv7::launch_step_gdn<__nv_bfloat16>(q, k, v, g, beta, state, o, units, K, stream)
             : wkv7::launch_step_gdn<float>(q, k, v, g, beta, state, o, units, K, stream);
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V) {
+    if (B < 0 || T < 0 || H <= 0 || K != 64 || V != 64) return 0;
+    return wkv7::bwd::workspace_floats((long long)B * H, T) * sizeof(float);
+}
+
+wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
+                     const void* b, const float* s0, const uint8_t* mask, const void* dout,
+                     const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
+                     void* db, float* ds0, int B, int T, int H, int K, int V,
+                     wkv7_dtype dtype, void* workspace, size_t workspace_bytes,
+                     void* stream_) {
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)B * H;
+    if (units > 0x7fffffffLL || (long long)B * T * H > (1LL << 40)) return WKV7_ERR_UNSUPPORTED;
+    if (units == 0) return WKV7_OK;
+    const bool tokens = (long long)B * T > 0;
+    if (tokens && (!ok_ptr(r) || !ok_ptr(w) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(a) ||
+                   !ok_ptr(b) || !ok_ptr(dout) || !ok_ptr(dr) || !ok_ptr(dw) || !ok_ptr(dk) ||
+                   !ok_ptr(dv) || !ok_ptr(da) || !ok_ptr(db)))
+        return WKV7_ERR_INVALID_ARG;
+    if ((s0 && !aligned16(s0)) || (dsT && !aligned16(dsT)) || (ds0 && !aligned16(ds0)))
+        return WKV7_ERR_INVALID_ARG;
+    const void* ins[8] = {r, w, k, v, a, b, dout, s0};
+    const void* outs[7] = {dr, dw, dk, dv, da, db, ds0};
+    for (const void* x : outs)
+        for (const void* y : ins)
+            if (x && x == y) return WKV7_ERR_INVALID_ARG;
+    if (!ok_ptr(workspace) || workspace_bytes < wkv7_bwd_workspace_bytes(B, T, H, K, V))
+        return WKV7_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const cudaError_t err =
+        dtype == WKV7_BF16
+            ? wkv7::launch_bwd<__nv_bfloat16>(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk,
+                                              dv, da, db, ds0, B, T, H,
+                                              static_cast<float*>(workspace), stream)
+            : wkv7::launch_bwd<float>(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da,
+                                      db, ds0, B, T, H, static_cast<float*>(workspace), stream);
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 

@@ -33,8 +33,9 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     names = declared_functions()
-    for required in ("wkv7_fwd", "wkv7_step", "wkv7_gdn_fwd", "wkv7_gdn_step",
-                     "wkv7_get_last_error", "wkv7_status_string"):
+    for required in ("wkv7_fwd", "wkv7_step", "wkv7_bwd", "wkv7_bwd_workspace_bytes",
+                     "wkv7_gdn_fwd", "wkv7_gdn_step", "wkv7_get_last_error",
+                     "wkv7_status_string"):
         assert required in names
 
 
@@ -164,3 +165,26 @@ def test_gdn_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         wkv7.wkv7_gdn_step(x[:, 0], x[:, 0], x[:, 0], s[:, 0], s[:, 0],
                            torch.zeros(1, 1, 64, 64))
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    ins = [ctypes.c_void_p(P + 0x1000 * i) for i in range(6)]
+    dout = ctypes.c_void_p(P + 0x8000)
+    outs = [ctypes.c_void_p(P + 0x10000 + 0x1000 * i) for i in range(6)]
+    ws = ctypes.c_void_p(P + 0x100000)
+    need = lib.wkv7_bwd_workspace_bytes(1, 16, 2, 64, 64)
+    assert need == 2 * ((16 // 8 + 1) * 4096 + 16 * 64) * 4
+    assert lib.wkv7_bwd_workspace_bytes(1, 16, 2, 128, 128) == 0
+
+    def call(B=1, T=16, H=2, K=64, V=64, dtype=BF16, d=dout, o=outs, w=ws, n=need):
+        return lib.wkv7_bwd(*ins, None, None, d, None, *o, None, B, T, H, K, V, dtype, w, n, None)
+
+    assert call(K=128, V=128) == ERR_UNSUPPORTED
+    assert call(H=0) == ERR_INVALID_ARG
+    assert call(dtype=4) == ERR_INVALID_ARG
+    assert call(d=None) == ERR_INVALID_ARG
+    assert call(d=ctypes.c_void_p(P + 0x8008)) == ERR_INVALID_ARG  # misaligned dout
+    assert call(o=[ins[0]] + outs[1:]) == ERR_INVALID_ARG  # dr aliases r
+    assert call(n=need - 1) == ERR_INVALID_ARG  # workspace too small
+    assert call(w=None) == ERR_INVALID_ARG
+    assert call(B=0) == OK
