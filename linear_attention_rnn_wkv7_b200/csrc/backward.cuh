@@ -30,6 +30,10 @@ namespace bwd {
 
 constexpr int kCkpt = 8;  // tokens between checkpoints (one reverse tile)
 constexpr int kRow = 68;  // padded row length of the adjoint in shared memory
+// Threads per state row in the reverse pass.  One: splitting rows over 2 or 4 lanes
+// (shorter per-thread chains, but shuffle sums on every token's chain and twice or
+// four times the warps at each barrier) measured 1.4x and 2.5x slower.
+constexpr int kRowThreads = 1;
 
 // Workspace: checkpoints [units][nC + 1][64][64] fp32, then u [units][T][64] fp32.
 inline size_t workspace_floats(long long units, int T) {
@@ -114,8 +118,17 @@ ckpt_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
     for (int i = 0; i < 64; ++i) dst[i * 64 + j] = S[i];
 }
 
-template <typename Tin>
-__global__ void __launch_bounds__(64)
+// Sum of x over the P adjacent lanes that share a state row.
+template <int P>
+__device__ __forceinline__ float row_sum(float x) {
+#pragma unroll
+    for (int m = 1; m < P; m *= 2) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+// P threads per state row (adjacent lanes), 64 / P columns each.
+template <typename Tin, int P>
+__global__ void __launch_bounds__(64 * P)
 bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
            const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
            const uint8_t* __restrict__ mask, const Tin* __restrict__ dout,
@@ -123,6 +136,7 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
            const float* __restrict__ uws, Tin* __restrict__ dr, Tin* __restrict__ dw,
            Tin* __restrict__ dk, Tin* __restrict__ dv, Tin* __restrict__ da,
            Tin* __restrict__ db, float* __restrict__ ds0, int T, int H) {
+    constexpr int NC = 64 / P;  // columns (and, for the column sums, rows) per thread
     // per token of the tile: K-side r, e^{w}, e^{-w}, k, a, b; V-side v, do, u
     __shared__ __align__(16) float sK[6][kCkpt][64];
     __shared__ __align__(16) float sV[3][kCkpt][64];
@@ -131,49 +145,56 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
     __shared__ uint8_t smask[kCkpt];
     const int unit = blockIdx.x;
     const int h = unit % H, bb = unit / H;
-    const int i = threadIdx.x;  // state row
+    const int tid = threadIdx.x;
+    const int i = tid / P, part = tid % P;  // state row; columns c0 .. c0 + NC - 1
+    const int c0 = part * NC;
     const int nC = (T + kCkpt - 1) / kCkpt;
     const float* ck = ckpt + (size_t)unit * (nC + 1) * 4096;
     const float* uu = uws + (size_t)unit * T * 64;
 
-    float S[64], G[64];
-    {
-        const float4* src = reinterpret_cast<const float4*>(ck + (size_t)nC * 4096 + i * 64);
+    float S[NC], G[NC];
+    auto load_state = [&](int slot) {
+        const float4* src = reinterpret_cast<const float4*>(ck + (size_t)slot * 4096 + i * 64 + c0);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < NC / 4; ++q) {
             const float4 x = src[q];
             S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
         }
-    }
+    };
+    load_state(nC);
 #pragma unroll
-    for (int jj = 0; jj < 64; ++jj) G[jj] = dsT ? dsT[(size_t)unit * 4096 + i * 64 + jj] : 0.f;
+    for (int jj = 0; jj < NC; ++jj)
+        G[jj] = dsT ? dsT[(size_t)unit * 4096 + i * 64 + c0 + jj] : 0.f;
 
     for (int c = nC - 1; c >= 0; --c) {
         const int t0 = c * kCkpt, cnt = min(kCkpt, T - t0);
         __syncthreads();  // the previous tile's reads of the stage are done
-        for (int tt = 0; tt < cnt; ++tt) {
-            const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
-            const float wv = to_f32(w[row + i]);
-            sK[0][tt][i] = to_f32(r[row + i]);
-            sK[1][tt][i] = expf(wv);
-            sK[2][tt][i] = expf(-wv);
-            sK[3][tt][i] = to_f32(k[row + i]);
-            sK[4][tt][i] = to_f32(a[row + i]);
-            sK[5][tt][i] = to_f32(b[row + i]);
-            sV[0][tt][i] = to_f32(v[row + i]);
-            sV[1][tt][i] = to_f32(dout[row + i]);
-            sV[2][tt][i] = uu[(size_t)(t0 + tt) * 64 + i];
+        if (tid < 64) {
+            for (int tt = 0; tt < cnt; ++tt) {
+                const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
+                const float wv = to_f32(w[row + tid]);
+                sK[0][tt][tid] = to_f32(r[row + tid]);
+                sK[1][tt][tid] = expf(wv);
+                sK[2][tt][tid] = expf(-wv);
+                sK[3][tt][tid] = to_f32(k[row + tid]);
+                sK[4][tt][tid] = to_f32(a[row + tid]);
+                sK[5][tt][tid] = to_f32(b[row + tid]);
+                sV[0][tt][tid] = to_f32(v[row + tid]);
+                sV[1][tt][tid] = to_f32(dout[row + tid]);
+                sV[2][tt][tid] = uu[(size_t)(t0 + tt) * 64 + tid];
+            }
+            if (tid < cnt) smask[tid] = mask ? (mask[(size_t)bb * T + t0 + tid] != 0) : 1;
         }
-        if (i < cnt) smask[i] = mask ? (mask[(size_t)bb * T + t0 + i] != 0) : 1;
         __syncthreads();
 
         for (int tt = cnt - 1; tt >= 0; --tt) {
             const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
+            const bool out = part == 0;  // the lane that writes row i's results
             const float ri = sK[0][tt][i];
-            const float4* do4 = reinterpret_cast<const float4*>(sV[1][tt]);
+            const float4* do4 = reinterpret_cast<const float4*>(sV[1][tt] + c0);
             float dri = 0.f;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {  // G += r do^T;  dr = S_t do
+            for (int q = 0; q < NC / 4; ++q) {  // G += r do^T;  dr = S_t do
                 const float4 x = do4[q];
                 G[4 * q] = fmaf(ri, x.x, G[4 * q]);
                 G[4 * q + 1] = fmaf(ri, x.y, G[4 * q + 1]);
@@ -182,31 +203,27 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
                 dri = fmaf(S[4 * q], x.x, fmaf(S[4 * q + 1], x.y,
                       fmaf(S[4 * q + 2], x.z, fmaf(S[4 * q + 3], x.w, dri))));
             }
-            dr[row + i] = from_f32<Tin>(dri);
+            dri = row_sum<P>(dri);
+            if (out) dr[row + i] = from_f32<Tin>(dri);
             const bool upd = smask[tt] != 0;  // block-uniform
             if (!upd) {
-                dw[row + i] = from_f32<Tin>(0.f);
-                dk[row + i] = from_f32<Tin>(0.f);
-                dv[row + i] = from_f32<Tin>(0.f);
-                da[row + i] = from_f32<Tin>(0.f);
-                db[row + i] = from_f32<Tin>(0.f);
-                if (tt == 0) {  // the state before the tile is the checkpoint (unchanged here)
-                    const float4* src = reinterpret_cast<const float4*>(ck + (size_t)c * 4096 + i * 64);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 x = src[q];
-                        S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
-                    }
+                if (out) {
+                    dw[row + i] = from_f32<Tin>(0.f);
+                    dk[row + i] = from_f32<Tin>(0.f);
+                    dv[row + i] = from_f32<Tin>(0.f);
+                    da[row + i] = from_f32<Tin>(0.f);
+                    db[row + i] = from_f32<Tin>(0.f);
                 }
+                if (tt == 0) load_state(c);  // the state before the tile (unchanged here)
                 continue;
             }
             // dk = G v, db = G u (row sums); G row to shared memory for the column sums
-            const float4* v4 = reinterpret_cast<const float4*>(sV[0][tt]);
-            const float4* u4 = reinterpret_cast<const float4*>(sV[2][tt]);
+            const float4* v4 = reinterpret_cast<const float4*>(sV[0][tt] + c0);
+            const float4* u4 = reinterpret_cast<const float4*>(sV[2][tt] + c0);
             float dki = 0.f, dbi = 0.f;
-            float4* gr = reinterpret_cast<float4*>(sG + i * kRow);
+            float4* gr = reinterpret_cast<float4*>(sG + i * kRow + c0);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
+            for (int q = 0; q < NC / 4; ++q) {
                 const float4 xv = v4[q], xu = u4[q];
                 dki = fmaf(G[4 * q], xv.x, fmaf(G[4 * q + 1], xv.y,
                       fmaf(G[4 * q + 2], xv.z, fmaf(G[4 * q + 3], xv.w, dki))));
@@ -214,37 +231,39 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
                       fmaf(G[4 * q + 2], xu.z, fmaf(G[4 * q + 3], xu.w, dbi))));
                 gr[q] = make_float4(G[4 * q], G[4 * q + 1], G[4 * q + 2], G[4 * q + 3]);
             }
-            dk[row + i] = from_f32<Tin>(dki);
-            db[row + i] = from_f32<Tin>(dbi);
+            dki = row_sum<P>(dki);
+            dbi = row_sum<P>(dbi);
+            if (out) {
+                dk[row + i] = from_f32<Tin>(dki);
+                db[row + i] = from_f32<Tin>(dbi);
+            }
             __syncthreads();
-            {  // thread i as column i: dv_i = sum_m G[m][i] k_m, du_i = sum_m G[m][i] b_m
+            {  // as column i over rows c0 .. c0 + NC - 1: dv_i = sum_m G[m][i] k_m, du_i = G^T b
                 const float* kk = sK[3][tt];
                 const float* bbv = sK[5][tt];
                 float sv0 = 0.f, sv1 = 0.f, su0 = 0.f, su1 = 0.f;
-#pragma unroll 16
-                for (int m = 0; m < 64; m += 2) {
+#pragma unroll
+                for (int m = c0; m < c0 + NC; m += 2) {
                     const float g0 = sG[m * kRow + i], g1 = sG[(m + 1) * kRow + i];
                     sv0 = fmaf(g0, kk[m], sv0);
                     sv1 = fmaf(g1, kk[m + 1], sv1);
                     su0 = fmaf(g0, bbv[m], su0);
                     su1 = fmaf(g1, bbv[m + 1], su1);
                 }
-                dv[row + i] = from_f32<Tin>(sv0 + sv1);
-                sdu[i] = su0 + su1;
+                const float dvi = row_sum<P>(sv0 + sv1), dui = row_sum<P>(su0 + su1);
+                if (out) {
+                    dv[row + i] = from_f32<Tin>(dvi);
+                    sdu[i] = dui;
+                }
             }
             __syncthreads();
             // S becomes S_{t-1}: the checkpoint at the tile start, else rebuilt from S_t
             if (tt == 0) {
-                const float4* src = reinterpret_cast<const float4*>(ck + (size_t)c * 4096 + i * 64);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float4 x = src[q];
-                    S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
-                }
+                load_state(c);
             } else {
                 const float ki = sK[3][tt][i], bi = sK[5][tt][i], dinv = sK[2][tt][i];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
+                for (int q = 0; q < NC / 4; ++q) {
                     const float4 xv = v4[q], xu = u4[q];
                     S[4 * q] = (S[4 * q] - fmaf(bi, xu.x, ki * xv.x)) * dinv;
                     S[4 * q + 1] = (S[4 * q + 1] - fmaf(bi, xu.y, ki * xv.y)) * dinv;
@@ -252,11 +271,11 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
                     S[4 * q + 3] = (S[4 * q + 3] - fmaf(bi, xu.w, ki * xv.w)) * dinv;
                 }
             }
-            const float4* du4 = reinterpret_cast<const float4*>(sdu);
+            const float4* du4 = reinterpret_cast<const float4*>(sdu + c0);
             const float di = sK[1][tt][i], ai = sK[4][tt][i];
             float dai = 0.f, dwi = 0.f;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
+            for (int q = 0; q < NC / 4; ++q) {
                 const float4 x = du4[q];
                 dai = fmaf(S[4 * q], x.x, fmaf(S[4 * q + 1], x.y,
                       fmaf(S[4 * q + 2], x.z, fmaf(S[4 * q + 3], x.w, dai))));
@@ -267,14 +286,18 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
                 G[4 * q + 2] = fmaf(di, G[4 * q + 2], ai * x.z);
                 G[4 * q + 3] = fmaf(di, G[4 * q + 3], ai * x.w);
             }
-            da[row + i] = from_f32<Tin>(dai);
-            dw[row + i] = from_f32<Tin>(di * dwi);
+            dai = row_sum<P>(dai);
+            dwi = row_sum<P>(dwi);
+            if (out) {
+                da[row + i] = from_f32<Tin>(dai);
+                dw[row + i] = from_f32<Tin>(di * dwi);
+            }
         }
     }
     if (ds0) {
-        float4* dst = reinterpret_cast<float4*>(ds0 + (size_t)unit * 4096 + i * 64);
+        float4* dst = reinterpret_cast<float4*>(ds0 + (size_t)unit * 4096 + i * 64 + c0);
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
+        for (int q = 0; q < NC / 4; ++q)
             dst[q] = make_float4(G[4 * q], G[4 * q + 1], G[4 * q + 2], G[4 * q + 3]);
     }
 }
@@ -296,7 +319,7 @@ cudaError_t launch_bwd(const void* r, const void* w, const void* k, const void* 
               *a_ = static_cast<const Tin*>(a), *b_ = static_cast<const Tin*>(b);
     bwd::ckpt_kernel<Tin><<<(unsigned)units, 64, 0, stream>>>(r_, w_, k_, v_, a_, b_, s0, mask,
                                                               ckpt, uws, T, H);
-    bwd::bwd_kernel<Tin><<<(unsigned)units, 64, 0, stream>>>(
+    bwd::bwd_kernel<Tin, bwd::kRowThreads><<<(unsigned)units, 64 * bwd::kRowThreads, 0, stream>>>(
         r_, w_, k_, v_, a_, b_, mask, static_cast<const Tin*>(dout), dsT, ckpt, uws,
         static_cast<Tin*>(dr), static_cast<Tin*>(dw), static_cast<Tin*>(dk),
         static_cast<Tin*>(dv), static_cast<Tin*>(da), static_cast<Tin*>(db), ds0, T, H);
