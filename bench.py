@@ -497,8 +497,8 @@ def bwd_leg(args, device, stream, wkv7_bwd, hbm_peak, peak_kind, max_over_ranks,
 
 
 def wkv7_bwd_workspace_nbytes(B, T, H):
-    from linear_attention_rnn_wkv7_b200 import library
-    return int(library().wkv7_bwd_workspace_bytes(B, T, H, 64, 64))
+    from linear_attention_rnn_wkv7_b200.wkv7 import wkv7_bwd_workspace_bytes
+    return wkv7_bwd_workspace_bytes(B, T, H)
 
 
 def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank,

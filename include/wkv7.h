@@ -137,13 +137,13 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
  *     dw_t = e^{w_t} * rowsum(G * S_{t-1});  G <- diag(e^{w_t}) G + a_t du_t^T;
  *     ds0 = G after the first token.
  *
- *   r, w, k, v, a, b, s0, mask   as for wkv7_fwd ([B, T, H, 64], token-major, no varlen)
- *   dout           [B, T, H, V]  dtype   dL/do (required)
- *   dsT            [B, H, K, V]  fp32    dL/dS_T, or NULL for zero
- *   dr, dw, dk, da, db [B, T, H, K], dv [B, T, H, V]   dtype   outputs (fully written;
+ *   r, w, k, v, a, b, s0, mask, cu_seqlens, N, layout   as for wkv7_fwd (K = V = 64)
+ *   dout           shaped like v dtype   dL/do (required)
+ *   dsT            [N, H, K, V]  fp32    dL/dS_T, or NULL for zero
+ *   dr, dw, dk, da, db (shaped like r), dv (like v)   dtype   outputs (fully written;
  *                                        must not alias an input)
- *   ds0            [B, H, K, V]  fp32    dL/ds0, or NULL to skip
- *   workspace      device buffer of at least wkv7_bwd_workspace_bytes(B, T, H, K, V)
+ *   ds0            [N, H, K, V]  fp32    dL/ds0, or NULL to skip
+ *   workspace      device buffer of at least wkv7_bwd_workspace_bytes(B, T, H, K, V, N)
  *                  bytes (16-byte aligned; the caller owns it): the forward states
  *                  every 8 tokens and every token's u = S_{t-1}^T a, recomputed here
  *
@@ -151,13 +151,14 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
  * dw, dk, dv, da, db.  Two kernels on `stream`: a forward that writes the
  * checkpoints, then the reverse pass.
  */
-size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V);
+size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N);
 
 wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
                      const void* b, const float* s0, const uint8_t* mask, const void* dout,
                      const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
                      void* db, float* ds0, int B, int T, int H, int K, int V,
-                     wkv7_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+                     const int32_t* cu_seqlens, int N, wkv7_layout layout, wkv7_dtype dtype,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * wkv7_gdn_fwd -- Gated DeltaNet forward over whole sequences

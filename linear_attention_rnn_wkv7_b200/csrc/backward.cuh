@@ -35,10 +35,40 @@ constexpr int kRow = 68;  // padded row length of the adjoint in shared memory
 // four times the warps at each barrier) measured 1.4x and 2.5x slower.
 constexpr int kRowThreads = 1;
 
-// Workspace: checkpoints [units][nC + 1][64][64] fp32, then u [units][T][64] fp32.
-inline size_t workspace_floats(long long units, int T) {
-    const long long nC = (T + kCkpt - 1) / kCkpt;
-    return (size_t)units * ((size_t)(nC + 1) * 4096 + (size_t)T * 64);
+// Workspace, fp32: checkpoints [slots][H][64][64] (the heads of one slot side by
+// side, so the blocks writing checkpoints at the same time write neighbouring 16 KB
+// blocks), then u [H][B*T token rows][64].
+// Sequence n (packed rows [bos_n, eos_n)) of head h keeps its ceil(L/kCkpt) + 1
+// checkpoints from slot floor(bos_n / kCkpt) + 2 n on; these ranges never overlap
+// (floor((bos + L) / 8) + 1 >= floor(bos / 8) + ceil(L / 8)), so
+// slots = floor(B*T / kCkpt) + 2 N + 1 per head covers every layout and length mix.
+inline long long ckpt_slots(long long rows, int N) { return rows / kCkpt + 2LL * N + 1; }
+inline size_t workspace_floats(long long rows, int N, int H) {
+    return (size_t)H * ckpt_slots(rows, N) * 4096 + (size_t)rows * H * 64;
+}
+
+// The unit's sequence: packed rows [bos, eos) of batch row bb, and its first slot.
+struct Seq {
+    int bb, bos, eos;
+    long long slot0;
+    bool ok;
+};
+__device__ __forceinline__ Seq unit_seq(int n, int T, const int32_t* cu_seqlens) {
+    Seq q;
+    if (cu_seqlens) {
+        q.bb = 0;
+        q.bos = cu_seqlens[n];
+        q.eos = cu_seqlens[n + 1];
+        q.ok = q.bos >= 0 && q.eos >= q.bos && q.eos <= T;
+        q.slot0 = (long long)q.bos / kCkpt + 2LL * n;
+    } else {
+        q.bb = n;
+        q.bos = 0;
+        q.eos = T;
+        q.ok = true;
+        q.slot0 = (long long)n * T / kCkpt + 2LL * n;
+    }
+    return q;
 }
 
 template <typename Tin>
@@ -46,40 +76,66 @@ __global__ void __launch_bounds__(64)
 ckpt_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
             const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
             const float* __restrict__ s0, const uint8_t* __restrict__ mask,
-            float* __restrict__ ckpt, float* __restrict__ uws, int T, int H) {
+            float* __restrict__ ckpt, float* __restrict__ uws, int T, int H, int N,
+            const int32_t* __restrict__ cu_seqlens, int head_first, long long slots) {
     constexpr int kTile = 16;
     __shared__ __align__(16) float sm[4][kTile][64];  // d = exp(w), k, a, b
     __shared__ float sv[kTile][64];
     __shared__ uint8_t smask[kTile];
     const int unit = blockIdx.x;
-    const int h = unit % H, bb = unit / H;
+    const int h = unit % H, n = unit / H;
     const int j = threadIdx.x;
-    const int nC = (T + kCkpt - 1) / kCkpt;
-    float* ck = ckpt + (size_t)unit * (nC + 1) * 4096;
-    float* uu = uws + (size_t)unit * T * 64;
+    const Seq sq = unit_seq(n, T, cu_seqlens);
+    if (!sq.ok) {  // block-uniform; reported by the reverse pass
+        return;
+    }
+    const int L = sq.eos - sq.bos;
+    const long long rows = cu_seqlens ? (long long)T : (long long)N * T;
+    // token p of the unit: row tb + p * ts of the inputs; u row bb*T + bos + p of head h
+    const size_t tb = head_first ? ((size_t)sq.bb * H + h) * T + sq.bos
+                                 : ((size_t)sq.bb * T + sq.bos) * H + h;
+    const size_t ts = head_first ? 1 : (size_t)H;
+    float* ck = ckpt + ((size_t)sq.slot0 * H + h) * 4096;
+    float* uu = uws + ((size_t)h * rows + (size_t)sq.bb * T + sq.bos) * 64;
     (void)r;
 
     float S[64];
 #pragma unroll
     for (int i = 0; i < 64; ++i) S[i] = s0 ? s0[(size_t)unit * 4096 + i * 64 + j] : 0.f;
 
-    for (int t0 = 0; t0 < T; t0 += kTile) {
-        const int cnt = min(kTile, T - t0);
+    for (int t0 = 0; t0 < L; t0 += kTile) {
+        const int cnt = min(kTile, L - t0);
         __syncthreads();
-        for (int tt = 0; tt < cnt; ++tt) {
-            const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
-            sm[0][tt][j] = expf(to_f32(w[row + j]));
-            sm[1][tt][j] = to_f32(k[row + j]);
-            sm[2][tt][j] = to_f32(a[row + j]);
-            sm[3][tt][j] = to_f32(b[row + j]);
-            sv[tt][j] = to_f32(v[row + j]);
+        {  // every load of the tile is issued before the first store (one latency per tile)
+            float xw[kTile], xk[kTile], xa[kTile], xb[kTile], xv[kTile];
+#pragma unroll
+            for (int tt = 0; tt < kTile; ++tt) {
+                if (tt < cnt) {
+                    const size_t row = (tb + (size_t)(t0 + tt) * ts) * 64;
+                    xw[tt] = to_f32(w[row + j]);
+                    xk[tt] = to_f32(k[row + j]);
+                    xa[tt] = to_f32(a[row + j]);
+                    xb[tt] = to_f32(b[row + j]);
+                    xv[tt] = to_f32(v[row + j]);
+                }
+            }
+#pragma unroll
+            for (int tt = 0; tt < kTile; ++tt) {
+                if (tt < cnt) {
+                    sm[0][tt][j] = expf(xw[tt]);
+                    sm[1][tt][j] = xk[tt];
+                    sm[2][tt][j] = xa[tt];
+                    sm[3][tt][j] = xb[tt];
+                    sv[tt][j] = xv[tt];
+                }
+            }
         }
-        if (j < cnt) smask[j] = mask ? (mask[(size_t)bb * T + t0 + j] != 0) : 1;
+        if (j < cnt) smask[j] = mask ? (mask[(size_t)sq.bb * T + sq.bos + t0 + j] != 0) : 1;
         __syncthreads();
         for (int tt = 0; tt < cnt; ++tt) {
             const int p = t0 + tt;
             if (p % kCkpt == 0) {  // the state before token p
-                float* dst = ck + (size_t)(p / kCkpt) * 4096;
+                float* dst = ck + (size_t)(p / kCkpt) * H * 4096;
 #pragma unroll
                 for (int i = 0; i < 64; ++i) dst[i * 64 + j] = S[i];
             }
@@ -113,7 +169,7 @@ ckpt_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
             }
         }
     }
-    float* dst = ck + (size_t)nC * 4096;  // the final state
+    float* dst = ck + (size_t)((L + kCkpt - 1) / kCkpt) * H * 4096;  // the final state
 #pragma unroll
     for (int i = 0; i < 64; ++i) dst[i * 64 + j] = S[i];
 }
@@ -135,7 +191,8 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
            const float* __restrict__ dsT, const float* __restrict__ ckpt,
            const float* __restrict__ uws, Tin* __restrict__ dr, Tin* __restrict__ dw,
            Tin* __restrict__ dk, Tin* __restrict__ dv, Tin* __restrict__ da,
-           Tin* __restrict__ db, float* __restrict__ ds0, int T, int H) {
+           Tin* __restrict__ db, float* __restrict__ ds0, int T, int H, int N,
+           const int32_t* __restrict__ cu_seqlens, int head_first, long long slots) {
     constexpr int NC = 64 / P;  // columns (and, for the column sums, rows) per thread
     // per token of the tile: K-side r, e^{w}, e^{-w}, k, a, b; V-side v, do, u
     __shared__ __align__(16) float sK[6][kCkpt][64];
@@ -144,17 +201,27 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
     __shared__ __align__(16) float sdu[64];
     __shared__ uint8_t smask[kCkpt];
     const int unit = blockIdx.x;
-    const int h = unit % H, bb = unit / H;
+    const int h = unit % H, n = unit / H;
     const int tid = threadIdx.x;
     const int i = tid / P, part = tid % P;  // state row; columns c0 .. c0 + NC - 1
     const int c0 = part * NC;
-    const int nC = (T + kCkpt - 1) / kCkpt;
-    const float* ck = ckpt + (size_t)unit * (nC + 1) * 4096;
-    const float* uu = uws + (size_t)unit * T * 64;
+    const Seq sq = unit_seq(n, T, cu_seqlens);
+    if (!sq.ok) {  // block-uniform: the sequence is skipped and reported
+        if (tid == 0) raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
+        return;
+    }
+    const int L = sq.eos - sq.bos;
+    const int nC = (L + kCkpt - 1) / kCkpt;
+    const size_t tb = head_first ? ((size_t)sq.bb * H + h) * T + sq.bos
+                                 : ((size_t)sq.bb * T + sq.bos) * H + h;
+    const size_t ts = head_first ? 1 : (size_t)H;
+    const float* ck = ckpt + ((size_t)sq.slot0 * H + h) * 4096;
+    const long long rows = cu_seqlens ? (long long)T : (long long)N * T;
+    const float* uu = uws + ((size_t)h * rows + (size_t)sq.bb * T + sq.bos) * 64;
 
     float S[NC], G[NC];
     auto load_state = [&](int slot) {
-        const float4* src = reinterpret_cast<const float4*>(ck + (size_t)slot * 4096 + i * 64 + c0);
+        const float4* src = reinterpret_cast<const float4*>(ck + (size_t)slot * H * 4096 + i * 64 + c0);
 #pragma unroll
         for (int q = 0; q < NC / 4; ++q) {
             const float4 x = src[q];
@@ -167,28 +234,44 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
         G[jj] = dsT ? dsT[(size_t)unit * 4096 + i * 64 + c0 + jj] : 0.f;
 
     for (int c = nC - 1; c >= 0; --c) {
-        const int t0 = c * kCkpt, cnt = min(kCkpt, T - t0);
+        const int t0 = c * kCkpt, cnt = min(kCkpt, L - t0);
         __syncthreads();  // the previous tile's reads of the stage are done
-        if (tid < 64) {
-            for (int tt = 0; tt < cnt; ++tt) {
-                const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
-                const float wv = to_f32(w[row + tid]);
-                sK[0][tt][tid] = to_f32(r[row + tid]);
-                sK[1][tt][tid] = expf(wv);
-                sK[2][tt][tid] = expf(-wv);
-                sK[3][tt][tid] = to_f32(k[row + tid]);
-                sK[4][tt][tid] = to_f32(a[row + tid]);
-                sK[5][tt][tid] = to_f32(b[row + tid]);
-                sV[0][tt][tid] = to_f32(v[row + tid]);
-                sV[1][tt][tid] = to_f32(dout[row + tid]);
-                sV[2][tt][tid] = uu[(size_t)(t0 + tt) * 64 + tid];
+        if (tid < 64) {  // every load of the tile is issued before the first store
+            float x[8][kCkpt];
+#pragma unroll
+            for (int tt = 0; tt < kCkpt; ++tt) {
+                if (tt < cnt) {
+                    const size_t row = (tb + (size_t)(t0 + tt) * ts) * 64;
+                    x[0][tt] = to_f32(r[row + tid]);
+                    x[1][tt] = to_f32(w[row + tid]);
+                    x[2][tt] = to_f32(k[row + tid]);
+                    x[3][tt] = to_f32(a[row + tid]);
+                    x[4][tt] = to_f32(b[row + tid]);
+                    x[5][tt] = to_f32(v[row + tid]);
+                    x[6][tt] = to_f32(dout[row + tid]);
+                    x[7][tt] = uu[(size_t)(t0 + tt) * 64 + tid];
+                }
             }
-            if (tid < cnt) smask[tid] = mask ? (mask[(size_t)bb * T + t0 + tid] != 0) : 1;
+#pragma unroll
+            for (int tt = 0; tt < kCkpt; ++tt) {
+                if (tt < cnt) {
+                    sK[0][tt][tid] = x[0][tt];
+                    sK[1][tt][tid] = expf(x[1][tt]);
+                    sK[2][tt][tid] = expf(-x[1][tt]);
+                    sK[3][tt][tid] = x[2][tt];
+                    sK[4][tt][tid] = x[3][tt];
+                    sK[5][tt][tid] = x[4][tt];
+                    sV[0][tt][tid] = x[5][tt];
+                    sV[1][tt][tid] = x[6][tt];
+                    sV[2][tt][tid] = x[7][tt];
+                }
+            }
+            if (tid < cnt) smask[tid] = mask ? (mask[(size_t)sq.bb * T + sq.bos + t0 + tid] != 0) : 1;
         }
         __syncthreads();
 
         for (int tt = cnt - 1; tt >= 0; --tt) {
-            const size_t row = (((size_t)bb * T + t0 + tt) * H + h) * 64;
+            const size_t row = (tb + (size_t)(t0 + tt) * ts) * 64;
             const bool out = part == 0;  // the lane that writes row i's results
             const float ri = sK[0][tt][i];
             const float4* do4 = reinterpret_cast<const float4*>(sV[1][tt] + c0);
@@ -308,21 +391,25 @@ template <typename Tin>
 cudaError_t launch_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
                        const void* b, const float* s0, const uint8_t* mask, const void* dout,
                        const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
-                       void* db, float* ds0, int B, int T, int H, float* ws,
+                       void* db, float* ds0, int B, int T, int H, int N,
+                       const int32_t* cu_seqlens, int head_first, float* ws,
                        cudaStream_t stream) {
-    const long long units = (long long)B * H;
-    const long long nC = (T + bwd::kCkpt - 1) / bwd::kCkpt;
+    const long long units = (long long)N * H;
+    const long long rows = (long long)B * T;
+    const long long slots = bwd::ckpt_slots(rows, N);
     float* ckpt = ws;
-    float* uws = ws + (size_t)units * (nC + 1) * 4096;
+    float* uws = ws + (size_t)H * slots * 4096;
     const Tin *r_ = static_cast<const Tin*>(r), *w_ = static_cast<const Tin*>(w),
               *k_ = static_cast<const Tin*>(k), *v_ = static_cast<const Tin*>(v),
               *a_ = static_cast<const Tin*>(a), *b_ = static_cast<const Tin*>(b);
     bwd::ckpt_kernel<Tin><<<(unsigned)units, 64, 0, stream>>>(r_, w_, k_, v_, a_, b_, s0, mask,
-                                                              ckpt, uws, T, H);
+                                                              ckpt, uws, T, H, N, cu_seqlens,
+                                                              head_first, slots);
     bwd::bwd_kernel<Tin, bwd::kRowThreads><<<(unsigned)units, 64 * bwd::kRowThreads, 0, stream>>>(
         r_, w_, k_, v_, a_, b_, mask, static_cast<const Tin*>(dout), dsT, ckpt, uws,
         static_cast<Tin*>(dr), static_cast<Tin*>(dw), static_cast<Tin*>(dk),
-        static_cast<Tin*>(dv), static_cast<Tin*>(da), static_cast<Tin*>(db), ds0, T, H);
+        static_cast<Tin*>(dv), static_cast<Tin*>(da), static_cast<Tin*>(db), ds0, T, H, N,
+        cu_seqlens, head_first, slots);
     return cudaGetLastError();
 }
 

@@ -192,21 +192,28 @@ wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const voi
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 
-size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V) {
-    if (B < 0 || T < 0 || H <= 0 || K != 64 || V != 64) return 0;
-    return wkv7::bwd::workspace_floats((long long)B * H, T) * sizeof(float);
+size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N) {
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || K != 64 || V != 64) return 0;
+    return wkv7::bwd::workspace_floats((long long)B * T, N, H) * sizeof(float);
 }
 
 wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
                      const void* b, const float* s0, const uint8_t* mask, const void* dout,
                      const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
                      void* db, float* ds0, int B, int T, int H, int K, int V,
-                     wkv7_dtype dtype, void* workspace, size_t workspace_bytes,
-                     void* stream_) {
-    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
+                     const int32_t* cu_seqlens, int N, wkv7_layout layout, wkv7_dtype dtype,
+                     void* workspace, size_t workspace_bytes, void* stream_) {
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0 || N < 0) return WKV7_ERR_INVALID_ARG;
     if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (layout != WKV7_LAYOUT_BTHK && layout != WKV7_LAYOUT_BHTK) return WKV7_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (B != 1) return WKV7_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return WKV7_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return WKV7_ERR_INVALID_ARG;
+    }
     if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
-    const long long units = (long long)B * H;
+    const long long units = (long long)N * H;
     if (units > 0x7fffffffLL || (long long)B * T * H > (1LL << 40)) return WKV7_ERR_UNSUPPORTED;
     if (units == 0) return WKV7_OK;
     const bool tokens = (long long)B * T > 0;
@@ -221,16 +228,18 @@ wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v,
     for (const void* x : outs)
         for (const void* y : ins)
             if (x && x == y) return WKV7_ERR_INVALID_ARG;
-    if (!ok_ptr(workspace) || workspace_bytes < wkv7_bwd_workspace_bytes(B, T, H, K, V))
+    if (!ok_ptr(workspace) || workspace_bytes < wkv7_bwd_workspace_bytes(B, T, H, K, V, N))
         return WKV7_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const int hf = layout == WKV7_LAYOUT_BHTK;
     const cudaError_t err =
         dtype == WKV7_BF16
             ? wkv7::launch_bwd<__nv_bfloat16>(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk,
-                                              dv, da, db, ds0, B, T, H,
+                                              dv, da, db, ds0, B, T, H, N, cu_seqlens, hf,
                                               static_cast<float*>(workspace), stream)
             : wkv7::launch_bwd<float>(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da,
-                                      db, ds0, B, T, H, static_cast<float*>(workspace), stream);
+                                      db, ds0, B, T, H, N, cu_seqlens, hf,
+                                      static_cast<float*>(workspace), stream);
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 

@@ -50,9 +50,9 @@ def library() -> ctypes.CDLL:
         lib.wkv7_step.restype = i
         lib.wkv7_step.argtypes = [p, p, p, p, p, p, p, p, i, i, i, i, i, p]
         lib.wkv7_bwd_workspace_bytes.restype = ctypes.c_size_t
-        lib.wkv7_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+        lib.wkv7_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
         lib.wkv7_bwd.restype = i
-        lib.wkv7_bwd.argtypes = [p] * 17 + [i, i, i, i, i, i, p, ctypes.c_size_t, p]
+        lib.wkv7_bwd.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i, i, p, ctypes.c_size_t, p]
         lib.wkv7_gdn_fwd.restype = i
         lib.wkv7_gdn_fwd.argtypes = [p, p, p, p, p, p, i, p, p, i, i, i, i, i, p, i, i, i, i, p]
         lib.wkv7_gdn_step.restype = i
@@ -168,40 +168,56 @@ def wkv7_step(r, w, k, v, a, b, state, o=None):
     return o
 
 
-def wkv7_bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, workspace=None):
+def wkv7_bwd_workspace_bytes(B, T, H, K=64, V=64, N=None) -> int:
+    return int(library().wkv7_bwd_workspace_bytes(B, T, H, K, V, B if N is None else N))
+
+
+def wkv7_bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=None,
+             head_first: bool = False, workspace=None):
     """Backward of wkv7_fwd for L = sum(o * dout) + sum(S_T * dsT).  Inputs as for
-    wkv7_fwd (token-major, no varlen); dout [B,T,H,V]; dsT [B,H,K,V] fp32 or None.
-    Returns a dict: dr, dw, dk, dv, da, db (input dtype) and ds0 (fp32).  The
-    workspace (uint8 device tensor of at least wkv7_bwd_workspace_bytes) is
-    allocated here when not given."""
+    wkv7_fwd (K = V = 64); dout shaped like v; dsT [N,H,K,V] fp32 or None.
+    Returns a dict: dr, dw, dk, dv, da, db (input dtype, shaped like the inputs) and
+    ds0 (fp32 [N,H,K,V]).  The workspace (uint8 device tensor of at least
+    wkv7_bwd_workspace_bytes) is allocated here when not given."""
     _check(r, "r")
     dt = r.dtype
-    B, T, H, K = r.shape
+    if head_first:
+        B, H, T, K = r.shape
+    else:
+        B, T, H, K = r.shape
     V = v.shape[-1]
+    kshape = (B, H, T, K) if head_first else (B, T, H, K)
+    vshape = (B, H, T, V) if head_first else (B, T, H, V)
     for name, t in (("w", w), ("k", k), ("a", a), ("b", b)):
-        _check(t, name, dt, (B, T, H, K))
-    _check(v, "v", dt, (B, T, H, V))
-    _check(dout, "dout", dt, (B, T, H, V))
+        _check(t, name, dt, kshape)
+    _check(v, "v", dt, vshape)
+    _check(dout, "dout", dt, vshape)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
     if s0 is not None:
-        _check(s0, "s0", torch.float32, (B, H, K, V))
+        _check(s0, "s0", torch.float32, (N, H, K, V))
     if dsT is not None:
-        _check(dsT, "dsT", torch.float32, (B, H, K, V))
+        _check(dsT, "dsT", torch.float32, (N, H, K, V))
     if mask is not None:
         if mask.dtype == torch.bool:
             mask = mask.to(torch.uint8)
         _check(mask, "mask", torch.uint8, (B, T))
-    nbytes = library().wkv7_bwd_workspace_bytes(B, T, H, K, V)
+    nbytes = wkv7_bwd_workspace_bytes(B, T, H, K, V, N)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=r.device)
     else:
         _check(workspace, "workspace", torch.uint8)
-    g = {n: torch.empty((B, T, H, K), dtype=dt, device=r.device) for n in ("dr", "dw", "dk", "da", "db")}
-    g["dv"] = torch.empty((B, T, H, V), dtype=dt, device=r.device)
-    g["ds0"] = torch.empty((B, H, K, V), dtype=torch.float32, device=r.device)
+    g = {n: torch.empty(kshape, dtype=dt, device=r.device) for n in ("dr", "dw", "dk", "da", "db")}
+    g["dv"] = torch.empty(vshape, dtype=dt, device=r.device)
+    g["ds0"] = torch.empty((N, H, K, V), dtype=torch.float32, device=r.device)
     st = library().wkv7_bwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0),
                             _ptr(mask), _ptr(dout), _ptr(dsT), _ptr(g["dr"]), _ptr(g["dw"]),
                             _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["db"]),
-                            _ptr(g["ds0"]), B, T, H, K, V, _dtype_code(r), _ptr(workspace),
+                            _ptr(g["ds0"]), B, T, H, K, V, _ptr(cu_seqlens), N,
+                            int(bool(head_first)), _dtype_code(r), _ptr(workspace),
                             workspace.numel(), _stream(r.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_bwd")
@@ -213,25 +229,30 @@ class GeneralizedDeltaRule(torch.autograd.Function):
     through wkv7_bwd (token-major inputs, K = V = 64, no varlen)."""
 
     @staticmethod
-    def forward(ctx, r, w, k, v, a, b, s0, mask):
-        o, sT = wkv7_fwd(r, w, k, v, a, b, s0=s0, mask=mask)
-        ctx.save_for_backward(r, w, k, v, a, b, s0, mask)
+    def forward(ctx, r, w, k, v, a, b, s0, mask, cu_seqlens, head_first):
+        o, sT = wkv7_fwd(r, w, k, v, a, b, s0=s0, mask=mask, cu_seqlens=cu_seqlens,
+                         head_first=head_first)
+        ctx.save_for_backward(r, w, k, v, a, b, s0, mask, cu_seqlens)
+        ctx.head_first = head_first
         return o, sT
 
     @staticmethod
     def backward(ctx, do, dsT):
-        r, w, k, v, a, b, s0, mask = ctx.saved_tensors
-        do = torch.zeros_like(r[..., :v.shape[-1]]) if do is None else do.contiguous()
+        r, w, k, v, a, b, s0, mask, cu_seqlens = ctx.saved_tensors
+        do = torch.zeros_like(v) if do is None else do.contiguous()
         dsT = None if dsT is None else dsT.contiguous().float()
-        g = wkv7_bwd(r, w, k, v, a, b, do.to(r.dtype), s0=s0, mask=mask, dsT=dsT)
+        g = wkv7_bwd(r, w, k, v, a, b, do.to(r.dtype), s0=s0, mask=mask, dsT=dsT,
+                     cu_seqlens=cu_seqlens, head_first=ctx.head_first)
         ds0 = g["ds0"] if s0 is not None else None
-        return g["dr"], g["dw"], g["dk"], g["dv"], g["da"], g["db"], ds0, None
+        return g["dr"], g["dw"], g["dk"], g["dv"], g["da"], g["db"], ds0, None, None, None
 
 
 def generalized_delta_rule(r, w, k, v, a, b, initial_state=None, output_final_state=True,
-                           mask=None):
-    """Differentiable forward (README: generalized_delta_rule); returns (o, final state or None)."""
-    o, sT = GeneralizedDeltaRule.apply(r, w, k, v, a, b, initial_state, mask)
+                           mask=None, cu_seqlens=None, head_first: bool = False):
+    """Differentiable forward (README: generalized_delta_rule); returns (o, final state or
+    None).  Backward through wkv7_bwd."""
+    o, sT = GeneralizedDeltaRule.apply(r, w, k, v, a, b, initial_state, mask, cu_seqlens,
+                                       head_first)
     return o, (sT if output_final_state else None)
 
 

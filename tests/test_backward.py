@@ -116,3 +116,36 @@ def test_bwd_rejects_small_workspace(cuda_device):
     with pytest.raises(WKV7Error) as e:
         wkv7_bwd(*(x[n] for n in NAMES), dout, workspace=ws)
     assert e.value.status == ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("head_first", [False, True])
+def test_bwd_varlen(cuda_device, head_first):
+    """Packed sequences (lengths 0 … 130, checkpoint boundaries inside and at the ends)
+    with per-sequence s0 and dL/dS_T, token-major and head-first."""
+    lengths = torch.tensor([17, 0, 8, 1, 130, 63])
+    x = synth.varlen_inputs(lengths, 2, dtype=torch.float32, seed=650, s0_std=0.1)
+    cu = x.pop("cu_seqlens")
+    total, N = int(lengths.sum()), lengths.numel()
+    dout, _ = upstream(1, total, 2, torch.float32, 651)
+    dsT = torch.randn(N, 2, 64, 64, generator=torch.Generator().manual_seed(652)) * 0.1
+    ref = oracle.bwd(*(x[n] for n in NAMES), dout, s0=x["s0"], dsT=dsT, cu_seqlens=cu)
+    xd = to_dev(x, cuda_device)
+    lay = (lambda t: t.transpose(1, 2).contiguous()) if head_first else (lambda t: t)
+    g = wkv7_bwd(*(lay(xd[n]) for n in NAMES), lay(dout.to(cuda_device)), s0=xd["s0"],
+                 dsT=dsT.to(cuda_device), cu_seqlens=cu.to(cuda_device), head_first=head_first)
+    if head_first:
+        g = {n: (t.transpose(1, 2) if n != "ds0" else t) for n, t in g.items()}
+    check_grads(g, ref, torch.float32, f"bwd varlen head_first={head_first}")
+    assert wkv7_get_last_error() == OK
+
+
+def test_bwd_head_first_batched(cuda_device):
+    x = synth.fwd_inputs(2, 45, 3, dtype=torch.bfloat16, seed=660, s0_std=0.1)
+    dout, dsT = upstream(2, 45, 3, torch.bfloat16, 661)
+    ref = oracle.bwd(*(x[n] for n in NAMES), dout, s0=x["s0"], dsT=dsT)
+    xd = to_dev(x, cuda_device)
+    hf = lambda t: t.transpose(1, 2).contiguous()
+    g = wkv7_bwd(*(hf(xd[n]) for n in NAMES), hf(dout.to(cuda_device)), s0=xd["s0"],
+                 dsT=dsT.to(cuda_device), head_first=True)
+    g = {n: (t.transpose(1, 2) if n != "ds0" else t) for n, t in g.items()}
+    check_grads(g, ref, torch.bfloat16, "bwd head_first")

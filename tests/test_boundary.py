@@ -172,12 +172,14 @@ def test_bwd_rejects_bad_arguments(lib):
     dout = ctypes.c_void_p(P + 0x8000)
     outs = [ctypes.c_void_p(P + 0x10000 + 0x1000 * i) for i in range(6)]
     ws = ctypes.c_void_p(P + 0x100000)
-    need = lib.wkv7_bwd_workspace_bytes(1, 16, 2, 64, 64)
-    assert need == 2 * ((16 // 8 + 1) * 4096 + 16 * 64) * 4
-    assert lib.wkv7_bwd_workspace_bytes(1, 16, 2, 128, 128) == 0
+    need = lib.wkv7_bwd_workspace_bytes(1, 16, 2, 64, 64, 1)
+    assert need == (2 * (16 // 8 + 2 * 1 + 1) * 4096 + 16 * 2 * 64) * 4
+    assert lib.wkv7_bwd_workspace_bytes(1, 16, 2, 128, 128, 1) == 0
 
-    def call(B=1, T=16, H=2, K=64, V=64, dtype=BF16, d=dout, o=outs, w=ws, n=need):
-        return lib.wkv7_bwd(*ins, None, None, d, None, *o, None, B, T, H, K, V, dtype, w, n, None)
+    def call(B=1, T=16, H=2, K=64, V=64, dtype=BF16, d=dout, o=outs, w=ws, n=need, N=None,
+             layout=0):
+        return lib.wkv7_bwd(*ins, None, None, d, None, *o, None, B, T, H, K, V, None,
+                            B if N is None else N, layout, dtype, w, n, None)
 
     assert call(K=128, V=128) == ERR_UNSUPPORTED
     assert call(H=0) == ERR_INVALID_ARG
@@ -187,4 +189,6 @@ def test_bwd_rejects_bad_arguments(lib):
     assert call(o=[ins[0]] + outs[1:]) == ERR_INVALID_ARG  # dr aliases r
     assert call(n=need - 1) == ERR_INVALID_ARG  # workspace too small
     assert call(w=None) == ERR_INVALID_ARG
+    assert call(N=2) == ERR_INVALID_ARG  # N must equal B without cu_seqlens
+    assert call(layout=3) == ERR_INVALID_ARG
     assert call(B=0) == OK
