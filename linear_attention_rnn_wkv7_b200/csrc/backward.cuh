@@ -73,11 +73,11 @@ __device__ __forceinline__ Seq unit_seq(int n, int T, const int32_t* cu_seqlens)
 
 template <typename Tin>
 __global__ void __launch_bounds__(64)
-ckpt_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
-            const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
+ckpt_kernel(const Tin* __restrict__ w, const Tin* __restrict__ k, const Tin* __restrict__ v,
+            const Tin* __restrict__ a, const Tin* __restrict__ b,
             const float* __restrict__ s0, const uint8_t* __restrict__ mask,
             float* __restrict__ ckpt, float* __restrict__ uws, int T, int H, int N,
-            const int32_t* __restrict__ cu_seqlens, int head_first, long long slots) {
+            const int32_t* __restrict__ cu_seqlens, int head_first) {
     constexpr int kTile = 16;
     __shared__ __align__(16) float sm[4][kTile][64];  // d = exp(w), k, a, b
     __shared__ float sv[kTile][64];
@@ -97,7 +97,6 @@ ckpt_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
     const size_t ts = head_first ? 1 : (size_t)H;
     float* ck = ckpt + ((size_t)sq.slot0 * H + h) * 4096;
     float* uu = uws + ((size_t)h * rows + (size_t)sq.bb * T + sq.bos) * 64;
-    (void)r;
 
     float S[64];
 #pragma unroll
@@ -192,7 +191,7 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
            const float* __restrict__ uws, Tin* __restrict__ dr, Tin* __restrict__ dw,
            Tin* __restrict__ dk, Tin* __restrict__ dv, Tin* __restrict__ da,
            Tin* __restrict__ db, float* __restrict__ ds0, int T, int H, int N,
-           const int32_t* __restrict__ cu_seqlens, int head_first, long long slots) {
+           const int32_t* __restrict__ cu_seqlens, int head_first) {
     constexpr int NC = 64 / P;  // columns (and, for the column sums, rows) per thread
     // per token of the tile: K-side r, e^{w}, e^{-w}, k, a, b; V-side v, do, u
     __shared__ __align__(16) float sK[6][kCkpt][64];
@@ -402,14 +401,14 @@ cudaError_t launch_bwd(const void* r, const void* w, const void* k, const void* 
     const Tin *r_ = static_cast<const Tin*>(r), *w_ = static_cast<const Tin*>(w),
               *k_ = static_cast<const Tin*>(k), *v_ = static_cast<const Tin*>(v),
               *a_ = static_cast<const Tin*>(a), *b_ = static_cast<const Tin*>(b);
-    bwd::ckpt_kernel<Tin><<<(unsigned)units, 64, 0, stream>>>(r_, w_, k_, v_, a_, b_, s0, mask,
-                                                              ckpt, uws, T, H, N, cu_seqlens,
-                                                              head_first, slots);
+    bwd::ckpt_kernel<Tin><<<(unsigned)units, 64, 0, stream>>>(w_, k_, v_, a_, b_, s0, mask, ckpt,
+                                                              uws, T, H, N, cu_seqlens,
+                                                              head_first);
     bwd::bwd_kernel<Tin, bwd::kRowThreads><<<(unsigned)units, 64 * bwd::kRowThreads, 0, stream>>>(
         r_, w_, k_, v_, a_, b_, mask, static_cast<const Tin*>(dout), dsT, ckpt, uws,
         static_cast<Tin*>(dr), static_cast<Tin*>(dw), static_cast<Tin*>(dk),
         static_cast<Tin*>(dv), static_cast<Tin*>(da), static_cast<Tin*>(db), ds0, T, H, N,
-        cu_seqlens, head_first, slots);
+        cu_seqlens, head_first);
     return cudaGetLastError();
 }
 
