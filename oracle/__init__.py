@@ -16,6 +16,10 @@ pin this one on tiny inputs.
 ``bwd`` is the backward of ``fwd`` (plain reverse-mode differentiation of the
 same recurrence, every state kept), for dL/do and dL/dS_T given.
 
+``gdn_bwd`` is the Gated DeltaNet backward: the generalized-rule backward on the
+substituted inputs, then the chain rule through that substitution and through the
+L2 normalisation of q and k (numpy, written out below).
+
 ``gdn_fwd`` / ``gdn_step`` are the Gated DeltaNet operator of the same README
 (sections "gdn_recurrent 使用方法" and "gdn_chunk 使用方法": q, k L2-normalised
 inside, g a log-space decay gate per (b, t, h), beta a write strength in (0, 1)
@@ -211,3 +215,45 @@ def bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=None,
     if rc != 0:
         raise ValueError("wkv7_oracle_bwd rejected its arguments")
     return g
+
+
+def gdn_bwd(q, k, v, g, beta, dout, s0=None, dsT=None, cu_seqlens=None, nthreads: int = 0):
+    """Gated DeltaNet backward for L = sum(o * dout) + sum(S_T * dsT).  Returns float64
+    dq, dk, dv [B,T,H,*], dg, dbeta [B,T,H] and ds0 (shaped like s0, or [N,H,K,V]).
+
+    Gated DeltaNet is the generalized rule with r = qh, w = g on every channel, write
+    key beta kh, a = kh and b = -e^g beta kh (qh = q/|q|, kh = k/|k|).  The gradients
+    of those inputs come from ``bwd``; then, by the chain rule,
+        dkh = beta dk_w + da - e^g beta db,   dg = sum(dw) + db . b,
+        dbeta = kh . dk_w - e^g (kh . db),
+        dx = (dxh - xh (xh . dxh)) / |x| for x = q (dxh = dr) and x = k (a zero x gets 0).
+    """
+    q, k, v, g, beta, dout = (_f64(x) for x in (q, k, v, g, beta, dout))
+    B, T, H, K = q.shape
+    cu = _cu(cu_seqlens)
+    N = B if cu is None else cu.shape[0] - 1
+    s0 = _f64(s0)
+    shared = s0 is not None and s0.shape[0] == 1 and N != 1
+    s0_full = np.repeat(s0, N, axis=0) if shared else s0
+    nq = np.linalg.norm(q, axis=-1, keepdims=True)
+    nk = np.linalg.norm(k, axis=-1, keepdims=True)
+    qh = np.where(nq > 0, q / np.where(nq > 0, nq, 1.0), 0.0)
+    kh = np.where(nk > 0, k / np.where(nk > 0, nk, 1.0), 0.0)
+    eg = np.exp(g)[..., None]
+    bt = beta[..., None]
+    w = np.repeat(g[..., None], K, axis=-1)
+    gr = bwd(qh, w, bt * kh, v, kh, -eg * bt * kh, dout, s0=s0_full, dsT=_f64(dsT),
+             cu_seqlens=cu, nthreads=nthreads)
+    dkh = bt * gr["dk"] + gr["da"] - eg * bt * gr["db"]
+    out = {"dv": gr["dv"]}
+    out["dg"] = gr["dw"].sum(-1) + np.sum(gr["db"] * (-eg * bt * kh), axis=-1)
+    out["dbeta"] = np.sum(kh * gr["dk"], axis=-1) - eg[..., 0] * np.sum(kh * gr["db"], axis=-1)
+
+    def through_norm(xh, n, dxh):
+        proj = dxh - xh * np.sum(xh * dxh, axis=-1, keepdims=True)
+        return np.where(n > 0, proj / np.where(n > 0, n, 1.0), 0.0)
+
+    out["dq"] = through_norm(qh, nq, gr["dr"])
+    out["dk"] = through_norm(kh, nk, dkh)
+    out["ds0"] = gr["ds0"].sum(axis=0, keepdims=True) if shared else gr["ds0"]
+    return out

@@ -273,3 +273,33 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     ob1, _ = brute.gdn_fwd(q, k, v, g, beta, s0=np.repeat(s1, 2, axis=0))
     failures += not np.allclose(o1, ob1, atol=1e-9)
     assert failures > 0, f"mutant {name} passed every pin"
+
+
+# --- the Gated DeltaNet backward --------------------------------------------------
+
+def _gdn_loss(x, dout, dsT):
+    o, sT, _ = oracle.gdn_fwd(*(x[n] for n in ("q", "k", "v", "g", "beta")), s0=x["s0"])
+    return float(np.sum(o * dout) + np.sum(sT * dsT))
+
+
+@pytest.mark.parametrize("seed,shared", [(20, False), (21, True)])
+def test_gdn_bwd_matches_finite_differences(seed, shared):
+    rng = np.random.default_rng(seed)
+    q, k, v, g, beta, _ = rand_gdn(rng, 2, 6, 1, 3, 2, s0=False)
+    s0 = rng.standard_normal((1 if shared else 2, 1, 3, 2))
+    x = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "s0": s0}
+    dout = rng.standard_normal(v.shape)
+    dsT = rng.standard_normal((2, 1, 3, 2))
+    gr = oracle.gdn_bwd(q, k, v, g, beta, dout, s0=s0, dsT=dsT)
+    eps = 1e-6
+    for n in ("q", "k", "v", "g", "beta", "s0"):
+        fd = np.zeros_like(x[n])
+        for idx in np.ndindex(x[n].shape):
+            keep = x[n][idx]
+            x[n][idx] = keep + eps
+            lp = _gdn_loss(x, dout, dsT)
+            x[n][idx] = keep - eps
+            lm = _gdn_loss(x, dout, dsT)
+            x[n][idx] = keep
+            fd[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(gr["d" + n], fd, rtol=1e-6, atol=1e-7, err_msg=n)
