@@ -213,6 +213,34 @@ wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const voi
                           wkv7_dtype dtype, void* stream);
 
 /*
+ * wkv7_gdn_bwd -- backward of wkv7_gdn_fwd (the README's gated_delta_net_recurrent
+ * and gated_delta_net_chunk support backpropagation), for
+ * L = sum(o * dout) + sum(S_T * dsT): the generalized-rule backward (wkv7_bwd) on the
+ * substituted inputs r = qh, w = g, write key beta kh, a = kh, b = -e^g beta kh, then
+ * the chain rule through the substitution and the L2 normalisation of q and k (the
+ * gradient of a zero q or k is zero).
+ *
+ *   q, k, v, g, beta, s0, s0_shared, cu_seqlens, N, layout   as for wkv7_gdn_fwd (K = V = 64)
+ *   dout           shaped like v dtype   dL/do (required)
+ *   dsT            [N, H, K, V]  fp32    dL/dS_T, or NULL
+ *   dq, dk (like q), dv (like v), dg, dbeta (like g)   dtype   outputs
+ *   ds0            fp32, shaped like s0 ([1, H, K, V] when shared: summed over the
+ *                  sequences), or NULL
+ *   workspace      at least wkv7_gdn_bwd_workspace_bytes(B, T, H, K, V, N, dtype,
+ *                  s0_shared) bytes of device memory (16-byte aligned)
+ */
+size_t wkv7_gdn_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N, wkv7_dtype dtype,
+                                     int s0_shared);
+
+wkv7_status wkv7_gdn_bwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* s0, int s0_shared, const void* dout,
+                         const float* dsT, void* dq, void* dk, void* dv, void* dg, void* dbeta,
+                         float* ds0, int B, int T, int H, int K, int V,
+                         const int32_t* cu_seqlens, int N, wkv7_layout layout,
+                         wkv7_dtype dtype, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
  * wkv7_get_last_error -- synchronises `stream`, returns and clears the sticky
  * device-side flag (WKV7_ERR_DEVICE_TIMEOUT / WKV7_ERR_DEVICE_BAD_SEQLENS) of
  * the current device, or WKV7_ERR_CUDA if the stream reports a CUDA error,

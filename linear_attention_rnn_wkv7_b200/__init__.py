@@ -6,9 +6,10 @@
 not load the CUDA library; the first call does, and fails loudly if it is
 missing.
 """
-from .wkv7 import (WKV7Error, generalized_delta_rule, library, status_string,  # noqa: F401
-                   wkv7_bwd, wkv7_fwd, wkv7_gdn_fwd, wkv7_gdn_step, wkv7_get_last_error,
-                   wkv7_step)
+from .wkv7 import (WKV7Error, gated_delta_net, generalized_delta_rule, library,  # noqa: F401
+                   status_string, wkv7_bwd, wkv7_fwd, wkv7_gdn_bwd, wkv7_gdn_fwd,
+                   wkv7_gdn_step, wkv7_get_last_error, wkv7_step)
 
 __all__ = ["wkv7_fwd", "wkv7_step", "wkv7_bwd", "generalized_delta_rule", "wkv7_gdn_fwd",
-           "wkv7_gdn_step", "wkv7_get_last_error", "library", "status_string", "WKV7Error"]
+           "wkv7_gdn_step", "wkv7_gdn_bwd", "gated_delta_net", "wkv7_get_last_error",
+           "library", "status_string", "WKV7Error"]

@@ -9,6 +9,7 @@
 #include "recurrent.cuh"
 #include "chunked.cuh"
 #include "backward.cuh"
+#include "gdn_backward.cuh"
 
 namespace {
 
@@ -240,6 +241,64 @@ wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v,
             : wkv7::launch_bwd<float>(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da,
                                       db, ds0, B, T, H, N, cu_seqlens, hf,
                                       static_cast<float*>(workspace), stream);
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+size_t wkv7_gdn_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N, wkv7_dtype dtype,
+                                     int s0_shared) {
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || K != 64 || V != 64) return 0;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return 0;
+    return wkv7::gdnb::workspace_bytes((long long)B * T, N, H, s0_shared != 0);
+}
+
+wkv7_status wkv7_gdn_bwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* s0, int s0_shared, const void* dout,
+                         const float* dsT, void* dq, void* dk, void* dv, void* dg, void* dbeta,
+                         float* ds0, int B, int T, int H, int K, int V,
+                         const int32_t* cu_seqlens, int N, wkv7_layout layout,
+                         wkv7_dtype dtype, void* workspace, size_t workspace_bytes,
+                         void* stream_) {
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0 || N < 0) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (layout != WKV7_LAYOUT_BTHK && layout != WKV7_LAYOUT_BHTK) return WKV7_ERR_INVALID_ARG;
+    if (s0_shared != 0 && s0_shared != 1) return WKV7_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (B != 1) return WKV7_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return WKV7_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return WKV7_ERR_INVALID_ARG;
+    }
+    if (K != 64 || V != 64) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)N * H;
+    if (units > 0x7fffffffLL || (long long)B * T * H > (1LL << 40)) return WKV7_ERR_UNSUPPORTED;
+    if (units == 0) return WKV7_OK;
+    const bool tokens = (long long)B * T > 0;
+    if (tokens && (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(dout) || !ok_ptr(dq) ||
+                   !ok_ptr(dk) || !ok_ptr(dv) || !ok_scalar_ptr(g, dtype) ||
+                   !ok_scalar_ptr(beta, dtype) || !ok_scalar_ptr(dg, dtype) ||
+                   !ok_scalar_ptr(dbeta, dtype)))
+        return WKV7_ERR_INVALID_ARG;
+    if ((s0 && !aligned16(s0)) || (dsT && !aligned16(dsT)) || (ds0 && !aligned16(ds0)))
+        return WKV7_ERR_INVALID_ARG;
+    const void* ins[7] = {q, k, v, g, beta, dout, s0};
+    const void* outs[6] = {dq, dk, dv, dg, dbeta, ds0};
+    for (const void* x : outs)
+        for (const void* y : ins)
+            if (x && x == y) return WKV7_ERR_INVALID_ARG;
+    if (!s0) s0_shared = 0;
+    if (!ok_ptr(workspace) ||
+        workspace_bytes < wkv7_gdn_bwd_workspace_bytes(B, T, H, K, V, N, dtype, s0_shared))
+        return WKV7_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const int hf = layout == WKV7_LAYOUT_BHTK;
+    const cudaError_t err =
+        dtype == WKV7_BF16
+            ? wkv7::launch_gdn_bwd<__nv_bfloat16>(q, k, v, g, beta, s0, s0_shared, dout, dsT, dq,
+                                                  dk, dv, dg, dbeta, ds0, B, T, H, N, cu_seqlens,
+                                                  hf, workspace, stream)
+            : wkv7::launch_gdn_bwd<float>(q, k, v, g, beta, s0, s0_shared, dout, dsT, dq, dk, dv,
+                                          dg, dbeta, ds0, B, T, H, N, cu_seqlens, hf, workspace,
+                                          stream);
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 

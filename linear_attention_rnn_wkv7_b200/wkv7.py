@@ -53,6 +53,11 @@ def library() -> ctypes.CDLL:
         lib.wkv7_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
         lib.wkv7_bwd.restype = i
         lib.wkv7_bwd.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i, i, p, ctypes.c_size_t, p]
+        lib.wkv7_gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.wkv7_gdn_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+        lib.wkv7_gdn_bwd.restype = i
+        lib.wkv7_gdn_bwd.argtypes = ([p] * 6 + [i] + [p] * 8 + [i] * 5 + [p, i, i, i, p,
+                                                                         ctypes.c_size_t, p])
         lib.wkv7_gdn_fwd.restype = i
         lib.wkv7_gdn_fwd.argtypes = [p, p, p, p, p, p, i, p, p, i, i, i, i, i, p, i, i, i, i, p]
         lib.wkv7_gdn_step.restype = i
@@ -330,3 +335,90 @@ def wkv7_gdn_step(q, k, v, g, beta, state, o=None):
 def wkv7_get_last_error(device=None) -> int:
     """Synchronise the current stream; return and clear the device-side flag."""
     return library().wkv7_get_last_error(_stream(device))
+
+
+def wkv7_gdn_bwd(q, k, v, g, beta, dout, s0=None, dsT=None, cu_seqlens=None,
+                 head_first: bool = False, workspace=None):
+    """Backward of wkv7_gdn_fwd for L = sum(o * dout) + sum(S_T * dsT).  Returns a dict:
+    dq, dk, dv, dg, dbeta (input dtype, shaped like the inputs) and ds0 (fp32, shaped
+    like s0; [N,H,K,V] when s0 is None)."""
+    _check(q, "q")
+    dt = q.dtype
+    if head_first:
+        B, H, T, K = q.shape
+    else:
+        B, T, H, K = q.shape
+    V = v.shape[-1]
+    kshape = (B, H, T, K) if head_first else (B, T, H, K)
+    vshape = (B, H, T, V) if head_first else (B, T, H, V)
+    _check(k, "k", dt, kshape)
+    _check(v, "v", dt, vshape)
+    _check(g, "g", dt, kshape[:3])
+    _check(beta, "beta", dt, kshape[:3])
+    _check(dout, "dout", dt, vshape)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    shared = 0
+    if s0 is not None:
+        _check(s0, "s0", torch.float32)
+        if tuple(s0.shape) == (1, H, K, V) and N != 1:
+            shared = 1
+        elif tuple(s0.shape) != (N, H, K, V):
+            raise ValueError(f"s0 must have shape {(N, H, K, V)} or {(1, H, K, V)}")
+    if dsT is not None:
+        _check(dsT, "dsT", torch.float32, (N, H, K, V))
+    nbytes = int(library().wkv7_gdn_bwd_workspace_bytes(B, T, H, K, V, N, _dtype_code(q), shared))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    else:
+        _check(workspace, "workspace", torch.uint8)
+    out = {"dq": torch.empty(kshape, dtype=dt, device=q.device),
+           "dk": torch.empty(kshape, dtype=dt, device=q.device),
+           "dv": torch.empty(vshape, dtype=dt, device=q.device),
+           "dg": torch.empty(kshape[:3], dtype=dt, device=q.device),
+           "dbeta": torch.empty(kshape[:3], dtype=dt, device=q.device),
+           "ds0": torch.empty(tuple(s0.shape) if s0 is not None else (N, H, K, V),
+                              dtype=torch.float32, device=q.device)}
+    st = library().wkv7_gdn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0), shared,
+                                _ptr(dout), _ptr(dsT), _ptr(out["dq"]), _ptr(out["dk"]),
+                                _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+                                _ptr(out["ds0"]), B, T, H, K, V, _ptr(cu_seqlens), N,
+                                int(bool(head_first)), _dtype_code(q), _ptr(workspace),
+                                workspace.numel(), _stream(q.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_gdn_bwd")
+    return out
+
+
+class GatedDeltaNet(torch.autograd.Function):
+    """gated_delta_net_chunk / gated_delta_net_recurrent as a differentiable op: forward
+    through wkv7_gdn_fwd, backward through wkv7_gdn_bwd (K = V = 64)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, beta, s0, cu_seqlens, head_first):
+        o, sT = wkv7_gdn_fwd(q, k, v, g, beta, s0=s0, cu_seqlens=cu_seqlens,
+                             head_first=head_first)
+        ctx.save_for_backward(q, k, v, g, beta, s0, cu_seqlens)
+        ctx.head_first = head_first
+        return o, sT
+
+    @staticmethod
+    def backward(ctx, do, dsT):
+        q, k, v, g, beta, s0, cu_seqlens = ctx.saved_tensors
+        do = torch.zeros_like(v) if do is None else do.contiguous()
+        dsT = None if dsT is None else dsT.contiguous().float()
+        gr = wkv7_gdn_bwd(q, k, v, g, beta, do.to(q.dtype), s0=s0, dsT=dsT,
+                          cu_seqlens=cu_seqlens, head_first=ctx.head_first)
+        ds0 = gr["ds0"] if s0 is not None else None
+        return gr["dq"], gr["dk"], gr["dv"], gr["dg"], gr["dbeta"], ds0, None, None
+
+
+def gated_delta_net(q, k, v, g, beta, initial_state=None, output_final_state=True,
+                    cu_seqlens=None, head_first: bool = False):
+    """Differentiable Gated DeltaNet (README: gated_delta_net_recurrent / _chunk);
+    returns (o, final state or None)."""
+    o, sT = GatedDeltaNet.apply(q, k, v, g, beta, initial_state, cu_seqlens, head_first)
+    return o, (sT if output_final_state else None)

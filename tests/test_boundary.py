@@ -34,7 +34,8 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for required in ("wkv7_fwd", "wkv7_step", "wkv7_bwd", "wkv7_bwd_workspace_bytes",
-                     "wkv7_gdn_fwd", "wkv7_gdn_step", "wkv7_get_last_error",
+                     "wkv7_gdn_fwd", "wkv7_gdn_step", "wkv7_gdn_bwd",
+                     "wkv7_gdn_bwd_workspace_bytes", "wkv7_get_last_error",
                      "wkv7_status_string"):
         assert required in names
 
