@@ -260,8 +260,8 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
-    from linear_attention_rnn_wkv7_b200 import (library, wkv7_bwd, wkv7_fwd, wkv7_gdn_fwd,
-                                                wkv7_gdn_step, wkv7_step)
+    from linear_attention_rnn_wkv7_b200 import (library, wkv7_bwd, wkv7_fwd, wkv7_gdn_bwd,
+                                                wkv7_gdn_fwd, wkv7_gdn_step, wkv7_step)
     library()  # fail loudly if the CUDA library is missing
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
@@ -292,10 +292,10 @@ def main():
         decode = decode_leg(device, stream, wkv7_gdn_step if gdn else wkv7_step, hbm_peak,
                             peak_kind, max_over_ranks, barrier, rank, gdn, args.head_size)
     backward = None
-    if (args.only in ("all", "bwd") and not args.no_bwd and not gdn and args.head_size == 64
+    if (args.only in ("all", "bwd") and not args.no_bwd and args.head_size == 64
             and args.workload == "b8_t4096_h64"):
-        backward = bwd_leg(args, device, stream, wkv7_bwd, hbm_peak, peak_kind, max_over_ranks,
-                           barrier, rank)
+        backward = bwd_leg(args, device, stream, wkv7_gdn_bwd if gdn else wkv7_bwd, hbm_peak,
+                           peak_kind, max_over_ranks, barrier, rank, gdn)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu and args.only == "all" and args.head_size == 64:
         cpu = cpu_oracle_sample(gdn=gdn)
@@ -456,21 +456,33 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
             "clocks": clock_info, "desc": desc}
 
 
-def bwd_leg(args, device, stream, wkv7_bwd, hbm_peak, peak_kind, max_over_ranks, barrier, rank):
-    """wkv7_bwd on the B=8, T=4096, H=64 bf16 forward workload (random dL/do and
-    dL/dS_T), inputs and workspace resident; up to 20 timed launches."""
+def bwd_leg(args, device, stream, bwd_fn, hbm_peak, peak_kind, max_over_ranks, barrier, rank,
+            gdn=False):
+    """wkv7_bwd (or wkv7_gdn_bwd) on the B=8, T=4096, H=64 bf16 forward workload (random
+    dL/do and dL/dS_T), inputs and workspace resident; up to 20 timed launches."""
     B, T, H = args.batch, FWD["T"], FWD["H"]
-    x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16,
-                         seed=replicas.replica_seed(FWD["seed"], rank), s0_std=FWD["s0_std"])
+    if gdn:
+        x = synth.gdn_inputs(B, T, H, dtype=torch.bfloat16,
+                             seed=replicas.replica_seed(GDN_FWD["seed"], rank),
+                             s0_std=GDN_FWD["s0_std"])
+        names = ("q", "k", "v", "g", "beta")
+    else:
+        x = synth.fwd_inputs(B, T, H, dtype=torch.bfloat16,
+                             seed=replicas.replica_seed(FWD["seed"], rank), s0_std=FWD["s0_std"])
+        names = ("r", "w", "k", "v", "a", "b")
     gen = torch.Generator().manual_seed(replicas.replica_seed(620, rank))
     dout = torch.randn(B, T, H, 64, generator=gen).to(torch.bfloat16).to(device)
     dsT = (torch.randn(B, H, 64, 64, generator=gen) * 0.1).to(device)
     xd = {k: v.to(device) for k, v in x.items()}
-    ws = torch.empty(wkv7_bwd_workspace_nbytes(B, T, H), dtype=torch.uint8, device=device)
+    if gdn:
+        from linear_attention_rnn_wkv7_b200 import library
+        nbytes = int(library().wkv7_gdn_bwd_workspace_bytes(B, T, H, 64, 64, B, 0, 0))
+    else:
+        nbytes = wkv7_bwd_workspace_nbytes(B, T, H)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
     def step():
-        wkv7_bwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], dout, s0=xd["s0"],
-                 dsT=dsT, workspace=ws)
+        bwd_fn(*(xd[n] for n in names), dout, s0=xd["s0"], dsT=dsT, workspace=ws)
 
     for _ in range(3):
         step()
@@ -485,15 +497,21 @@ def bwd_leg(args, device, stream, wkv7_bwd, hbm_peak, peak_kind, max_over_ranks,
     torch.cuda.synchronize(device)
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
-    # inputs r,w,k,v,a,b and dout read, six gradients written (bf16), s0 and dsT read and
-    # ds0 written (fp32); the workspace (checkpoints, u) is not counted
-    nbytes = B * T * H * 13 * 64 * 2 + 3 * B * H * STATE_BYTES
+    # WKV7: r,w,k,v,a,b and dout read, six gradients written (bf16); Gated DeltaNet:
+    # q,k,v,dout read and dq,dk,dv written (bf16 vectors), g,beta read and dg,dbeta
+    # written (bf16 scalars); s0 and dsT read and ds0 written (fp32).  The workspace
+    # (checkpoints, u, and for Gated DeltaNet the fp32 substituted inputs) is not counted.
+    per_th = (7 * 64 * 2 + 4 * 2) if gdn else 13 * 64 * 2
+    nbytes = B * T * H * per_th + 3 * B * H * STATE_BYTES
     gbs = nbytes / (ms / 1e3) / 1e9
-    return {"workload": f"bwd_bf16_b{B}_t{T}_h{H}", "steps": steps, "ms_per_step": ms,
+    return {"workload": ("gdn_" if gdn else "") + f"bwd_bf16_b{B}_t{T}_h{H}", "steps": steps,
+            "ms_per_step": ms,
             "tokens/s": B * T / (ms / 1e3), "algorithmic_bytes_per_step": nbytes, "GB/s": gbs,
             "peak": hbm_peak, "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
             "workspace_bytes": ws.numel(), "gpu_launches": 2 * steps,
-            "kernels": "ckpt_kernel (forward, checkpoints) + bwd_kernel (reverse)"}
+            "kernels": ("gdn_map_kernel + " if gdn else "")
+            + "ckpt_kernel (forward, checkpoints) + bwd_kernel (reverse)"
+            + (" + gdn_chain_kernel" if gdn else "")}
 
 
 def wkv7_bwd_workspace_nbytes(B, T, H):
