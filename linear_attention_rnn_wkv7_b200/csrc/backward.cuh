@@ -105,27 +105,38 @@ ckpt_kernel(const Tin* __restrict__ w, const Tin* __restrict__ k, const Tin* __r
     for (int t0 = 0; t0 < L; t0 += kTile) {
         const int cnt = min(kTile, L - t0);
         __syncthreads();
-        {  // every load of the tile is issued before the first store (one latency per tile)
-            float xw[kTile], xk[kTile], xa[kTile], xb[kTile], xv[kTile];
+        {  // 16-byte loads: EPL elements per thread, 64 / EPL threads per row; all of
+           // the tile's loads are issued before the first store
+            constexpr int EPL = 16 / (int)sizeof(Tin);  // elements per load
+            constexpr int TPR = 64 / EPL;               // threads per row
+            constexpr int RPS = 64 / TPR;               // rows (tokens) per sweep
+            constexpr int SW = kTile / RPS;             // sweeps per tile
+            const int e0 = (j % TPR) * EPL, rr = j / TPR;
+            uint4 raw[5][SW];
 #pragma unroll
-            for (int tt = 0; tt < kTile; ++tt) {
+            for (int s2 = 0; s2 < SW; ++s2) {
+                const int tt = s2 * RPS + rr;
                 if (tt < cnt) {
-                    const size_t row = (tb + (size_t)(t0 + tt) * ts) * 64;
-                    xw[tt] = to_f32(w[row + j]);
-                    xk[tt] = to_f32(k[row + j]);
-                    xa[tt] = to_f32(a[row + j]);
-                    xb[tt] = to_f32(b[row + j]);
-                    xv[tt] = to_f32(v[row + j]);
+                    const size_t row = (tb + (size_t)(t0 + tt) * ts) * 64 + e0;
+                    raw[0][s2] = *reinterpret_cast<const uint4*>(w + row);
+                    raw[1][s2] = *reinterpret_cast<const uint4*>(k + row);
+                    raw[2][s2] = *reinterpret_cast<const uint4*>(a + row);
+                    raw[3][s2] = *reinterpret_cast<const uint4*>(b + row);
+                    raw[4][s2] = *reinterpret_cast<const uint4*>(v + row);
                 }
             }
 #pragma unroll
-            for (int tt = 0; tt < kTile; ++tt) {
+            for (int s2 = 0; s2 < SW; ++s2) {
+                const int tt = s2 * RPS + rr;
                 if (tt < cnt) {
-                    sm[0][tt][j] = expf(xw[tt]);
-                    sm[1][tt][j] = xk[tt];
-                    sm[2][tt][j] = xa[tt];
-                    sm[3][tt][j] = xb[tt];
-                    sv[tt][j] = xv[tt];
+#pragma unroll
+                    for (int q = 0; q < 5; ++q) {
+                        const Tin* x = reinterpret_cast<const Tin*>(&raw[q][s2]);
+                        float* dst = q == 4 ? &sv[tt][e0] : &sm[q][tt][e0];
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e)
+                            dst[e] = q == 0 ? expf(to_f32(x[e])) : to_f32(x[e]);
+                    }
                 }
             }
         }
@@ -235,35 +246,60 @@ bwd_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __re
     for (int c = nC - 1; c >= 0; --c) {
         const int t0 = c * kCkpt, cnt = min(kCkpt, L - t0);
         __syncthreads();  // the previous tile's reads of the stage are done
-        if (tid < 64) {  // every load of the tile is issued before the first store
-            float x[8][kCkpt];
+        if (tid < 64) {  // 16-byte loads, all issued before the first store
+            constexpr int EPL = 16 / (int)sizeof(Tin);  // input elements per load
+            constexpr int TPR = 64 / EPL;               // threads per row
+            constexpr int RPS = 64 / TPR;               // rows (tokens) per sweep
+            constexpr int SW = (kCkpt + RPS - 1) / RPS; // sweeps per tile
+            const int e0 = (tid % TPR) * EPL, rr = tid / TPR;
+            uint4 raw[7][SW];
 #pragma unroll
-            for (int tt = 0; tt < kCkpt; ++tt) {
+            for (int s2 = 0; s2 < SW; ++s2) {
+                const int tt = s2 * RPS + rr;
                 if (tt < cnt) {
-                    const size_t row = (tb + (size_t)(t0 + tt) * ts) * 64;
-                    x[0][tt] = to_f32(r[row + tid]);
-                    x[1][tt] = to_f32(w[row + tid]);
-                    x[2][tt] = to_f32(k[row + tid]);
-                    x[3][tt] = to_f32(a[row + tid]);
-                    x[4][tt] = to_f32(b[row + tid]);
-                    x[5][tt] = to_f32(v[row + tid]);
-                    x[6][tt] = to_f32(dout[row + tid]);
-                    x[7][tt] = uu[(size_t)(t0 + tt) * 64 + tid];
+                    const size_t row = (tb + (size_t)(t0 + tt) * ts) * 64 + e0;
+                    raw[0][s2] = *reinterpret_cast<const uint4*>(r + row);
+                    raw[1][s2] = *reinterpret_cast<const uint4*>(w + row);
+                    raw[2][s2] = *reinterpret_cast<const uint4*>(k + row);
+                    raw[3][s2] = *reinterpret_cast<const uint4*>(a + row);
+                    raw[4][s2] = *reinterpret_cast<const uint4*>(b + row);
+                    raw[5][s2] = *reinterpret_cast<const uint4*>(v + row);
+                    raw[6][s2] = *reinterpret_cast<const uint4*>(dout + row);
+                }
+            }
+            // u (fp32): 16 threads per row, 4 rows per sweep
+            float4 ru[kCkpt / 4];
+#pragma unroll
+            for (int s2 = 0; s2 < kCkpt / 4; ++s2) {
+                const int tt = s2 * 4 + tid / 16;
+                if (tt < cnt)
+                    ru[s2] = *reinterpret_cast<const float4*>(uu + (size_t)(t0 + tt) * 64 + (tid % 16) * 4);
+            }
+#pragma unroll
+            for (int s2 = 0; s2 < SW; ++s2) {
+                const int tt = s2 * RPS + rr;
+                if (tt < cnt) {
+                    const Tin* x[7];
+#pragma unroll
+                    for (int q = 0; q < 7; ++q) x[q] = reinterpret_cast<const Tin*>(&raw[q][s2]);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) {
+                        const float wv = to_f32(x[1][e]);
+                        sK[0][tt][e0 + e] = to_f32(x[0][e]);
+                        sK[1][tt][e0 + e] = expf(wv);
+                        sK[2][tt][e0 + e] = expf(-wv);
+                        sK[3][tt][e0 + e] = to_f32(x[2][e]);
+                        sK[4][tt][e0 + e] = to_f32(x[3][e]);
+                        sK[5][tt][e0 + e] = to_f32(x[4][e]);
+                        sV[0][tt][e0 + e] = to_f32(x[5][e]);
+                        sV[1][tt][e0 + e] = to_f32(x[6][e]);
+                    }
                 }
             }
 #pragma unroll
-            for (int tt = 0; tt < kCkpt; ++tt) {
-                if (tt < cnt) {
-                    sK[0][tt][tid] = x[0][tt];
-                    sK[1][tt][tid] = expf(x[1][tt]);
-                    sK[2][tt][tid] = expf(-x[1][tt]);
-                    sK[3][tt][tid] = x[2][tt];
-                    sK[4][tt][tid] = x[3][tt];
-                    sK[5][tt][tid] = x[4][tt];
-                    sV[0][tt][tid] = x[5][tt];
-                    sV[1][tt][tid] = x[6][tt];
-                    sV[2][tt][tid] = x[7][tt];
-                }
+            for (int s2 = 0; s2 < kCkpt / 4; ++s2) {
+                const int tt = s2 * 4 + tid / 16;
+                if (tt < cnt) *reinterpret_cast<float4*>(&sV[2][tt][(tid % 16) * 4]) = ru[s2];
             }
             if (tid < cnt) smask[tid] = mask ? (mask[(size_t)sq.bb * T + sq.bos + t0 + tid] != 0) : 1;
         }
