@@ -161,6 +161,25 @@ wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * wkv7_bwd_noalloc -- wkv7_bwd with the library's own scratch instead of a caller
+ * workspace.  The pages have no counterpart to this entry point: it exists so that a
+ * caller without a device allocator can run the backward.  The scratch is a file-scope
+ * device array of WKV7_STATIC_SCRATCH_BYTES, reserved when libwkv7.so's device code is
+ * loaded (no allocation at call time).  Problems whose wkv7_bwd_workspace_bytes exceed
+ * it return WKV7_ERR_UNSUPPORTED.  Calls share that one scratch: they must not overlap
+ * in time (issue them on one stream, or synchronise between streams).  Arguments and
+ * results are those of wkv7_bwd.
+ */
+#define WKV7_STATIC_SCRATCH_BYTES (64u << 20)
+
+wkv7_status wkv7_bwd_noalloc(const void* r, const void* w, const void* k, const void* v,
+                             const void* a, const void* b, const float* s0,
+                             const uint8_t* mask, const void* dout, const float* dsT, void* dr,
+                             void* dw, void* dk, void* dv, void* da, void* db, float* ds0, int B,
+                             int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
+                             wkv7_layout layout, wkv7_dtype dtype, void* stream);
+
+/*
  * wkv7_gdn_fwd -- Gated DeltaNet forward over whole sequences
  * (gated_delta_net_recurrent / gated_delta_net_recurrent_inference /
  * gated_delta_net_chunk; rwkv-ops 0.9.0 README, "gdn_recurrent 使用方法" and

@@ -15,6 +15,11 @@ namespace {
 
 constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
 
+// Scratch of wkv7_bwd_noalloc: a file-scope device array, reserved when the library's
+// module is loaded, so that entry point allocates nothing at call time.
+constexpr size_t kStaticScratchBytes = WKV7_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
@@ -249,6 +254,20 @@ size_t wkv7_gdn_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N, wk
     if (B < 0 || T < 0 || H <= 0 || N < 0 || K != 64 || V != 64) return 0;
     if (dtype != WKV7_BF16 && dtype != WKV7_F32) return 0;
     return wkv7::gdnb::workspace_bytes((long long)B * T, N, H, s0_shared != 0);
+}
+
+wkv7_status wkv7_bwd_noalloc(const void* r, const void* w, const void* k, const void* v,
+                             const void* a, const void* b, const float* s0,
+                             const uint8_t* mask, const void* dout, const float* dsT, void* dr,
+                             void* dw, void* dk, void* dv, void* da, void* db, float* ds0, int B,
+                             int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
+                             wkv7_layout layout, wkv7_dtype dtype, void* stream) {
+    const size_t need = wkv7_bwd_workspace_bytes(B, T, H, K, V, N);
+    if (need > kStaticScratchBytes) return WKV7_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    if (cudaGetSymbolAddress(&scratch, g_static_scratch) != cudaSuccess) return WKV7_ERR_CUDA;
+    return wkv7_bwd(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da, db, ds0, B, T, H,
+                    K, V, cu_seqlens, N, layout, dtype, scratch, kStaticScratchBytes, stream);
 }
 
 wkv7_status wkv7_gdn_bwd(const void* q, const void* k, const void* v, const void* g,

@@ -53,6 +53,8 @@ def library() -> ctypes.CDLL:
         lib.wkv7_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
         lib.wkv7_bwd.restype = i
         lib.wkv7_bwd.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i, i, p, ctypes.c_size_t, p]
+        lib.wkv7_bwd_noalloc.restype = i
+        lib.wkv7_bwd_noalloc.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i, i, p]
         lib.wkv7_gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_gdn_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
         lib.wkv7_gdn_bwd.restype = i
@@ -226,6 +228,40 @@ def wkv7_bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=No
                             workspace.numel(), _stream(r.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_bwd")
+    return g
+
+
+def wkv7_bwd_noalloc(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=None,
+                     head_first: bool = False):
+    """wkv7_bwd on the library's static scratch (no workspace argument; small problems
+    only -- larger ones raise WKV7Error with WKV7_ERR_UNSUPPORTED).  Same results."""
+    _check(r, "r")
+    dt = r.dtype
+    if head_first:
+        B, H, T, K = r.shape
+    else:
+        B, T, H, K = r.shape
+    V = v.shape[-1]
+    kshape = (B, H, T, K) if head_first else (B, T, H, K)
+    vshape = (B, H, T, V) if head_first else (B, T, H, V)
+    for name, t in (("w", w), ("k", k), ("a", a), ("b", b)):
+        _check(t, name, dt, kshape)
+    _check(v, "v", dt, vshape)
+    _check(dout, "dout", dt, vshape)
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if mask is not None and mask.dtype == torch.bool:
+        mask = mask.to(torch.uint8)
+    g = {n: torch.empty(kshape, dtype=dt, device=r.device) for n in ("dr", "dw", "dk", "da", "db")}
+    g["dv"] = torch.empty(vshape, dtype=dt, device=r.device)
+    g["ds0"] = torch.empty((N, H, K, V), dtype=torch.float32, device=r.device)
+    st = library().wkv7_bwd_noalloc(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                    _ptr(s0), _ptr(mask), _ptr(dout), _ptr(dsT), _ptr(g["dr"]),
+                                    _ptr(g["dw"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]),
+                                    _ptr(g["db"]), _ptr(g["ds0"]), B, T, H, K, V,
+                                    _ptr(cu_seqlens), N, int(bool(head_first)), _dtype_code(r),
+                                    _stream(r.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_bwd_noalloc")
     return g
 
 

@@ -1,0 +1,64 @@
+"""wkv7_bwd_noalloc: the backward on the library's static scratch (a file-scope device
+array) instead of a caller workspace.  It must give exactly wkv7_bwd's results on
+problems that fit, and refuse larger ones before touching the device."""
+import ctypes
+
+import pytest
+import torch
+
+import oracle
+from linear_attention_rnn_wkv7_b200 import build as wkv7_build
+from linear_attention_rnn_wkv7_b200 import library, synth, wkv7_bwd
+from linear_attention_rnn_wkv7_b200.wkv7 import (ERR_UNSUPPORTED, BF16, WKV7Error,
+                                                 wkv7_bwd_noalloc, wkv7_bwd_workspace_bytes)
+from parity_util import rel_err, to_dev
+
+NAMES = ("r", "w", "k", "v", "a", "b")
+STATIC_SCRATCH_BYTES = 64 << 20  # WKV7_STATIC_SCRATCH_BYTES in include/wkv7.h
+
+
+def test_header_constant_and_refusal_on_cpu():
+    """The header's scratch size; a problem whose workspace exceeds it is refused by the
+    host check (nothing is launched, so this runs without a GPU)."""
+    import os
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "wkv7.h")).read()
+    assert "#define WKV7_STATIC_SCRATCH_BYTES (64u << 20)" in hdr
+    wkv7_build.build()
+    lib = library()
+    B, T, H = 8, 4096, 64
+    assert wkv7_bwd_workspace_bytes(B, T, H) > STATIC_SCRATCH_BYTES
+    fake = [ctypes.c_void_p(0x7f0000000000 + 0x1000 * i) for i in range(16)]
+    st = lib.wkv7_bwd_noalloc(*fake[:6], None, None, fake[6], None, *fake[7:13], None,
+                              B, T, H, 64, 64, None, B, 0, BF16, None)
+    assert st == ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_noalloc_equals_workspace_call(cuda_device, dtype):
+    B, T, H = 2, 100, 3
+    assert wkv7_bwd_workspace_bytes(B, T, H) <= STATIC_SCRATCH_BYTES
+    x = synth.fwd_inputs(B, T, H, dtype=dtype, seed=800, s0_std=0.1)
+    gen = torch.Generator().manual_seed(801)
+    dout = torch.randn(B, T, H, 64, generator=gen).to(dtype)
+    dsT = torch.randn(B, H, 64, 64, generator=gen) * 0.1
+    xd = to_dev(x, cuda_device)
+    args = [xd[n] for n in NAMES] + [dout.to(cuda_device)]
+    g0 = wkv7_bwd(*args, s0=xd["s0"], dsT=dsT.to(cuda_device))
+    g1 = wkv7_bwd_noalloc(*args, s0=xd["s0"], dsT=dsT.to(cuda_device))
+    for n in g0:
+        assert torch.equal(g0[n], g1[n]), n
+    ref = oracle.bwd(*(x[n] for n in NAMES), dout, s0=x["s0"], dsT=dsT)
+    limit = 1e-4 if dtype == torch.float32 else 2e-2
+    for n in ("dr", "dw", "dk", "dv", "da", "db"):
+        assert rel_err(g1[n], ref[n]) <= limit, n
+
+
+@pytest.mark.gpu
+def test_noalloc_refuses_large_problem(cuda_device):
+    x = to_dev(synth.fwd_inputs(2, 4096, 16, dtype=torch.bfloat16, seed=802, s0_std=0.1),
+               cuda_device)
+    dout = torch.zeros(2, 4096, 16, 64, dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(WKV7Error) as e:
+        wkv7_bwd_noalloc(*(x[n] for n in NAMES), dout, s0=x["s0"])
+    assert e.value.status == ERR_UNSUPPORTED
