@@ -248,9 +248,19 @@ def wkv7_bwd_noalloc(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_se
         _check(t, name, dt, kshape)
     _check(v, "v", dt, vshape)
     _check(dout, "dout", dt, vshape)
-    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
-    if mask is not None and mask.dtype == torch.bool:
-        mask = mask.to(torch.uint8)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if s0 is not None:
+        _check(s0, "s0", torch.float32, (N, H, K, V))
+    if dsT is not None:
+        _check(dsT, "dsT", torch.float32, (N, H, K, V))
+    if mask is not None:
+        if mask.dtype == torch.bool:
+            mask = mask.to(torch.uint8)
+        _check(mask, "mask", torch.uint8, (B, T))
     g = {n: torch.empty(kshape, dtype=dt, device=r.device) for n in ("dr", "dw", "dk", "da", "db")}
     g["dv"] = torch.empty(vshape, dtype=dt, device=r.device)
     g["ds0"] = torch.empty((N, H, K, V), dtype=torch.float32, device=r.device)
