@@ -16,6 +16,11 @@ pin this one on tiny inputs.
 ``bwd`` is the backward of ``fwd`` (plain reverse-mode differentiation of the
 same recurrence, every state kept), for dL/do and dL/dS_T given.
 
+``sane_fwd`` is the State Anomaly Neutralization variant (README, "rwkv7op_sane
+使用方法"): the same recurrence with a soft clip of the state after every 16th token;
+the clip function is not on the pages (reading: tau * tanh(S / tau)), so its parity
+is unpinned beyond the structure the tests check.
+
 ``gdn_bwd`` is the Gated DeltaNet backward: the generalized-rule backward on the
 substituted inputs, then the chain rule through that substitution and through the
 L2 normalisation of q and k (numpy, written out below).
@@ -64,6 +69,9 @@ def load_library(path: str):
         lib.wkv7_oracle_bwd.restype = ctypes.c_int
         lib.wkv7_oracle_bwd.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i,
                                                    ctypes.POINTER(ctypes.c_int)]
+    if hasattr(lib, "wkv7_oracle_sane_fwd"):
+        lib.wkv7_oracle_sane_fwd.restype = ctypes.c_int
+        lib.wkv7_oracle_sane_fwd.argtypes = [p] * 11 + [i, i, i, i, i]
     if hasattr(lib, "gdn_oracle_fwd"):
         lib.gdn_oracle_fwd.restype = ctypes.c_int
         lib.gdn_oracle_fwd.argtypes = [p, p, p, p, p, p, i, p, p,
@@ -257,3 +265,27 @@ def gdn_bwd(q, k, v, g, beta, dout, s0=None, dsT=None, cu_seqlens=None, nthreads
     out["dk"] = through_norm(kh, nk, dkh)
     out["ds0"] = gr["ds0"].sum(axis=0, keepdims=True) if shared else gr["ds0"]
     return out
+
+
+def sane_fwd(r, w, k, v, a, b, tau, sane_mask=None, s0=None, library=None):
+    """SANE forward.  r,w,k,a,b [B,T,H,K]; v [B,T,H,V]; tau [B,T//16,H] (> 0);
+    sane_mask [B,T//16] (nonzero = clip that chunk) or None (every chunk); s0
+    [B,H,K,V] or None.  Returns (o [B,T,H,V], sT [B,H,K,V]) in float64."""
+    r, w, k, v, a, b, tau = (_f64(x) for x in (r, w, k, v, a, b, tau))
+    B, T, H, K = r.shape
+    V = v.shape[-1]
+    assert tau.shape == (B, T // 16, H)
+    m = None
+    if sane_mask is not None:
+        m = sane_mask.cpu().numpy() if hasattr(sane_mask, "cpu") else np.asarray(sane_mask)
+        m = np.ascontiguousarray((m != 0).astype(np.uint8))
+        assert m.shape == (B, T // 16)
+    s0 = _f64(s0)
+    o = np.zeros((B, T, H, V))
+    sT = np.zeros((B, H, K, V))
+    lib = _load() if library is None else library
+    rc = lib.wkv7_oracle_sane_fwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                  _ptr(tau), _ptr(m), _ptr(s0), _ptr(o), _ptr(sT), B, T, H, K, V)
+    if rc != 0:
+        raise ValueError("wkv7_oracle_sane_fwd rejected its arguments")
+    return o, sT

@@ -418,3 +418,66 @@ int wkv7_oracle_bwd(const double* r, const double* w, const double* k,
     if (threads_used) *threads_used = used;
     return 0;
 }
+
+/*
+ * The generalized delta rule with State Anomaly Neutralization (SANE; rwkv-ops
+ * 0.9.0 README, "rwkv7op_sane 使用方法" and "rwkv7_op_sane_rnn 使用方法"): the
+ * recurrence of wkv7_oracle_fwd, and after every 16th token of a sequence (a chunk
+ * boundary) the state is soft-clipped with that chunk's tau[b, c, h] > 0 when the
+ * chunk's flag sane_mask[b, c] is nonzero (NULL: every chunk).  The outputs are read
+ * from the state before the clip (README: "output based on the state before SANE").
+ * The README defers the clip function to an external paper; the reading here is the
+ * elementwise soft clip S <- tau * tanh(S / tau).  A partial last chunk is not
+ * clipped (tau has T / 16 entries per sequence).  No token mask: padding is input
+ * values (README: k = 0, a = 0, w = -inf).
+ *
+ * Layouts: r, w, k, a, b [B,T,H,K]; v, o [B,T,H,V]; tau [B, T/16, H] (fp64 here);
+ * sane_mask [B, T/16] or NULL; s0 / sT [B,H,K,V].
+ */
+int wkv7_oracle_sane_fwd(const double* r, const double* w, const double* k,
+                         const double* v, const double* a, const double* b,
+                         const double* tau, const unsigned char* sane_mask,
+                         const double* s0, double* o, double* sT, int B, int T,
+                         int H, int K, int V) {
+    if (!r || !w || !k || !v || !a || !b || !tau || !o) return 1;
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0) return 1;
+    const int C = T / 16;  /* full 16-token chunks */
+    const size_t KV = (size_t)K * V;
+    double* S = (double*)malloc(sizeof(double) * (KV + V));
+    double* u = S + KV;
+    for (int bb = 0; bb < B; ++bb) {
+        for (int h = 0; h < H; ++h) {
+            const size_t state_off = ((size_t)bb * H + h) * KV;
+            if (s0)
+                memcpy(S, s0 + state_off, sizeof(double) * KV);
+            else
+                memset(S, 0, sizeof(double) * KV);
+            for (int t = 0; t < T; ++t) {
+                const size_t rowK = (((size_t)bb * T + t) * H + h) * (size_t)K;
+                const size_t rowV = (((size_t)bb * T + t) * H + h) * (size_t)V;
+                for (int j = 0; j < V; ++j) {
+                    u[j] = 0.0;
+                    for (int i = 0; i < K; ++i) u[j] += S[(size_t)i * V + j] * a[rowK + i];
+                }
+                for (int i = 0; i < K; ++i)
+                    for (int j = 0; j < V; ++j)
+                        S[(size_t)i * V + j] = exp(w[rowK + i]) * S[(size_t)i * V + j] +
+                                               b[rowK + i] * u[j] + k[rowK + i] * v[rowV + j];
+                for (int j = 0; j < V; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < K; ++i) acc += S[(size_t)i * V + j] * r[rowK + i];
+                    o[rowV + j] = acc;
+                }
+                const int c = t / 16;
+                if (t % 16 == 15 && c < C &&
+                    (!sane_mask || sane_mask[(size_t)bb * C + c] != 0)) {
+                    const double tc = tau[((size_t)bb * C + c) * H + h];
+                    for (size_t e = 0; e < KV; ++e) S[e] = tc * tanh(S[e] / tc);
+                }
+            }
+            if (sT) memcpy(sT + state_off, S, sizeof(double) * KV);
+        }
+    }
+    free(S);
+    return 0;
+}
