@@ -74,3 +74,34 @@ def test_backward_equals_finite_differences(sh):
         lm = loss()
         x[n][idx] = keep
         np.testing.assert_allclose(g["d" + n][idx], (lp - lm) / (2 * eps), rtol=1e-5, atol=1e-6)
+
+
+@settings(max_examples=10, deadline=None)
+@given(st.tuples(st.integers(1, 5), st.integers(1, 3), st.integers(1, 3), st.booleans(),
+                 st.integers(0, 2**31 - 1)))
+def test_gdn_backward_equals_finite_differences(sh):
+    T, K, V, shared, seed = sh
+    rng = np.random.default_rng(seed)
+    x = {"q": rng.standard_normal((2, T, 1, K)), "k": rng.standard_normal((2, T, 1, K)),
+         "v": rng.standard_normal((2, T, 1, V)), "g": -rng.random((2, T, 1)),
+         "beta": rng.random((2, T, 1)),
+         "s0": rng.standard_normal((1 if shared else 2, 1, K, V))}
+    dout = rng.standard_normal((2, T, 1, V))
+    dsT = rng.standard_normal((2, 1, K, V))
+    names = ("q", "k", "v", "g", "beta")
+    g = oracle.gdn_bwd(*(x[n] for n in names), dout, s0=x["s0"], dsT=dsT)
+
+    def loss():
+        o, sT, _ = oracle.gdn_fwd(*(x[n] for n in names), s0=x["s0"])
+        return float(np.sum(o * dout) + np.sum(sT * dsT))
+
+    eps = 1e-6
+    for n in names + ("s0",):
+        idx = tuple(rng.integers(0, d) for d in x[n].shape)
+        keep = x[n][idx]
+        x[n][idx] = keep + eps
+        lp = loss()
+        x[n][idx] = keep - eps
+        lm = loss()
+        x[n][idx] = keep
+        np.testing.assert_allclose(g["d" + n][idx], (lp - lm) / (2 * eps), rtol=1e-5, atol=1e-6)
