@@ -82,7 +82,8 @@ typedef enum {
  *   v              [B, T, H, V]  dtype
  *   s0             [N, H, K, V]  fp32    initial states, or NULL for zeros
  *                                        (README: initial_state=None)
- *   mask           [B, T]        uint8   nonzero = update, 0 = keep the state; NULL = all 1
+ *   mask           [B, T]        uint8   nonzero = update, 0 = keep the state; NULL = all 1;
+ *                                        with cu_seqlens it is [1, T] over the packed rows
  *   o              [B, T, H, V]  dtype   output, fully written (must not alias an input)
  *   sT             [N, H, K, V]  fp32    final states, or NULL to skip
  *                                        (README: output_final_state=False); may equal s0
@@ -162,13 +163,20 @@ wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v,
 
 /*
  * wkv7_bwd_noalloc -- wkv7_bwd with the library's own scratch instead of a caller
- * workspace.  The pages have no counterpart to this entry point: it exists so that a
- * caller without a device allocator can run the backward.  The scratch is a file-scope
- * device array of WKV7_STATIC_SCRATCH_BYTES, reserved when libwkv7.so's device code is
- * loaded (no allocation at call time).  Problems whose wkv7_bwd_workspace_bytes exceed
- * it return WKV7_ERR_UNSUPPORTED.  Calls share that one scratch: they must not overlap
- * in time (issue them on one stream, or synchronise between streams).  Arguments and
- * results are those of wkv7_bwd.
+ * workspace.  The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory (code that runs where cudaMalloc is forbidden or
+ * unavailable, such as a host framework that owns every allocation, or a path that
+ * must not call into the allocator).  The scratch is a file-scope device array of
+ * WKV7_STATIC_SCRATCH_BYTES that every GPU which loads the library keeps until exit.
+ * Problems whose wkv7_bwd_workspace_bytes exceed it return WKV7_ERR_UNSUPPORTED before
+ * anything is launched.  The call allocates nothing itself; it runs on the CURRENT
+ * device, which must be the device of every pointer and of the stream.  Its first call
+ * on a device looks up the array's address there (cudaGetSymbolAddress, cached per
+ * device); with CUDA's lazy module loading that first call may also load the library's
+ * device code, which is when the array is reserved -- make a first call (or any other
+ * call into the library) on each device before capturing a stream.  Every call shares
+ * the one array: calls that overlap on the GPU race (issue them on one stream, or
+ * synchronise between streams).  Arguments and results are those of wkv7_bwd.
  */
 #define WKV7_STATIC_SCRATCH_BYTES (64u << 20)
 
@@ -272,6 +280,22 @@ const char* wkv7_status_string(wkv7_status s);
 
 /* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
 int wkv7_version(void);
+
+/*
+ * wkv7_test_stall_next_chunked -- test hook of the failure path (no counterpart on the
+ * pages).  Every wait of the chunked kernel on an asynchronous copy or MMA is bounded
+ * (one second of device time); a thread that gives up raises WKV7_ERR_DEVICE_TIMEOUT,
+ * the CTA agrees on abandoning its sequence at its next barrier, waits (bounded) for
+ * the copies and MMAs it issued, frees its tensor memory and returns, so the context
+ * stays usable.  This call makes the NEXT chunked wkv7_fwd launch exercise that path
+ * without any fault: thread `tid` of the first CTA waits, with a 2 ms limit, on an
+ * mbarrier that nothing arrives at, right after its first chunk's inputs have landed
+ * (no copy or MMA in flight).  That sequence's outputs and final state are then not
+ * written; wkv7_get_last_error reports WKV7_ERR_DEVICE_TIMEOUT.  tid = -1 cancels;
+ * the hook is consumed by one launch.  Returns WKV7_ERR_INVALID_ARG for tid outside
+ * [-1, 256).
+ */
+wkv7_status wkv7_test_stall_next_chunked(int tid);
 
 #ifdef __cplusplus
 }

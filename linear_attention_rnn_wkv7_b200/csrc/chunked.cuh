@@ -249,10 +249,14 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
 }
 
 
-__device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int* abort_flag) {
+// Bounded wait on an mbarrier phase.  A thread that gives up raises the timeout flag
+// and records it in `timed_out`; it then carries on to the next CTA barrier, where
+// __syncthreads_or makes the decision to abandon the sequence the same for every
+// thread (no thread leaves while others wait at a barrier).
+__device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int& timed_out) {
     if (!sm100::mbar_wait(bar, parity)) {
         raise_flag(4 /* WKV7_ERR_DEVICE_TIMEOUT */);
-        *abort_flag = 1;
+        timed_out = 1;
     }
 }
 
@@ -270,7 +274,13 @@ struct Ctx {
     long long gb0;     // Gated DeltaNet: index of the first token's g / beta; gbs apart
     int gbs;
     int tma_y, tma_z;  // tile coordinates of the sequence start (dims 1 and 2 of the maps)
-    int* abort_flag;
+    int timed_out;     // this thread gave up on a wait (agreed on at the next CTA barrier)
+    uint32_t tma_par_last;  // parity of the last input load issued (drained on abort)
+    // Test hook of the timeout path: thread `stall_tid` of CTA 0 waits, with a short
+    // limit, on an mbarrier nothing arrives at (after chunk 0's inputs have landed, with
+    // no copy or MMA in flight).  -1 (every normal launch): off.
+    int stall_tid;
+    uint32_t bar_never;
     float* gamma_s;
     const CUtensorMap *tm_r, *tm_w, *tm_k, *tm_v, *tm_a, *tm_b;
     const __nv_bfloat16 *g, *beta;  // Gated DeltaNet only: [rows, H]
@@ -307,8 +317,10 @@ __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
 }
 
 // One 64-token chunk starting at token c0, in layout P (its inputs already requested).
+// Returns false, the same in every thread, when a bounded wait ran out: the caller then
+// abandons the sequence.
 template <bool kGdn, bool kHf>
-__device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
+__device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
     const LayR L = lay_of(par);
     using namespace sm100;
     uint8_t* smem = cx.smem;
@@ -319,7 +331,6 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
     const long long row0 = cx.row0;
     const uint8_t* mask = cx.mask;
     __nv_bfloat16* o = cx.o;
-    int* abort_flag = cx.abort_flag;
     float* gamma_s = cx.gamma_s;
     uint32_t& mma_phase = cx.mma_phase;
     float* scratch = reinterpret_cast<float*>(smem + L.ARK);  // prologue only
@@ -339,7 +350,11 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             bq[1] = __bfloat162float(cx.beta[tok + gbs]);
         }
     }
-    wait_or_abort(cx.bar_tma, par, abort_flag);
+    wait_or_abort(cx.bar_tma, par, cx.timed_out);
+    if (c0 == 0 && tid == cx.stall_tid && !sm100::mbar_wait_short(cx.bar_never, 0)) {
+        raise_flag(4 /* WKV7_ERR_DEVICE_TIMEOUT */);
+        cx.timed_out = 1;
+    }
 
         // ---- 2. prefix sums of w (mask folded) and every scaled operand, in one pass.
         //         Thread (q, j) owns tokens 2q, 2q+1 and channels 8j..8j+7: a shuffle
@@ -406,7 +421,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     nq[it] = sq > 0.f ? rsqrtf(sq) : 0.f;  // a zero vector stays zero
                     nk[it] = sk > 0.f ? rsqrtf(sk) : 0.f;
                 }
-                __syncthreads();
+                if (__syncthreads_or(cx.timed_out)) return false;  // a wait ran out: stop
                 float pre = 0.f, gL = 0.f;  // earlier warps' sum; g_L (log2 units)
 #pragma unroll
                 for (int w2 = 0; w2 < 8; ++w2) {
@@ -474,7 +489,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                     *reinterpret_cast<float4*>(wt + warp * 64 + h1) =
                         make_float4(incl[4], incl[5], incl[6], incl[7]);
                 }
-                __syncthreads();
+                if (__syncthreads_or(cx.timed_out)) return false;  // a wait ran out: stop
                 if (warp == 0) {  // per channel: exclusive prefixes over the warps, c = g_L, e^{g_L}
                     const int ch = cswz(2 * lane);  // channels 2 lane, 2 lane + 1
                     float2 gL = make_float2(0.f, 0.f);
@@ -579,7 +594,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         }
 
         // ---- 4. Gram wait ------------------------------------------------------------------
-        wait_or_abort(bar_mma, mma_phase, abort_flag);
+        wait_or_abort(bar_mma, mma_phase, cx.timed_out);
         mma_phase ^= 1;
         tc_fence_after();
 
@@ -665,7 +680,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             emit(1);
             fence_proxy_async();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(cx.timed_out)) return false;
         }
 
         // ---- 6. [W | Z] = T [Abar | A_ak], T = (I - A_ab)^-1, by block forward
@@ -801,7 +816,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
                           smem_desc(sbase + L.ABAR + 2048 * kk, L.AAK - L.ABAR, 1024), id, kk > 0);
             umma_commit(bar_mma);
         }
-        wait_or_abort(bar_mma, mma_phase, abort_flag);
+        wait_or_abort(bar_mma, mma_phase, cx.timed_out);
         mma_phase ^= 1;
         tc_fence_after();
 
@@ -890,12 +905,15 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             // previous chunk's epilogue 4 (or at the start).
             fence_proxy_async();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(cx.timed_out)) return false;
         }
 
         // The next chunk's inputs go to the other layout's input tiles, all of which
         // are dead now; the copy overlaps this chunk's final MMA and epilogue.
-        if (has_next && warp == 1) issue_loads<kGdn, kHf>(cx, c0 + 64, par ^ 1);
+        if (has_next) {
+            if (warp == 1) issue_loads<kGdn, kHf>(cx, c0 + 64, par ^ 1);
+            cx.tma_par_last = par ^ 1;
+        }
 
         // ---- 9. final MMA: [S upd; O] = A_fin [S0; V]  (128 x 64 x 128, fp16) ------------
         if (tid == 0) {
@@ -912,7 +930,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
             }
             umma_commit(bar_mma);
         }
-        wait_or_abort(bar_mma, mma_phase, abort_flag);
+        wait_or_abort(bar_mma, mma_phase, cx.timed_out);
         mma_phase ^= 1;
         tc_fence_after();
 
@@ -939,6 +957,7 @@ __device__ __forceinline__ void chunk(Ctx& cx, int c0, bool has_next, int par) {
         // No barrier: nothing the next chunk does before its own first barrier touches
         // what this epilogue reads or writes (o, the final product's output rows).
         tc_fence_before();
+        return true;
 }
 
 // kGdn: Gated DeltaNet (tm_r, tm_k, tm_v map q, k, v; g and beta per token; s0 may be
@@ -952,7 +971,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
                float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens,
                const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ beta,
-               int s0_shared) {
+               int s0_shared, int stall_tid) {
     extern __shared__ __align__(1024) uint8_t smem[];
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1028,7 +1047,10 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         cx.tma_y = h;
         cx.tma_z = (int)cx.row0;
     }
-    cx.abort_flag = reinterpret_cast<int*>(smem + OFF_MISC + 20);
+    cx.timed_out = 0;
+    cx.tma_par_last = 0;
+    cx.stall_tid = blockIdx.x == 0 ? stall_tid : -1;
+    cx.bar_never = sbase + OFF_MISC + 24;
     cx.gamma_s = reinterpret_cast<float*>(smem + OFF_GAMMA);
     cx.tm_r = &tm_r;
     cx.tm_w = &tm_w;
@@ -1047,7 +1069,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     if (tid == 0) {
         mbar_init(cx.bar_tma, 1);
         mbar_init(cx.bar_mma, 1);
-        *cx.abort_flag = 0;
+        mbar_init(cx.bar_never, 1);  // nothing ever arrives (the timeout test hook)
         fence_mbar_init();
     }
     tc_fence_before();
@@ -1093,13 +1115,22 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     tc_fence_before();
 
     // Chunks alternate between the two shared-memory layouts.
-    for (int c0 = 0, par = 0; c0 < cx.len; c0 += 64, par ^= 1) {
-        chunk<kGdn, kHf>(cx, c0, c0 + 64 < cx.len, par);
-        if (*cx.abort_flag) break;
-    }
+    bool ok = true;
+    for (int c0 = 0, par = 0; c0 < cx.len && ok; c0 += 64, par ^= 1)
+        ok = chunk<kGdn, kHf>(cx, c0, c0 + 64 < cx.len, par);
+    // The last chunk's final-MMA wait is agreed on here (it has no barrier of its own).
+    if (ok && __syncthreads_or(cx.timed_out)) ok = false;
 
     tc_fence_after();
-    if (cx.state_thread && sT && !*cx.abort_flag) {
+    if (!ok) {
+        // Abandoned: before the tensor memory is freed, wait (bounded again) for the
+        // last issued input copy and MMA, so that neither lands in memory this CTA no
+        // longer owns.  Waiting on a phase that has already completed returns at once.
+        if (tid == 0) {
+            (void)mbar_wait(cx.bar_tma, cx.tma_par_last);
+            (void)mbar_wait(cx.bar_mma, cx.mma_phase ^ 1u);
+        }
+    } else if (cx.state_thread && sT) {
         float sv[32];
         tmem_row<2>(cx.tmem + TM_DF, wq, 32 * wh, sv);
         float4* dst = reinterpret_cast<float4*>(sT + state_off + m_row * 64 + 32 * wh);
@@ -1163,7 +1194,7 @@ template <bool kGdn, bool kHf>
 inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float* s0,
                           const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
                           const int32_t* cu_seqlens, const void* g, const void* beta,
-                          int s0_shared, cudaStream_t stream) {
+                          int s0_shared, int stall_tid, cudaStream_t stream) {
     CUtensorMap maps[6];
     for (int i = 0; i < nmaps; ++i)
         if (!make_map(&maps[i], ptrs[i], B, T, H, kHf)) return cudaErrorInvalidValue;
@@ -1179,19 +1210,20 @@ inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float
     chunked_kernel<kGdn, kHf><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], s0, mask,
         static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens,
-        static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(beta), s0_shared);
+        static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(beta), s0_shared,
+        stall_tid);
     return cudaGetLastError();
 }
 template <bool kGdn>
 inline cudaError_t launch(const void* const* ptrs, int nmaps, const float* s0,
                           const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
                           const int32_t* cu_seqlens, const void* g, const void* beta,
-                          int s0_shared, int head_first, cudaStream_t stream) {
+                          int s0_shared, int head_first, int stall_tid, cudaStream_t stream) {
     return head_first
                ? launch_layout<kGdn, true>(ptrs, nmaps, s0, mask, o, sT, B, T, H, N, cu_seqlens,
-                                           g, beta, s0_shared, stream)
+                                           g, beta, s0_shared, stall_tid, stream)
                : launch_layout<kGdn, false>(ptrs, nmaps, s0, mask, o, sT, B, T, H, N, cu_seqlens,
-                                            g, beta, s0_shared, stream);
+                                            g, beta, s0_shared, stall_tid, stream);
 }
 }  // namespace chunked
 
@@ -1199,10 +1231,10 @@ inline cudaError_t launch_chunked(const void* r, const void* w, const void* k, c
                                   const void* a, const void* b, const float* s0,
                                   const uint8_t* mask, void* o, float* sT, int B, int T, int H,
                                   int N, const int32_t* cu_seqlens, int head_first,
-                                  cudaStream_t stream) {
+                                  int stall_tid, cudaStream_t stream) {
     const void* ptrs[6] = {r, w, k, v, a, b};
     return chunked::launch<false>(ptrs, 6, s0, mask, o, sT, B, T, H, N, cu_seqlens, nullptr,
-                                  nullptr, 0, head_first, stream);
+                                  nullptr, 0, head_first, stall_tid, stream);
 }
 
 // Gated DeltaNet: q, k, v [B*T, H, 64] bf16 through the r, k, v maps; g, beta [B*T, H]
@@ -1215,7 +1247,7 @@ inline cudaError_t launch_chunked_gdn(const void* q, const void* k, const void* 
     // map order r, w, k, v: the unused w slot repeats q
     const void* ptrs[4] = {q, q, k, v};
     return chunked::launch<true>(ptrs, 4, s0, nullptr, o, sT, B, T, H, N, cu_seqlens, g, beta,
-                                 s0_shared, head_first, stream);
+                                 s0_shared, head_first, -1, stream);
 }
 
 }  // namespace wkv7

@@ -32,13 +32,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: gives up after ~0.3 s and returns false (the caller flags it).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < (1u << 22); ++i) {
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait: gives up after kLimitNs of device time (or 2^30 polls, should the
+// timer not advance) and returns false; the caller flags it.
+template <uint64_t kLimitNs>
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0; i < (1u << 30); ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if (i > 32) __nanosleep(64);
+        if ((i & 63u) == 63u && globaltimer_ns() - t0 > kLimitNs) return false;
     }
     return false;
+}
+// The kernels' waits: one second (a TMA copy or an MMA group takes microseconds).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    return mbar_wait_for<1000000000ull>(bar, parity);
+}
+// Two milliseconds: only the timeout test hook uses it.
+__device__ __forceinline__ bool mbar_wait_short(uint32_t bar, uint32_t parity) {
+    return mbar_wait_for<2000000ull>(bar, parity);
 }
 
 // ---- proxies / fences -----------------------------------------------------------

@@ -3,6 +3,8 @@
 // in the kernels included below; this file only validates and launches.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "wkv7.h"
 #include "common.cuh"
 #include "step.cuh"
@@ -20,9 +22,29 @@ constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
 constexpr size_t kStaticScratchBytes = WKV7_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
+// The array's device address, looked up once per device with that device current (in
+// host code the symbol is only a host-side stand-in, never a device address).
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_scratch_addr[kMaxDevices];
+
+// Address of the static scratch on the current device, or nullptr on a CUDA error.
+void* static_scratch_on_current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_scratch_addr[dev].store(p, std::memory_order_release);
+    return p;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+
+// Test hook of the chunked kernel's timeout path (wkv7_test_stall_next_chunked):
+// consumed, and reset to -1, by the next chunked WKV7 launch.
+std::atomic<int> g_stall_tid{-1};
 
 // Head sizes with a kernel: K == V in {64, 128, 256} (the chunked form: 64 only).
 inline bool head_size_ok(int K, int V) { return K == V && (K == 64 || K == 128 || K == 256); }
@@ -50,6 +72,12 @@ const char* wkv7_status_string(wkv7_status s) {
 }
 
 int wkv7_version(void) { return kVersion; }
+
+wkv7_status wkv7_test_stall_next_chunked(int tid) {
+    if (tid < -1 || tid >= wkv7::chunked::kThreads) return WKV7_ERR_INVALID_ARG;
+    g_stall_tid.store(tid);
+    return WKV7_OK;
+}
 
 wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
                      const void* a, const void* b, const float* s0, const uint8_t* mask,
@@ -91,7 +119,7 @@ wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
     if (chunked) {
         if (dtype != WKV7_BF16 || K != 64 || !wkv7::kChunkedBuilt) return WKV7_ERR_UNSUPPORTED;
         err = wkv7::launch_chunked(r, w, k, v, a, b, s0, mask, o, sT, B, T, H, N, cu_seqlens,
-                                   hf, stream);
+                                   hf, g_stall_tid.exchange(-1), stream);
     } else if (dtype == WKV7_BF16) {
         err = wkv7::launch_recurrent<__nv_bfloat16>(r, w, k, v, a, b, s0, mask, o, sT, T, H, N,
                                                     cu_seqlens, hf, K, stream);
@@ -264,8 +292,8 @@ wkv7_status wkv7_bwd_noalloc(const void* r, const void* w, const void* k, const 
                              wkv7_layout layout, wkv7_dtype dtype, void* stream) {
     const size_t need = wkv7_bwd_workspace_bytes(B, T, H, K, V, N);
     if (need > kStaticScratchBytes) return WKV7_ERR_UNSUPPORTED;
-    void* scratch = nullptr;
-    if (cudaGetSymbolAddress(&scratch, g_static_scratch) != cudaSuccess) return WKV7_ERR_CUDA;
+    void* scratch = static_scratch_on_current_device();
+    if (!scratch) return WKV7_ERR_CUDA;
     return wkv7_bwd(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da, db, ds0, B, T, H,
                     K, V, cu_seqlens, N, layout, dtype, scratch, kStaticScratchBytes, stream);
 }

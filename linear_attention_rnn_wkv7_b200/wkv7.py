@@ -70,6 +70,8 @@ def library() -> ctypes.CDLL:
         lib.wkv7_status_string.argtypes = [i]
         lib.wkv7_version.restype = i
         lib.wkv7_version.argtypes = []
+        lib.wkv7_test_stall_next_chunked.restype = i
+        lib.wkv7_test_stall_next_chunked.argtypes = [i]
         _lib = lib
     return _lib
 
@@ -264,12 +266,20 @@ def wkv7_bwd_noalloc(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_se
     g = {n: torch.empty(kshape, dtype=dt, device=r.device) for n in ("dr", "dw", "dk", "da", "db")}
     g["dv"] = torch.empty(vshape, dtype=dt, device=r.device)
     g["ds0"] = torch.empty((N, H, K, V), dtype=torch.float32, device=r.device)
-    st = library().wkv7_bwd_noalloc(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
-                                    _ptr(s0), _ptr(mask), _ptr(dout), _ptr(dsT), _ptr(g["dr"]),
-                                    _ptr(g["dw"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]),
-                                    _ptr(g["db"]), _ptr(g["ds0"]), B, T, H, K, V,
-                                    _ptr(cu_seqlens), N, int(bool(head_first)), _dtype_code(r),
-                                    _stream(r.device))
+    for name, t in (("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("dout", dout),
+                    ("s0", s0), ("dsT", dsT), ("mask", mask), ("cu_seqlens", cu_seqlens)):
+        if t is not None and t.device != r.device:
+            raise ValueError(f"{name} is on {t.device}, r on {r.device}: one device only")
+    # The library's static scratch is per device: the call must run with r's device
+    # current, which is also the device of the stream passed.
+    with torch.cuda.device(r.device):
+        st = library().wkv7_bwd_noalloc(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                        _ptr(s0), _ptr(mask), _ptr(dout), _ptr(dsT),
+                                        _ptr(g["dr"]), _ptr(g["dw"]), _ptr(g["dk"]),
+                                        _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["db"]),
+                                        _ptr(g["ds0"]), B, T, H, K, V, _ptr(cu_seqlens), N,
+                                        int(bool(head_first)), _dtype_code(r),
+                                        _stream(r.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_bwd_noalloc")
     return g

@@ -149,3 +149,31 @@ def test_bwd_head_first_batched(cuda_device):
                  dsT=dsT.to(cuda_device), head_first=True)
     g = {n: (t.transpose(1, 2) if n != "ds0" else t) for n, t in g.items()}
     check_grads(g, ref, torch.bfloat16, "bwd head_first")
+
+
+def test_bwd_varlen_with_mask(cuda_device):
+    """Packed sequences with a padding mask over the packed rows (masked tokens at
+    sequence starts and ends and at checkpoint boundaries)."""
+    lengths = torch.tensor([17, 0, 8, 1, 130, 63])
+    x = synth.varlen_inputs(lengths, 2, dtype=torch.float32, seed=670, s0_std=0.1)
+    cu = x.pop("cu_seqlens")
+    total, N = int(lengths.sum()), lengths.numel()
+    g = torch.Generator().manual_seed(671)
+    mask = (torch.rand(1, total, generator=g) >= 0.2).to(torch.uint8)
+    for s0_, L in zip(cu[:-1].tolist(), lengths.tolist()):
+        if L > 0:
+            mask[0, s0_] = 0
+            mask[0, s0_ + L - 1] = 0
+        if L > 16:
+            mask[0, s0_ + 8] = 0
+            mask[0, s0_ + 15] = 0
+    dout, _ = upstream(1, total, 2, torch.float32, 672)
+    dsT = torch.randn(N, 2, 64, 64, generator=torch.Generator().manual_seed(673)) * 0.1
+    ref = oracle.bwd(*(x[n] for n in NAMES), dout, s0=x["s0"], mask=mask, dsT=dsT,
+                     cu_seqlens=cu)
+    xd = to_dev(x, cuda_device)
+    gr = wkv7_bwd(*(xd[n] for n in NAMES), dout.to(cuda_device), s0=xd["s0"],
+                  mask=mask.to(cuda_device), dsT=dsT.to(cuda_device),
+                  cu_seqlens=cu.to(cuda_device))
+    check_grads(gr, ref, torch.float32, "bwd varlen + mask")
+    assert wkv7_get_last_error() == OK

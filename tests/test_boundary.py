@@ -193,3 +193,12 @@ def test_bwd_rejects_bad_arguments(lib):
     assert call(N=2) == ERR_INVALID_ARG  # N must equal B without cu_seqlens
     assert call(layout=3) == ERR_INVALID_ARG
     assert call(B=0) == OK
+
+
+def test_stall_hook_arguments(lib):
+    """The timeout-path test hook takes a thread index of the chunked kernel's CTA, or
+    -1 to cancel; nothing is launched by the call itself."""
+    assert lib.wkv7_test_stall_next_chunked(-2) == ERR_INVALID_ARG
+    assert lib.wkv7_test_stall_next_chunked(256) == ERR_INVALID_ARG
+    assert lib.wkv7_test_stall_next_chunked(5) == OK
+    assert lib.wkv7_test_stall_next_chunked(-1) == OK

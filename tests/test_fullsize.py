@@ -78,18 +78,28 @@ def test_fwd_varlen_64seq_h32(cuda_device):
 
 
 def test_step_b1024_h32(cuda_device):
+    """The decode workload at its stated length: 256 consecutive in-place steps over
+    1024 x 32 states.  o is compared at every step (rel <= 2e-2) and the state after
+    the last step (rel <= 1e-3) on 64 sampled states, the first and last included;
+    the oracle steps those states in fp64 from the same initial values."""
     p = synth.WORKLOADS["step_bf16_b1024_h32_256steps"]
-    B, H, steps = p["B"], p["H"], 16
+    B, H, steps = p["B"], p["H"], p["steps"]
+    assert steps == 256
     state = synth.decode_state(B, H, seed=p["seed"], std=p["s0_std"])
-    units = _sample_units(B, H, 8, p["seed"])
+    units = _sample_units(B, H, 64, p["seed"])
+    assert (0, 0) in units and (B - 1, H - 1) in units
     idx_b = [u[0] for u in units]
     idx_h = [u[1] for u in units]
     ref = state[idx_b, idx_h].double().numpy()[:, None]  # [U,1,K,V]
     st = state.to(cuda_device)
+    worst_o = 0.0
     for i in range(steps):
         x = synth.decode_step_inputs(B, H, dtype=torch.bfloat16, seed=p["seed"], step=i)
         o = wkv7_step(*(x[n].to(cuda_device) for n in "rwkvab"), st)
         sub = {n: x[n][idx_b, idx_h][:, None] for n in "rwkvab"}  # [U,1,K]
         o_ref, ref = oracle.step(*(sub[n] for n in "rwkvab"), ref)
-        assert rel_err(o[idx_b, idx_h][:, None], o_ref) <= BF16_O_REL
-    assert rel_err(st[idx_b, idx_h][:, None], ref) <= BF16_S_REL
+        e = rel_err(o[idx_b, idx_h][:, None], o_ref)
+        worst_o = max(worst_o, e)
+        assert e <= BF16_O_REL, f"step {i}: o rel {e:.3e}"
+    es = rel_err(st[idx_b, idx_h][:, None], ref)
+    assert es <= BF16_S_REL, f"state after {steps} steps: rel {es:.3e} (worst o {worst_o:.3e})"

@@ -247,3 +247,37 @@ def test_head_first_varlen(cuda_device, algo):
     o, s = wkv7_fwd(*(hf[n] for n in "rwkvab"), s0=hf["s0"], cu_seqlens=cu.to(cuda_device),
                     algo=algo, head_first=True)
     check(o.transpose(1, 2), s, o_ref, s_ref, torch.bfloat16, f"head_first varlen {algo}")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("head_first", [False, True])
+def test_varlen_with_mask(cuda_device, algo, head_first):
+    """Packed sequences (cu_seqlens) together with a padding mask: the mask is [1, sum L]
+    over the packed token rows (rwkv-ops 0.9.0 README, "rwkv7op 使用方法": mask[b, t] = 0
+    leaves the state unchanged at that token).  Masked tokens fall at sequence starts,
+    ends, chunk boundaries and the interior; one sequence is masked throughout."""
+    lengths = torch.tensor([70, 0, 1, 129, 64, 200, 33], dtype=torch.int64)
+    x = synth.varlen_inputs(lengths, 2, dtype=torch.bfloat16, seed=320, s0_std=0.1)
+    cu = x.pop("cu_seqlens")
+    total = int(lengths.sum())
+    g = torch.Generator().manual_seed(321)
+    mask = (torch.rand(1, total, generator=g) >= 0.15).to(torch.uint8)
+    starts = cu[:-1].tolist()
+    for s0_, L in zip(starts, lengths.tolist()):
+        if L > 0:
+            mask[0, s0_] = 0               # first token of every sequence
+            mask[0, s0_ + L - 1] = 0       # last token
+        if L > 64:
+            mask[0, s0_ + 63] = 0          # a chunk's last token
+            mask[0, s0_ + 64] = 0          # and the next chunk's first
+    mask[0, starts[4]:starts[4] + 64] = 0  # the 64-token sequence is masked throughout
+    o_ref, s_ref = ref(x, mask=mask, cu=cu)
+    xd = to_dev(x, cuda_device)
+    if head_first:
+        xd = {n: (_head_first(xd[n]) if n != "s0" else xd[n]) for n in xd}
+    o, s = wkv7_fwd(*(xd[n] for n in "rwkvab"), s0=xd["s0"], mask=mask.to(cuda_device),
+                    cu_seqlens=cu.to(cuda_device), algo=algo, head_first=head_first)
+    if head_first:
+        o = o.transpose(1, 2)
+    check(o, s, o_ref, s_ref, torch.bfloat16, f"varlen+mask {algo} head_first={head_first}")
+    torch.testing.assert_close(s[4].cpu(), x["s0"][4], rtol=0, atol=0)
