@@ -138,12 +138,11 @@ __device__ __forceinline__ uint32_t swe(uint32_t row, uint32_t col) {
     return sw(row, col >> 3) + ((col & 7u) << 1);
 }
 
-// Float index of element (r, c) of diagonal 16x16 block bb of A_ab, kept in fp32
-// (rows 20 floats apart, so the float4 chunks eight rows write together fall in eight
-// different bank groups; blocks 324 floats apart, so the two blocks a warp reads
-// together do too).
-__device__ __forceinline__ int didx(int bb, int r, int c) {
-    return bb * 324 + r * 20 + c;
+// Float index of element (row t, column s) of diagonal 16x16 block bb of A_ab, kept in
+// fp32 and stored transposed (s-major, rows 20 floats apart; blocks 336 floats apart,
+// so the two blocks one warp writes and reads together sit 16 banks apart).
+__device__ __forceinline__ int dtidx(int bb, int s, int t) {
+    return bb * 336 + s * 20 + t;
 }
 
 // Position of channel c in a 64-float per-channel row (prologue scratch, e^{g_L},
@@ -656,17 +655,10 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                         float* dg = reinterpret_cast<float*>(smem + L.A);
 #pragma unroll
                         for (int b2 = 2 * h; b2 < 2 * h + 2; ++b2) {
-                            if (bt == b2) {
+                            if (bt == b2) {  // the diagonal block, transposed
 #pragma unroll
-                                for (int c4 = 0; c4 < 4; ++c4) {
-                                    const int s0_ = 16 * b2 + 4 * c4;
-                                    float4 x;
-                                    x.x = (s0_ + 0 < t) ? v[s0_ + 0] : 0.f;
-                                    x.y = (s0_ + 1 < t) ? v[s0_ + 1] : 0.f;
-                                    x.z = (s0_ + 2 < t) ? v[s0_ + 2] : 0.f;
-                                    x.w = (s0_ + 3 < t) ? v[s0_ + 3] : 0.f;
-                                    *reinterpret_cast<float4*>(dg + didx(b2, t & 15, 4 * c4)) = x;
-                                }
+                                for (int s2 = 0; s2 < 16; ++s2)
+                                    dg[dtidx(b2, s2, t & 15)] = (16 * b2 + s2 < t) ? v[16 * b2 + s2] : 0.f;
                             }
                         }
                     }
@@ -678,6 +670,38 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             emit(0);
             tmem_ld_wait();
             emit(1);
+            if (wq >= 2 && wh == 1) {
+                // The warps holding A_ab's rows invert their own two diagonal blocks,
+                // T_bb = (I - N_bb)^-1 with N_bb strictly lower, while the other warps
+                // finish this epilogue.  Lane (block, column c) solves (I - N) x = e_c
+                // column-wise: once x[s] is final it is added into every later x[t], so
+                // the dependent chain is one FMA per row.  T_bb goes out as fp16.
+                __syncwarp();
+                const int bb = 2 * (wq - 2) + (lane >> 4), c = lane & 15;
+                const float* nt = reinterpret_cast<const float*>(smem + L.A) + dtidx(bb, 0, 0);
+                float x[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) x[t] = (t == c) ? 1.f : 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 15; ++s2) {
+                    const float xs = x[s2];
+#pragma unroll
+                    for (int t4 = ((s2 + 1) >> 2) << 2; t4 < 16; t4 += 4) {
+                        const float4 n4 = *reinterpret_cast<const float4*>(nt + s2 * 20 + t4);
+                        const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (t4 + e > s2) x[t4 + e] = fmaf(nv[e], xs, x[t4 + e]);
+                    }
+                }
+                uint8_t* Tb = smem + L.K;  // fp16 16x16 blocks with 48-byte rows
+#pragma unroll
+                for (int t = 0; t < 16; t += 2) {  // column c: rows t and t + 1
+                    const uint32_t hp = pack2h(x[t], x[t + 1]);
+                    *reinterpret_cast<uint16_t*>(Tb + bb * 768 + t * 48 + 2 * c) = (uint16_t)(hp & 0xFFFFu);
+                    *reinterpret_cast<uint16_t*>(Tb + bb * 768 + (t + 1) * 48 + 2 * c) = (uint16_t)(hp >> 16);
+                }
+            }
             fence_proxy_async();
             tc_fence_before();
             if (__syncthreads_or(cx.timed_out)) return false;
@@ -693,37 +717,10 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
         //         place over the right-hand side (fp16), where MMA-3 reads it as its
         //         MN-major B operand. ------------------------------------------------
         {
-            const float* Dg = reinterpret_cast<const float*>(smem + L.A);  // diagonal blocks of A_ab
-            // fp16 16x16 blocks with rows of 48 bytes: T_ii (4), then T_ii A_im (6).
+            // fp16 16x16 blocks with rows of 48 bytes: T_ii (4, from epilogue 1), then
+            // T_ii A_im (6).
             uint8_t* Tb = smem + L.K;
             uint8_t* Tab = Tb + 4 * 768;
-            if (tid < 64) {  // diagonal block b, column c
-                const int b = tid >> 4, c = tid & 15;
-                float x[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) x[i] = 0.f;
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                    for (int s4 = 0; s4 < t; s4 += 4) {
-                        const float4 a4 = *reinterpret_cast<const float4*>(Dg + didx(b, t, s4));
-                        acc0 = fmaf(a4.x, x[s4 + 0], acc0);
-                        acc1 = fmaf(a4.y, x[s4 + 1], acc1);
-                        acc0 = fmaf(a4.z, x[s4 + 2], acc0);
-                        acc1 = fmaf(a4.w, x[s4 + 3], acc1);
-                    }
-                    x[t] = (t == c) ? 1.f : acc0 + acc1;
-                }
-#pragma unroll
-#pragma unroll
-                for (int t = 0; t < 16; t += 2) {  // fp16, column c: rows t and t + 1
-                    const uint32_t hp = pack2h(x[t], x[t + 1]);
-                    *reinterpret_cast<uint16_t*>(Tb + b * 768 + t * 48 + 2 * c) = (uint16_t)(hp & 0xFFFFu);
-                    *reinterpret_cast<uint16_t*>(Tb + b * 768 + (t + 1) * 48 + 2 * c) = (uint16_t)(hp >> 16);
-                }
-            }
-            __syncthreads();
             const int g = lane >> 2, q = lane & 3;
             uint8_t* xt = smem + (warp < 4 ? L.ABAR : L.AAK);  // tile of this warp's columns
             const int nb = 2 * (warp & 3);                     // first 16-byte chunk of them
