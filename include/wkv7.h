@@ -188,6 +188,63 @@ wkv7_status wkv7_bwd_noalloc(const void* r, const void* w, const void* k, const 
                              wkv7_layout layout, wkv7_dtype dtype, void* stream);
 
 /*
+ * wkv7_sane_fwd -- the WKV7 forward with State Anomaly Neutralization
+ * (generalized_delta_rule_sane / generalized_delta_rule_sane_inference; rwkv-ops 0.9.0
+ * README, "rwkv7op_sane 使用方法").  The recurrence of wkv7_fwd, and after the last
+ * token of every full 16-token chunk c (tokens 16 c .. 16 c + 15, c < T / 16) whose
+ * flag is set, the state is soft-clipped elementwise with that chunk's tau:
+ *
+ *     S <- tau[b, c, h] * tanh(S / tau[b, c, h])
+ *
+ * The output of token 16 c + 15 is read from the state before the clip (README: the
+ * output is based on the state before SANE).  A partial last chunk is not clipped
+ * (tau holds T / 16 chunks; README: the inference kernel reads tau per chunk, so T
+ * need not be a multiple of 16).  The README defers the clip function to the SANE
+ * paper; tau * tanh(S / tau) is the reading implemented (parity for the function
+ * itself is unpinned by the pages).
+ *
+ *   r, w, k, v, a, b  as for wkv7_fwd ([B, T, H, *], or [B, H, T, *] with
+ *                     WKV7_LAYOUT_BHTK); no token mask and no packed sequences
+ *   tau            [B, T / 16, H]  fp32  > 0 (README: softplus(param) + 1); may be NULL
+ *                                        only when T < 16
+ *   sane_mask      [B, T / 16]   uint8   nonzero = clip after that chunk, 0 = skip (README:
+ *                                        per-chunk 0/1 shared by all heads); NULL = every chunk
+ *   s0             [B, H, K, V]  fp32    initial states or NULL; with s0_shared = 1 a single
+ *                                        [1, H, K, V] state used by every batch row
+ *   o              [B, T, H, V]  dtype   output; sT [B, H, K, V] fp32 or NULL (may equal s0
+ *                                        unless s0_shared with B > 1)
+ *   K = V in {64, 128, 256}; dtype bf16 or fp32 (fp32 state and arithmetic throughout).
+ *
+ * Runs on the fp32 CUDA-core recurrent kernel.  Returns WKV7_ERR_INVALID_ARG /
+ * WKV7_ERR_UNSUPPORTED before any launch on bad arguments, WKV7_ERR_CUDA if the
+ * launch fails.  The caller owns every buffer.
+ */
+wkv7_status wkv7_sane_fwd(const void* r, const void* w, const void* k, const void* v,
+                          const void* a, const void* b, const float* tau,
+                          const uint8_t* sane_mask, const float* s0, int s0_shared, void* o,
+                          float* sT, int B, int T, int H, int K, int V, wkv7_layout layout,
+                          wkv7_dtype dtype, void* stream);
+
+/*
+ * wkv7_sane_step -- one decode token with State Anomaly Neutralization
+ * (rwkv7_op_sane_rnn; rwkv-ops 0.9.0 README, "rwkv7_op_sane_rnn 使用方法").  The step
+ * of wkv7_step; then, for the batch rows whose flag is set, the state written back is
+ * soft-clipped with tau[b, h] as in wkv7_sane_fwd.  o is read from the state before
+ * the clip.  The README's loop calls it with do_sane = (step % 16 == 15).
+ *
+ *   r, w, k, v, a, b, state, o   as for wkv7_step ([B, H, K], state [B, H, K, V] in place)
+ *   tau            [B, H]        fp32    > 0
+ *   do_sane        [B]           uint8   nonzero = clip that row; NULL = do_sane_all (0 or 1)
+ *                                        for every row (README: do_sane is a bool or [B])
+ *
+ * Errors and ownership as for wkv7_step.
+ */
+wkv7_status wkv7_sane_step(const void* r, const void* w, const void* k, const void* v,
+                           const void* a, const void* b, const float* tau,
+                           const uint8_t* do_sane, int do_sane_all, float* state, void* o,
+                           int B, int H, int K, int V, wkv7_dtype dtype, void* stream);
+
+/*
  * wkv7_gdn_fwd -- Gated DeltaNet forward over whole sequences
  * (gated_delta_net_recurrent / gated_delta_net_recurrent_inference /
  * gated_delta_net_chunk; rwkv-ops 0.9.0 README, "gdn_recurrent 使用方法" and

@@ -24,6 +24,14 @@
 // packed varlen sequences and null s0 / sT are handled here exactly as in the
 // chunked kernel.
 //
+// kSane: State Anomaly Neutralization (rwkv-ops 0.9.0 README, "rwkv7op_sane 使用方法"):
+// after token 16 c + 15 of a sequence (c < T / 16, a full 16-token chunk) whose flag
+// sane[b, c] is set (no flags: every chunk), each state entry is soft-clipped,
+// S <- tau * tanh(S / tau) with tau = tau[b, c, h] > 0.  The token's output is read
+// before the clip.  The README defers the clip function to its paper; tau * tanh(S /
+// tau) is the reading taken (the state stays within (-tau, tau) and is unchanged to
+// first order where |S| << tau).
+//
 // kGdn: Gated DeltaNet (rwkv-ops 0.9.0 README, "gdn_recurrent 使用方法").  The
 // conversion turns q, k, v, g, beta into the generalized rule's per-token vectors:
 // r = qh, exp(w) = e^{g} on every channel, write key beta kh, a = kh and
@@ -52,14 +60,15 @@ __device__ __forceinline__ void cp_async_wait() {
 }  // namespace rec
 
 // K (= V): head size.  Block: 64 columns x P = K / 64 threads per column, 64 rows each.
-template <typename Tin, bool kGdn, int K>
+template <typename Tin, bool kGdn, int K, bool kSane = false>
 __global__ void __launch_bounds__(K)
 recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
                  const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
                  const float* s0, const uint8_t* __restrict__ mask, Tin* __restrict__ o,
                  float* sT, int T, int H, const int32_t* __restrict__ cu_seqlens,
                  const Tin* __restrict__ g, const Tin* __restrict__ beta, int s0_shared,
-                 int head_first) {
+                 int head_first, const float* __restrict__ tau,
+                 const uint8_t* __restrict__ sane_flags) {
     using namespace rec;
     constexpr int P = K / 64;        // threads per state column
     constexpr int R = 64;            // rows per thread
@@ -233,6 +242,15 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
                 const size_t row = (tb + (size_t)(t0 + tt) * ts) * K;
                 o[row + col] = from_f32<Tin>(ov);
             }
+            if constexpr (kSane) {  // the output above was read before the clip
+                const int tg = t0 + tt, ch = tg >> 4, C = T >> 4;  // no packed sequences here
+                if ((tg & 15) == 15 && ch < C &&
+                    (!sane_flags || sane_flags[(size_t)bb * C + ch] != 0)) {
+                    const float tc = tau[((size_t)bb * C + ch) * H + h];
+#pragma unroll
+                    for (int i = 0; i < R; ++i) S[i] = tc * tanhf(S[i] / tc);
+                }
+            }
         }
     }
     cp_async_wait<0>();  // nothing is left in flight when the block exits
@@ -242,18 +260,19 @@ recurrent_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
     }
 }
 
-template <typename Tin, bool kGdn, int K>
+template <typename Tin, bool kGdn, int K, bool kSane = false>
 cudaError_t launch_recurrent_k(const void* r, const void* w, const void* k, const void* v,
                                const void* a, const void* b, const float* s0,
                                const uint8_t* mask, void* o, float* sT, int T, int H, int N,
                                const int32_t* cu_seqlens, const void* g, const void* beta,
-                               int s0_shared, int head_first, cudaStream_t stream) {
+                               int s0_shared, int head_first, cudaStream_t stream,
+                               const float* tau = nullptr, const uint8_t* sane_flags = nullptr) {
     const long long blocks = (long long)N * H * (K / 64);
-    recurrent_kernel<Tin, kGdn, K><<<(unsigned)blocks, K, 0, stream>>>(
+    recurrent_kernel<Tin, kGdn, K, kSane><<<(unsigned)blocks, K, 0, stream>>>(
         static_cast<const Tin*>(r), static_cast<const Tin*>(w), static_cast<const Tin*>(k),
         static_cast<const Tin*>(v), static_cast<const Tin*>(a), static_cast<const Tin*>(b), s0,
         mask, static_cast<Tin*>(o), sT, T, H, cu_seqlens, static_cast<const Tin*>(g),
-        static_cast<const Tin*>(beta), s0_shared, head_first);
+        static_cast<const Tin*>(beta), s0_shared, head_first, tau, sane_flags);
     return cudaGetLastError();
 }
 
@@ -300,6 +319,35 @@ cudaError_t launch_recurrent_gdn(const void* q, const void* k, const void* v, co
     return launch_recurrent_any<Tin, true>(K, q, nullptr, k, v, nullptr, nullptr, s0, nullptr,
                                            o, sT, T, H, N, cu_seqlens, g, beta, s0_shared,
                                            head_first, stream);
+}
+
+// SANE forward: the WKV7 recurrence with the soft clip after every 16th token (kSane);
+// tau [B, T / 16, H] fp32, sane_flags [B, T / 16] (or NULL: every full chunk); no mask and
+// no packed sequences; s0 may be one [1, H, K, V] state shared by every batch row.
+template <typename Tin>
+cudaError_t launch_recurrent_sane(const void* r, const void* w, const void* k, const void* v,
+                                  const void* a, const void* b, const float* tau,
+                                  const uint8_t* sane_flags, const float* s0, int s0_shared,
+                                  void* o, float* sT, int B, int T, int H, int head_first, int K,
+                                  cudaStream_t stream) {
+    switch (K) {
+        case 64:
+            return launch_recurrent_k<Tin, false, 64, true>(r, w, k, v, a, b, s0, nullptr, o, sT, T,
+                                                            H, B, nullptr, nullptr, nullptr,
+                                                            s0_shared, head_first, stream, tau,
+                                                            sane_flags);
+        case 128:
+            return launch_recurrent_k<Tin, false, 128, true>(r, w, k, v, a, b, s0, nullptr, o, sT,
+                                                             T, H, B, nullptr, nullptr, nullptr,
+                                                             s0_shared, head_first, stream, tau,
+                                                             sane_flags);
+        case 256:
+            return launch_recurrent_k<Tin, false, 256, true>(r, w, k, v, a, b, s0, nullptr, o, sT,
+                                                             T, H, B, nullptr, nullptr, nullptr,
+                                                             s0_shared, head_first, stream, tau,
+                                                             sane_flags);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace wkv7

@@ -21,6 +21,12 @@
 // norms, reduced across the warp), so the same update applies
 // e^{g} (I - beta kh kh^T) S + beta kh v^T.
 //
+// kSane: rwkv7_op_sane_rnn (rwkv-ops 0.9.0 README, "rwkv7_op_sane_rnn 使用方法"): when
+// the unit's batch row is flagged (do_sane[b], or one flag for all), the state written
+// back is soft-clipped, S <- tau * tanh(S / tau) with tau[b, h] > 0, while the output
+// is read from the state before the clip (the reading of the clip function is the
+// forward's, see recurrent.cuh).
+//
 // Head sizes 128 and 256 (step_kernel_wide): one block per (unit, 64-column slab)
 // with K / 64 warps, warp p holding rows 64 p .. 64 p + 63 of the slab in the same
 // lane layout as above; the K-reductions of u and o add the warps' partial sums
@@ -32,12 +38,20 @@ namespace wkv7 {
 
 constexpr int kStepWarps = 4;  // units per block
 
-template <typename Tin, bool kGdn>
+// Soft clip of the SANE step (4 state entries).
+__device__ __forceinline__ float4 sane_clip4(float4 s, float tc) {
+    return make_float4(tc * tanhf(s.x / tc), tc * tanhf(s.y / tc), tc * tanhf(s.z / tc),
+                       tc * tanhf(s.w / tc));
+}
+
+template <typename Tin, bool kGdn, bool kSane = false>
 __global__ void __launch_bounds__(kStepWarps * 32)
 step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
             const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
             float* __restrict__ state, Tin* __restrict__ o, long long units,
-            const Tin* __restrict__ g, const Tin* __restrict__ beta) {
+            const Tin* __restrict__ g, const Tin* __restrict__ beta,
+            const float* __restrict__ tau, const uint8_t* __restrict__ do_sane,
+            int do_sane_all, int H) {
     __shared__ __align__(16) float vec[kStepWarps][5][64];  // r, d = exp(w), k, a, b
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -48,6 +62,12 @@ step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
     float4* S_g = reinterpret_cast<float4*>(state + (size_t)unit * 64 * 64);
     const int c = lane & 15;  // float4 column group
     const int p = lane >> 4;  // row half
+    bool clip = false;  // SANE: this unit's state is clipped after the step (warp-uniform)
+    float tc = 1.f;
+    if constexpr (kSane) {
+        clip = do_sane ? do_sane[unit / H] != 0 : do_sane_all != 0;
+        if (clip) tc = tau[unit];
+    }
 
     // Issue the 16 KiB state read first so it overlaps the vector staging.
     float4 S[32];
@@ -138,7 +158,7 @@ step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
             acc.y = fmaf(s.y, rv[q], acc.y);
             acc.z = fmaf(s.z, rv[q], acc.z);
             acc.w = fmaf(s.w, rv[q], acc.w);
-            S_g[(32 * p + 4 * m4 + q) * 16 + c] = s;
+            S_g[(32 * p + 4 * m4 + q) * 16 + c] = (kSane && clip) ? sane_clip4(s, tc) : s;
         }
     }
     acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
@@ -149,12 +169,13 @@ step_kernel(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __r
 }
 
 // K = V in {128, 256}: block = K / 64 warps on one 64-column slab of one unit.
-template <typename Tin, bool kGdn, int K>
+template <typename Tin, bool kGdn, int K, bool kSane = false>
 __global__ void __launch_bounds__(32 * (K / 64))
 step_kernel_wide(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin* __restrict__ k,
                  const Tin* __restrict__ v, const Tin* __restrict__ a, const Tin* __restrict__ b,
                  float* __restrict__ state, Tin* __restrict__ o, const Tin* __restrict__ g,
-                 const Tin* __restrict__ beta) {
+                 const Tin* __restrict__ beta, const float* __restrict__ tau,
+                 const uint8_t* __restrict__ do_sane, int do_sane_all, int H) {
     constexpr int P = K / 64;  // warps = row parts = column slabs per unit
     __shared__ __align__(16) float vec[5][K];  // r, d = exp(w), k, a, b
     __shared__ __align__(16) float part_u[P][64];
@@ -170,6 +191,12 @@ step_kernel_wide(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
     const int ph = lane >> 4; // row half of the part
     const int row0 = 64 * warp + 32 * ph;
     const int col0 = 64 * slab + 4 * c;
+    bool clip = false;  // SANE (block-uniform)
+    float tc = 1.f;
+    if constexpr (kSane) {
+        clip = do_sane ? do_sane[unit / H] != 0 : do_sane_all != 0;
+        if (clip) tc = tau[unit];
+    }
 
     float4 S[32];
 #pragma unroll
@@ -269,7 +296,8 @@ step_kernel_wide(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
             acc.y = fmaf(s.y, rv[q], acc.y);
             acc.z = fmaf(s.z, rv[q], acc.z);
             acc.w = fmaf(s.w, rv[q], acc.w);
-            *reinterpret_cast<float4*>(Su + (size_t)(row0 + 4 * m4 + q) * K + col0) = s;
+            *reinterpret_cast<float4*>(Su + (size_t)(row0 + 4 * m4 + q) * K + col0) =
+                (kSane && clip) ? sane_clip4(s, tc) : s;
         }
     }
     acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
@@ -292,10 +320,12 @@ step_kernel_wide(const Tin* __restrict__ r, const Tin* __restrict__ w, const Tin
     }
 }
 
-template <typename Tin, bool kGdn>
+template <typename Tin, bool kGdn, bool kSane = false>
 cudaError_t launch_step_any(int K, const void* r, const void* w, const void* k, const void* v,
                             const void* a, const void* b, float* state, void* o, long long units,
-                            const void* g, const void* beta, cudaStream_t stream) {
+                            const void* g, const void* beta, cudaStream_t stream,
+                            const float* tau = nullptr, const uint8_t* do_sane = nullptr,
+                            int do_sane_all = 0, int H = 1) {
     const Tin *r_ = static_cast<const Tin*>(r), *w_ = static_cast<const Tin*>(w),
               *k_ = static_cast<const Tin*>(k), *v_ = static_cast<const Tin*>(v),
               *a_ = static_cast<const Tin*>(a), *b_ = static_cast<const Tin*>(b),
@@ -303,14 +333,14 @@ cudaError_t launch_step_any(int K, const void* r, const void* w, const void* k, 
     Tin* o_ = static_cast<Tin*>(o);
     if (K == 64) {
         const long long blocks = (units + kStepWarps - 1) / kStepWarps;
-        step_kernel<Tin, kGdn><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
-            r_, w_, k_, v_, a_, b_, state, o_, units, g_, be_);
+        step_kernel<Tin, kGdn, kSane><<<(unsigned)blocks, kStepWarps * 32, 0, stream>>>(
+            r_, w_, k_, v_, a_, b_, state, o_, units, g_, be_, tau, do_sane, do_sane_all, H);
     } else if (K == 128) {
-        step_kernel_wide<Tin, kGdn, 128><<<(unsigned)(units * 2), 64, 0, stream>>>(
-            r_, w_, k_, v_, a_, b_, state, o_, g_, be_);
+        step_kernel_wide<Tin, kGdn, 128, kSane><<<(unsigned)(units * 2), 64, 0, stream>>>(
+            r_, w_, k_, v_, a_, b_, state, o_, g_, be_, tau, do_sane, do_sane_all, H);
     } else if (K == 256) {
-        step_kernel_wide<Tin, kGdn, 256><<<(unsigned)(units * 4), 128, 0, stream>>>(
-            r_, w_, k_, v_, a_, b_, state, o_, g_, be_);
+        step_kernel_wide<Tin, kGdn, 256, kSane><<<(unsigned)(units * 4), 128, 0, stream>>>(
+            r_, w_, k_, v_, a_, b_, state, o_, g_, be_, tau, do_sane, do_sane_all, H);
     } else {
         return cudaErrorInvalidValue;
     }
@@ -333,6 +363,17 @@ cudaError_t launch_step_gdn(const void* q, const void* k, const void* v, const v
                             cudaStream_t stream) {
     return launch_step_any<Tin, true>(K, q, nullptr, k, v, nullptr, nullptr, state, o, units, g,
                                       beta, stream);
+}
+
+// SANE step: the WKV7 step, then the soft clip of the written state for flagged batch
+// rows; tau [units] = [B, H] fp32, do_sane [B] (or NULL: do_sane_all for every row).
+template <typename Tin>
+cudaError_t launch_step_sane(const void* r, const void* w, const void* k, const void* v,
+                             const void* a, const void* b, const float* tau,
+                             const uint8_t* do_sane, int do_sane_all, float* state, void* o,
+                             long long units, int H, int K, cudaStream_t stream) {
+    return launch_step_any<Tin, false, true>(K, r, w, k, v, a, b, state, o, units, nullptr,
+                                             nullptr, stream, tau, do_sane, do_sane_all, H);
 }
 
 }  // namespace wkv7

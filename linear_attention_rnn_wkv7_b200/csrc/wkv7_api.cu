@@ -226,6 +226,68 @@ wkv7_status wkv7_gdn_step(const void* q, const void* k, const void* v, const voi
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 
+wkv7_status wkv7_sane_fwd(const void* r, const void* w, const void* k, const void* v,
+                          const void* a, const void* b, const float* tau,
+                          const uint8_t* sane_mask, const float* s0, int s0_shared, void* o,
+                          float* sT, int B, int T, int H, int K, int V, wkv7_layout layout,
+                          wkv7_dtype dtype, void* stream_) {
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
+    if (layout != WKV7_LAYOUT_BTHK && layout != WKV7_LAYOUT_BHTK) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (s0_shared != 0 && s0_shared != 1) return WKV7_ERR_INVALID_ARG;
+    if (!head_size_ok(K, V)) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)B * H;
+    const long long rows = (long long)B * T * H;
+    if (units * (K / 64) > 0x7fffffffLL || rows > (1LL << 40) || (long long)B * T > 0x7fffffffLL)
+        return WKV7_ERR_UNSUPPORTED;
+    const bool tokens = rows > 0;
+    if (tokens && (!ok_ptr(r) || !ok_ptr(w) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(a) ||
+                   !ok_ptr(b) || !ok_ptr(o)))
+        return WKV7_ERR_INVALID_ARG;
+    if (T >= 16 && B > 0 && !ok_scalar_ptr(tau, WKV7_F32)) return WKV7_ERR_INVALID_ARG;
+    if ((s0 && !aligned16(s0)) || (sT && !aligned16(sT))) return WKV7_ERR_INVALID_ARG;
+    if (tokens && (o == r || o == w || o == k || o == v || o == a || o == b))
+        return WKV7_ERR_INVALID_ARG;
+    if (s0_shared && sT && s0 == sT && B > 1) return WKV7_ERR_INVALID_ARG;
+    if (units == 0) return WKV7_OK;
+    if (!s0) s0_shared = 0;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const int hf = layout == WKV7_LAYOUT_BHTK;
+    const cudaError_t err =
+        dtype == WKV7_BF16
+            ? wkv7::launch_recurrent_sane<__nv_bfloat16>(r, w, k, v, a, b, tau, sane_mask, s0,
+                                                         s0_shared, o, sT, B, T, H, hf, K, stream)
+            : wkv7::launch_recurrent_sane<float>(r, w, k, v, a, b, tau, sane_mask, s0, s0_shared,
+                                                 o, sT, B, T, H, hf, K, stream);
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+wkv7_status wkv7_sane_step(const void* r, const void* w, const void* k, const void* v,
+                           const void* a, const void* b, const float* tau,
+                           const uint8_t* do_sane, int do_sane_all, float* state, void* o,
+                           int B, int H, int K, int V, wkv7_dtype dtype, void* stream_) {
+    if (B < 0 || H <= 0 || K <= 0 || V <= 0) return WKV7_ERR_INVALID_ARG;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
+    if (do_sane_all != 0 && do_sane_all != 1) return WKV7_ERR_INVALID_ARG;
+    if (!head_size_ok(K, V)) return WKV7_ERR_UNSUPPORTED;
+    const long long units = (long long)B * H;
+    if (units == 0) return WKV7_OK;
+    if (units > (1LL << 33) || units * (K / 64) > 0x7fffffffLL) return WKV7_ERR_UNSUPPORTED;
+    if (!ok_ptr(r) || !ok_ptr(w) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(a) || !ok_ptr(b) ||
+        !ok_ptr(state) || !ok_ptr(o) || !ok_scalar_ptr(tau, WKV7_F32))
+        return WKV7_ERR_INVALID_ARG;
+    if (o == state || o == r || o == w || o == k || o == v || o == a || o == b)
+        return WKV7_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const cudaError_t err =
+        dtype == WKV7_BF16
+            ? wkv7::launch_step_sane<__nv_bfloat16>(r, w, k, v, a, b, tau, do_sane, do_sane_all,
+                                                    state, o, units, H, K, stream)
+            : wkv7::launch_step_sane<float>(r, w, k, v, a, b, tau, do_sane, do_sane_all, state,
+                                            o, units, H, K, stream);
+    return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
 size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N) {
     if (B < 0 || T < 0 || H <= 0 || N < 0 || K != 64 || V != 64) return 0;
     return wkv7::bwd::workspace_floats((long long)B * T, N, H) * sizeof(float);

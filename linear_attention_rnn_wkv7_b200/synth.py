@@ -25,7 +25,7 @@ import math
 import torch
 import torch.nn.functional as F
 
-__all__ = ["fwd_inputs", "padding_mask", "varlen_lengths", "decode_state",
+__all__ = ["fwd_inputs", "padding_mask", "sane_tau", "varlen_lengths", "decode_state",
            "decode_step_inputs", "gdn_inputs", "gdn_varlen_inputs", "gdn_step_inputs",
            "WORKLOADS"]
 
@@ -104,6 +104,13 @@ def gdn_step_inputs(B: int, H: int, K: int = 64, V: int = 64,
     """One Gated DeltaNet decode step: q, k [B,H,K], v [B,H,V], g, beta [B,H]."""
     g = torch.Generator().manual_seed(seed * 1_000_003 + 1 + step)
     return _gdn_vectors(g, (B, H, K), (B, H, V), dtype)
+
+
+def sane_tau(B: int, C: int, H: int, seed: int) -> torch.Tensor:
+    """fp32 [B, C, H] SANE clip levels, softplus(z) + 1 with z ~ N(0, 1) (the README's
+    preprocessing of tau: softplus(param) + 1, so tau > 1)."""
+    g = torch.Generator().manual_seed(seed * 7177 + 11)
+    return (F.softplus(torch.randn(B, C, H, generator=g)) + 1.0).contiguous()
 
 
 def padding_mask(B: int, T: int, seed: int, max_suffix: int = 1024,

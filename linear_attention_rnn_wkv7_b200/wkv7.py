@@ -72,6 +72,10 @@ def library() -> ctypes.CDLL:
         lib.wkv7_version.argtypes = []
         lib.wkv7_test_stall_next_chunked.restype = i
         lib.wkv7_test_stall_next_chunked.argtypes = [i]
+        lib.wkv7_sane_fwd.restype = i
+        lib.wkv7_sane_fwd.argtypes = [p] * 9 + [i, p, p, i, i, i, i, i, i, i, p]
+        lib.wkv7_sane_step.restype = i
+        lib.wkv7_sane_step.argtypes = [p] * 8 + [i, p, p, i, i, i, i, i, p]
         _lib = lib
     return _lib
 
@@ -174,6 +178,95 @@ def wkv7_step(r, w, k, v, a, b, state, o=None):
                              _ptr(o), B, H, K, V, _dtype_code(r), _stream(r.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_step")
+    return o
+
+
+def _flags_u8(x, name, shape):
+    """A 0/1 flag tensor (bool, uint8 or float 0/1, as the README's SANE flags) as uint8."""
+    if x.dtype != torch.uint8:
+        x = (x != 0).to(torch.uint8)
+    _check(x.contiguous(), name, torch.uint8, shape)
+    return x.contiguous()
+
+
+def wkv7_sane_fwd(r, w, k, v, a, b, tau, sane_mask=None, s0=None,
+                  output_final_state: bool = True, o=None, sT=None, head_first: bool = False):
+    """WKV7 forward with State Anomaly Neutralization (generalized_delta_rule_sane): the
+    state is soft-clipped, S <- tau * tanh(S / tau), after every full 16-token chunk
+    whose flag is set; outputs are read before the clip.  r,w,k,a,b [B,T,H,K], v
+    [B,T,H,V] (or [B,H,T,*] with head_first), bf16 or fp32; tau [B,T//16,H] fp32 > 0;
+    sane_mask [B,T//16] (bool / uint8 / float 0-1) or None (every chunk); s0 [B,H,K,V]
+    or [1,H,K,V] fp32 or None.  Returns (o shaped like v, sT [B,H,K,V] or None).
+    Unlike the README's wrapper, the final state is returned whenever asked for, with or
+    without sane_mask."""
+    _check(r, "r")
+    dt = r.dtype
+    if head_first:
+        B, H, T, K = r.shape
+    else:
+        B, T, H, K = r.shape
+    V = v.shape[-1]
+    kshape = (B, H, T, K) if head_first else (B, T, H, K)
+    vshape = (B, H, T, V) if head_first else (B, T, H, V)
+    for name, t in (("w", w), ("k", k), ("a", a), ("b", b)):
+        _check(t, name, dt, kshape)
+    _check(v, "v", dt, vshape)
+    C = T // 16
+    _check(tau, "tau", torch.float32, (B, C, H))
+    if sane_mask is not None:
+        sane_mask = _flags_u8(sane_mask, "sane_mask", (B, C))
+    shared = 0
+    if s0 is not None:
+        _check(s0, "s0", torch.float32)
+        if tuple(s0.shape) == (1, H, K, V) and B != 1:
+            shared = 1
+        elif tuple(s0.shape) != (B, H, K, V):
+            raise ValueError(f"s0 must have shape {(B, H, K, V)} or {(1, H, K, V)}")
+    if o is None:
+        o = torch.empty(vshape, dtype=dt, device=r.device)
+    else:
+        _check(o, "o", dt, vshape)
+    if output_final_state and sT is None:
+        sT = torch.empty((B, H, K, V), dtype=torch.float32, device=r.device)
+    elif sT is not None:
+        _check(sT, "sT", torch.float32, (B, H, K, V))
+    st = library().wkv7_sane_fwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                 _ptr(tau), _ptr(sane_mask), _ptr(s0), shared, _ptr(o), _ptr(sT),
+                                 B, T, H, K, V, int(bool(head_first)), _dtype_code(r),
+                                 _stream(r.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_sane_fwd")
+    return o, sT
+
+
+def wkv7_sane_step(r, w, k, v, a, b, tau, do_sane, state, o=None):
+    """One decode token with State Anomaly Neutralization (rwkv7_op_sane_rnn).
+    r,w,k,a,b [B,H,K]; v [B,H,V]; tau [B,H] fp32 > 0; do_sane a bool (every row) or a
+    [B] flag tensor; state [B,H,K,V] fp32, updated in place (clipped where flagged).
+    Returns o [B,H,V], read from the state before the clip."""
+    _check(r, "r")
+    dt = r.dtype
+    B, H, K = r.shape
+    V = v.shape[-1]
+    for name, t in (("w", w), ("k", k), ("a", a), ("b", b)):
+        _check(t, name, dt, (B, H, K))
+    _check(v, "v", dt, (B, H, V))
+    _check(tau, "tau", torch.float32, (B, H))
+    _check(state, "state", torch.float32, (B, H, K, V))
+    flags, every = None, 0
+    if isinstance(do_sane, torch.Tensor):
+        flags = _flags_u8(do_sane, "do_sane", (B,))
+    else:
+        every = int(bool(do_sane))
+    if o is None:
+        o = torch.empty((B, H, V), dtype=dt, device=r.device)
+    else:
+        _check(o, "o", dt, (B, H, V))
+    st = library().wkv7_sane_step(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                  _ptr(tau), _ptr(flags), every, _ptr(state), _ptr(o), B, H, K,
+                                  V, _dtype_code(r), _stream(r.device))
+    if st != OK:
+        raise WKV7Error(st, "wkv7_sane_step")
     return o
 
 

@@ -289,3 +289,22 @@ def sane_fwd(r, w, k, v, a, b, tau, sane_mask=None, s0=None, library=None):
     if rc != 0:
         raise ValueError("wkv7_oracle_sane_fwd rejected its arguments")
     return o, sT
+
+
+def sane_step(r, w, k, v, a, b, tau, do_sane, state, nthreads: int = 0):
+    """SANE single step (README, "rwkv7_op_sane_rnn 使用方法"): one step of the recurrence
+    (``step``), the output read from the state before the clip, then the soft clip
+    S <- tau * tanh(S / tau) of the rows whose flag is set.  r,w,k,a,b [B,H,K], v [B,H,V],
+    tau [B,H] (> 0), do_sane a bool or [B] flags, state [B,H,K,V] (not modified).
+    Returns (o [B,H,V], new_state [B,H,K,V]) in float64.  The clip function is the
+    reading taken for SANE (parity unpinned by the pages)."""
+    o, new = step(r, w, k, v, a, b, state, nthreads=nthreads)
+    tau = _f64(tau)
+    B = new.shape[0]
+    flags = np.broadcast_to(np.asarray(
+        do_sane.cpu().numpy() if hasattr(do_sane, "cpu") else do_sane) != 0, (B,))
+    for bb in range(B):
+        if flags[bb]:
+            tc = tau[bb][:, None, None]
+            new[bb] = tc * np.tanh(new[bb] / tc)
+    return o, new

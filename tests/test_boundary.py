@@ -202,3 +202,32 @@ def test_stall_hook_arguments(lib):
     assert lib.wkv7_test_stall_next_chunked(256) == ERR_INVALID_ARG
     assert lib.wkv7_test_stall_next_chunked(5) == OK
     assert lib.wkv7_test_stall_next_chunked(-1) == OK
+
+
+def test_sane_entry_points_reject_bad_arguments(lib):
+    """wkv7_sane_fwd / wkv7_sane_step: host checks before any launch."""
+    p = [ctypes.c_void_p(P + 0x1000 * i) for i in range(8)]
+    tau = ctypes.c_void_p(P + 0x20000)
+    o = ctypes.c_void_p(P + 0x30000)
+    # forward: T >= 16 needs tau; layout, dtype and s0_shared range; head size; aliasing
+    assert lib.wkv7_sane_fwd(*p[:6], None, None, None, 0, o, None, 1, 32, 2, 64, 64, 0, 0,
+                             None) == ERR_INVALID_ARG
+    assert lib.wkv7_sane_fwd(*p[:6], tau, None, None, 0, o, None, 1, 32, 2, 64, 64, 2, 0,
+                             None) == ERR_INVALID_ARG
+    assert lib.wkv7_sane_fwd(*p[:6], tau, None, None, 2, o, None, 1, 32, 2, 64, 64, 0, 0,
+                             None) == ERR_INVALID_ARG
+    assert lib.wkv7_sane_fwd(*p[:6], tau, None, None, 0, o, None, 1, 32, 2, 96, 96, 0, 0,
+                             None) == ERR_UNSUPPORTED
+    assert lib.wkv7_sane_fwd(*p[:6], tau, None, None, 0, p[0], None, 1, 32, 2, 64, 64, 0, 0,
+                             None) == ERR_INVALID_ARG
+    assert lib.wkv7_sane_fwd(*p[:6], ctypes.c_void_p(P + 2), None, None, 0, o, None, 1, 32, 2,
+                             64, 64, 0, 0, None) == ERR_INVALID_ARG
+    # T < 16 needs no tau; B = 0 launches nothing
+    assert lib.wkv7_sane_fwd(*p[:6], None, None, None, 0, o, None, 0, 15, 2, 64, 64, 0, 0,
+                             None) == OK
+    # step: tau required, do_sane_all in {0, 1}, state and o distinct
+    st = ctypes.c_void_p(P + 0x40000)
+    assert lib.wkv7_sane_step(*p[:6], None, None, 1, st, o, 2, 2, 64, 64, 0, None) == ERR_INVALID_ARG
+    assert lib.wkv7_sane_step(*p[:6], tau, None, 2, st, o, 2, 2, 64, 64, 0, None) == ERR_INVALID_ARG
+    assert lib.wkv7_sane_step(*p[:6], tau, None, 1, st, st, 2, 2, 64, 64, 0, None) == ERR_INVALID_ARG
+    assert lib.wkv7_sane_step(*p[:6], tau, None, 1, st, o, 2, 2, 96, 96, 0, None) == ERR_UNSUPPORTED

@@ -94,3 +94,19 @@ def test_clip_bounds_the_state():
     _, sT = oracle.sane_fwd(*(x[n] for n in NAMES), tau, s0=s0 * 10)
     assert np.all(np.abs(sT) <= tau[:, 0][:, :, None, None])
     assert np.abs(sT).max() > 0.5 * tau.min()
+
+
+def test_sane_step_matches_the_forward():
+    """oracle.sane_step (NumPy, per step) driven as the README's loop (do_sane at step %
+    16 == 15, per-row flags) equals the C SANE forward on the same tokens."""
+    rng = np.random.default_rng(5)
+    x, s0, tau = problem(rng, B=3, T=48, scale=2.0)
+    mask = np.array([[1, 1, 0], [0, 1, 1], [1, 0, 1]])
+    o, sT = oracle.sane_fwd(*(x[n] for n in NAMES), tau, sane_mask=mask, s0=s0)
+    state = s0.copy()
+    for t in range(48):
+        c = t // 16
+        flags = mask[:, c] if t % 16 == 15 else np.zeros(3)
+        ot, state = oracle.sane_step(*(x[n][:, t] for n in NAMES), tau[:, c], flags, state)
+        np.testing.assert_allclose(ot, o[:, t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(state, sT, rtol=1e-12, atol=1e-12)
