@@ -13,7 +13,9 @@ Under torchrun (N > 1) every rank runs its own replica of the workload (the
 rank 0 prints the whole-job throughput: all ranks' tokens / max-over-ranks time.
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample instead.
 ``--family gdn`` measures the Gated DeltaNet entry points (wkv7_gdn_fwd /
-wkv7_gdn_step) on workloads of the same shapes instead.
+wkv7_gdn_step) on workloads of the same shapes instead; ``--family sane`` the
+State Anomaly Neutralization ones (wkv7_sane_fwd with the clip after every 16-token
+chunk, wkv7_sane_step with do_sane every 16th step).
 """
 from __future__ import annotations
 
@@ -42,6 +44,8 @@ GDN_METRIC = "Gated DeltaNet fwd tokens/s (B=8,T=4096,H=64,D=64 bf16) + decode H
 GDN_FWD = synth.WORKLOADS["gdn_fwd_bf16_b8_t4096_h64"]
 GDN_DEC = synth.WORKLOADS["gdn_step_bf16_b1024_h32_256steps"]
 GDN_TOKEN_HEAD_BYTES = 3 * 64 * 2 + 2 * 2 + 64 * 2  # q,k,v + g,beta in, o out, bf16
+SANE_METRIC = ("SANE fwd tokens/s (B=8,T=4096,H=64,D=64 bf16, clip every 16 tokens) + decode "
+               "HBM GB/s vs peak")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -185,7 +189,9 @@ def reference_arm(args, rank: int):
         return
     import oracle
     gdn = args.family == "gdn"
+    sane = args.family == "sane"
     H, T = FWD["H"], FWD["T"]
+    tau = None
     if gdn:
         x = synth.gdn_inputs(1, T, H, dtype=torch.bfloat16, seed=GDN_FWD["seed"],
                              s0_std=GDN_FWD["s0_std"])
@@ -195,9 +201,15 @@ def reference_arm(args, rank: int):
                              s0_std=FWD["s0_std"])
         names, call = tuple("rwkvab"), oracle.fwd
     units = min(H, max(4, os.cpu_count() or 1))  # one whole (b, h) unit per host thread
+    if sane:  # the SANE oracle runs its units one after another on one host thread
+        units = 2
+        tau = synth.sane_tau(1, T // 16, H, FWD["seed"])[:, :, :units]
     sl = {n: x[n][:, :, :units] for n in names}
 
     def one():
+        if sane:
+            oracle.sane_fwd(*(sl[n] for n in names), tau, s0=x["s0"][:, :units])
+            return 1
         return call(*(sl[n] for n in names), s0=x["s0"][:, :units])[2]
 
     for _ in range(args.warmup):
@@ -209,12 +221,13 @@ def reference_arm(args, rank: int):
     dt = time.perf_counter() - t0
     tokens = args.steps * units * T / H
     value = tokens / dt
-    line = {"metric": GDN_METRIC if gdn else METRIC, "value": value, "unit": "tokens/s",
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+    fam = "gdn_" if gdn else "sane_" if sane else ""
+    line = {"metric": GDN_METRIC if gdn else SANE_METRIC if sane else METRIC, "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": fwd_config({"workload": ("gdn_" if gdn else "") + "fwd_bf16_b8_t4096_h64",
+            "config": fwd_config({"workload": fam + "fwd_bf16_b8_t4096_h64",
                                   "B": FWD["B"], "T": T, "H": H}, "oracle", args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
                              "sample": f"each step: {units} of the 512 (b,h) units of "
@@ -246,9 +259,9 @@ def main():
     ap.add_argument("--head-size", type=int, choices=[64, 128, 256], default=64,
                     help="K = V; 128 / 256 keep C = H x head size at 4096 (forward) and "
                          "2048 (decode), and run on the CUDA-core kernels")
-    ap.add_argument("--family", choices=["wkv7", "gdn"], default="wkv7",
+    ap.add_argument("--family", choices=["wkv7", "gdn", "sane"], default="wkv7",
                     help="gdn: the Gated DeltaNet entry points on the B=8,T=4096,H=64 "
-                         "forward and 1024x32 decode workloads")
+                         "forward and 1024x32 decode workloads; sane: the SANE ones")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -261,7 +274,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
 
     from linear_attention_rnn_wkv7_b200 import (library, wkv7_bwd, wkv7_fwd, wkv7_gdn_bwd,
-                                                wkv7_gdn_fwd, wkv7_gdn_step, wkv7_step)
+                                                wkv7_gdn_fwd, wkv7_gdn_step, wkv7_sane_fwd,
+                                                wkv7_sane_step, wkv7_step)
     library()  # fail loudly if the CUDA library is missing
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
@@ -284,25 +298,30 @@ def main():
     stream = torch.cuda.current_stream(device)
     fwd = None
     gdn = args.family == "gdn"
+    sane = args.family == "sane"
+    fwd_fn = wkv7_gdn_fwd if gdn else wkv7_sane_fwd if sane else wkv7_fwd
+    step_fn = wkv7_gdn_step if gdn else wkv7_sane_step if sane else wkv7_step
     if args.only in ("all", "fwd"):
-        fwd = fwd_leg(args, device, stream, wkv7_gdn_fwd if gdn else wkv7_fwd, hbm_peak,
-                      peak_kind, max_over_ranks, barrier, rank, world)
+        fwd = fwd_leg(args, device, stream, fwd_fn, hbm_peak, peak_kind, max_over_ranks,
+                      barrier, rank, world)
     decode = None
     if args.only in ("all", "decode") and not args.no_decode:
-        decode = decode_leg(device, stream, wkv7_gdn_step if gdn else wkv7_step, hbm_peak,
-                            peak_kind, max_over_ranks, barrier, rank, gdn, args.head_size)
+        decode = decode_leg(device, stream, step_fn, hbm_peak, peak_kind, max_over_ranks,
+                            barrier, rank, gdn, args.head_size, sane=sane)
     backward = None
     if (args.only in ("all", "bwd") and not args.no_bwd and args.head_size == 64
-            and args.workload == "b8_t4096_h64"):
+            and args.workload == "b8_t4096_h64" and not sane):
         backward = bwd_leg(args, device, stream, wkv7_gdn_bwd if gdn else wkv7_bwd, hbm_peak,
                            peak_kind, max_over_ranks, barrier, rank, gdn)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu and args.only == "all" and args.head_size == 64:
+    if (rank == 0 and world == 1 and not args.no_cpu and args.only == "all"
+            and args.head_size == 64 and not sane):
         cpu = cpu_oracle_sample(gdn=gdn)
 
     if rank == 0:
         desc = fwd["desc"] if fwd else {"workload": "none"}
-        line = {"metric": GDN_METRIC if gdn else METRIC, "value": fwd and fwd["value"],
+        line = {"metric": GDN_METRIC if gdn else SANE_METRIC if sane else METRIC,
+                "value": fwd and fwd["value"],
                 "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": fwd and fwd["ms_per_step"], "higher_is_better": True,
@@ -332,6 +351,20 @@ def fwd_workload(args, rank):
                 {"workload": f"gdn_fwd_bf16_b{B}_t{T}_h{H}{tag}", "B": B, "T": T, "H": H})
     if args.head_size != 64 and args.workload != "b8_t4096_h64":
         raise SystemExit("--head-size applies to the b8_t4096_h64 workload only")
+    if args.family == "sane":
+        if args.workload != "b8_t4096_h64":
+            raise SystemExit("--family sane runs the b8_t4096_h64 workload only")
+        D = args.head_size
+        B, T, H = args.batch, FWD["T"], FWD["H"] * 64 // D
+        seed = replicas.replica_seed(FWD["seed"], rank)
+        x = synth.fwd_inputs(B, T, H, K=D, V=D, dtype=torch.bfloat16, seed=seed,
+                             s0_std=FWD["s0_std"])
+        x["tau"] = synth.sane_tau(B, T // 16, H, seed)
+        tag = "" if D == 64 else f"_d{D}"
+        nbytes = fwd_algorithmic_bytes(B, T, H, D) + x["tau"].numel() * 4
+        return (x, None, None, B, T, H, B * T, nbytes,
+                {"workload": f"sane_fwd_bf16_b{B}_t{T}_h{H}{tag}", "B": B, "T": T, "H": H,
+                 "sane": "clip after every 16-token chunk"})
     if args.workload == "b8_t4096_h64":
         D = args.head_size
         B, T, H = args.batch, FWD["T"], FWD["H"] * 64 // D
@@ -386,6 +419,10 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
         def step():
             wkv7_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], s0=xd["s0"],
                      algo=args.algo, o=o, sT=sT)
+    elif args.family == "sane":
+        def step():
+            wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], xd["tau"],
+                     s0=xd["s0"], o=o, sT=sT)
     else:
         def step():
             wkv7_fwd(xd["r"], xd["w"], xd["k"], xd["v"], xd["a"], xd["b"], s0=xd["s0"],
@@ -413,6 +450,8 @@ def fwd_leg(args, device, stream, wkv7_fwd, hbm_peak, peak_kind, max_over_ranks,
     kernel = "chunked" if args.algo in ("auto", "chunked") and D == 64 else "recurrent"
     if args.family == "gdn":
         kernel = "gdn_" + kernel
+    elif args.family == "sane":
+        kernel = "sane_recurrent"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
                 "kernel": kernel,
@@ -520,9 +559,10 @@ def wkv7_bwd_workspace_nbytes(B, T, H):
 
 
 def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank,
-               gdn=False, D=64):
-    """256 consecutive wkv7_step (or wkv7_gdn_step) calls over 1024 x 32 fp32 states
-    (512 MiB, > L2).  Step inputs: 32 independently drawn step sets, used in turn."""
+               gdn=False, D=64, sane=False):
+    """256 consecutive wkv7_step (or wkv7_gdn_step, wkv7_sane_step) calls over 1024 x 32
+    fp32 states (512 MiB, > L2).  Step inputs: 32 independently drawn step sets, used in
+    turn; SANE clips every state after every 16th step (do_sane = step % 16 == 15)."""
     p = GDN_DEC if gdn else DEC
     B, H, steps = p["B"], p["H"] * 64 // D, p["steps"]
     state = synth.decode_state(B, H, K=D, V=D, seed=replicas.replica_seed(p["seed"], rank),
@@ -535,10 +575,14 @@ def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, b
                  seed=replicas.replica_seed(p["seed"], rank), step=i)
         sets.append(tuple(x[n].to(device) for n in names))
     o = torch.empty(B, H, D, dtype=torch.bfloat16, device=device)
+    tau = synth.sane_tau(B, 1, H, replicas.replica_seed(p["seed"], rank))[:, 0].contiguous().to(device)
 
     def run(n):
         for i in range(n):
-            wkv7_step(*sets[i % len(sets)], state, o=o)
+            if sane:
+                wkv7_step(*sets[i % len(sets)], tau, i % 16 == 15, state, o=o)
+            else:
+                wkv7_step(*sets[i % len(sets)], state, o=o)
 
     run(3)
     torch.cuda.synchronize(device)
@@ -551,15 +595,18 @@ def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, b
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
     nbytes = gdn_step_algorithmic_bytes(B, H, D) if gdn else step_algorithmic_bytes(B, H, D)
+    if sane:
+        nbytes += B * H * 4  # tau
     gbs = nbytes / (ms / 1e3) / 1e9
     tag = "" if D == 64 else f"_d{D}"
-    return {"workload": ("gdn_" if gdn else "") + f"step_bf16_b{B}_h{H}_256steps{tag}",
+    fam = "gdn_" if gdn else "sane_" if sane else ""
+    return {"workload": fam + f"step_bf16_b{B}_h{H}_256steps{tag}",
             "steps": steps,
             "us_per_step": 1e3 * ms,
             "algorithmic_bytes_per_step": nbytes, "GB/s": gbs, "peak": hbm_peak,
             "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
             "tokens/s": B / (ms / 1e3), "gpu_launches": steps,
-            "traffic": profiled_traffic(("gdn_" if gdn else "") + f"step_b{B}_h{H}{tag}")}
+            "traffic": profiled_traffic(fam + f"step_b{B}_h{H}{tag}")}
 
 
 if __name__ == "__main__":

@@ -138,11 +138,16 @@ __device__ __forceinline__ uint32_t swe(uint32_t row, uint32_t col) {
 }
 
 // Float index of element (row t, column s) of diagonal 16x16 block bb of A_ab, kept in
-// fp32 and stored transposed (s-major, rows 20 floats apart; blocks 336 floats apart,
-// so the two blocks one warp writes and reads together sit 16 banks apart).
+// fp32 and stored transposed (s-major rows of 16; blocks 272 floats apart, so the two
+// blocks one warp writes and reads together sit 16 banks apart).  They and the fp16
+// inverses T_bb live in the S0 tile, which nothing else uses between the previous
+// chunk's output store and this chunk's epilogue 3.
 __device__ __forceinline__ int dtidx(int bb, int s, int t) {
-    return bb * 336 + s * 20 + t;
+    return bb * 272 + s * 16 + t;
 }
+constexpr uint32_t kDiagBytes = 4 * 272 * 4;         // the four fp32 diagonal blocks
+constexpr uint32_t OFF_TB = OFF_S0 + kDiagBytes;     // T_bb: fp16 16x16, 48-byte rows
+static_assert(OFF_TB + 4 * 768 <= OFF_S0 + kTile, "diagonal blocks and T_bb fit the S0 tile");
 
 // Position of channel c in a 64-float per-channel row (prologue scratch, e^{g_L},
 // Khat rows): the two 16-byte halves of each 32-byte group swap places in the upper
@@ -262,6 +267,7 @@ __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int
 struct Ctx {
     uint8_t* smem;
     uint32_t sbase, tmem, bar_tma, bar_mma, mma_phase;
+    uint32_t bar_g2, g2_phase;  // the Gram's second commit group (see the Gram issue)
     int tid, warp, lane, wq, wh, m_row;
     bool state_thread;
     long long row0;  // token row of the sequence start in the [B*T] token space (mask)
@@ -544,10 +550,17 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             tc_fence_before();
             __syncthreads();
 
-            // Gram: D1 = [r~; a~] [k~; b~]^T  (128 x 128 x 64) on the tensor cores.
+            // Gram: D1 = [r~; a~] [k~; b~]^T  (128 x 128 x 64) on the tensor cores, in two
+            // commit groups: first the b~ columns (A_rb, A_ab), so that the warps holding
+            // A_ab start on its diagonal inverses while the k~ columns and A_rb^T run.
             if (tid == 0) {
                 tc_fence_after();
-                constexpr uint32_t id = idesc_bf16(128, 128, false, false);
+                constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_D1 + 64, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
+                              smem_desc(sbase + L.B + 32 * kk, 16, 1024), id, kk > 0);
+                umma_commit(bar_mma);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem + TM_D1, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
@@ -559,7 +572,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.B + 32 * kk, 16, 1024),
                               smem_desc(sbase + L.R + 32 * kk, 16, 1024), id2, kk > 0);
-                umma_commit(bar_mma);
+                umma_commit(cx.bar_g2);
             }
             // While it runs: Abar = a~ e^{g_L} (fp16) and Rbar = r~ e^{g_L} (tiles the Gram
             // does not read, first read after epilogue 1's barrier).
@@ -580,51 +593,111 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             }
         }
 
-        // ---- 4. Gram wait ------------------------------------------------------------------
-        wait_or_abort(bar_mma, mma_phase, cx.timed_out);
-        mma_phase ^= 1;
+        // ---- 4. Gram waits: the warps holding A_ab need only the first group ------------
+        const bool ab_warp = wq >= 2 && wh == 1;
+        wait_or_abort(ab_warp ? bar_mma : cx.bar_g2, ab_warp ? mma_phase : cx.g2_phase,
+                      cx.timed_out);
         tc_fence_after();
 
-        // ---- 5. epilogue 1: masked A_rk, A_rb^T, A_ak (bf16) and A_ab (fp32), each row-wise;
-        //         the second 32 columns load from tensor memory while the first are stored.
+        // ---- 5. epilogue 1: masked A_rk (bf16), A_rb^T, A_ak (fp16) and A_ab, each
+        //         row-wise; the second 32 columns load from tensor memory while the first
+        //         are stored.  A_ab: its diagonal 16x16 blocks (fp32) are inverted at once
+        //         by the two warps holding them, the blocks left of them (fp16) are stored
+        //         over r~ once the second group has read it.
         {
             float v[64];
-            // Warps 4 and 5 read A_rb^T (lanes 0..63 of D1b); the others read D1.
-            const uint32_t ta = tmem + ((uint32_t)(32 * wq) << 16) +
-                                ((wq < 2 && wh == 1) ? TM_D1B : TM_D1 + 64 * wh);
-            auto load32 = [&](int h) {
+            if (ab_warp) {
+                const int t = m_row - 64, bt = t >> 4;  // row of a~, its 16-row block
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                for (int i = 0; i < 4; ++i) {
                     float tmp[16];
-                    tmem_ld16(ta + 32 * h + 16 * i, tmp);
+                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1 + 64 + 16 * i, tmp);
 #pragma unroll
-                    for (int j2 = 0; j2 < 16; ++j2) v[32 * h + 16 * i + j2] = tmp[j2];
+                    for (int j2 = 0; j2 < 16; ++j2) v[16 * i + j2] = tmp[j2];
                 }
-            };
-            auto emit = [&](int h) {  // columns [32h, 32h + 32)
-                if (wq < 2) {
-                    const int t = m_row;  // row of r~
-                    if (wh == 0) {  // A_rk[t][s] = v[s], kept for s <= t -> row t
+                tmem_ld_wait();
+                float* dg = reinterpret_cast<float*>(smem + OFF_S0);
 #pragma unroll
-                        for (int c = 4 * h; c < 4 * h + 4; ++c) {
-                            float x[8];
+                for (int b2 = 0; b2 < 4; ++b2) {
+                    if (bt == b2) {  // the diagonal block, transposed, strictly lower
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
-                            *reinterpret_cast<uint4*>(smem + L.ARK + sw(t, c)) = pack8(x);
-                        }
-                    } else {  // row s = m_row of A_rb^T: A_rb[t][s] = v[t], kept for s <= t
-                        const int s_ = m_row;
+                        for (int s2 = 0; s2 < 16; ++s2)
+                            dg[dtidx(b2, s2, t & 15)] = (16 * b2 + s2 < t) ? v[16 * b2 + s2] : 0.f;
+                    }
+                }
+                // T_bb = (I - N_bb)^-1 with N_bb strictly lower, for this warp's two blocks:
+                // lane (block, column c) solves (I - N) x = e_c column-wise; once x[s] is
+                // final it is added into every later x[t], so the dependent chain is one
+                // FMA per row.  T_bb goes out as fp16.
+                __syncwarp();
+                {
+                    const int bb = 2 * (wq - 2) + (lane >> 4), c = lane & 15;
+                    const float* nt = dg + dtidx(bb, 0, 0);
+                    float x[16];
 #pragma unroll
-                        for (int c = 4 * h; c < 4 * h + 4; ++c) {
-                            float x[8];
+                    for (int t2 = 0; t2 < 16; ++t2) x[t2] = (t2 == c) ? 1.f : 0.f;
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] = (s_ <= 8 * c + e) ? v[8 * c + e] : 0.f;
-                            *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8h(x);
+                    for (int s2 = 0; s2 < 15; ++s2) {
+                        const float xs = x[s2];
+#pragma unroll
+                        for (int t4 = ((s2 + 1) >> 2) << 2; t4 < 16; t4 += 4) {
+                            const float4 n4 = *reinterpret_cast<const float4*>(nt + s2 * 16 + t4);
+                            const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                if (t4 + e > s2) x[t4 + e] = fmaf(nv[e], xs, x[t4 + e]);
                         }
                     }
-                } else {
-                    const int t = m_row - 64;  // row of a~
-                    if (wh == 0) {  // A_ak[t][s] = v[s], kept for s < t -> row t
+                    uint8_t* Tb = smem + OFF_TB;  // fp16 16x16 blocks with 48-byte rows
+#pragma unroll
+                    for (int t2 = 0; t2 < 16; t2 += 2) {  // column c: rows t2 and t2 + 1
+                        const uint32_t hp = pack2h(x[t2], x[t2 + 1]);
+                        *reinterpret_cast<uint16_t*>(Tb + bb * 768 + t2 * 48 + 2 * c) = (uint16_t)(hp & 0xFFFFu);
+                        *reinterpret_cast<uint16_t*>(Tb + bb * 768 + (t2 + 1) * 48 + 2 * c) = (uint16_t)(hp >> 16);
+                    }
+                }
+                wait_or_abort(cx.bar_g2, cx.g2_phase, cx.timed_out);  // r~ has been read
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 8; ++c)  // A_ab[t][s], the blocks left of the diagonal
+                    if (c < 2 * bt)
+                        *reinterpret_cast<uint4*>(smem + L.R + sw(t, c)) = pack8h(v + 8 * c);
+            } else {
+                // Warps 4 and 5 read A_rb^T (lanes 0..63 of D1b); the others read D1.
+                const uint32_t ta = tmem + ((uint32_t)(32 * wq) << 16) +
+                                    ((wq < 2 && wh == 1) ? TM_D1B : TM_D1 + 64 * wh);
+                auto load32 = [&](int h) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        float tmp[16];
+                        tmem_ld16(ta + 32 * h + 16 * i, tmp);
+#pragma unroll
+                        for (int j2 = 0; j2 < 16; ++j2) v[32 * h + 16 * i + j2] = tmp[j2];
+                    }
+                };
+                auto emit = [&](int h) {  // columns [32h, 32h + 32)
+                    if (wq < 2) {
+                        const int t = m_row;  // row of r~
+                        if (wh == 0) {  // A_rk[t][s] = v[s], kept for s <= t -> row t
+#pragma unroll
+                            for (int c = 4 * h; c < 4 * h + 4; ++c) {
+                                float x[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
+                                *reinterpret_cast<uint4*>(smem + L.ARK + sw(t, c)) = pack8(x);
+                            }
+                        } else {  // row s = m_row of A_rb^T: A_rb[t][s] = v[t], kept for s <= t
+                            const int s_ = m_row;
+#pragma unroll
+                            for (int c = 4 * h; c < 4 * h + 4; ++c) {
+                                float x[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) x[e] = (s_ <= 8 * c + e) ? v[8 * c + e] : 0.f;
+                                *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8h(x);
+                            }
+                        }
+                    } else {  // A_ak[t][s] = v[s], kept for s < t -> row t
+                        const int t = m_row - 64;  // row of a~
 #pragma unroll
                         for (int c = 4 * h; c < 4 * h + 4; ++c) {
                             float x[8];
@@ -632,64 +705,17 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                             for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
                             *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8h(x);
                         }
-                    } else {  // A_ab[t][s], s < t: the blocks left of row t's diagonal block
-                        // (all kept) as fp16 for the T_ii A_im products, the diagonal block
-                        // (masked) in fp32 for the T_ii substitution.
-                        const int bt = t >> 4;
-#pragma unroll
-                        for (int c = 4 * h; c < 4 * h + 4; ++c)
-                            if (c < 2 * bt)
-                                *reinterpret_cast<uint4*>(smem + L.R + sw(t, c)) = pack8h(v + 8 * c);
-                        float* dg = reinterpret_cast<float*>(smem + L.A);
-#pragma unroll
-                        for (int b2 = 2 * h; b2 < 2 * h + 2; ++b2) {
-                            if (bt == b2) {  // the diagonal block, transposed
-#pragma unroll
-                                for (int s2 = 0; s2 < 16; ++s2)
-                                    dg[dtidx(b2, s2, t & 15)] = (16 * b2 + s2 < t) ? v[16 * b2 + s2] : 0.f;
-                            }
-                        }
                     }
-                }
-            };
-            load32(0);
-            tmem_ld_wait();
-            load32(1);
-            emit(0);
-            tmem_ld_wait();
-            emit(1);
-            if (wq >= 2 && wh == 1) {
-                // The warps holding A_ab's rows invert their own two diagonal blocks,
-                // T_bb = (I - N_bb)^-1 with N_bb strictly lower, while the other warps
-                // finish this epilogue.  Lane (block, column c) solves (I - N) x = e_c
-                // column-wise: once x[s] is final it is added into every later x[t], so
-                // the dependent chain is one FMA per row.  T_bb goes out as fp16.
-                __syncwarp();
-                const int bb = 2 * (wq - 2) + (lane >> 4), c = lane & 15;
-                const float* nt = reinterpret_cast<const float*>(smem + L.A) + dtidx(bb, 0, 0);
-                float x[16];
-#pragma unroll
-                for (int t = 0; t < 16; ++t) x[t] = (t == c) ? 1.f : 0.f;
-#pragma unroll
-                for (int s2 = 0; s2 < 15; ++s2) {
-                    const float xs = x[s2];
-#pragma unroll
-                    for (int t4 = ((s2 + 1) >> 2) << 2; t4 < 16; t4 += 4) {
-                        const float4 n4 = *reinterpret_cast<const float4*>(nt + s2 * 20 + t4);
-                        const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (t4 + e > s2) x[t4 + e] = fmaf(nv[e], xs, x[t4 + e]);
-                    }
-                }
-                uint8_t* Tb = smem + L.K;  // fp16 16x16 blocks with 48-byte rows
-#pragma unroll
-                for (int t = 0; t < 16; t += 2) {  // column c: rows t and t + 1
-                    const uint32_t hp = pack2h(x[t], x[t + 1]);
-                    *reinterpret_cast<uint16_t*>(Tb + bb * 768 + t * 48 + 2 * c) = (uint16_t)(hp & 0xFFFFu);
-                    *reinterpret_cast<uint16_t*>(Tb + bb * 768 + (t + 1) * 48 + 2 * c) = (uint16_t)(hp >> 16);
-                }
+                };
+                load32(0);
+                tmem_ld_wait();
+                load32(1);
+                emit(0);
+                tmem_ld_wait();
+                emit(1);
             }
+            mma_phase ^= 1;
+            cx.g2_phase ^= 1;
             fence_proxy_async();
             tc_fence_before();
             if (__syncthreads_or(cx.timed_out)) return false;
@@ -705,10 +731,10 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
         //         place over the right-hand side (fp16), where MMA-3 reads it as its
         //         MN-major B operand. ------------------------------------------------
         {
-            // fp16 16x16 blocks with rows of 48 bytes: T_ii (4, from epilogue 1), then
-            // T_ii A_im (6).
-            uint8_t* Tb = smem + L.K;
-            uint8_t* Tab = Tb + 4 * 768;
+            // fp16 16x16 blocks with rows of 48 bytes: T_ii (4, from epilogue 1) and
+            // T_ii A_im (6, in the dead k~ tile).
+            uint8_t* Tb = smem + OFF_TB;
+            uint8_t* Tab = smem + L.K;
             const int g = lane >> 2, q = lane & 3;
             uint8_t* xt = smem + (warp < 4 ? L.ABAR : L.AAK);  // tile of this warp's columns
             const int nb = 2 * (warp & 3);                     // first 16-byte chunk of them
@@ -1021,6 +1047,8 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     cx.sbase = sbase;
     cx.bar_tma = sbase + OFF_MISC;
     cx.bar_mma = sbase + OFF_MISC + 8;
+    cx.bar_g2 = sbase + OFF_MISC + 32;
+    cx.g2_phase = 0;
     cx.mma_phase = 0;
     cx.tid = tid;
     cx.warp = warp;
@@ -1071,6 +1099,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     if (tid == 0) {
         mbar_init(cx.bar_tma, 1);
         mbar_init(cx.bar_mma, 1);
+        mbar_init(cx.bar_g2, 1);
         mbar_init(cx.bar_never, 1);  // nothing ever arrives (the timeout test hook)
         fence_mbar_init();
     }
@@ -1131,6 +1160,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         if (tid == 0) {
             (void)mbar_wait(cx.bar_tma, cx.tma_par_last);
             (void)mbar_wait(cx.bar_mma, cx.mma_phase ^ 1u);
+            (void)mbar_wait(cx.bar_g2, cx.g2_phase ^ 1u);
         }
     } else if (cx.state_thread && sT) {
         float sv[32];

@@ -26,7 +26,7 @@ def run(args, env=None):
     return [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
 
 
-@pytest.mark.parametrize("family", ["wkv7", "gdn"])
+@pytest.mark.parametrize("family", ["wkv7", "gdn", "sane"])
 def test_reference_arm_line(family):
     lines = run(["--impl", "reference", "--steps", "1", "--warmup", "1", "--family", family])
     assert len(lines) == 1
@@ -39,7 +39,8 @@ def test_reference_arm_line(family):
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
-    assert d["metric"] == (bench.GDN_METRIC if family == "gdn" else bench.METRIC)
+    assert d["metric"] == {"gdn": bench.GDN_METRIC, "sane": bench.SANE_METRIC}.get(family,
+                                                                                  bench.METRIC)
     assert d["config"]["workload"].endswith("fwd_bf16_b8_t4096_h64")
 
 
