@@ -10,22 +10,25 @@
 //   A_rk[t][s] = r~_t.k~_s (s<=t), A_rb = r~.b~ (s<=t), A_ak = a~.k~ (s<t), A_ab = a~.b~ (s<t)
 //   T = (I - A_ab)^-1 (the UT / WY representation of the chunk's rank-1 products)
 //   Abar = a e^{g_{t-1}} = a~ e^{g_L}, Rbar = r e^{g_t} = r~ e^{g_L},
-//   Bhat = b e^{g_L - g_t} = b~, Khat = k e^{g_L - g_t} = k~ (kept in fp32)
-//   W = T Abar, Z = T A_ak              (so the read vectors are U = W S0 + Z V)
-//   S_L = diag(e^{g_L}) S0 + (Bhat^T W) S0 + (Khat^T + Bhat^T Z) V
-//   O   = (Rbar + A_rb W) S0 + (A_rk + A_rb Z) V
-// Only the last product depends on S0.  One chunk costs three tcgen05 MMA groups
-// (the Gram matrix, the Bhat/A_rb products with [W | Z], and the final product
-// with [S0; V]) with fp32 accumulators in tensor memory.  [W | Z] = T [Abar | A_ak]
+//   Bhat = b e^{g_L - g_t} = b~, Khat = k e^{g_L - g_t} = k~
+//   W = T Abar, Z = T A_ak,  U = W S0 + Z V   (U: the chunk's read vectors u_t)
+//   S_L = diag(e^{g_L}) S0 + Bhat^T U + Khat^T V
+//   O   = Rbar S0 + A_rb U + A_rk V
+// Only U and what follows depend on S0.  One chunk costs three rounds of tcgen05
+// MMAs with fp32 accumulators in tensor memory: the Gram matrices (two commit
+// groups), MMA-U (U = [W | Z] [S0; V], M = 64, K = 128), and the final products (the
+// state accumulating onto itself scaled by e^{g_L}, and O).  [W | Z] = T [Abar | A_ak]
 // comes from a block forward substitution on warp-level MMAs (each warp owns 16 of
 // its 128 columns), after the 16x16 diagonal blocks of T by fp32 forward
 // substitution.  CUDA cores do the prefix sums and exps and the tensor-memory ->
-// shared-memory epilogues that re-layout each result as the next product's operand.
+// shared-memory epilogues that re-layout each result as the next product's operand;
+// the M = 64 accumulators are read 16 lanes x 32 columns at a time in the warp-MMA
+// fragment layout (all 32 threads busy) and written back with stmatrix.
 // Precision: the Gram operands need bf16's exponent range (E_t spans e^{+-40}).  Every
-// later operand (the substitution, MMA-3, the final product, the fp16 copy of S0 and
-// V) stays near 1 in magnitude and is fp16, with three more significant bits than
+// later operand (the substitution, MMA-U, the final products, the fp16 copies of S0,
+// V and U) stays near 1 in magnitude and is fp16, with three more significant bits than
 // bf16; that keeps the fp32 final state within 1e-3 of the fp64 recurrence (measured
-// over every unit of the B=8, T=4096, H=64 workload: 5.2e-4 of max |S|).
+// over every unit of the B=8, T=4096, H=64 workload: 4.8e-4 of max |S|).
 //
 // A masked or out-of-range token is folded into the loads as w = 0 and zero a, k, b
 // scales: its transition is then the identity and it writes nothing, and its output
@@ -57,74 +60,50 @@ constexpr int kThreads = 256;
 constexpr int kStoreTid = 64;  // issues the output tile stores (an output warp's lane 0)
 // Shared-memory map.  Fourteen 8 KB tiles (64 rows x 128 B, 1024-aligned, 128B
 // swizzle) plus a small control block.  Consecutive chunks alternate between two
-// layouts of the same tiles, so that the next chunk's six input tiles can be
-// loaded by TMA into tiles this chunk no longer needs while its final MMA runs.
+// layouts of the same tiles: the next chunk's six input tiles are exactly the tiles
+// this chunk no longer needs once its MMA-U has read W and Z, so their TMA loads
+// overlap this chunk's last epilogue and final products.
 constexpr uint32_t kTile = 8192;
-constexpr uint32_t OFF_S0 = 11 * kTile;    // S0 bf16 [k][v] (final MMA B, MN-major), both layouts
-constexpr uint32_t OFF_MISC = 14 * kTile;  // mbarriers, TMEM address, abort flag
+constexpr uint32_t OFF_S0 = 12 * kTile;    // S0 fp16 [k][v] (MMA-U and O's B operand), then
+                                           // the output staging; both layouts
+constexpr uint32_t OFF_MISC = 14 * kTile;  // mbarriers, TMEM address
 constexpr uint32_t OFF_GAMMA = OFF_MISC + 64;  // e^{g_L}, channel c at cswz(c) (64 fp32)
 constexpr uint32_t kSmemBytes = OFF_GAMMA + 256;
 
-template <int P>
-struct Lay;
-// Even chunks.
-template <>
-struct Lay<0> {
-    static constexpr uint32_t R = 0 * kTile;      // raw r -> r~   (Gram A rows 0..63)
-    static constexpr uint32_t A = 1 * kTile;      // raw a -> a~   (Gram A rows 64..127)
-    static constexpr uint32_t K = 2 * kTile;      // raw k -> k~   (Gram B rows 0..63)
-    static constexpr uint32_t B = 3 * kTile;      // raw b -> b~   (Gram B rows 64..127)
-    static constexpr uint32_t W = 4 * kTile;      // raw w -> Bhat (MMA-3 A, MN-major atom 0)
-    static constexpr uint32_t V = 5 * kTile;      // raw v         (final MMA B, MN-major)
-    static constexpr uint32_t ABAR = 6 * kTile;   // Abar [s][k] -> W [t][k]  (MMA-3 B, MN-major atom 0)
-    static constexpr uint32_t AAK = 7 * kTile;    // A_ak [s][s'] -> Z [t][s'] (MMA-3 B, MN-major atom 1)
-    static constexpr uint32_t ARBT = 8 * kTile;   // A_rb^T [s][t] (MMA-3 A, MN-major atom 1)
-    static constexpr uint32_t ARK = 9 * kTile;    // A_rk [t][s] (epilogue 3); prologue scratch
-    static constexpr uint32_t RBAR = 10 * kTile;  // Rbar [t][k] (epilogue 3)
-    static constexpr uint32_t F0 = 12 * kTile;    // fp32 64x64 (2 tiles): Khat [s][cswz(k)]
-};
-// Odd chunks: the six input tiles land in tiles the even layout no longer needs
-// once its epilogue 3 is done (Bhat, A_rb^T, A_rk, Rbar, Khat), and vice versa.
-template <>
-struct Lay<1> {
-    static constexpr uint32_t R = 12 * kTile;
-    static constexpr uint32_t A = 13 * kTile;
-    static constexpr uint32_t K = 8 * kTile;
-    static constexpr uint32_t B = 9 * kTile;
-    static constexpr uint32_t W = 4 * kTile;
-    static constexpr uint32_t V = 10 * kTile;
-    static constexpr uint32_t ABAR = 6 * kTile;
-    static constexpr uint32_t AAK = 7 * kTile;
-    static constexpr uint32_t ARBT = 5 * kTile;
-    static constexpr uint32_t ARK = 0 * kTile;
-    static constexpr uint32_t RBAR = 1 * kTile;
-    static constexpr uint32_t F0 = 2 * kTile;
-};
-// The two layouts as run-time offsets (one copy of the chunk code keeps the
-// kernel's instruction footprint small).
+// Tile roles of one chunk (byte offsets):
+//   R     raw r -> r~ (B of A_rk^T / A_rb^T) -> A_ab's blocks left of the diagonal
+//   A     raw a -> a~ (A of the Gram) -> U fp16 [t][v] (B of the final products)
+//   K, B  raw k, b -> k~, b~ (B of the Gram, and together [k~; b~] the A of A_rk^T /
+//         A_rb^T); K then holds T_ii A_im during [W|Z]
+//   W     raw w -> Bhat fp16 [s][k] (A of S's U block, MN-major)
+//   V     raw v -> fp16 in place [s][v] (B of the V blocks)
+//   KHAT  Khat fp16 [s][k] (A of S's V block)     RBAR  Rbar fp16 [t][k] (A of O's S0 block)
+//   ARKT  A_rk^T fp16 [s][t], ARBT A_rb^T fp16 [s][t] (A of O's V and U blocks)
+//   ABAR  Abar fp16 [t][k] -> W [t][k];  AAK  A_ak [t][s] -> Z [t][s]  (A of MMA-U)
+//   SP    prologue scratch, then A_ab's fp32 diagonal blocks and T_ii (epilogue 1 -> [W|Z])
 struct LayR {
-    uint32_t R, A, K, B, W, V, ABAR, AAK, ARBT, ARK, RBAR, F0;
+    uint32_t R, A, K, B, W, V, KHAT, ARKT, ARBT, RBAR, ABAR, AAK, SP;
 };
-template <int P>
-__device__ __forceinline__ LayR lay_const() {
-    return LayR{Lay<P>::R,    Lay<P>::A,   Lay<P>::K,    Lay<P>::B,   Lay<P>::W,    Lay<P>::V,
-                Lay<P>::ABAR, Lay<P>::AAK, Lay<P>::ARBT, Lay<P>::ARK, Lay<P>::RBAR, Lay<P>::F0};
-}
+// Even chunks (tiles 0..13, 12 is S0) and odd chunks: each layout's inputs
+// {R, A, K, B, W, V} are the other's {R, K, B, ABAR, AAK, SP}, all dead once that
+// chunk's MMA-U is done; K and B are adjacent in both ([k~; b~] is one 128-row operand).
 __device__ __forceinline__ LayR lay_of(int par) {
-    return par ? lay_const<1>() : lay_const<0>();
+    return par ? LayR{0 * kTile, 13 * kTile, 2 * kTile, 3 * kTile, 10 * kTile, 11 * kTile,
+                      6 * kTile, 7 * kTile,  8 * kTile, 9 * kTile, 1 * kTile,  4 * kTile,
+                      5 * kTile}
+               : LayR{0 * kTile, 1 * kTile,  2 * kTile, 3 * kTile, 4 * kTile,  5 * kTile,
+                      6 * kTile, 7 * kTile,  8 * kTile, 9 * kTile, 10 * kTile, 11 * kTile,
+                      13 * kTile};
 }
-// Aliases inside one chunk (lifetimes do not overlap):
-//   A_ab [t][s]          R: fp16 blocks left of the diagonal; A: fp32 diagonal
-//                        blocks (epilogue 1 -> W|Z substitution)
-//   T_ii, T_ii A_im      K: fp16 16x16 blocks with 48-byte rows (W|Z substitution)
-//   [M'; Rbar + A_rb W]  R (2 tiles)   epilogue 3 -> final MMA A, K block 0 (B: S0)
-//   [P_N; A_rk + A_rb Z] ABAR (2)      epilogue 3 -> final MMA A, K block 1 (B: V)
-// Prologue scratch inside the A_rk tile (free until epilogue 1), in floats.
+// Prologue scratch in the SP tile, in floats.
 constexpr int SCR_TOT = 0, SCR_C = 512, SCR_PRE = 576;  // floats (SCR_PRE: 8 x 64)
-// Tensor-memory columns (fp32 accumulators, 128 lanes).
-constexpr uint32_t TM_D1 = 0;    // Gram, later MMA-3 (128 cols)
-constexpr uint32_t TM_D1B = 128; // A_rb^T = b~ r~^T (64 cols)
-constexpr uint32_t TM_DF = 192;  // [S update; O] (64 cols)
+// Tensor-memory columns.  An M = 64 accumulator holds row m in lane (m % 16) +
+// 32 (m / 16): lanes 0..15 of each 32-lane quadrant; M = 128 uses all 128 lanes.
+constexpr uint32_t TM_D1 = 0;    // [A_ak | A_ab] = a~ [k~; b~]^T, M = 64 (128 cols); then U
+constexpr uint32_t TM_DU = 0;    // U = [W | Z] [S0; V], M = 64 (64 cols)
+constexpr uint32_t TM_D1B = 128; // [A_rk^T; A_rb^T] = [k~; b~] r~^T, M = 128 (64 cols); then O
+constexpr uint32_t TM_DFO = 128; // O, M = 64 (64 cols)
+constexpr uint32_t TM_DFS = 192; // the fp32 state S, M = 64 (64 cols), for the whole sequence
 constexpr uint32_t kTmemCols = 256;
 constexpr float kExpClamp = 80.f;
 
@@ -138,16 +117,16 @@ __device__ __forceinline__ uint32_t swe(uint32_t row, uint32_t col) {
 }
 
 // Float index of element (row t, column s) of diagonal 16x16 block bb of A_ab, kept in
-// fp32 and stored transposed (s-major rows of 16; blocks 272 floats apart, so the two
-// blocks one warp writes and reads together sit 16 banks apart).  They and the fp16
-// inverses T_bb live in the S0 tile, which nothing else uses between the previous
-// chunk's output store and this chunk's epilogue 3.
+// fp32 and stored transposed (s-major rows of 16 floats padded to 20, so that the
+// fragment-layout writes of rows s = 2q + e, q = 0..3, fall in four different 8-bank
+// groups).  They and the fp16 inverses T_bb (48-byte rows) live in the SP tile, free
+// once the prologue is done.
+constexpr int kDgRow = 20;
 __device__ __forceinline__ int dtidx(int bb, int s, int t) {
-    return bb * 272 + s * 16 + t;
+    return bb * 16 * kDgRow + s * kDgRow + t;
 }
-constexpr uint32_t kDiagBytes = 4 * 272 * 4;         // the four fp32 diagonal blocks
-constexpr uint32_t OFF_TB = OFF_S0 + kDiagBytes;     // T_bb: fp16 16x16, 48-byte rows
-static_assert(OFF_TB + 4 * 768 <= OFF_S0 + kTile, "diagonal blocks and T_bb fit the S0 tile");
+constexpr uint32_t kDiagBytes = 4 * 16 * kDgRow * 4;  // the four fp32 diagonal blocks, then T_bb
+static_assert(kDiagBytes + 4 * 768 <= kTile, "diagonal blocks and T_bb fit one tile");
 
 // Position of channel c in a 64-float per-channel row (prologue scratch, e^{g_L},
 // Khat rows): the two 16-byte halves of each 32-byte group swap places in the upper
@@ -243,6 +222,48 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                  : "r"(addr));
 }
 
+// Four 8x8 b16 matrices from warp-MMA fragment registers (lane l: row l / 4, columns
+// 2 (l % 4), +1 of each) to shared memory; lane l gives the address of row l % 8 of
+// matrix l / 8 (16 bytes per row).
+__device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                        uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
+// Half h (columns 16h .. 16h + 15) of a 16-row x 32-column block held in fragment
+// layout (sm100::tmem_ld16x32) to a 128B-swizzled tile: rows row0 .. row0 + 15, 16-byte
+// chunks chunk0 + 2h, +1; each element pair packed by `pk` (fp16 or bf16).  One
+// stmatrix.x4, whose matrices are (chunk 2h, rows +0), (2h, +8), (2h + 1, +0), (2h + 1, +8).
+template <typename Pack>
+__device__ __forceinline__ void frag_half_to_tile(uint32_t tile, int row0, int chunk0, int h,
+                                                  const float (&v)[16], int lane, Pack pk) {
+    const int mi = lane >> 3;  // the matrix this lane addresses
+    const uint32_t addr = tile + sw(row0 + 8 * (mi & 1) + (lane & 7), chunk0 + 2 * h + (mi >> 1));
+    stsm_x4(addr, pk(v[8 * h + 0], v[8 * h + 1]), pk(v[8 * h + 2], v[8 * h + 3]),
+            pk(v[8 * h + 4], v[8 * h + 5]), pk(v[8 * h + 6], v[8 * h + 7]));
+}
+template <typename Pack>
+__device__ __forceinline__ void frag_to_tile(uint32_t tile, int row0, int chunk0, const float (&v)[16],
+                                             int lane, Pack pk) {
+    frag_half_to_tile(tile, row0, chunk0, 0, v, lane, pk);
+    frag_half_to_tile(tile, row0, chunk0, 1, v, lane, pk);
+}
+struct PackH {
+    __device__ __forceinline__ uint32_t operator()(float a, float b) const { return pack2h(a, b); }
+};
+struct PackB {
+    __device__ __forceinline__ uint32_t operator()(float a, float b) const { return pack2(a, b); }
+};
+
+// The 16 rows of an M = 64 accumulator that warp quadrant wq owns (rows 16 wq .. 16 wq + 15,
+// lanes 0..15 of the quadrant), columns col .. col + 31, in fragment layout.
+__device__ __forceinline__ void tmem_frag(uint32_t tmem, int wq, uint32_t col, float (&v)[16]) {
+    sm100::tmem_ld16x32(tmem + ((uint32_t)(32 * wq) << 16) + col, v);
+    sm100::tmem_ld_wait();
+}
+
 // Transpose of an 8x8 b16 matrix held one 32-bit pair per lane (lane l: row l / 4,
 // columns 2 (l % 4), +1), returned in the same layout.
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
@@ -268,8 +289,7 @@ struct Ctx {
     uint8_t* smem;
     uint32_t sbase, tmem, bar_tma, bar_mma, mma_phase;
     uint32_t bar_g2, g2_phase;  // the Gram's second commit group (see the Gram issue)
-    int tid, warp, lane, wq, wh, m_row;
-    bool state_thread;
+    int tid, warp, lane, wq, wh;
     long long row0;  // token row of the sequence start in the [B*T] token space (mask)
     int len;
     const uint8_t* mask;
@@ -330,15 +350,12 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
     uint8_t* smem = cx.smem;
     const uint32_t sbase = cx.sbase, tmem = cx.tmem, bar_mma = cx.bar_mma;
     const int tid = cx.tid, warp = cx.warp, lane = cx.lane, wq = cx.wq, wh = cx.wh;
-    const int m_row = cx.m_row;
-    const bool state_thread = cx.state_thread;
     const long long row0 = cx.row0;
     const uint8_t* mask = cx.mask;
     __nv_bfloat16* o = cx.o;
     float* gamma_s = cx.gamma_s;
     uint32_t& mma_phase = cx.mma_phase;
-    float* scratch = reinterpret_cast<float*>(smem + L.ARK);  // prologue only
-    float* F0 = reinterpret_cast<float*>(smem + L.F0);
+    float* scratch = reinterpret_cast<float*>(smem + L.SP);  // prologue only
     const int nv = min(64, cx.len - c0);
     // The previous chunk's output store has read the S0 tile before this chunk's
     // epilogue 3 writes it (ordered by the barriers in between).
@@ -377,7 +394,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             const int h0 = cswz(8 * j), h1 = cswz(8 * j + 4);  // this thread's channel halves
             float rts[2][8], ats[2][8], ec[8];  // fp32 r~ and a~, kept for Rbar and Abar; e^{g_L}
             // The token's operands to shared memory: r~, a~, k~ (bf16), b~ (bf16 and fp16
-            // as Bhat), Khat (fp32).
+            // as Bhat), Khat (fp16).
             auto put = [&](int it, const float* kt, const float* btl) {
                 const uint32_t off = it ? offb : offa;
                 *reinterpret_cast<uint4*>(smem + L.R + off) = pack8(rts[it]);
@@ -386,9 +403,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                 *reinterpret_cast<uint4*>(smem + L.K + off) = kq;
                 *reinterpret_cast<uint4*>(smem + L.B + off) = pack8(btl);
                 *reinterpret_cast<uint4*>(smem + L.W + off) = pack8h(btl);  // Bhat (fp16)
-                float* kh = F0 + (t0 + it) * 64;
-                *reinterpret_cast<float4*>(kh + h0) = make_float4(kt[0], kt[1], kt[2], kt[3]);
-                *reinterpret_cast<float4*>(kh + h1) = make_float4(kt[4], kt[5], kt[6], kt[7]);
+                *reinterpret_cast<uint4*>(smem + L.KHAT + off) = pack8h(kt);  // Khat (fp16)
             };
             if constexpr (kGdn) {
                 // Gated DeltaNet: one log decay per token, so the scan runs on one value per
@@ -550,32 +565,31 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             tc_fence_before();
             __syncthreads();
 
-            // Gram: D1 = [r~; a~] [k~; b~]^T  (128 x 128 x 64) on the tensor cores, in two
-            // commit groups: first the b~ columns (A_rb, A_ab), so that the warps holding
-            // A_ab start on its diagonal inverses while the k~ columns and A_rb^T run.
+            // Gram on the tensor cores, in two commit groups: first A_ab = a~ b~^T (M = 64),
+            // so that the warps holding it start on its diagonal inverses while the second
+            // group runs: A_ak = a~ k~^T (M = 64) and [A_rk^T; A_rb^T] = [k~; b~] r~^T
+            // (M = 128), the transposes the output product takes as MN-major operands.
             if (tid == 0) {
                 tc_fence_after();
-                constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+                constexpr uint32_t id64 = idesc_bf16(64, 64, false, false);
+                constexpr uint32_t id128 = idesc_bf16(128, 64, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + TM_D1 + 64, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
-                              smem_desc(sbase + L.B + 32 * kk, 16, 1024), id, kk > 0);
+                    umma_bf16(tmem + TM_D1 + 64, smem_desc(sbase + L.A + 32 * kk, 16, 1024),
+                              smem_desc(sbase + L.B + 32 * kk, 16, 1024), id64, kk > 0);
                 umma_commit(bar_mma);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + TM_D1, smem_desc(sbase + L.R + 32 * kk, 16, 1024),
-                              smem_desc(sbase + L.K + 32 * kk, 16, 1024), id, kk > 0);
-                // A_rb^T directly: rows s of b~ against r~ (rows 64..127 of this A operand
-                // read the next tile and are never used).
-                constexpr uint32_t id2 = idesc_bf16(128, 64, false, false);
+                    umma_bf16(tmem + TM_D1, smem_desc(sbase + L.A + 32 * kk, 16, 1024),
+                              smem_desc(sbase + L.K + 32 * kk, 16, 1024), id64, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.B + 32 * kk, 16, 1024),
-                              smem_desc(sbase + L.R + 32 * kk, 16, 1024), id2, kk > 0);
+                    umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.K + 32 * kk, 16, 1024),
+                              smem_desc(sbase + L.R + 32 * kk, 16, 1024), id128, kk > 0);
                 umma_commit(cx.bar_g2);
             }
-            // While it runs: Abar = a~ e^{g_L} (fp16) and Rbar = r~ e^{g_L} (tiles the Gram
-            // does not read, first read after epilogue 1's barrier).
+            // While it runs: Abar = a~ e^{g_L} and Rbar = r~ e^{g_L} (fp16), V to fp16 in
+            // place (tiles the Gram does not read).
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const uint32_t off = it ? offb : offa;
@@ -586,52 +600,75 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                     rbar[e] = rts[it][e] * ec[e];
                 }
                 *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8h(abar);
-                *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8(rbar);
-                float vf[8];  // V to fp16 in place (the final MMA's B operand)
+                *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8h(rbar);
+                float vf[8];
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.V + off), vf);
                 *reinterpret_cast<uint4*>(smem + L.V + off) = pack8h(vf);
+            }
+            // And the state this chunk starts from (rows k = 16 wq + lane of the M = 64
+            // accumulator, lanes 0..15): its fp16 copy, the B operand of MMA-U and of O's S0
+            // block, and the state itself scaled by e^{g_L} in tensor memory, where the
+            // final product S_L += Bhat^T U + Khat^T V accumulates onto it.
+            {
+                float sv[16];
+                tmem_frag(tmem + TM_DFS, wq, 32 * wh, sv);
+                frag_to_tile(sbase + OFF_S0, 16 * wq, 4 * wh, sv, lane, PackH{});
+                const float g0 = gamma_s[cswz(16 * wq + (lane >> 2))];
+                const float g1 = gamma_s[cswz(16 * wq + (lane >> 2) + 8)];
+#pragma unroll
+                for (int j2 = 0; j2 < 4; ++j2) {
+                    sv[4 * j2 + 0] *= g0;
+                    sv[4 * j2 + 1] *= g0;
+                    sv[4 * j2 + 2] *= g1;
+                    sv[4 * j2 + 3] *= g1;
+                }
+                sm100::tmem_st16x32(tmem + TM_DFS + ((uint32_t)(32 * wq) << 16) + 32 * wh, sv);
+                tmem_st_wait();
             }
         }
 
         // ---- 4. Gram waits: the warps holding A_ab need only the first group ------------
-        const bool ab_warp = wq >= 2 && wh == 1;
+        const bool ab_warp = wh == 1;
         wait_or_abort(ab_warp ? bar_mma : cx.bar_g2, ab_warp ? mma_phase : cx.g2_phase,
                       cx.timed_out);
         tc_fence_after();
 
-        // ---- 5. epilogue 1: masked A_rk (bf16), A_rb^T, A_ak (fp16) and A_ab, each
-        //         row-wise; the second 32 columns load from tensor memory while the first
-        //         are stored.  A_ab: its diagonal 16x16 blocks (fp32) are inverted at once
-        //         by the two warps holding them, the blocks left of them (fp16) are stored
-        //         over r~ once the second group has read it.
+        // ---- 5. epilogue 1.  M = 64 rows t = 16 wq + lane (lanes 0..15) of [A_ak | A_ab]:
+        //         warps 4..7 hold A_ab's block row wq, write its diagonal block (fp32,
+        //         transposed) and invert it at once, then, once the second group has read
+        //         r~, store the blocks left of it (fp16) over r~; warps 0..3 store masked
+        //         A_ak and all of [A_rk^T; A_rb^T] (M = 128, rows s = 32 wq + lane),
+        //         masked s <= t, as fp16 [s][t]. ------------------------------------------
         {
-            float v[64];
+            const int g = lane >> 2, q = lane & 3;
+            const int t0 = 16 * wq + g;  // fragment rows t0 and t0 + 8 of a~
             if (ab_warp) {
-                const int t = m_row - 64, bt = t >> 4;  // row of a~, its 16-row block
+                float v[2][16];  // A_ab columns 0..31, 32..63
+                tmem_frag(tmem + TM_D1 + 64, wq, 0, v[0]);
+                tmem_frag(tmem + TM_D1 + 64, wq, 32, v[1]);
+                float* dg = reinterpret_cast<float*>(smem + L.SP);
+                {   // the diagonal block (columns 16 wq ..), transposed, strictly lower
+                    const bool hi = wq >= 2, odd = wq & 1;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float tmp[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1 + 64 + 16 * i, tmp);
+                    for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-                    for (int j2 = 0; j2 < 16; ++j2) v[16 * i + j2] = tmp[j2];
+                        for (int e = 0; e < 2; ++e) {
+                            const int s2 = 8 * jj + 2 * q + e;  // column within the block
+                            const int i0 = 4 * jj + e, i1 = 4 * (2 + jj) + e;
+                            const float lo0 = odd ? v[0][i1] : v[0][i0], hi0 = odd ? v[1][i1] : v[1][i0];
+                            const float lo1 = odd ? v[0][i1 + 2] : v[0][i0 + 2];
+                            const float hi1 = odd ? v[1][i1 + 2] : v[1][i0 + 2];
+                            dg[dtidx(wq, s2, g)] = (s2 < g) ? (hi ? hi0 : lo0) : 0.f;
+                            dg[dtidx(wq, s2, g + 8)] = (s2 < g + 8) ? (hi ? hi1 : lo1) : 0.f;
+                        }
                 }
-                tmem_ld_wait();
-                float* dg = reinterpret_cast<float*>(smem + OFF_S0);
-#pragma unroll
-                for (int b2 = 0; b2 < 4; ++b2) {
-                    if (bt == b2) {  // the diagonal block, transposed, strictly lower
-#pragma unroll
-                        for (int s2 = 0; s2 < 16; ++s2)
-                            dg[dtidx(b2, s2, t & 15)] = (16 * b2 + s2 < t) ? v[16 * b2 + s2] : 0.f;
-                    }
-                }
-                // T_bb = (I - N_bb)^-1 with N_bb strictly lower, for this warp's two blocks:
-                // lane (block, column c) solves (I - N) x = e_c column-wise; once x[s] is
-                // final it is added into every later x[t], so the dependent chain is one
-                // FMA per row.  T_bb goes out as fp16.
+                // T_bb = (I - N_bb)^-1 with N_bb strictly lower, for this warp's block:
+                // lane c < 16 solves (I - N) x = e_c column-wise; once x[s] is final it is
+                // added into every later x[t], so the dependent chain is one FMA per row.
+                // T_bb goes out as fp16.
                 __syncwarp();
-                {
-                    const int bb = 2 * (wq - 2) + (lane >> 4), c = lane & 15;
+                if (lane < 16) {
+                    const int bb = wq, c = lane;
                     const float* nt = dg + dtidx(bb, 0, 0);
                     float x[16];
 #pragma unroll
@@ -641,14 +678,14 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                         const float xs = x[s2];
 #pragma unroll
                         for (int t4 = ((s2 + 1) >> 2) << 2; t4 < 16; t4 += 4) {
-                            const float4 n4 = *reinterpret_cast<const float4*>(nt + s2 * 16 + t4);
+                            const float4 n4 = *reinterpret_cast<const float4*>(nt + s2 * kDgRow + t4);
                             const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
                                 if (t4 + e > s2) x[t4 + e] = fmaf(nv[e], xs, x[t4 + e]);
                         }
                     }
-                    uint8_t* Tb = smem + OFF_TB;  // fp16 16x16 blocks with 48-byte rows
+                    uint8_t* Tb = smem + L.SP + kDiagBytes;  // fp16 16x16 blocks, 48-byte rows
 #pragma unroll
                     for (int t2 = 0; t2 < 16; t2 += 2) {  // column c: rows t2 and t2 + 1
                         const uint32_t hp = pack2h(x[t2], x[t2 + 1]);
@@ -658,61 +695,48 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                 }
                 wait_or_abort(cx.bar_g2, cx.g2_phase, cx.timed_out);  // r~ has been read
                 tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < 8; ++c)  // A_ab[t][s], the blocks left of the diagonal
-                    if (c < 2 * bt)
-                        *reinterpret_cast<uint4*>(smem + L.R + sw(t, c)) = pack8h(v + 8 * c);
+                // A_ab[t][s] over r~: the 16-column blocks left of the diagonal
+                if (wq > 0) frag_half_to_tile(sbase + L.R, 16 * wq, 0, 0, v[0], lane, PackH{});
+                if (wq > 1) frag_half_to_tile(sbase + L.R, 16 * wq, 0, 1, v[0], lane, PackH{});
+                if (wq > 2) frag_half_to_tile(sbase + L.R, 16 * wq, 4, 0, v[1], lane, PackH{});
             } else {
-                // Warps 4 and 5 read A_rb^T (lanes 0..63 of D1b); the others read D1.
-                const uint32_t ta = tmem + ((uint32_t)(32 * wq) << 16) +
-                                    ((wq < 2 && wh == 1) ? TM_D1B : TM_D1 + 64 * wh);
-                auto load32 = [&](int h) {
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {  // A_ak[t][s], kept for s < t
+                    float v[16];
+                    tmem_frag(tmem + TM_D1, wq, 32 * h2, v);
+#pragma unroll
+                    for (int j2 = 0; j2 < 4; ++j2)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int s2 = 32 * h2 + 8 * j2 + 2 * q + e;
+                            if (s2 >= t0) v[4 * j2 + e] = 0.f;
+                            if (s2 >= t0 + 8) v[4 * j2 + 2 + e] = 0.f;
+                        }
+                    frag_to_tile(sbase + L.AAK, 16 * wq, 4 * h2, v, lane, PackH{});
+                }
+                // row s of A_rk^T (wq 0, 1) or A_rb^T (wq 2, 3): A_x[t][s] = v[t], kept s <= t
+                const int s_ = 32 * (wq & 1) + lane;
+                const uint32_t dst = wq < 2 ? L.ARKT : L.ARBT;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    float v[32];
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
                         float tmp[16];
-                        tmem_ld16(ta + 32 * h + 16 * i, tmp);
+                        tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1B + 32 * h2 + 16 * i, tmp);
 #pragma unroll
-                        for (int j2 = 0; j2 < 16; ++j2) v[32 * h + 16 * i + j2] = tmp[j2];
+                        for (int j2 = 0; j2 < 16; ++j2) v[16 * i + j2] = tmp[j2];
                     }
-                };
-                auto emit = [&](int h) {  // columns [32h, 32h + 32)
-                    if (wq < 2) {
-                        const int t = m_row;  // row of r~
-                        if (wh == 0) {  // A_rk[t][s] = v[s], kept for s <= t -> row t
+                    tmem_ld_wait();
 #pragma unroll
-                            for (int c = 4 * h; c < 4 * h + 4; ++c) {
-                                float x[8];
+                    for (int c = 0; c < 4; ++c) {
+                        float x[8];
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= t) ? v[8 * c + e] : 0.f;
-                                *reinterpret_cast<uint4*>(smem + L.ARK + sw(t, c)) = pack8(x);
-                            }
-                        } else {  // row s = m_row of A_rb^T: A_rb[t][s] = v[t], kept for s <= t
-                            const int s_ = m_row;
-#pragma unroll
-                            for (int c = 4 * h; c < 4 * h + 4; ++c) {
-                                float x[8];
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) x[e] = (s_ <= 8 * c + e) ? v[8 * c + e] : 0.f;
-                                *reinterpret_cast<uint4*>(smem + L.ARBT + sw(s_, c)) = pack8h(x);
-                            }
-                        }
-                    } else {  // A_ak[t][s] = v[s], kept for s < t -> row t
-                        const int t = m_row - 64;  // row of a~
-#pragma unroll
-                        for (int c = 4 * h; c < 4 * h + 4; ++c) {
-                            float x[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < t) ? v[8 * c + e] : 0.f;
-                            *reinterpret_cast<uint4*>(smem + L.AAK + sw(t, c)) = pack8h(x);
-                        }
+                        for (int e = 0; e < 8; ++e)
+                            x[e] = (s_ <= 32 * h2 + 8 * c + e) ? v[8 * c + e] : 0.f;
+                        *reinterpret_cast<uint4*>(smem + dst + sw(s_, 4 * h2 + c)) = pack8h(x);
                     }
-                };
-                load32(0);
-                tmem_ld_wait();
-                load32(1);
-                emit(0);
-                tmem_ld_wait();
-                emit(1);
+                }
             }
             mma_phase ^= 1;
             cx.g2_phase ^= 1;
@@ -733,7 +757,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
         {
             // fp16 16x16 blocks with rows of 48 bytes: T_ii (4, from epilogue 1) and
             // T_ii A_im (6, in the dead k~ tile).
-            uint8_t* Tb = smem + OFF_TB;
+            uint8_t* Tb = smem + L.SP + kDiagBytes;
             uint8_t* Tab = smem + L.K;
             const int g = lane >> 2, q = lane & 3;
             uint8_t* xt = smem + (warp < 4 ? L.ABAR : L.AAK);  // tile of this warp's columns
@@ -817,171 +841,109 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             __syncthreads();
         }
 
-        // ---- 7. MMA-3: [Bhat^T; A_rb] [W | Z]  (128 x 128 x 64) ----------------------------
+        // ---- 7. MMA-U: U = [W | Z] [S0; V], the chunk's read vectors u_t = S_{t-1}^T a_t
+        //         (M = 64, K = 128, fp16). ---------------------------------------------------
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id = idesc_f16(128, 128, true, true);  // fp16 operands
+            constexpr uint32_t idu = idesc_f16(64, 64, false, true);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_D1, smem_desc(sbase + L.W + 2048 * kk, L.ARBT - L.W, 1024),
-                          smem_desc(sbase + L.ABAR + 2048 * kk, L.AAK - L.ABAR, 1024), id, kk > 0);
+                umma_bf16(tmem + TM_DU, smem_desc(sbase + L.ABAR + 32 * kk, 16, 1024),
+                          smem_desc(sbase + OFF_S0 + 2048 * kk, 8192, 1024), idu, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_DU, smem_desc(sbase + L.AAK + 32 * kk, 16, 1024),
+                          smem_desc(sbase + L.V + 2048 * kk, 8192, 1024), idu, 1u);
             umma_commit(bar_mma);
         }
         wait_or_abort(bar_mma, mma_phase, cx.timed_out);
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 8. epilogue 3: assemble the final A operand.  Rows k (lanes 0..63): M'
-        //         and P_N; warps 0/1 take columns 0..31 of both, warps 4/5 columns
-        //         32..63.  Rows t (lanes 64..127): Q (warps 2/3) and P_O (warps 6/7). --
-        {
-            if (wq < 2) {
-                const int k = m_row;
-                float v[64];  // M' = Bhat^T W, then P_N - Khat^T = Bhat^T Z, 32 columns each
-                auto load16 = [&](int i) {
-                    float tmp[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1 + (i >> 1) * 64 + 32 * wh + 16 * (i & 1),
-                              tmp);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
-                };
-                float sv[32];  // this thread's fp32 state row, loaded with M'
-                load16(0);
-                load16(1);
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    float tmp[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_DF + 32 * wh + 16 * i, tmp);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) sv[16 * i + j] = tmp[j];
-                }
-                tmem_ld_wait();
-                load16(2);  // P_N columns load while M' is stored and the state is scaled
-                load16(3);
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + L.R + sw(k, 4 * wh + c)) = pack8h(v + 8 * c);
-                // The final MMA's S0 operand: the fp16 copy of the state this chunk starts from.
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(k, 4 * wh + c)) = pack8h(sv + 8 * c);
-                {  // the final MMA accumulates onto the state row scaled by e^{g_L}
-                    const float gamma = gamma_s[cswz(m_row)];
-#pragma unroll
-                    for (int j2 = 0; j2 < 32; ++j2) sv[j2] *= gamma;
-                    tmem_row_st32(tmem + TM_DF, wq, 32 * wh, sv);
-                }
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {  // P_N = Bhat^T Z + Khat^T
-                    float pn[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) pn[e] = v[32 + 8 * c + e] + F0[(8 * (4 * wh + c) + e) * 64 + cswz(k)];
-                    *reinterpret_cast<uint4*>(smem + L.ABAR + sw(k, 4 * wh + c)) = pack8h(pn);
-                }
-                tmem_st_wait();
-            } else {
-                const int tp = m_row - 64;
-                float v[64];
-                auto load16 = [&](int i) {
-                    float tmp[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + TM_D1 + 64 * wh + 16 * i, tmp);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) v[16 * i + j] = tmp[j];
-                };
-                // Q = A_rb W + Rbar (wh 0) or P_O = A_rb Z + A_rk (wh 1).  The second 32
-                // columns load while the first are stored.
-                const uint32_t src = wh ? L.ARK : L.RBAR, dst = wh ? L.ABAR : L.R;
-                auto emit = [&](int h) {
-#pragma unroll
-                    for (int c = 4 * h; c < 4 * h + 4; ++c) {
-                        float x[8];
-                        unpack8(*reinterpret_cast<const uint4*>(smem + src + sw(tp, c)), x);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] += v[8 * c + e];
-                        *reinterpret_cast<uint4*>(smem + dst + sw(m_row, c)) = pack8h(x);
-                    }
-                };
-                load16(0);
-                load16(1);
-                tmem_ld_wait();
-                load16(2);
-                load16(3);
-                emit(0);
-                tmem_ld_wait();
-                emit(1);
-            }
-            // The final MMA accumulates onto its tensor-memory columns: rows 0..63 hold
-            // the scaled fp32 state (above); rows 64..127 (outputs) were cleared by the
-            // previous chunk's epilogue 4 (or at the start).
-            fence_proxy_async();
-            tc_fence_before();
-            if (__syncthreads_or(cx.timed_out)) return false;
-        }
-
-        // The next chunk's inputs go to the other layout's input tiles, all of which
-        // are dead now; the copy overlaps this chunk's final MMA and epilogue.
+        // W and Z have been read: every tile the next chunk loads into is dead now.
         if (has_next) {
             if (warp == 1) issue_loads<kGdn, kHf>(cx, c0 + 64, par ^ 1);
             cx.tma_par_last = par ^ 1;
         }
 
-        // ---- 9. final MMA: [S upd; O] = A_fin [S0; V]  (128 x 64 x 128, fp16) ------------
+        // ---- 8. epilogue U: U (rows t = 16 wq + lane, lanes 0..15) to fp16 [t][v] over a~,
+        //         the B operand of both final products. -------------------------------------
+        {
+            float v[16];
+            tmem_frag(tmem + TM_DU, wq, 32 * wh, v);
+            frag_to_tile(sbase + L.A, 16 * wq, 4 * wh, v, lane, PackH{});
+            fence_proxy_async();
+            tc_fence_before();
+            if (__syncthreads_or(cx.timed_out)) return false;
+        }
+
+        // ---- 9. the final products (M = 64, fp16):
+        //         S_L += Bhat^T U + Khat^T V   (onto the state scaled by e^{g_L})
+        //         O    = A_rb U + A_rk V + Rbar S0 ------------------------------------------
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id = idesc_f16(128, 64, false, true);
+            constexpr uint32_t idmm = idesc_f16(64, 64, true, true);   // A and B MN-major
+            constexpr uint32_t idkm = idesc_f16(64, 64, false, true);  // A K-major
 #pragma unroll
-            for (int blk = 0; blk < 2; ++blk) {
-                const uint32_t aoff = blk == 0 ? L.R : L.ABAR;
-                const uint32_t boff = blk == 0 ? OFF_S0 : L.V;
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_DFS, smem_desc(sbase + L.W + 2048 * kk, 8192, 1024),
+                          smem_desc(sbase + L.A + 2048 * kk, 8192, 1024), idmm, 1u);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + TM_DF, smem_desc(sbase + aoff + 32 * kk, 16, 1024),
-                              smem_desc(sbase + boff + 2048 * kk, 8192, 1024), id, 1u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_DFS, smem_desc(sbase + L.KHAT + 2048 * kk, 8192, 1024),
+                          smem_desc(sbase + L.V + 2048 * kk, 8192, 1024), idmm, 1u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.ARBT + 2048 * kk, 8192, 1024),
+                          smem_desc(sbase + L.A + 2048 * kk, 8192, 1024), idmm, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.ARKT + 2048 * kk, 8192, 1024),
+                          smem_desc(sbase + L.V + 2048 * kk, 8192, 1024), idmm, 1u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.RBAR + 32 * kk, 16, 1024),
+                          smem_desc(sbase + OFF_S0 + 2048 * kk, 8192, 1024), idkm, 1u);
             umma_commit(bar_mma);
         }
         wait_or_abort(bar_mma, mma_phase, cx.timed_out);
         mma_phase ^= 1;
         tc_fence_after();
 
-        // ---- 10. epilogue 4: the chunk's outputs (rows 64..127 of the final product); the
-        //          new fp32 state stays in tensor memory (its fp16 copy is written by the
-        //          next chunk's epilogue 3) ----------------------------------------------
-        if (!state_thread) {
-            float v[32];
-            tmem_row<2>(tmem + TM_DF, wq, 32 * wh, v);
-            {  // cleared for the next chunk's final MMA, which accumulates onto them
-                float z[32];
-#pragma unroll
-                for (int j2 = 0; j2 < 32; ++j2) z[j2] = 0.f;
-                tmem_row_st32(tmem + TM_DF, wq, 32 * wh, z);
-            }
-            const int t = m_row - 64;
+        // ---- 10. epilogue 4: the chunk's outputs (rows t = 16 wq + lane of O); the new fp32
+        //          state stays in tensor memory. ---------------------------------------------
+        {
+            float v[16];
+            tmem_frag(tmem + TM_DFO, wq, 32 * wh, v);
             if (nv == 64) {
                 // A full chunk: the bf16 rows are staged in the (now dead) S0 tile in the
                 // inputs' swizzled layout and leave as one TMA tile store, so each output
-                // row is written by whole lines instead of 16-byte pieces of 32 rows.
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S0 + sw(t, 4 * wh + c)) = pack8(v + 8 * c);
+                // row is written by whole lines instead of 16-byte pieces of many rows.
+                frag_to_tile(sbase + OFF_S0, 16 * wq, 4 * wh, v, lane, PackB{});
                 fence_proxy_async();
-                asm volatile("bar.sync 1, 128;" ::: "memory");  // the four output warps
+                __syncthreads();
                 if (tid == kStoreTid) {
                     const int cy = kHf ? cx.tma_y + c0 : cx.tma_y;
                     const int cz = kHf ? cx.tma_z : cx.tma_z + c0;
                     tma_store_3d(cx.tm_o, sbase + OFF_S0, 0, cy, cz);
                     bulk_commit();
                 }
-            } else if (t < nv) {  // a partial last chunk: only the sequence's own rows
-                uint4* dst = reinterpret_cast<uint4*>(o + (c0 + t) * (kHf ? 64 : cx.o_ts) + 32 * wh);
+            } else {  // a partial last chunk: the sequence's own rows, element pairs
 #pragma unroll
-                for (int c = 0; c < 4; ++c) dst[c] = pack8(v + 8 * c);
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int t = 16 * wq + (lane >> 2) + 8 * hr;
+                    if (t < nv) {
+                        uint32_t* dst = reinterpret_cast<uint32_t*>(
+                            o + (c0 + t) * (kHf ? 64 : cx.o_ts) + 32 * wh + 2 * (lane & 3));
+#pragma unroll
+                        for (int j2 = 0; j2 < 4; ++j2)
+                            dst[4 * j2] = pack2(v[4 * j2 + 2 * hr], v[4 * j2 + 2 * hr + 1]);
+                    }
+                }
             }
         }
-        if (!state_thread) tmem_st_wait();
-        // No barrier: nothing the next chunk does before its own first barrier touches
-        // what this epilogue reads or writes (o, the final product's output rows).
+        // No barrier: the next chunk reads and writes nothing this epilogue touches before
+        // its own first barrier (its prologue waits for the output store's reads).
         tc_fence_before();
         return true;
 }
@@ -1055,8 +1017,6 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     cx.lane = lane;
     cx.wq = wq;
     cx.wh = wh;
-    cx.m_row = 32 * wq + lane;
-    cx.state_thread = wq < 2;
     cx.row0 = (long long)bb * T + bos;
     cx.len = eos - bos;
     cx.mask = mask;
@@ -1112,19 +1072,18 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                            : lane == 3 ? &tm_b : lane == 4 ? &tm_w : lane == 5 ? &tm_v : &tm_o);
     if (warp == 0 && cx.len > 0) issue_loads<kGdn, kHf>(cx, 0, 0);
 
-    // The fp32 state lives in tensor memory, rows 0..63 of the final product's
-    // columns: warps with lane quarter 0/1 own row m = 32*wq + lane, columns
-    // [32*wh, 32*wh + 32).  Each chunk's epilogue 3 writes the fp16 copy in shared
-    // memory that feeds its final MMA.
-    const int m_row = cx.m_row;
+    // The fp32 state lives in tensor memory as an M = 64 accumulator: row k in lane
+    // (k % 16) + 32 (k / 16), so lanes 0..15 of warp w hold rows 16 (w % 4) + lane,
+    // columns [32 (w / 4), 32 (w / 4) + 32).  The other lanes of those columns stay unused.
+    const int srow = 16 * wq + lane;  // state row of this thread (lanes 0..15)
     const size_t state_off = ((size_t)n * H + h) * 4096;
-    if (cx.state_thread) {
+    {
         float sv[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) sv[j] = 0.f;
-        if (s0) {
+        if (s0 && lane < 16) {
             const size_t init_off = s0_shared ? (size_t)h * 4096 : state_off;
-            const float4* src = reinterpret_cast<const float4*>(s0 + init_off + m_row * 64 + 32 * wh);
+            const float4* src = reinterpret_cast<const float4*>(s0 + init_off + srow * 64 + 32 * wh);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float4 f = src[j];
@@ -1134,13 +1093,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                 sv[4 * j + 3] = f.w;
             }
         }
-        tmem_row_st32(cx.tmem + TM_DF, wq, 32 * wh, sv);
-        tmem_st_wait();
-    } else {  // output rows start at 0 (the final MMA accumulates onto them)
-        float z[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) z[j] = 0.f;
-        tmem_row_st32(cx.tmem + TM_DF, wq, 32 * wh, z);
+        tmem_row_st32(cx.tmem + TM_DFS, wq, 32 * wh, sv);
         tmem_st_wait();
     }
     tc_fence_before();
@@ -1162,13 +1115,15 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             (void)mbar_wait(cx.bar_mma, cx.mma_phase ^ 1u);
             (void)mbar_wait(cx.bar_g2, cx.g2_phase ^ 1u);
         }
-    } else if (cx.state_thread && sT) {
+    } else if (sT) {
         float sv[32];
-        tmem_row<2>(cx.tmem + TM_DF, wq, 32 * wh, sv);
-        float4* dst = reinterpret_cast<float4*>(sT + state_off + m_row * 64 + 32 * wh);
+        tmem_row<2>(cx.tmem + TM_DFS, wq, 32 * wh, sv);
+        if (lane < 16) {
+            float4* dst = reinterpret_cast<float4*>(sT + state_off + srow * 64 + 32 * wh);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+            for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+        }
     }
     if (tid == kStoreTid) bulk_wait0();  // the output stores are complete
     tc_fence_before();
