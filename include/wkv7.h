@@ -145,12 +145,25 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
  *                                        must not alias an input)
  *   ds0            [N, H, K, V]  fp32    dL/ds0, or NULL to skip
  *   workspace      device buffer of at least wkv7_bwd_workspace_bytes(B, T, H, K, V, N)
- *                  bytes (16-byte aligned; the caller owns it): the forward states
- *                  every 8 tokens and every token's u = S_{t-1}^T a, recomputed here
+ *                  bytes (16-byte aligned; the caller owns it; contents on return are
+ *                  scratch)
  *
  * K = V = 64 only.  A masked token passes the state gradient through and has zero
- * dw, dk, dv, da, db.  Two kernels on `stream`: a forward that writes the
- * checkpoints, then the reverse pass.
+ * dw, dk, dv, da, db.  Two kernel families (wkv7_bwd picks as AUTO does):
+ *   - bf16 (AUTO, WKV7_ALGO_CHUNKED): the chunked form on tcgen05 tensor cores.  The
+ *     state gradient G_t = dL/dS_t obeys G_t = r_t do_t^T + (diag(e^{w_{t+1}}) +
+ *     a_{t+1} b_{t+1}^T) G_{t+1}: a WKV7 recurrence read backwards in time (a and b
+ *     swapped, r and do as the write pair), so it runs on the chunked forward kernel
+ *     over reversed copies of the inputs, from dsT; its final state is ds0 and its
+ *     outputs (with k as the read vector) are dv.  A forward pass stores the fp16 state
+ *     at every 64-token chunk start, the reversed pass the state gradient at every
+ *     chunk end, and one kernel then forms every chunk's dr, dw, dk, da, db in
+ *     parallel from the chunk's inputs and those two 64 x 64 checkpoints (the adjoint
+ *     of the chunk's WY products).  Six launches on `stream`.
+ *   - fp32 (AUTO, WKV7_ALGO_RECURRENT): fp32 recurrences on CUDA cores: a forward that
+ *     stores the states every 8 tokens and every token's u = S_{t-1}^T a, then the
+ *     reverse pass.  Two launches on `stream`.
+ * The workspace bound covers both.
  */
 size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N);
 
@@ -160,6 +173,20 @@ wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v,
                      void* db, float* ds0, int B, int T, int H, int K, int V,
                      const int32_t* cu_seqlens, int N, wkv7_layout layout, wkv7_dtype dtype,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * wkv7_bwd_with_algo -- wkv7_bwd with the kernel family chosen by the caller:
+ * WKV7_ALGO_AUTO (as wkv7_bwd), WKV7_ALGO_RECURRENT (the fp32 CUDA-core recurrences,
+ * bf16 or fp32 inputs) or WKV7_ALGO_CHUNKED (bf16 only; fp32 returns
+ * WKV7_ERR_UNSUPPORTED).  Arguments and results are otherwise those of wkv7_bwd.
+ */
+wkv7_status wkv7_bwd_with_algo(const void* r, const void* w, const void* k, const void* v,
+                               const void* a, const void* b, const float* s0,
+                               const uint8_t* mask, const void* dout, const float* dsT, void* dr,
+                               void* dw, void* dk, void* dv, void* da, void* db, float* ds0,
+                               int B, int T, int H, int K, int V, const int32_t* cu_seqlens,
+                               int N, wkv7_layout layout, wkv7_dtype dtype, wkv7_algo algo,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * wkv7_bwd_noalloc -- wkv7_bwd with the library's own scratch instead of a caller

@@ -307,6 +307,11 @@ struct Ctx {
     uint32_t bar_never;
     float* gamma_s;
     const CUtensorMap *tm_r, *tm_w, *tm_k, *tm_v, *tm_a, *tm_b, *tm_o;
+    // State checkpoints (the backward's): when `ck` is set, each chunk's fp16 starting
+    // state (the S0 operand tile) is stored to checkpoint slice ck_z0 + chunk index.
+    const CUtensorMap* tm_ck;
+    bool ck;
+    int ck_z0;
     const __nv_bfloat16 *g, *beta;  // Gated DeltaNet only: [rows, H]
 };
 
@@ -743,6 +748,13 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             fence_proxy_async();
             tc_fence_before();
             if (__syncthreads_or(cx.timed_out)) return false;
+            // The chunk's fp16 starting state (written in the Gram window) to its
+            // checkpoint slice; the tile is next overwritten by epilogue 4's staging, and
+            // the same thread waits for this store's reads before that (epilogue U).
+            if (cx.ck && tid == kStoreTid) {
+                tma_store_3d(cx.tm_ck, sbase + OFF_S0, 0, 0, cx.ck_z0 + (c0 >> 6));
+                bulk_commit();
+            }
         }
 
         // ---- 6. [W | Z] = T [Abar | A_ak], T = (I - A_ab)^-1, by block forward
@@ -872,6 +884,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             float v[16];
             tmem_frag(tmem + TM_DU, wq, 32 * wh, v);
             frag_to_tile(sbase + L.A, 16 * wq, 4 * wh, v, lane, PackH{});
+            if (cx.ck && tid == kStoreTid) sm100::bulk_wait_read0();  // the S0 tile is read
             fence_proxy_async();
             tc_fence_before();
             if (__syncthreads_or(cx.timed_out)) return false;
@@ -912,7 +925,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
 
         // ---- 10. epilogue 4: the chunk's outputs (rows t = 16 wq + lane of O); the new fp32
         //          state stays in tensor memory. ---------------------------------------------
-        {
+        if (o != nullptr) {  // (no outputs: a state-only run)
             float v[16];
             tmem_frag(tmem + TM_DFO, wq, 32 * wh, v);
             if (nv == 64) {
@@ -957,10 +970,11 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                const __grid_constant__ CUtensorMap tm_o,
+               const __grid_constant__ CUtensorMap tm_ck,
                const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
                float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens,
                const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ beta,
-               int s0_shared, int stall_tid) {
+               int s0_shared, int stall_tid, int ck_slots) {
     extern __shared__ __align__(1024) uint8_t smem[];
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1022,14 +1036,14 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     cx.mask = mask;
     if (kHf) {
         const long long u0 = ((long long)bb * H + h) * T + bos;  // [B, H, T] token index
-        cx.o = o + u0 * 64;
+        cx.o = o ? o + u0 * 64 : nullptr;
         cx.o_ts = 64;
         cx.gb0 = u0;
         cx.gbs = 1;
         cx.tma_y = bos;
         cx.tma_z = bb * H + h;
     } else {
-        cx.o = o + (cx.row0 * H + h) * 64;
+        cx.o = o ? o + (cx.row0 * H + h) * 64 : nullptr;
         cx.o_ts = (long long)H * 64;
         cx.gb0 = cx.row0 * H + h;
         cx.gbs = H;
@@ -1048,6 +1062,9 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     cx.tm_a = &tm_a;
     cx.tm_b = &tm_b;
     cx.tm_o = &tm_o;
+    cx.tm_ck = &tm_ck;
+    cx.ck = ck_slots > 0;
+    cx.ck_z0 = h * ck_slots + (int)(cx.row0 >> 6) + n;  // slot: floor(row0 / 64) + n + chunk
     cx.g = g;
     cx.beta = beta;
 
@@ -1175,19 +1192,51 @@ inline bool make_map(CUtensorMap* map, const void* ptr, int B, int T, int H, int
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// State checkpoints: [H * slots][64][64] 16-bit (fp16) tiles, viewed as (64, 64,
+// H * slots), box = one whole tile.
+inline bool make_ck_map(CUtensorMap* map, const void* ptr, long long slices) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || slices <= 0 || slices > 0x7fffffffLL) return false;
+    cuuint64_t dims[3] = {64, 64, (cuuint64_t)slices};
+    cuuint64_t strides[2] = {64 * 2, 64 * 64 * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace chunked
 
 namespace chunked {
+// Optional extras of a launch: per-chunk state checkpoints (ck != nullptr: H * ck_slots
+// fp16 tiles; chunk c of unit (n, h) goes to slice h * ck_slots + floor(row0 / 64) + n + c,
+// row0 the sequence's first token row); o may be nullptr (no outputs).
+struct Extras {
+    void* ck = nullptr;
+    int ck_slots = 0;
+};
 template <bool kGdn, bool kHf>
 inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float* s0,
                           const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
                           const int32_t* cu_seqlens, const void* g, const void* beta,
-                          int s0_shared, int stall_tid, cudaStream_t stream) {
-    CUtensorMap maps[7];
+                          int s0_shared, int stall_tid, const Extras& ex,
+                          cudaStream_t stream) {
+    CUtensorMap maps[8];
     for (int i = 0; i < nmaps; ++i)
         if (!make_map(&maps[i], ptrs[i], B, T, H, kHf)) return cudaErrorInvalidValue;
     for (int i = nmaps; i < 6; ++i) maps[i] = maps[0];  // unused by the kernel
-    if (!make_map(&maps[6], o, B, T, H, kHf)) return cudaErrorInvalidValue;  // the output
+    if (o) {
+        if (!make_map(&maps[6], o, B, T, H, kHf)) return cudaErrorInvalidValue;  // the output
+    } else {
+        maps[6] = maps[0];  // unused: no outputs
+    }
+    if (ex.ck) {
+        if (ex.ck_slots <= 0 || !make_ck_map(&maps[7], ex.ck, (long long)H * ex.ck_slots))
+            return cudaErrorInvalidValue;
+    } else {
+        maps[7] = maps[0];  // unused: no checkpoints
+    }
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf>,
@@ -1197,22 +1246,23 @@ inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float
         attr_set = true;
     }
     chunked_kernel<kGdn, kHf><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], s0, mask,
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7], s0, mask,
         static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens,
         static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(beta), s0_shared,
-        stall_tid);
+        stall_tid, ex.ck ? ex.ck_slots : 0);
     return cudaGetLastError();
 }
 template <bool kGdn>
 inline cudaError_t launch(const void* const* ptrs, int nmaps, const float* s0,
                           const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
                           const int32_t* cu_seqlens, const void* g, const void* beta,
-                          int s0_shared, int head_first, int stall_tid, cudaStream_t stream) {
+                          int s0_shared, int head_first, int stall_tid, const Extras& ex,
+                          cudaStream_t stream) {
     return head_first
                ? launch_layout<kGdn, true>(ptrs, nmaps, s0, mask, o, sT, B, T, H, N, cu_seqlens,
-                                           g, beta, s0_shared, stall_tid, stream)
+                                           g, beta, s0_shared, stall_tid, ex, stream)
                : launch_layout<kGdn, false>(ptrs, nmaps, s0, mask, o, sT, B, T, H, N, cu_seqlens,
-                                            g, beta, s0_shared, stall_tid, stream);
+                                            g, beta, s0_shared, stall_tid, ex, stream);
 }
 }  // namespace chunked
 
@@ -1220,10 +1270,11 @@ inline cudaError_t launch_chunked(const void* r, const void* w, const void* k, c
                                   const void* a, const void* b, const float* s0,
                                   const uint8_t* mask, void* o, float* sT, int B, int T, int H,
                                   int N, const int32_t* cu_seqlens, int head_first,
-                                  int stall_tid, cudaStream_t stream) {
+                                  int stall_tid, cudaStream_t stream,
+                                  const chunked::Extras& ex = chunked::Extras{}) {
     const void* ptrs[6] = {r, w, k, v, a, b};
     return chunked::launch<false>(ptrs, 6, s0, mask, o, sT, B, T, H, N, cu_seqlens, nullptr,
-                                  nullptr, 0, head_first, stall_tid, stream);
+                                  nullptr, 0, head_first, stall_tid, ex, stream);
 }
 
 // Gated DeltaNet: q, k, v [B*T, H, 64] bf16 through the r, k, v maps; g, beta [B*T, H]
@@ -1236,7 +1287,7 @@ inline cudaError_t launch_chunked_gdn(const void* q, const void* k, const void* 
     // map order r, w, k, v: the unused w slot repeats q
     const void* ptrs[4] = {q, q, k, v};
     return chunked::launch<true>(ptrs, 4, s0, nullptr, o, sT, B, T, H, N, cu_seqlens, g, beta,
-                                 s0_shared, head_first, -1, stream);
+                                 s0_shared, head_first, -1, chunked::Extras{}, stream);
 }
 
 }  // namespace wkv7

@@ -1,0 +1,1088 @@
+// chunked_bwd.cuh -- backward of the WKV7 forward in the chunked (WY) form on tcgen05
+// tensor cores, bf16, K = V = 64 (the README's training entry, generalized_delta_rule,
+// supports backpropagation; rwkv-ops 0.9.0 README, "rwkv7op 使用方法").
+//
+// For L = sum(o * dout) + sum(S_T * dsT), with G_t = dL/dS_t,
+//     G_t = r_t do_t^T + (diag(e^{w_{t+1}}) + a_{t+1} b_{t+1}^T) G_{t+1},   G_{T-1} = r do^T + dsT,
+// and ds0 = (diag(e^{w_0}) + a_0 b_0^T) G_0.  Read backwards in time, that is itself a
+// WKV7 recurrence: with X_tau = G_{L-1-tau},
+//     X_tau = (diag(e^{w'_tau}) + b'_tau a'_tau^T) X_{tau-1} + k'_tau v'_tau^T
+// where w'_tau = w_{L-tau}, b' = a_{L-tau}, a' = b_{L-tau} (tau >= 1; the identity at
+// tau = 0) and k'_tau = r_{L-1-tau}, v'_tau = do_{L-1-tau} (tau < L), started from dsT;
+// one more transition (tau = L, no input) gives ds0.  So the backward runs in four
+// launches of its own plus two of the forward kernel:
+//   1. prep:     offsets of the reversed sequences (each padded at its start to a
+//                multiple of 64 tokens: p = 63 - L % 64 identity steps, then L + 1 steps);
+//   2. forward:  the chunked forward with per-chunk fp16 checkpoints of the state
+//                S0 at every chunk start, and no outputs;
+//   3. reverse:  the reversed, shifted inputs above (a masked token's transition is the
+//                identity, its output still feeds G) plus r' = k reversed, so that the
+//                reversed run's outputs o'_tau = X_tau^T k_{L-1-tau} = G_t^T k_t are dv;
+//   4. forward on the reversed inputs from dsT: its final state is ds0 and its
+//                per-chunk checkpoints hold G at the last token of every chunk of the
+//                original sequence (the padding puts chunk boundaries there);
+//   5. grad:     one CTA per original chunk, all chunks in parallel: the chunk's
+//                gradients from its inputs, S0 and dSL = G_e - r_e do_e^T (e its last
+//                token; dSL = dsT for a partial last chunk), on tcgen05;
+//   6. dv:       o' back to token order (zero for masked tokens).
+//
+// The per-chunk adjoint (grad kernel), with the forward's chunk algebra (chunked.cuh):
+//   X = Abar S0 + A_ak V,  U = T X                     (U = W S0 + Z V)
+//   dU = A_rb^T dO + Bhat dSL,  dX = T^T dU,  dT = dU X^T
+//   dA_rk = (dO V^T)_{s<=t}, dA_rb = (dO U^T)_{s<=t}, dA_ak = (dX V^T)_{s<t},
+//   dA_ab = (T^T dT T^T)_{s<t}
+//   acc_r = dA_rk k~ + dA_rb b~,  dRbar = dO S0^T       dr = E acc_r + e^{g_t} dRbar
+//   acc_a = dA_ak k~ + dA_ab b~,  dAbar = dX S0^T       da = E_{t-1} acc_a + e^{g_{t-1}} dAbar
+//   acc_k = dA_rk^T r~ + dA_ak^T a~ + V dSL^T            dk = acc_k / E
+//   acc_b = dA_rb^T r~ + dA_ab^T a~ + U dSL^T            db = acc_b / E
+//   dw_t = R - a_t da_t - sum_{t' < t} (r dr - k dk - b db + a da)_{t'}
+//   R = rowsum(S0 * (Rbar^T dO + Abar^T dX + e^{g_L} dSL))        (per channel)
+// (the adjoint of the E_t, E_{t-1} and e^{g_L} factors, summed back over the in-chunk
+// prefix of w).  e^{g_t} = E_t e^{g_L} is applied in fp32 in the last step: folded into
+// an fp16 operand (e^{g_L} S0) it would underflow once a chunk's decay is strong.  A masked token has zero dw, dk, da, db (its fold w = 0, a = k = b = 0
+// has no derivative); dv comes from the reversed run.
+#pragma once
+#include <cuda.h>
+
+#include "chunked.cuh"
+
+namespace wkv7 {
+namespace cbwd {
+
+using namespace chunked;
+using namespace sm100;
+
+constexpr int kThreads = 256;
+
+// ---------------------------------------------------------------------------------
+// Workspace layout (bytes, each region 256-aligned).
+// ---------------------------------------------------------------------------------
+struct Ws {
+    long long rows, rowsR;   // token rows of the inputs; bound on the reversed rows
+    long long slotsF, slotsR;  // checkpoint slots per head (forward, reversed)
+    size_t off_cu, off_ckF, off_ckR, off_rev, rev_stride, total;
+};
+inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline Ws ws_layout(long long rows, int N, int H) {
+    Ws w;
+    w.rows = rows;
+    w.rowsR = rows + 64LL * N;
+    w.slotsF = rows / 64 + N + 1;
+    w.slotsR = w.rowsR / 64 + N + 1;
+    w.off_cu = 0;
+    w.off_ckF = al256((size_t)(N + 1) * 4);
+    w.off_ckR = al256(w.off_ckF + (size_t)H * w.slotsF * 8192);
+    w.off_rev = al256(w.off_ckR + (size_t)H * w.slotsR * 8192);
+    w.rev_stride = al256((size_t)w.rowsR * H * 128);  // one reversed [rowsR, H, 64] bf16 tensor
+    w.total = w.off_rev + 7 * w.rev_stride;           // w', a', b', k', v', r', o'
+    return w;
+}
+
+// Sequence n: first token row in the [B*T] row space and length.
+__device__ __forceinline__ void seq_of(int n, int T, const int32_t* cu, long long& row0, int& L,
+                                       bool& ok) {
+    if (cu) {
+        const int bos = cu[n], eos = cu[n + 1];
+        ok = bos >= 0 && eos >= bos && eos <= T;
+        row0 = bos;
+        L = eos - bos;
+    } else {
+        ok = true;
+        row0 = (long long)n * T;
+        L = T;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// 1. prep: cu'[n] = sum_{m<n} 64 (floor(L_m / 64) + 1), one CTA.
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ cu, int T, int N,
+                                                    int32_t* __restrict__ cur) {
+    __shared__ int32_t tot[32];
+    __shared__ int32_t carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < N; base += 1024) {
+        const int n = base + tid;
+        int lr = 0;
+        if (n < N) {
+            long long row0;
+            int L;
+            bool ok;
+            seq_of(n, T, cu, row0, L, ok);
+            if (!ok) {
+                raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
+                L = 0;
+            }
+            lr = 64 * (L / 64 + 1);
+        }
+        int incl = lr;
+#pragma unroll
+        for (int d = 1; d < 32; d *= 2) {
+            const int up = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += up;
+        }
+        if (lane == 31) tot[warp] = incl;
+        __syncthreads();
+        int pre = carry;
+        for (int w2 = 0; w2 < warp; ++w2) pre += tot[w2];
+        if (n < N) cur[n] = pre + incl - lr;
+        __syncthreads();
+        if (tid == 1023) carry = pre + incl;
+        __syncthreads();
+    }
+    if (tid == 0) cur[N] = carry;
+}
+
+// ---------------------------------------------------------------------------------
+// 3. reverse: one CTA per (reversed 64-row chunk, head); thread = (row, 16 channels).
+// ---------------------------------------------------------------------------------
+template <bool kHf>
+__global__ void __launch_bounds__(256) reverse_kernel(
+    const __nv_bfloat16* __restrict__ r, const __nv_bfloat16* __restrict__ w,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ a,
+    const __nv_bfloat16* __restrict__ b, const __nv_bfloat16* __restrict__ dout,
+    const uint8_t* __restrict__ mask, const int32_t* __restrict__ cu,
+    const int32_t* __restrict__ cur, int T, int H, int N, __nv_bfloat16* __restrict__ rev,
+    size_t rev_stride_elems) {
+    const int gchunk = blockIdx.x, h = blockIdx.y;
+    const long long grow0 = 64LL * gchunk;
+    if (grow0 >= cur[N]) return;
+    int lo = 0, hi = N - 1;  // last n with cur[n] <= grow0
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cur[mid] <= grow0) lo = mid; else hi = mid - 1;
+    }
+    const int n = lo;
+    long long row0;
+    int L;
+    bool ok;
+    seq_of(n, T, cu, row0, L, ok);
+    if (!ok) L = 0;  // flagged by prep; the reversed sequence is all identity
+    const int p = 63 - (L & 63);
+    const int row = threadIdx.x >> 2, qq = threadIdx.x & 3;
+    const long long tp = grow0 + row - cur[n];  // tau' within the reversed sequence
+    const int tau = (int)tp - p;
+    const int t1 = L - tau;      // transition token (tau >= 1)
+    const int t2 = L - 1 - tau;  // input token (tau < L)
+    const bool has1 = tau >= 1 && tau <= L && (!mask || mask[row0 + t1] != 0);
+    const bool has2 = tau >= 0 && tau < L;
+    auto src = [&](const __nv_bfloat16* x, int t) -> const uint4* {
+        const long long e = kHf ? (((row0 / T) * H + h) * (long long)T + (row0 % T) + t) * 64
+                                : ((row0 + t) * H + h) * 64;
+        return reinterpret_cast<const uint4*>(x + e) + 2 * qq;
+    };
+    const size_t dst = ((size_t)(grow0 + row) * H + h) * 64;
+    uint4* out = reinterpret_cast<uint4*>(rev + dst) + 2 * qq;
+    const size_t str = rev_stride_elems / 8;  // in uint4
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    // w' a' b' k' v' r' = w[t1] b[t1] a[t1] r[t2] do[t2] k[t2]
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        out[0 * str + i] = has1 ? src(w, t1)[i] : z;
+        out[1 * str + i] = has1 ? src(b, t1)[i] : z;
+        out[2 * str + i] = has1 ? src(a, t1)[i] : z;
+        out[3 * str + i] = has2 ? src(r, t2)[i] : z;
+        out[4 * str + i] = has2 ? src(dout, t2)[i] : z;
+        out[5 * str + i] = has2 ? src(k, t2)[i] : z;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// 6. dv: dv[t] = o'[cur_n + p + L - 1 - t] (zero for a masked token); thread = 16 bytes.
+// ---------------------------------------------------------------------------------
+template <bool kHf>
+__global__ void __launch_bounds__(256) dv_kernel(const __nv_bfloat16* __restrict__ orev,
+                                                 const uint8_t* __restrict__ mask,
+                                                 const int32_t* __restrict__ cu,
+                                                 const int32_t* __restrict__ cur, int T, int H,
+                                                 int N, long long rows,
+                                                 __nv_bfloat16* __restrict__ dv) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // (row, h, 8 pieces)
+    if (i >= rows * H * 8) return;
+    const int piece = (int)(i & 7);
+    const int h = (int)((i >> 3) % H);
+    const long long grow = (i >> 3) / H;  // token row in [B*T]
+    int n;
+    if (cu) {
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (cu[mid] <= grow) lo = mid; else hi = mid - 1;
+        }
+        n = lo;
+        if (grow >= cu[N] || grow < cu[n]) return;  // rows outside every sequence: untouched
+    } else {
+        n = (int)(grow / T);
+    }
+    long long row0;
+    int L;
+    bool ok;
+    seq_of(n, T, cu, row0, L, ok);
+    if (!ok) return;
+    const int t = (int)(grow - row0);
+    const int p = 63 - (L & 63);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (!mask || mask[grow] != 0) {
+        const long long rr = cur[n] + p + L - 1 - t;
+        val = reinterpret_cast<const uint4*>(orev + (rr * H + h) * 64)[piece];
+    }
+    const long long e = kHf ? (((row0 / T) * H + h) * (long long)T + (row0 % T) + t) * 64
+                            : (grow * H + h) * 64;
+    reinterpret_cast<uint4*>(dv + e)[piece] = val;
+}
+
+// ---------------------------------------------------------------------------------
+// 5. grad: the per-chunk adjoint on tcgen05.
+// ---------------------------------------------------------------------------------
+// Shared-memory tiles (8 KB, 64 rows x 128 B, 128B swizzle).
+enum : uint32_t {
+    G_R = 0, G_A, G_K, G_B,  // r, a, k, b -> r~, a~, k~, b~ (bf16)
+    G_W,                     // w -> Abar (fp16)
+    G_V, G_DO,               // v, dO -> fp16 in place (dO rows past the chunk zeroed)
+    G_S0, G_DS,              // S0 (fp16 checkpoint), G -> dSL (fp16)
+    G_BH, G_RB, G_SPARE,     // Bhat, Rbar (fp16); a spare tile
+    G_E, G_E2,               // E (fp32, two tiles)
+    G_SP,                    // prologue scratch -> A_ab's diagonal blocks and T_ii; reloaded r
+    G_AB,                    // A_ab's blocks left of the diagonal (fp16); reloaded k
+    G_AAK, G_ARB,            // A_ak, A_rb (fp16, masked); reloaded a, b
+    G_T,                     // T = (I - A_ab)^-1 (fp16)
+    G_X, G_DU, G_DT,         // X -> U;  dU -> dX;  T_ii A_im scratch -> dT -> Y (fp16)
+    G_DARK, G_DAAK, G_DARB, G_DAAB,  // dA_rk, dA_ak, dA_rb, dA_ab (bf16); then staging
+    kNumTiles
+};
+constexpr uint32_t gt(uint32_t i) { return i * kTile; }
+constexpr uint32_t GOFF_MISC = kNumTiles * kTile;
+// misc: mbarriers (tma, mma, reload) at +0, +8, +16; TMEM address at +32;
+constexpr uint32_t GOFF_GAMMA = GOFF_MISC + 64;      // e^{g_L} (64 fp32, plain order)
+constexpr uint32_t GOFF_R = GOFF_GAMMA + 256;        // R per channel (64 fp32)
+constexpr uint32_t GOFF_EM0 = GOFF_R + 256;          // E_{-1} per channel (64 fp32)
+constexpr uint32_t GOFF_RAW = GOFF_EM0 + 256;        // raw r and dO of token 63 (2 x 64 fp32)
+constexpr uint32_t GOFF_TOT = GOFF_RAW + 512;        // scan totals [4 quadrants][64]
+constexpr uint32_t kGSmemBytes = GOFF_TOT + 1024;
+static_assert(kGSmemBytes <= 232448, "fits one CTA per SM");
+constexpr uint32_t kGTmemCols = 512;
+// TMEM columns (every accumulator M = 64): C0..C2 rotate through the phases' products;
+// dRbar, dAbar (phase C), acc_k, acc_b (D), acc_r (E, over C2) and acc_a (E) stay to the end.
+constexpr uint32_t C0 = 0, C1 = 64, C2 = 128, C_DRB = 192, C_DAB = 256, C_AK = 320, C_AB = 384,
+                   C_AR = 128, C_AA = 448;
+
+// E tile index (fp32 [t][c], groups of 8 channels XOR-swizzled by row).
+__device__ __forceinline__ int eidx(int t, int c) { return t * 64 + (c ^ ((t & 7) << 3)); }
+
+// Store one warp's share (rows 16 wq.., columns 32 wh..) of the M = 64 accumulator at
+// TMEM column `col` as a 16-bit tile; mode 1 keeps s <= t, mode 2 keeps s < t.
+template <typename Pack>
+__device__ __forceinline__ void acc_to_tile(uint32_t tmem, uint32_t col, uint32_t tile, int wq,
+                                            int wh, int lane, int mode, Pack pk) {
+    float v[16];
+    tmem_frag(tmem + col, wq, 32 * wh, v);
+    if (mode) {
+        const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = 16 * wq + g + 8 * hr, s = 32 * wh + 8 * j + 2 * q + e;
+                    if (mode == 1 ? s > t : s >= t) v[4 * j + 2 * hr + e] = 0.f;
+                }
+    }
+    frag_to_tile(tile, 16 * wq, 4 * wh, v, lane, pk);
+}
+
+// D (+)= A B over K = 64 (four K16 steps) from 64-row tiles; a_mn / b_mn: the tile is
+// stored MN-major for that operand (rows = the K index), else K-major (rows = M / N).
+__device__ __forceinline__ void mma64(uint32_t tmem_d, uint32_t a, bool a_mn, uint32_t b, bool b_mn,
+                                      bool bf16, bool acc) {
+    const uint32_t id = bf16 ? idesc_bf16(64, 64, a_mn, b_mn) : idesc_f16(64, 64, a_mn, b_mn);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t da = a_mn ? smem_desc(a + 2048 * kk, 8192, 1024) : smem_desc(a + 32 * kk, 16, 1024);
+        const uint64_t db = b_mn ? smem_desc(b + 2048 * kk, 8192, 1024) : smem_desc(b + 32 * kk, 16, 1024);
+        umma_bf16(tmem_d, da, db, id, (acc || kk > 0) ? 1u : 0u);
+    }
+}
+
+template <bool kHf>
+__global__ void __launch_bounds__(kThreads, 1)
+grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
+            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+            const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+            const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_ckf,
+            const __grid_constant__ CUtensorMap tm_ckr, const __grid_constant__ CUtensorMap tm_dr,
+            const __grid_constant__ CUtensorMap tm_dw, const __grid_constant__ CUtensorMap tm_dk,
+            const __grid_constant__ CUtensorMap tm_da, const __grid_constant__ CUtensorMap tm_db,
+            const uint8_t* __restrict__ mask, const int32_t* __restrict__ cu,
+            const int32_t* __restrict__ cur, int T, int H, int N, int slotsF, int slotsR,
+            __nv_bfloat16* __restrict__ dr, __nv_bfloat16* __restrict__ dw,
+            __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ da,
+            __nv_bfloat16* __restrict__ db) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    using namespace sm100;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wq = warp & 3, wh = warp >> 2;
+    const int g = lane >> 2, q = lane & 3;
+    const int slot = blockIdx.x, h = blockIdx.y;
+
+    // The chunk of this slot: sequence n with floor(row0_n / 64) + n <= slot, chunk c.
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const long long r0 = cu ? (long long)cu[mid] : (long long)mid * T;
+        if ((r0 >> 6) + mid <= slot) lo = mid; else hi = mid - 1;
+    }
+    const int n = lo;
+    long long row0;
+    int L;
+    bool ok;
+    seq_of(n, T, cu, row0, L, ok);
+    if (!ok) return;  // flagged by prep
+    const int c = slot - (int)((row0 >> 6) + n);
+    if (c < 0 || 64 * c >= L) return;
+    const int nv = min(64, L - 64 * c);
+    const long long crow = row0 + 64LL * c;  // first token row of the chunk
+    const int rslot = cur[n] / 64 + n + L / 64 - c;
+
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_tma = sbase + GOFF_MISC, bar_mma = sbase + GOFF_MISC + 8,
+                   bar_rl = sbase + GOFF_MISC + 16;
+    float* gam = reinterpret_cast<float*>(smem + GOFF_GAMMA);
+    float* Rc = reinterpret_cast<float*>(smem + GOFF_R);
+    float* em0 = reinterpret_cast<float*>(smem + GOFF_EM0);
+    float* raw = reinterpret_cast<float*>(smem + GOFF_RAW);
+    float* tot = reinterpret_cast<float*>(smem + GOFF_TOT);
+    float* Ef = reinterpret_cast<float*>(smem + gt(G_E));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GOFF_MISC + 32);
+    int timed_out = 0;
+    uint32_t mph = 0;
+
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), kGTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_rl, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // token-major maps: (channel, head, token row); head first: (channel, token, b*H + h)
+    const int cy = kHf ? (int)(crow % T) : h;
+    const int cz = kHf ? (int)((crow / T) * H + h) : (int)crow;
+    if (warp == 0) {
+        if (lane == 0) mbar_arrive_expect_tx(bar_tma, 9 * kTile);
+        __syncwarp();
+        if (lane < 9) {
+            const CUtensorMap* map = lane == 0 ? &tm_r : lane == 1 ? &tm_a : lane == 2 ? &tm_k
+                                   : lane == 3 ? &tm_b : lane == 4 ? &tm_w : lane == 5 ? &tm_v
+                                   : lane == 6 ? &tm_do : lane == 7 ? &tm_ckf : &tm_ckr;
+            const uint32_t dst = lane == 0 ? G_R : lane == 1 ? G_A : lane == 2 ? G_K
+                               : lane == 3 ? G_B : lane == 4 ? G_W : lane == 5 ? G_V
+                               : lane == 6 ? G_DO : lane == 7 ? G_S0 : G_DS;
+            if (lane < 7)
+                tma_load_3d(sbase + gt(dst), map, bar_tma, 0, cy, cz);
+            else
+                tma_load_3d(sbase + gt(dst), map, bar_tma, 0, 0,
+                            lane == 7 ? h * slotsF + slot : h * slotsR + rslot);
+        }
+    }
+    wait_or_abort(bar_tma, 0, timed_out);
+
+    // ---- prologue: prefix sums of w (mask folded), E, and the operands --------------
+    {
+        float* scratch = reinterpret_cast<float*>(smem + gt(G_SP));
+        const int j = tid & 7, t0 = 2 * (tid >> 3);
+        const bool ina = t0 < nv, inb = t0 + 1 < nv;
+        const bool va = ina && (!mask || mask[crow + t0] != 0);
+        const bool vb = inb && (!mask || mask[crow + t0 + 1] != 0);
+        const uint32_t offa = sw(t0, j), offb = sw(t0 + 1, j);
+        const int h0 = cswz(8 * j), h1 = cswz(8 * j + 4);
+        float wa[8], wb[8], incl[8];
+        {
+            const uint32_t ma = va ? 0xFFFFFFFFu : 0u, mb = vb ? 0xFFFFFFFFu : 0u;
+            uint4 qa = *reinterpret_cast<const uint4*>(smem + gt(G_W) + offa);
+            uint4 qb = *reinterpret_cast<const uint4*>(smem + gt(G_W) + offb);
+            qa.x &= ma; qa.y &= ma; qa.z &= ma; qa.w &= ma;
+            qb.x &= mb; qb.y &= mb; qb.z &= mb; qb.w &= mb;
+            unpack8(qa, wa);
+            unpack8(qb, wb);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            wa[e] *= kLog2e;
+            wb[e] *= kLog2e;
+            incl[e] = wa[e] + wb[e];
+        }
+#pragma unroll
+        for (int d = 8; d < 32; d *= 2) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float up = __shfl_up_sync(0xffffffffu, incl[e], d);
+                if (lane >= d) incl[e] += up;
+            }
+        }
+        float* wt = scratch + SCR_TOT;
+        if (lane >= 24) {
+            *reinterpret_cast<float4*>(wt + warp * 64 + h0) = make_float4(incl[0], incl[1], incl[2], incl[3]);
+            *reinterpret_cast<float4*>(wt + warp * 64 + h1) = make_float4(incl[4], incl[5], incl[6], incl[7]);
+        }
+        if (__syncthreads_or(timed_out)) goto teardown;
+        if (warp == 0) {
+            const int ch = cswz(2 * lane);
+            float2 gL = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int w2 = 0; w2 < 8; ++w2) {
+                const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
+                *reinterpret_cast<float2*>(scratch + SCR_PRE + w2 * 64 + ch) = gL;
+                gL.x += x.x;
+                gL.y += x.y;
+            }
+            *reinterpret_cast<float2*>(scratch + SCR_C + ch) = gL;
+            // plain channel order from here on: ch holds channels 2 lane, 2 lane + 1 (cswz
+            // permutes 4-channel groups, so the pair stays together)
+            const int c2 = 2 * lane;
+            const float2 gLp = *reinterpret_cast<const float2*>(scratch + SCR_C + ch);
+            gam[c2] = ex2(gLp.x);
+            gam[c2 + 1] = ex2(gLp.y);
+        }
+        __syncthreads();
+        float ga[8];
+        {
+            const float4 x0 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + h0);
+            const float4 x1 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + h1);
+            const float pre[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ga[e] = pre[e] + (incl[e] - wb[e]);
+        }
+        float cc[8], ec[8];
+        *reinterpret_cast<float4*>(cc) = *reinterpret_cast<const float4*>(scratch + SCR_C + h0);
+        *reinterpret_cast<float4*>(cc + 4) = *reinterpret_cast<const float4*>(scratch + SCR_C + h1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ec[e] = gam[8 * j + e];
+        float Ep[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) Ep[e] = ex2(clamp2(ga[e] - wa[e] - cc[e]));
+        if (t0 == 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) em0[8 * j + e] = Ep[e];
+        }
+        __syncthreads();  // every thread has read the scan scratch (the SP tile)
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const uint32_t off = it ? offb : offa;
+            const bool val = it ? vb : va;
+            const bool in = it ? inb : ina;
+            const int t = t0 + it;
+            float rv[8], av[8], kv[8], bv[8], vv[8], dv[8];
+            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_R) + off), rv);
+            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_A) + off), av);
+            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_K) + off), kv);
+            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_B) + off), bv);
+            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_V) + off), vv);
+            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_DO) + off), dv);
+            if (t == 63) {  // raw r and dO of the last token (dSL = G - r do^T)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    raw[8 * j + e] = rv[e];
+                    raw[64 + 8 * j + e] = dv[e];
+                }
+            }
+            float rt[8], at[8], kt[8], bt[8], ab[8], rb[8], Ev[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float gg = it ? ga[e] + wb[e] : ga[e];
+                const float d = clamp2(gg - cc[e]);
+                const float E = ex2(d);
+                const float inv = val ? ex2(-d) : 0.f;
+                const float ep = val ? Ep[e] : 0.f;
+                rt[e] = in ? rv[e] * E : 0.f;
+                at[e] = av[e] * ep;
+                kt[e] = kv[e] * inv;
+                bt[e] = bv[e] * inv;
+                ab[e] = at[e] * ec[e];  // Abar = a~ e^{g_L}
+                rb[e] = rt[e] * ec[e];  // Rbar = r~ e^{g_L}
+                Ev[e] = E;
+                Ep[e] = E;
+                if (!in) dv[e] = 0.f;
+            }
+            *reinterpret_cast<uint4*>(smem + gt(G_R) + off) = pack8(rt);
+            *reinterpret_cast<uint4*>(smem + gt(G_A) + off) = pack8(at);
+            *reinterpret_cast<uint4*>(smem + gt(G_K) + off) = pack8(kt);
+            *reinterpret_cast<uint4*>(smem + gt(G_B) + off) = pack8(bt);
+            *reinterpret_cast<uint4*>(smem + gt(G_W) + off) = pack8h(ab);
+            *reinterpret_cast<uint4*>(smem + gt(G_RB) + off) = pack8h(rb);
+            *reinterpret_cast<uint4*>(smem + gt(G_BH) + off) = pack8h(bt);
+            *reinterpret_cast<uint4*>(smem + gt(G_V) + off) = pack8h(vv);
+            *reinterpret_cast<uint4*>(smem + gt(G_DO) + off) = pack8h(dv);
+            *reinterpret_cast<float4*>(Ef + eidx(t, 8 * j)) = make_float4(Ev[0], Ev[1], Ev[2], Ev[3]);
+            *reinterpret_cast<float4*>(Ef + eidx(t, 8 * j + 4)) = make_float4(Ev[4], Ev[5], Ev[6], Ev[7]);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    // ---- Gram: [A_ak | A_ab] = a~ [k~ | b~]^T, A_rb = r~ b~^T (bf16) ----------------
+    if (tid == 0) {
+        tc_fence_after();
+        mma64(tmem + C0, sbase + gt(G_A), false, sbase + gt(G_K), false, true, false);
+        mma64(tmem + C1, sbase + gt(G_A), false, sbase + gt(G_B), false, true, false);
+        mma64(tmem + C2, sbase + gt(G_R), false, sbase + gt(G_B), false, true, false);
+        umma_commit(bar_mma);
+    }
+    // While it runs: dSL (fp16) and R = e^{g_L} rowsum(S0 dSL).
+    {
+        const int row = tid >> 2, qq = tid & 3;  // state row (channel) and 16 of its columns
+        const float gm = gam[row];
+        const bool full = nv == 64;
+        const float rr = full ? raw[row] : 0.f;
+        float part = 0.f;
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+            const int chk = 2 * qq + hc;
+            const uint32_t off = sw(row, chk);
+            const uint4 s4 = *reinterpret_cast<const uint4*>(smem + gt(G_S0) + off);
+            const uint4 g4 = *reinterpret_cast<const uint4*>(smem + gt(G_DS) + off);
+            const uint32_t sw4[4] = {s4.x, s4.y, s4.z, s4.w}, gw4[4] = {g4.x, g4.y, g4.z, g4.w};
+            uint32_t go[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sw4[i]));
+                float2 gf = __half22float2(*reinterpret_cast<const __half2*>(&gw4[i]));
+                const int v0 = 8 * chk + 2 * i;
+                gf.x -= rr * raw[64 + v0];
+                gf.y -= rr * raw[64 + v0 + 1];
+                part = fmaf(sf.x, gf.x, fmaf(sf.y, gf.y, part));
+                go[i] = pack2h(gf.x, gf.y);
+            }
+            *reinterpret_cast<uint4*>(smem + gt(G_DS) + off) = make_uint4(go[0], go[1], go[2], go[3]);
+        }
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        if (qq == 0) Rc[row] = gm * part;
+        fence_proxy_async();
+    }
+    wait_or_abort(bar_mma, mph, timed_out);
+    mph ^= 1;
+    tc_fence_after();
+
+    // ---- Gram epilogue: A_ab's diagonal inverses and left blocks; A_ak, A_rb --------
+    if (wh == 1) {
+        float v[2][16];
+        tmem_frag(tmem + C1, wq, 0, v[0]);
+        tmem_frag(tmem + C1, wq, 32, v[1]);
+        float* dg = reinterpret_cast<float*>(smem + gt(G_SP));
+        {
+            const bool hi = wq >= 2, odd = wq & 1;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int s2 = 8 * jj + 2 * q + e;
+                    const int i0 = 4 * jj + e, i1 = 4 * (2 + jj) + e;
+                    const float lo0 = odd ? v[0][i1] : v[0][i0], hi0 = odd ? v[1][i1] : v[1][i0];
+                    const float lo1 = odd ? v[0][i1 + 2] : v[0][i0 + 2];
+                    const float hi1 = odd ? v[1][i1 + 2] : v[1][i0 + 2];
+                    dg[dtidx(wq, s2, g)] = (s2 < g) ? (hi ? hi0 : lo0) : 0.f;
+                    dg[dtidx(wq, s2, g + 8)] = (s2 < g + 8) ? (hi ? hi1 : lo1) : 0.f;
+                }
+        }
+        __syncwarp();
+        if (lane < 16) {
+            const int bb = wq, cidx = lane;
+            const float* nt = dg + dtidx(bb, 0, 0);
+            float x[16];
+#pragma unroll
+            for (int t2 = 0; t2 < 16; ++t2) x[t2] = (t2 == cidx) ? 1.f : 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < 15; ++s2) {
+                const float xs = x[s2];
+#pragma unroll
+                for (int t4 = ((s2 + 1) >> 2) << 2; t4 < 16; t4 += 4) {
+                    const float4 n4 = *reinterpret_cast<const float4*>(nt + s2 * kDgRow + t4);
+                    const float nvv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (t4 + e > s2) x[t4 + e] = fmaf(nvv[e], xs, x[t4 + e]);
+                }
+            }
+            uint8_t* Tb = smem + gt(G_SP) + kDiagBytes;
+#pragma unroll
+            for (int t2 = 0; t2 < 16; t2 += 2) {
+                const uint32_t hp = pack2h(x[t2], x[t2 + 1]);
+                *reinterpret_cast<uint16_t*>(Tb + bb * 768 + t2 * 48 + 2 * cidx) = (uint16_t)(hp & 0xFFFFu);
+                *reinterpret_cast<uint16_t*>(Tb + bb * 768 + (t2 + 1) * 48 + 2 * cidx) = (uint16_t)(hp >> 16);
+            }
+        }
+        if (wq > 0) frag_half_to_tile(sbase + gt(G_AB), 16 * wq, 0, 0, v[0], lane, PackH{});
+        if (wq > 1) frag_half_to_tile(sbase + gt(G_AB), 16 * wq, 0, 1, v[0], lane, PackH{});
+        if (wq > 2) frag_half_to_tile(sbase + gt(G_AB), 16 * wq, 4, 0, v[1], lane, PackH{});
+    } else {
+        acc_to_tile(tmem, C0, sbase + gt(G_AAK), wq, 0, lane, 2, PackH{});
+        acc_to_tile(tmem, C0, sbase + gt(G_AAK), wq, 1, lane, 2, PackH{});
+        acc_to_tile(tmem, C2, sbase + gt(G_ARB), wq, 0, lane, 1, PackH{});
+        acc_to_tile(tmem, C2, sbase + gt(G_ARB), wq, 1, lane, 1, PackH{});
+    }
+    tc_fence_before();
+    if (__syncthreads_or(timed_out)) goto teardown;
+
+    // ---- T = (I - A_ab)^-1 by block forward substitution (warp-level fp16 MMAs):
+    //      warps 0..5 form T_ii A_im (m < i); warp w < 4 then builds column block w:
+    //      X_w = T_ww, X_i = sum_{w<=m<i} (T_ii A_im) X_m. ------------------------------
+    {
+        uint8_t* Tb = smem + gt(G_SP) + kDiagBytes;
+        uint8_t* Tab = smem + gt(G_DT);
+        const int lr = (lane & 7) + 8 * ((lane >> 3) & 1), lc = 8 * (lane >> 4);
+        const uint32_t a_lane = lr * 48 + 2 * lc;
+        auto a_frag = [&](const uint8_t* blk, uint32_t (&af)[4]) {
+            ldsm_x4(smem_u32(blk) + a_lane, af[0], af[1], af[2], af[3]);
+        };
+        if (warp < 6) {
+            const int i = warp < 1 ? 1 : (warp < 3 ? 2 : 3);
+            const int m = warp < 1 ? 0 : (warp < 3 ? warp - 1 : warp - 3);
+            uint32_t af[4];
+            a_frag(Tb + i * 768, af);
+            float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            uint32_t bfa[4];
+            ldsm_x4_t(sbase + gt(G_AB) + sw(16 * i + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * m + (lane >> 4)),
+                      bfa[0], bfa[1], bfa[2], bfa[3]);
+            mma_f16_16816(z[0], af[0], af[1], af[2], af[3], bfa[0], bfa[1]);
+            mma_f16_16816(z[1], af[0], af[1], af[2], af[3], bfa[2], bfa[3]);
+            uint8_t* dst = Tab + warp * 768;  // blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                *reinterpret_cast<uint32_t*>(dst + g * 48 + 2 * (8 * nt + 2 * q)) = pack2h(z[nt][0], z[nt][1]);
+                *reinterpret_cast<uint32_t*>(dst + (g + 8) * 48 + 2 * (8 * nt + 2 * q)) = pack2h(z[nt][2], z[nt][3]);
+            }
+        }
+        __syncthreads();
+        if (warp < 4) {
+            const int wcol = warp;  // column block of T
+            uint8_t* tt = smem + gt(G_T);
+            uint32_t xb[3][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t top[2], bot[2];
+                if (i < wcol) {
+                    top[0] = top[1] = bot[0] = bot[1] = 0u;
+                } else if (i == wcol) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        top[nt] = *reinterpret_cast<const uint32_t*>(Tb + i * 768 + g * 48 + 2 * (8 * nt + 2 * q));
+                        bot[nt] = *reinterpret_cast<const uint32_t*>(Tb + i * 768 + (g + 8) * 48 + 2 * (8 * nt + 2 * q));
+                    }
+                } else {
+                    float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                    for (int m = 0; m < 3; ++m) {
+                        if (m < wcol || m >= i) continue;
+                        const int blk = (i == 1) ? 0 : (i == 2 ? 1 + m : 3 + m);
+                        uint32_t af[4];
+                        a_frag(Tab + blk * 768, af);
+                        mma_f16_16816(y[0], af[0], af[1], af[2], af[3], xb[m][0], xb[m][1]);
+                        mma_f16_16816(y[1], af[0], af[1], af[2], af[3], xb[m][2], xb[m][3]);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        top[nt] = pack2h(y[nt][0], y[nt][1]);
+                        bot[nt] = pack2h(y[nt][2], y[nt][3]);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int col = 16 * wcol + 8 * nt + 2 * q;
+                    *reinterpret_cast<uint32_t*>(tt + swe(16 * i + g, col)) = top[nt];
+                    *reinterpret_cast<uint32_t*>(tt + swe(16 * i + g + 8, col)) = bot[nt];
+                    if (i < 3) {
+                        xb[i][2 * nt] = movmatrix_t(top[nt]);
+                        xb[i][2 * nt + 1] = movmatrix_t(bot[nt]);
+                    }
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    // ---- A: X = Abar S0 + A_ak V;  dU = A_rb^T dO + Bhat dSL;  dA_rk = dO V^T ---------
+    if (tid == 0) {
+        tc_fence_after();
+        mma64(tmem + C0, sbase + gt(G_W), false, sbase + gt(G_S0), true, false, false);
+        mma64(tmem + C0, sbase + gt(G_AAK), false, sbase + gt(G_V), true, false, true);
+        mma64(tmem + C1, sbase + gt(G_ARB), true, sbase + gt(G_DO), true, false, false);
+        mma64(tmem + C1, sbase + gt(G_BH), false, sbase + gt(G_DS), true, false, true);
+        mma64(tmem + C2, sbase + gt(G_DO), false, sbase + gt(G_V), false, false, false);
+        umma_commit(bar_mma);
+    }
+    wait_or_abort(bar_mma, mph, timed_out);
+    mph ^= 1;
+    tc_fence_after();
+    // The original r, k, a, b again (for dw), into tiles that are dead now.
+    if (tid == 32) {
+        mbar_arrive_expect_tx(bar_rl, 4 * kTile);
+        tma_load_3d(sbase + gt(G_SP), &tm_r, bar_rl, 0, cy, cz);
+        tma_load_3d(sbase + gt(G_AB), &tm_k, bar_rl, 0, cy, cz);
+        tma_load_3d(sbase + gt(G_AAK), &tm_a, bar_rl, 0, cy, cz);
+        tma_load_3d(sbase + gt(G_ARB), &tm_b, bar_rl, 0, cy, cz);
+    }
+    acc_to_tile(tmem, C0, sbase + gt(G_X), wq, wh, lane, 0, PackH{});
+    acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, wh, lane, 0, PackH{});
+    acc_to_tile(tmem, C2, sbase + gt(G_DARK), wq, wh, lane, 1, PackB{});
+    fence_proxy_async();
+    tc_fence_before();
+    if (__syncthreads_or(timed_out)) goto teardown;
+
+    // ---- B: U = T X;  dX = T^T dU;  dT = dU X^T ------------------------------------
+    if (tid == 0) {
+        tc_fence_after();
+        mma64(tmem + C0, sbase + gt(G_T), false, sbase + gt(G_X), true, false, false);
+        mma64(tmem + C1, sbase + gt(G_T), true, sbase + gt(G_DU), true, false, false);
+        mma64(tmem + C2, sbase + gt(G_DU), false, sbase + gt(G_X), false, false, false);
+        umma_commit(bar_mma);
+    }
+    wait_or_abort(bar_mma, mph, timed_out);
+    mph ^= 1;
+    tc_fence_after();
+    acc_to_tile(tmem, C0, sbase + gt(G_X), wq, wh, lane, 0, PackH{});   // U
+    acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, wh, lane, 0, PackH{});  // dX
+    acc_to_tile(tmem, C2, sbase + gt(G_DT), wq, wh, lane, 0, PackH{});  // dT
+    fence_proxy_async();
+    tc_fence_before();
+    if (__syncthreads_or(timed_out)) goto teardown;
+
+    // ---- C: dA_rb = dO U^T; dA_ak = dX V^T; Y = dT T^T; dRbar = dO S0^T; dAbar = dX S0^T
+    if (tid == 0) {
+        tc_fence_after();
+        mma64(tmem + C0, sbase + gt(G_DO), false, sbase + gt(G_X), false, false, false);
+        mma64(tmem + C1, sbase + gt(G_DU), false, sbase + gt(G_V), false, false, false);
+        mma64(tmem + C2, sbase + gt(G_DT), false, sbase + gt(G_T), false, false, false);
+        mma64(tmem + C_DRB, sbase + gt(G_DO), false, sbase + gt(G_S0), false, false, false);
+        mma64(tmem + C_DAB, sbase + gt(G_DU), false, sbase + gt(G_S0), false, false, false);
+        umma_commit(bar_mma);
+    }
+    wait_or_abort(bar_mma, mph, timed_out);
+    mph ^= 1;
+    tc_fence_after();
+    acc_to_tile(tmem, C0, sbase + gt(G_DARB), wq, wh, lane, 1, PackB{});
+    acc_to_tile(tmem, C1, sbase + gt(G_DAAK), wq, wh, lane, 2, PackB{});
+    acc_to_tile(tmem, C2, sbase + gt(G_DT), wq, wh, lane, 0, PackH{});  // Y
+    fence_proxy_async();
+    tc_fence_before();
+    if (__syncthreads_or(timed_out)) goto teardown;
+
+    // ---- D: dA_ab = T^T Y; P = Rbar^T dO + Abar^T dX; acc_k = V dSL^T; acc_b = U dSL^T
+    if (tid == 0) {
+        tc_fence_after();
+        mma64(tmem + C0, sbase + gt(G_T), true, sbase + gt(G_DT), true, false, false);
+        mma64(tmem + C1, sbase + gt(G_RB), true, sbase + gt(G_DO), true, false, false);
+        mma64(tmem + C1, sbase + gt(G_W), true, sbase + gt(G_DU), true, false, true);
+        mma64(tmem + C_AK, sbase + gt(G_V), false, sbase + gt(G_DS), false, false, false);
+        mma64(tmem + C_AB, sbase + gt(G_X), false, sbase + gt(G_DS), false, false, false);
+        umma_commit(bar_mma);
+    }
+    wait_or_abort(bar_mma, mph, timed_out);
+    mph ^= 1;
+    tc_fence_after();
+    acc_to_tile(tmem, C0, sbase + gt(G_DAAB), wq, wh, lane, 2, PackB{});
+    {  // R += rowsum(S0 * P) over this warp's 32 columns
+        float v[16];
+        tmem_frag(tmem + C1, wq, 32 * wh, v);
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int row = 16 * wq + g + 8 * hr;
+            float part = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(
+                    smem + gt(G_S0) + swe(row, 32 * wh + 8 * j + 2 * q)));
+                part = fmaf(s2.x, v[4 * j + 2 * hr], fmaf(s2.y, v[4 * j + 2 * hr + 1], part));
+            }
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (q == 0) atomicAdd(Rc + row, part);
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    if (__syncthreads_or(timed_out)) goto teardown;
+
+    // ---- E: the four gradient accumulators (bf16 against the Gram operands) ----------
+    if (tid == 0) {
+        tc_fence_after();
+        mma64(tmem + C_AR, sbase + gt(G_DARK), false, sbase + gt(G_K), true, true, false);
+        mma64(tmem + C_AR, sbase + gt(G_DARB), false, sbase + gt(G_B), true, true, true);
+        mma64(tmem + C_AA, sbase + gt(G_DAAK), false, sbase + gt(G_K), true, true, false);
+        mma64(tmem + C_AA, sbase + gt(G_DAAB), false, sbase + gt(G_B), true, true, true);
+        mma64(tmem + C_AK, sbase + gt(G_DARK), true, sbase + gt(G_R), true, true, true);
+        mma64(tmem + C_AK, sbase + gt(G_DAAK), true, sbase + gt(G_A), true, true, true);
+        mma64(tmem + C_AB, sbase + gt(G_DARB), true, sbase + gt(G_R), true, true, true);
+        mma64(tmem + C_AB, sbase + gt(G_DAAB), true, sbase + gt(G_A), true, true, true);
+        umma_commit(bar_mma);
+    }
+    wait_or_abort(bar_mma, mph, timed_out);
+    mph ^= 1;
+    tc_fence_after();
+    wait_or_abort(bar_rl, 0, timed_out);
+
+    // ---- final epilogue: dr, da, dk, db, and dw by an exclusive prefix over tokens ----
+    {
+        float ar[16], aa[16], ak[16], abv[16], drb[16], dab[16];
+        tmem_frag(tmem + C_AR, wq, 32 * wh, ar);
+        tmem_frag(tmem + C_AA, wq, 32 * wh, aa);
+        tmem_frag(tmem + C_AK, wq, 32 * wh, ak);
+        tmem_frag(tmem + C_AB, wq, 32 * wh, abv);
+        tmem_frag(tmem + C_DRB, wq, 32 * wh, drb);
+        tmem_frag(tmem + C_DAB, wq, 32 * wh, dab);
+        float hv[16], fv[16];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int t = 16 * wq + g + 8 * hr;
+            const bool in = t < nv;
+            const bool val = in && (!mask || mask[crow + t] != 0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int cidx = 32 * wh + 8 * j + 2 * q;
+                const float2 E2 = *reinterpret_cast<const float2*>(Ef + eidx(t, cidx));
+                const float2 Em = t > 0 ? *reinterpret_cast<const float2*>(Ef + eidx(t - 1, cidx))
+                                        : make_float2(em0[cidx], em0[cidx + 1]);
+                const uint32_t bo = swe(t, cidx);
+                const float2 r2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_SP) + bo));
+                const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_AB) + bo));
+                const float2 a2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_AAK) + bo));
+                const float2 b2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_ARB) + bo));
+                const float Ee[2] = {E2.x, E2.y}, Eme[2] = {Em.x, Em.y};
+                const float re[2] = {r2.x, r2.y}, ke[2] = {k2.x, k2.y}, ae[2] = {a2.x, a2.y},
+                            be[2] = {b2.x, b2.y};
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int ix = 4 * j + 2 * hr + e;
+                    const float gm = gam[cidx + e];
+                    const float vdr = in ? fmaf(Ee[e], ar[ix], (Ee[e] * gm) * drb[ix]) : 0.f;
+                    const float vdk = val ? ak[ix] / Ee[e] : 0.f;
+                    const float vdb = val ? abv[ix] / Ee[e] : 0.f;
+                    const float vda = val ? fmaf(Eme[e], aa[ix], (Eme[e] * gm) * dab[ix]) : 0.f;
+                    ar[ix] = vdr;
+                    ak[ix] = vdk;
+                    abv[ix] = vdb;
+                    aa[ix] = vda;
+                    fv[ix] = ae[e] * vda;
+                    hv[ix] = in ? re[e] * vdr - ke[e] * vdk - be[e] * vdb + fv[ix] : 0.f;
+                }
+            }
+        }
+        // stage dr, dk, db, da (bf16) in the dA tiles (read by MMA-E, done)
+        frag_to_tile(sbase + gt(G_DARK), 16 * wq, 4 * wh, ar, lane, PackB{});
+        frag_to_tile(sbase + gt(G_DAAK), 16 * wq, 4 * wh, ak, lane, PackB{});
+        frag_to_tile(sbase + gt(G_DARB), 16 * wq, 4 * wh, abv, lane, PackB{});
+        frag_to_tile(sbase + gt(G_DAAB), 16 * wq, 4 * wh, aa, lane, PackB{});
+        // exclusive prefix of h over the tokens: rows g (lanes 4 g + q) within the warp,
+        // then rows g + 8, then the quadrants before this one
+        float ex[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int i0 = 4 * j + e, i1 = 4 * j + 2 + e;
+                float s0v = hv[i0], s1v = hv[i1];
+#pragma unroll
+                for (int d = 4; d < 32; d *= 2) {
+                    const float u0 = __shfl_up_sync(0xffffffffu, s0v, d);
+                    const float u1 = __shfl_up_sync(0xffffffffu, s1v, d);
+                    if (lane >= d) {
+                        s0v += u0;
+                        s1v += u1;
+                    }
+                }
+                const float tot0 = __shfl_sync(0xffffffffu, s0v, 28 + q);
+                const float tot1 = __shfl_sync(0xffffffffu, s1v, 28 + q);
+                ex[i0] = s0v - hv[i0];
+                ex[i1] = tot0 + s1v - hv[i1];
+                if (g == 0) tot[wq * 64 + 32 * wh + 8 * j + 2 * q + e] = tot0 + tot1;
+            }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int cidx = 32 * wh + 8 * j + 2 * q + e;
+                float pre = 0.f;
+                for (int w2 = 0; w2 < wq; ++w2) pre += tot[w2 * 64 + cidx];
+                const float R = Rc[cidx];
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int ix = 4 * j + 2 * hr + e;
+                    const int t = 16 * wq + g + 8 * hr;
+                    const bool val = t < nv && (!mask || mask[crow + t] != 0);
+                    hv[ix] = val ? R - fv[ix] - (pre + ex[ix]) : 0.f;
+                }
+            }
+        frag_to_tile(sbase + gt(G_X), 16 * wq, 4 * wh, hv, lane, PackB{});  // dw
+        fence_proxy_async();
+        __syncthreads();
+        const uint32_t stg[5] = {G_DARK, G_X, G_DAAK, G_DAAB, G_DARB};  // dr dw dk da db
+        if (nv == 64) {
+            if (tid == 0) {
+                const CUtensorMap* maps[5] = {&tm_dr, &tm_dw, &tm_dk, &tm_da, &tm_db};
+#pragma unroll
+                for (int i = 0; i < 5; ++i) tma_store_3d(maps[i], sbase + gt(stg[i]), 0, cy, cz);
+                bulk_commit();
+                bulk_wait0();
+            }
+        } else {
+            // a partial chunk: rows < nv only (the rows after belong to another sequence)
+            __nv_bfloat16* outs[5] = {dr, dw, dk, da, db};
+            for (int i = tid; i < 5 * 64 * 8; i += kThreads) {
+                const int which = i / 512, rem = i % 512, t = rem >> 3, chk = rem & 7;
+                if (t >= nv) continue;
+                const long long e = kHf ? (((crow / T) * H + h) * (long long)T + (crow % T) + t) * 64
+                                        : ((crow + t) * H + h) * 64;
+                *reinterpret_cast<uint4*>(outs[which] + e + 8 * chk) =
+                    *reinterpret_cast<const uint4*>(smem + gt(stg[which]) + sw(t, chk));
+            }
+        }
+    }
+
+teardown:
+    if (timed_out) {
+        // bounded drains of what may still be in flight, then free the tensor memory
+        if (tid == 0) {
+            (void)mbar_wait(bar_tma, 0);
+            (void)mbar_wait(bar_mma, mph ^ 1u);
+            (void)mbar_wait(bar_rl, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kGTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// host
+// ---------------------------------------------------------------------------------
+template <bool kHf>
+inline cudaError_t launch_grad(const void* r, const void* w, const void* k, const void* v,
+                               const void* a, const void* b, const void* dout,
+                               const uint8_t* mask, void* dr, void* dw, void* dk, void* da,
+                               void* db, int B, int T, int H, int N, const int32_t* cu,
+                               const int32_t* cur, const void* ckF, const void* ckR,
+                               const Ws& lay, cudaStream_t stream) {
+    CUtensorMap m[14];
+    const void* ins[7] = {r, w, k, v, a, b, dout};
+    for (int i = 0; i < 7; ++i)
+        if (!make_map(&m[i], ins[i], B, T, H, kHf)) return cudaErrorInvalidValue;
+    if (!make_ck_map(&m[7], ckF, (long long)H * lay.slotsF)) return cudaErrorInvalidValue;
+    if (!make_ck_map(&m[8], ckR, (long long)H * lay.slotsR)) return cudaErrorInvalidValue;
+    void* outs[5] = {dr, dw, dk, da, db};
+    for (int i = 0; i < 5; ++i)
+        if (!make_map(&m[9 + i], outs[i], B, T, H, kHf)) return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(grad_kernel<kHf>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kGSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const dim3 grid((unsigned)lay.slotsF, (unsigned)H);
+    grad_kernel<kHf><<<grid, kThreads, kGSmemBytes, stream>>>(
+        m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], m[9], m[10], m[11], m[12], m[13],
+        mask, cu, cur, T, H, N, (int)lay.slotsF, (int)lay.slotsR,
+        static_cast<__nv_bfloat16*>(dr), static_cast<__nv_bfloat16*>(dw),
+        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(da),
+        static_cast<__nv_bfloat16*>(db));
+    return cudaGetLastError();
+}
+
+}  // namespace cbwd
+
+inline size_t bwd_chunked_workspace_bytes(long long rows, int N, int H) {
+    return cbwd::ws_layout(rows, N, H).total;
+}
+
+// The whole chunked backward (bf16, K = V = 64) on `stream`.
+inline cudaError_t launch_bwd_chunked(const void* r, const void* w, const void* k, const void* v,
+                                      const void* a, const void* b, const float* s0,
+                                      const uint8_t* mask, const void* dout, const float* dsT,
+                                      void* dr, void* dw, void* dk, void* dv, void* da, void* db,
+                                      float* ds0, int B, int T, int H, int N,
+                                      const int32_t* cu_seqlens, int head_first, void* workspace,
+                                      cudaStream_t stream) {
+    using namespace cbwd;
+    const long long rows = (long long)B * T;
+    const Ws lay = ws_layout(rows, N, H);
+    if (lay.slotsF > 0x7fffffffLL || lay.slotsR > 0x7fffffffLL || (long long)H * lay.slotsR > 0x7fffffffLL)
+        return cudaErrorInvalidValue;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* cur = reinterpret_cast<int32_t*>(ws + lay.off_cu);
+    void* ckF = ws + lay.off_ckF;
+    void* ckR = ws + lay.off_ckR;
+    __nv_bfloat16* rev = reinterpret_cast<__nv_bfloat16*>(ws + lay.off_rev);
+    const size_t rs = lay.rev_stride / 2;  // elements
+    __nv_bfloat16 *wr = rev, *ar = rev + rs, *br = rev + 2 * rs, *kr = rev + 3 * rs,
+                  *vr = rev + 4 * rs, *rr = rev + 5 * rs, *orv = rev + 6 * rs;
+    cudaError_t e;
+    // 1. reversed sequence offsets
+    prep_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, T, N, cur);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 2. forward with per-chunk checkpoints, no outputs
+    chunked::Extras exF;
+    exF.ck = ckF;
+    exF.ck_slots = (int)lay.slotsF;
+    if ((e = launch_chunked(r, w, k, v, a, b, s0, mask, nullptr, nullptr, B, T, H, N, cu_seqlens,
+                            head_first, -1, stream, exF)) != cudaSuccess)
+        return e;
+    // 3. reversed inputs
+    const dim3 rgrid((unsigned)(lay.rowsR / 64), (unsigned)H);
+    const __nv_bfloat16 *pr = static_cast<const __nv_bfloat16*>(r),
+                        *pw = static_cast<const __nv_bfloat16*>(w),
+                        *pk = static_cast<const __nv_bfloat16*>(k),
+                        *pa = static_cast<const __nv_bfloat16*>(a),
+                        *pb = static_cast<const __nv_bfloat16*>(b),
+                        *pd = static_cast<const __nv_bfloat16*>(dout);
+    if (head_first)
+        reverse_kernel<true><<<rgrid, 256, 0, stream>>>(pr, pw, pk, pa, pb, pd, mask, cu_seqlens,
+                                                        cur, T, H, N, rev, rs);
+    else
+        reverse_kernel<false><<<rgrid, 256, 0, stream>>>(pr, pw, pk, pa, pb, pd, mask, cu_seqlens,
+                                                         cur, T, H, N, rev, rs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 4. the adjoint as a forward run over the reversed sequences, from dsT
+    chunked::Extras exR;
+    exR.ck = ckR;
+    exR.ck_slots = (int)lay.slotsR;
+    if ((e = launch_chunked(rr, wr, kr, vr, ar, br, dsT, nullptr, orv, ds0, 1, (int)lay.rowsR, H,
+                            N, cur, 0, -1, stream, exR)) != cudaSuccess)
+        return e;
+    // 5. per-chunk gradients
+    e = head_first ? launch_grad<true>(r, w, k, v, a, b, dout, mask, dr, dw, dk, da, db, B, T, H,
+                                       N, cu_seqlens, cur, ckF, ckR, lay, stream)
+                   : launch_grad<false>(r, w, k, v, a, b, dout, mask, dr, dw, dk, da, db, B, T,
+                                        H, N, cu_seqlens, cur, ckF, ckR, lay, stream);
+    if (e != cudaSuccess) return e;
+    // 6. dv in token order
+    const long long nthr = rows * H * 8;
+    if (nthr > 0) {
+        const unsigned blocks = (unsigned)((nthr + 255) / 256);
+        if (head_first)
+            dv_kernel<true><<<blocks, 256, 0, stream>>>(orv, mask, cu_seqlens, cur, T, H, N, rows,
+                                                        static_cast<__nv_bfloat16*>(dv));
+        else
+            dv_kernel<false><<<blocks, 256, 0, stream>>>(orv, mask, cu_seqlens, cur, T, H, N, rows,
+                                                         static_cast<__nv_bfloat16*>(dv));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace wkv7

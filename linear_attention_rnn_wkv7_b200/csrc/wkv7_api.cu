@@ -11,6 +11,7 @@
 #include "recurrent.cuh"
 #include "chunked.cuh"
 #include "backward.cuh"
+#include "chunked_bwd.cuh"
 #include "gdn_backward.cuh"
 
 namespace {
@@ -290,7 +291,10 @@ wkv7_status wkv7_sane_step(const void* r, const void* w, const void* k, const vo
 
 size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N) {
     if (B < 0 || T < 0 || H <= 0 || N < 0 || K != 64 || V != 64) return 0;
-    return wkv7::bwd::workspace_floats((long long)B * T, N, H) * sizeof(float);
+    const long long rows = (long long)B * T;
+    const size_t rec = wkv7::bwd::workspace_floats(rows, N, H) * sizeof(float);
+    const size_t chk = wkv7::bwd_chunked_workspace_bytes(rows, N, H);
+    return rec > chk ? rec : chk;
 }
 
 wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
@@ -299,7 +303,21 @@ wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v,
                      void* db, float* ds0, int B, int T, int H, int K, int V,
                      const int32_t* cu_seqlens, int N, wkv7_layout layout, wkv7_dtype dtype,
                      void* workspace, size_t workspace_bytes, void* stream_) {
+    return wkv7_bwd_with_algo(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da, db, ds0,
+                              B, T, H, K, V, cu_seqlens, N, layout, dtype, WKV7_ALGO_AUTO,
+                              workspace, workspace_bytes, stream_);
+}
+
+wkv7_status wkv7_bwd_with_algo(const void* r, const void* w, const void* k, const void* v,
+                               const void* a, const void* b, const float* s0,
+                               const uint8_t* mask, const void* dout, const float* dsT, void* dr,
+                               void* dw, void* dk, void* dv, void* da, void* db, float* ds0,
+                               int B, int T, int H, int K, int V, const int32_t* cu_seqlens,
+                               int N, wkv7_layout layout, wkv7_dtype dtype, wkv7_algo algo,
+                               void* workspace, size_t workspace_bytes, void* stream_) {
     if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0 || N < 0) return WKV7_ERR_INVALID_ARG;
+    if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_RECURRENT && algo != WKV7_ALGO_CHUNKED)
+        return WKV7_ERR_INVALID_ARG;
     if (dtype != WKV7_BF16 && dtype != WKV7_F32) return WKV7_ERR_INVALID_ARG;
     if (layout != WKV7_LAYOUT_BTHK && layout != WKV7_LAYOUT_BHTK) return WKV7_ERR_INVALID_ARG;
     if (cu_seqlens) {
@@ -326,8 +344,15 @@ wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v,
             if (x && x == y) return WKV7_ERR_INVALID_ARG;
     if (!ok_ptr(workspace) || workspace_bytes < wkv7_bwd_workspace_bytes(B, T, H, K, V, N))
         return WKV7_ERR_INVALID_ARG;
+    if (algo == WKV7_ALGO_CHUNKED && dtype != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const int hf = layout == WKV7_LAYOUT_BHTK;
+    if (dtype == WKV7_BF16 && algo != WKV7_ALGO_RECURRENT) {
+        const cudaError_t err = wkv7::launch_bwd_chunked(r, w, k, v, a, b, s0, mask, dout, dsT,
+                                                         dr, dw, dk, dv, da, db, ds0, B, T, H, N,
+                                                         cu_seqlens, hf, workspace, stream);
+        return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+    }
     const cudaError_t err =
         dtype == WKV7_BF16
             ? wkv7::launch_bwd<__nv_bfloat16>(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk,

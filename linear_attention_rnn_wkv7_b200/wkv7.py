@@ -53,6 +53,9 @@ def library() -> ctypes.CDLL:
         lib.wkv7_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
         lib.wkv7_bwd.restype = i
         lib.wkv7_bwd.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i, i, p, ctypes.c_size_t, p]
+        lib.wkv7_bwd_with_algo.restype = i
+        lib.wkv7_bwd_with_algo.argtypes = ([p] * 17 + [i, i, i, i, i, p, i, i, i, i, p,
+                                                       ctypes.c_size_t, p])
         lib.wkv7_bwd_noalloc.restype = i
         lib.wkv7_bwd_noalloc.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i, i, p]
         lib.wkv7_gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
@@ -275,12 +278,14 @@ def wkv7_bwd_workspace_bytes(B, T, H, K=64, V=64, N=None) -> int:
 
 
 def wkv7_bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=None,
-             head_first: bool = False, workspace=None):
+             head_first: bool = False, workspace=None, algo: str = "auto"):
     """Backward of wkv7_fwd for L = sum(o * dout) + sum(S_T * dsT).  Inputs as for
     wkv7_fwd (K = V = 64); dout shaped like v; dsT [N,H,K,V] fp32 or None.
     Returns a dict: dr, dw, dk, dv, da, db (input dtype, shaped like the inputs) and
     ds0 (fp32 [N,H,K,V]).  The workspace (uint8 device tensor of at least
-    wkv7_bwd_workspace_bytes) is allocated here when not given."""
+    wkv7_bwd_workspace_bytes) is allocated here when not given.  algo: "auto" (the
+    tensor-core chunked form for bf16, the fp32 recurrences for fp32), "chunked"
+    (bf16 only) or "recurrent"."""
     _check(r, "r")
     dt = r.dtype
     if head_first:
@@ -315,12 +320,12 @@ def wkv7_bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=No
     g = {n: torch.empty(kshape, dtype=dt, device=r.device) for n in ("dr", "dw", "dk", "da", "db")}
     g["dv"] = torch.empty(vshape, dtype=dt, device=r.device)
     g["ds0"] = torch.empty((N, H, K, V), dtype=torch.float32, device=r.device)
-    st = library().wkv7_bwd(_ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0),
-                            _ptr(mask), _ptr(dout), _ptr(dsT), _ptr(g["dr"]), _ptr(g["dw"]),
-                            _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["db"]),
-                            _ptr(g["ds0"]), B, T, H, K, V, _ptr(cu_seqlens), N,
-                            int(bool(head_first)), _dtype_code(r), _ptr(workspace),
-                            workspace.numel(), _stream(r.device))
+    st = library().wkv7_bwd_with_algo(
+        _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0), _ptr(mask), _ptr(dout),
+        _ptr(dsT), _ptr(g["dr"]), _ptr(g["dw"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]),
+        _ptr(g["db"]), _ptr(g["ds0"]), B, T, H, K, V, _ptr(cu_seqlens), N,
+        int(bool(head_first)), _dtype_code(r), ALGO[algo], _ptr(workspace), workspace.numel(),
+        _stream(r.device))
     if st != OK:
         raise WKV7Error(st, "wkv7_bwd")
     return g
