@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------------
-// 3. reverse: one CTA per (reversed 64-row chunk, head); thread = (row, 16 channels).
+// 3. reverse: one CTA per (reversed 64-row chunk, head); thread = 16 bytes of two rows
+//    (rows i and i + 32); the six loads of a row are issued before its six stores.
 // ---------------------------------------------------------------------------------
 template <bool kHf>
 __global__ void __launch_bounds__(256) reverse_kernel(
@@ -161,31 +162,37 @@ __global__ void __launch_bounds__(256) reverse_kernel(
     seq_of(n, T, cu, row0, L, ok);
     if (!ok) L = 0;  // flagged by prep; the reversed sequence is all identity
     const int p = 63 - (L & 63);
-    const int row = threadIdx.x >> 2, qq = threadIdx.x & 3;
-    const long long tp = grow0 + row - cur[n];  // tau' within the reversed sequence
-    const int tau = (int)tp - p;
-    const int t1 = L - tau;      // transition token (tau >= 1)
-    const int t2 = L - 1 - tau;  // input token (tau < L)
-    const bool has1 = tau >= 1 && tau <= L && (!mask || mask[row0 + t1] != 0);
-    const bool has2 = tau >= 0 && tau < L;
-    auto src = [&](const __nv_bfloat16* x, int t) -> const uint4* {
-        const long long e = kHf ? (((row0 / T) * H + h) * (long long)T + (row0 % T) + t) * 64
-                                : ((row0 + t) * H + h) * 64;
-        return reinterpret_cast<const uint4*>(x + e) + 2 * qq;
-    };
-    const size_t dst = ((size_t)(grow0 + row) * H + h) * 64;
-    uint4* out = reinterpret_cast<uint4*>(rev + dst) + 2 * qq;
-    const size_t str = rev_stride_elems / 8;  // in uint4
+    const int piece = threadIdx.x & 7;
+    // element offset of token t of the sequence (head h) in the inputs
+    const long long base = kHf ? (((row0 / T) * H + h) * (long long)T + (row0 % T)) * 64
+                               : (row0 * H + h) * 64;
+    const long long tstride = kHf ? 64 : (long long)H * 64;
+    const size_t str = rev_stride_elems / 8;  // tensors apart, in uint4
     const uint4 z = make_uint4(0, 0, 0, 0);
-    // w' a' b' k' v' r' = w[t1] b[t1] a[t1] r[t2] do[t2] k[t2]
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        out[0 * str + i] = has1 ? src(w, t1)[i] : z;
-        out[1 * str + i] = has1 ? src(b, t1)[i] : z;
-        out[2 * str + i] = has1 ? src(a, t1)[i] : z;
-        out[3 * str + i] = has2 ? src(r, t2)[i] : z;
-        out[4 * str + i] = has2 ? src(dout, t2)[i] : z;
-        out[5 * str + i] = has2 ? src(k, t2)[i] : z;
+    for (int half = 0; half < 2; ++half) {
+        const int row = (threadIdx.x >> 3) + 32 * half;
+        const long long tp = grow0 + row - cur[n];  // tau' within the reversed sequence
+        const int tau = (int)tp - p;
+        const int t1 = L - tau;      // transition token (tau >= 1)
+        const int t2 = L - 1 - tau;  // input token (tau < L)
+        const bool in1 = tau >= 1 && tau <= L, in2 = tau >= 0 && tau < L;
+        const bool has1 = in1 && (!mask || mask[row0 + t1] != 0);
+        uint4 x[6] = {z, z, z, z, z, z};
+        if (L > 0) {
+            const int c1 = min(max(t1, 0), L - 1), c2 = min(max(t2, 0), L - 1);
+            const long long e1 = base + c1 * tstride, e2 = base + c2 * tstride;
+            x[0] = __ldg(reinterpret_cast<const uint4*>(w + e1) + piece);
+            x[1] = __ldg(reinterpret_cast<const uint4*>(b + e1) + piece);
+            x[2] = __ldg(reinterpret_cast<const uint4*>(a + e1) + piece);
+            x[3] = __ldg(reinterpret_cast<const uint4*>(r + e2) + piece);
+            x[4] = __ldg(reinterpret_cast<const uint4*>(dout + e2) + piece);
+            x[5] = __ldg(reinterpret_cast<const uint4*>(k + e2) + piece);
+        }
+        // w' a' b' k' v' r' = w[t1] b[t1] a[t1] r[t2] do[t2] k[t2]
+        uint4* out = reinterpret_cast<uint4*>(rev + ((size_t)(grow0 + row) * H + h) * 64) + piece;
+#pragma unroll
+        for (int i = 0; i < 6; ++i) out[i * str] = (i < 3 ? has1 : in2) ? x[i] : z;
     }
 }
 
@@ -260,13 +267,15 @@ constexpr uint32_t GOFF_R = GOFF_GAMMA + 256;        // R per channel (64 fp32)
 constexpr uint32_t GOFF_EM0 = GOFF_R + 256;          // E_{-1} per channel (64 fp32)
 constexpr uint32_t GOFF_RAW = GOFF_EM0 + 256;        // raw r and dO of token 63 (2 x 64 fp32)
 constexpr uint32_t GOFF_TOT = GOFF_RAW + 512;        // scan totals [4 quadrants][64]
-constexpr uint32_t kGSmemBytes = GOFF_TOT + 1024;
+constexpr uint32_t GOFF_NEXT = GOFF_TOT + 1024;      // the CTA's next work item (and index)
+constexpr uint32_t kGSmemBytes = GOFF_NEXT + 128;
 static_assert(kGSmemBytes <= 232448, "fits one CTA per SM");
 constexpr uint32_t kGTmemCols = 512;
-// TMEM columns (every accumulator M = 64): C0..C2 rotate through the phases' products;
-// dRbar, dAbar (phase C), acc_k, acc_b (D), acc_r (E, over C2) and acc_a (E) stay to the end.
+// TMEM columns (every accumulator M = 64): C0..C2 hold each phase's products for its
+// epilogue; dRbar, dAbar, acc_k, acc_b and P have their own columns; acc_r and acc_a
+// take C2 and C1 once phase C's epilogue has read them.
 constexpr uint32_t C0 = 0, C1 = 64, C2 = 128, C_DRB = 192, C_DAB = 256, C_AK = 320, C_AB = 384,
-                   C_AR = 128, C_AA = 448;
+                   C_P = 448, C_AR = 128, C_AA = 64;
 
 // E tile index (fp32 [t][c], groups of 8 channels XOR-swizzled by row).
 __device__ __forceinline__ int eidx(int t, int c) { return t * 64 + (c ^ ((t & 7) << 3)); }
@@ -306,6 +315,49 @@ __device__ __forceinline__ void mma64(uint32_t tmem_d, uint32_t a, bool a_mn, ui
     }
 }
 
+// Work item `it` (slot fastest, then head) -> the chunk: sequence n with
+// floor(row0_n / 64) + n <= slot, its chunk c; false for a slot that no chunk maps to.
+struct Item {
+    int n, c, h, L, nv, slot, rslot;
+    long long row0, crow;
+};
+__device__ __forceinline__ bool item_of(int it, int slotsF, int T, int N, const int32_t* cu,
+                                        Item& I) {
+    I.h = it / slotsF;
+    I.slot = it - I.h * slotsF;
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const long long r0 = cu ? (long long)cu[mid] : (long long)mid * T;
+        if ((r0 >> 6) + mid <= I.slot) lo = mid; else hi = mid - 1;
+    }
+    I.n = lo;
+    bool ok;
+    seq_of(I.n, T, cu, I.row0, I.L, ok);
+    if (!ok) return false;  // flagged by prep
+    I.c = I.slot - (int)((I.row0 >> 6) + I.n);
+    if (I.c < 0 || 64 * I.c >= I.L) return false;
+    I.nv = min(64, I.L - 64 * I.c);
+    I.crow = I.row0 + 64LL * I.c;
+    return true;
+}
+// The first item with a chunk among it, it + gridDim.x, ..., or -1; with the slot of its
+// state-gradient checkpoint (reversed sequence n starts at cur[n]).
+__device__ __forceinline__ int next_item(int it, int total, int slotsF, int T, int N,
+                                         const int32_t* cu, const int32_t* cur, Item& I) {
+    for (; it < total; it += gridDim.x)
+        if (item_of(it, slotsF, T, N, cu, I)) {
+            // reversed sequences are 64 (floor(L / 64) + 1) rows each: closed form for
+            // equal lengths
+            const int c0r = cu ? cur[I.n] / 64 : I.n * (T / 64 + 1);
+            I.rslot = c0r + I.n + I.L / 64 - I.c;
+            return it;
+        }
+    return -1;
+}
+
+// Persistent: CTA b takes work items b, b + gridDim.x, ... (one CTA per SM); each
+// chunk's nine input tiles are loaded while the previous chunk's final epilogue runs.
 template <bool kHf>
 __global__ void __launch_bounds__(kThreads, 1)
 grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
@@ -324,26 +376,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wq = warp & 3, wh = warp >> 2;
     const int g = lane >> 2, q = lane & 3;
-    const int slot = blockIdx.x, h = blockIdx.y;
-
-    // The chunk of this slot: sequence n with floor(row0_n / 64) + n <= slot, chunk c.
-    int lo = 0, hi = N - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        const long long r0 = cu ? (long long)cu[mid] : (long long)mid * T;
-        if ((r0 >> 6) + mid <= slot) lo = mid; else hi = mid - 1;
-    }
-    const int n = lo;
-    long long row0;
-    int L;
-    bool ok;
-    seq_of(n, T, cu, row0, L, ok);
-    if (!ok) return;  // flagged by prep
-    const int c = slot - (int)((row0 >> 6) + n);
-    if (c < 0 || 64 * c >= L) return;
-    const int nv = min(64, L - 64 * c);
-    const long long crow = row0 + 64LL * c;  // first token row of the chunk
-    const int rslot = cur[n] / 64 + n + L / 64 - c;
+    const int total = slotsF * H;  // below 2^31 (checked on the host)
 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_tma = sbase + GOFF_MISC, bar_mma = sbase + GOFF_MISC + 8,
@@ -356,7 +389,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     float* Ef = reinterpret_cast<float*>(smem + gt(G_E));
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GOFF_MISC + 32);
     int timed_out = 0;
-    uint32_t mph = 0;
+    uint32_t mph = 0, tph = 0, rph = 0;
+
+    Item I, In;
+    int it = next_item(blockIdx.x, total, slotsF, T, N, cu, cur, I);
+    if (it < 0) return;
 
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), kGTmemCols);
@@ -372,28 +409,43 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (warp == 1 && lane < 14) {
+        const CUtensorMap* maps[14] = {&tm_r, &tm_w, &tm_k, &tm_v, &tm_a, &tm_b, &tm_do,
+                                       &tm_ckf, &tm_ckr, &tm_dr, &tm_dw, &tm_dk, &tm_da, &tm_db};
+        prefetch_tensormap(maps[lane]);
+    }
 
-    // token-major maps: (channel, head, token row); head first: (channel, token, b*H + h)
-    const int cy = kHf ? (int)(crow % T) : h;
-    const int cz = kHf ? (int)((crow / T) * H + h) : (int)crow;
+    // Input tile i (0..8) of item J: r, a, k, b, w, v, dO by the input maps (token-major:
+    // (channel, head, token row); head first: (channel, token, b*H + h)), S0 and G from
+    // the two checkpoint arrays.  Each TMA instruction takes a few hundred cycles to
+    // issue, so the nine are spread over the warps.
+    auto load_in = [&](const Item& J, int i) {
+        const int jy = kHf ? (int)(J.crow % T) : J.h;
+        const int jz = kHf ? (int)((J.crow / T) * H + J.h) : (int)J.crow;
+        const CUtensorMap* map = i == 0 ? &tm_r : i == 1 ? &tm_a : i == 2 ? &tm_k
+                               : i == 3 ? &tm_b : i == 4 ? &tm_w : i == 5 ? &tm_v
+                               : i == 6 ? &tm_do : i == 7 ? &tm_ckf : &tm_ckr;
+        const uint32_t dst = i == 0 ? G_R : i == 1 ? G_A : i == 2 ? G_K : i == 3 ? G_B
+                           : i == 4 ? G_W : i == 5 ? G_V : i == 6 ? G_DO : i == 7 ? G_S0 : G_DS;
+        if (i < 7)
+            tma_load_3d(sbase + gt(dst), map, bar_tma, 0, jy, jz);
+        else
+            tma_load_3d(sbase + gt(dst), map, bar_tma, 0, 0,
+                        i == 7 ? J.h * slotsF + J.slot : J.h * slotsR + J.rslot);
+    };
     if (warp == 0) {
         if (lane == 0) mbar_arrive_expect_tx(bar_tma, 9 * kTile);
         __syncwarp();
-        if (lane < 9) {
-            const CUtensorMap* map = lane == 0 ? &tm_r : lane == 1 ? &tm_a : lane == 2 ? &tm_k
-                                   : lane == 3 ? &tm_b : lane == 4 ? &tm_w : lane == 5 ? &tm_v
-                                   : lane == 6 ? &tm_do : lane == 7 ? &tm_ckf : &tm_ckr;
-            const uint32_t dst = lane == 0 ? G_R : lane == 1 ? G_A : lane == 2 ? G_K
-                               : lane == 3 ? G_B : lane == 4 ? G_W : lane == 5 ? G_V
-                               : lane == 6 ? G_DO : lane == 7 ? G_S0 : G_DS;
-            if (lane < 7)
-                tma_load_3d(sbase + gt(dst), map, bar_tma, 0, cy, cz);
-            else
-                tma_load_3d(sbase + gt(dst), map, bar_tma, 0, 0,
-                            lane == 7 ? h * slotsF + slot : h * slotsR + rslot);
-        }
+        if (lane < 9) load_in(I, lane);
     }
-    wait_or_abort(bar_tma, 0, timed_out);
+
+    while (it >= 0) {
+    const int h = I.h, nv = I.nv;
+    const long long crow = I.crow;
+    const int cy = kHf ? (int)(crow % T) : h;
+    const int cz = kHf ? (int)((crow / T) * H + h) : (int)crow;
+    wait_or_abort(bar_tma, tph, timed_out);
+    tph ^= 1;
 
     // ---- prologue: prefix sums of w (mask folded), E, and the operands --------------
     {
@@ -473,7 +525,6 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
 #pragma unroll
             for (int e = 0; e < 8; ++e) em0[8 * j + e] = Ep[e];
         }
-        __syncthreads();  // every thread has read the scan scratch (the SP tile)
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
             const uint32_t off = it ? offb : offa;
@@ -630,13 +681,32 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         acc_to_tile(tmem, C2, sbase + gt(G_ARB), wq, 0, lane, 1, PackH{});
         acc_to_tile(tmem, C2, sbase + gt(G_ARB), wq, 1, lane, 1, PackH{});
     }
+    // the previous chunk's output stores have read the staging tiles before phase A's
+    // epilogue writes them
+    if (lane == 0 && warp < 5) bulk_wait_read0();
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
 
-    // ---- T = (I - A_ab)^-1 by block forward substitution (warp-level fp16 MMAs):
-    //      warps 0..5 form T_ii A_im (m < i); warp w < 4 then builds column block w:
-    //      X_w = T_ww, X_i = sum_{w<=m<i} (T_ii A_im) X_m. ------------------------------
-    {
+    // ---- A: X = Abar S0 + A_ak V;  dU = A_rb^T dO + Bhat dSL;  dA_rk = dO V^T ---------
+    if (tid == 0) {
+        tc_fence_after();
+        mma64(tmem + C0, sbase + gt(G_W), false, sbase + gt(G_S0), true, false, false);
+        mma64(tmem + C0, sbase + gt(G_AAK), false, sbase + gt(G_V), true, false, true);
+        mma64(tmem + C1, sbase + gt(G_ARB), true, sbase + gt(G_DO), true, false, false);
+        mma64(tmem + C1, sbase + gt(G_BH), false, sbase + gt(G_DS), true, false, true);
+        mma64(tmem + C2, sbase + gt(G_DO), false, sbase + gt(G_V), false, false, false);
+        umma_commit(bar_mma);
+        // background (read after later commits): dRbar = dO S0^T, acc_k = V dSL^T,
+        // P = Rbar^T dO
+        mma64(tmem + C_DRB, sbase + gt(G_DO), false, sbase + gt(G_S0), false, false, false);
+        mma64(tmem + C_AK, sbase + gt(G_V), false, sbase + gt(G_DS), false, false, false);
+        mma64(tmem + C_P, sbase + gt(G_RB), true, sbase + gt(G_DO), true, false, false);
+    }
+    // ---- T = (I - A_ab)^-1 by block forward substitution (warp-level fp16 MMAs) on
+    //      warps 0..3: the six products T_ii A_im (m < i), then warp w builds column
+    //      block w: X_w = T_ww, X_i = sum_{w<=m<i} (T_ii A_im) X_m.  Meanwhile warps
+    //      4..7 store phase A's products (issued above; they do not need T). ---------
+    if (warp < 4) {
         uint8_t* Tb = smem + gt(G_SP) + kDiagBytes;
         uint8_t* Tab = smem + gt(G_DT);
         const int lr = (lane & 7) + 8 * ((lane >> 3) & 1), lc = 8 * (lane >> 4);
@@ -644,9 +714,12 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         auto a_frag = [&](const uint8_t* blk, uint32_t (&af)[4]) {
             ldsm_x4(smem_u32(blk) + a_lane, af[0], af[1], af[2], af[3]);
         };
-        if (warp < 6) {
-            const int i = warp < 1 ? 1 : (warp < 3 ? 2 : 3);
-            const int m = warp < 1 ? 0 : (warp < 3 ? warp - 1 : warp - 3);
+#pragma unroll
+        for (int rep = 0; rep < 2; ++rep) {
+            const int blk = warp + 4 * rep;
+            if (blk >= 6) break;
+            const int i = blk < 1 ? 1 : (blk < 3 ? 2 : 3);
+            const int m = blk < 1 ? 0 : (blk < 3 ? blk - 1 : blk - 3);
             uint32_t af[4];
             a_frag(Tb + i * 768, af);
             float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -655,15 +728,15 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                       bfa[0], bfa[1], bfa[2], bfa[3]);
             mma_f16_16816(z[0], af[0], af[1], af[2], af[3], bfa[0], bfa[1]);
             mma_f16_16816(z[1], af[0], af[1], af[2], af[3], bfa[2], bfa[3]);
-            uint8_t* dst = Tab + warp * 768;  // blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+            uint8_t* dst = Tab + blk * 768;  // blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 *reinterpret_cast<uint32_t*>(dst + g * 48 + 2 * (8 * nt + 2 * q)) = pack2h(z[nt][0], z[nt][1]);
                 *reinterpret_cast<uint32_t*>(dst + (g + 8) * 48 + 2 * (8 * nt + 2 * q)) = pack2h(z[nt][2], z[nt][3]);
             }
         }
-        __syncthreads();
-        if (warp < 4) {
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // warps 0..3: T_ii A_im visible
+        {
             const int wcol = warp;  // column block of T
             uint8_t* tt = smem + gt(G_T);
             uint32_t xb[3][4];
@@ -707,42 +780,27 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                 }
             }
         }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-    }
-
-    // ---- A: X = Abar S0 + A_ak V;  dU = A_rb^T dO + Bhat dSL;  dA_rk = dO V^T ---------
-    if (tid == 0) {
+    } else {
+        wait_or_abort(bar_mma, mph, timed_out);
         tc_fence_after();
-        mma64(tmem + C0, sbase + gt(G_W), false, sbase + gt(G_S0), true, false, false);
-        mma64(tmem + C0, sbase + gt(G_AAK), false, sbase + gt(G_V), true, false, true);
-        mma64(tmem + C1, sbase + gt(G_ARB), true, sbase + gt(G_DO), true, false, false);
-        mma64(tmem + C1, sbase + gt(G_BH), false, sbase + gt(G_DS), true, false, true);
-        mma64(tmem + C2, sbase + gt(G_DO), false, sbase + gt(G_V), false, false, false);
-        umma_commit(bar_mma);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            acc_to_tile(tmem, C0, sbase + gt(G_X), wq, hh, lane, 0, PackH{});
+            acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, hh, lane, 0, PackH{});
+            acc_to_tile(tmem, C2, sbase + gt(G_DARK), wq, hh, lane, 1, PackB{});
+        }
     }
-    wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
-    tc_fence_after();
-    // The original r, k, a, b again (for dw), into tiles that are dead now.
-    if (tid == 32) {
-        mbar_arrive_expect_tx(bar_rl, 4 * kTile);
-        tma_load_3d(sbase + gt(G_SP), &tm_r, bar_rl, 0, cy, cz);
-        tma_load_3d(sbase + gt(G_AB), &tm_k, bar_rl, 0, cy, cz);
-        tma_load_3d(sbase + gt(G_AAK), &tm_a, bar_rl, 0, cy, cz);
-        tma_load_3d(sbase + gt(G_ARB), &tm_b, bar_rl, 0, cy, cz);
-    }
-    acc_to_tile(tmem, C0, sbase + gt(G_X), wq, wh, lane, 0, PackH{});
-    acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, wh, lane, 0, PackH{});
-    acc_to_tile(tmem, C2, sbase + gt(G_DARK), wq, wh, lane, 1, PackB{});
     fence_proxy_async();
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
 
     // ---- B: U = T X;  dX = T^T dU;  dT = dU X^T ------------------------------------
+    //      (and the original r, k, a, b again, for dw, into tiles that are dead now:
+    //      armed here, issued by warps 4..7 below)
     if (tid == 0) {
         tc_fence_after();
+        mbar_arrive_expect_tx(bar_rl, 4 * kTile);
         mma64(tmem + C0, sbase + gt(G_T), false, sbase + gt(G_X), true, false, false);
         mma64(tmem + C1, sbase + gt(G_T), true, sbase + gt(G_DU), true, false, false);
         mma64(tmem + C2, sbase + gt(G_DU), false, sbase + gt(G_X), false, false, false);
@@ -751,6 +809,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
     tc_fence_after();
+    if (warp >= 4 && lane == 0) {
+        const int i = warp - 4;
+        tma_load_3d(sbase + gt(i == 0 ? G_SP : i == 1 ? G_AB : i == 2 ? G_AAK : G_ARB),
+                    i == 0 ? &tm_r : i == 1 ? &tm_k : i == 2 ? &tm_a : &tm_b, bar_rl, 0, cy, cz);
+    }
     acc_to_tile(tmem, C0, sbase + gt(G_X), wq, wh, lane, 0, PackH{});   // U
     acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, wh, lane, 0, PackH{});  // dX
     acc_to_tile(tmem, C2, sbase + gt(G_DT), wq, wh, lane, 0, PackH{});  // dT
@@ -758,15 +821,17 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
 
-    // ---- C: dA_rb = dO U^T; dA_ak = dX V^T; Y = dT T^T; dRbar = dO S0^T; dAbar = dX S0^T
+    // ---- C: dA_rb = dO U^T; dA_ak = dX V^T; Y = dT T^T;
+    //      background: dAbar = dX S0^T, acc_b = U dSL^T, P += Abar^T dX
     if (tid == 0) {
         tc_fence_after();
         mma64(tmem + C0, sbase + gt(G_DO), false, sbase + gt(G_X), false, false, false);
         mma64(tmem + C1, sbase + gt(G_DU), false, sbase + gt(G_V), false, false, false);
         mma64(tmem + C2, sbase + gt(G_DT), false, sbase + gt(G_T), false, false, false);
-        mma64(tmem + C_DRB, sbase + gt(G_DO), false, sbase + gt(G_S0), false, false, false);
-        mma64(tmem + C_DAB, sbase + gt(G_DU), false, sbase + gt(G_S0), false, false, false);
         umma_commit(bar_mma);
+        mma64(tmem + C_DAB, sbase + gt(G_DU), false, sbase + gt(G_S0), false, false, false);
+        mma64(tmem + C_AB, sbase + gt(G_X), false, sbase + gt(G_DS), false, false, false);
+        mma64(tmem + C_P, sbase + gt(G_W), true, sbase + gt(G_DU), true, false, true);
     }
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
@@ -778,15 +843,27 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
 
-    // ---- D: dA_ab = T^T Y; P = Rbar^T dO + Abar^T dX; acc_k = V dSL^T; acc_b = U dSL^T
+    // ---- D: dA_ab = T^T Y (the commit also covers P, finished in the background of C);
+    //      background: every gradient-accumulator term that does not need dA_ab
+    //      (bf16 against the Gram operands)
     if (tid == 0) {
         tc_fence_after();
         mma64(tmem + C0, sbase + gt(G_T), true, sbase + gt(G_DT), true, false, false);
-        mma64(tmem + C1, sbase + gt(G_RB), true, sbase + gt(G_DO), true, false, false);
-        mma64(tmem + C1, sbase + gt(G_W), true, sbase + gt(G_DU), true, false, true);
-        mma64(tmem + C_AK, sbase + gt(G_V), false, sbase + gt(G_DS), false, false, false);
-        mma64(tmem + C_AB, sbase + gt(G_X), false, sbase + gt(G_DS), false, false, false);
         umma_commit(bar_mma);
+        mma64(tmem + C_AR, sbase + gt(G_DARK), false, sbase + gt(G_K), true, true, false);
+        mma64(tmem + C_AR, sbase + gt(G_DARB), false, sbase + gt(G_B), true, true, true);
+        mma64(tmem + C_AA, sbase + gt(G_DAAK), false, sbase + gt(G_K), true, true, false);
+        mma64(tmem + C_AK, sbase + gt(G_DARK), true, sbase + gt(G_R), true, true, true);
+        mma64(tmem + C_AK, sbase + gt(G_DAAK), true, sbase + gt(G_A), true, true, true);
+        mma64(tmem + C_AB, sbase + gt(G_DARB), true, sbase + gt(G_R), true, true, true);
+    }
+    if (warp == 4) {  // the next chunk of this CTA: shared, and its load barrier armed
+        const int itn = next_item(it + gridDim.x, total, slotsF, T, N, cu, cur, In);
+        if (lane == 0) {
+            *reinterpret_cast<Item*>(smem + GOFF_NEXT) = In;
+            *reinterpret_cast<int*>(smem + GOFF_NEXT + 64) = itn;
+            if (itn >= 0) mbar_arrive_expect_tx(bar_tma, 9 * kTile);
+        }
     }
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
@@ -794,7 +871,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     acc_to_tile(tmem, C0, sbase + gt(G_DAAB), wq, wh, lane, 2, PackB{});
     {  // R += rowsum(S0 * P) over this warp's 32 columns
         float v[16];
-        tmem_frag(tmem + C1, wq, 32 * wh, v);
+        tmem_frag(tmem + C_P, wq, 32 * wh, v);
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int row = 16 * wq + g + 8 * hr;
@@ -814,33 +891,42 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
 
-    // ---- E: the four gradient accumulators (bf16 against the Gram operands) ----------
+    // ---- E: the dA_ab terms of acc_a and acc_b ---------------------------------------
     if (tid == 0) {
         tc_fence_after();
-        mma64(tmem + C_AR, sbase + gt(G_DARK), false, sbase + gt(G_K), true, true, false);
-        mma64(tmem + C_AR, sbase + gt(G_DARB), false, sbase + gt(G_B), true, true, true);
-        mma64(tmem + C_AA, sbase + gt(G_DAAK), false, sbase + gt(G_K), true, true, false);
         mma64(tmem + C_AA, sbase + gt(G_DAAB), false, sbase + gt(G_B), true, true, true);
-        mma64(tmem + C_AK, sbase + gt(G_DARK), true, sbase + gt(G_R), true, true, true);
-        mma64(tmem + C_AK, sbase + gt(G_DAAK), true, sbase + gt(G_A), true, true, true);
-        mma64(tmem + C_AB, sbase + gt(G_DARB), true, sbase + gt(G_R), true, true, true);
         mma64(tmem + C_AB, sbase + gt(G_DAAB), true, sbase + gt(G_A), true, true, true);
         umma_commit(bar_mma);
     }
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
     tc_fence_after();
-    wait_or_abort(bar_rl, 0, timed_out);
+    // Every input tile is dead now: the next chunk's loads (one per warp, warp 0 two)
+    // overlap the final epilogue.
+    it = *reinterpret_cast<const volatile int*>(smem + GOFF_NEXT + 64);
+    if (it >= 0) {
+        I = *reinterpret_cast<const Item*>(smem + GOFF_NEXT);
+        if (lane == 0) {
+            load_in(I, warp);
+            if (warp == 0) load_in(I, 8);
+        }
+    }
+    wait_or_abort(bar_rl, rph, timed_out);
+    rph ^= 1;
 
     // ---- final epilogue: dr, da, dk, db, and dw by an exclusive prefix over tokens ----
     {
         float ar[16], aa[16], ak[16], abv[16], drb[16], dab[16];
-        tmem_frag(tmem + C_AR, wq, 32 * wh, ar);
-        tmem_frag(tmem + C_AA, wq, 32 * wh, aa);
-        tmem_frag(tmem + C_AK, wq, 32 * wh, ak);
-        tmem_frag(tmem + C_AB, wq, 32 * wh, abv);
-        tmem_frag(tmem + C_DRB, wq, 32 * wh, drb);
-        tmem_frag(tmem + C_DAB, wq, 32 * wh, dab);
+        {
+            const uint32_t ta = tmem + ((uint32_t)(32 * wq) << 16) + 32 * wh;
+            tmem_ld16x32(ta + C_AR, ar);
+            tmem_ld16x32(ta + C_AA, aa);
+            tmem_ld16x32(ta + C_AK, ak);
+            tmem_ld16x32(ta + C_AB, abv);
+            tmem_ld16x32(ta + C_DRB, drb);
+            tmem_ld16x32(ta + C_DAB, dab);
+            tmem_ld_wait();
+        }
         float hv[16], fv[16];
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
@@ -866,8 +952,8 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                     const int ix = 4 * j + 2 * hr + e;
                     const float gm = gam[cidx + e];
                     const float vdr = in ? fmaf(Ee[e], ar[ix], (Ee[e] * gm) * drb[ix]) : 0.f;
-                    const float vdk = val ? ak[ix] / Ee[e] : 0.f;
-                    const float vdb = val ? abv[ix] / Ee[e] : 0.f;
+                    const float vdk = val ? __fdividef(ak[ix], Ee[e]) : 0.f;
+                    const float vdb = val ? __fdividef(abv[ix], Ee[e]) : 0.f;
                     const float vda = val ? fmaf(Eme[e], aa[ix], (Eme[e] * gm) * dab[ix]) : 0.f;
                     ar[ix] = vdr;
                     ak[ix] = vdk;
@@ -929,12 +1015,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         __syncthreads();
         const uint32_t stg[5] = {G_DARK, G_X, G_DAAK, G_DAAB, G_DARB};  // dr dw dk da db
         if (nv == 64) {
-            if (tid == 0) {
-                const CUtensorMap* maps[5] = {&tm_dr, &tm_dw, &tm_dk, &tm_da, &tm_db};
-#pragma unroll
-                for (int i = 0; i < 5; ++i) tma_store_3d(maps[i], sbase + gt(stg[i]), 0, cy, cz);
+            if (lane == 0 && warp < 5) {  // one tile store per warp
+                const CUtensorMap* map = warp == 0 ? &tm_dr : warp == 1 ? &tm_dw : warp == 2 ? &tm_dk
+                                       : warp == 3 ? &tm_da : &tm_db;
+                tma_store_3d(map, sbase + gt(stg[warp]), 0, cy, cz);
                 bulk_commit();
-                bulk_wait0();
             }
         } else {
             // a partial chunk: rows < nv only (the rows after belong to another sequence)
@@ -950,14 +1035,18 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         }
     }
 
+    }  // chunks
+    if (lane == 0 && warp < 5) bulk_wait0();  // the last output stores are complete
+
 teardown:
     if (timed_out) {
         // bounded drains of what may still be in flight, then free the tensor memory
         if (tid == 0) {
-            (void)mbar_wait(bar_tma, 0);
+            (void)mbar_wait(bar_tma, tph);
             (void)mbar_wait(bar_mma, mph ^ 1u);
-            (void)mbar_wait(bar_rl, 0);
+            (void)mbar_wait(bar_rl, rph);
         }
+        if (lane == 0 && warp < 5) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
@@ -994,7 +1083,13 @@ inline cudaError_t launch_grad(const void* r, const void* w, const void* k, cons
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const dim3 grid((unsigned)lay.slotsF, (unsigned)H);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaErrorInvalidValue;
+    const long long items = lay.slotsF * H;
+    if (items > 0x7fffffffLL - 4096) return cudaErrorInvalidValue;  // item + grid stays an int
+    const unsigned grid = (unsigned)(items < sms ? items : sms);
     grad_kernel<kHf><<<grid, kThreads, kGSmemBytes, stream>>>(
         m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], m[9], m[10], m[11], m[12], m[13],
         mask, cu, cur, T, H, N, (int)lay.slotsF, (int)lay.slotsR,
