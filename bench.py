@@ -547,12 +547,12 @@ def bwd_leg(args, device, stream, bwd_fn, hbm_peak, peak_kind, max_over_ranks, b
             "ms_per_step": ms,
             "tokens/s": B * T / (ms / 1e3), "algorithmic_bytes_per_step": nbytes, "GB/s": gbs,
             "peak": hbm_peak, "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} burst copy",
-            "workspace_bytes": ws.numel(), "gpu_launches": (4 if gdn else 6) * steps,
+            "workspace_bytes": ws.numel(), "gpu_launches": 4 * steps,
             "kernels": ("gdn_map_kernel + ckpt_kernel (forward, checkpoints) + bwd_kernel "
                         "(reverse) + gdn_chain_kernel" if gdn else
                         "prep_kernel + chunked_kernel (forward, state checkpoints) + "
-                        "reverse_kernel + chunked_kernel (state gradient, reversed) + "
-                        "grad_kernel (per-chunk gradients) + dv_kernel")}
+                        "chunked_kernel (state gradient over the reversed sequences, dv) + "
+                        "grad_kernel (per-chunk gradients)")}
 
 
 def wkv7_bwd_workspace_nbytes(B, T, H):

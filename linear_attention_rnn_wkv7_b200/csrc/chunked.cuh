@@ -284,6 +284,19 @@ __device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, int
     }
 }
 
+// The reversed run (kRev) of the backward's state gradient reads the original tensors
+// itself: reversed sequence n is p = 63 - L % 64 identity steps, then step tau = 0..L with
+// transition w, b, a of token L - tau (tau >= 1; identity for a masked token) and write
+// pair r, dO of token L - 1 - tau (tau < L); its read vector is k of token L - 1 - tau,
+// so the outputs are dv of that token (zero for a masked token), written in place.
+struct RevIn {
+    const __nv_bfloat16 *w, *a, *b, *r, *dout, *k;  // original tensors
+    const uint8_t* mask;                             // [B, T] or nullptr
+    const int32_t* cu;                               // original cu_seqlens or nullptr
+    int T, hf;                                       // original T and layout
+    __nv_bfloat16* dv;                               // dv, the original layout
+};
+
 // Everything one CTA keeps for its (sequence, head) between chunks.
 struct Ctx {
     uint8_t* smem;
@@ -312,6 +325,11 @@ struct Ctx {
     const CUtensorMap* tm_ck;
     bool ck;
     int ck_z0;
+    // kRev: the original sequence (length, padding, first token's element offset and
+    // token stride in the inputs, row in the mask, and its dv tile coordinates)
+    const RevIn* ri;
+    int rv_L, rv_p, rv_y0, rv_z0;
+    long long rv_base, rv_ts, rv_row0;
     const __nv_bfloat16 *g, *beta;  // Gated DeltaNet only: [rows, H]
 };
 
@@ -345,10 +363,41 @@ __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
     }
 }
 
+// kRev, every thread: 12 of the chunk's 6 x 64 x 8 16-byte pieces by cp.async, each
+// from its original token (zero-filled where the step has no transition or no write),
+// then the mbarrier tracks this thread's copies (one plain arrive after the next CTA
+// barrier completes the count).
+__device__ __forceinline__ void issue_loads_rev(const Ctx& cx, int c0, int par) {
+    const LayR L = lay_of(par);
+    const RevIn& ri = *cx.ri;
+#pragma unroll 2
+    for (int i = 0; i < 12; ++i) {
+        const int pidx = cx.tid + kThreads * i;
+        const int tile = pidx >> 9, j = (pidx >> 3) & 63, cc = pidx & 7;
+        const int tau = c0 + j - cx.rv_p;
+        int t;
+        bool ok;
+        if (tile < 3) {  // w', a', b' = w, b, a of token L - tau
+            t = cx.rv_L - tau;
+            ok = tau >= 1 && tau <= cx.rv_L && (!ri.mask || ri.mask[cx.rv_row0 + t] != 0);
+        } else {         // k', v', r' = r, dO, k of token L - 1 - tau
+            t = cx.rv_L - 1 - tau;
+            ok = tau >= 0 && tau < cx.rv_L;
+        }
+        const __nv_bfloat16* src = tile == 0 ? ri.w : tile == 1 ? ri.b : tile == 2 ? ri.a
+                                 : tile == 3 ? ri.r : tile == 4 ? ri.dout : ri.k;
+        const uint32_t dst = tile == 0 ? L.W : tile == 1 ? L.A : tile == 2 ? L.B
+                           : tile == 3 ? L.K : tile == 4 ? L.V : L.R;
+        if (ok) src += cx.rv_base + (long long)t * cx.rv_ts + 8 * cc;
+        sm100::cp_async_16(cx.sbase + dst + sw(j, cc), src, ok ? 16u : 0u);
+    }
+    sm100::cp_async_mbar_arrive(cx.bar_tma);
+}
+
 // One 64-token chunk starting at token c0, in layout P (its inputs already requested).
 // Returns false, the same in every thread, when a bounded wait ran out: the caller then
 // abandons the sequence.
-template <bool kGdn, bool kHf>
+template <bool kGdn, bool kHf, bool kRev>
 __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
     const LayR L = lay_of(par);
     using namespace sm100;
@@ -874,7 +923,10 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
 
         // W and Z have been read: every tile the next chunk loads into is dead now.
         if (has_next) {
-            if (warp == 1) issue_loads<kGdn, kHf>(cx, c0 + 64, par ^ 1);
+            if constexpr (kRev)
+                issue_loads_rev(cx, c0 + 64, par ^ 1);
+            else if (warp == 1)
+                issue_loads<kGdn, kHf>(cx, c0 + 64, par ^ 1);
             cx.tma_par_last = par ^ 1;
         }
 
@@ -888,6 +940,8 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             fence_proxy_async();
             tc_fence_before();
             if (__syncthreads_or(cx.timed_out)) return false;
+            // every thread's copies are tracked by now: complete the arrival count
+            if (kRev && has_next && tid == 0) sm100::mbar_arrive(cx.bar_tma);
         }
 
         // ---- 9. the final products (M = 64, fp16):
@@ -925,7 +979,49 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
 
         // ---- 10. epilogue 4: the chunk's outputs (rows t = 16 wq + lane of O); the new fp32
         //          state stays in tensor memory. ---------------------------------------------
-        if (o != nullptr) {  // (no outputs: a state-only run)
+        if constexpr (kRev) {
+            // row j is dv of original token tb - j (zero for a masked one); rows staged
+            // reversed, so the tile is tokens tb - 63 .. tb in order
+            float v[16];
+            tmem_frag(tmem + TM_DFO, wq, 32 * wh, v);
+            const RevIn& ri = *cx.ri;
+            const int tb = cx.rv_L - 1 - (c0 - cx.rv_p);
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int t = tb - (16 * wq + (lane >> 2) + 8 * hr);
+                const bool keep = t >= 0 && t < cx.rv_L && (!ri.mask || ri.mask[cx.rv_row0 + t] != 0);
+                if (!keep) {
+#pragma unroll
+                    for (int j2 = 0; j2 < 4; ++j2) v[4 * j2 + 2 * hr] = v[4 * j2 + 2 * hr + 1] = 0.f;
+                }
+            }
+            {
+                const int mi = lane >> 3;
+                const int row = 16 * wq + 8 * (mi & 1) + (lane & 7);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    stsm_x4(sbase + OFF_S0 + sw(63 - row, 4 * wh + 2 * hh + (mi >> 1)),
+                            pack2(v[8 * hh + 0], v[8 * hh + 1]), pack2(v[8 * hh + 2], v[8 * hh + 3]),
+                            pack2(v[8 * hh + 4], v[8 * hh + 5]), pack2(v[8 * hh + 6], v[8 * hh + 7]));
+            }
+            fence_proxy_async();
+            __syncthreads();
+            const int t0s = tb - 63;  // token of staging row 0
+            if (t0s >= 0 && t0s + 63 < cx.rv_L) {
+                if (tid == kStoreTid) {
+                    tma_store_3d(cx.tm_o, sbase + OFF_S0, 0, ri.hf ? cx.rv_y0 + t0s : cx.rv_y0,
+                                 ri.hf ? cx.rv_z0 : cx.rv_z0 + t0s);
+                    bulk_commit();
+                }
+            } else {
+                for (int i = tid; i < 512; i += kThreads) {
+                    const int r = i >> 3, cc = i & 7, t = t0s + r;
+                    if (t >= 0 && t < cx.rv_L)
+                        *reinterpret_cast<uint4*>(ri.dv + cx.rv_base + (long long)t * cx.rv_ts + 8 * cc) =
+                            *reinterpret_cast<const uint4*>(smem + OFF_S0 + sw(r, cc));
+                }
+            }
+        } else if (o != nullptr) {  // (no outputs: a state-only run)
             float v[16];
             tmem_frag(tmem + TM_DFO, wq, 32 * wh, v);
             if (nv == 64) {
@@ -964,7 +1060,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
 // kGdn: Gated DeltaNet (tm_r, tm_k, tm_v map q, k, v; g and beta per token; s0 may be
 // one state per head shared by every sequence, s0_shared != 0).  kHf (head first):
 // inputs, o (and g, beta) are [B, H, T, *] instead of [B, T, H, *]; the maps follow.
-template <bool kGdn, bool kHf>
+template <bool kGdn, bool kHf, bool kRev>
 __global__ void __launch_bounds__(kThreads, 2)
 chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -974,7 +1070,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
                const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
                float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens,
                const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ beta,
-               int s0_shared, int stall_tid, int ck_slots) {
+               int s0_shared, int stall_tid, int ck_slots, const __grid_constant__ RevIn rin) {
     extern __shared__ __align__(1024) uint8_t smem[];
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1063,6 +1159,30 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     cx.tm_b = &tm_b;
     cx.tm_o = &tm_o;
     cx.tm_ck = &tm_ck;
+    cx.ri = &rin;
+    if constexpr (kRev) {
+        int bb_o = n, bos_o = 0, L_o = rin.T;
+        if (rin.cu) {
+            bb_o = 0;
+            bos_o = rin.cu[n];
+            L_o = rin.cu[n + 1] - bos_o;
+            if (bos_o < 0 || L_o < 0 || bos_o + L_o > rin.T) bos_o = L_o = 0;  // flagged by prep
+        }
+        cx.rv_L = L_o;
+        cx.rv_p = 63 - (L_o & 63);
+        cx.rv_row0 = (long long)bb_o * rin.T + bos_o;
+        if (rin.hf) {
+            cx.rv_base = (((long long)bb_o * H + h) * rin.T + bos_o) * 64;
+            cx.rv_ts = 64;
+            cx.rv_y0 = bos_o;
+            cx.rv_z0 = bb_o * H + h;
+        } else {
+            cx.rv_base = (cx.rv_row0 * H + h) * 64;
+            cx.rv_ts = (long long)H * 64;
+            cx.rv_y0 = h;
+            cx.rv_z0 = (int)cx.rv_row0;
+        }
+    }
     cx.ck = ck_slots > 0;
     cx.ck_z0 = h * ck_slots + (int)(cx.row0 >> 6) + n;  // slot: floor(row0 / 64) + n + chunk
     cx.g = g;
@@ -1087,7 +1207,15 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     if (warp == 0 && lane < 7)
         prefetch_tensormap(lane == 0 ? &tm_r : lane == 1 ? &tm_a : lane == 2 ? &tm_k
                            : lane == 3 ? &tm_b : lane == 4 ? &tm_w : lane == 5 ? &tm_v : &tm_o);
-    if (warp == 0 && cx.len > 0) issue_loads<kGdn, kHf>(cx, 0, 0);
+    if constexpr (kRev) {
+        if (cx.len > 0) {
+            issue_loads_rev(cx, 0, 0);
+            __syncthreads();  // every thread's copies are tracked: complete the count
+            if (tid == 0) mbar_arrive(cx.bar_tma);
+        }
+    } else if (warp == 0 && cx.len > 0) {
+        issue_loads<kGdn, kHf>(cx, 0, 0);
+    }
 
     // The fp32 state lives in tensor memory as an M = 64 accumulator: row k in lane
     // (k % 16) + 32 (k / 16), so lanes 0..15 of warp w hold rows 16 (w % 4) + lane,
@@ -1118,7 +1246,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     // Chunks alternate between the two shared-memory layouts.
     bool ok = true;
     for (int c0 = 0, par = 0; c0 < cx.len && ok; c0 += 64, par ^= 1)
-        ok = chunk<kGdn, kHf>(cx, c0, c0 + 64 < cx.len, par);
+        ok = chunk<kGdn, kHf, kRev>(cx, c0, c0 + 64 < cx.len, par);
     // The last chunk's final-MMA wait is agreed on here (it has no barrier of its own).
     if (ok && __syncthreads_or(cx.timed_out)) ok = false;
 
@@ -1216,17 +1344,23 @@ struct Extras {
     void* ck = nullptr;
     int ck_slots = 0;
 };
-template <bool kGdn, bool kHf>
+template <bool kGdn, bool kHf, bool kRev = false>
 inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float* s0,
                           const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
                           const int32_t* cu_seqlens, const void* g, const void* beta,
                           int s0_shared, int stall_tid, const Extras& ex,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const RevIn* rin = nullptr,
+                          int B_o = 0, int T_o = 0) {
     CUtensorMap maps[8];
+    if (kRev) {  // the output is dv in the original layout; no input maps (cp.async loads)
+        if (!make_map(&maps[6], rin->dv, B_o, T_o, H, rin->hf)) return cudaErrorInvalidValue;
+        for (int i = 0; i < 6; ++i) maps[i] = maps[6];  // unused by the kernel
+    }
     for (int i = 0; i < nmaps; ++i)
         if (!make_map(&maps[i], ptrs[i], B, T, H, kHf)) return cudaErrorInvalidValue;
-    for (int i = nmaps; i < 6; ++i) maps[i] = maps[0];  // unused by the kernel
-    if (o) {
+    for (int i = nmaps; i < 6 && !kRev; ++i) maps[i] = maps[0];  // unused by the kernel
+    if (kRev) {
+    } else if (o) {
         if (!make_map(&maps[6], o, B, T, H, kHf)) return cudaErrorInvalidValue;  // the output
     } else {
         maps[6] = maps[0];  // unused: no outputs
@@ -1239,17 +1373,18 @@ inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float
     }
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf>,
+        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf, kRev>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    chunked_kernel<kGdn, kHf><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
+    const RevIn rv = rin ? *rin : RevIn{};
+    chunked_kernel<kGdn, kHf, kRev><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7], s0, mask,
         static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens,
         static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(beta), s0_shared,
-        stall_tid, ex.ck ? ex.ck_slots : 0);
+        stall_tid, ex.ck ? ex.ck_slots : 0, rv);
     return cudaGetLastError();
 }
 template <bool kGdn>
@@ -1275,6 +1410,18 @@ inline cudaError_t launch_chunked(const void* r, const void* w, const void* k, c
     const void* ptrs[6] = {r, w, k, v, a, b};
     return chunked::launch<false>(ptrs, 6, s0, mask, o, sT, B, T, H, N, cu_seqlens, nullptr,
                                   nullptr, 0, head_first, stall_tid, ex, stream);
+}
+
+// The backward's reversed run of the state gradient (see RevIn): unit n of the packed
+// reversed sequences `cur` ([N + 1], multiples of 64, rows_r in all) for every head, from
+// the state dsT (or zero) to ds0, with per-chunk checkpoints and dv written in the
+// original layout ([B_o, T_o, H, 64] or head first).  The input maps are not read.
+inline cudaError_t launch_chunked_rev(const chunked::RevIn& rin, int B_o, const float* dsT, float* ds0,
+                                      int rows_r, int H, int N, const int32_t* cur,
+                                      const chunked::Extras& ex, cudaStream_t stream) {
+    return chunked::launch_layout<false, false, true>(nullptr, 0, dsT, nullptr, nullptr, ds0, 1,
+                                                      rows_r, H, N, cur, nullptr, nullptr, 0, -1,
+                                                      ex, stream, &rin, B_o, rin.T);
 }
 
 // Gated DeltaNet: q, k, v [B*T, H, 64] bf16 through the r, k, v maps; g, beta [B*T, H]

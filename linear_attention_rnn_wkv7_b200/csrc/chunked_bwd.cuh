@@ -9,22 +9,21 @@
 //     X_tau = (diag(e^{w'_tau}) + b'_tau a'_tau^T) X_{tau-1} + k'_tau v'_tau^T
 // where w'_tau = w_{L-tau}, b' = a_{L-tau}, a' = b_{L-tau} (tau >= 1; the identity at
 // tau = 0) and k'_tau = r_{L-1-tau}, v'_tau = do_{L-1-tau} (tau < L), started from dsT;
-// one more transition (tau = L, no input) gives ds0.  So the backward runs in four
-// launches of its own plus two of the forward kernel:
+// one more transition (tau = L, no input) gives ds0.  So the backward is four launches:
 //   1. prep:     offsets of the reversed sequences (each padded at its start to a
 //                multiple of 64 tokens: p = 63 - L % 64 identity steps, then L + 1 steps);
 //   2. forward:  the chunked forward with per-chunk fp16 checkpoints of the state
 //                S0 at every chunk start, and no outputs;
-//   3. reverse:  the reversed, shifted inputs above (a masked token's transition is the
-//                identity, its output still feeds G) plus r' = k reversed, so that the
-//                reversed run's outputs o'_tau = X_tau^T k_{L-1-tau} = G_t^T k_t are dv;
-//   4. forward on the reversed inputs from dsT: its final state is ds0 and its
-//                per-chunk checkpoints hold G at the last token of every chunk of the
-//                original sequence (the padding puts chunk boundaries there);
-//   5. grad:     one CTA per original chunk, all chunks in parallel: the chunk's
+//   3. reversed: the same kernel over the reversed sequences from dsT, reading the
+//                original tensors itself (a masked token's transition is the identity,
+//                its output still feeds G; r' = k, so its outputs X_tau^T k_{L-1-tau} =
+//                G_t^T k_t are dv, written in place, zero for a masked token): its final
+//                state is ds0 and its per-chunk checkpoints hold G at the last token of
+//                every chunk of the original sequence (the padding puts chunk boundaries
+//                there);
+//   4. grad:     the chunks in parallel (persistent, one CTA per SM): each chunk's
 //                gradients from its inputs, S0 and dSL = G_e - r_e do_e^T (e its last
-//                token; dSL = dsT for a partial last chunk), on tcgen05;
-//   6. dv:       o' back to token order (zero for masked tokens).
+//                token; dSL = dsT for a partial last chunk), on tcgen05.
 //
 // The per-chunk adjoint (grad kernel), with the forward's chunk algebra (chunked.cuh):
 //   X = Abar S0 + A_ak V,  U = T X                     (U = W S0 + Z V)
@@ -60,7 +59,7 @@ constexpr int kThreads = 256;
 struct Ws {
     long long rows, rowsR;   // token rows of the inputs; bound on the reversed rows
     long long slotsF, slotsR;  // checkpoint slots per head (forward, reversed)
-    size_t off_cu, off_ckF, off_ckR, off_rev, rev_stride, total;
+    size_t off_cu, off_ckF, off_ckR, total;
 };
 inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 inline Ws ws_layout(long long rows, int N, int H) {
@@ -72,9 +71,7 @@ inline Ws ws_layout(long long rows, int N, int H) {
     w.off_cu = 0;
     w.off_ckF = al256((size_t)(N + 1) * 4);
     w.off_ckR = al256(w.off_ckF + (size_t)H * w.slotsF * 8192);
-    w.off_rev = al256(w.off_ckR + (size_t)H * w.slotsR * 8192);
-    w.rev_stride = al256((size_t)w.rowsR * H * 128);  // one reversed [rowsR, H, 64] bf16 tensor
-    w.total = w.off_rev + 7 * w.rev_stride;           // w', a', b', k', v', r', o'
+    w.total = al256(w.off_ckR + (size_t)H * w.slotsR * 8192);
     return w;
 }
 
@@ -136,111 +133,6 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------------
-// 3. reverse: one CTA per (reversed 64-row chunk, head); thread = 16 bytes of two rows
-//    (rows i and i + 32); the six loads of a row are issued before its six stores.
-// ---------------------------------------------------------------------------------
-template <bool kHf>
-__global__ void __launch_bounds__(256) reverse_kernel(
-    const __nv_bfloat16* __restrict__ r, const __nv_bfloat16* __restrict__ w,
-    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ a,
-    const __nv_bfloat16* __restrict__ b, const __nv_bfloat16* __restrict__ dout,
-    const uint8_t* __restrict__ mask, const int32_t* __restrict__ cu,
-    const int32_t* __restrict__ cur, int T, int H, int N, __nv_bfloat16* __restrict__ rev,
-    size_t rev_stride_elems) {
-    const int gchunk = blockIdx.x, h = blockIdx.y;
-    const long long grow0 = 64LL * gchunk;
-    if (grow0 >= cur[N]) return;
-    int lo = 0, hi = N - 1;  // last n with cur[n] <= grow0
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (cur[mid] <= grow0) lo = mid; else hi = mid - 1;
-    }
-    const int n = lo;
-    long long row0;
-    int L;
-    bool ok;
-    seq_of(n, T, cu, row0, L, ok);
-    if (!ok) L = 0;  // flagged by prep; the reversed sequence is all identity
-    const int p = 63 - (L & 63);
-    const int piece = threadIdx.x & 7;
-    // element offset of token t of the sequence (head h) in the inputs
-    const long long base = kHf ? (((row0 / T) * H + h) * (long long)T + (row0 % T)) * 64
-                               : (row0 * H + h) * 64;
-    const long long tstride = kHf ? 64 : (long long)H * 64;
-    const size_t str = rev_stride_elems / 8;  // tensors apart, in uint4
-    const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int row = (threadIdx.x >> 3) + 32 * half;
-        const long long tp = grow0 + row - cur[n];  // tau' within the reversed sequence
-        const int tau = (int)tp - p;
-        const int t1 = L - tau;      // transition token (tau >= 1)
-        const int t2 = L - 1 - tau;  // input token (tau < L)
-        const bool in1 = tau >= 1 && tau <= L, in2 = tau >= 0 && tau < L;
-        const bool has1 = in1 && (!mask || mask[row0 + t1] != 0);
-        uint4 x[6] = {z, z, z, z, z, z};
-        if (L > 0) {
-            const int c1 = min(max(t1, 0), L - 1), c2 = min(max(t2, 0), L - 1);
-            const long long e1 = base + c1 * tstride, e2 = base + c2 * tstride;
-            x[0] = __ldg(reinterpret_cast<const uint4*>(w + e1) + piece);
-            x[1] = __ldg(reinterpret_cast<const uint4*>(b + e1) + piece);
-            x[2] = __ldg(reinterpret_cast<const uint4*>(a + e1) + piece);
-            x[3] = __ldg(reinterpret_cast<const uint4*>(r + e2) + piece);
-            x[4] = __ldg(reinterpret_cast<const uint4*>(dout + e2) + piece);
-            x[5] = __ldg(reinterpret_cast<const uint4*>(k + e2) + piece);
-        }
-        // w' a' b' k' v' r' = w[t1] b[t1] a[t1] r[t2] do[t2] k[t2]
-        uint4* out = reinterpret_cast<uint4*>(rev + ((size_t)(grow0 + row) * H + h) * 64) + piece;
-#pragma unroll
-        for (int i = 0; i < 6; ++i) out[i * str] = (i < 3 ? has1 : in2) ? x[i] : z;
-    }
-}
-
-// ---------------------------------------------------------------------------------
-// 6. dv: dv[t] = o'[cur_n + p + L - 1 - t] (zero for a masked token); thread = 16 bytes.
-// ---------------------------------------------------------------------------------
-template <bool kHf>
-__global__ void __launch_bounds__(256) dv_kernel(const __nv_bfloat16* __restrict__ orev,
-                                                 const uint8_t* __restrict__ mask,
-                                                 const int32_t* __restrict__ cu,
-                                                 const int32_t* __restrict__ cur, int T, int H,
-                                                 int N, long long rows,
-                                                 __nv_bfloat16* __restrict__ dv) {
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // (row, h, 8 pieces)
-    if (i >= rows * H * 8) return;
-    const int piece = (int)(i & 7);
-    const int h = (int)((i >> 3) % H);
-    const long long grow = (i >> 3) / H;  // token row in [B*T]
-    int n;
-    if (cu) {
-        int lo = 0, hi = N - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (cu[mid] <= grow) lo = mid; else hi = mid - 1;
-        }
-        n = lo;
-        if (grow >= cu[N] || grow < cu[n]) return;  // rows outside every sequence: untouched
-    } else {
-        n = (int)(grow / T);
-    }
-    long long row0;
-    int L;
-    bool ok;
-    seq_of(n, T, cu, row0, L, ok);
-    if (!ok) return;
-    const int t = (int)(grow - row0);
-    const int p = 63 - (L & 63);
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (!mask || mask[grow] != 0) {
-        const long long rr = cur[n] + p + L - 1 - t;
-        val = reinterpret_cast<const uint4*>(orev + (rr * H + h) * 64)[piece];
-    }
-    const long long e = kHf ? (((row0 / T) * H + h) * (long long)T + (row0 % T) + t) * 64
-                            : (grow * H + h) * 64;
-    reinterpret_cast<uint4*>(dv + e)[piece] = val;
-}
-
-// ---------------------------------------------------------------------------------
 // 5. grad: the per-chunk adjoint on tcgen05.
 // ---------------------------------------------------------------------------------
 // Shared-memory tiles (8 KB, 64 rows x 128 B, 128B swizzle).
@@ -268,7 +160,8 @@ constexpr uint32_t GOFF_EM0 = GOFF_R + 256;          // E_{-1} per channel (64 f
 constexpr uint32_t GOFF_RAW = GOFF_EM0 + 256;        // raw r and dO of token 63 (2 x 64 fp32)
 constexpr uint32_t GOFF_TOT = GOFF_RAW + 512;        // scan totals [4 quadrants][64]
 constexpr uint32_t GOFF_NEXT = GOFF_TOT + 1024;      // the CTA's next work item (and index)
-constexpr uint32_t kGSmemBytes = GOFF_NEXT + 128;
+constexpr uint32_t GOFF_RP = GOFF_NEXT + 128;        // rowsum(S0 P) halves [2][64] (fixed order)
+constexpr uint32_t kGSmemBytes = GOFF_RP + 512;
 static_assert(kGSmemBytes <= 232448, "fits one CTA per SM");
 constexpr uint32_t kGTmemCols = 512;
 // TMEM columns (every accumulator M = 64): C0..C2 hold each phase's products for its
@@ -386,6 +279,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     float* em0 = reinterpret_cast<float*>(smem + GOFF_EM0);
     float* raw = reinterpret_cast<float*>(smem + GOFF_RAW);
     float* tot = reinterpret_cast<float*>(smem + GOFF_TOT);
+    float* Rp = reinterpret_cast<float*>(smem + GOFF_RP);
     float* Ef = reinterpret_cast<float*>(smem + gt(G_E));
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GOFF_MISC + 32);
     int timed_out = 0;
@@ -869,7 +763,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     mph ^= 1;
     tc_fence_after();
     acc_to_tile(tmem, C0, sbase + gt(G_DAAB), wq, wh, lane, 2, PackB{});
-    {  // R += rowsum(S0 * P) over this warp's 32 columns
+    {  // rowsum(S0 * P) over this warp's 32 columns (added to R in the final epilogue)
         float v[16];
         tmem_frag(tmem + C_P, wq, 32 * wh, v);
 #pragma unroll
@@ -884,7 +778,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
             }
             part += __shfl_xor_sync(0xffffffffu, part, 1);
             part += __shfl_xor_sync(0xffffffffu, part, 2);
-            if (q == 0) atomicAdd(Rc + row, part);
+            if (q == 0) Rp[64 * wh + row] = part;
         }
     }
     fence_proxy_async();
@@ -1001,7 +895,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                 const int cidx = 32 * wh + 8 * j + 2 * q + e;
                 float pre = 0.f;
                 for (int w2 = 0; w2 < wq; ++w2) pre += tot[w2 * 64 + cidx];
-                const float R = Rc[cidx];
+                const float R = Rc[cidx] + Rp[cidx] + Rp[64 + cidx];  // fixed order
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {
                     const int ix = 4 * j + 2 * hr + e;
@@ -1116,16 +1010,13 @@ inline cudaError_t launch_bwd_chunked(const void* r, const void* w, const void* 
     using namespace cbwd;
     const long long rows = (long long)B * T;
     const Ws lay = ws_layout(rows, N, H);
-    if (lay.slotsF > 0x7fffffffLL || lay.slotsR > 0x7fffffffLL || (long long)H * lay.slotsR > 0x7fffffffLL)
+    if (lay.slotsF > 0x7fffffffLL || lay.slotsR > 0x7fffffffLL ||
+        (long long)H * lay.slotsR > 0x7fffffffLL || lay.rowsR > 0x7fffffffLL)
         return cudaErrorInvalidValue;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* cur = reinterpret_cast<int32_t*>(ws + lay.off_cu);
     void* ckF = ws + lay.off_ckF;
     void* ckR = ws + lay.off_ckR;
-    __nv_bfloat16* rev = reinterpret_cast<__nv_bfloat16*>(ws + lay.off_rev);
-    const size_t rs = lay.rev_stride / 2;  // elements
-    __nv_bfloat16 *wr = rev, *ar = rev + rs, *br = rev + 2 * rs, *kr = rev + 3 * rs,
-                  *vr = rev + 4 * rs, *rr = rev + 5 * rs, *orv = rev + 6 * rs;
     cudaError_t e;
     // 1. reversed sequence offsets
     prep_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, T, N, cur);
@@ -1137,46 +1028,31 @@ inline cudaError_t launch_bwd_chunked(const void* r, const void* w, const void* 
     if ((e = launch_chunked(r, w, k, v, a, b, s0, mask, nullptr, nullptr, B, T, H, N, cu_seqlens,
                             head_first, -1, stream, exF)) != cudaSuccess)
         return e;
-    // 3. reversed inputs
-    const dim3 rgrid((unsigned)(lay.rowsR / 64), (unsigned)H);
-    const __nv_bfloat16 *pr = static_cast<const __nv_bfloat16*>(r),
-                        *pw = static_cast<const __nv_bfloat16*>(w),
-                        *pk = static_cast<const __nv_bfloat16*>(k),
-                        *pa = static_cast<const __nv_bfloat16*>(a),
-                        *pb = static_cast<const __nv_bfloat16*>(b),
-                        *pd = static_cast<const __nv_bfloat16*>(dout);
-    if (head_first)
-        reverse_kernel<true><<<rgrid, 256, 0, stream>>>(pr, pw, pk, pa, pb, pd, mask, cu_seqlens,
-                                                        cur, T, H, N, rev, rs);
-    else
-        reverse_kernel<false><<<rgrid, 256, 0, stream>>>(pr, pw, pk, pa, pb, pd, mask, cu_seqlens,
-                                                         cur, T, H, N, rev, rs);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 4. the adjoint as a forward run over the reversed sequences, from dsT
+    // 3. the state gradient as a forward run over the reversed sequences, from dsT
+    chunked::RevIn rin;
+    rin.w = static_cast<const __nv_bfloat16*>(w);
+    rin.a = static_cast<const __nv_bfloat16*>(a);
+    rin.b = static_cast<const __nv_bfloat16*>(b);
+    rin.r = static_cast<const __nv_bfloat16*>(r);
+    rin.dout = static_cast<const __nv_bfloat16*>(dout);
+    rin.k = static_cast<const __nv_bfloat16*>(k);
+    rin.mask = mask;
+    rin.cu = cu_seqlens;
+    rin.T = T;
+    rin.hf = head_first;
+    rin.dv = static_cast<__nv_bfloat16*>(dv);
     chunked::Extras exR;
     exR.ck = ckR;
     exR.ck_slots = (int)lay.slotsR;
-    if ((e = launch_chunked(rr, wr, kr, vr, ar, br, dsT, nullptr, orv, ds0, 1, (int)lay.rowsR, H,
-                            N, cur, 0, -1, stream, exR)) != cudaSuccess)
+    if ((e = launch_chunked_rev(rin, B, dsT, ds0, (int)lay.rowsR, H, N, cur, exR, stream)) !=
+        cudaSuccess)
         return e;
-    // 5. per-chunk gradients
+    // 4. per-chunk gradients
     e = head_first ? launch_grad<true>(r, w, k, v, a, b, dout, mask, dr, dw, dk, da, db, B, T, H,
                                        N, cu_seqlens, cur, ckF, ckR, lay, stream)
                    : launch_grad<false>(r, w, k, v, a, b, dout, mask, dr, dw, dk, da, db, B, T,
                                         H, N, cu_seqlens, cur, ckF, ckR, lay, stream);
     if (e != cudaSuccess) return e;
-    // 6. dv in token order
-    const long long nthr = rows * H * 8;
-    if (nthr > 0) {
-        const unsigned blocks = (unsigned)((nthr + 255) / 256);
-        if (head_first)
-            dv_kernel<true><<<blocks, 256, 0, stream>>>(orv, mask, cu_seqlens, cur, T, H, N, rows,
-                                                        static_cast<__nv_bfloat16*>(dv));
-        else
-            dv_kernel<false><<<blocks, 256, 0, stream>>>(orv, mask, cu_seqlens, cur, T, H, N, rows,
-                                                         static_cast<__nv_bfloat16*>(dv));
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
     return cudaSuccess;
 }
 

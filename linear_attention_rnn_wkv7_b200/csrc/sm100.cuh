@@ -83,6 +83,24 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
         : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared; src_bytes 0 fills the 16 bytes with zeros
+// (no global read).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+// The mbarrier tracks this thread's earlier cp.async copies: its pending count rises by
+// one now and falls by one when they have landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+// A plain arrive on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+                 : "memory");
+}
+
 // Tile store shared -> global through a tensor map (bulk async group of this thread).
 __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int c0, int c1,
                                              int c2) {

@@ -175,17 +175,15 @@ def test_bwd_rejects_bad_arguments(lib):
     ws = ctypes.c_void_p(P + 0x100000)
     need = lib.wkv7_bwd_workspace_bytes(1, 16, 2, 64, 64, 1)
     # the larger of the two families' needs: the fp32 recurrences (checkpoints every
-    # 8 tokens and every token's u) and the chunked form (reversed-sequence offsets,
-    # fp16 state checkpoints of both passes, seven reversed [rows + 64 N, H, 64] bf16
-    # tensors; every region 256-byte aligned)
+    # 8 tokens and every token's u) and the chunked form (reversed-sequence offsets and
+    # the fp16 state checkpoints of both passes; every region 256-byte aligned)
     rows, N, H = 16, 1, 2
     rec = (H * (rows // 8 + 2 * N + 1) * 4096 + rows * H * 64) * 4
     al = lambda x: (x + 255) // 256 * 256
     rows_r = rows + 64 * N
     ck_f = al(4 * (N + 1))
     ck_r = al(ck_f + H * (rows // 64 + N + 1) * 8192)
-    rev = al(ck_r + H * (rows_r // 64 + N + 1) * 8192)
-    chk = rev + 7 * al(rows_r * H * 128)
+    chk = al(ck_r + H * (rows_r // 64 + N + 1) * 8192)
     assert need == max(rec, chk)
     assert lib.wkv7_bwd_workspace_bytes(1, 16, 2, 128, 128, 1) == 0
 
