@@ -370,26 +370,24 @@ __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
 __device__ __forceinline__ void issue_loads_rev(const Ctx& cx, int c0, int par) {
     const LayR L = lay_of(par);
     const RevIn& ri = *cx.ri;
-#pragma unroll 2
-    for (int i = 0; i < 12; ++i) {
-        const int pidx = cx.tid + kThreads * i;
-        const int tile = pidx >> 9, j = (pidx >> 3) & 63, cc = pidx & 7;
+    const int cc = cx.tid & 7;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {  // rows j and j + 32, 16-byte piece cc of each
+        const int j = (cx.tid >> 3) + 32 * half;
         const int tau = c0 + j - cx.rv_p;
-        int t;
-        bool ok;
-        if (tile < 3) {  // w', a', b' = w, b, a of token L - tau
-            t = cx.rv_L - tau;
-            ok = tau >= 1 && tau <= cx.rv_L && (!ri.mask || ri.mask[cx.rv_row0 + t] != 0);
-        } else {         // k', v', r' = r, dO, k of token L - 1 - tau
-            t = cx.rv_L - 1 - tau;
-            ok = tau >= 0 && tau < cx.rv_L;
-        }
-        const __nv_bfloat16* src = tile == 0 ? ri.w : tile == 1 ? ri.b : tile == 2 ? ri.a
-                                 : tile == 3 ? ri.r : tile == 4 ? ri.dout : ri.k;
-        const uint32_t dst = tile == 0 ? L.W : tile == 1 ? L.A : tile == 2 ? L.B
-                           : tile == 3 ? L.K : tile == 4 ? L.V : L.R;
-        if (ok) src += cx.rv_base + (long long)t * cx.rv_ts + 8 * cc;
-        sm100::cp_async_16(cx.sbase + dst + sw(j, cc), src, ok ? 16u : 0u);
+        const int t1 = cx.rv_L - tau, t2 = t1 - 1;  // transition token, write-pair token
+        const bool ok1 = tau >= 1 && tau <= cx.rv_L && (!ri.mask || ri.mask[cx.rv_row0 + t1] != 0);
+        const bool ok2 = tau >= 0 && tau < cx.rv_L;
+        const long long o1 = ok1 ? cx.rv_base + (long long)t1 * cx.rv_ts + 8 * cc : 0;
+        const long long o2 = ok2 ? cx.rv_base + (long long)t2 * cx.rv_ts + 8 * cc : 0;
+        const uint32_t n1 = ok1 ? 16u : 0u, n2 = ok2 ? 16u : 0u, d = cx.sbase + sw(j, cc);
+        // w', a', b' = w, b, a of token t1;  k', v', r' = r, dO, k of token t2
+        sm100::cp_async_16(d + L.W, ri.w + o1, n1);
+        sm100::cp_async_16(d + L.A, ri.b + o1, n1);
+        sm100::cp_async_16(d + L.B, ri.a + o1, n1);
+        sm100::cp_async_16(d + L.K, ri.r + o2, n2);
+        sm100::cp_async_16(d + L.V, ri.dout + o2, n2);
+        sm100::cp_async_16(d + L.R, ri.k + o2, n2);
     }
     sm100::cp_async_mbar_arrive(cx.bar_tma);
 }
@@ -407,6 +405,8 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
     const long long row0 = cx.row0;
     const uint8_t* mask = cx.mask;
     __nv_bfloat16* o = cx.o;
+    // a state-only run (no outputs): the work that only feeds O is skipped
+    const bool so = !kRev && o == nullptr;
     float* gamma_s = cx.gamma_s;
     uint32_t& mma_phase = cx.mma_phase;
     float* scratch = reinterpret_cast<float*>(smem + L.SP);  // prologue only
@@ -636,10 +636,12 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem + TM_D1, smem_desc(sbase + L.A + 32 * kk, 16, 1024),
                               smem_desc(sbase + L.K + 32 * kk, 16, 1024), id64, kk > 0);
+                if (!so) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.K + 32 * kk, 16, 1024),
-                              smem_desc(sbase + L.R + 32 * kk, 16, 1024), id128, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + TM_D1B, smem_desc(sbase + L.K + 32 * kk, 16, 1024),
+                                  smem_desc(sbase + L.R + 32 * kk, 16, 1024), id128, kk > 0);
+                }
                 umma_commit(cx.bar_g2);
             }
             // While it runs: Abar = a~ e^{g_L} and Rbar = r~ e^{g_L} (fp16), V to fp16 in
@@ -654,7 +656,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                     rbar[e] = rts[it][e] * ec[e];
                 }
                 *reinterpret_cast<uint4*>(smem + L.ABAR + off) = pack8h(abar);
-                *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8h(rbar);
+                if (!so) *reinterpret_cast<uint4*>(smem + L.RBAR + off) = pack8h(rbar);
                 float vf[8];
                 unpack8(*reinterpret_cast<const uint4*>(smem + L.V + off), vf);
                 *reinterpret_cast<uint4*>(smem + L.V + off) = pack8h(vf);
@@ -772,7 +774,7 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
                 const int s_ = 32 * (wq & 1) + lane;
                 const uint32_t dst = wq < 2 ? L.ARKT : L.ARBT;
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
+                for (int h2 = 0; h2 < (so ? 0 : 2); ++h2) {
                     float v[32];
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
@@ -959,18 +961,20 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             for (int kk = 0; kk < 4; ++kk)
                 umma_bf16(tmem + TM_DFS, smem_desc(sbase + L.KHAT + 2048 * kk, 8192, 1024),
                           smem_desc(sbase + L.V + 2048 * kk, 8192, 1024), idmm, 1u);
+            if (!so) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.ARBT + 2048 * kk, 8192, 1024),
-                          smem_desc(sbase + L.A + 2048 * kk, 8192, 1024), idmm, kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.ARBT + 2048 * kk, 8192, 1024),
+                              smem_desc(sbase + L.A + 2048 * kk, 8192, 1024), idmm, kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.ARKT + 2048 * kk, 8192, 1024),
-                          smem_desc(sbase + L.V + 2048 * kk, 8192, 1024), idmm, 1u);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.ARKT + 2048 * kk, 8192, 1024),
+                              smem_desc(sbase + L.V + 2048 * kk, 8192, 1024), idmm, 1u);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.RBAR + 32 * kk, 16, 1024),
-                          smem_desc(sbase + OFF_S0 + 2048 * kk, 8192, 1024), idkm, 1u);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_DFO, smem_desc(sbase + L.RBAR + 32 * kk, 16, 1024),
+                              smem_desc(sbase + OFF_S0 + 2048 * kk, 8192, 1024), idkm, 1u);
+            }
             umma_commit(bar_mma);
         }
         wait_or_abort(bar_mma, mma_phase, cx.timed_out);

@@ -218,6 +218,17 @@ __device__ __forceinline__ bool item_of(int it, int slotsF, int T, int N, const 
                                         Item& I) {
     I.h = it / slotsF;
     I.slot = it - I.h * slotsF;
+    if (!cu && (T & 63) == 0) {  // equal lengths, a multiple of 64: T / 64 + 1 slots each
+        const int per = T / 64 + 1;
+        I.n = I.slot / per;
+        I.c = I.slot - I.n * per;
+        I.L = T;
+        I.row0 = (long long)I.n * T;
+        if (I.n >= N || I.c >= T / 64) return false;
+        I.nv = 64;
+        I.crow = I.row0 + 64LL * I.c;
+        return true;
+    }
     int lo = 0, hi = N - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -333,6 +344,35 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         if (lane < 9) load_in(I, lane);
     }
 
+    // The previous chunk's outputs (dr dw dk da db), staged in the dA tiles and X: five
+    // TMA tile stores (one per warp), or the rows < nv copied for a partial chunk (the
+    // rows after belong to another sequence).  Called by every thread after a barrier.
+    int p_nv = 0, p_h = 0, p_cy = 0, p_cz = 0;
+    long long p_crow = 0;
+    auto flush = [&]() {
+        if (p_nv == 0) return;
+        const uint32_t stg[5] = {G_DARK, G_X, G_DAAK, G_DAAB, G_DARB};  // dr dw dk da db
+        if (p_nv == 64) {
+            if (lane == 0 && warp < 5) {
+                const CUtensorMap* map = warp == 0 ? &tm_dr : warp == 1 ? &tm_dw : warp == 2 ? &tm_dk
+                                       : warp == 3 ? &tm_da : &tm_db;
+                tma_store_3d(map, sbase + gt(stg[warp]), 0, p_cy, p_cz);
+                bulk_commit();
+            }
+        } else {
+            __nv_bfloat16* outs[5] = {dr, dw, dk, da, db};
+            for (int i = tid; i < 5 * 64 * 8; i += kThreads) {
+                const int which = i / 512, rem = i % 512, t = rem >> 3, chk = rem & 7;
+                if (t >= p_nv) continue;
+                const long long e = kHf ? (((p_crow / T) * H + p_h) * (long long)T + (p_crow % T) + t) * 64
+                                        : ((p_crow + t) * H + p_h) * 64;
+                *reinterpret_cast<uint4*>(outs[which] + e + 8 * chk) =
+                    *reinterpret_cast<const uint4*>(smem + gt(stg[which]) + sw(t, chk));
+            }
+        }
+        p_nv = 0;
+    };
+
     while (it >= 0) {
     const int h = I.h, nv = I.nv;
     const long long crow = I.crow;
@@ -380,6 +420,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
             *reinterpret_cast<float4*>(wt + warp * 64 + h1) = make_float4(incl[4], incl[5], incl[6], incl[7]);
         }
         if (__syncthreads_or(timed_out)) goto teardown;
+        flush();  // the previous chunk's outputs
         if (warp == 0) {
             const int ch = cswz(2 * lane);
             float2 gL = make_float2(0.f, 0.f);
@@ -821,6 +862,23 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
             tmem_ld16x32(ta + C_DAB, dab);
             tmem_ld_wait();
         }
+        // the original r, k, a, b at this thread's fragment positions: ldmatrix of the
+        // 16 x 32 block gives register 4 (j / 2) + 2 (j % 2) + hr = (row g + 8 hr,
+        // columns 8 j + 2 q, +1)
+        uint32_t fr_r[8], fr_k[8], fr_a[8], fr_b[8];
+        {
+            const int lrow = 16 * wq + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t o = sw(lrow, 4 * wh + 2 * hh + (lane >> 4));
+                ldsm_x4(sbase + gt(G_SP) + o, fr_r[4 * hh], fr_r[4 * hh + 1], fr_r[4 * hh + 2], fr_r[4 * hh + 3]);
+                ldsm_x4(sbase + gt(G_AB) + o, fr_k[4 * hh], fr_k[4 * hh + 1], fr_k[4 * hh + 2], fr_k[4 * hh + 3]);
+                ldsm_x4(sbase + gt(G_AAK) + o, fr_a[4 * hh], fr_a[4 * hh + 1], fr_a[4 * hh + 2], fr_a[4 * hh + 3]);
+                ldsm_x4(sbase + gt(G_ARB) + o, fr_b[4 * hh], fr_b[4 * hh + 1], fr_b[4 * hh + 2], fr_b[4 * hh + 3]);
+            }
+        }
+        // a bf16 pair (low half first) as two floats: bf16 is the top half of an fp32
+        auto bf2 = [](uint32_t u) { return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)); };
         float hv[16], fv[16];
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
@@ -833,11 +891,9 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                 const float2 E2 = *reinterpret_cast<const float2*>(Ef + eidx(t, cidx));
                 const float2 Em = t > 0 ? *reinterpret_cast<const float2*>(Ef + eidx(t - 1, cidx))
                                         : make_float2(em0[cidx], em0[cidx + 1]);
-                const uint32_t bo = swe(t, cidx);
-                const float2 r2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_SP) + bo));
-                const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_AB) + bo));
-                const float2 a2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_AAK) + bo));
-                const float2 b2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + gt(G_ARB) + bo));
+                const int fi = 4 * (j >> 1) + 2 * (j & 1) + hr;
+                const float2 r2 = bf2(fr_r[fi]), k2 = bf2(fr_k[fi]), a2 = bf2(fr_a[fi]),
+                             b2 = bf2(fr_b[fi]);
                 const float Ee[2] = {E2.x, E2.y}, Eme[2] = {Em.x, Em.y};
                 const float re[2] = {r2.x, r2.y}, ke[2] = {k2.x, k2.y}, ae[2] = {a2.x, a2.y},
                             be[2] = {b2.x, b2.y};
@@ -906,30 +962,18 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
             }
         frag_to_tile(sbase + gt(G_X), 16 * wq, 4 * wh, hv, lane, PackB{});  // dw
         fence_proxy_async();
-        __syncthreads();
-        const uint32_t stg[5] = {G_DARK, G_X, G_DAAK, G_DAAB, G_DARB};  // dr dw dk da db
-        if (nv == 64) {
-            if (lane == 0 && warp < 5) {  // one tile store per warp
-                const CUtensorMap* map = warp == 0 ? &tm_dr : warp == 1 ? &tm_dw : warp == 2 ? &tm_dk
-                                       : warp == 3 ? &tm_da : &tm_db;
-                tma_store_3d(map, sbase + gt(stg[warp]), 0, cy, cz);
-                bulk_commit();
-            }
-        } else {
-            // a partial chunk: rows < nv only (the rows after belong to another sequence)
-            __nv_bfloat16* outs[5] = {dr, dw, dk, da, db};
-            for (int i = tid; i < 5 * 64 * 8; i += kThreads) {
-                const int which = i / 512, rem = i % 512, t = rem >> 3, chk = rem & 7;
-                if (t >= nv) continue;
-                const long long e = kHf ? (((crow / T) * H + h) * (long long)T + (crow % T) + t) * 64
-                                        : ((crow + t) * H + h) * 64;
-                *reinterpret_cast<uint4*>(outs[which] + e + 8 * chk) =
-                    *reinterpret_cast<const uint4*>(smem + gt(stg[which]) + sw(t, chk));
-            }
-        }
+        // The stores leave after the next CTA barrier (the next chunk's first, or the
+        // one after the loop), which orders them after every thread's staging writes.
+        p_nv = nv;
+        p_h = h;
+        p_cy = cy;
+        p_cz = cz;
+        p_crow = crow;
     }
 
     }  // chunks
+    __syncthreads();
+    flush();
     if (lane == 0 && warp < 5) bulk_wait0();  // the last output stores are complete
 
 teardown:
@@ -995,6 +1039,30 @@ inline cudaError_t launch_grad(const void* r, const void* w, const void* k, cons
 
 }  // namespace cbwd
 
+// A second stream and two events per (host thread, device): the checkpointing forward
+// and the reversed run are independent, and run side by side so that each one's last
+// partial wave of CTAs overlaps the other.
+struct ForkJoin {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+inline cudaError_t fork_join_for_current_device(ForkJoin*& out) {
+    constexpr int kMaxDev = 64;
+    thread_local ForkJoin fj[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    ForkJoin& f = fj[dev];
+    if (!f.side) {
+        if ((e = cudaStreamCreateWithFlags(&f.side, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&f.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&f.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    out = &f;
+    return cudaSuccess;
+}
+
 inline size_t bwd_chunked_workspace_bytes(long long rows, int N, int H) {
     return cbwd::ws_layout(rows, N, H).total;
 }
@@ -1021,7 +1089,12 @@ inline cudaError_t launch_bwd_chunked(const void* r, const void* w, const void* 
     // 1. reversed sequence offsets
     prep_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, T, N, cur);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 2. forward with per-chunk checkpoints, no outputs
+    // 2. forward with per-chunk checkpoints, no outputs, and 3. (below) the reversed run,
+    //    side by side: the reversed run goes to a second stream forked after prep
+    ForkJoin* fj = nullptr;
+    if ((e = fork_join_for_current_device(fj)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(fj->fork, stream)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(fj->side, fj->fork, 0)) != cudaSuccess) return e;
     chunked::Extras exF;
     exF.ck = ckF;
     exF.ck_slots = (int)lay.slotsF;
@@ -1044,9 +1117,11 @@ inline cudaError_t launch_bwd_chunked(const void* r, const void* w, const void* 
     chunked::Extras exR;
     exR.ck = ckR;
     exR.ck_slots = (int)lay.slotsR;
-    if ((e = launch_chunked_rev(rin, B, dsT, ds0, (int)lay.rowsR, H, N, cur, exR, stream)) !=
+    if ((e = launch_chunked_rev(rin, B, dsT, ds0, (int)lay.rowsR, H, N, cur, exR, fj->side)) !=
         cudaSuccess)
         return e;
+    if ((e = cudaEventRecord(fj->join, fj->side)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(stream, fj->join, 0)) != cudaSuccess) return e;
     // 4. per-chunk gradients
     e = head_first ? launch_grad<true>(r, w, k, v, a, b, dout, mask, dr, dw, dk, da, db, B, T, H,
                                        N, cu_seqlens, cur, ckF, ckR, lay, stream)
