@@ -363,6 +363,28 @@ __device__ __forceinline__ void issue_loads(const Ctx& cx, int c0, int par) {
     }
 }
 
+// Input tile i (0..5: r, a, k, b, w, v; Gated DeltaNet 0..2: q, k, v) of the chunk at
+// token c0 into layout `par`, by the calling thread (the barrier is armed elsewhere).
+// Each TMA instruction takes a few hundred cycles to issue, so a chunk's loads come
+// from one thread of each of several warps.
+template <bool kGdn, bool kHf>
+__device__ __forceinline__ void issue_load_one(const Ctx& cx, int c0, int par, int i) {
+    const LayR L = lay_of(par);
+    const int cy = kHf ? cx.tma_y + c0 : cx.tma_y;
+    const int cz = kHf ? cx.tma_z : cx.tma_z + c0;
+    const CUtensorMap* map;
+    uint32_t dst;
+    if constexpr (kGdn) {
+        map = i == 0 ? cx.tm_r : i == 1 ? cx.tm_k : cx.tm_v;
+        dst = i == 0 ? L.R : i == 1 ? L.K : L.V;
+    } else {
+        map = i == 0 ? cx.tm_r : i == 1 ? cx.tm_a : i == 2 ? cx.tm_k : i == 3 ? cx.tm_b
+            : i == 4 ? cx.tm_w : cx.tm_v;
+        dst = i == 0 ? L.R : i == 1 ? L.A : i == 2 ? L.K : i == 3 ? L.B : i == 4 ? L.W : L.V;
+    }
+    sm100::tma_load_3d(cx.sbase + dst, map, cx.bar_tma, 0, cy, cz);
+}
+
 // kRev, every thread: 12 of the chunk's 6 x 64 x 8 16-byte pieces by cp.async, each
 // from its original token (zero-filled where the step has no transition or no write),
 // then the mbarrier tracks this thread's copies (one plain arrive after the next CTA
@@ -625,6 +647,9 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
             // (M = 128), the transposes the output product takes as MN-major operands.
             if (tid == 0) {
                 tc_fence_after();
+                // the next chunk's input barrier, armed now (its loads are issued after
+                // MMA-U, several CTA barriers later)
+                if (!kRev && has_next) mbar_arrive_expect_tx(cx.bar_tma, (kGdn ? 3 : 6) * kTile);
                 constexpr uint32_t id64 = idesc_bf16(64, 64, false, false);
                 constexpr uint32_t id128 = idesc_bf16(128, 64, false, false);
 #pragma unroll
@@ -927,8 +952,8 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
         if (has_next) {
             if constexpr (kRev)
                 issue_loads_rev(cx, c0 + 64, par ^ 1);
-            else if (warp == 1)
-                issue_loads<kGdn, kHf>(cx, c0 + 64, par ^ 1);
+            else if (lane == 0 && warp >= 1 && warp <= (kGdn ? 3 : 6))
+                issue_load_one<kGdn, kHf>(cx, c0 + 64, par ^ 1, warp - 1);
             cx.tma_par_last = par ^ 1;
         }
 
