@@ -556,8 +556,9 @@ def bwd_leg(args, device, stream, bwd_fn, hbm_peak, peak_kind, max_over_ranks, b
 
 
 def wkv7_bwd_workspace_nbytes(B, T, H):
+    """The workspace of the kernel family wkv7_bwd picks for bf16 inputs."""
     from linear_attention_rnn_wkv7_b200.wkv7 import wkv7_bwd_workspace_bytes
-    return wkv7_bwd_workspace_bytes(B, T, H)
+    return wkv7_bwd_workspace_bytes(B, T, H, dtype=torch.bfloat16, algo="auto")
 
 
 def decode_leg(device, stream, wkv7_step, hbm_peak, peak_kind, max_over_ranks, barrier, rank,

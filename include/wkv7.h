@@ -145,8 +145,8 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
  *                                        must not alias an input)
  *   ds0            [N, H, K, V]  fp32    dL/ds0, or NULL to skip
  *   workspace      device buffer of at least wkv7_bwd_workspace_bytes(B, T, H, K, V, N)
- *                  bytes (16-byte aligned; the caller owns it; contents on return are
- *                  scratch)
+ *                  bytes, or of wkv7_bwd_workspace_bytes_algo for the family that runs
+ *                  (16-byte aligned; the caller owns it; contents on return are scratch)
  *
  * K = V = 64 only.  A masked token passes the state gradient through and has zero
  * dw, dk, dv, da, db.  Two kernel families (wkv7_bwd picks as AUTO does):
@@ -166,6 +166,18 @@ wkv7_status wkv7_step(const void* r, const void* w, const void* k, const void* v
  * The workspace bound covers both.
  */
 size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N);
+
+/*
+ * wkv7_bwd_workspace_bytes_algo -- the workspace one kernel family needs (what
+ * wkv7_bwd_with_algo checks): the chunked form (dtype bf16 with WKV7_ALGO_CHUNKED or
+ * WKV7_ALGO_AUTO) needs the reversed-sequence offsets and the fp16 state checkpoints of
+ * its two passes, about 2 x 8 KiB per 64-token chunk and head; the fp32 recurrences
+ * (WKV7_ALGO_RECURRENT, or AUTO with fp32) the states every 8 tokens and every token's
+ * u.  Returns 0 for unsupported arguments (K != 64, fp32 with WKV7_ALGO_CHUNKED).
+ * wkv7_bwd_workspace_bytes is the larger of the two.
+ */
+size_t wkv7_bwd_workspace_bytes_algo(int B, int T, int H, int K, int V, int N, wkv7_dtype dtype,
+                                     wkv7_algo algo);
 
 wkv7_status wkv7_bwd(const void* r, const void* w, const void* k, const void* v, const void* a,
                      const void* b, const float* s0, const uint8_t* mask, const void* dout,

@@ -289,11 +289,21 @@ wkv7_status wkv7_sane_step(const void* r, const void* w, const void* k, const vo
     return err == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
 }
 
-size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N) {
+size_t wkv7_bwd_workspace_bytes_algo(int B, int T, int H, int K, int V, int N, wkv7_dtype dtype,
+                                     wkv7_algo algo) {
     if (B < 0 || T < 0 || H <= 0 || N < 0 || K != 64 || V != 64) return 0;
+    if (dtype != WKV7_BF16 && dtype != WKV7_F32) return 0;
     const long long rows = (long long)B * T;
-    const size_t rec = wkv7::bwd::workspace_floats(rows, N, H) * sizeof(float);
-    const size_t chk = wkv7::bwd_chunked_workspace_bytes(rows, N, H);
+    if (algo == WKV7_ALGO_CHUNKED || (algo == WKV7_ALGO_AUTO && dtype == WKV7_BF16))
+        return dtype == WKV7_BF16 ? wkv7::bwd_chunked_workspace_bytes(rows, N, H) : 0;
+    if (algo == WKV7_ALGO_RECURRENT || algo == WKV7_ALGO_AUTO)
+        return wkv7::bwd::workspace_floats(rows, N, H) * sizeof(float);
+    return 0;
+}
+
+size_t wkv7_bwd_workspace_bytes(int B, int T, int H, int K, int V, int N) {
+    const size_t rec = wkv7_bwd_workspace_bytes_algo(B, T, H, K, V, N, WKV7_F32, WKV7_ALGO_RECURRENT);
+    const size_t chk = wkv7_bwd_workspace_bytes_algo(B, T, H, K, V, N, WKV7_BF16, WKV7_ALGO_CHUNKED);
     return rec > chk ? rec : chk;
 }
 
@@ -342,7 +352,8 @@ wkv7_status wkv7_bwd_with_algo(const void* r, const void* w, const void* k, cons
     for (const void* x : outs)
         for (const void* y : ins)
             if (x && x == y) return WKV7_ERR_INVALID_ARG;
-    if (!ok_ptr(workspace) || workspace_bytes < wkv7_bwd_workspace_bytes(B, T, H, K, V, N))
+    if (!ok_ptr(workspace) ||
+        workspace_bytes < wkv7_bwd_workspace_bytes_algo(B, T, H, K, V, N, dtype, algo))
         return WKV7_ERR_INVALID_ARG;
     if (algo == WKV7_ALGO_CHUNKED && dtype != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
@@ -377,7 +388,7 @@ wkv7_status wkv7_bwd_noalloc(const void* r, const void* w, const void* k, const 
                              void* dw, void* dk, void* dv, void* da, void* db, float* ds0, int B,
                              int T, int H, int K, int V, const int32_t* cu_seqlens, int N,
                              wkv7_layout layout, wkv7_dtype dtype, void* stream) {
-    const size_t need = wkv7_bwd_workspace_bytes(B, T, H, K, V, N);
+    const size_t need = wkv7_bwd_workspace_bytes_algo(B, T, H, K, V, N, dtype, WKV7_ALGO_AUTO);
     if (need > kStaticScratchBytes) return WKV7_ERR_UNSUPPORTED;
     void* scratch = static_scratch_on_current_device();
     if (!scratch) return WKV7_ERR_CUDA;

@@ -53,6 +53,8 @@ def library() -> ctypes.CDLL:
         lib.wkv7_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
         lib.wkv7_bwd.restype = i
         lib.wkv7_bwd.argtypes = [p] * 17 + [i, i, i, i, i, p, i, i, i, p, ctypes.c_size_t, p]
+        lib.wkv7_bwd_workspace_bytes_algo.restype = ctypes.c_size_t
+        lib.wkv7_bwd_workspace_bytes_algo.argtypes = [i] * 8
         lib.wkv7_bwd_with_algo.restype = i
         lib.wkv7_bwd_with_algo.argtypes = ([p] * 17 + [i, i, i, i, i, p, i, i, i, i, p,
                                                        ctypes.c_size_t, p])
@@ -273,8 +275,15 @@ def wkv7_sane_step(r, w, k, v, a, b, tau, do_sane, state, o=None):
     return o
 
 
-def wkv7_bwd_workspace_bytes(B, T, H, K=64, V=64, N=None) -> int:
-    return int(library().wkv7_bwd_workspace_bytes(B, T, H, K, V, B if N is None else N))
+def wkv7_bwd_workspace_bytes(B, T, H, K=64, V=64, N=None, dtype=None, algo: str = None) -> int:
+    """Workspace bytes of wkv7_bwd: with dtype (torch.bfloat16 / torch.float32) and algo,
+    the need of the kernel family that runs; without, the larger of the two."""
+    N = B if N is None else N
+    if dtype is None and algo is None:
+        return int(library().wkv7_bwd_workspace_bytes(B, T, H, K, V, N))
+    code = 0 if (dtype is None or dtype == torch.bfloat16) else 1
+    return int(library().wkv7_bwd_workspace_bytes_algo(B, T, H, K, V, N, code,
+                                                        ALGO[algo or "auto"]))
 
 
 def wkv7_bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=None,
@@ -312,7 +321,7 @@ def wkv7_bwd(r, w, k, v, a, b, dout, s0=None, mask=None, dsT=None, cu_seqlens=No
         if mask.dtype == torch.bool:
             mask = mask.to(torch.uint8)
         _check(mask, "mask", torch.uint8, (B, T))
-    nbytes = wkv7_bwd_workspace_bytes(B, T, H, K, V, N)
+    nbytes = wkv7_bwd_workspace_bytes(B, T, H, K, V, N, dtype=dt, algo=algo)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=r.device)
     else:

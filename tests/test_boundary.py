@@ -185,6 +185,15 @@ def test_bwd_rejects_bad_arguments(lib):
     ck_r = al(ck_f + H * (rows // 64 + N + 1) * 8192)
     chk = al(ck_r + H * (rows_r // 64 + N + 1) * 8192)
     assert need == max(rec, chk)
+    q = lib.wkv7_bwd_workspace_bytes_algo
+    q.restype = ctypes.c_size_t
+    AUTO, RECURRENT, CHUNKED = 0, 1, 2
+    assert q(1, 16, 2, 64, 64, 1, BF16, AUTO) == chk
+    assert q(1, 16, 2, 64, 64, 1, BF16, CHUNKED) == chk
+    assert q(1, 16, 2, 64, 64, 1, BF16, RECURRENT) == rec
+    assert q(1, 16, 2, 64, 64, 1, F32, AUTO) == rec
+    assert q(1, 16, 2, 64, 64, 1, F32, CHUNKED) == 0
+    assert q(1, 16, 2, 128, 128, 1, BF16, AUTO) == 0
     assert lib.wkv7_bwd_workspace_bytes(1, 16, 2, 128, 128, 1) == 0
 
     def call(B=1, T=16, H=2, K=64, V=64, dtype=BF16, d=dout, o=outs, w=ws, n=need, N=None,
@@ -198,7 +207,8 @@ def test_bwd_rejects_bad_arguments(lib):
     assert call(d=None) == ERR_INVALID_ARG
     assert call(d=ctypes.c_void_p(P + 0x8008)) == ERR_INVALID_ARG  # misaligned dout
     assert call(o=[ins[0]] + outs[1:]) == ERR_INVALID_ARG  # dr aliases r
-    assert call(n=need - 1) == ERR_INVALID_ARG  # workspace too small
+    assert call(n=chk - 1) == ERR_INVALID_ARG  # workspace too small (bf16: the chunked form)
+    assert call(n=rec - 1, dtype=F32) == ERR_INVALID_ARG  # (fp32: the recurrences)
     assert call(w=None) == ERR_INVALID_ARG
     assert call(N=2) == ERR_INVALID_ARG  # N must equal B without cu_seqlens
     assert call(layout=3) == ERR_INVALID_ARG
