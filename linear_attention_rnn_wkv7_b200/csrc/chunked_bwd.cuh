@@ -51,7 +51,7 @@ namespace cbwd {
 using namespace chunked;
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;  // the gradient kernel: 16 warps
 
 // ---------------------------------------------------------------------------------
 // Workspace layout (bytes, each region 256-aligned).
@@ -160,8 +160,8 @@ constexpr uint32_t GOFF_EM0 = GOFF_R + 256;          // E_{-1} per channel (64 f
 constexpr uint32_t GOFF_RAW = GOFF_EM0 + 256;        // raw r and dO of token 63 (2 x 64 fp32)
 constexpr uint32_t GOFF_TOT = GOFF_RAW + 512;        // scan totals [4 quadrants][64]
 constexpr uint32_t GOFF_NEXT = GOFF_TOT + 1024;      // the CTA's next work item (and index)
-constexpr uint32_t GOFF_RP = GOFF_NEXT + 128;        // rowsum(S0 P) halves [2][64] (fixed order)
-constexpr uint32_t kGSmemBytes = GOFF_RP + 512;
+constexpr uint32_t GOFF_RP = GOFF_NEXT + 128;        // rowsum(S0 P) quarters [4][64] (fixed order)
+constexpr uint32_t kGSmemBytes = GOFF_RP + 1024;
 static_assert(kGSmemBytes <= 232448, "fits one CTA per SM");
 constexpr uint32_t kGTmemCols = 512;
 // TMEM columns (every accumulator M = 64): C0..C2 hold each phase's products for its
@@ -193,6 +193,38 @@ __device__ __forceinline__ void acc_to_tile(uint32_t tmem, uint32_t col, uint32_
                 }
     }
     frag_to_tile(tile, 16 * wq, 4 * wh, v, lane, pk);
+}
+
+// One 16 x 16 block in fragment layout (sm100::tmem_ld16x16) to a 128B-swizzled tile:
+// rows row0 .. row0 + 15, 16-byte chunks chunk0, chunk0 + 1 (one stmatrix.x4).
+template <typename Pack>
+__device__ __forceinline__ void frag8_to_tile(uint32_t tile, int row0, int chunk0, const float (&v)[8],
+                                              int lane, Pack pk) {
+    const int mi = lane >> 3;
+    const uint32_t addr = tile + sw(row0 + 8 * (mi & 1) + (lane & 7), chunk0 + (mi >> 1));
+    stsm_x4(addr, pk(v[0], v[1]), pk(v[2], v[3]), pk(v[4], v[5]), pk(v[6], v[7]));
+}
+// One warp's 16 x 16 block (rows 16 wq .., columns 16 wc ..) of the M = 64 accumulator at
+// TMEM column `col` as a 16-bit tile; mode 1 keeps s <= t, mode 2 keeps s < t.
+template <typename Pack>
+__device__ __forceinline__ void acc16_to_tile(uint32_t tmem, uint32_t col, uint32_t tile, int wq,
+                                              int wc, int lane, int mode, Pack pk) {
+    float v[8];
+    sm100::tmem_ld16x16(tmem + ((uint32_t)(32 * wq) << 16) + col + 16 * wc, v);
+    sm100::tmem_ld_wait();
+    if (mode) {
+        const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = 16 * wq + g + 8 * hr, s = 16 * wc + 8 * j + 2 * q + e;
+                    if (mode == 1 ? s > t : s >= t) v[4 * j + 2 * hr + e] = 0.f;
+                }
+    }
+    frag8_to_tile(tile, 16 * wq, 2 * wc, v, lane, pk);
 }
 
 // D (+)= A B over K = 64 (four K16 steps) from 64-row tiles; a_mn / b_mn: the tile is
@@ -278,7 +310,10 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
             __nv_bfloat16* __restrict__ db) {
     extern __shared__ __align__(1024) uint8_t smem[];
     using namespace sm100;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wq = warp & 3, wh = warp >> 2;
+    // 16 warps: wq = TMEM lane quadrant (rows 16 wq .. of an M = 64 accumulator), wc =
+    // 16-column quarter of it in the epilogues; warps 0..7 keep the single-thread and
+    // warp roles (MMA issue, T, the A_ab inverses, TMA issue)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wq = warp & 3, wc = warp >> 2;
     const int g = lane >> 2, q = lane & 3;
     const int total = slotsF * H;  // below 2^31 (checked on the host)
 
@@ -290,7 +325,6 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     float* em0 = reinterpret_cast<float*>(smem + GOFF_EM0);
     float* raw = reinterpret_cast<float*>(smem + GOFF_RAW);
     float* tot = reinterpret_cast<float*>(smem + GOFF_TOT);
-    float* Rp = reinterpret_cast<float*>(smem + GOFF_RP);
     float* Ef = reinterpret_cast<float*>(smem + gt(G_E));
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GOFF_MISC + 32);
     int timed_out = 0;
@@ -343,6 +377,8 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         __syncwarp();
         if (lane < 9) load_in(I, lane);
     }
+    // rowsum(S0 P) partials, one per 16-column quarter (added in a fixed order)
+    float* Rq = reinterpret_cast<float*>(smem + GOFF_RP);
 
     // The previous chunk's outputs (dr dw dk da db), staged in the dA tiles and X: five
     // TMA tile stores (one per warp), or the rows < nv copied for a partial chunk (the
@@ -381,135 +417,114 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     wait_or_abort(bar_tma, tph, timed_out);
     tph ^= 1;
 
-    // ---- prologue: prefix sums of w (mask folded), E, and the operands --------------
+    // ---- prologue: prefix sums of w (mask folded), E, and the operands; thread = one
+    //      token t of the chunk, channels 8 j .. 8 j + 7 -------------------------------
     {
-        float* scratch = reinterpret_cast<float*>(smem + gt(G_SP));
-        const int j = tid & 7, t0 = 2 * (tid >> 3);
-        const bool ina = t0 < nv, inb = t0 + 1 < nv;
-        const bool va = ina && (!mask || mask[crow + t0] != 0);
-        const bool vb = inb && (!mask || mask[crow + t0 + 1] != 0);
-        const uint32_t offa = sw(t0, j), offb = sw(t0 + 1, j);
+        float* scr = reinterpret_cast<float*>(smem + gt(G_SP));  // warp totals [16][64], g_L
+        float* pre_s = reinterpret_cast<float*>(smem + gt(G_DT));  // exclusive prefixes [16][64]
+        const int j = tid & 7, t = tid >> 3;
+        const bool in = t < nv, val = in && (!mask || mask[crow + t] != 0);
+        const uint32_t off = sw(t, j);
         const int h0 = cswz(8 * j), h1 = cswz(8 * j + 4);
-        float wa[8], wb[8], incl[8];
+        float wv[8], incl[8];
         {
-            const uint32_t ma = va ? 0xFFFFFFFFu : 0u, mb = vb ? 0xFFFFFFFFu : 0u;
-            uint4 qa = *reinterpret_cast<const uint4*>(smem + gt(G_W) + offa);
-            uint4 qb = *reinterpret_cast<const uint4*>(smem + gt(G_W) + offb);
-            qa.x &= ma; qa.y &= ma; qa.z &= ma; qa.w &= ma;
-            qb.x &= mb; qb.y &= mb; qb.z &= mb; qb.w &= mb;
-            unpack8(qa, wa);
-            unpack8(qb, wb);
+            uint4 qa = *reinterpret_cast<const uint4*>(smem + gt(G_W) + off);
+            if (!val) qa = make_uint4(0, 0, 0, 0);  // a masked token's w is zero
+            unpack8(qa, wv);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            wa[e] *= kLog2e;
-            wb[e] *= kLog2e;
-            incl[e] = wa[e] + wb[e];
+            wv[e] *= kLog2e;  // log decays in log2 units from here on
+            incl[e] = wv[e];
         }
 #pragma unroll
-        for (int d = 8; d < 32; d *= 2) {
+        for (int d = 8; d < 32; d *= 2) {  // the warp's four tokens
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float up = __shfl_up_sync(0xffffffffu, incl[e], d);
                 if (lane >= d) incl[e] += up;
             }
         }
-        float* wt = scratch + SCR_TOT;
         if (lane >= 24) {
-            *reinterpret_cast<float4*>(wt + warp * 64 + h0) = make_float4(incl[0], incl[1], incl[2], incl[3]);
-            *reinterpret_cast<float4*>(wt + warp * 64 + h1) = make_float4(incl[4], incl[5], incl[6], incl[7]);
+            *reinterpret_cast<float4*>(scr + warp * 64 + h0) = make_float4(incl[0], incl[1], incl[2], incl[3]);
+            *reinterpret_cast<float4*>(scr + warp * 64 + h1) = make_float4(incl[4], incl[5], incl[6], incl[7]);
         }
         if (__syncthreads_or(timed_out)) goto teardown;
         flush();  // the previous chunk's outputs
-        if (warp == 0) {
+        if (warp == 0) {  // per channel pair: exclusive prefixes over the warps, g_L, e^{g_L}
             const int ch = cswz(2 * lane);
             float2 gL = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int w2 = 0; w2 < 8; ++w2) {
-                const float2 x = *reinterpret_cast<const float2*>(wt + w2 * 64 + ch);
-                *reinterpret_cast<float2*>(scratch + SCR_PRE + w2 * 64 + ch) = gL;
+            for (int w2 = 0; w2 < kThreads / 32; ++w2) {
+                const float2 x = *reinterpret_cast<const float2*>(scr + w2 * 64 + ch);
+                *reinterpret_cast<float2*>(pre_s + w2 * 64 + ch) = gL;
                 gL.x += x.x;
                 gL.y += x.y;
             }
-            *reinterpret_cast<float2*>(scratch + SCR_C + ch) = gL;
-            // plain channel order from here on: ch holds channels 2 lane, 2 lane + 1 (cswz
-            // permutes 4-channel groups, so the pair stays together)
-            const int c2 = 2 * lane;
-            const float2 gLp = *reinterpret_cast<const float2*>(scratch + SCR_C + ch);
-            gam[c2] = ex2(gLp.x);
-            gam[c2 + 1] = ex2(gLp.y);
+            *reinterpret_cast<float2*>(scr + 1024 + ch) = gL;
+            gam[2 * lane] = ex2(gL.x);  // plain channel order (cswz keeps pairs together)
+            gam[2 * lane + 1] = ex2(gL.y);
         }
         __syncthreads();
-        float ga[8];
+        float ga[8], cc[8], ec[8];
         {
-            const float4 x0 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + h0);
-            const float4 x1 = *reinterpret_cast<const float4*>(scratch + SCR_PRE + warp * 64 + h1);
+            const float4 x0 = *reinterpret_cast<const float4*>(pre_s + warp * 64 + h0);
+            const float4 x1 = *reinterpret_cast<const float4*>(pre_s + warp * 64 + h1);
             const float pre[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ga[e] = pre[e] + (incl[e] - wb[e]);
+            for (int e = 0; e < 8; ++e) ga[e] = pre[e] + incl[e];  // g at token t
         }
-        float cc[8], ec[8];
-        *reinterpret_cast<float4*>(cc) = *reinterpret_cast<const float4*>(scratch + SCR_C + h0);
-        *reinterpret_cast<float4*>(cc + 4) = *reinterpret_cast<const float4*>(scratch + SCR_C + h1);
+        *reinterpret_cast<float4*>(cc) = *reinterpret_cast<const float4*>(scr + 1024 + h0);
+        *reinterpret_cast<float4*>(cc + 4) = *reinterpret_cast<const float4*>(scr + 1024 + h1);
 #pragma unroll
         for (int e = 0; e < 8; ++e) ec[e] = gam[8 * j + e];
-        float Ep[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) Ep[e] = ex2(clamp2(ga[e] - wa[e] - cc[e]));
-        if (t0 == 0) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) em0[8 * j + e] = Ep[e];
-        }
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const uint32_t off = it ? offb : offa;
-            const bool val = it ? vb : va;
-            const bool in = it ? inb : ina;
-            const int t = t0 + it;
-            float rv[8], av[8], kv[8], bv[8], vv[8], dv[8];
-            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_R) + off), rv);
-            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_A) + off), av);
-            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_K) + off), kv);
-            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_B) + off), bv);
-            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_V) + off), vv);
-            unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_DO) + off), dv);
-            if (t == 63) {  // raw r and dO of the last token (dSL = G - r do^T)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    raw[8 * j + e] = rv[e];
-                    raw[64 + 8 * j + e] = dv[e];
-                }
-            }
-            float rt[8], at[8], kt[8], bt[8], ab[8], rb[8], Ev[8];
+        float rv[8], av[8], kv[8], bv[8], vv[8], dv[8];
+        unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_R) + off), rv);
+        unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_A) + off), av);
+        unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_K) + off), kv);
+        unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_B) + off), bv);
+        unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_V) + off), vv);
+        unpack8(*reinterpret_cast<const uint4*>(smem + gt(G_DO) + off), dv);
+        if (t == 63) {  // raw r and dO of the last token (dSL = G - r do^T)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float gg = it ? ga[e] + wb[e] : ga[e];
-                const float d = clamp2(gg - cc[e]);
-                const float E = ex2(d);
-                const float inv = val ? ex2(-d) : 0.f;
-                const float ep = val ? Ep[e] : 0.f;
-                rt[e] = in ? rv[e] * E : 0.f;
-                at[e] = av[e] * ep;
-                kt[e] = kv[e] * inv;
-                bt[e] = bv[e] * inv;
-                ab[e] = at[e] * ec[e];  // Abar = a~ e^{g_L}
-                rb[e] = rt[e] * ec[e];  // Rbar = r~ e^{g_L}
-                Ev[e] = E;
-                Ep[e] = E;
-                if (!in) dv[e] = 0.f;
+                raw[8 * j + e] = rv[e];
+                raw[64 + 8 * j + e] = dv[e];
             }
-            *reinterpret_cast<uint4*>(smem + gt(G_R) + off) = pack8(rt);
-            *reinterpret_cast<uint4*>(smem + gt(G_A) + off) = pack8(at);
-            *reinterpret_cast<uint4*>(smem + gt(G_K) + off) = pack8(kt);
-            *reinterpret_cast<uint4*>(smem + gt(G_B) + off) = pack8(bt);
-            *reinterpret_cast<uint4*>(smem + gt(G_W) + off) = pack8h(ab);
-            *reinterpret_cast<uint4*>(smem + gt(G_RB) + off) = pack8h(rb);
-            *reinterpret_cast<uint4*>(smem + gt(G_BH) + off) = pack8h(bt);
-            *reinterpret_cast<uint4*>(smem + gt(G_V) + off) = pack8h(vv);
-            *reinterpret_cast<uint4*>(smem + gt(G_DO) + off) = pack8h(dv);
-            *reinterpret_cast<float4*>(Ef + eidx(t, 8 * j)) = make_float4(Ev[0], Ev[1], Ev[2], Ev[3]);
-            *reinterpret_cast<float4*>(Ef + eidx(t, 8 * j + 4)) = make_float4(Ev[4], Ev[5], Ev[6], Ev[7]);
         }
+        float Ev[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float d = clamp2(ga[e] - cc[e]);
+            const float E = ex2(d);                              // e^{g_t - g_L}
+            const float Ep = ex2(clamp2(ga[e] - wv[e] - cc[e]));  // e^{g_{t-1} - g_L}
+            if (t == 0) em0[8 * j + e] = Ep;
+            const float inv = val ? ex2(-d) : 0.f;
+            const float ep = val ? Ep : 0.f;
+            rv[e] = in ? rv[e] * E : 0.f;  // r~
+            av[e] = av[e] * ep;            // a~
+            kv[e] = kv[e] * inv;           // k~
+            bv[e] = bv[e] * inv;           // b~
+            Ev[e] = E;
+            if (!in) dv[e] = 0.f;
+        }
+        float ab[8], rb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            ab[e] = av[e] * ec[e];  // Abar = a~ e^{g_L}
+            rb[e] = rv[e] * ec[e];  // Rbar = r~ e^{g_L}
+        }
+        *reinterpret_cast<uint4*>(smem + gt(G_R) + off) = pack8(rv);
+        *reinterpret_cast<uint4*>(smem + gt(G_A) + off) = pack8(av);
+        *reinterpret_cast<uint4*>(smem + gt(G_K) + off) = pack8(kv);
+        *reinterpret_cast<uint4*>(smem + gt(G_B) + off) = pack8(bv);
+        *reinterpret_cast<uint4*>(smem + gt(G_W) + off) = pack8h(ab);
+        *reinterpret_cast<uint4*>(smem + gt(G_RB) + off) = pack8h(rb);
+        *reinterpret_cast<uint4*>(smem + gt(G_BH) + off) = pack8h(bv);
+        *reinterpret_cast<uint4*>(smem + gt(G_V) + off) = pack8h(vv);
+        *reinterpret_cast<uint4*>(smem + gt(G_DO) + off) = pack8h(dv);
+        *reinterpret_cast<float4*>(Ef + eidx(t, 8 * j)) = make_float4(Ev[0], Ev[1], Ev[2], Ev[3]);
+        *reinterpret_cast<float4*>(Ef + eidx(t, 8 * j + 4)) = make_float4(Ev[4], Ev[5], Ev[6], Ev[7]);
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -523,44 +538,42 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         mma64(tmem + C2, sbase + gt(G_R), false, sbase + gt(G_B), false, true, false);
         umma_commit(bar_mma);
     }
-    // While it runs: dSL (fp16) and R = e^{g_L} rowsum(S0 dSL).
+    // While it runs: dSL (fp16) and R = e^{g_L} rowsum(S0 dSL); thread = state row c,
+    // 8 of its columns.
     {
-        const int row = tid >> 2, qq = tid & 3;  // state row (channel) and 16 of its columns
+        const int row = tid >> 3, chk = tid & 7;
         const float gm = gam[row];
-        const bool full = nv == 64;
-        const float rr = full ? raw[row] : 0.f;
+        const float rr = nv == 64 ? raw[row] : 0.f;
+        const uint32_t off = sw(row, chk);
+        const uint4 s4 = *reinterpret_cast<const uint4*>(smem + gt(G_S0) + off);
+        const uint4 g4 = *reinterpret_cast<const uint4*>(smem + gt(G_DS) + off);
+        const uint32_t sw4[4] = {s4.x, s4.y, s4.z, s4.w}, gw4[4] = {g4.x, g4.y, g4.z, g4.w};
+        uint32_t go[4];
         float part = 0.f;
 #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-            const int chk = 2 * qq + hc;
-            const uint32_t off = sw(row, chk);
-            const uint4 s4 = *reinterpret_cast<const uint4*>(smem + gt(G_S0) + off);
-            const uint4 g4 = *reinterpret_cast<const uint4*>(smem + gt(G_DS) + off);
-            const uint32_t sw4[4] = {s4.x, s4.y, s4.z, s4.w}, gw4[4] = {g4.x, g4.y, g4.z, g4.w};
-            uint32_t go[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sw4[i]));
-                float2 gf = __half22float2(*reinterpret_cast<const __half2*>(&gw4[i]));
-                const int v0 = 8 * chk + 2 * i;
-                gf.x -= rr * raw[64 + v0];
-                gf.y -= rr * raw[64 + v0 + 1];
-                part = fmaf(sf.x, gf.x, fmaf(sf.y, gf.y, part));
-                go[i] = pack2h(gf.x, gf.y);
-            }
-            *reinterpret_cast<uint4*>(smem + gt(G_DS) + off) = make_uint4(go[0], go[1], go[2], go[3]);
+        for (int i = 0; i < 4; ++i) {
+            const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sw4[i]));
+            float2 gf = __half22float2(*reinterpret_cast<const __half2*>(&gw4[i]));
+            const int v0 = 8 * chk + 2 * i;
+            gf.x -= rr * raw[64 + v0];
+            gf.y -= rr * raw[64 + v0 + 1];
+            part = fmaf(sf.x, gf.x, fmaf(sf.y, gf.y, part));
+            go[i] = pack2h(gf.x, gf.y);
         }
+        *reinterpret_cast<uint4*>(smem + gt(G_DS) + off) = make_uint4(go[0], go[1], go[2], go[3]);
         part += __shfl_xor_sync(0xffffffffu, part, 1);
         part += __shfl_xor_sync(0xffffffffu, part, 2);
-        if (qq == 0) Rc[row] = gm * part;
+        part += __shfl_xor_sync(0xffffffffu, part, 4);
+        if (chk == 0) Rc[row] = gm * part;
         fence_proxy_async();
     }
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
     tc_fence_after();
 
-    // ---- Gram epilogue: A_ab's diagonal inverses and left blocks; A_ak, A_rb --------
-    if (wh == 1) {
+    // ---- Gram epilogue: warps 4..7 A_ab's diagonal inverses and left blocks; warps
+    //      8..11 masked A_ak, 12..15 masked A_rb ------------------------------------------
+    if (warp >= 4 && warp < 8) {
         float v[2][16];
         tmem_frag(tmem + C1, wq, 0, v[0]);
         tmem_frag(tmem + C1, wq, 32, v[1]);
@@ -610,9 +623,10 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         if (wq > 0) frag_half_to_tile(sbase + gt(G_AB), 16 * wq, 0, 0, v[0], lane, PackH{});
         if (wq > 1) frag_half_to_tile(sbase + gt(G_AB), 16 * wq, 0, 1, v[0], lane, PackH{});
         if (wq > 2) frag_half_to_tile(sbase + gt(G_AB), 16 * wq, 4, 0, v[1], lane, PackH{});
-    } else {
+    } else if (warp >= 8 && warp < 12) {
         acc_to_tile(tmem, C0, sbase + gt(G_AAK), wq, 0, lane, 2, PackH{});
         acc_to_tile(tmem, C0, sbase + gt(G_AAK), wq, 1, lane, 2, PackH{});
+    } else if (warp >= 12) {
         acc_to_tile(tmem, C2, sbase + gt(G_ARB), wq, 0, lane, 1, PackH{});
         acc_to_tile(tmem, C2, sbase + gt(G_ARB), wq, 1, lane, 1, PackH{});
     }
@@ -640,7 +654,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     // ---- T = (I - A_ab)^-1 by block forward substitution (warp-level fp16 MMAs) on
     //      warps 0..3: the six products T_ii A_im (m < i), then warp w builds column
     //      block w: X_w = T_ww, X_i = sum_{w<=m<i} (T_ii A_im) X_m.  Meanwhile warps
-    //      4..7 store phase A's products (issued above; they do not need T). ---------
+    //      4..15 store phase A's products (issued above; they do not need T). ---------
     if (warp < 4) {
         uint8_t* Tb = smem + gt(G_SP) + kDiagBytes;
         uint8_t* Tab = smem + gt(G_DT);
@@ -718,11 +732,14 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     } else {
         wait_or_abort(bar_mma, mph, timed_out);
         tc_fence_after();
+        const uint32_t col = warp < 8 ? C0 : warp < 12 ? C2 : C1;
+        const uint32_t dst = warp < 8 ? G_X : warp < 12 ? G_DARK : G_DU;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            acc_to_tile(tmem, C0, sbase + gt(G_X), wq, hh, lane, 0, PackH{});
-            acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, hh, lane, 0, PackH{});
-            acc_to_tile(tmem, C2, sbase + gt(G_DARK), wq, hh, lane, 1, PackB{});
+            if (warp >= 8 && warp < 12)
+                acc_to_tile(tmem, col, sbase + gt(dst), wq, hh, lane, 1, PackB{});  // dA_rk
+            else
+                acc_to_tile(tmem, col, sbase + gt(dst), wq, hh, lane, 0, PackH{});  // X, dU
         }
     }
     mph ^= 1;
@@ -744,14 +761,14 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
     tc_fence_after();
-    if (warp >= 4 && lane == 0) {
+    if (warp >= 4 && warp < 8 && lane == 0) {
         const int i = warp - 4;
         tma_load_3d(sbase + gt(i == 0 ? G_SP : i == 1 ? G_AB : i == 2 ? G_AAK : G_ARB),
                     i == 0 ? &tm_r : i == 1 ? &tm_k : i == 2 ? &tm_a : &tm_b, bar_rl, 0, cy, cz);
     }
-    acc_to_tile(tmem, C0, sbase + gt(G_X), wq, wh, lane, 0, PackH{});   // U
-    acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, wh, lane, 0, PackH{});  // dX
-    acc_to_tile(tmem, C2, sbase + gt(G_DT), wq, wh, lane, 0, PackH{});  // dT
+    acc16_to_tile(tmem, C0, sbase + gt(G_X), wq, wc, lane, 0, PackH{});   // U
+    acc16_to_tile(tmem, C1, sbase + gt(G_DU), wq, wc, lane, 0, PackH{});  // dX
+    acc16_to_tile(tmem, C2, sbase + gt(G_DT), wq, wc, lane, 0, PackH{});  // dT
     fence_proxy_async();
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
@@ -771,9 +788,9 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
     tc_fence_after();
-    acc_to_tile(tmem, C0, sbase + gt(G_DARB), wq, wh, lane, 1, PackB{});
-    acc_to_tile(tmem, C1, sbase + gt(G_DAAK), wq, wh, lane, 2, PackB{});
-    acc_to_tile(tmem, C2, sbase + gt(G_DT), wq, wh, lane, 0, PackH{});  // Y
+    acc16_to_tile(tmem, C0, sbase + gt(G_DARB), wq, wc, lane, 1, PackB{});
+    acc16_to_tile(tmem, C1, sbase + gt(G_DAAK), wq, wc, lane, 2, PackB{});
+    acc16_to_tile(tmem, C2, sbase + gt(G_DT), wq, wc, lane, 0, PackH{});  // Y
     fence_proxy_async();
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
@@ -803,23 +820,24 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
     tc_fence_after();
-    acc_to_tile(tmem, C0, sbase + gt(G_DAAB), wq, wh, lane, 2, PackB{});
-    {  // rowsum(S0 * P) over this warp's 32 columns (added to R in the final epilogue)
-        float v[16];
-        tmem_frag(tmem + C_P, wq, 32 * wh, v);
+    acc16_to_tile(tmem, C0, sbase + gt(G_DAAB), wq, wc, lane, 2, PackB{});
+    {  // rowsum(S0 * P) over this warp's 16 columns (added to R in the final epilogue)
+        float v[8];
+        tmem_ld16x16(tmem + ((uint32_t)(32 * wq) << 16) + C_P + 16 * wc, v);
+        tmem_ld_wait();
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int row = 16 * wq + g + 8 * hr;
             float part = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
                 const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(
-                    smem + gt(G_S0) + swe(row, 32 * wh + 8 * j + 2 * q)));
+                    smem + gt(G_S0) + swe(row, 16 * wc + 8 * j + 2 * q)));
                 part = fmaf(s2.x, v[4 * j + 2 * hr], fmaf(s2.y, v[4 * j + 2 * hr + 1], part));
             }
             part += __shfl_xor_sync(0xffffffffu, part, 1);
             part += __shfl_xor_sync(0xffffffffu, part, 2);
-            if (q == 0) Rp[64 * wh + row] = part;
+            if (q == 0) Rq[64 * wc + row] = part;
         }
     }
     fence_proxy_async();
@@ -836,62 +854,55 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     wait_or_abort(bar_mma, mph, timed_out);
     mph ^= 1;
     tc_fence_after();
-    // Every input tile is dead now: the next chunk's loads (one per warp, warp 0 two)
-    // overlap the final epilogue.
+    // Every input tile is dead now: the next chunk's nine loads (one per warp) overlap
+    // the final epilogue.
     it = *reinterpret_cast<const volatile int*>(smem + GOFF_NEXT + 64);
     if (it >= 0) {
         I = *reinterpret_cast<const Item*>(smem + GOFF_NEXT);
-        if (lane == 0) {
-            load_in(I, warp);
-            if (warp == 0) load_in(I, 8);
-        }
+        if (lane == 0 && warp < 9) load_in(I, warp);
     }
     wait_or_abort(bar_rl, rph, timed_out);
     rph ^= 1;
 
-    // ---- final epilogue: dr, da, dk, db, and dw by an exclusive prefix over tokens ----
+    // ---- final epilogue: dr, da, dk, db, and dw by an exclusive prefix over tokens;
+    //      thread = rows 16 wq + g (+8) x columns 16 wc + 8 j + 2 q (+1), j = 0, 1 ------
     {
-        float ar[16], aa[16], ak[16], abv[16], drb[16], dab[16];
+        float ar[8], aa[8], ak[8], abv[8], drb[8], dab[8];
         {
-            const uint32_t ta = tmem + ((uint32_t)(32 * wq) << 16) + 32 * wh;
-            tmem_ld16x32(ta + C_AR, ar);
-            tmem_ld16x32(ta + C_AA, aa);
-            tmem_ld16x32(ta + C_AK, ak);
-            tmem_ld16x32(ta + C_AB, abv);
-            tmem_ld16x32(ta + C_DRB, drb);
-            tmem_ld16x32(ta + C_DAB, dab);
+            const uint32_t ta = tmem + ((uint32_t)(32 * wq) << 16) + 16 * wc;
+            tmem_ld16x16(ta + C_AR, ar);
+            tmem_ld16x16(ta + C_AA, aa);
+            tmem_ld16x16(ta + C_AK, ak);
+            tmem_ld16x16(ta + C_AB, abv);
+            tmem_ld16x16(ta + C_DRB, drb);
+            tmem_ld16x16(ta + C_DAB, dab);
             tmem_ld_wait();
         }
-        // the original r, k, a, b at this thread's fragment positions: ldmatrix of the
-        // 16 x 32 block gives register 4 (j / 2) + 2 (j % 2) + hr = (row g + 8 hr,
-        // columns 8 j + 2 q, +1)
-        uint32_t fr_r[8], fr_k[8], fr_a[8], fr_b[8];
+        // the original r, k, a, b at this thread's fragment positions (ldmatrix of the
+        // 16 x 16 block: register 2 j + hr = rows g + 8 hr, columns 8 j + 2 q, +1)
+        uint32_t fr_r[4], fr_k[4], fr_a[4], fr_b[4];
         {
-            const int lrow = 16 * wq + (lane & 7) + 8 * ((lane >> 3) & 1);
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const uint32_t o = sw(lrow, 4 * wh + 2 * hh + (lane >> 4));
-                ldsm_x4(sbase + gt(G_SP) + o, fr_r[4 * hh], fr_r[4 * hh + 1], fr_r[4 * hh + 2], fr_r[4 * hh + 3]);
-                ldsm_x4(sbase + gt(G_AB) + o, fr_k[4 * hh], fr_k[4 * hh + 1], fr_k[4 * hh + 2], fr_k[4 * hh + 3]);
-                ldsm_x4(sbase + gt(G_AAK) + o, fr_a[4 * hh], fr_a[4 * hh + 1], fr_a[4 * hh + 2], fr_a[4 * hh + 3]);
-                ldsm_x4(sbase + gt(G_ARB) + o, fr_b[4 * hh], fr_b[4 * hh + 1], fr_b[4 * hh + 2], fr_b[4 * hh + 3]);
-            }
+            const uint32_t o = sw(16 * wq + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * wc + (lane >> 4));
+            ldsm_x4(sbase + gt(G_SP) + o, fr_r[0], fr_r[1], fr_r[2], fr_r[3]);
+            ldsm_x4(sbase + gt(G_AB) + o, fr_k[0], fr_k[1], fr_k[2], fr_k[3]);
+            ldsm_x4(sbase + gt(G_AAK) + o, fr_a[0], fr_a[1], fr_a[2], fr_a[3]);
+            ldsm_x4(sbase + gt(G_ARB) + o, fr_b[0], fr_b[1], fr_b[2], fr_b[3]);
         }
         // a bf16 pair (low half first) as two floats: bf16 is the top half of an fp32
         auto bf2 = [](uint32_t u) { return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)); };
-        float hv[16], fv[16];
+        float hv[8], fv[8];
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int t = 16 * wq + g + 8 * hr;
             const bool in = t < nv;
             const bool val = in && (!mask || mask[crow + t] != 0);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int cidx = 32 * wh + 8 * j + 2 * q;
+            for (int j = 0; j < 2; ++j) {
+                const int cidx = 16 * wc + 8 * j + 2 * q;
                 const float2 E2 = *reinterpret_cast<const float2*>(Ef + eidx(t, cidx));
                 const float2 Em = t > 0 ? *reinterpret_cast<const float2*>(Ef + eidx(t - 1, cidx))
                                         : make_float2(em0[cidx], em0[cidx + 1]);
-                const int fi = 4 * (j >> 1) + 2 * (j & 1) + hr;
+                const int fi = 2 * j + hr;
                 const float2 r2 = bf2(fr_r[fi]), k2 = bf2(fr_k[fi]), a2 = bf2(fr_a[fi]),
                              b2 = bf2(fr_b[fi]);
                 const float Ee[2] = {E2.x, E2.y}, Eme[2] = {Em.x, Em.y};
@@ -915,15 +926,15 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
             }
         }
         // stage dr, dk, db, da (bf16) in the dA tiles (read by MMA-E, done)
-        frag_to_tile(sbase + gt(G_DARK), 16 * wq, 4 * wh, ar, lane, PackB{});
-        frag_to_tile(sbase + gt(G_DAAK), 16 * wq, 4 * wh, ak, lane, PackB{});
-        frag_to_tile(sbase + gt(G_DARB), 16 * wq, 4 * wh, abv, lane, PackB{});
-        frag_to_tile(sbase + gt(G_DAAB), 16 * wq, 4 * wh, aa, lane, PackB{});
+        frag8_to_tile(sbase + gt(G_DARK), 16 * wq, 2 * wc, ar, lane, PackB{});
+        frag8_to_tile(sbase + gt(G_DAAK), 16 * wq, 2 * wc, ak, lane, PackB{});
+        frag8_to_tile(sbase + gt(G_DARB), 16 * wq, 2 * wc, abv, lane, PackB{});
+        frag8_to_tile(sbase + gt(G_DAAB), 16 * wq, 2 * wc, aa, lane, PackB{});
         // exclusive prefix of h over the tokens: rows g (lanes 4 g + q) within the warp,
         // then rows g + 8, then the quadrants before this one
-        float ex[16];
+        float ex[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int i0 = 4 * j + e, i1 = 4 * j + 2 + e;
@@ -941,17 +952,17 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                 const float tot1 = __shfl_sync(0xffffffffu, s1v, 28 + q);
                 ex[i0] = s0v - hv[i0];
                 ex[i1] = tot0 + s1v - hv[i1];
-                if (g == 0) tot[wq * 64 + 32 * wh + 8 * j + 2 * q + e] = tot0 + tot1;
+                if (g == 0) tot[wq * 64 + 16 * wc + 8 * j + 2 * q + e] = tot0 + tot1;
             }
         __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int cidx = 32 * wh + 8 * j + 2 * q + e;
+                const int cidx = 16 * wc + 8 * j + 2 * q + e;
                 float pre = 0.f;
                 for (int w2 = 0; w2 < wq; ++w2) pre += tot[w2 * 64 + cidx];
-                const float R = Rc[cidx] + Rp[cidx] + Rp[64 + cidx];  // fixed order
+                const float R = Rc[cidx] + Rq[cidx] + Rq[64 + cidx] + Rq[128 + cidx] + Rq[192 + cidx];
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {
                     const int ix = 4 * j + 2 * hr + e;
@@ -960,7 +971,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                     hv[ix] = val ? R - fv[ix] - (pre + ex[ix]) : 0.f;
                 }
             }
-        frag_to_tile(sbase + gt(G_X), 16 * wq, 4 * wh, hv, lane, PackB{});  // dw
+        frag8_to_tile(sbase + gt(G_X), 16 * wq, 2 * wc, hv, lane, PackB{});  // dw
         fence_proxy_async();
         // The stores leave after the next CTA barrier (the next chunk's first, or the
         // one after the loop), which orders them after every thread's staging writes.

@@ -163,6 +163,18 @@ __device__ __forceinline__ void tmem_ld16x32(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 16 lanes x 16 columns in the same fragment layout: v[4j], v[4j+1] (lane +i/4) and
+// v[4j+2], v[4j+3] (lane +i/4+8), columns 8j + 2(i%4), +1, j = 0, 1.
+__device__ __forceinline__ void tmem_ld16x16(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
 // Inverse of tmem_ld16x32 (same register layout).
 __device__ __forceinline__ void tmem_st16x32(uint32_t taddr, const float (&v)[16]) {
     asm volatile(

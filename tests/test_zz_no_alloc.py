@@ -56,9 +56,11 @@ def test_noalloc_equals_workspace_call(cuda_device, dtype):
 
 @pytest.mark.gpu
 def test_noalloc_refuses_large_problem(cuda_device):
-    x = to_dev(synth.fwd_inputs(2, 4096, 16, dtype=torch.bfloat16, seed=802, s0_std=0.1),
+    B, T, H = 4, 4096, 32  # the bf16 (chunked) workspace is over the static scratch
+    assert wkv7_bwd_workspace_bytes(B, T, H, dtype=torch.bfloat16, algo="auto") > STATIC_SCRATCH_BYTES
+    x = to_dev(synth.fwd_inputs(B, T, H, dtype=torch.bfloat16, seed=802, s0_std=0.1),
                cuda_device)
-    dout = torch.zeros(2, 4096, 16, 64, dtype=torch.bfloat16, device=cuda_device)
+    dout = torch.zeros(B, T, H, 64, dtype=torch.bfloat16, device=cuda_device)
     with pytest.raises(WKV7Error) as e:
         wkv7_bwd_noalloc(*(x[n] for n in NAMES), dout, s0=x["s0"])
     assert e.value.status == ERR_UNSUPPORTED
