@@ -43,6 +43,8 @@
 #pragma once
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "chunked.cuh"
 
 namespace wkv7 {
@@ -389,10 +391,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         if (p_nv == 0) return;
         const uint32_t stg[5] = {G_DARK, G_X, G_DAAK, G_DAAB, G_DARB};  // dr dw dk da db
         if (p_nv == 64) {
-            if (lane == 0 && warp < 5) {
-                const CUtensorMap* map = warp == 0 ? &tm_dr : warp == 1 ? &tm_dw : warp == 2 ? &tm_dk
-                                       : warp == 3 ? &tm_da : &tm_db;
-                tma_store_3d(map, sbase + gt(stg[warp]), 0, p_cy, p_cz);
+            if (lane == 0 && warp >= 8 && warp < 13) {  // warps 8..12 (warp 0 scans next)
+                const int ws = warp - 8;
+                const CUtensorMap* map = ws == 0 ? &tm_dr : ws == 1 ? &tm_dw : ws == 2 ? &tm_dk
+                                       : ws == 3 ? &tm_da : &tm_db;
+                tma_store_3d(map, sbase + gt(stg[ws]), 0, p_cy, p_cz);
                 bulk_commit();
             }
         } else {
@@ -632,7 +635,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     }
     // the previous chunk's output stores have read the staging tiles before phase A's
     // epilogue writes them
-    if (lane == 0 && warp < 5) bulk_wait_read0();
+    if (lane == 0 && warp >= 8 && warp < 13) bulk_wait_read0();
     tc_fence_before();
     if (__syncthreads_or(timed_out)) goto teardown;
 
@@ -652,10 +655,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         mma64(tmem + C_P, sbase + gt(G_RB), true, sbase + gt(G_DO), true, false, false);
     }
     // ---- T = (I - A_ab)^-1 by block forward substitution (warp-level fp16 MMAs) on
-    //      warps 0..3: the six products T_ii A_im (m < i), then warp w builds column
-    //      block w: X_w = T_ww, X_i = sum_{w<=m<i} (T_ii A_im) X_m.  Meanwhile warps
-    //      4..15 store phase A's products (issued above; they do not need T). ---------
-    if (warp < 4) {
+    //      warps 0..7: warps 0..5 form the six products T_ii A_im (m < i); then warp w
+    //      builds columns 8 w .. 8 w + 7 (column block w / 2, MMA n-tile w % 2):
+    //      X_b = T_bb, X_i = sum_{b<=m<i} (T_ii A_im) X_m.  Meanwhile warps 8..15 store
+    //      phase A's products (issued above; they do not need T). ------------------------
+    if (warp < 8) {
         uint8_t* Tb = smem + gt(G_SP) + kDiagBytes;
         uint8_t* Tab = smem + gt(G_DT);
         const int lr = (lane & 7) + 8 * ((lane >> 3) & 1), lc = 8 * (lane >> 4);
@@ -663,10 +667,8 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         auto a_frag = [&](const uint8_t* blk, uint32_t (&af)[4]) {
             ldsm_x4(smem_u32(blk) + a_lane, af[0], af[1], af[2], af[3]);
         };
-#pragma unroll
-        for (int rep = 0; rep < 2; ++rep) {
-            const int blk = warp + 4 * rep;
-            if (blk >= 6) break;
+        if (warp < 6) {
+            const int blk = warp;
             const int i = blk < 1 ? 1 : (blk < 3 ? 2 : 3);
             const int m = blk < 1 ? 0 : (blk < 3 ? blk - 1 : blk - 3);
             uint32_t af[4];
@@ -684,62 +686,52 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                 *reinterpret_cast<uint32_t*>(dst + (g + 8) * 48 + 2 * (8 * nt + 2 * q)) = pack2h(z[nt][2], z[nt][3]);
             }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // warps 0..3: T_ii A_im visible
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // warps 0..7: T_ii A_im visible
         {
-            const int wcol = warp;  // column block of T
+            const int cb = warp >> 1, nt = warp & 1;  // column block, n-tile
             uint8_t* tt = smem + gt(G_T);
-            uint32_t xb[3][4];
+            uint32_t xb[3][2];  // B fragments of X_0..X_2 in this n-tile
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint32_t top[2], bot[2];
-                if (i < wcol) {
-                    top[0] = top[1] = bot[0] = bot[1] = 0u;
-                } else if (i == wcol) {
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        top[nt] = *reinterpret_cast<const uint32_t*>(Tb + i * 768 + g * 48 + 2 * (8 * nt + 2 * q));
-                        bot[nt] = *reinterpret_cast<const uint32_t*>(Tb + i * 768 + (g + 8) * 48 + 2 * (8 * nt + 2 * q));
-                    }
+                uint32_t top, bot;
+                if (i < cb) {
+                    top = bot = 0u;
+                } else if (i == cb) {
+                    top = *reinterpret_cast<const uint32_t*>(Tb + i * 768 + g * 48 + 2 * (8 * nt + 2 * q));
+                    bot = *reinterpret_cast<const uint32_t*>(Tb + i * 768 + (g + 8) * 48 + 2 * (8 * nt + 2 * q));
                 } else {
-                    float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int m = 0; m < 3; ++m) {
-                        if (m < wcol || m >= i) continue;
+                        if (m < cb || m >= i) continue;
                         const int blk = (i == 1) ? 0 : (i == 2 ? 1 + m : 3 + m);
                         uint32_t af[4];
                         a_frag(Tab + blk * 768, af);
-                        mma_f16_16816(y[0], af[0], af[1], af[2], af[3], xb[m][0], xb[m][1]);
-                        mma_f16_16816(y[1], af[0], af[1], af[2], af[3], xb[m][2], xb[m][3]);
+                        mma_f16_16816(y, af[0], af[1], af[2], af[3], xb[m][0], xb[m][1]);
                     }
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        top[nt] = pack2h(y[nt][0], y[nt][1]);
-                        bot[nt] = pack2h(y[nt][2], y[nt][3]);
-                    }
+                    top = pack2h(y[0], y[1]);
+                    bot = pack2h(y[2], y[3]);
                 }
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int col = 16 * wcol + 8 * nt + 2 * q;
-                    *reinterpret_cast<uint32_t*>(tt + swe(16 * i + g, col)) = top[nt];
-                    *reinterpret_cast<uint32_t*>(tt + swe(16 * i + g + 8, col)) = bot[nt];
-                    if (i < 3) {
-                        xb[i][2 * nt] = movmatrix_t(top[nt]);
-                        xb[i][2 * nt + 1] = movmatrix_t(bot[nt]);
-                    }
+                const int col = 16 * cb + 8 * nt + 2 * q;
+                *reinterpret_cast<uint32_t*>(tt + swe(16 * i + g, col)) = top;
+                *reinterpret_cast<uint32_t*>(tt + swe(16 * i + g + 8, col)) = bot;
+                if (i < 3) {
+                    xb[i][0] = movmatrix_t(top);
+                    xb[i][1] = movmatrix_t(bot);
                 }
             }
         }
     } else {
         wait_or_abort(bar_mma, mph, timed_out);
         tc_fence_after();
-        const uint32_t col = warp < 8 ? C0 : warp < 12 ? C2 : C1;
-        const uint32_t dst = warp < 8 ? G_X : warp < 12 ? G_DARK : G_DU;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            if (warp >= 8 && warp < 12)
-                acc_to_tile(tmem, col, sbase + gt(dst), wq, hh, lane, 1, PackB{});  // dA_rk
-            else
-                acc_to_tile(tmem, col, sbase + gt(dst), wq, hh, lane, 0, PackH{});  // X, dU
+        if (warp < 12) {  // X, and dA_rk's first half
+            acc_to_tile(tmem, C0, sbase + gt(G_X), wq, 0, lane, 0, PackH{});
+            acc_to_tile(tmem, C0, sbase + gt(G_X), wq, 1, lane, 0, PackH{});
+            acc_to_tile(tmem, C2, sbase + gt(G_DARK), wq, 0, lane, 1, PackB{});
+        } else {          // dU, and dA_rk's second half
+            acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, 0, lane, 0, PackH{});
+            acc_to_tile(tmem, C1, sbase + gt(G_DU), wq, 1, lane, 0, PackH{});
+            acc_to_tile(tmem, C2, sbase + gt(G_DARK), wq, 1, lane, 1, PackB{});
         }
     }
     mph ^= 1;
@@ -891,11 +883,14 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
         // a bf16 pair (low half first) as two floats: bf16 is the top half of an fp32
         auto bf2 = [](uint32_t u) { return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)); };
         float hv[8], fv[8];
+        // kPlain: a full chunk without a mask (every row in and valid, known at compile time)
+        auto elem = [&](auto plain_c) {
+        constexpr bool kPlain = decltype(plain_c)::value;
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int t = 16 * wq + g + 8 * hr;
-            const bool in = t < nv;
-            const bool val = in && (!mask || mask[crow + t] != 0);
+            const bool in = kPlain || t < nv;
+            const bool val = kPlain || (in && (!mask || mask[crow + t] != 0));
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int cidx = 16 * wc + 8 * j + 2 * q;
@@ -925,6 +920,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
                 }
             }
         }
+        };
+        if (nv == 64 && !mask)
+            elem(std::true_type{});
+        else
+            elem(std::false_type{});
         // stage dr, dk, db, da (bf16) in the dA tiles (read by MMA-E, done)
         frag8_to_tile(sbase + gt(G_DARK), 16 * wq, 2 * wc, ar, lane, PackB{});
         frag8_to_tile(sbase + gt(G_DAAK), 16 * wq, 2 * wc, ak, lane, PackB{});
@@ -985,7 +985,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CU
     }  // chunks
     __syncthreads();
     flush();
-    if (lane == 0 && warp < 5) bulk_wait0();  // the last output stores are complete
+    if (lane == 0 && warp >= 8 && warp < 13) bulk_wait0();  // the last output stores are complete
 
 teardown:
     if (timed_out) {
@@ -995,7 +995,7 @@ teardown:
             (void)mbar_wait(bar_mma, mph ^ 1u);
             (void)mbar_wait(bar_rl, rph);
         }
-        if (lane == 0 && warp < 5) bulk_wait0();
+        if (lane == 0 && warp >= 8 && warp < 13) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
