@@ -76,10 +76,12 @@ def load_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest() -> str:
+def source_digest(files=None) -> str:
+    """Digest of the kernel sources: the named files of csrc/ (the ones a kernel is
+    built from), or all of them."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_rnn_wkv7_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -87,14 +89,14 @@ def source_digest() -> str:
 
 def profiled_traffic(kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+    current sources of that kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         entries = json.load(f)
     e = entries.get(kernel)
-    if not e or e.get("source_digest") != source_digest():
+    if not e or e.get("source_digest") != source_digest(e.get("sources")):
         return None
     return e.get("dram_bytes_per_launch")
 
