@@ -143,3 +143,16 @@ def test_chunked_bwd_is_deterministic(cuda_device):
     g1 = _run(x, dout, cuda_device, s0=x["s0"], dsT=dsT.to(cuda_device))
     for n in GRADS:
         assert torch.equal(g0[n], g1[n]), n
+
+
+def test_chunked_bwd_larger_magnitudes(cuda_device):
+    """States around 10 and values around 100 (the gradient kernel carries V, dO, S0 and
+    dSL as fp16 operands, exact in range up to 65504), as the forward's test does."""
+    B, T, H = 2, 200, 2
+    x = synth.fwd_inputs(B, T, H, dtype=BF, seed=760, s0_std=10.0)
+    x["v"] = (x["v"].float() * 100.0).to(BF).contiguous()
+    dout, dsT = upstream(B, T, H, BF, 761)
+    ref = oracle.bwd(*(x[n] for n in NAMES), dout, s0=x["s0"], dsT=dsT)
+    xd = to_dev(x, cuda_device)
+    g = _run(xd, dout, cuda_device, s0=xd["s0"], dsT=dsT.to(cuda_device), algo="chunked")
+    check_grads(g, ref, BF, "chunked larger magnitudes")
