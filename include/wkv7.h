@@ -21,7 +21,10 @@
  * Conventions shared by every entry point:
  *  - All pointers are DEVICE pointers of the current CUDA device, dense,
  *    row-major and 16-byte aligned.  The caller owns and allocates every
- *    buffer; the library allocates nothing and frees nothing.
+ *    buffer; the library frees nothing and allocates one thing of its own: the
+ *    chunked kernel's handoff area (about 4.9 MB per host thread, device and
+ *    stream, made by the first launch on that stream that splits sequences
+ *    between CTAs, outside stream capture; see wkv7_fwd).
  *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
  *    stream).  A non-OK return means either nothing was launched (argument
  *    check on the host) or the launch itself failed (WKV7_ERR_CUDA).
@@ -104,6 +107,14 @@ typedef enum {
  * average); the state and v enter its last tensor-core product as fp16 operands,
  * so their magnitudes must stay below 65504 (larger values saturate).  The
  * recurrent form has neither limit.
+ *
+ * Scheduling of the chunked form: an unpacked problem (cu_seqlens == NULL) with more
+ * (sequence, head) units than the GPU holds CTAs at once (two per SM) is cut into
+ * equal runs of chunks, one per CTA, a sequence split between two CTAs passing its
+ * fp32 state through the library's handoff area (see the conventions above); the
+ * results are bit-identical to one CTA per unit.  Packed problems, smaller ones, and a
+ * launch being captured on a stream that has no handoff area yet run one CTA per
+ * unit (packed sequences longest first).
  */
 wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
                      const void* a, const void* b, const float* s0, const uint8_t* mask,
@@ -392,6 +403,20 @@ int wkv7_version(void);
  * [-1, 256).
  */
 wkv7_status wkv7_test_stall_next_chunked(int tid);
+
+/*
+ * wkv7_test_chunked_schedule -- test hook (no counterpart on the pages): the launch
+ * geometry the chunked kernel takes for `units` (sequence, head) units all `len` tokens
+ * long (unpacked problems) on the current device.  *resident receives the CTAs of the
+ * token-major WKV7 kernel resident at once; when units > *resident the balanced
+ * schedule cuts the units' chunks, laid end to end, into *ctas runs of *cmax chunks (one
+ * CTA each; a unit cut between CTAs m and m+1 runs its first chunks on m+1 and its last
+ * ones on m), else *ctas = *cmax = 0 (one unit per CTA).  Host memory pointers, written
+ * only on success.  Returns WKV7_ERR_INVALID_ARG for a null pointer, units < 0 or
+ * len < 0, WKV7_ERR_CUDA when the device cannot be queried.  Launches nothing.
+ */
+wkv7_status wkv7_test_chunked_schedule(long long units, int len, int* resident, long long* ctas,
+                                       long long* cmax);
 
 #ifdef __cplusplus
 }

@@ -1,5 +1,6 @@
 // chunked.cuh -- 64-token chunked WKV7 forward on tcgen05 tensor cores (bf16 in,
-// fp32 state), one CTA per (sequence, head), two CTAs resident per SM.
+// fp32 state), two CTAs resident per SM, each running one (sequence, head) unit or,
+// for units of one length, an equal run of the units' chunks (Sched).
 //
 // The recurrence (rwkv-ops 0.9.0 README, "rwkv7op 使用方法")
 //     u_t = S_{t-1}^T a_t;  S_t = diag(exp w_t) S_{t-1} + b_t u_t^T + k_t v_t^T;  o_t = S_t^T r_t
@@ -47,6 +48,9 @@
 #pragma once
 #include <cuda.h>
 
+#include <algorithm>
+#include <climits>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -57,6 +61,7 @@ constexpr bool kChunkedBuilt = true;
 namespace chunked {
 
 constexpr int kThreads = 256;
+constexpr int kMinCtasPerSm = 2;  // registers (128 per thread) and shared memory allow two
 constexpr int kStoreTid = 64;  // issues the output tile stores (an output warp's lane 0)
 // Shared-memory map.  Fourteen 8 KB tiles (64 rows x 128 B, 1024-aligned, 128B
 // swizzle) plus a small control block.  Consecutive chunks alternate between two
@@ -66,7 +71,7 @@ constexpr int kStoreTid = 64;  // issues the output tile stores (an output warp'
 constexpr uint32_t kTile = 8192;
 constexpr uint32_t OFF_S0 = 12 * kTile;    // S0 fp16 [k][v] (MMA-U and O's B operand), then
                                            // the output staging; both layouts
-constexpr uint32_t OFF_MISC = 14 * kTile;  // mbarriers, TMEM address
+constexpr uint32_t OFF_MISC = 14 * kTile;  // mbarriers, TMEM address, unit index
 constexpr uint32_t OFF_GAMMA = OFF_MISC + 64;  // e^{g_L}, channel c at cswz(c) (64 fp32)
 constexpr uint32_t kSmemBytes = OFF_GAMMA + 256;
 
@@ -412,6 +417,41 @@ __device__ __forceinline__ void issue_loads_rev(const Ctx& cx, int c0, int par) 
         sm100::cp_async_16(d + L.R, ri.k + o2, n2);
     }
     sm100::cp_async_mbar_arrive(cx.bar_tma);
+}
+
+// Work of one CTA.  When every unit (sequence, head) has the same length, the units'
+// chunks, laid end to end unit by unit, are cut into equal runs of `cmax` >= C chunks
+// (C per unit), one run per CTA, with no more CTAs than fit on the GPU at once
+// (McNaughton's wrap-around rule for preemptive scheduling on identical machines).  A
+// unit cut between CTAs m and m + 1 still runs in order: m + 1 takes the unit's first
+// chunks at the start of its run, m the unit's last chunks at the end of its run, and
+// the fp32 state passes between them through handoff slot m.  Because cmax >= C, the
+// later part starts (no earlier than cmax minus its length) after the earlier part has
+// ended (no later than C minus the later part's length), so the wait is normally nil;
+// it is bounded all the same.  Otherwise (packed sequences of different lengths) each
+// CTA runs one unit.
+struct Sched {
+    int Lu;              // the common unit length in tokens; 0: one unit per CTA
+    long long cmax;      // chunks per CTA
+    float* ho_state;     // [slots][64][64] fp32 handoff states
+    unsigned* ho_flag;   // [slots]: equals `epoch` once the slot's state is written
+    unsigned epoch;      // this launch's (nonzero) flag value
+};
+
+// Bounded wait (one second of device time) until *f == want, with acquire ordering.
+__device__ __forceinline__ bool wait_flag(const unsigned* f, unsigned want) {
+    const uint64_t t0 = sm100::globaltimer_ns();
+    for (uint32_t i = 0; i < (1u << 30); ++i) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+        if (v == want) return true;
+        __nanosleep(128);
+        if ((i & 15u) == 15u && sm100::globaltimer_ns() - t0 > 1000000000ull) return false;
+    }
+    return false;
+}
+__device__ __forceinline__ void st_release(unsigned* f, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
 }
 
 // One 64-token chunk starting at token c0, in layout P (its inputs already requested).
@@ -1089,76 +1129,51 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
 // kGdn: Gated DeltaNet (tm_r, tm_k, tm_v map q, k, v; g and beta per token; s0 may be
 // one state per head shared by every sequence, s0_shared != 0).  kHf (head first):
 // inputs, o (and g, beta) are [B, H, T, *] instead of [B, T, H, *]; the maps follow.
-template <bool kGdn, bool kHf, bool kRev>
-__global__ void __launch_bounds__(kThreads, 2)
-chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
-               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-               const __grid_constant__ CUtensorMap tm_o,
-               const __grid_constant__ CUtensorMap tm_ck,
-               const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
-               float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens,
-               const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ beta,
-               int s0_shared, int stall_tid, int ck_slots, const __grid_constant__ RevIn rin) {
-    extern __shared__ __align__(1024) uint8_t smem[];
-    using namespace sm100;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
-    const uint32_t sbase = smem_u32(smem);
-    if (sbase & 1023u) {  // the swizzled tiles need a 1024-byte aligned base
-        if (tid == 0) raise_flag(3 /* WKV7_ERR_CUDA */);
-        return;
+// Piece k of CTA blockIdx.x's run under the balanced schedule (Sched): unit (n, h),
+// its chunks [cb, ce), and the handoff slots its first and final states come from and
+// go to (-1: s0 and sT).  False past the run's end.
+struct Piece {
+    int n, h, cb, ce, in_slot, out_slot;
+};
+__device__ __forceinline__ bool piece_of(int k, const Sched& sc, int N, int H, Piece& pc) {
+    const long long C = (sc.Lu + 63) / 64;
+    const long long p0 = (long long)blockIdx.x * sc.cmax;
+    const long long pe = min(p0 + sc.cmax, (long long)N * H * C);
+    const long long u = p0 / C + k;  // piece 0 starts at p0, piece k > 0 at unit u's start
+    const long long p = k == 0 ? p0 : u * C;
+    if (p >= pe) return false;
+    const long long uend = (u + 1) * C;
+    pc.n = (int)(u / H);
+    pc.h = (int)(u - (long long)pc.n * H);
+    pc.cb = 0;
+    pc.ce = (int)C;
+    pc.in_slot = pc.out_slot = -1;
+    if (p != u * C) {  // list part [p, uend): the unit's first uend - p chunks
+        pc.ce = (int)(uend - p);
+        pc.out_slot = blockIdx.x - 1;
+    } else if (uend > pe) {  // list part [p, pe): the unit's last pe - p chunks
+        pc.cb = (int)(C - (pe - p));
+        pc.in_slot = blockIdx.x;
     }
-    const int h = blockIdx.x % H;
-    int n = blockIdx.x / H;
-    if (cu_seqlens && N <= kThreads) {
-        // Packed sequences are taken longest first (ties by index): blocks start in
-        // index order, so the long sequences do not end up in the last wave.  Each CTA
-        // ranks the lengths itself, in a tile that is free until the first chunk.
-        int* lens = reinterpret_cast<int*>(smem + 9 * kTile);
-        int* pick = lens + kThreads;
-        if (tid < N) lens[tid] = cu_seqlens[tid + 1] - cu_seqlens[tid];
-        __syncthreads();
-        if (tid < N) {
-            const int mine = lens[tid];
-            int rank = 0;
-            for (int j = 0; j < N; ++j) {
-                const int lj = lens[j];
-                rank += (lj > mine) || (lj == mine && j < tid);
-            }
-            if (rank == n) *pick = tid;
-        }
-        __syncthreads();
-        n = *pick;
-        __syncthreads();  // the tile is reused later
-    }
+    return true;
+}
+
+// The per-unit fields of cx for unit (sequence n, head h): the sequence's token rows,
+// output, gate and checkpoint offsets, its TMA coordinates and, for kRev, the original
+// sequence.  Packed offsets are valid here (checked by the caller or built by the
+// backward's preparation kernel).
+template <bool kHf, bool kRev>
+__device__ __forceinline__ void set_unit(Ctx& cx, int n, int h, int T, int H,
+                                         const int32_t* cu_seqlens, __nv_bfloat16* o,
+                                         int ck_slots, const RevIn& rin) {
     int bb = n, bos = 0, eos = T;
     if (cu_seqlens) {
         bb = 0;
         bos = cu_seqlens[n];
         eos = cu_seqlens[n + 1];
-        if (bos < 0 || eos < bos || eos > T) {
-            if (tid == 0) raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
-            return;
-        }
     }
-
-    Ctx cx;
-    cx.smem = smem;
-    cx.sbase = sbase;
-    cx.bar_tma = sbase + OFF_MISC;
-    cx.bar_mma = sbase + OFF_MISC + 8;
-    cx.bar_g2 = sbase + OFF_MISC + 32;
-    cx.g2_phase = 0;
-    cx.mma_phase = 0;
-    cx.tid = tid;
-    cx.warp = warp;
-    cx.lane = lane;
-    cx.wq = wq;
-    cx.wh = wh;
     cx.row0 = (long long)bb * T + bos;
     cx.len = eos - bos;
-    cx.mask = mask;
     if (kHf) {
         const long long u0 = ((long long)bb * H + h) * T + bos;  // [B, H, T] token index
         cx.o = o ? o + u0 * 64 : nullptr;
@@ -1175,20 +1190,6 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         cx.tma_y = h;
         cx.tma_z = (int)cx.row0;
     }
-    cx.timed_out = 0;
-    cx.tma_par_last = 0;
-    cx.stall_tid = blockIdx.x == 0 ? stall_tid : -1;
-    cx.bar_never = sbase + OFF_MISC + 24;
-    cx.gamma_s = reinterpret_cast<float*>(smem + OFF_GAMMA);
-    cx.tm_r = &tm_r;
-    cx.tm_w = &tm_w;
-    cx.tm_k = &tm_k;
-    cx.tm_v = &tm_v;
-    cx.tm_a = &tm_a;
-    cx.tm_b = &tm_b;
-    cx.tm_o = &tm_o;
-    cx.tm_ck = &tm_ck;
-    cx.ri = &rin;
     if constexpr (kRev) {
         int bb_o = n, bos_o = 0, L_o = rin.T;
         if (rin.cu) {
@@ -1212,8 +1213,90 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             cx.rv_z0 = (int)cx.rv_row0;
         }
     }
-    cx.ck = ck_slots > 0;
     cx.ck_z0 = h * ck_slots + (int)(cx.row0 >> 6) + n;  // slot: floor(row0 / 64) + n + chunk
+}
+
+template <bool kGdn, bool kHf, bool kRev>
+__global__ void __launch_bounds__(kThreads, kMinCtasPerSm)
+chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const __grid_constant__ CUtensorMap tm_o,
+               const __grid_constant__ CUtensorMap tm_ck,
+               const float* s0, const uint8_t* __restrict__ mask, __nv_bfloat16* __restrict__ o,
+               float* sT, int T, int H, int N, const int32_t* __restrict__ cu_seqlens,
+               const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ beta,
+               int s0_shared, int stall_tid, int ck_slots, const __grid_constant__ RevIn rin,
+               const __grid_constant__ Sched sc) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    using namespace sm100;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
+    const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {  // the swizzled tiles need a 1024-byte aligned base
+        if (tid == 0) raise_flag(3 /* WKV7_ERR_CUDA */);
+        return;
+    }
+    const bool bal = sc.Lu > 0;
+    int n = blockIdx.x / H;
+    if (!bal && cu_seqlens && N <= kThreads) {
+        // Packed sequences are taken longest first (ties by index): blocks start in
+        // index order, so the long sequences do not end up in the last wave.  Each CTA
+        // ranks the lengths itself, in a tile that is free until the first chunk.
+        int* lens = reinterpret_cast<int*>(smem + 9 * kTile);
+        int* pick = lens + kThreads;
+        if (tid < N) lens[tid] = cu_seqlens[tid + 1] - cu_seqlens[tid];
+        __syncthreads();
+        if (tid < N) {
+            const int mine = lens[tid];
+            int rank = 0;
+            for (int j = 0; j < N; ++j) {
+                const int lj = lens[j];
+                rank += (lj > mine) || (lj == mine && j < tid);
+            }
+            if (rank == n) *pick = tid;
+        }
+        __syncthreads();
+        n = *pick;
+        __syncthreads();  // the tile is reused later
+    }
+    if (!bal && cu_seqlens) {
+        const int bos = cu_seqlens[n], eos = cu_seqlens[n + 1];
+        if (bos < 0 || eos < bos || eos > T) {
+            if (tid == 0) raise_flag(5 /* WKV7_ERR_DEVICE_BAD_SEQLENS */);
+            return;
+        }
+    }
+
+    Ctx cx;
+    cx.smem = smem;
+    cx.sbase = sbase;
+    cx.bar_tma = sbase + OFF_MISC;
+    cx.bar_mma = sbase + OFF_MISC + 8;
+    cx.bar_g2 = sbase + OFF_MISC + 32;
+    cx.g2_phase = 0;
+    cx.mma_phase = 0;
+    cx.tid = tid;
+    cx.warp = warp;
+    cx.lane = lane;
+    cx.wq = wq;
+    cx.wh = wh;
+    cx.mask = mask;
+    cx.timed_out = 0;
+    cx.tma_par_last = 0;
+    cx.stall_tid = blockIdx.x == 0 ? stall_tid : -1;
+    cx.bar_never = sbase + OFF_MISC + 24;
+    cx.gamma_s = reinterpret_cast<float*>(smem + OFF_GAMMA);
+    cx.tm_r = &tm_r;
+    cx.tm_w = &tm_w;
+    cx.tm_k = &tm_k;
+    cx.tm_v = &tm_v;
+    cx.tm_a = &tm_a;
+    cx.tm_b = &tm_b;
+    cx.tm_o = &tm_o;
+    cx.tm_ck = &tm_ck;
+    cx.ri = &rin;
+    cx.ck = ck_slots > 0;
     cx.g = g;
     cx.beta = beta;
 
@@ -1223,6 +1306,7 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
         tmem_relinquish();
     }
     if (tid == 0) {
+        *reinterpret_cast<int*>(smem + OFF_MISC + 40) = n;  // the unit of a one-unit CTA
         mbar_init(cx.bar_tma, 1);
         mbar_init(cx.bar_mma, 1);
         mbar_init(cx.bar_g2, 1);
@@ -1236,48 +1320,123 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
     if (warp == 0 && lane < 7)
         prefetch_tensormap(lane == 0 ? &tm_r : lane == 1 ? &tm_a : lane == 2 ? &tm_k
                            : lane == 3 ? &tm_b : lane == 4 ? &tm_w : lane == 5 ? &tm_v : &tm_o);
-    if constexpr (kRev) {
-        if (cx.len > 0) {
-            issue_loads_rev(cx, 0, 0);
-            __syncthreads();  // every thread's copies are tracked: complete the count
-            if (tid == 0) mbar_arrive(cx.bar_tma);
-        }
-    } else if (warp == 0 && cx.len > 0) {
-        issue_loads<kGdn, kHf>(cx, 0, 0);
-    }
 
     // The fp32 state lives in tensor memory as an M = 64 accumulator: row k in lane
     // (k % 16) + 32 (k / 16), so lanes 0..15 of warp w hold rows 16 (w % 4) + lane,
     // columns [32 (w / 4), 32 (w / 4) + 32).  The other lanes of those columns stay unused.
     const int srow = 16 * wq + lane;  // state row of this thread (lanes 0..15)
-    const size_t state_off = ((size_t)n * H + h) * 4096;
-    {
-        float sv[32];
+
+    // This CTA's pieces, in time order (see Sched): with the balanced schedule, piece k
+    // of its run of the unit-major chunk list (recomputed where needed, so that nothing
+    // of it stays live across the chunks); otherwise the one unit n, h.
+    bool ok = true;
+    int par = 0;  // layout of the next chunk (chunks alternate between the two)
+    for (int piece = 0; ok; ++piece) {
+        Piece pc;
+        if (bal) {
+            if (!piece_of(piece, sc, N, H, pc)) break;
+        } else {
+            if (piece > 0) break;
+            pc = Piece{*reinterpret_cast<const int*>(smem + OFF_MISC + 40), (int)(blockIdx.x % H),
+                       0, INT_MAX, -1, -1};
+        }
+        const int cb = pc.cb, ce = pc.ce, in_slot = pc.in_slot, h = pc.h;
+        set_unit<kHf, kRev>(cx, pc.n, h, T, H, cu_seqlens, o, ck_slots, rin);
+        const int tb = 64 * cb;
+        const int te = ce == INT_MAX ? cx.len : min(cx.len, 64 * ce);
+
+        // the piece's first loads (they do not depend on the state)
+        if (tb < te) {
+            if constexpr (kRev) {
+                issue_loads_rev(cx, tb, par);
+                __syncthreads();  // every thread's copies are tracked: complete the count
+                if (tid == 0) mbar_arrive(cx.bar_tma);
+            } else if (warp == 0) {
+                issue_loads<kGdn, kHf>(cx, tb, par);
+            }
+            cx.tma_par_last = par;
+        }
+
+        // the starting state: s0 (or zeros) at a unit's start, else the handoff slot
+        {
+            const float* src = nullptr;
+            if (in_slot >= 0) {
+                int late = 0;
+                if (tid == 0 && !wait_flag(sc.ho_flag + in_slot, sc.epoch)) {
+                    raise_flag(4 /* WKV7_ERR_DEVICE_TIMEOUT */);
+                    late = 1;
+                }
+                if (__syncthreads_or(late)) {
+                    ok = false;
+                    break;
+                }
+                src = sc.ho_state + (size_t)in_slot * 4096;
+            } else if (s0 && cb == 0) {
+                src = s0 + (s0_shared ? (size_t)h : (size_t)pc.n * H + h) * 4096;
+            }
+            float sv[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sv[j] = 0.f;
-        if (s0 && lane < 16) {
-            const size_t init_off = s0_shared ? (size_t)h * 4096 : state_off;
-            const float4* src = reinterpret_cast<const float4*>(s0 + init_off + srow * 64 + 32 * wh);
+            for (int j = 0; j < 32; ++j) sv[j] = 0.f;
+            if (src && lane < 16) {
+                const float4* s4 = reinterpret_cast<const float4*>(src + srow * 64 + 32 * wh);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 f = src[j];
-                sv[4 * j] = f.x;
-                sv[4 * j + 1] = f.y;
-                sv[4 * j + 2] = f.z;
-                sv[4 * j + 3] = f.w;
+                for (int j = 0; j < 8; ++j) {
+                    const float4 f = in_slot >= 0 ? __ldcg(s4 + j) : s4[j];
+                    sv[4 * j] = f.x;
+                    sv[4 * j + 1] = f.y;
+                    sv[4 * j + 2] = f.z;
+                    sv[4 * j + 3] = f.w;
+                }
+            }
+            tmem_row_st32(cx.tmem + TM_DFS, wq, 32 * wh, sv);
+            tmem_st_wait();
+            if (in_slot >= 0) {  // consumed: clear the flag for the next launch
+                __syncthreads();
+                if (tid == 0) *reinterpret_cast<volatile unsigned*>(sc.ho_flag + in_slot) = 0u;
             }
         }
-        tmem_row_st32(cx.tmem + TM_DFS, wq, 32 * wh, sv);
-        tmem_st_wait();
-    }
-    tc_fence_before();
+        tc_fence_before();
 
-    // Chunks alternate between the two shared-memory layouts.
-    bool ok = true;
-    for (int c0 = 0, par = 0; c0 < cx.len && ok; c0 += 64, par ^= 1)
-        ok = chunk<kGdn, kHf, kRev>(cx, c0, c0 + 64 < cx.len, par);
-    // The last chunk's final-MMA wait is agreed on here (it has no barrier of its own).
-    if (ok && __syncthreads_or(cx.timed_out)) ok = false;
+        for (int c0 = tb; c0 < te && ok; c0 += 64, par ^= 1)
+            ok = chunk<kGdn, kHf, kRev>(cx, c0, c0 + 64 < te, par);
+        // The last chunk's final-MMA wait is agreed on here (it has no barrier of its own).
+        if (ok && __syncthreads_or(cx.timed_out)) ok = false;
+        tc_fence_after();
+        if (!ok) break;
+
+        // the final state: to sT at a unit's end, else to the handoff slot
+        int out_slot = -1, un, uh;
+        if (bal) {
+            (void)piece_of(piece, sc, N, H, pc);
+            out_slot = pc.out_slot;
+            un = pc.n;
+            uh = pc.h;
+        } else {
+            un = *reinterpret_cast<const int*>(smem + OFF_MISC + 40);
+            uh = (int)(blockIdx.x % H);
+        }
+        const size_t state_off = ((size_t)un * H + uh) * 4096;
+        float* dst = out_slot >= 0 ? sc.ho_state + (size_t)out_slot * 4096
+                                   : (sT ? sT + state_off : nullptr);
+        if (dst) {
+            float sv[32];
+            tmem_row<2>(cx.tmem + TM_DFS, wq, 32 * wh, sv);
+            if (lane < 16) {
+                float4* d4 = reinterpret_cast<float4*>(dst + srow * 64 + 32 * wh);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    d4[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+            }
+        }
+        if (out_slot >= 0) {
+            __syncthreads();  // every thread's part of the state is written
+            if (tid == 0) {
+                __threadfence();
+                st_release(sc.ho_flag + out_slot, sc.epoch);
+            }
+        }
+        tc_fence_before();
+    }
 
     tc_fence_after();
     if (!ok) {
@@ -1288,15 +1447,6 @@ chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__
             (void)mbar_wait(cx.bar_tma, cx.tma_par_last);
             (void)mbar_wait(cx.bar_mma, cx.mma_phase ^ 1u);
             (void)mbar_wait(cx.bar_g2, cx.g2_phase ^ 1u);
-        }
-    } else if (sT) {
-        float sv[32];
-        tmem_row<2>(cx.tmem + TM_DFS, wq, 32 * wh, sv);
-        if (lane < 16) {
-            float4* dst = reinterpret_cast<float4*>(sT + state_off + srow * 64 + 32 * wh);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                dst[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
         }
     }
     if (tid == kStoreTid) bulk_wait0();  // the output stores are complete
@@ -1328,8 +1478,12 @@ inline EncodeTiledFn encode_fn() {
 
 // [B*T, H, 64] bf16 tensor viewed as (64, H, B*T), box = 64 tokens of one head; or,
 // head first, [B*H, T, 64] viewed as (64, T, B*H), box = 64 tokens of one (b, h).  Both
-// boxes land as 64 rows of 128 bytes, token-major.
-inline bool make_map(CUtensorMap* map, const void* ptr, int B, int T, int H, int head_first) {
+// boxes land as 64 rows of 128 bytes, token-major.  L2 fetches are promoted to 256 bytes
+// (a token-major row and the next head's, which the CTA of that head, running at the
+// same time, reads) unless `wide_l2` is false (128 bytes: when the CTAs running at once
+// do not hold neighbouring heads, the other half would be fetched for nobody).
+inline bool make_map(CUtensorMap* map, const void* ptr, int B, int T, int H, int head_first,
+                     bool wide_l2 = true) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t rows = (cuuint64_t)B * T;
@@ -1346,7 +1500,8 @@ inline bool make_map(CUtensorMap* map, const void* ptr, int B, int T, int H, int
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               wide_l2 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // State checkpoints: [H * slots][64][64] 16-bit (fp16) tiles, viewed as (64, 64,
@@ -1373,6 +1528,124 @@ struct Extras {
     void* ck = nullptr;
     int ck_slots = 0;
 };
+
+// The kernel's dynamic shared-memory size (above the default limit) and the largest
+// shared-memory carveout (two CTAs per SM need all of it), set once.
+template <bool kGdn, bool kHf, bool kRev>
+inline cudaError_t ensure_smem_attr() {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf, kRev>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kSmemBytes);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf, kRev>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    return cudaSuccess;
+}
+
+// Launch geometry of the balanced schedule (Sched) for `units` units of Lu tokens with
+// `slots` CTAs resident at once: `ctas` runs of `cmax` chunks.  False (one unit per
+// CTA) unless there are more units than slots.
+inline bool balanced_geometry(long long units, int Lu, long long slots, long long& ctas,
+                              long long& cmax) {
+    if (Lu <= 0 || slots <= 0 || units <= slots) return false;
+    const long long C = (Lu + 63) / 64, total = units * C;
+    cmax = std::max(C, (total + slots - 1) / slots);
+    ctas = (total + cmax - 1) / cmax;
+    return true;
+}
+
+// CTAs of chunked_kernel<kGdn, kHf, kRev> resident on the current device at once (its
+// dynamic shared-memory size already set), 0 if unknown.
+template <bool kGdn, bool kHf, bool kRev>
+inline int resident_ctas() {
+    constexpr int kMaxDev = 64;
+    static int cached[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    if (cached[dev] == 0) {
+        int per_sm = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunked_kernel<kGdn, kHf, kRev>,
+                                                          kThreads, kSmemBytes) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return 0;
+        }
+        // The occupancy query answers one per SM for this kernel, while it runs two
+        // (its registers and shared memory are sized for two; the launch list shows
+        // it): take the design's two unless the query allows more.
+        cached[dev] = std::max(per_sm, kMinCtasPerSm) * sms;
+    }
+    return cached[dev];
+}
+
+// The handoff slots of the balanced schedule (Sched): one area per (host thread, device,
+// stream), so launches that may run at the same time never share one.  It is made on
+// first use (outside stream capture: a launch being captured with no area yet runs one
+// unit per CTA) and kept for the life of the process; a captured launch keeps the area
+// and epoch it was captured with, and each consumer clears its flag, so replays work.
+struct Handoff {
+    int dev = -1;
+    cudaStream_t stream = nullptr;
+    int slots = 0;
+    float* state = nullptr;
+    unsigned* flag = nullptr;
+    unsigned epoch = 0;
+};
+inline Handoff* handoff_for(cudaStream_t stream, int slots) {
+    constexpr int kMax = 16;
+    thread_local Handoff cache[kMax];
+    thread_local int used = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    for (int i = 0; i < used; ++i)
+        if (cache[i].dev == dev && cache[i].stream == stream && cache[i].slots >= slots)
+            return &cache[i];
+    if (used == kMax) return nullptr;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    if (cs != cudaStreamCaptureStatusNone) return nullptr;
+    const size_t state_bytes = (size_t)slots * 4096 * sizeof(float);
+    void* mem = nullptr;
+    // relaxed capture mode for this thread: the allocation must not disturb a capture
+    // that another thread may have open
+    cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+    (void)cudaThreadExchangeStreamCaptureMode(&mode);
+    const cudaError_t e = cudaMalloc(&mem, state_bytes + (size_t)slots * sizeof(unsigned));
+    (void)cudaThreadExchangeStreamCaptureMode(&mode);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    unsigned* flag = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(mem) + state_bytes);
+    if (cudaMemsetAsync(flag, 0, (size_t)slots * sizeof(unsigned), stream) != cudaSuccess) {
+        (void)cudaGetLastError();
+        (void)cudaFree(mem);
+        return nullptr;
+    }
+    Handoff& hb = cache[used++];
+    hb.dev = dev;
+    hb.stream = stream;
+    hb.slots = slots;
+    hb.state = static_cast<float*>(mem);
+    hb.flag = flag;
+    hb.epoch = 0;
+    return &hb;
+}
 template <bool kGdn, bool kHf, bool kRev = false>
 inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float* s0,
                           const uint8_t* mask, void* o, float* sT, int B, int T, int H, int N,
@@ -1380,17 +1653,28 @@ inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float
                           int s0_shared, int stall_tid, const Extras& ex,
                           cudaStream_t stream, const RevIn* rin = nullptr,
                           int B_o = 0, int T_o = 0) {
+    if (const cudaError_t e = ensure_smem_attr<kGdn, kHf, kRev>(); e != cudaSuccess) return e;
+    // Units of one length (no packed sequences; for kRev, reversed sequences of an
+    // unpacked problem) take the balanced schedule when there are more units than
+    // resident CTAs (and a handoff area is at hand).
+    long long grid = (long long)N * H, ctas = 0, cmax = 0;
+    const int Lu = kRev ? (rin && !rin->cu ? 64 * (T_o / 64 + 1) : 0) : (cu_seqlens ? 0 : T);
+    Handoff* hb = nullptr;
+    if (Lu > 0 && balanced_geometry(grid, Lu, resident_ctas<kGdn, kHf, kRev>(), ctas, cmax))
+        hb = handoff_for(stream, (int)ctas);
+    const bool wide_l2 = hb == nullptr;  // neighbouring heads run at once only without it
+
     CUtensorMap maps[8];
     if (kRev) {  // the output is dv in the original layout; no input maps (cp.async loads)
-        if (!make_map(&maps[6], rin->dv, B_o, T_o, H, rin->hf)) return cudaErrorInvalidValue;
+        if (!make_map(&maps[6], rin->dv, B_o, T_o, H, rin->hf, wide_l2)) return cudaErrorInvalidValue;
         for (int i = 0; i < 6; ++i) maps[i] = maps[6];  // unused by the kernel
     }
     for (int i = 0; i < nmaps; ++i)
-        if (!make_map(&maps[i], ptrs[i], B, T, H, kHf)) return cudaErrorInvalidValue;
+        if (!make_map(&maps[i], ptrs[i], B, T, H, kHf, wide_l2)) return cudaErrorInvalidValue;
     for (int i = nmaps; i < 6 && !kRev; ++i) maps[i] = maps[0];  // unused by the kernel
     if (kRev) {
     } else if (o) {
-        if (!make_map(&maps[6], o, B, T, H, kHf)) return cudaErrorInvalidValue;  // the output
+        if (!make_map(&maps[6], o, B, T, H, kHf, wide_l2)) return cudaErrorInvalidValue;  // the output
     } else {
         maps[6] = maps[0];  // unused: no outputs
     }
@@ -1400,20 +1684,22 @@ inline cudaError_t launch_layout(const void* const* ptrs, int nmaps, const float
     } else {
         maps[7] = maps[0];  // unused: no checkpoints
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf, kRev>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
     const RevIn rv = rin ? *rin : RevIn{};
-    chunked_kernel<kGdn, kHf, kRev><<<(unsigned)((long long)N * H), kThreads, kSmemBytes, stream>>>(
+    Sched sc{};
+    if (hb) {
+        if (++hb->epoch == 0) hb->epoch = 1;
+        sc.Lu = Lu;
+        sc.cmax = cmax;
+        sc.ho_state = hb->state;
+        sc.ho_flag = hb->flag;
+        sc.epoch = hb->epoch;
+        grid = ctas;
+    }
+    chunked_kernel<kGdn, kHf, kRev><<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7], s0, mask,
         static_cast<__nv_bfloat16*>(o), sT, T, H, N, cu_seqlens,
         static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(beta), s0_shared,
-        stall_tid, ex.ck ? ex.ck_slots : 0, rv);
+        stall_tid, ex.ck ? ex.ck_slots : 0, rv, sc);
     return cudaGetLastError();
 }
 template <bool kGdn>

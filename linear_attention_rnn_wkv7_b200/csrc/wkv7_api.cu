@@ -80,6 +80,24 @@ wkv7_status wkv7_test_stall_next_chunked(int tid) {
     return WKV7_OK;
 }
 
+wkv7_status wkv7_test_chunked_schedule(long long units, int len, int* resident, long long* ctas,
+                                       long long* cmax) {
+    using namespace wkv7::chunked;
+    if (!resident || !ctas || !cmax || units < 0 || len < 0) return WKV7_ERR_INVALID_ARG;
+    if (ensure_smem_attr<false, false, false>() != cudaSuccess) {
+        (void)cudaGetLastError();
+        return WKV7_ERR_CUDA;
+    }
+    const int slots = resident_ctas<false, false, false>();
+    if (slots <= 0) return WKV7_ERR_CUDA;
+    long long c = 0, m = 0;
+    if (!balanced_geometry(units, len, slots, c, m)) c = m = 0;
+    *resident = slots;
+    *ctas = c;
+    *cmax = m;
+    return WKV7_OK;
+}
+
 wkv7_status wkv7_fwd(const void* r, const void* w, const void* k, const void* v,
                      const void* a, const void* b, const float* s0, const uint8_t* mask,
                      void* o, float* sT, int B, int T, int H, int K, int V,

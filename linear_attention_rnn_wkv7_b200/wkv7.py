@@ -77,6 +77,10 @@ def library() -> ctypes.CDLL:
         lib.wkv7_version.argtypes = []
         lib.wkv7_test_stall_next_chunked.restype = i
         lib.wkv7_test_stall_next_chunked.argtypes = [i]
+        lib.wkv7_test_chunked_schedule.restype = i
+        lib.wkv7_test_chunked_schedule.argtypes = [ctypes.c_longlong, i, ctypes.POINTER(i),
+                                                   ctypes.POINTER(ctypes.c_longlong),
+                                                   ctypes.POINTER(ctypes.c_longlong)]
         lib.wkv7_sane_fwd.restype = i
         lib.wkv7_sane_fwd.argtypes = [p] * 9 + [i, p, p, i, i, i, i, i, i, i, p]
         lib.wkv7_sane_step.restype = i
