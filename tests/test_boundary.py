@@ -6,10 +6,12 @@ import os
 import re
 
 import pytest
+import torch
 
 import linear_attention_rnn_wkv7_b200 as wkv7
 from linear_attention_rnn_wkv7_b200 import build as wkv7_build
-from linear_attention_rnn_wkv7_b200.wkv7 import (ERR_INVALID_ARG, ERR_UNSUPPORTED, OK, BF16, F32)
+from linear_attention_rnn_wkv7_b200.wkv7 import (BF16, ERR_CUDA, ERR_INVALID_ARG, ERR_UNSUPPORTED,
+                                                 F32, OK)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
@@ -222,6 +224,20 @@ def test_stall_hook_arguments(lib):
     assert lib.wkv7_test_stall_next_chunked(256) == ERR_INVALID_ARG
     assert lib.wkv7_test_stall_next_chunked(5) == OK
     assert lib.wkv7_test_stall_next_chunked(-1) == OK
+
+
+def test_schedule_hook_arguments(lib):
+    """The chunked kernel's schedule query checks its arguments on the host; with no
+    device to query it reports WKV7_ERR_CUDA and writes nothing."""
+    r, c, m = ctypes.c_int(-7), ctypes.c_longlong(-7), ctypes.c_longlong(-7)
+    out = (ctypes.byref(r), ctypes.byref(c), ctypes.byref(m))
+    assert lib.wkv7_test_chunked_schedule(512, 4096, None, out[1], out[2]) == ERR_INVALID_ARG
+    assert lib.wkv7_test_chunked_schedule(512, 4096, out[0], None, out[2]) == ERR_INVALID_ARG
+    assert lib.wkv7_test_chunked_schedule(-1, 4096, *out) == ERR_INVALID_ARG
+    assert lib.wkv7_test_chunked_schedule(512, -1, *out) == ERR_INVALID_ARG
+    if not torch.cuda.is_available():
+        assert lib.wkv7_test_chunked_schedule(512, 4096, *out) == ERR_CUDA
+    assert (r.value, c.value, m.value) == (-7, -7, -7)
 
 
 def test_sane_entry_points_reject_bad_arguments(lib):
