@@ -1530,20 +1530,24 @@ struct Extras {
 };
 
 // The kernel's dynamic shared-memory size (above the default limit) and the largest
-// shared-memory carveout (two CTAs per SM need all of it), set once.
+// shared-memory carveout (two CTAs per SM need all of it), set once per device.
 template <bool kGdn, bool kHf, bool kRev>
 inline cudaError_t ensure_smem_attr() {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf, kRev>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
+    constexpr int kMaxDev = 64;
+    static bool attr_set[kMaxDev] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf, kRev>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(chunked_kernel<kGdn, kHf, kRev>,
                                  cudaFuncAttributePreferredSharedMemoryCarveout,
                                  (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set[dev] = true;
     }
     return cudaSuccess;
 }

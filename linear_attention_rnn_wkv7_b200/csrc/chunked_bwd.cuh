@@ -1024,18 +1024,20 @@ inline cudaError_t launch_grad(const void* r, const void* w, const void* k, cons
     void* outs[5] = {dr, dw, dk, da, db};
     for (int i = 0; i < 5; ++i)
         if (!make_map(&m[9 + i], outs[i], B, T, H, kHf)) return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(grad_kernel<kHf>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kGSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return cudaErrorInvalidValue;
+    constexpr int kMaxDev = 64;  // the dynamic shared-memory size, set once per device
+    static bool attr_set[kMaxDev] = {};
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(grad_kernel<kHf>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kGSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
     const long long items = lay.slotsF * H;
     if (items > 0x7fffffffLL - 4096) return cudaErrorInvalidValue;  // item + grid stays an int
     const unsigned grid = (unsigned)(items < sms ? items : sms);
