@@ -219,7 +219,9 @@ wkv7_status wkv7_bwd_with_algo(const void* r, const void* w, const void* k, cons
  * must not call into the allocator).  The scratch is a file-scope device array of
  * WKV7_STATIC_SCRATCH_BYTES that every GPU which loads the library keeps until exit.
  * Problems whose wkv7_bwd_workspace_bytes exceed it return WKV7_ERR_UNSUPPORTED before
- * anything is launched.  The call allocates nothing itself; it runs on the CURRENT
+ * anything is launched.  The call allocates nothing itself (its chunked forward runs
+ * take the balanced schedule only on a stream that already has a handoff area, else
+ * one CTA per unit, with the same results); it runs on the CURRENT
  * device, which must be the device of every pointer and of the stream.  Its first call
  * on a device looks up the array's address there (cudaGetSymbolAddress, cached per
  * device); with CUDA's lazy module loading that first call may also load the library's

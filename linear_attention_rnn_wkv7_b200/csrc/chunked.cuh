@@ -1596,6 +1596,12 @@ inline int resident_ctas() {
 // first use (outside stream capture: a launch being captured with no area yet runs one
 // unit per CTA) and kept for the life of the process; a captured launch keeps the area
 // and epoch it was captured with, and each consumer clears its flag, so replays work.
+// Set (per host thread) while an entry point that promises no allocation runs: the
+// balanced schedule then takes an existing handoff area or none.
+inline bool& handoff_alloc_forbidden() {
+    thread_local bool forbidden = false;
+    return forbidden;
+}
 struct Handoff {
     int dev = -1;
     cudaStream_t stream = nullptr;
@@ -1616,7 +1622,7 @@ inline Handoff* handoff_for(cudaStream_t stream, int slots) {
     for (int i = 0; i < used; ++i)
         if (cache[i].dev == dev && cache[i].stream == stream && cache[i].slots >= slots)
             return &cache[i];
-    if (used == kMax) return nullptr;
+    if (used == kMax || handoff_alloc_forbidden()) return nullptr;
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
         (void)cudaGetLastError();

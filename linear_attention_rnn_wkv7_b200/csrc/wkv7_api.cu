@@ -410,8 +410,15 @@ wkv7_status wkv7_bwd_noalloc(const void* r, const void* w, const void* k, const 
     if (need > kStaticScratchBytes) return WKV7_ERR_UNSUPPORTED;
     void* scratch = static_scratch_on_current_device();
     if (!scratch) return WKV7_ERR_CUDA;
-    return wkv7_bwd(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da, db, ds0, B, T, H,
-                    K, V, cu_seqlens, N, layout, dtype, scratch, kStaticScratchBytes, stream);
+    // the chunked forward runs must not make a handoff area here (they use an existing one
+    // or run one unit per CTA)
+    bool& forbid = wkv7::chunked::handoff_alloc_forbidden();
+    forbid = true;
+    const wkv7_status st = wkv7_bwd(r, w, k, v, a, b, s0, mask, dout, dsT, dr, dw, dk, dv, da,
+                                    db, ds0, B, T, H, K, V, cu_seqlens, N, layout, dtype, scratch,
+                                    kStaticScratchBytes, stream);
+    forbid = false;
+    return st;
 }
 
 wkv7_status wkv7_gdn_bwd(const void* q, const void* k, const void* v, const void* g,

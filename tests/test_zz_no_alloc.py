@@ -2,6 +2,7 @@
 array) instead of a caller workspace.  It must give exactly wkv7_bwd's results on
 problems that fit, and refuse larger ones before touching the device."""
 import ctypes
+import threading
 
 import pytest
 import torch
@@ -64,3 +65,37 @@ def test_noalloc_refuses_large_problem(cuda_device):
     with pytest.raises(WKV7Error) as e:
         wkv7_bwd_noalloc(*(x[n] for n in NAMES), dout, s0=x["s0"])
     assert e.value.status == ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+def test_noalloc_makes_no_handoff_area(cuda_device):
+    """More (sequence, head) units than the GPU holds CTAs at once: wkv7_bwd runs its
+    two chunked forward runs on the balanced schedule (with the library's handoff area),
+    while wkv7_bwd_noalloc, called from a host thread that has no handoff area yet, must
+    not make one and runs them one unit per CTA.  The results are the same bits."""
+    B, T, H = 5, 200, 64
+    assert wkv7_bwd_workspace_bytes(B, T, H, dtype=torch.bfloat16, algo="auto") <= STATIC_SCRATCH_BYTES
+    x = to_dev(synth.fwd_inputs(B, T, H, dtype=torch.bfloat16, seed=803, s0_std=0.1), cuda_device)
+    gen = torch.Generator().manual_seed(804)
+    dout = torch.randn(B, T, H, 64, generator=gen).to(torch.bfloat16).to(cuda_device)
+    dsT = (torch.randn(B, H, 64, 64, generator=gen) * 0.1).to(cuda_device)
+    args = [x[n] for n in NAMES] + [dout]
+    g0 = wkv7_bwd(*args, s0=x["s0"], dsT=dsT)
+    torch.cuda.synchronize()
+    out = {}
+
+    def run():
+        try:
+            torch.cuda.set_device(cuda_device)
+            out["g"] = wkv7_bwd_noalloc(*args, s0=x["s0"], dsT=dsT)
+            torch.cuda.synchronize()
+        except Exception as e:  # re-raised below, in the test's thread
+            out["err"] = e
+
+    t = threading.Thread(target=run)
+    t.start()
+    t.join()
+    if "err" in out:
+        raise out["err"]
+    for n in g0:
+        assert torch.equal(g0[n], out["g"][n]), n
