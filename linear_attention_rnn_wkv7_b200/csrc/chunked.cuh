@@ -1126,9 +1126,6 @@ __device__ __forceinline__ bool chunk(Ctx& cx, int c0, bool has_next, int par) {
         return true;
 }
 
-// kGdn: Gated DeltaNet (tm_r, tm_k, tm_v map q, k, v; g and beta per token; s0 may be
-// one state per head shared by every sequence, s0_shared != 0).  kHf (head first):
-// inputs, o (and g, beta) are [B, H, T, *] instead of [B, T, H, *]; the maps follow.
 // Piece k of CTA blockIdx.x's run under the balanced schedule (Sched): unit (n, h),
 // its chunks [cb, ce), and the handoff slots its first and final states come from and
 // go to (-1: s0 and sT).  False past the run's end.
@@ -1216,6 +1213,9 @@ __device__ __forceinline__ void set_unit(Ctx& cx, int n, int h, int T, int H,
     cx.ck_z0 = h * ck_slots + (int)(cx.row0 >> 6) + n;  // slot: floor(row0 / 64) + n + chunk
 }
 
+// kGdn: Gated DeltaNet (tm_r, tm_k, tm_v map q, k, v; g and beta per token; s0 may be
+// one state per head shared by every sequence, s0_shared != 0).  kHf (head first):
+// inputs, o (and g, beta) are [B, H, T, *] instead of [B, T, H, *]; the maps follow.
 template <bool kGdn, bool kHf, bool kRev>
 __global__ void __launch_bounds__(kThreads, kMinCtasPerSm)
 chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_w,
